@@ -1,0 +1,506 @@
+"""Pins of the CPU oracle to facts outside itself (runs without a GPU).
+
+Each test checks the oracle against something it does not compute the same
+way: a value the pages print, a published table, a closed form, a library
+routine, an invariant, or brute force on tiny inputs.
+"""
+
+import json
+import math
+import os
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.integrate
+import scipy.linalg
+from scipy.special import gamma
+
+from oracle import tq_oracle as O
+
+D = 128
+
+
+def _golden(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+def fmt(bits, sizes, H=1, seed=0, d=D, rng=None):
+    high = None
+    if len(bits) == 2:
+        rng = rng or np.random.default_rng(5)
+        high = np.stack([np.sort(rng.choice(d, sizes[0], replace=False)) for _ in range(H)])
+    return O.Format(d, H, tuple(bits), tuple(sizes), high, seed)
+
+
+FORMATS = {
+    "4u": ((4,), (128,)),
+    "3p5": ((4, 3), (64, 64)),
+    "2p5k": ((4, 2), (32, 96)),
+    "3u": ((3,), (128,)),
+    "2u": ((2,), (128,)),
+}
+
+
+# --- rotation ---------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [1, 2, 4, 8, 16, 32, 64, 128])
+def test_hadamard_matches_library_and_is_orthogonal(d):
+    H = O.hadamard_matrix(d)
+    assert np.array_equal(H, scipy.linalg.hadamard(d).astype(float))
+    assert np.array_equal(H @ H.T, d * np.eye(d))
+    assert np.array_equal(H, H.T)
+    K = np.array([[1.0]])
+    while K.shape[0] < d:  # Sylvester recursion H_2n = [[H, H], [H, -H]]
+        K = np.kron(np.array([[1.0, 1.0], [1.0, -1.0]]), K)
+    assert np.array_equal(H, K)
+
+
+def test_rotation_orthonormal_and_self_inverse():
+    rng = np.random.default_rng(0)
+    s = O.hadamard_signs(7, D)
+    R = O.rotate(np.eye(D), s)  # row i = R e_i, so R here is the transpose of the map
+    assert np.allclose(R @ R.T, np.eye(D), atol=1e-14)
+    x = rng.standard_normal((50, D))
+    y = O.rotate(x, s)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+    assert np.allclose(O.unrotate(y, s), x, atol=1e-13)
+    # rotating twice without signs is the identity up to scale 1 (H/sqrt(d) is an involution)
+    ones = np.ones(D)
+    assert np.allclose(O.rotate(O.rotate(x, ones), ones), x, atol=1e-13)
+
+
+def test_splitmix64_reference_outputs(golden_dir):
+    g = _golden(golden_dir, "splitmix64_seed0.json")
+    got = O.splitmix64(g["seed"], len(g["outputs_hex"]))
+    assert [f"{z:016x}" for z in got] == g["outputs_hex"]
+    s = O.hadamard_signs(0, 3)
+    assert list(s) == [-1.0 if int(h, 16) & 1 else 1.0 for h in g["outputs_hex"]]
+
+
+# --- coordinate density and codebooks ----------------------------------------
+
+@pytest.mark.parametrize("d", [3, 8, 128])
+def test_density_mass_and_moments_match_quadrature(d):
+    C = O.coord_density_const(d)
+    f = lambda x: C * (1 - x * x) ** ((d - 3) / 2)  # noqa: E731
+    for a, b in [(-1, 1), (-0.3, 0.05), (0.02, 0.2), (-0.9, -0.1), (0.2, 1.0)]:
+        m, _ = scipy.integrate.quad(f, a, b, epsabs=1e-15, epsrel=1e-13, limit=200)
+        m1, _ = scipy.integrate.quad(lambda x: x * f(x), a, b, epsabs=1e-15, epsrel=1e-13, limit=200)
+        m2, _ = scipy.integrate.quad(lambda x: x * x * f(x), a, b, epsabs=1e-15, epsrel=1e-13, limit=200)
+        assert O.cell_mass(a, b, d) == pytest.approx(m, rel=1e-11, abs=1e-15)
+        assert O.cell_first_moment(a, b, d) == pytest.approx(m1, rel=1e-11, abs=1e-15)
+        assert O.cell_second_moment(a, b, d) == pytest.approx(m2, rel=1e-11, abs=1e-15)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_codebook_d3_is_uniform_quantizer(bits):
+    # A coordinate of a uniform point on S^2 is uniform on [-1, 1] (Archimedes),
+    # whose Lloyd-Max quantizer is the uniform one.
+    L = 1 << bits
+    c = O.lloyd_max(bits, 3)
+    assert np.allclose(c, -1 + (2 * np.arange(L) + 1) / L, atol=1e-12)
+
+
+@pytest.mark.parametrize("d", [16, 128, 1000])
+def test_codebook_one_bit_closed_form(d):
+    c = O.lloyd_max(1, d)
+    e_abs = gamma(d / 2) / (math.sqrt(math.pi) * gamma((d + 1) / 2)) if d < 300 else \
+        math.exp(math.lgamma(d / 2) - math.lgamma((d + 1) / 2)) / math.sqrt(math.pi)
+    assert np.allclose(c, [-e_abs, e_abs], rtol=1e-13)
+
+
+def test_codebook_large_d_tends_to_gaussian_table(golden_dir):
+    # sqrt(d) X -> N(0, 1): the codebook tends to Max's Gaussian quantizer.
+    g = _golden(golden_dir, "gaussian_lloyd_max.json")["levels"]
+    d = 1 << 16
+    for bits in (1, 2, 3, 4):
+        ref = g[str(1 << bits)]
+        c = O.lloyd_max(bits, d, tol=1e-11) * math.sqrt(d)  # betainc noise floor is higher at d = 2^16
+        pos = c[len(c) // 2:]
+        assert np.allclose(pos, ref["outputs"], rtol=1.5e-3, atol=6e-4)
+        edges = np.concatenate(([-1.0], 0.5 * (c[:-1] + c[1:]) / math.sqrt(d), [1.0]))
+        cu = c / math.sqrt(d)
+        dist = (O.cell_second_moment(edges[:-1], edges[1:], d) - 2 * cu * O.cell_first_moment(edges[:-1], edges[1:], d)
+                + cu * cu * O.cell_mass(edges[:-1], edges[1:], d)).sum() * d
+        assert dist == pytest.approx(ref["mse"], rel=2e-3)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_codebook_optimality_conditions_d128(bits):
+    c = O.lloyd_max(bits, D)
+    assert np.allclose(c, -c[::-1], atol=0)
+    edges = np.concatenate(([-1.0], 0.5 * (c[:-1] + c[1:]), [1.0]))
+    C = O.coord_density_const(D)
+    for i in range(len(c)):
+        a, b = edges[i], edges[i + 1]
+        num, _ = scipy.integrate.quad(lambda x: x * C * (1 - x * x) ** 62.5, a, b, epsabs=1e-17, epsrel=1e-14)
+        den, _ = scipy.integrate.quad(lambda x: C * (1 - x * x) ** 62.5, a, b, epsabs=1e-17, epsrel=1e-14)
+        assert c[i] == pytest.approx(num / den, rel=1e-11, abs=1e-14)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_fp16_codebook_and_fp32_boundaries(bits):
+    c, beta = O.codebook(bits, D)
+    assert np.array_equal(c.astype(np.float16).astype(np.float64), c)
+    assert np.array_equal(beta, 0.5 * (c[:-1] + c[1:]))
+    assert np.array_equal(beta.astype(np.float32).astype(np.float64), beta)
+    assert np.all(np.diff(beta) > 0)
+    assert np.max(np.abs(c - O.lloyd_max(bits, D))) <= 2.0 ** -11 * np.max(np.abs(c))
+
+
+# --- quantizer -----------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_boundary_count_equals_nearest_centroid(bits):
+    c, beta = O.codebook(bits, D)
+    rng = np.random.default_rng(bits)
+    u = np.concatenate((rng.uniform(-0.4, 0.4, 4000), beta, np.nextafter(beta, 1), np.nextafter(beta, -1)))
+    idx = np.searchsorted(beta, u, side="left")
+    cf = [Fraction(float(ci)) for ci in c]
+    for x, i in zip(u, idx):
+        xf = Fraction(float(x))
+        dist = [abs(xf - ci) for ci in cf]  # exact rational distances
+        best = min(range(len(c)), key=lambda k: (dist[k], k))  # ties to the lower index
+        assert i == best
+
+
+def test_product_codeword_bruteforce_d4():
+    d, bits = 4, 2
+    f = O.Format(d, 1, (bits,), (d,), None, 3)
+    c, _ = O.codebook(bits, d)
+    grid = np.array(np.meshgrid(*[np.arange(4)] * d, indexing="ij")).reshape(d, -1).T  # 4^4 codewords
+    words = c[grid]
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((300, d))
+    idx, _, u = O.quantize(x, f, 0)
+    for k in range(len(x)):
+        best = np.argmin(((words - u[k]) ** 2).sum(axis=1))
+        assert np.array_equal(grid[best], idx[k])
+
+
+def test_norm_is_fp16_round_half_even_of_exact_norm():
+    rng = np.random.default_rng(2)
+    x = O.bf16_round(rng.standard_normal((400, D)) * rng.uniform(0.1, 50, (400, 1))).astype(np.float64)
+    f = fmt((4,), (128,))
+    _, n16, _ = O.quantize(x, f, 0)
+    for k in range(len(x)):
+        exact = math.sqrt(math.fsum(v * v for v in x[k]))
+        ref = struct.unpack("<e", struct.pack("<e", exact))[0]  # Python's IEEE half, RNE
+        assert n16[k] == ref
+
+
+def test_zero_vector_row():
+    f = fmt((4,), (128,))
+    idx, n16, u = O.quantize(np.zeros((1, D)), f, 0)
+    assert n16[0] == 0.0 and np.all(u == 0) and np.all(idx == 7)
+    assert np.all(O.dequantize_rows(idx, n16, f, 0) == 0)
+
+
+# --- row format ---------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,expected", [("4u", 66), ("3p5", 58), ("2p5k", 42), ("3u", 50), ("2u", 34)])
+def test_row_bytes(name, expected):
+    bits, sizes = FORMATS[name]
+    assert O.row_bytes(fmt(bits, sizes)) == expected
+
+
+@pytest.mark.parametrize("name", list(FORMATS))
+def test_pack_roundtrip_exhaustive(name):
+    bits, sizes = FORMATS[name]
+    f = fmt(bits, sizes)
+    pb = O.position_bits(f)
+    L = 1 << int(pb.max())
+    idx = (np.arange(D)[None, :] + np.arange(L)[:, None]) % (1 << pb)[None, :]  # every value at every position
+    n16 = O.fp16_round(np.linspace(0, 300, L))
+    rows = O.encode_rows(idx, n16, f)
+    assert rows.shape == (L, O.row_bytes(f))
+    back, nb = O.decode_rows(rows, f)
+    assert np.array_equal(back, idx) and np.array_equal(nb, n16)
+
+
+def test_row_bit_layout_golden(golden_dir):
+    for case in _golden(golden_dir, "row_bit_layout.json")["cases"]:
+        d = sum(case["group_size"])
+        high = np.arange(case["group_size"][0])[None, :] if len(case["group_bits"]) == 2 else None
+        f = O.Format(d, 1, tuple(case["group_bits"]), tuple(case["group_size"]), high, 0)
+        row = O.encode_rows(np.array([case["indices"]]), np.array([case["norm"]]), f)[0]
+        assert bytes(row).hex() == case["row_hex"]
+
+
+def test_permutation_puts_high_coords_first():
+    f = fmt((4, 3), (64, 64), H=3)
+    for h in range(3):
+        p = O.permutation(f, h)
+        assert sorted(p) == list(range(D))
+        assert list(p[:64]) == sorted(f.high_coords[h]) and list(p[64:]) == sorted(set(range(D)) - set(p[:64]))
+
+
+# --- reconstruction invariant -------------------------------------------------
+
+@pytest.mark.parametrize("name", ["4u", "3p5", "2p5k", "3u"])
+def test_reconstruction_error_matches_codebook_distortion(name):
+    bits, sizes = FORMATS[name]
+    f = fmt(bits, sizes)
+    expected = 0.0
+    for b, n in zip(bits, sizes):
+        c, beta = O.codebook(b, D)
+        e = np.concatenate(([-1.0], beta, [1.0]))
+        per = (O.cell_second_moment(e[:-1], e[1:], D) - 2 * c * O.cell_first_moment(e[:-1], e[1:], D)
+               + c * c * O.cell_mass(e[:-1], e[1:], D)).sum()
+        expected += n * per
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((20000, D))
+    idx, _, u = O.quantize(x, f, 0)
+    chat = np.empty_like(u)
+    start = 0
+    for b, n in zip(bits, sizes):
+        c, _ = O.codebook(b, D)
+        chat[:, start:start + n] = c[idx[:, start:start + n]]
+        start += n
+    err = ((u - chat) ** 2).sum(axis=1)
+    sigma = err.std() / math.sqrt(len(err))
+    assert abs(err.mean() - expected) < 4 * sigma
+    # reconstruction through rows and the inverse rotation gives the same error up to the fp16 norm
+    xr = O.dequantize_rows(idx[:200], np.linalg.norm(x[:200], axis=1), f, 0)
+    n = np.linalg.norm(x[:200], axis=1)
+    assert np.allclose(((xr - x[:200]) ** 2).sum(axis=1) / n ** 2, err[:200], rtol=1e-9, atol=1e-13)
+
+
+# --- pages, addressing --------------------------------------------------------
+
+def test_pack_addressing_by_formula():
+    rng = np.random.default_rng(4)
+    H, bs, nb, T = 2, 4, 6, 17
+    kf, vf = fmt((4,), (128,), H=H, seed=0), fmt((4, 3), (64, 64), H=H, seed=1)
+    k = O.bf16_round(rng.standard_normal((T, H, D))).astype(np.float64)
+    v = O.bf16_round(rng.standard_normal((T, H, D))).astype(np.float64)
+    slots = rng.permutation(nb * bs)[:T]
+    slots[3] = -1
+    kp, vp = O.pack_kv(k, v, slots, kf, vf, nb, bs)
+    for t in range(T):
+        for h in range(H):
+            if slots[t] < 0:
+                continue
+            ki, kn, _ = O.quantize(k[t, h][None], kf, h)
+            vi, vn, _ = O.quantize(v[t, h][None], vf, h)
+            assert np.array_equal(O.read_row(kp, slots[t], h, bs), O.encode_rows(ki, kn, kf)[0])
+            assert np.array_equal(O.read_row(vp, slots[t], h, bs), O.encode_rows(vi, vn, vf)[0])
+    written = {(s // bs, s % bs) for s in slots if s >= 0}
+    for blk in range(nb):
+        for off in range(bs):
+            if (blk, off) not in written:
+                assert not kp[blk, :, off].any()
+    with pytest.raises(IndexError):
+        O.pack_kv(k, v, np.full(T, nb * bs), kf, vf, nb, bs)
+
+
+# --- attention ---------------------------------------------------------------
+
+def _pages_for(seq_keys, seq_vals, kf, vf, bs, rng):
+    """Pack one sequence's tokens into a permuted block pool."""
+    P = len(seq_keys)
+    nblk = max(1, -(-P // bs))
+    table = rng.permutation(nblk + 2)[:nblk]
+    slots = table[np.arange(P) // bs] * bs + np.arange(P) % bs
+    kp, vp = O.pack_kv(seq_keys, seq_vals, slots, kf, vf, nblk + 2, bs)
+    return kp, vp, table
+
+
+def test_attention_single_token_returns_its_value():
+    rng = np.random.default_rng(6)
+    kf, vf = fmt((4,), (128,)), fmt((3,), (128,), seed=1)
+    k = O.bf16_round(rng.standard_normal((1, 1, D))).astype(np.float64)
+    v = O.bf16_round(rng.standard_normal((1, 1, D))).astype(np.float64)
+    kp, vp, table = _pages_for(k, v, kf, vf, 16, rng)
+    q = rng.standard_normal((1, 4, D))
+    out = O.decode_attention(q, kp, vp, table[None], [1], None, None, 0, 0.1, kf, vf, 16)
+    vi, vn = O.decode_rows(vp[table[0], 0, 0][None], vf)
+    vhat = O.dequantize_rows(vi, vn, vf, 0)[0]
+    for g in range(4):
+        assert np.allclose(out[0, g], vhat, atol=1e-13)
+
+
+def test_attention_identical_keys_average_values():
+    rng = np.random.default_rng(7)
+    kf, vf = fmt((4,), (128,)), fmt((4,), (128,), seed=1)
+    P = 37
+    k = np.repeat(O.bf16_round(rng.standard_normal((1, 1, D))).astype(np.float64), P, axis=0)
+    v = O.bf16_round(rng.standard_normal((P, 1, D))).astype(np.float64)
+    kp, vp, table = _pages_for(k, v, kf, vf, 8, rng)
+    q = rng.standard_normal((1, 2, D))
+    out = O.decode_attention(q, kp, vp, table[None], [P], None, None, 0, 0.3, kf, vf, 8)
+    vi, vn, _ = O.quantize(v[:, 0], vf, 0)
+    mean = O.dequantize_rows(vi, vn, vf, 0).mean(axis=0)
+    assert np.allclose(out[0, 0], mean, atol=1e-12) and np.allclose(out[0, 1], mean, atol=1e-12)
+
+
+def test_attention_window_only_is_dense_softmax_by_hand():
+    rng = np.random.default_rng(8)
+    kf, vf = fmt((4,), (128,)), fmt((4,), (128,))
+    W, L, d = 5, 3, D
+    kw = np.zeros((1, 1, W, d))
+    vw = np.zeros((1, 1, W, d))
+    kw[0, 0, :L] = rng.standard_normal((L, d))
+    vw[0, 0, :L] = rng.standard_normal((L, d))
+    q = rng.standard_normal((1, 1, d))
+    pages = np.zeros((1, 1, 4, O.row_bytes(kf)), dtype=np.uint8)
+    out = O.decode_attention(q, pages, pages, np.zeros((1, 1), np.int64), [L], kw, vw, W, 0.2, kf, vf, 4)
+    s = [0.2 * sum(q[0, 0, j] * kw[0, 0, t, j] for j in range(d)) for t in range(L)]
+    m = max(s)
+    w = [math.exp(x - m) for x in s]
+    ref = [sum(w[t] * vw[0, 0, t, j] for t in range(L)) / sum(w) for j in range(d)]
+    assert np.allclose(out[0, 0], ref, atol=1e-12)
+
+
+def test_sixteen_bit_codebook_reproduces_dense_attention():
+    rng = np.random.default_rng(9)
+    f16 = O.Format(D, 1, (16,), (D,), None, 5)
+    P = 64
+    k = rng.standard_normal((P, D)) * 3
+    v = rng.standard_normal((P, D)) * 3
+    q = rng.standard_normal(D)
+    ki, kn, _ = O.quantize(k, f16, 0)
+    vi, vn, _ = O.quantize(v, f16, 0)
+    kh, vh = O.dequantize_rows(ki, kn, f16, 0), O.dequantize_rows(vi, vn, f16, 0)
+    scale = 1 / math.sqrt(D)
+    ref = O.dense_attention(q, k, v, scale)
+    got = O.dense_attention(q, kh, vh, scale)
+    # Perturbation bound: |d out| <= max_t |dv_t| + 2 max|v| max_t |d s_t|.
+    dv = np.abs(vh - v).max()
+    ds = scale * np.abs((kh - k) @ q).max()
+    bound = dv + 2 * np.abs(v).max() * ds
+    err = np.abs(got - ref).max()
+    assert err <= bound
+    assert err < 5e-5 * np.abs(v).max()
+    # the same comparison with the 4-bit codebook is three orders of magnitude worse
+    f4 = O.Format(D, 1, (4,), (D,), None, 5)
+    k4 = O.dequantize_rows(*O.quantize(k, f4, 0)[:2], f4, 0)
+    v4 = O.dequantize_rows(*O.quantize(v, f4, 0)[:2], f4, 0)
+    assert np.abs(O.dense_attention(q, k4, v4, scale) - ref).max() > 1000 * err
+
+
+def _bruteforce_row_decode(row, bits, sizes, perm):
+    """Read a row bit by bit (pure Python) into (rotated-order indices, norm)."""
+    idx = [0] * sum(sizes)
+    bitpos = 0
+    p = 0
+    for b, n in zip(bits, sizes):
+        for _ in range(n):
+            val = 0
+            for k in range(b):
+                byte, bit = divmod(bitpos, 8)
+                val |= ((int(row[byte]) >> bit) & 1) << k
+                bitpos += 1
+            idx[perm[p]] = val
+            p += 1
+    norm = struct.unpack("<e", bytes(row[bitpos // 8: bitpos // 8 + 2]))[0]
+    return idx, norm
+
+
+def test_attention_bruteforce_tiny():
+    rng = np.random.default_rng(10)
+    d, H, G, bs, W = 8, 2, 2, 2, 2
+    high = np.stack([np.sort(rng.choice(d, 4, replace=False)) for _ in range(H)])
+    kf = O.Format(d, H, (4, 2), (4, 4), high, 3)
+    vf = O.Format(d, H, (3,), (d,), None, 9)
+    lens = [3, 5]
+    B = len(lens)
+    maxb = 2
+    tables = np.array([[4, 1], [0, 3]])
+    nb = 5
+    kp = np.zeros((nb, H, bs, O.row_bytes(kf)), np.uint8)
+    vp = np.zeros((nb, H, bs, O.row_bytes(vf)), np.uint8)
+    kw = np.zeros((B, H, W, d))
+    vw = np.zeros((B, H, W, d))
+    hist_k, hist_v = {}, {}
+    for b, L in enumerate(lens):
+        P = L - min(W, L)
+        kk = O.bf16_round(rng.standard_normal((L, H, d)) * 2).astype(np.float64)
+        vv = O.bf16_round(rng.standard_normal((L, H, d)) * 2).astype(np.float64)
+        slots = tables[b, np.arange(P) // bs] * bs + np.arange(P) % bs
+        O.pack_kv(kk[:P], vv[:P], slots, kf, vf, nb, bs, kp, vp)
+        kw[b, :, :L - P] = kk[P:].transpose(1, 0, 2)
+        vw[b, :, :L - P] = vv[P:].transpose(1, 0, 2)
+        hist_k[b], hist_v[b] = kk, vv
+    q = rng.standard_normal((B, H * G, d))
+    out = O.decode_attention(q, kp, vp, tables, lens, kw, vw, W, 0.7, kf, vf, bs)
+
+    def hand_dequant(row, f, h):
+        perm = list(O.permutation(f, h))
+        idx, norm = _bruteforce_row_decode(row, f.group_bits, f.group_size, perm)
+        bits_of = {}
+        p = 0
+        for b_, n_ in zip(f.group_bits, f.group_size):
+            for _ in range(n_):
+                bits_of[perm[p]] = b_
+                p += 1
+        cent = [O.codebook(bits_of[j], d)[0][idx[j]] for j in range(d)]
+        z = O.splitmix64(f.seed, d)
+        s = [-1.0 if zz & 1 else 1.0 for zz in z]
+        return [norm * s[i] * sum((-1) ** bin(i & j).count("1") * cent[j] for j in range(d)) / math.sqrt(d)
+                for i in range(d)]
+
+    for b, L in enumerate(lens):
+        P = L - min(W, L)
+        for hq in range(H * G):
+            h = hq // G
+            keys, vals = [], []
+            for t in range(P):
+                blk, off = tables[b][t // bs], t % bs
+                keys.append(hand_dequant(kp[blk, h, off], kf, h))
+                vals.append(hand_dequant(vp[blk, h, off], vf, h))
+            for t in range(L - P):
+                keys.append(list(kw[b, h, t]))
+                vals.append(list(vw[b, h, t]))
+            s = [0.7 * sum(q[b, hq, j] * kk[j] for j in range(d)) for kk in keys]
+            m = max(s)
+            w = [math.exp(x - m) for x in s]
+            ref = [sum(w[t] * vals[t][j] for t in range(L)) / sum(w) for j in range(d)]
+            assert np.allclose(out[b, hq], ref, atol=1e-12)
+
+
+# --- byte ledger --------------------------------------------------------------
+
+def test_ledger_ratios_match_server_page(golden_dir):
+    g = _golden(golden_dir, "server_page_table.json")
+    tol = g["printed_precision"]
+    for key, (bits, sizes) in (("tq35", ((4, 3), (64, 64))), ("tq25", ((4, 2), (32, 96)))):
+        f = fmt(bits, sizes, H=8)
+        assert f.mean_bits == g["bits_per_channel"][key]
+        led = O.byte_ledger(f, f, [4096] * 4, 0, 16, 1024)
+        ratio = led.dense_bytes / led.index_bytes  # index-only ratio, as the page reports
+        assert abs(ratio - g["compression_ratio"][key]) <= tol["compression_ratio"]
+        equiv = g["equivalent_context_tokens_80gb_a100"]["full"] * ratio
+        assert equiv == pytest.approx(g["equivalent_context_tokens_80gb_a100"][key], rel=tol["equivalent_context_relative"])
+    # with the 2-byte norm included, per-row ratios are 256/66, 256/58, 256/42, 256/50
+    for (bits, sizes), rb in (((4,), (128,)), 66), (((4, 3), (64, 64)), 58), (((4, 2), (32, 96)), 42), (((3,), (128,)), 50):
+        f = fmt(bits, sizes, H=8)
+        led = O.byte_ledger(f, f, [100], 0, 16, 7)
+        assert led.dense_bytes / (led.index_bytes + led.norm_bytes) == pytest.approx(256 / rb)
+
+
+def test_ledger_counts_what_the_oracle_allocates():
+    rng = np.random.default_rng(12)
+    H, bs, W = 2, 4, 3
+    kf, vf = fmt((4, 3), (64, 64), H=H), fmt((3,), (128,), H=H, seed=2)
+    lens = [2, 9, 13]
+    packed = [L - min(W, L) for L in lens]
+    nblk = [-(-p // bs) for p in packed]
+    nb = sum(nblk) + 1
+    led = O.byte_ledger(kf, vf, lens, W, bs, nb, workspace_bytes=123)
+    k = O.bf16_round(rng.standard_normal((sum(packed), H, D))).astype(np.float64)
+    kp, vp = O.pack_kv(k, k, np.arange(sum(packed)), kf, vf, nb, bs)
+    assert led.page_pool_bytes == kp.nbytes + vp.nbytes
+    assert led.index_bytes + led.norm_bytes == sum(packed) * H * (O.row_bytes(kf) + O.row_bytes(vf))
+    assert led.window_bytes == 2 * np.zeros((len(lens), H, W, D), np.float16).nbytes
+    assert led.block_table_bytes == np.zeros(sum(nblk), np.int32).nbytes
+    cb = sum(O.codebook(b, D)[0].astype(np.float16).nbytes + O.codebook(b, D)[1].astype(np.float32).nbytes
+             for f in (kf, vf) for b in f.group_bits)
+    assert led.codebook_bytes == cb
+    assert led.dense_bytes == 2 * np.zeros((sum(lens), H, D), np.float16).nbytes
+    assert led.workspace_bytes == 123
+    assert led.metadata_bytes == led.norm_bytes + led.codebook_bytes + led.transform_bytes + led.window_bytes \
+        + led.block_table_bytes + 123
