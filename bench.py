@@ -1,0 +1,556 @@
+"""Benchmark of the compressed paged KV cache on B200: one JSON line on rank 0.
+
+A step is one serving decode step of the whole hot path over the workload's
+batch: tq_pack_kv writes the step's new K/V vector per (sequence, KV head)
+into its page slot (the token that leaves the dense window), then
+tq_decode_paged attends every query head over the packed history plus the
+bf16 window. Inputs are resident in HBM before timing; the page pools are far
+larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+--impl reference times the CPU oracle (fp64 NumPy) on a bounded sample of the
+same workload: it is a deliberately slow baseline, not a target.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from quantized_paged_kv_pack_b200 import tq  # noqa: E402
+from quantized_paged_kv_pack_b200 import workloads as WL  # noqa: E402
+
+HEADLINE = "decode_llama70b_3p5bit"
+EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "pack_llama8b_4bit"]
+D = 128
+METRIC = "paged TQ decode HBM GB/s (algorithmic bytes / step time)"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash(name):
+    with open(os.path.join(ROOT, "quantized_paged_kv_pack_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def stored_traffic(workload, kernel_file):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        t = json.load(f)
+    e = t.get(workload)
+    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
+        return None
+    return e.get("bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- workload setup
+
+class DecodeSetup:
+    """A decode workload resident on the GPU, with the pages written by tq_pack_kv."""
+
+    def __init__(self, w: WL.Workload, seed_offset: int = 0):
+        if seed_offset:
+            w = WL.Workload(**{**w.__dict__, "seed": w.seed + 1000 * seed_offset})
+        self.w = w
+        ks, vs = WL.codec_specs(w)
+        self.kspec, self.vspec = ks, vs
+        self.kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed)
+        self.vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed)
+        lay = WL.page_layout(w)
+        B = len(lay.seq_lens)
+        # one spare block per sequence takes the step's appended row
+        self.num_blocks = lay.num_blocks + B
+        self.append_block = np.arange(lay.num_blocks, lay.num_blocks + B)
+        self.layout = lay
+        bs = w.block_size
+        self.kp = tq.page_pool(self.kc, self.num_blocks, bs)
+        self.vp = tq.page_pool(self.vc, self.num_blocks, bs)
+        for b in range(B):
+            P = int(lay.packed_lens[b])
+            for t0 in range(0, P, 32768):
+                t1 = min(P, t0 + 32768)
+                k, v = WL.sequence_kv(w, b, t0, t1, device="cuda")
+                slots = torch.as_tensor(WL.slot_mapping(lay, b, t0, t1, bs), device="cuda")
+                tq.pack_kv(self.kc, self.vc, k, v, slots, self.kp, self.vp)
+        self.kw, self.vw = WL.windows(w, lay, device="cuda")
+        self.q = WL.queries(w, device="cuda")
+        self.bt = torch.as_tensor(lay.block_tables, device="cuda")
+        self.sl = torch.as_tensor(lay.seq_lens.astype(np.int32), device="cuda")
+        self.max_len = int(lay.seq_lens.max())
+        self.scale = 1.0 / math.sqrt(D)
+        self.ws = tq.alloc_workspace(B, w.num_q_heads, w.num_kv_heads, self.max_len, bs)
+        self.out = torch.empty(B, w.num_q_heads, D, dtype=torch.float32, device="cuda")
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        # the step's appended vector per (sequence, head): the token leaving the window
+        g = torch.Generator(device="cuda")
+        g.manual_seed(w.seed + 99)
+        self.new_k = (torch.randn(B, w.num_kv_heads, D, generator=g, device="cuda") * 2).to(torch.bfloat16)
+        self.new_v = (torch.randn(B, w.num_kv_heads, D, generator=g, device="cuda") * 2).to(torch.bfloat16)
+        self.new_slots = torch.as_tensor(self.append_block.astype(np.int64) * bs, device="cuda")
+        torch.cuda.synchronize()
+
+    # algorithmic bytes -----------------------------------------------------
+    def decode_split_bytes(self):
+        w, lay = self.w, self.layout
+        rows = int(lay.packed_lens.sum()) * w.num_kv_heads * (self.kc.row_bytes + self.vc.row_bytes)
+        win = int(np.minimum(w.window, lay.seq_lens).sum()) * w.num_kv_heads * D * 2 * 2
+        bt = 4 * int((-(-lay.packed_lens // w.block_size)).sum())
+        q = len(lay.seq_lens) * w.num_q_heads * D * 2
+        return rows + win + bt + q
+
+    def out_bytes(self):
+        return len(self.layout.seq_lens) * self.w.num_q_heads * D * 4
+
+    def pack_bytes(self):
+        B, H = len(self.layout.seq_lens), self.w.num_kv_heads
+        return B * H * D * 2 * 2 + B * H * (self.kc.row_bytes + self.vc.row_bytes) + B * 8
+
+    def step_bytes(self):
+        return self.decode_split_bytes() + self.out_bytes() + self.pack_bytes()
+
+    def kv_tokens(self):
+        return int(self.layout.seq_lens.sum())
+
+    # the step ---------------------------------------------------------------
+    def pack(self, k=None, v=None, slots=None):
+        tq.pack_kv(self.kc, self.vc, self.new_k if k is None else k, self.new_v if v is None else v,
+                   self.new_slots if slots is None else slots, self.kp, self.vp, d_err=self.err)
+
+    def decode(self, phase="all", q=None, out=None):
+        w = self.w
+        return tq.decode_paged(self.kc, self.vc, self.q if q is None else q, self.kp, self.vp, self.bt, self.sl,
+                               self.max_len, self.kw if w.window else None, self.vw if w.window else None, w.window,
+                               self.scale, out=self.out if out is None else out, workspace=self.ws, d_err=self.err,
+                               phase=phase)
+
+
+class PackSetup:
+    def __init__(self, w: WL.Workload):
+        self.w = w
+        ks, vs = WL.codec_specs(w)
+        self.kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed)
+        self.vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed)
+        self.k, self.v, slots, lay = WL.pack_batch(w, device="cuda")
+        self.slots = torch.as_tensor(slots, device="cuda")
+        self.kp = tq.page_pool(self.kc, lay.num_blocks, w.block_size)
+        self.vp = tq.page_pool(self.vc, lay.num_blocks, w.block_size)
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        torch.cuda.synchronize()
+
+    def bytes(self):
+        T, H = self.k.shape[0], self.w.num_kv_heads
+        return T * H * D * 2 * 2 + T * H * (self.kc.row_bytes + self.vc.row_bytes) + T * 8
+
+    def step(self):
+        tq.pack_kv(self.kc, self.vc, self.k, self.v, self.slots, self.kp, self.vp, d_err=self.err)
+
+
+# --------------------------------------------------------------------------- measurement
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index=0):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            sel = str(device_index)
+        self.sel = sel
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        time.sleep(0.15)
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def time_steps(fns, steps, stream):
+    """Run `steps` iterations of the callables in `fns` with events between them.
+
+    Returns (total ms, [per-callable mean ms]). Events are recorded on the
+    stream the library launches on (torch's current stream).
+    """
+    n = len(fns)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for s in range(steps):
+        ev[s][0].record(stream)
+        for i, f in enumerate(fns):
+            f()
+            ev[s][i + 1].record(stream)
+    torch.cuda.synchronize()
+    total = sum(ev[s][0].elapsed_time(ev[s][n]) for s in range(steps))
+    parts = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps for i in range(n)]
+    return total, parts
+
+
+def measure_decode(setup: DecodeSetup, steps, warmup, dist_ctx=None, clocks=True):
+    stream = torch.cuda.current_stream()
+    fns = [setup.pack, lambda: setup.decode("partials"), lambda: setup.decode("combine")]
+    for _ in range(warmup):
+        for f in fns:
+            f()
+    torch.cuda.synchronize()
+    if setup.err.item():
+        raise RuntimeError(f"device error word {setup.err.item()} during warm-up")
+    barrier(dist_ctx)
+    sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if sampler:
+        sampler.__enter__()
+    total_ms, parts = time_steps(fns, steps, stream)
+    if sampler:
+        sampler.__exit__(None, None, None)
+    barrier(dist_ctx)
+    total_ms = max_over_ranks(total_ms, dist_ctx)
+    return total_ms / steps, parts, (sampler.summary() if sampler else None)
+
+
+def measure_decode_e2e(setup: DecodeSetup, steps, warmup):
+    """Same step through the public API from pinned host buffers (H2D in, D2H out, inside the timing)."""
+    B, Hq, H = setup.q.shape[0], setup.q.shape[1], setup.w.num_kv_heads
+    hq = setup.q.cpu().pin_memory()
+    hk = setup.new_k.cpu().pin_memory()
+    hv = setup.new_v.cpu().pin_memory()
+    hs = setup.new_slots.cpu().pin_memory()
+    hout = torch.empty(B, Hq, D, dtype=torch.float32).pin_memory()
+    dq, dk, dv, ds = torch.empty_like(setup.q), torch.empty_like(setup.new_k), torch.empty_like(setup.new_v), \
+        torch.empty_like(setup.new_slots)
+    dout = torch.empty_like(setup.out)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        ds.copy_(hs, non_blocking=True)
+        setup.pack(dk, dv, ds)
+        setup.decode("all", q=dq, out=dout)
+        hout.copy_(dout, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    total, _ = time_steps([step], steps, torch.cuda.current_stream())
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + hs.numel() * 8
+    d2h = hout.numel() * 4
+    return total / steps, h2d, d2h
+
+
+def measure_pack(setup: PackSetup, steps, warmup):
+    for _ in range(warmup):
+        setup.step()
+    torch.cuda.synchronize()
+    total, _ = time_steps([setup.step], steps, torch.cuda.current_stream())
+    return total / steps
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+
+def init_dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return dist
+
+
+def barrier(dist_ctx):
+    if dist_ctx is not None:
+        dist_ctx.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, dist_ctx):
+    if dist_ctx is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist_ctx.all_reduce(t, op=dist_ctx.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- CPU oracle legs
+
+def _oracle_formats(w, kspec, vspec, h):
+    from oracle import tq_oracle as O
+
+    hk = None if kspec.high_coords is None else kspec.high_coords[h:h + 1]
+    hv = None if vspec.high_coords is None else vspec.high_coords[h:h + 1]
+    return (O.Format(D, 1, kspec.group_bits, kspec.group_size, hk, kspec.seed),
+            O.Format(D, 1, vspec.group_bits, vspec.group_size, hv, vspec.seed))
+
+
+def _median_sequence(lay):
+    order = np.argsort(lay.seq_lens, kind="stable")
+    return int(order[len(order) // 2])
+
+
+def gpu_pages_unit(setup: "DecodeSetup", b: int, h: int):
+    """(kp, vp, table, q, kw, vw) of unit (b, h) from the GPU-written cache."""
+    w, lay = setup.w, setup.layout
+    G = w.num_q_heads // w.num_kv_heads
+    P = int(lay.packed_lens[b])
+    nblk = -(-P // w.block_size)
+    blocks = torch.as_tensor(lay.block_tables[b, :max(nblk, 1)].astype(np.int64).clip(0), device="cuda")
+    return (setup.kp[blocks][:, h:h + 1].cpu().numpy(), setup.vp[blocks][:, h:h + 1].cpu().numpy(),
+            np.arange(max(nblk, 1))[None], setup.q[b:b + 1, h * G:(h + 1) * G].float().cpu().numpy().astype(np.float64),
+            setup.kw[b:b + 1, h:h + 1].float().cpu().numpy(), setup.vw[b:b + 1, h:h + 1].float().cpu().numpy())
+
+
+def oracle_pages_unit(w, kspec, vspec, lay, b, h, cache={}):
+    """(kp, vp, table, q, kw, vw) of unit (b, h) built on the CPU by the oracle's own pack."""
+    from oracle import tq_oracle as O
+
+    key = (w.name, b)
+    if key not in cache:
+        cache.clear()
+        L = int(lay.seq_lens[b])
+        k, v = WL.sequence_kv(w, b, 0, L, device="cpu")
+        cache[key] = (k.float().numpy(), v.float().numpy(), WL.queries(w, device="cpu").float().numpy())
+    k, v, q = cache[key]
+    G = w.num_q_heads // w.num_kv_heads
+    L, P = int(lay.seq_lens[b]), int(lay.packed_lens[b])
+    kf1, vf1 = _oracle_formats(w, kspec, vspec, h)
+    nblk = max(1, -(-P // w.block_size))
+    kp, vp = O.pack_kv(k[:P, h:h + 1], v[:P, h:h + 1], np.arange(P), kf1, vf1, nblk, w.block_size)
+    Wn = max(w.window, 1)
+    kw = np.zeros((1, 1, Wn, D))
+    vw = np.zeros((1, 1, Wn, D))
+    kw[0, 0, :L - P] = k[P:L, h]
+    vw[0, 0, :L - P] = v[P:L, h]
+    return kp, vp, np.arange(nblk)[None], q[b:b + 1, h * G:(h + 1) * G].astype(np.float64), kw, vw
+
+
+def oracle_decode_sample(w, kspec, vspec, lay, unit_source, budget_s: float, row_bytes):
+    """Time the oracle's decode attention on (sequence, KV head) units until ~budget_s of CPU work.
+
+    Returns (GB/s of algorithmic bytes, KV token-heads/s, description, threads).
+    """
+    from oracle import tq_oracle as O
+
+    G = w.num_q_heads // w.num_kv_heads
+    b = _median_sequence(lay)
+    L, P = int(lay.seq_lens[b]), int(lay.packed_lens[b])
+    done_bytes = done_tok = 0
+    elapsed = 0.0
+    units = 0
+    for h in range(w.num_kv_heads):
+        kp, vp, table, q, kw, vw = unit_source(b, h)
+        kf1, vf1 = _oracle_formats(w, kspec, vspec, h)
+        t0 = time.perf_counter()
+        O.decode_attention(q, kp, vp, table, [L], kw, vw, w.window, 1.0 / math.sqrt(D), kf1, vf1, w.block_size)
+        elapsed += time.perf_counter() - t0
+        units += 1
+        n_win = min(w.window, L)
+        done_bytes += P * row_bytes + n_win * D * 4 + 4 * (-(-P // w.block_size)) + G * D * 6
+        done_tok += L
+        if elapsed >= budget_s:
+            break
+    threads = len(os.sched_getaffinity(0))
+    desc = (f"oracle decode of sequence {b} (L={L}, the median length), {units} of {w.num_kv_heads} KV heads, "
+            f"all {G} query heads of each")
+    return done_bytes / elapsed / 1e9, done_tok / elapsed, desc, threads
+
+
+# --------------------------------------------------------------------------- main
+
+def run_reference(args):
+    """--impl reference: the CPU oracle as the reference arm (rank 0 only, no GPU code)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WL.WORKLOADS[args.workload]
+    kspec, vspec = WL.codec_specs(w)
+    lay = WL.page_layout(w)
+    from oracle import tq_oracle as O
+
+    rb = sum(O.row_bytes(O.Format(D, 1, s.group_bits, s.group_size,
+                                  None if s.high_coords is None else s.high_coords[:1], s.seed)) for s in (kspec, vspec))
+    src = lambda b, h: oracle_pages_unit(w, kspec, vspec, lay, b, h)  # noqa: E731
+    for _ in range(args.warmup):
+        oracle_decode_sample(w, kspec, vspec, lay, src, 0.0, rb)
+    vals, desc, threads = [], None, None
+    for _ in range(args.steps):
+        gbs, tps, desc, threads = oracle_decode_sample(w, kspec, vspec, lay, src, args.reference_budget, rb)
+        vals.append(gbs)
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "description": w.description},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    dist_ctx = init_dist()
+    rank = dist_ctx.get_rank() if dist_ctx else 0
+    world = dist_ctx.get_world_size() if dist_ctx else 1
+    if world == 1:
+        torch.cuda.set_device(0)
+    w = WL.WORKLOADS[args.workload]
+    setup = DecodeSetup(w, seed_offset=rank)
+    step_ms, parts, clocks = measure_decode(setup, args.steps, args.warmup, dist_ctx)
+    e2e_ms, h2d, d2h = measure_decode_e2e(setup, max(3, args.steps // 2), args.warmup)
+    e2e_ms = max_over_ranks(e2e_ms, dist_ctx)
+    peak, peak_kind = peaks()
+    split_bytes = setup.decode_split_bytes()
+    achieved = split_bytes / (parts[1] * 1e-3) / 1e9
+    step_bytes = setup.step_bytes()
+    value = world * step_bytes / (step_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+        "config": {"workload": w.name, "description": w.description, "batch": w.batch,
+                   "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": D,
+                   "block_size": w.block_size, "window": w.window,
+                   "k_format": {"bits": list(w.k_bits), "sizes": list(w.k_sizes)},
+                   "v_format": {"bits": list(w.v_bits), "sizes": list(w.v_sizes)},
+                   "parallelism": f"{world} independent replicas (no collective)",
+                   "l2": f"no flush: {split_bytes / 1e9:.2f} GB of pages read per step, L2 is 126 MB"},
+        "kv_tokens_per_s": world * setup.kv_tokens() / (step_ms * 1e-3),
+        "step_breakdown_ms": {"pack": parts[0], "decode_partials": parts[1], "decode_combine": parts[2]},
+        "algorithmic_bytes_per_step": step_bytes,
+        "roofline": {"bound": "hbm", "kernel": "decode_partials", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "frac_of_8TBs": achieved / 8000.0,
+                     "traffic": stored_traffic(w.name, "tq_decode.cu")},
+        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        gbs, tps, desc, threads = oracle_decode_sample(
+            w, setup.kspec, setup.vspec, setup.layout, lambda b, h: gpu_pages_unit(setup, b, h), args.cpu_budget,
+            setup.kc.row_bytes + setup.vc.row_bytes)
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
+                                "kv_token_heads_per_s": tps}
+    if world == 1 and not args.no_extra:
+        extra = {}
+        for name in EXTRA:
+            ew = WL.WORKLOADS[name]
+            if ew.kind == "decode":
+                del setup
+                torch.cuda.empty_cache()
+                setup = DecodeSetup(ew)
+                ms, p, _ = measure_decode(setup, max(5, args.steps // 2), args.warmup, None, clocks=False)
+                sb = setup.decode_split_bytes()
+                extra[name] = {"GB/s": setup.step_bytes() / (ms * 1e-3) / 1e9,
+                               "kv_tokens_per_s": setup.kv_tokens() / (ms * 1e-3), "ms_per_step": ms,
+                               "decode_partials_GB/s": sb / (p[1] * 1e-3) / 1e9,
+                               "decode_partials_frac": sb / (p[1] * 1e-3) / 1e9 / peak,
+                               "traffic": stored_traffic(name, "tq_decode.cu")}
+            else:
+                del setup
+                torch.cuda.empty_cache()
+                setup = PackSetup(ew)
+                ms = measure_pack(setup, max(5, args.steps // 2), args.warmup)
+                gbs = setup.bytes() / (ms * 1e-3) / 1e9
+                extra[name] = {"GB/s": gbs, "tokens_per_s": setup.k.shape[0] / (ms * 1e-3), "ms_per_step": ms,
+                               "frac": gbs / peak, "traffic": stored_traffic(name, "tq_pack.cu")}
+                line["gpu_launches"] += max(5, args.steps // 2)
+        line["per_workload"] = extra
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_ctx is not None:
+        dist_ctx.barrier()
+        dist_ctx.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--reference-budget", type=float, default=4.0, help="seconds of oracle work per reference step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

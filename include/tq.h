@@ -1,0 +1,255 @@
+/*
+ * tq.h - C ABI of the compressed paged KV cache library (libtq.so, sm_100a).
+ *
+ * Two device calls make up the hot path, plus host-only helpers:
+ *
+ *   tq_pack_kv       quantize K/V token vectors and write packed rows into
+ *                    persistent uint8 pages (the serving route's write).
+ *   tq_decode_paged  single-token decode attention that reads those pages
+ *                    through a block table without rebuilding the history.
+ *
+ * Pages cited by title and section:
+ *   [Design]  TurboQuant documentation, "Design" page.
+ *   [Server]  TurboQuant Inference Server README.
+ *
+ * Conventions for every call:
+ *   - Pointers named d_* or documented as "device" are CUDA device memory of
+ *     the current device; all others are host memory.
+ *   - The caller owns every buffer, the stream and the workspace. The library
+ *     allocates device memory only inside tq_make_codec (its tables, under
+ *     4 KB), freed by tq_free_codec.
+ *   - Device calls only enqueue work on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and return without synchronizing. Conditions the
+ *     device detects (a slot or block id outside the pool, a bounded wait that
+ *     gave up) are OR-ed into the int32 device word `d_err` (TQ_DERR_* bits)
+ *     when it is not NULL; the kernel then skips the offending access instead
+ *     of faulting. With the environment variable TQ_CHECKED=1 every device call
+ *     synchronizes `stream` and turns a nonzero `d_err` into a status.
+ *   - On error no work is enqueued and tq_last_error() describes the cause
+ *     (thread-local, valid until the next call on the same thread).
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes; the mapping follows the [Design] "Error Model" section. */
+typedef enum {
+    TQ_OK = 0,
+    TQ_ERR_VALUE = 1,       /* ValueError: bad shapes, bit widths, metadata, argument combinations */
+    TQ_ERR_INDEX = 2,       /* IndexError: slot mapping or block id outside the allocated pages */
+    TQ_ERR_NOT_FOUND = 3,   /* FileNotFoundError: missing recipe metadata (raised by loaders) */
+    TQ_ERR_UNSUPPORTED = 4, /* UnsupportedFormatError: the kernels do not implement this format */
+    TQ_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+    TQ_ERR_TIMEOUT = 6      /* a bounded pipeline wait inside a kernel gave up */
+} tq_status;
+
+/* Bits of the device error word. */
+#define TQ_DERR_SLOT 1      /* tq_pack_kv: slot >= num_blocks * block_size (row skipped) */
+#define TQ_DERR_BLOCK 2     /* tq_decode_paged: block table entry outside [0, num_blocks) */
+#define TQ_DERR_TIMEOUT 4   /* a kernel's bounded wait expired; its results are invalid */
+
+/*
+ * One codec (format) for the keys or for the values of a layer.
+ * [Design] "System Invariants": key and value formats are independent, so a
+ * decode call takes two codecs. [Design] "Recipe Strategy": channels split
+ * into a high and a low group, the high group named by sorted calibration
+ * indices; a row stores each group's indices, then the vector norm.
+ *
+ * head_dim       must be 128 on the GPU path (TQ_ERR_UNSUPPORTED otherwise).
+ * num_kv_heads   number of KV heads sharing this codec, 1..1024.
+ * n_groups       1 (uniform) or 2 (high/low mix).
+ * group_bits     bits per index of each group; 2, 3 or 4 on the GPU path.
+ * group_size     coordinates per group; multiples of 16 summing to head_dim.
+ * high_coords    host int16 [num_kv_heads][group_size[0]]: for each KV head,
+ *                the rotated coordinates of group 0, strictly ascending.
+ *                NULL when n_groups == 1. Copied by tq_make_codec.
+ * hadamard_seed  SplitMix64 seed of the sign vector of the rotation.
+ */
+typedef struct {
+    int32_t head_dim;
+    int32_t num_kv_heads;
+    int32_t n_groups;
+    int32_t group_bits[2];
+    int32_t group_size[2];
+    const int16_t* high_coords;
+    uint64_t hadamard_seed;
+} tq_format_desc;
+
+typedef struct tq_codec tq_codec; /* opaque, immutable after tq_make_codec */
+
+/*
+ * Host tables of a codec, for inspection and tests; no CUDA call is made.
+ * Codebook: Lloyd-Max quantizer of one coordinate of a random unit vector in
+ * R^head_dim ([Server] "Codebook caching"), centroids rounded to fp16,
+ * boundaries the fp32 midpoints of adjacent centroids. Rotation:
+ * y = H diag(s) x / sqrt(d), H the natural-order Sylvester matrix,
+ * s_i = -1 when bit 0 of the i-th SplitMix64 output is 1.
+ *
+ * centroids_f16  out, uint16 [2][16]: fp16 bit patterns, ascending, per group
+ * boundaries     out, float  [2][15]
+ * signs          out, int8   [head_dim], +1 or -1
+ * perm           out, int16  [num_kv_heads][head_dim]: packed position ->
+ *                rotated coordinate (group 0 coordinates ascending, then the rest)
+ * row_bytes      out: index bytes of all groups + 2 (fp16 norm)
+ * Any output pointer may be NULL. Returns TQ_ERR_VALUE / TQ_ERR_UNSUPPORTED
+ * for an invalid descriptor (the GPU format limits apply here too).
+ */
+tq_status tq_codec_host_tables(const tq_format_desc* desc, uint16_t* centroids_f16, float* boundaries,
+                               int8_t* signs, int16_t* perm, int32_t* row_bytes);
+
+/*
+ * Validate `desc`, build the codec tables on the host and copy them to the
+ * current device. *out receives the codec; free it with tq_free_codec (not
+ * while kernels that use it are in flight).
+ */
+tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out);
+void tq_free_codec(tq_codec* codec);
+
+/* Bytes of one packed row of this codec (index bytes of every group + 2). */
+int32_t tq_codec_row_bytes(const tq_codec* codec);
+
+/*
+ * tq_pack_kv - the quantize-and-pack write.
+ * [Design] "Serving Route Design": write packed rows into persistent pages;
+ * slot id -> physical block -> token offset -> packed row bytes, with
+ * block = slot / block_size and offset = slot % block_size.
+ *
+ * k, v           device bf16 [num_tokens][num_kv_heads][head_dim], contiguous.
+ * slot_mapping   device int64 [num_tokens]; a negative slot marks a padding
+ *                token, which is skipped.
+ * k_pages        device uint8 [num_blocks][num_kv_heads][block_size][kc row_bytes]
+ * v_pages        device uint8 [num_blocks][num_kv_heads][block_size][vc row_bytes]
+ *                (separate pools that share block ids).
+ * Row of one (token, head): [group-0 bitstream][group-1 bitstream][fp16 norm],
+ * bitstreams LSB-first, the norm little endian; see tq_codec_host_tables for
+ * the rotation and codebook. Each row is written whole; bytes of other rows
+ * are untouched.
+ * Errors: TQ_ERR_VALUE for inconsistent arguments (num_kv_heads or head_dim
+ * differing between the codecs, block_size < 1, null pointers with
+ * num_tokens > 0). A slot >= num_blocks * block_size sets TQ_DERR_SLOT in
+ * d_err and its row is not written ([Design] "Error Model": IndexError).
+ */
+tq_status tq_pack_kv(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
+                     const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
+                     int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream);
+
+/*
+ * Workspace bytes that tq_decode_paged needs for these sizes; bounded by the
+ * runtime shape ([Design] "Serving Route Design": keep workspace bounded).
+ * Returns 0 for invalid sizes.
+ */
+size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,
+                                 int32_t block_size);
+
+/*
+ * tq_decode_paged - single-token decode attention over packed pages.
+ * [Design] "Serving Route Design": use block tables for logical-to-physical
+ * mapping, read K rows inside score computation, read and dequantize V rows
+ * inside accumulation. [Design] "System Invariants": production routes
+ * consume packed historical K/V (no dense rebuild of the history).
+ * [Design] "Format Strategy": recent dense window.
+ *
+ * For sequence b with seq_lens[b] = L_b tokens (window included), the last
+ * n_win = min(window, L_b) tokens are the dense window and the first
+ * P_b = L_b - n_win tokens are packed, logical token i in physical block
+ * block_tables[b][i / block_size] at offset i % block_size.
+ * Query head g reads KV head g / (num_q_heads / num_kv_heads).
+ *
+ * q              device bf16 [batch][num_q_heads][head_dim]
+ * k_pages,
+ * v_pages        as written by tq_pack_kv with the same codecs
+ * block_tables   device int32 [batch][max_blocks_per_seq]; entries past
+ *                ceil(P_b / block_size) are not read
+ * seq_lens       device int32 [batch], 0 <= L_b <= max_seq_len
+ * max_seq_len    host bound on every L_b (sizes the workspace)
+ * k_win, v_win   device bf16 [batch][num_kv_heads][window][head_dim]; slot j
+ *                holds logical token P_b + j for j < n_win. May be NULL when
+ *                window == 0.
+ * softmax_scale  multiplies q.k before the softmax (1/sqrt(128) is usual)
+ * out            device fp32 [batch][num_q_heads][head_dim]; a sequence with
+ *                L_b = 0 gets zeros
+ * workspace      device buffer of at least tq_decode_workspace_bytes(...)
+ *                bytes, 256-byte aligned, owned by the caller; it holds the
+ *                split-K partials and is fully rewritten by each call.
+ * Errors: TQ_ERR_VALUE for inconsistent sizes or a short workspace,
+ * TQ_ERR_UNSUPPORTED for a format the kernels lack. A block id outside
+ * [0, num_blocks) sets TQ_DERR_BLOCK (block 0 is read instead, no fault);
+ * an expired wait sets TQ_DERR_TIMEOUT.
+ */
+tq_status tq_decode_paged(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
+                          const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t max_seq_len,
+                          const void* k_win, const void* v_win, int32_t window, float softmax_scale,
+                          int64_t num_blocks, int32_t block_size, float* out, void* workspace,
+                          size_t workspace_bytes, int32_t* d_err, void* stream);
+
+/*
+ * The two phases of tq_decode_paged, exposed so a caller can time them
+ * apart; tq_decode_paged is exactly tq_decode_partials then tq_decode_combine
+ * on the same stream. tq_decode_partials writes one (max, sum, accumulator)
+ * record per (sequence, KV head, split) into the workspace; tq_decode_combine
+ * merges them by log-sum-exp, undoes the value rotation once per (sequence,
+ * query head) and writes `out`. Arguments mean what they mean above.
+ */
+tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
+                             const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                             const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t max_seq_len,
+                             const void* k_win, const void* v_win, int32_t window, float softmax_scale,
+                             int64_t num_blocks, int32_t block_size, void* workspace, size_t workspace_bytes,
+                             int32_t* d_err, void* stream);
+tq_status tq_decode_combine(const tq_codec* vc, const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                            int32_t max_seq_len, int32_t window, int32_t block_size, float* out,
+                            const void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Byte ledger ([Design] "System Invariants": storage bytes and metadata bytes
+ * are reported separately; the ratio includes norms, codebooks, transforms,
+ * recent windows and workspace). Host arithmetic only.
+ *
+ * dense_bytes        bf16 K and V of every token: 4 * num_kv_heads * head_dim * sum L_b
+ * index_bytes        packed index bytes of the P_b packed tokens, K and V (storage)
+ * norm_bytes         2 bytes per packed row, K and V
+ * codebook_bytes     fp16 centroids + fp32 boundaries of every group of both codecs
+ * transform_bytes    per codec: head_dim int8 signs + num_kv_heads*head_dim int16 permutation
+ * window_bytes       the allocated bf16 windows, K and V
+ * block_table_bytes  one int32 per used block
+ * workspace_bytes    tq_decode_workspace_bytes for these sizes
+ * page_pool_bytes    the allocated K and V page pools (num_blocks blocks)
+ * metadata_bytes     norms + codebooks + transforms + window + block tables + workspace
+ * index_only_ratio   dense_bytes / index_bytes (how the [Server] "What it does" table counts)
+ * all_in_ratio       dense_bytes / (index_bytes + metadata_bytes)
+ */
+typedef struct {
+    int64_t dense_bytes;
+    int64_t index_bytes;
+    int64_t norm_bytes;
+    int64_t codebook_bytes;
+    int64_t transform_bytes;
+    int64_t window_bytes;
+    int64_t block_table_bytes;
+    int64_t workspace_bytes;
+    int64_t page_pool_bytes;
+    int64_t metadata_bytes;
+    double index_only_ratio;
+    double all_in_ratio;
+} tq_ledger;
+
+/* seq_lens is host int32 [batch]. */
+tq_status tq_byte_ledger(const tq_format_desc* kdesc, const tq_format_desc* vdesc, int32_t batch,
+                         const int32_t* seq_lens, int32_t window, int32_t num_q_heads, int32_t block_size,
+                         int64_t num_blocks, int32_t max_seq_len, tq_ledger* out);
+
+/* Message describing the last error on this thread ("" if none). */
+const char* tq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

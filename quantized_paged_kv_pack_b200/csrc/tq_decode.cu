@@ -1,0 +1,396 @@
+// tq_decode_paged: split-K decode attention over packed pages.
+//
+// TurboQuant "Design" page, "Serving Route Design": block tables map logical
+// to physical blocks, K rows are read inside the score computation and V rows
+// are read and dequantized inside the accumulation; "System Invariants": the
+// historical cache is consumed packed, never rebuilt densely.
+//
+// With q_r = pi_K(R_K q) (rotated once per query head, in packed order) and
+// centroids c, the score of packed token t is
+//     s_t = scale * n_K[t] * sum_p q_r[p] c_K[idx_t[p]]            (R orthogonal)
+// and the value accumulator stays in the rotated, packed domain of V:
+//     acc[p] += softmax weight * n_V[t] * c_V[idx_t[p]],
+// so the inverse rotation R_V^T pi_V^-1 runs once per (sequence, query head)
+// in the combine. The bf16 recent window is scored exactly in the original
+// domain and merged through the same log-sum-exp.
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kWarps = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecodeArgs {
+    DevCodec kc, vc;
+    const __nv_bfloat16* q;
+    const uint8_t* k_pages;
+    const uint8_t* v_pages;
+    const int32_t* block_tables;
+    int32_t max_blocks;
+    const int32_t* seq_lens;
+    int32_t batch, num_q_heads, max_seq_len;
+    const __nv_bfloat16* k_win;
+    const __nv_bfloat16* v_win;
+    int32_t window;
+    float scale_log2;  // softmax_scale * log2(e)
+    int64_t num_blocks;
+    int32_t block_size;
+    int32_t split_tokens, max_splits, items_per_unit;
+    float* ws;
+    int* d_err;
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int m = 16; m; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+    return v;
+}
+
+// Index at packed position p of a row (generic bit extraction).
+__device__ __forceinline__ int row_index(const uint8_t* row, const DevCodec& c, int p, int& g) {
+    g = (c.n_groups == 2 && p >= c.pos0[1]) ? 1 : 0;
+    const int b = c.bits[g];
+    const int bit = 8 * c.byte_off[g] + (p - c.pos0[g]) * b;
+    const int byte = bit >> 3, sh = bit & 7;
+    unsigned w = row[byte];
+    if (sh + b > 8) w |= static_cast<unsigned>(row[byte + 1]) << 8;
+    return static_cast<int>((w >> sh) & ((1u << b) - 1u));
+}
+
+__device__ __forceinline__ float row_norm(const uint8_t* row, const DevCodec& c) {
+    unsigned short h = static_cast<unsigned short>(row[c.index_bytes] | (row[c.index_bytes + 1] << 8));
+    return __half2float(__ushort_as_half(h));
+}
+
+// Sequence geometry of item (b, split): returns false when the item is empty.
+__device__ __forceinline__ bool item_range(const DecodeArgs& a, int b, int split, int& t0, int& t1, bool& is_win) {
+    int L = a.seq_lens[b];
+    if (L < 0 || L > a.max_seq_len) {
+        if (a.d_err && threadIdx.x == 0) atomicOr(a.d_err, TQ_DERR_BLOCK);
+        L = L < 0 ? 0 : a.max_seq_len;
+    }
+    const int n_win = min(a.window, L), P = L - n_win;
+    const int ns = (P + a.split_tokens - 1) / a.split_tokens;
+    if (split == a.max_splits) {
+        is_win = true;
+        t0 = 0;
+        t1 = n_win;
+        return n_win > 0;
+    }
+    is_win = false;
+    if (split >= ns) return false;
+    t0 = split * a.split_tokens;
+    t1 = min(P, t0 + a.split_tokens);
+    return true;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs a) {
+    __shared__ float qs[G][kHeadDim];
+    __shared__ float red_m[kWarps][G], red_l[kWarps][G];
+    __shared__ float red_acc[kWarps][G][kHeadDim];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    int t0, t1;
+    bool is_win;
+    if (!item_range(a, b, split, t0, t1, is_win)) return;
+    const int H = a.kc.num_heads;
+
+    // Query prep: q_r = pi_K(H(s_K q)/sqrt(d)) * scale * log2(e) for packed items;
+    // q * scale * log2(e) in the original domain for the window item.
+    for (int g = warp; g < G; g += kWarps) {
+        const __nv_bfloat16* qp = a.q + (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
+        float z[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) z[i] = __bfloat162float(qp[4 * lane + i]);
+        if (is_win) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) qs[g][4 * lane + i] = z[i] * a.scale_log2;
+            continue;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) z[i] *= a.kc.sign[4 * lane + i];
+        {
+            float p0 = z[0] + z[1], p1 = z[0] - z[1], p2 = z[2] + z[3], p3 = z[2] - z[3];
+            z[0] = p0 + p2;
+            z[2] = p0 - p2;
+            z[1] = p1 + p3;
+            z[3] = p1 - p3;
+        }
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float p = __shfl_xor_sync(kFull, z[i], m);
+                z[i] = (lane & m) ? (p - z[i]) : (z[i] + p);
+            }
+        const float sc = a.scale_log2 * 0.08838834764831845f;  // 1/sqrt(128)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) qs[g][a.kc.pos[h * kHeadDim + 4 * lane + i]] = z[i] * sc;
+    }
+    __syncthreads();
+
+    float m[G], l[G], acc[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = -INFINITY;
+        l[g] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[g][i] = 0.0f;
+    }
+    const int bs = a.block_size;
+    for (int t = t0 + warp; t < t1; t += kWarps) {
+        float kv[4], vv[4], nk = 1.0f, nv = 1.0f;
+        if (is_win) {
+            const int64_t base = ((static_cast<int64_t>(b) * H + h) * a.window + t) * kHeadDim + 4 * lane;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                kv[i] = __bfloat162float(a.k_win[base + i]);
+                vv[i] = __bfloat162float(a.v_win[base + i]);
+            }
+        } else {
+            int64_t blk = a.block_tables[static_cast<int64_t>(b) * a.max_blocks + t / bs];
+            if (blk < 0 || blk >= a.num_blocks) {
+                if (a.d_err && lane == 0) atomicOr(a.d_err, TQ_DERR_BLOCK);
+                blk = 0;
+            }
+            const int64_t r = (blk * H + h) * bs + t % bs;
+            const uint8_t* krow = a.k_pages + r * a.kc.row_bytes;
+            const uint8_t* vrow = a.v_pages + r * a.vc.row_bytes;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int g;
+                int ix = row_index(krow, a.kc, 4 * lane + i, g);
+                kv[i] = a.kc.cent[g * 16 + ix];
+                ix = row_index(vrow, a.vc, 4 * lane + i, g);
+                vv[i] = a.vc.cent[g * 16 + ix];
+            }
+            nk = row_norm(krow, a.kc);
+            nv = row_norm(vrow, a.vc);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float s = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s += qs[g][4 * lane + i] * kv[i];
+            s = warp_sum(s) * nk;
+            const float mn = fmaxf(m[g], s);
+            const float alpha = exp2f(m[g] - mn);
+            const float p = exp2f(s - mn);
+            l[g] = l[g] * alpha + p;
+            const float pv = p * nv;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[g][i] = acc[g][i] * alpha + pv * vv[i];
+            m[g] = mn;
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        if (lane == 0) {
+            red_m[warp][g] = m[g];
+            red_l[warp][g] = l[g];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) red_acc[warp][g][4 * lane + i] = acc[g][i];
+    }
+    __syncthreads();
+    float* rec = a.ws + ((static_cast<int64_t>(b) * H + h) * a.items_per_unit + split) *
+                            static_cast<int64_t>(G) * (kHeadDim + 2);
+    for (int e = threadIdx.x; e < G * kHeadDim; e += kWarps * 32) {
+        const int g = e / kHeadDim, j = e - g * kHeadDim;
+        float M = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red_m[w][g]);
+        float L = 0.0f, A = 0.0f;
+        if (M != -INFINITY)
+            for (int w = 0; w < kWarps; ++w) {
+                const float f = exp2f(red_m[w][g] - M);
+                L += red_l[w][g] * f;
+                A += red_acc[w][g][j] * f;
+            }
+        float* rg = rec + g * (kHeadDim + 2);
+        rg[2 + j] = A;
+        if (j == 0) {
+            rg[0] = M;
+            rg[1] = L;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, const int32_t* seq_lens,
+                                                                   int32_t num_q_heads, int32_t max_seq_len,
+                                                                   int32_t window, int32_t split_tokens,
+                                                                   int32_t max_splits, int32_t items_per_unit,
+                                                                   int32_t G, const float* ws, float* out) {
+    __shared__ float y[kHeadDim];
+    const int hq = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
+    const int H = vc.num_heads, h = hq / G, g = hq - h * G;
+    int L = seq_lens[b];
+    L = L < 0 ? 0 : (L > max_seq_len ? max_seq_len : L);
+    const int n_win = min(window, L), P = L - n_win;
+    const int ns = (P + split_tokens - 1) / split_tokens;
+    const float* unit = ws + (static_cast<int64_t>(b) * H + h) * items_per_unit * static_cast<int64_t>(G) * (kHeadDim + 2);
+    auto rec = [&](int i) { return unit + (static_cast<int64_t>(i) * G + g) * (kHeadDim + 2); };
+    float M = -INFINITY;
+    for (int i = 0; i < ns; ++i) M = fmaxf(M, rec(i)[0]);
+    if (n_win) M = fmaxf(M, rec(max_splits)[0]);
+    float Ls = 0.0f, rot = 0.0f, win = 0.0f;
+    if (M != -INFINITY) {
+        for (int i = 0; i < ns; ++i) {
+            const float f = exp2f(rec(i)[0] - M);
+            Ls += rec(i)[1] * f;
+            rot += rec(i)[2 + j] * f;
+        }
+        if (n_win) {
+            const float f = exp2f(rec(max_splits)[0] - M);
+            Ls += rec(max_splits)[1] * f;
+            win = rec(max_splits)[2 + j] * f;
+        }
+    }
+    y[vc.perm[h * kHeadDim + j]] = rot;  // back to rotated coordinate order
+    __syncthreads();
+    for (int len = 1; len < kHeadDim; len <<= 1) {  // Walsh-Hadamard, natural order
+        float mine = y[j], other = y[j ^ len];
+        __syncthreads();
+        y[j] = (j & len) ? (other - mine) : (mine + other);
+        __syncthreads();
+    }
+    const float x = vc.sign[j] * y[j] * 0.08838834764831845f;
+    out[(static_cast<int64_t>(b) * num_q_heads + hq) * kHeadDim + j] = Ls > 0.0f ? (x + win) / Ls : 0.0f;
+}
+
+tq_status check_decode_args(const tq_codec* kc, const tq_codec* vc, int32_t batch, int32_t num_q_heads,
+                            int32_t max_seq_len, int32_t window, int32_t block_size, size_t workspace_bytes,
+                            const void* workspace, SplitPlan* plan) {
+    if (!kc || !vc) return fail(TQ_ERR_VALUE, "null codec");
+    if (kc->desc.num_kv_heads != vc->desc.num_kv_heads || kc->desc.head_dim != vc->desc.head_dim)
+        return fail(TQ_ERR_VALUE, "K and V codecs disagree on num_kv_heads or head_dim");
+    const int H = kc->desc.num_kv_heads;
+    if (batch < 0 || window < 0 || max_seq_len < 0 || block_size < 1)
+        return fail(TQ_ERR_VALUE, "negative size");
+    if (num_q_heads < H || num_q_heads % H) return fail(TQ_ERR_VALUE, "num_q_heads must be a multiple of num_kv_heads");
+    const int G = num_q_heads / H;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
+        return fail(TQ_ERR_UNSUPPORTED, "query heads per KV head must be 1, 2, 4, 8 or 16");
+    if (!make_split_plan(batch, num_q_heads, H, max_seq_len, block_size, plan))
+        return fail(TQ_ERR_VALUE, "invalid decode sizes");
+    if (workspace_bytes < plan->workspace_bytes) return fail(TQ_ERR_VALUE, "workspace smaller than tq_decode_workspace_bytes");
+    if (batch > 0 && !workspace) return fail(TQ_ERR_VALUE, "null workspace");
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(TQ_ERR_VALUE, "workspace must be 256-byte aligned");
+    return TQ_OK;
+}
+
+tq_status finish(cudaStream_t s, int32_t* d_err, const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(TQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+    if (checked_mode()) {
+        if ((e = cudaStreamSynchronize(s)) != cudaSuccess)
+            return fail(TQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+        if (d_err) {
+            int32_t h = 0;
+            if (cudaMemcpy(&h, d_err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+                return fail(TQ_ERR_CUDA, "reading the device error word failed");
+            if (h & TQ_DERR_TIMEOUT) return fail(TQ_ERR_TIMEOUT, "a bounded wait in the decode kernel expired");
+            if (h & TQ_DERR_BLOCK) return fail(TQ_ERR_INDEX, "block table entry or length outside the pages");
+        }
+    }
+    return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
+                                        const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                        const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                        int32_t max_seq_len, const void* k_win, const void* v_win, int32_t window,
+                                        float softmax_scale, int64_t num_blocks, int32_t block_size,
+                                        void* workspace, size_t workspace_bytes, int32_t* d_err, void* stream) {
+    clear_error();
+    SplitPlan plan;
+    tq_status st = check_decode_args(kc, vc, batch, num_q_heads, max_seq_len, window, block_size, workspace_bytes,
+                                     workspace, &plan);
+    if (st != TQ_OK) return st;
+    if (batch == 0) return TQ_OK;
+    if (!q || !seq_lens || (max_seq_len > window && (!k_pages || !v_pages || !block_tables)))
+        return fail(TQ_ERR_VALUE, "null buffer");
+    if (window > 0 && (!k_win || !v_win)) return fail(TQ_ERR_VALUE, "window > 0 needs k_win and v_win");
+    if (num_blocks < 0 || max_blocks_per_seq < 0) return fail(TQ_ERR_VALUE, "negative size");
+    if (static_cast<int64_t>(max_blocks_per_seq) * block_size < static_cast<int64_t>(max_seq_len) - window)
+        return fail(TQ_ERR_VALUE, "max_blocks_per_seq * block_size cannot hold max_seq_len - window tokens");
+    DecodeArgs a;
+    a.kc = kc->dev;
+    a.vc = vc->dev;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k_pages = static_cast<const uint8_t*>(k_pages);
+    a.v_pages = static_cast<const uint8_t*>(v_pages);
+    a.block_tables = block_tables;
+    a.max_blocks = max_blocks_per_seq;
+    a.seq_lens = seq_lens;
+    a.batch = batch;
+    a.num_q_heads = num_q_heads;
+    a.max_seq_len = max_seq_len;
+    a.k_win = static_cast<const __nv_bfloat16*>(k_win);
+    a.v_win = static_cast<const __nv_bfloat16*>(v_win);
+    a.window = window;
+    a.scale_log2 = softmax_scale * kLog2e;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    a.split_tokens = plan.split_tokens;
+    a.max_splits = plan.max_splits;
+    a.items_per_unit = plan.items_per_unit;
+    a.ws = static_cast<float*>(workspace);
+    a.d_err = d_err;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dim3 grid(plan.items_per_unit, kc->desc.num_kv_heads, batch);
+    switch (plan.group) {
+        case 1: decode_partials_kernel<1><<<grid, kWarps * 32, 0, s>>>(a); break;
+        case 2: decode_partials_kernel<2><<<grid, kWarps * 32, 0, s>>>(a); break;
+        case 4: decode_partials_kernel<4><<<grid, kWarps * 32, 0, s>>>(a); break;
+        case 8: decode_partials_kernel<8><<<grid, kWarps * 32, 0, s>>>(a); break;
+        default: decode_partials_kernel<16><<<grid, kWarps * 32, 0, s>>>(a); break;
+    }
+    return finish(s, d_err, "decode partials");
+}
+
+extern "C" tq_status tq_decode_combine(const tq_codec* vc, const int32_t* seq_lens, int32_t batch,
+                                       int32_t num_q_heads, int32_t max_seq_len, int32_t window, int32_t block_size,
+                                       float* out, const void* workspace, size_t workspace_bytes, void* stream) {
+    clear_error();
+    SplitPlan plan;
+    tq_status st = check_decode_args(vc, vc, batch, num_q_heads, max_seq_len, window, block_size, workspace_bytes,
+                                     workspace, &plan);
+    if (st != TQ_OK) return st;
+    if (batch == 0) return TQ_OK;
+    if (!out || !seq_lens) return fail(TQ_ERR_VALUE, "null buffer");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    decode_combine_kernel<<<dim3(num_q_heads, batch), kHeadDim, 0, s>>>(
+        vc->dev, seq_lens, num_q_heads, max_seq_len, window, plan.split_tokens, plan.max_splits,
+        plan.items_per_unit, plan.group, static_cast<const float*>(workspace), out);
+    return finish(s, nullptr, "decode combine");
+}
+
+extern "C" tq_status tq_decode_paged(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
+                                     const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                     int32_t max_seq_len, const void* k_win, const void* v_win, int32_t window,
+                                     float softmax_scale, int64_t num_blocks, int32_t block_size, float* out,
+                                     void* workspace, size_t workspace_bytes, int32_t* d_err, void* stream) {
+    tq_status st = tq_decode_partials(kc, vc, q, k_pages, v_pages, block_tables, max_blocks_per_seq, seq_lens, batch,
+                                      num_q_heads, max_seq_len, k_win, v_win, window, softmax_scale, num_blocks,
+                                      block_size, workspace, workspace_bytes, d_err, stream);
+    if (st != TQ_OK) return st;
+    return tq_decode_combine(vc, seq_lens, batch, num_q_heads, max_seq_len, window, block_size, out, workspace,
+                             workspace_bytes, stream);
+}

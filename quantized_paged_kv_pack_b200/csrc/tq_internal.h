@@ -1,0 +1,78 @@
+// Internal declarations shared by the host codec and the CUDA kernels of libtq.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "tq.h"
+
+namespace tq {
+
+constexpr int kHeadDim = 128;   // the only head_dim the kernels implement
+constexpr int kMaxHeads = 1024;
+constexpr int kMaxLevels = 16;  // 4-bit codebooks at most on the GPU path
+
+// Device-side view of one codec, passed to kernels by value.
+struct DevCodec {
+    const float* sign;      // [128] +1 / -1
+    const float* cent;      // [2][16] centroids (fp16-exact values)
+    const float* bound;     // [2][16] boundaries, 15 used, entry 15 = +inf
+    const int16_t* perm;    // [H][128] packed position -> rotated coordinate
+    const int16_t* pos;     // [H][128] rotated coordinate -> packed position
+    int32_t num_heads;
+    int32_t n_groups;
+    int32_t bits[2];
+    int32_t size[2];
+    int32_t pos0[2];        // first packed position of each group
+    int32_t byte_off[2];    // byte offset of each group's bitstream in the row
+    int32_t index_bytes;
+    int32_t row_bytes;
+};
+
+}  // namespace tq
+
+struct tq_codec {
+    tq_format_desc desc;
+    std::vector<int16_t> high;     // owned copy of desc.high_coords
+    uint16_t cent16[2][16];
+    float cent[2][16];
+    float bound[2][16];
+    float sign[tq::kHeadDim];
+    std::vector<int16_t> perm;     // [H][d]
+    std::vector<int16_t> pos;      // [H][d]
+    int32_t row_bytes = 0;
+    int32_t index_bytes = 0;
+    int device = 0;
+    void* d_tables = nullptr;
+    tq::DevCodec dev{};
+};
+
+namespace tq {
+
+// Sets the thread-local error message and returns `st`.
+tq_status fail(tq_status st, const std::string& msg);
+void clear_error();
+
+// Validates a descriptor against the GPU format limits.
+tq_status validate_desc(const tq_format_desc* desc);
+
+// Builds every host table of a codec (no CUDA call).
+tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c);
+
+// True when TQ_CHECKED=1 is set in the environment.
+bool checked_mode();
+
+// Decode split-K geometry shared by the workspace sizing and the kernels.
+struct SplitPlan {
+    int32_t split_tokens;   // packed tokens per work item (multiple of block_size)
+    int32_t max_splits;     // packed work items per (sequence, KV head)
+    int32_t items_per_unit; // max_splits + 1 (the last one is the window)
+    int32_t group;          // query heads per KV head
+    size_t record_floats;   // floats per work item record
+    size_t workspace_bytes;
+};
+bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,
+                     int32_t block_size, SplitPlan* plan);
+
+}  // namespace tq

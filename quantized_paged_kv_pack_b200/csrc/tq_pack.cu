@@ -1,0 +1,193 @@
+// tq_pack_kv: quantize-and-pack write of K/V token vectors into uint8 pages.
+//
+// TurboQuant "Design" page, "Serving Route Design": the serving route writes
+// packed rows into persistent pages addressed slot -> physical block -> token
+// offset -> row bytes, block = slot / block_size, offset = slot % block_size.
+// Per (token, head) vector x (bf16, 128 values):
+//   n   = ||x||_2, stored as fp16 (round to nearest even)
+//   z   = H (s * x)              Sylvester Walsh-Hadamard, signs s of the codec
+//   u   = z / (sqrt(128) n)      the rotated unit vector
+//   idx = #{boundaries of its group below u_j}, placed at packed position pos[h][j]
+//   row = [group-0 bitstream][group-1 bitstream][n16], LSB-first.
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kPackWarps = 8;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int m = 16; m; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int m = 16; m; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+    return v;
+}
+
+// fp16 bits of the norm, equal to the correctly rounded fp16 of the exact norm.
+// The fp32 sum of exact squares is within 5e-7 (relative) of the exact sum, so
+// its square root decides the rounding unless it lies within 1e-6 of an fp16
+// rounding midpoint, or the fp32 sum under- or overflows; then the warp
+// recomputes the sum in fp64 and `n32` is replaced by that norm.
+__device__ __forceinline__ unsigned short norm_fp16_bits(const float (&x)[4], float ss, float& n32) {
+    bool risky = !(ss > 1e-30f && ss < 1e30f) || n32 > 60000.0f;
+    __half h = __float2half_rn(n32);
+    unsigned short hb = __half_as_ushort(h);
+    if (!risky) {
+        float hf = __half2float(h);
+        float up = __half2float(__ushort_as_half(static_cast<unsigned short>(hb + 1)));
+        float dn = __half2float(__ushort_as_half(static_cast<unsigned short>(hb - 1)));
+        float tol = 1e-6f * n32;
+        risky = fabsf(n32 - 0.5f * (hf + up)) <= tol || fabsf(n32 - 0.5f * (hf + dn)) <= tol;
+    }
+    if (risky) {  // warp-uniform: ss and n32 are warp-wide values
+        double sd = 0.0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sd += static_cast<double>(x[i]) * static_cast<double>(x[i]);
+        sd = warp_sum_d(sd);
+        const double nd = sqrt(sd);
+        hb = __half_as_ushort(__double2half(nd));
+        n32 = static_cast<float>(nd);
+    }
+    return hb;
+}
+
+__global__ void __launch_bounds__(kPackWarps * 32)
+pack_rows_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__ k,
+                 const __nv_bfloat16* __restrict__ v, const int64_t* __restrict__ slots, int64_t num_tokens,
+                 uint8_t* __restrict__ k_pages, uint8_t* __restrict__ v_pages, int64_t num_blocks,
+                 int block_size, int* __restrict__ d_err) {
+    __shared__ uint8_t idx_buf[kPackWarps][kHeadDim];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t H = kc.num_heads;
+    const int64_t n_vec = num_tokens * H * 2;
+    const int64_t capacity = num_blocks * block_size;
+    for (int64_t vec = static_cast<int64_t>(blockIdx.x) * kPackWarps + warp; vec < n_vec;
+         vec += static_cast<int64_t>(gridDim.x) * kPackWarps) {
+        const int which = static_cast<int>(vec & 1);
+        const int64_t th = vec >> 1;
+        const int64_t t = th / H;
+        const int h = static_cast<int>(th - t * H);
+        const int64_t slot = slots[t];
+        if (slot < 0) continue;
+        if (slot >= capacity) {
+            if (lane == 0 && d_err) atomicOr(d_err, TQ_DERR_SLOT);
+            continue;
+        }
+        const DevCodec& c = which ? vc : kc;
+        const __nv_bfloat16* src = (which ? v : k) + th * kHeadDim + 4 * lane;
+        uint2 raw = *reinterpret_cast<const uint2*>(src);
+        float x[4];
+        x[0] = __uint_as_float(raw.x << 16);
+        x[1] = __uint_as_float(raw.x & 0xffff0000u);
+        x[2] = __uint_as_float(raw.y << 16);
+        x[3] = __uint_as_float(raw.y & 0xffff0000u);
+
+        float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
+        float n32 = sqrtf(ss);
+        unsigned short n16 = norm_fp16_bits(x, ss, n32);
+
+        float z[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) z[i] = x[i] * c.sign[4 * lane + i];
+        {
+            float a = z[0] + z[1], b = z[0] - z[1], cc = z[2] + z[3], d = z[2] - z[3];
+            z[0] = a + cc;
+            z[2] = a - cc;
+            z[1] = b + d;
+            z[3] = b - d;
+        }
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float p = __shfl_xor_sync(kFull, z[i], m);
+                z[i] = (lane & m) ? (p - z[i]) : (z[i] + p);
+            }
+        }
+        const float inv = n32 > 0.0f ? 1.0f / (n32 * 11.313708498984761f) : 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = 4 * lane + i;
+            const int p = c.pos[h * kHeadDim + j];
+            const int g = (c.n_groups == 2 && p >= c.pos0[1]) ? 1 : 0;
+            const float u = z[i] * inv;
+            const int levels = 1 << c.bits[g];
+            int idx = 0;
+            for (int q = 0; q < levels - 1; ++q) idx += (c.bound[g * 16 + q] < u) ? 1 : 0;
+            idx_buf[warp][p] = static_cast<uint8_t>(idx);
+        }
+        __syncwarp();
+        const int half_words = c.index_bytes / 2;
+        unsigned word = 0;
+        if (lane < half_words) {
+            for (int i = 0; i < 16; ++i) {
+                const int B = 16 * lane + i;
+                const int g = (c.n_groups == 2 && B >= 8 * c.byte_off[1]) ? 1 : 0;
+                const int lb = B - 8 * c.byte_off[g];
+                const int b = c.bits[g];
+                const int q = lb / b, r = lb - q * b;
+                word |= ((idx_buf[warp][c.pos0[g] + q] >> r) & 1u) << i;
+            }
+        }
+        const int64_t blk = slot / block_size, off = slot - blk * block_size;
+        uint8_t* pages = which ? v_pages : k_pages;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(pages + ((blk * H + h) * block_size + off) * c.row_bytes);
+        if (lane < half_words) dst[lane] = static_cast<uint16_t>(word);
+        if (lane == 0) dst[half_words] = n16;
+        __syncwarp();
+    }
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" tq_status tq_pack_kv(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
+                                const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
+                                int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream) {
+    clear_error();
+    if (!kc || !vc) return fail(TQ_ERR_VALUE, "null codec");
+    if (kc->desc.num_kv_heads != vc->desc.num_kv_heads || kc->desc.head_dim != vc->desc.head_dim)
+        return fail(TQ_ERR_VALUE, "K and V codecs disagree on num_kv_heads or head_dim");
+    if (num_tokens < 0 || num_blocks < 0 || block_size < 1) return fail(TQ_ERR_VALUE, "negative size");
+    if (num_tokens == 0) return TQ_OK;
+    if (!k || !v || !slot_mapping || !k_pages || !v_pages) return fail(TQ_ERR_VALUE, "null buffer");
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 7)
+        return fail(TQ_ERR_VALUE, "k and v must be 8-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 1)
+        return fail(TQ_ERR_VALUE, "page pools must be 2-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t n_vec = num_tokens * kc->desc.num_kv_heads * 2;
+    const int64_t blocks = std::min<int64_t>((n_vec + kPackWarps - 1) / kPackWarps, 148 * 32);
+    pack_rows_kernel<<<static_cast<unsigned>(blocks), kPackWarps * 32, 0, s>>>(
+        kc->dev, vc->dev, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        slot_mapping, num_tokens, static_cast<uint8_t*>(k_pages), static_cast<uint8_t*>(v_pages), num_blocks,
+        block_size, d_err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(TQ_ERR_CUDA, std::string("pack launch: ") + cudaGetErrorString(e));
+    if (checked_mode()) {
+        if ((e = cudaStreamSynchronize(s)) != cudaSuccess)
+            return fail(TQ_ERR_CUDA, std::string("pack: ") + cudaGetErrorString(e));
+        if (d_err) {
+            int32_t h = 0;
+            if (cudaMemcpy(&h, d_err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+                return fail(TQ_ERR_CUDA, "reading the device error word failed");
+            if (h & TQ_DERR_SLOT) return fail(TQ_ERR_INDEX, "slot mapping points outside the allocated pages");
+        }
+    }
+    return TQ_OK;
+}

@@ -1,0 +1,330 @@
+"""Thin ctypes binding of libtq (include/tq.h): argument marshalling only.
+
+Every step of the pack and decode path runs in the CUDA library; this module
+checks tensor dtypes, shapes and devices, passes raw pointers and the current
+CUDA stream, and maps status codes to exceptions following the TurboQuant
+"Design" page, "Error Model" (ValueError, IndexError, FileNotFoundError,
+UnsupportedFormatError). There is no fallback: if libtq.so is missing or no
+CUDA device is present, the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import json
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_OK, TQ_ERR_VALUE, TQ_ERR_INDEX, TQ_ERR_NOT_FOUND, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_TIMEOUT = range(7)
+TQ_DERR_SLOT, TQ_DERR_BLOCK, TQ_DERR_TIMEOUT = 1, 2, 4
+HEAD_DIM = 128
+
+
+class UnsupportedFormatError(Exception):
+    """The kernels do not implement the requested format (no silent fallback)."""
+
+
+class TQTimeoutError(RuntimeError):
+    """A bounded wait inside a kernel expired."""
+
+
+class TQCudaError(RuntimeError):
+    """A CUDA runtime call inside the library failed."""
+
+
+class _FormatDesc(ctypes.Structure):
+    _fields_ = [("head_dim", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("n_groups", ctypes.c_int32),
+                ("group_bits", ctypes.c_int32 * 2), ("group_size", ctypes.c_int32 * 2),
+                ("high_coords", ctypes.POINTER(ctypes.c_int16)), ("hadamard_seed", ctypes.c_uint64)]
+
+
+class _Ledger(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "dense_bytes", "index_bytes", "norm_bytes", "codebook_bytes", "transform_bytes", "window_bytes",
+        "block_table_bytes", "workspace_bytes", "page_pool_bytes", "metadata_bytes")] + \
+        [("index_only_ratio", ctypes.c_double), ("all_in_ratio", ctypes.c_double)]
+
+
+_lib = None
+_VP, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+
+def lib():
+    """Load libtq.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with quantized_paged_kv_pack_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER
+        L.tq_last_error.restype = ctypes.c_char_p
+        L.tq_codec_host_tables.argtypes = [P(_FormatDesc), _VP, _VP, _VP, _VP, _VP]
+        L.tq_make_codec.argtypes = [P(_FormatDesc), P(_VP)]
+        L.tq_free_codec.argtypes = [_VP]
+        L.tq_free_codec.restype = None
+        L.tq_codec_row_bytes.argtypes = [_VP]
+        L.tq_codec_row_bytes.restype = _I32
+        L.tq_pack_kv.argtypes = [_VP, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _I64, _I32, _VP, _VP]
+        L.tq_decode_workspace_bytes.argtypes = [_I32, _I32, _I32, _I32, _I32]
+        L.tq_decode_workspace_bytes.restype = _SZ
+        dec = [_VP, _VP, _VP, _VP, _VP, _VP, _I32, _VP, _I32, _I32, _I32, _VP, _VP, _I32, ctypes.c_float, _I64, _I32]
+        L.tq_decode_paged.argtypes = dec + [_VP, _VP, _SZ, _VP, _VP]
+        L.tq_decode_partials.argtypes = dec + [_VP, _SZ, _VP, _VP]
+        L.tq_decode_combine.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _SZ, _VP]
+        L.tq_byte_ledger.argtypes = [P(_FormatDesc), P(_FormatDesc), _I32, _VP, _I32, _I32, _I32, _I64, _I32,
+                                     P(_Ledger)]
+        for name in ("tq_codec_host_tables", "tq_make_codec", "tq_pack_kv", "tq_decode_paged",
+                     "tq_decode_partials", "tq_decode_combine", "tq_byte_ledger"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status == TQ_OK:
+        return
+    msg = lib().tq_last_error().decode()
+    if status == TQ_ERR_VALUE:
+        raise ValueError(msg)
+    if status == TQ_ERR_INDEX:
+        raise IndexError(msg)
+    if status == TQ_ERR_NOT_FOUND:
+        raise FileNotFoundError(msg)
+    if status == TQ_ERR_UNSUPPORTED:
+        raise UnsupportedFormatError(msg)
+    if status == TQ_ERR_TIMEOUT:
+        raise TQTimeoutError(msg)
+    raise TQCudaError(msg or f"tq status {status}")
+
+
+def _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed):
+    bits, sizes = tuple(group_bits), tuple(group_size)
+    d = _FormatDesc()
+    d.head_dim, d.num_kv_heads, d.n_groups = head_dim, num_kv_heads, len(bits)
+    if len(bits) not in (1, 2) or len(sizes) != len(bits):
+        raise ValueError("one or two channel groups with matching sizes")
+    for i in range(len(bits)):
+        d.group_bits[i], d.group_size[i] = bits[i], sizes[i]
+    keep = None
+    if high_coords is not None:
+        keep = np.ascontiguousarray(np.asarray(high_coords, dtype=np.int16))
+        d.high_coords = keep.ctypes.data_as(ctypes.POINTER(ctypes.c_int16))
+    d.hadamard_seed = int(seed) & ((1 << 64) - 1)
+    return d, keep
+
+
+def codec_host_tables(head_dim, num_kv_heads, group_bits, group_size, high_coords=None, seed=0):
+    """Host-side codec tables (no CUDA call): codebooks, signs, permutation, row bytes."""
+    d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed)
+    c16 = np.zeros((2, 16), np.uint16)
+    bnd = np.zeros((2, 15), np.float32)
+    sg = np.zeros(head_dim, np.int8)
+    perm = np.zeros((num_kv_heads, head_dim), np.int16)
+    rb = ctypes.c_int32()
+    _check(lib().tq_codec_host_tables(ctypes.byref(d), c16.ctypes.data, bnd.ctypes.data, sg.ctypes.data,
+                                      perm.ctypes.data, ctypes.addressof(rb)))
+    del keep
+    return {"centroids_f16": c16, "boundaries": bnd, "signs": sg, "perm": perm, "row_bytes": rb.value}
+
+
+class Codec:
+    """A device codec (tq_make_codec); immutable, freed on close()."""
+
+    def __init__(self, num_kv_heads: int, group_bits: Sequence[int], group_size: Sequence[int],
+                 high_coords=None, seed: int = 0, head_dim: int = HEAD_DIM):
+        self.head_dim, self.num_kv_heads = head_dim, num_kv_heads
+        self.group_bits, self.group_size, self.seed = tuple(group_bits), tuple(group_size), seed
+        self.high_coords = None if high_coords is None else np.asarray(high_coords, dtype=np.int16)
+        d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed)
+        h = _VP()
+        _check(lib().tq_make_codec(ctypes.byref(d), ctypes.byref(h)))
+        del keep
+        self._h = h
+        self.row_bytes = lib().tq_codec_row_bytes(h)
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise ValueError("codec is closed")
+        return self._h
+
+    def desc(self):
+        return _desc(self.head_dim, self.num_kv_heads, self.group_bits, self.group_size, self.high_coords, self.seed)
+
+    def close(self):
+        if getattr(self, "_h", None) is not None:
+            lib().tq_free_codec(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def load_recipe_metadata(path: str) -> dict:
+    """Read a recipe metadata JSON (sorted high-precision channel indices per KV head).
+
+    TurboQuant "Design" page, "Recipe Strategy": activation energy -> sorted
+    high-precision indices -> metadata JSON; runtime loads and validates it.
+    "Error Model": a missing file raises FileNotFoundError. The keys are
+    head_dim, num_kv_heads, group_bits, group_size, high_coords, hadamard_seed.
+    """
+    if not os.path.exists(path):
+        raise FileNotFoundError(f"recipe metadata not found: {path}")
+    with open(path) as f:
+        meta = json.load(f)
+    try:
+        spec = dict(head_dim=int(meta["head_dim"]), num_kv_heads=int(meta["num_kv_heads"]),
+                    group_bits=tuple(meta["group_bits"]), group_size=tuple(meta["group_size"]),
+                    high_coords=None if meta.get("high_coords") is None else np.asarray(meta["high_coords"], np.int16),
+                    seed=int(meta.get("hadamard_seed", 0)))
+    except (KeyError, TypeError) as e:
+        raise ValueError(f"malformed recipe metadata: {e}") from e
+    codec_host_tables(spec["head_dim"], spec["num_kv_heads"], spec["group_bits"], spec["group_size"],
+                      spec["high_coords"], spec["seed"])  # validates
+    return spec
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, shape, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def page_pool(codec: Codec, num_blocks: int, block_size: int, device="cuda") -> torch.Tensor:
+    """Zeroed uint8 pool [num_blocks][H_kv][block_size][row_bytes]."""
+    return torch.zeros(num_blocks, codec.num_kv_heads, block_size, codec.row_bytes, dtype=torch.uint8, device=device)
+
+
+def pack_kv(kc: Codec, vc: Codec, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+            k_pages: torch.Tensor, v_pages: torch.Tensor, d_err: Optional[torch.Tensor] = None, stream=None):
+    """Quantize and write K/V rows into the page pools (tq_pack_kv)."""
+    T = k.shape[0] if k.dim() == 3 else -1
+    H = kc.num_kv_heads
+    _need(k, torch.bfloat16, (T, H, kc.head_dim), "k")
+    _need(v, torch.bfloat16, (T, H, kc.head_dim), "v")
+    _need(slot_mapping, torch.int64, (T,), "slot_mapping")
+    if k_pages.dim() != 4:
+        raise ValueError("page pools must be [num_blocks][H_kv][block_size][row_bytes]")
+    nb, _, bs, _ = k_pages.shape
+    _need(k_pages, torch.uint8, (nb, H, bs, kc.row_bytes), "k_pages")
+    _need(v_pages, torch.uint8, (nb, H, bs, vc.row_bytes), "v_pages")
+    if d_err is not None:
+        _need(d_err, torch.int32, (1,), "d_err")
+    _check(lib().tq_pack_kv(kc.handle, vc.handle, _ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_pages),
+                            _ptr(v_pages), nb, bs, _ptr(d_err), _stream(stream)))
+
+
+def decode_workspace_bytes(batch: int, num_q_heads: int, num_kv_heads: int, max_seq_len: int, block_size: int) -> int:
+    return int(lib().tq_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, max_seq_len, block_size))
+
+
+def alloc_workspace(batch, num_q_heads, num_kv_heads, max_seq_len, block_size, device="cuda") -> torch.Tensor:
+    n = decode_workspace_bytes(batch, num_q_heads, num_kv_heads, max_seq_len, block_size)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def decode_paged(kc: Codec, vc: Codec, q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                 block_tables: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
+                 k_win: Optional[torch.Tensor], v_win: Optional[torch.Tensor], window: int,
+                 softmax_scale: float, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 d_err: Optional[torch.Tensor] = None, stream=None, phase: str = "all") -> torch.Tensor:
+    """Decode attention over packed pages (tq_decode_paged); returns fp32 [B][H_q][d].
+
+    ``phase`` is "all" (tq_decode_paged), "partials" or "combine" (the two
+    halves, for timing them apart).
+    """
+    if q.dim() != 3:
+        raise ValueError("q must be [batch][num_q_heads][head_dim]")
+    B, Hq, d = q.shape
+    H = kc.num_kv_heads
+    _need(q, torch.bfloat16, (B, Hq, kc.head_dim), "q")
+    if k_pages.dim() != 4:
+        raise ValueError("page pools must be [num_blocks][H_kv][block_size][row_bytes]")
+    nb, _, bs, _ = k_pages.shape
+    _need(k_pages, torch.uint8, (nb, H, bs, kc.row_bytes), "k_pages")
+    _need(v_pages, torch.uint8, (nb, H, bs, vc.row_bytes), "v_pages")
+    if block_tables.dim() != 2:
+        raise ValueError("block_tables must be [batch][max_blocks_per_seq]")
+    _need(block_tables, torch.int32, (B, block_tables.shape[1]), "block_tables")
+    _need(seq_lens, torch.int32, (B,), "seq_lens")
+    if window > 0:
+        _need(k_win, torch.bfloat16, (B, H, window, kc.head_dim), "k_win")
+        _need(v_win, torch.bfloat16, (B, H, window, kc.head_dim), "v_win")
+    else:
+        k_win = v_win = None
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, (B, Hq, d), "out")
+    if workspace is None:
+        workspace = alloc_workspace(B, Hq, H, max_seq_len, bs, device=q.device)
+    if d_err is not None:
+        _need(d_err, torch.int32, (1,), "d_err")
+    L, s = lib(), _stream(stream)
+    common = (kc.handle, vc.handle, _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), block_tables.shape[1],
+              _ptr(seq_lens), B, Hq, int(max_seq_len), _ptr(k_win), _ptr(v_win), int(window), float(softmax_scale),
+              nb, bs)
+    ws = (_ptr(workspace), workspace.numel())
+    if phase == "all":
+        _check(L.tq_decode_paged(*common, _ptr(out), *ws, _ptr(d_err), s))
+    elif phase == "partials":
+        _check(L.tq_decode_partials(*common, *ws, _ptr(d_err), s))
+    elif phase == "combine":
+        _check(L.tq_decode_combine(vc.handle, _ptr(seq_lens), B, Hq, int(max_seq_len), int(window), bs, _ptr(out),
+                                   *ws, s))
+    else:
+        raise ValueError(f"unknown phase {phase!r}")
+    return out
+
+
+def byte_ledger(kc: Codec, vc: Codec, seq_lens: Sequence[int], window: int, num_q_heads: int, block_size: int,
+                num_blocks: int, max_seq_len: Optional[int] = None) -> dict:
+    """tq_byte_ledger for the host lengths ``seq_lens``; storage and metadata reported apart."""
+    lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    max_seq_len = int(lens.max()) if max_seq_len is None and len(lens) else int(max_seq_len or 0)
+    kd, kkeep = kc.desc()
+    vd, vkeep = vc.desc()
+    r = _Ledger()
+    _check(lib().tq_byte_ledger(ctypes.byref(kd), ctypes.byref(vd), len(lens), lens.ctypes.data, window, num_q_heads,
+                                block_size, num_blocks, max_seq_len, ctypes.byref(r)))
+    del kkeep, vkeep
+    return {name: getattr(r, name) for name, _ in _Ledger._fields_}
+
+
+def host_ledger(num_kv_heads, kspec: dict, vspec: dict, seq_lens, window, num_q_heads, block_size, num_blocks,
+                max_seq_len=None) -> dict:
+    """tq_byte_ledger from plain codec parameters (no device needed)."""
+    lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    max_seq_len = int(lens.max()) if max_seq_len is None and len(lens) else int(max_seq_len or 0)
+    kd, kkeep = _desc(HEAD_DIM, num_kv_heads, kspec["group_bits"], kspec["group_size"], kspec.get("high_coords"),
+                      kspec.get("seed", 0))
+    vd, vkeep = _desc(HEAD_DIM, num_kv_heads, vspec["group_bits"], vspec["group_size"], vspec.get("high_coords"),
+                      vspec.get("seed", 0))
+    r = _Ledger()
+    _check(lib().tq_byte_ledger(ctypes.byref(kd), ctypes.byref(vd), len(lens), lens.ctypes.data, window, num_q_heads,
+                                block_size, num_blocks, max_seq_len, ctypes.byref(r)))
+    del kkeep, vkeep
+    return {name: getattr(r, name) for name, _ in _Ledger._fields_}

@@ -1,0 +1,126 @@
+"""Shared test helpers: build both sides' codecs from plain specs, make decode problems."""
+
+import math
+
+import numpy as np
+import torch
+
+from oracle import tq_oracle as O
+from quantized_paged_kv_pack_b200 import tq
+from quantized_paged_kv_pack_b200 import workloads as W
+
+D = 128
+
+
+def random_high(H, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.stack([np.sort(rng.choice(D, n, replace=False)) for _ in range(H)]).astype(np.int16)
+
+
+def codec_pair(H, bits, sizes, seed, high=None):
+    """(device Codec, oracle Format) for the same plain parameters."""
+    if len(bits) == 2 and high is None:
+        high = random_high(H, sizes[0], seed + 17)
+    return tq.Codec(H, bits, sizes, high, seed), O.Format(D, H, tuple(bits), tuple(sizes), high, seed)
+
+
+def slice_format(f: O.Format, h: int) -> O.Format:
+    """The oracle format of KV head h alone (metadata sliced to one head)."""
+    hc = None if f.high_coords is None else np.asarray(f.high_coords)[h:h + 1]
+    return O.Format(f.head_dim, 1, f.group_bits, f.group_size, hc, f.seed)
+
+
+def random_kv(T, H, gen, scale_outliers=True):
+    """bf16 K/V [T][H][128] on the GPU: N(0,1), some channels x10, per-vector scales."""
+    k = torch.randn(T, H, D, generator=gen, device="cuda")
+    v = torch.randn(T, H, D, generator=gen, device="cuda")
+    if scale_outliers:
+        k[:, :, :4] *= 10
+        v[:, :, 5:9] *= 10
+        k *= torch.exp(torch.rand(T, H, 1, generator=gen, device="cuda") * math.log(8) + math.log(0.5))
+        v *= torch.exp(torch.rand(T, H, 1, generator=gen, device="cuda") * math.log(8) + math.log(0.5))
+    return k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+class DecodeProblem:
+    """A paged cache written by the GPU pack kernel, plus queries and windows."""
+
+    def __init__(self, lens, H, G, kspec, vspec, window, block_size, seed, slack=1.3):
+        self.lens = np.asarray(lens, dtype=np.int64)
+        self.B, self.H, self.G, self.Hq = len(lens), H, G, H * G
+        self.window, self.bs = window, block_size
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(seed)
+        rng = np.random.default_rng(seed)
+        self.kc, self.kf = codec_pair(H, *kspec)
+        self.vc, self.vf = codec_pair(H, *vspec)
+        packed = self.lens - np.minimum(window, self.lens)
+        nblk = -(-packed // block_size)
+        self.num_blocks = max(1, int(math.ceil(slack * nblk.sum())) + 1)
+        order = rng.permutation(self.num_blocks)
+        self.max_blocks = max(1, int(nblk.max()) if len(nblk) else 1)
+        bt = np.full((self.B, self.max_blocks), -1, np.int32)
+        pos = 0
+        for b in range(self.B):
+            bt[b, :nblk[b]] = order[pos:pos + nblk[b]]
+            pos += nblk[b]
+        self.block_tables_np = bt
+        self.k_pages = tq.page_pool(self.kc, self.num_blocks, block_size)
+        self.v_pages = tq.page_pool(self.vc, self.num_blocks, block_size)
+        Wn = max(window, 1)
+        self.k_win = torch.zeros(self.B, H, Wn, D, dtype=torch.bfloat16, device="cuda")
+        self.v_win = torch.zeros_like(self.k_win)
+        for b in range(self.B):
+            L, P = int(self.lens[b]), int(packed[b])
+            k, v = random_kv(L, H, gen)
+            if P:
+                t = np.arange(P)
+                slots = torch.as_tensor(bt[b, t // block_size].astype(np.int64) * block_size + t % block_size,
+                                        device="cuda")
+                tq.pack_kv(self.kc, self.vc, k[:P].contiguous(), v[:P].contiguous(), slots, self.k_pages,
+                           self.v_pages)
+            if L > P:
+                self.k_win[b, :, :L - P] = k[P:].transpose(0, 1)
+                self.v_win[b, :, :L - P] = v[P:].transpose(0, 1)
+        self.q = torch.randn(self.B, self.Hq, D, generator=gen, device="cuda").to(torch.bfloat16)
+        self.block_tables = torch.as_tensor(bt, device="cuda")
+        self.seq_lens = torch.as_tensor(self.lens.astype(np.int32), device="cuda")
+        self.max_seq_len = int(self.lens.max()) if self.B else 0
+        self.scale = 1.0 / math.sqrt(D)
+
+    def run(self, **kw):
+        return tq.decode_paged(self.kc, self.vc, self.q, self.k_pages, self.v_pages, self.block_tables,
+                               self.seq_lens, self.max_seq_len, self.k_win if self.window else None,
+                               self.v_win if self.window else None, self.window, self.scale, **kw)
+
+    def oracle(self, b, hq):
+        """fp64 oracle output of (sequence b, query head hq) over the GPU-written pages."""
+        h = hq // self.G
+        L = int(self.lens[b])
+        P = L - min(self.window, L)
+        nblk = -(-P // self.bs)
+        blocks = torch.as_tensor(self.block_tables_np[b, :nblk].astype(np.int64), device="cuda")
+        if nblk:
+            kp = self.k_pages[blocks][:, h:h + 1].cpu().numpy()
+            vp = self.v_pages[blocks][:, h:h + 1].cpu().numpy()
+        else:
+            kp = np.zeros((1, 1, self.bs, self.kc.row_bytes), np.uint8)
+            vp = np.zeros((1, 1, self.bs, self.vc.row_bytes), np.uint8)
+        table = np.arange(max(nblk, 1))[None]
+        q = self.q[b:b + 1, hq:hq + 1].float().cpu().numpy().astype(np.float64)
+        kw = self.k_win[b:b + 1, h:h + 1].float().cpu().numpy().astype(np.float64)
+        vw = self.v_win[b:b + 1, h:h + 1].float().cpu().numpy().astype(np.float64)
+        if L == 0:
+            return np.zeros(D)
+        return O.decode_attention(q, kp, vp, table, [L], kw, vw, self.window, self.scale,
+                                  slice_format(self.kf, h), slice_format(self.vf, h), self.bs)[0, 0]
+
+
+def workload_codecs(w):
+    """(device K codec, device V codec, oracle K format, oracle V format) of a named workload."""
+    ks, vs = W.codec_specs(w)
+    kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed)
+    vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed)
+    kf = O.Format(D, w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed)
+    vf = O.Format(D, w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed)
+    return kc, vc, kf, vf

@@ -1,0 +1,136 @@
+"""C-ABI checks that need no GPU: exports, host codec tables vs the oracle, errors, ledger."""
+
+import ctypes
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import tq_oracle as O
+from quantized_paged_kv_pack_b200 import tq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+D = 128
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "tq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert {"tq_make_codec", "tq_pack_kv", "tq_decode_paged", "tq_byte_ledger"} <= set(names)
+    L = ctypes.CDLL(tq.LIB_PATH)
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing
+
+
+def _high(H, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.stack([np.sort(rng.choice(D, n, replace=False)) for _ in range(H)]).astype(np.int16)
+
+
+CASES = [((4,), (128,), None, 0), ((3,), (128,), None, 1), ((2,), (128,), None, 7),
+         ((4, 3), (64, 64), "h", 0), ((4, 2), (32, 96), "h", 1), ((3, 2), (16, 112), "h", 12345678901234)]
+
+
+@pytest.mark.parametrize("bits,sizes,high,seed", CASES)
+def test_host_tables_equal_oracle(bits, sizes, high, seed):
+    H = 4
+    hc = _high(H, sizes[0], seed % 97) if high else None
+    t = tq.codec_host_tables(D, H, bits, sizes, hc, seed)
+    f = O.Format(D, H, bits, sizes, hc, seed)
+    for g, b in enumerate(bits):
+        c, beta = O.codebook(b, D)
+        L = 1 << b
+        assert np.array_equal(t["centroids_f16"][g, :L], c.astype(np.float16).view(np.uint16))
+        assert np.array_equal(t["boundaries"][g, :L - 1].astype(np.float64), beta)
+    assert np.array_equal(t["signs"].astype(np.float64), O.hadamard_signs(seed, D))
+    for h in range(H):
+        assert np.array_equal(t["perm"][h], O.permutation(f, h))
+    assert t["row_bytes"] == O.row_bytes(f)
+
+
+@pytest.mark.parametrize("kw,err", [
+    (dict(bits=(9,), sizes=(128,)), ValueError),
+    (dict(bits=(1,), sizes=(128,)), tq.UnsupportedFormatError),
+    (dict(bits=(5,), sizes=(128,)), tq.UnsupportedFormatError),
+    (dict(bits=(4,), sizes=(64,), d=64), tq.UnsupportedFormatError),
+    (dict(bits=(4,), sizes=(96,), d=96), ValueError),
+    (dict(bits=(4, 3), sizes=(64, 32)), ValueError),
+    (dict(bits=(4, 3), sizes=(60, 68)), tq.UnsupportedFormatError),
+    (dict(bits=(4, 3), sizes=(64, 64), high="missing"), ValueError),
+    (dict(bits=(4, 3), sizes=(64, 64), high="unsorted"), ValueError),
+    (dict(bits=(4, 3), sizes=(64, 64), high="range"), ValueError),
+    (dict(bits=(4,), sizes=(128,), high="extra"), ValueError),
+    (dict(bits=(4,), sizes=(128,), H=0), ValueError),
+])
+def test_descriptor_validation(kw, err):
+    d, H = kw.get("d", D), kw.get("H", 2)
+    hc = None
+    mode = kw.get("high")
+    if mode in ("unsorted", "range", "extra"):
+        hc = _high(max(H, 1), kw["sizes"][0], 3)
+        if mode == "unsorted":
+            hc[0, [0, 1]] = hc[0, [1, 0]]
+        elif mode == "range":
+            hc[1, -1] = 200
+    elif kw.get("bits") and len(kw["bits"]) == 2 and mode != "missing":
+        hc = _high(H, kw["sizes"][0], 3)
+    with pytest.raises(err):
+        tq.codec_host_tables(d, H, kw["bits"], kw["sizes"], hc, 0)
+
+
+def test_workspace_bytes_bounded_by_shape():
+    n = tq.decode_workspace_bytes(16, 64, 8, 131072, 16)
+    assert 0 < n < 64 << 20
+    assert tq.decode_workspace_bytes(16, 64, 8, 131072, 0) == 0
+    assert tq.decode_workspace_bytes(16, 60, 8, 131072, 16) == 0
+    assert tq.decode_workspace_bytes(64, 32, 8, 32768, 16) >= tq.decode_workspace_bytes(32, 32, 8, 32768, 16)
+
+
+def _spec(bits, sizes, seed, H):
+    return {"group_bits": bits, "group_size": sizes, "seed": seed,
+            "high_coords": _high(H, sizes[0], 5) if len(bits) == 2 else None}
+
+
+@pytest.mark.parametrize("kb,ks,vb,vs", [((4,), (128,), (4,), (128,)), ((4, 3), (64, 64), (4, 3), (64, 64)),
+                                          ((4, 2), (32, 96), (3,), (128,))])
+def test_ledger_matches_oracle(kb, ks, vb, vs):
+    H, Hq, W, bs = 8, 32, 64, 16
+    lens = [0, 5, 64, 65, 1000, 4097]
+    ksp, vsp = _spec(kb, ks, 0, H), _spec(vb, vs, 1, H)
+    nb = sum(-(-(L - min(W, L)) // bs) for L in lens) + 3
+    got = tq.host_ledger(H, ksp, vsp, lens, W, Hq, bs, nb)
+    kf = O.Format(D, H, kb, ks, ksp["high_coords"], 0)
+    vf = O.Format(D, H, vb, vs, vsp["high_coords"], 1)
+    ws = tq.decode_workspace_bytes(len(lens), Hq, H, max(lens), bs)
+    ref = O.byte_ledger(kf, vf, lens, W, bs, nb, workspace_bytes=ws)
+    for key in ("dense_bytes", "index_bytes", "norm_bytes", "codebook_bytes", "transform_bytes", "window_bytes",
+                "block_table_bytes", "workspace_bytes", "page_pool_bytes", "metadata_bytes"):
+        assert got[key] == getattr(ref, key), key
+    assert got["all_in_ratio"] == pytest.approx(ref.all_in_ratio, rel=1e-12)
+    assert got["index_only_ratio"] == pytest.approx(ref.dense_bytes / ref.index_bytes, rel=1e-12)
+
+
+def test_recipe_metadata_loader(tmp_path):
+    with pytest.raises(FileNotFoundError):
+        tq.load_recipe_metadata(str(tmp_path / "absent.json"))
+    hc = _high(8, 64, 9)
+    p = tmp_path / "recipe.json"
+    p.write_text(json.dumps({"head_dim": 128, "num_kv_heads": 8, "group_bits": [4, 3], "group_size": [64, 64],
+                             "high_coords": hc.tolist(), "hadamard_seed": 3}))
+    spec = tq.load_recipe_metadata(str(p))
+    assert spec["group_bits"] == (4, 3) and np.array_equal(spec["high_coords"], hc)
+    bad = tmp_path / "bad.json"
+    bad.write_text(json.dumps({"head_dim": 128, "num_kv_heads": 8, "group_bits": [4, 3], "group_size": [64, 64],
+                               "high_coords": hc[:, ::-1].tolist()}))
+    with pytest.raises(ValueError):
+        tq.load_recipe_metadata(str(bad))
+    with pytest.raises(ValueError):
+        bad.write_text(json.dumps({"head_dim": 128}))
+        tq.load_recipe_metadata(str(bad))

@@ -1,0 +1,175 @@
+"""GPU parity of tq_decode_paged against the fp64 oracle on the same (GPU-written) pages."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import tq_oracle as O
+from quantized_paged_kv_pack_b200 import tq
+from quantized_paged_kv_pack_b200 import workloads as W
+
+from helpers import D, DecodeProblem, slice_format, workload_codecs
+
+pytestmark = pytest.mark.gpu
+
+ATOL = 2e-3  # max-abs error of the fp32 decode vs the fp64 oracle on the same cache
+
+U4 = ((4,), (128,), 0)
+U3 = ((3,), (128,), 1)
+U2 = ((2,), (128,), 2)
+M35 = ((4, 3), (64, 64), 3)
+M25 = ((4, 2), (32, 96), 4)
+
+
+def check(prob, pairs=None):
+    out = prob.run()
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    pairs = pairs if pairs is not None else [(b, hq) for b in range(prob.B) for hq in range(prob.Hq)]
+    worst = scale = 0.0
+    for b, hq in pairs:
+        ref = prob.oracle(b, hq)
+        worst = max(worst, float(np.abs(got[b, hq] - ref).max()))
+        scale = max(scale, float(np.abs(ref).max()))
+    assert worst <= ATOL, worst
+    if any(prob.lens[b] for b, _ in pairs):
+        assert scale > 0.5  # the outputs are not trivially zero
+    return worst
+
+
+@pytest.mark.parametrize("kspec,vspec", [(U4, U4), (M35, M35), (M25, U3), (U2, M35), (U3, U2)])
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_decode_matches_oracle_small(kspec, vspec, G):
+    lens = [1, 15, 16, 17, 100, 700]
+    prob = DecodeProblem(lens, 2, G, kspec, (vspec[0], vspec[1], vspec[2] + 10), window=0, block_size=16, seed=G)
+    check(prob)
+
+
+@pytest.mark.parametrize("window,bs", [(8, 16), (64, 16), (128, 32), (5, 7)])
+def test_decode_with_window_and_ragged_lengths(window, bs):
+    lens = [0, 1, window, window + 1, 3 * window + 5, 2000, 4099]
+    prob = DecodeProblem(lens, 2, 4, M25, U3, window=window, block_size=bs, seed=window)
+    check(prob)
+
+
+def test_decode_gqa16_and_long_sequence_spans_many_splits():
+    prob = DecodeProblem([9000, 300], 1, 16, U4, M35, window=16, block_size=16, seed=5)
+    check(prob)
+
+
+def test_decode_full_small_workload():
+    """The oracle-sized workload in full: 1 sequence, GQA 8, context 4096, 4-bit."""
+    w = W.WORKLOADS["decode_gqa8_4k_4bit"]
+    kc, vc, kf, vf = workload_codecs(w)
+    layout = W.page_layout(w)
+    kp, vp = tq.page_pool(kc, layout.num_blocks, w.block_size), tq.page_pool(vc, layout.num_blocks, w.block_size)
+    L = int(layout.seq_lens[0])
+    k, v = W.sequence_kv(w, 0, 0, L, device="cuda")
+    slots = W.slot_mapping(layout, 0, 0, L, w.block_size)
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp)
+    q = W.queries(w, device="cuda")
+    bt = torch.as_tensor(layout.block_tables, device="cuda")
+    sl = torch.as_tensor(layout.seq_lens.astype(np.int32), device="cuda")
+    out = tq.decode_paged(kc, vc, q, kp, vp, bt, sl, L, None, None, 0, 1 / math.sqrt(D))
+    torch.cuda.synchronize()
+    ref = O.decode_attention(q.float().cpu().numpy().astype(np.float64), kp.cpu().numpy(), vp.cpu().numpy(),
+                             layout.block_tables, layout.seq_lens, None, None, 0, 1 / math.sqrt(D), kf, vf,
+                             w.block_size)
+    assert np.abs(out.cpu().numpy() - ref).max() <= ATOL
+    assert np.abs(ref).max() > 0.5
+
+
+def test_decode_empty_batch_and_zero_lengths():
+    prob = DecodeProblem([0, 0], 1, 2, U4, U4, window=4, block_size=16, seed=1)
+    out = prob.run()
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+
+
+def test_decode_bad_block_id_sets_error_without_fault():
+    prob = DecodeProblem([40], 1, 2, U4, U4, window=0, block_size=16, seed=2)
+    prob.block_tables[0, 1] = prob.num_blocks + 5
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    prob.run(d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() & tq.TQ_DERR_BLOCK
+
+
+def test_decode_argument_errors():
+    prob = DecodeProblem([40], 1, 2, U4, U4, window=0, block_size=16, seed=3)
+    small = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ValueError):
+        prob.run(workspace=small)
+    with pytest.raises(ValueError):
+        tq.decode_paged(prob.kc, prob.vc, prob.q, prob.k_pages, prob.v_pages, prob.block_tables, prob.seq_lens,
+                        prob.max_seq_len, None, None, 4, prob.scale)
+    q3 = torch.zeros(1, 3, D, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(tq.UnsupportedFormatError):  # 3 query heads per KV head
+        tq.decode_paged(prob.kc, prob.vc, q3, prob.k_pages, prob.v_pages, prob.block_tables, prob.seq_lens,
+                        prob.max_seq_len, None, None, 0, prob.scale)
+    prob2 = DecodeProblem([40], 2, 2, U4, U4, window=0, block_size=16, seed=4)
+    with pytest.raises(ValueError):  # 3 query heads over 2 KV heads
+        tq.decode_paged(prob2.kc, prob2.vc, q3, prob2.k_pages, prob2.v_pages, prob2.block_tables, prob2.seq_lens,
+                        prob2.max_seq_len, None, None, 0, prob2.scale)
+
+
+def test_decode_phases_equal_single_call():
+    prob = DecodeProblem([500, 1234], 2, 4, M35, U3, window=8, block_size=16, seed=9)
+    ws = tq.alloc_workspace(prob.B, prob.Hq, prob.H, prob.max_seq_len, prob.bs)
+    a = prob.run(workspace=ws).clone()
+    out = torch.empty_like(a)
+    prob.run(workspace=ws, phase="partials")
+    prob.run(workspace=ws, phase="combine", out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(a, out)
+
+
+def _workload_problem(name, n_seq):
+    """Build the named decode workload on the GPU (pages by the GPU pack kernel)."""
+    w = W.WORKLOADS[name]
+    kc, vc, kf, vf = workload_codecs(w)
+    layout = W.page_layout(w)
+    kp, vp = tq.page_pool(kc, layout.num_blocks, w.block_size), tq.page_pool(vc, layout.num_blocks, w.block_size)
+    for b in range(len(layout.seq_lens)):
+        P = int(layout.packed_lens[b])
+        for t0 in range(0, P, 16384):
+            t1 = min(P, t0 + 16384)
+            k, v = W.sequence_kv(w, b, t0, t1, device="cuda")
+            slots = W.slot_mapping(layout, b, t0, t1, w.block_size)
+            tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp)
+    kw, vw = W.windows(w, layout, device="cuda")
+    return w, kc, vc, kf, vf, layout, kp, vp, kw, vw
+
+
+@pytest.mark.parametrize("name", ["decode_llama8b_4bit", "decode_llama70b_3p5bit", "decode_llama8b_2p5bit"])
+def test_decode_full_size_workloads_sampled(name):
+    """Full-size workloads in the benchmark's launch; the oracle checks sampled outputs."""
+    w, kc, vc, kf, vf, layout, kp, vp, kw, vw = _workload_problem(name, None)
+    q = W.queries(w, device="cuda")
+    bt = torch.as_tensor(layout.block_tables, device="cuda")
+    sl = torch.as_tensor(layout.seq_lens.astype(np.int32), device="cuda")
+    maxL = int(layout.seq_lens.max())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = tq.decode_paged(kc, vc, q, kp, vp, bt, sl, maxL, kw, vw, w.window, 1 / math.sqrt(D), d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = out.cpu().numpy()
+    G = w.num_q_heads // w.num_kv_heads
+    order = np.argsort(layout.seq_lens)
+    picks = [int(order[0]), int(order[len(order) // 2]), int(order[-1])]
+    rng = np.random.default_rng(1)
+    for b in picks:
+        for hq in rng.choice(w.num_q_heads, 2, replace=False):
+            h = hq // G
+            L, P = int(layout.seq_lens[b]), int(layout.packed_lens[b])
+            nblk = -(-P // w.block_size)
+            blocks = torch.as_tensor(layout.block_tables[b, :nblk].astype(np.int64), device="cuda")
+            ref = O.decode_attention(q[b:b + 1, hq:hq + 1].float().cpu().numpy().astype(np.float64),
+                                     kp[blocks][:, h:h + 1].cpu().numpy(), vp[blocks][:, h:h + 1].cpu().numpy(),
+                                     np.arange(nblk)[None], [L], kw[b:b + 1, h:h + 1].float().cpu().numpy(),
+                                     vw[b:b + 1, h:h + 1].float().cpu().numpy(), w.window, 1 / math.sqrt(D),
+                                     slice_format(kf, h), slice_format(vf, h), w.block_size)[0, 0]
+            assert np.abs(got[b, hq] - ref).max() <= ATOL
+            assert np.abs(ref).max() > 0.5

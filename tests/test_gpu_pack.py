@@ -1,0 +1,188 @@
+"""GPU parity of tq_pack_kv against the oracle (through the C ABI)."""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import tq_oracle as O
+from quantized_paged_kv_pack_b200 import tq
+from quantized_paged_kv_pack_b200 import workloads as W
+
+from helpers import D, codec_pair, random_kv, slice_format, workload_codecs
+
+pytestmark = pytest.mark.gpu
+
+BOUNDARY_REL = 1e-5       # near-boundary exemption for index mismatches
+MAX_FLIP_FRACTION = 1e-4  # exempt mismatches allowed, as a fraction of coordinates
+
+FORMATS = [((4,), (128,)), ((3,), (128,)), ((2,), (128,)), ((4, 3), (64, 64)), ((4, 2), (32, 96)),
+           ((3, 2), (16, 112)), ((2, 4), (112, 16))]
+
+
+def compare_rows(gpu_rows, k_cpu, fmt, heads):
+    """Compare GPU rows [N][H][row] with the oracle's quantization of k_cpu [N][H][d].
+
+    Norms must be bit-identical; indices identical except near a boundary.
+    Returns (number of exempt index flips, number of coordinates).
+    """
+    flips = total = 0
+    for h in heads:
+        f1 = slice_format(fmt, h)
+        idx, n16, u = O.quantize(k_cpu[:, h], f1, 0)
+        gidx, gn16 = O.decode_rows(gpu_rows[:, h], f1)
+        assert np.array_equal(gn16.astype(np.float16).view(np.uint16), n16.astype(np.float16).view(np.uint16)), \
+            "fp16 norms differ"
+        bad = gidx != idx
+        if bad.any():
+            margin = O.boundary_margin(u, f1)
+            assert np.all(margin[bad] <= BOUNDARY_REL), "index mismatch away from a codebook boundary"
+            assert np.all(np.abs(gidx[bad] - idx[bad]) == 1)
+        flips += int(bad.sum())
+        total += idx.size
+    return flips, total
+
+
+@pytest.mark.parametrize("kfmt", FORMATS)
+@pytest.mark.parametrize("T,H,bs", [(1, 1, 16), (37, 2, 16), (300, 8, 32), (129, 3, 5)])
+def test_pack_matches_oracle(kfmt, T, H, bs):
+    vfmt = FORMATS[(FORMATS.index(kfmt) + 3) % len(FORMATS)]
+    kc, kf = codec_pair(H, *kfmt, 11)
+    vc, vf = codec_pair(H, *vfmt, 22)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(T * 131 + H)
+    k, v = random_kv(T, H, gen)
+    nb = -(-T // bs) + 3
+    rng = np.random.default_rng(T)
+    slots = rng.permutation(nb * bs)[:T].astype(np.int64)
+    slots[::7] = -1  # padding tokens
+    kp, vp = tq.page_pool(kc, nb, bs), tq.page_pool(vc, nb, bs)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    kcpu = k.float().cpu().numpy().astype(np.float64)
+    vcpu = v.float().cpu().numpy().astype(np.float64)
+    live = slots >= 0
+    ref_kp, ref_vp = O.pack_kv(kcpu, vcpu, slots, kf, vf, nb, bs)
+    gk, gv = kp.cpu().numpy(), vp.cpu().numpy()
+    s = slots[live]
+    for g, ref, src, f in ((gk, ref_kp, kcpu, kf), (gv, ref_vp, vcpu, vf)):
+        rows = g[s // bs, :, s % bs]
+        compare_rows(rows, src[live], f, range(H))
+        # bytes of slots nobody wrote stay zero, as in the oracle's pool
+        written = np.zeros((nb, bs), bool)
+        written[s // bs, s % bs] = True
+        assert not g.transpose(0, 2, 1, 3)[~written].any()
+        # where no index sits near a boundary the whole row is byte-identical
+        if len(s):
+            same = (rows == ref[s // bs, :, s % bs]).all(axis=-1)
+            assert same.mean() > 0.99
+            assert (rows[..., -2:] != 0).any(axis=-1).mean() > 0.99  # norms were written
+
+
+def test_pack_reconstruction_mse_within_two_percent():
+    H, T = 8, 2048
+    kc, kf = codec_pair(H, (4, 3), (64, 64), 5)
+    vc, vf = codec_pair(H, (4, 2), (32, 96), 6)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(77)
+    k, v = random_kv(T, H, gen)
+    kp, vp = tq.page_pool(kc, T // 16, 16), tq.page_pool(vc, T // 16, 16)
+    tq.pack_kv(kc, vc, k, v, torch.arange(T, device="cuda"), kp, vp)
+    torch.cuda.synchronize()
+    for pages, src, f in ((kp, k, kf), (vp, v, vf)):
+        x = src.float().cpu().numpy().astype(np.float64)
+        g = pages.cpu().numpy().reshape(T // 16, H, 16, -1).transpose(0, 2, 1, 3).reshape(T, H, -1)
+        mse_gpu = mse_ref = 0.0
+        for h in range(H):
+            f1 = slice_format(f, h)
+            gi, gn = O.decode_rows(g[:, h], f1)
+            ri, rn, _ = O.quantize(x[:, h], f1, 0)
+            mse_gpu += ((O.dequantize_rows(gi, gn, f1, 0) - x[:, h]) ** 2).sum()
+            mse_ref += ((O.dequantize_rows(ri, rn, f1, 0) - x[:, h]) ** 2).sum()
+        assert abs(mse_gpu / mse_ref - 1) <= 0.02
+
+
+def test_pack_edge_values():
+    H = 2
+    kc, kf = codec_pair(H, (4,), (128,), 0)
+    vc, vf = codec_pair(H, (3,), (128,), 1)
+    T = 6
+    k = torch.zeros(T, H, D, dtype=torch.bfloat16, device="cuda")
+    k[1] = 1e-30           # norm underflows fp16
+    k[2, :, 0] = 70000.0   # norm overflows fp16 -> inf
+    k[3] = 3.0e-3
+    k[4, :, 5] = -2.5      # one-hot
+    k[5] = torch.linspace(-300, 300, D, device="cuda").to(torch.bfloat16)
+    v = k.flip(0).contiguous()
+    kp, vp = tq.page_pool(kc, 1, 8), tq.page_pool(vc, 1, 8)
+    tq.pack_kv(kc, vc, k, v, torch.arange(T, device="cuda"), kp, vp)
+    torch.cuda.synchronize()
+    rk, rv = O.pack_kv(k.float().cpu().numpy(), v.float().cpu().numpy(), np.arange(T), kf, vf, 1, 8)
+    assert np.array_equal(kp.cpu().numpy(), rk)
+    assert np.array_equal(vp.cpu().numpy(), rv)
+
+
+def test_pack_empty_and_all_padding():
+    kc, _ = codec_pair(2, (4,), (128,), 0)
+    vc, _ = codec_pair(2, (4,), (128,), 1)
+    kp, vp = tq.page_pool(kc, 2, 16), tq.page_pool(vc, 2, 16)
+    e = torch.empty(0, 2, D, dtype=torch.bfloat16, device="cuda")
+    tq.pack_kv(kc, vc, e, e, torch.empty(0, dtype=torch.int64, device="cuda"), kp, vp)
+    k = torch.randn(5, 2, D, device="cuda").to(torch.bfloat16)
+    tq.pack_kv(kc, vc, k, k, torch.full((5,), -1, dtype=torch.int64, device="cuda"), kp, vp)
+    torch.cuda.synchronize()
+    assert not kp.any() and not vp.any()
+
+
+def test_pack_slot_outside_pool_sets_error_and_skips(monkeypatch):
+    kc, _ = codec_pair(1, (4,), (128,), 0)
+    vc, _ = codec_pair(1, (4,), (128,), 1)
+    kp, vp = tq.page_pool(kc, 2, 4), tq.page_pool(vc, 2, 4)
+    k = torch.randn(3, 1, D, device="cuda").to(torch.bfloat16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.pack_kv(kc, vc, k, k, torch.tensor([0, 8, 5], device="cuda"), kp, vp, d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() & tq.TQ_DERR_SLOT
+    assert kp[0, 0, 0].any() and kp[1, 0, 1].any()
+    assert not kp.view(-1, kp.shape[-1])[[1, 2, 3, 4, 6, 7]].any()
+    monkeypatch.setenv("TQ_CHECKED", "1")
+    err.zero_()
+    with pytest.raises(IndexError):
+        tq.pack_kv(kc, vc, k, k, torch.tensor([0, 8, 5], device="cuda"), kp, vp, d_err=err)
+
+
+def test_pack_argument_errors():
+    kc, _ = codec_pair(2, (4,), (128,), 0)
+    vc1, _ = codec_pair(1, (4,), (128,), 1)
+    kp = tq.page_pool(kc, 2, 4)
+    k = torch.randn(3, 2, D, device="cuda").to(torch.bfloat16)
+    with pytest.raises(ValueError):
+        tq.pack_kv(kc, vc1, k, k, torch.arange(3, device="cuda"), kp, tq.page_pool(vc1, 2, 4))
+    with pytest.raises(ValueError):
+        tq.pack_kv(kc, kc, k.float(), k, torch.arange(3, device="cuda"), kp, kp)
+
+
+def test_pack_workload_sample_full_size():
+    """The full pack workload in the benchmark's launch, checked on sampled rows."""
+    w = W.WORKLOADS["pack_llama8b_4bit"]
+    kc, vc, kf, vf = workload_codecs(w)
+    k, v, slots, layout = W.pack_batch(w, device="cuda")
+    kp, vp = tq.page_pool(kc, layout.num_blocks, w.block_size), tq.page_pool(vc, layout.num_blocks, w.block_size)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    rng = np.random.default_rng(3)
+    pick = np.sort(rng.choice(len(slots), 4096, replace=False))
+    s = slots[pick]
+    flips = total = 0
+    for pages, src, f in ((kp, k, kf), (vp, v, vf)):
+        rows = pages[torch.as_tensor(s // w.block_size, device="cuda"), :, torch.as_tensor(s % w.block_size, device="cuda")]
+        x = src[torch.as_tensor(pick, device="cuda")].float().cpu().numpy().astype(np.float64)
+        a, b = compare_rows(rows.cpu().numpy(), x, f, range(w.num_kv_heads))
+        flips, total = flips + a, total + b
+    assert flips <= MAX_FLIP_FRACTION * total
