@@ -96,7 +96,7 @@ class DecodeSetup:
                 t1 = min(P, t0 + 32768)
                 k, v = WL.sequence_kv(w, b, t0, t1, device="cuda")
                 slots = torch.as_tensor(WL.slot_mapping(lay, b, t0, t1, bs), device="cuda")
-                tq.pack_kv(self.kc, self.vc, k, v, slots, self.kp, self.vp)
+                tq.pack_kv(self.kc, self.vc, k, v, slots, self.kp, self.vp, bs)
         self.kw, self.vw = WL.windows(w, lay, device="cuda")
         self.q = WL.queries(w, device="cuda")
         self.bt = torch.as_tensor(lay.block_tables, device="cuda")
@@ -139,11 +139,12 @@ class DecodeSetup:
     # the step ---------------------------------------------------------------
     def pack(self, k=None, v=None, slots=None):
         tq.pack_kv(self.kc, self.vc, self.new_k if k is None else k, self.new_v if v is None else v,
-                   self.new_slots if slots is None else slots, self.kp, self.vp, d_err=self.err)
+                   self.new_slots if slots is None else slots, self.kp, self.vp, self.w.block_size, d_err=self.err)
 
     def decode(self, phase="all", q=None, out=None):
         w = self.w
-        return tq.decode_paged(self.kc, self.vc, self.q if q is None else q, self.kp, self.vp, self.bt, self.sl,
+        return tq.decode_paged(self.kc, self.vc, self.q if q is None else q, self.kp, self.vp, w.block_size,
+                               self.bt, self.sl,
                                self.max_len, self.kw if w.window else None, self.vw if w.window else None, w.window,
                                self.scale, out=self.out if out is None else out, workspace=self.ws, d_err=self.err,
                                phase=phase)
@@ -167,7 +168,7 @@ class PackSetup:
         return T * H * D * 2 * 2 + T * H * (self.kc.row_bytes + self.vc.row_bytes) + T * 8
 
     def step(self):
-        tq.pack_kv(self.kc, self.vc, self.k, self.v, self.slots, self.kp, self.vp, d_err=self.err)
+        tq.pack_kv(self.kc, self.vc, self.k, self.v, self.slots, self.kp, self.vp, self.w.block_size, d_err=self.err)
 
 
 # --------------------------------------------------------------------------- measurement

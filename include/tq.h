@@ -123,13 +123,16 @@ int32_t tq_codec_row_bytes(const tq_codec* codec);
  * k, v           device bf16 [num_tokens][num_kv_heads][head_dim], contiguous.
  * slot_mapping   device int64 [num_tokens]; a negative slot marks a padding
  *                token, which is skipped.
- * k_pages        device uint8 [num_blocks][num_kv_heads][block_size][kc row_bytes]
- * v_pages        device uint8 [num_blocks][num_kv_heads][block_size][vc row_bytes]
- *                (separate pools that share block ids).
+ * k_pages        device uint8 [num_blocks][num_kv_heads][block_size * kc row_bytes]
+ * v_pages        device uint8 [num_blocks][num_kv_heads][block_size * vc row_bytes]
+ *                (separate pools that share block ids; 8-byte aligned).
  * Row of one (token, head): [group-0 bitstream][group-1 bitstream][fp16 norm],
  * bitstreams LSB-first, the norm little endian; see tq_codec_host_tables for
- * the rotation and codebook. Each row is written whole; bytes of other rows
- * are untouched.
+ * the rotation and codebook. Within the sub-page of (block, head) the index
+ * bytes of the block_size rows come first, row after row (offset * index
+ * bytes), then the block_size norms (block_size * index bytes + 2 * offset),
+ * so index rows stay 8-byte aligned. Each row is written whole; bytes of
+ * other rows are untouched.
  * Errors: TQ_ERR_VALUE for inconsistent arguments (num_kv_heads or head_dim
  * differing between the codecs, block_size < 1, null pointers with
  * num_tokens > 0). A slot >= num_blocks * block_size sets TQ_DERR_SLOT in

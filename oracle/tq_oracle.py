@@ -46,8 +46,10 @@ R5  idx = #{boundaries strictly below u}: nearest centroid, ties to the lower
 R6  Row = [group-0 bitstream][group-1 bitstream][fp16 norm, little endian];
     each bitstream is LSB-first, index k at bits [k*b, (k+1)*b). Group 0 holds
     the high coordinates in ascending order, group 1 the rest ascending.
-    Pages are [num_blocks][H_kv][block_size][row_bytes]; K and V have separate
-    pools that share block ids.
+    Pages are [num_blocks][H_kv][block_size * row_bytes]: the sub-page of one
+    (block, head) holds the index bytes of its block_size rows, row after row,
+    then their block_size fp16 norms. A row is found from (block, offset)
+    alone; K and V have separate pools that share block ids.
 R7  The last min(W, L_b) tokens of a sequence live only in the dense bf16
     window; the first P_b = L_b - min(W, L_b) tokens are packed.
 R8  slot < 0 is a padding token and is skipped; slot >= num_blocks*block_size
@@ -70,7 +72,7 @@ __all__ = [
     "splitmix64", "hadamard_signs", "hadamard_matrix", "rotate", "unrotate",
     "permutation", "position_bits", "row_bytes", "index_bytes",
     "quantize", "encode_rows", "decode_rows", "dequantize_rows",
-    "pack_kv", "read_row", "decode_attention", "dense_attention",
+    "pack_kv", "read_row", "read_rows", "write_rows", "subpage_bytes", "decode_attention", "dense_attention",
     "boundary_margin", "byte_ledger", "Ledger", "fp16_round", "bf16_round",
 ]
 
@@ -434,6 +436,32 @@ def dequantize_rows(idx, n16, fmt: Format, head: int):
 # Page writes (serving route contract)
 # ---------------------------------------------------------------------------
 
+def subpage_bytes(fmt: Format, block_size: int) -> int:
+    return block_size * row_bytes(fmt)
+
+
+def write_rows(pages, blocks, head: int, offsets, rows, fmt: Format, block_size: int):
+    """Store logical rows at (block, offset) of one head's sub-pages (R6 layout)."""
+    ib = index_bytes(fmt)
+    blocks = np.asarray(blocks, dtype=np.int64)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.uint8)
+    cols = offsets[:, None] * ib + np.arange(ib)[None, :]
+    pages[blocks[:, None], head, cols] = rows[:, :ib]
+    ncols = block_size * ib + 2 * offsets[:, None] + np.arange(2)[None, :]
+    pages[blocks[:, None], head, ncols] = rows[:, ib:]
+
+
+def read_rows(pages, blocks, head: int, offsets, fmt: Format, block_size: int):
+    """Logical rows [n][row_bytes] at (block, offset) of one head's sub-pages."""
+    ib = index_bytes(fmt)
+    blocks = np.asarray(blocks, dtype=np.int64)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    cols = offsets[:, None] * ib + np.arange(ib)[None, :]
+    ncols = block_size * ib + 2 * offsets[:, None] + np.arange(2)[None, :]
+    return np.concatenate((pages[blocks[:, None], head, cols], pages[blocks[:, None], head, ncols]), axis=-1)
+
+
 def pack_kv(k, v, slot_mapping, kfmt: Format, vfmt: Format, num_blocks: int, block_size: int,
             k_pages=None, v_pages=None):
     """Quantize and write K and V rows into page pools.
@@ -452,32 +480,32 @@ def pack_kv(k, v, slot_mapping, kfmt: Format, vfmt: Format, num_blocks: int, blo
     if np.any(slots >= num_blocks * block_size):
         raise IndexError("slot mapping points outside the allocated pages")
     if k_pages is None:
-        k_pages = np.zeros((num_blocks, H, block_size, row_bytes(kfmt)), dtype=np.uint8)
+        k_pages = np.zeros((num_blocks, H, subpage_bytes(kfmt, block_size)), dtype=np.uint8)
     if v_pages is None:
-        v_pages = np.zeros((num_blocks, H, block_size, row_bytes(vfmt)), dtype=np.uint8)
+        v_pages = np.zeros((num_blocks, H, subpage_bytes(vfmt, block_size)), dtype=np.uint8)
     live = np.nonzero(slots >= 0)[0]
     blk = slots[live] // block_size
     off = slots[live] % block_size
     for h in range(H):
         for src, fmt, pages in ((k, kfmt, k_pages), (v, vfmt, v_pages)):
             idx, n16, _ = quantize(src[live, h, :], fmt, h)
-            pages[blk, h, off, :] = encode_rows(idx, n16, fmt)
+            write_rows(pages, blk, h, off, encode_rows(idx, n16, fmt), fmt, block_size)
     return k_pages, v_pages
 
 
-def read_row(pages, slot: int, head: int, block_size: int):
+def read_row(pages, slot: int, head: int, block_size: int, fmt: Format):
     """Row bytes of one token, by the page address formula."""
-    return pages[slot // block_size, head, slot % block_size, :]
+    return read_rows(pages, [slot // block_size], head, [slot % block_size], fmt, block_size)[0]
 
 
 # ---------------------------------------------------------------------------
 # Decode attention (dense reconstruction: diagnostic route only)
 # ---------------------------------------------------------------------------
 
-def _gather_rows(pages, block_table, count: int, head: int, block_size: int):
+def _gather_rows(pages, block_table, count: int, head: int, block_size: int, fmt: Format):
     i = np.arange(count)
     blocks = np.asarray(block_table, dtype=np.int64)[i // block_size]
-    return pages[blocks, head, i % block_size, :]
+    return read_rows(pages, blocks, head, i % block_size, fmt, block_size)
 
 
 def decode_attention(q, k_pages, v_pages, block_tables, seq_lens, k_win, v_win, window: int,
@@ -502,8 +530,8 @@ def decode_attention(q, k_pages, v_pages, block_tables, seq_lens, k_win, v_win, 
         n_win = min(window, L)
         P = L - n_win
         for h in range(H):
-            ki, kn = decode_rows(_gather_rows(k_pages, block_tables[b], P, h, block_size), kfmt)
-            vi, vn = decode_rows(_gather_rows(v_pages, block_tables[b], P, h, block_size), vfmt)
+            ki, kn = decode_rows(_gather_rows(k_pages, block_tables[b], P, h, block_size, kfmt), kfmt)
+            vi, vn = decode_rows(_gather_rows(v_pages, block_tables[b], P, h, block_size, vfmt), vfmt)
             keys = dequantize_rows(ki, kn, kfmt, h)
             vals = dequantize_rows(vi, vn, vfmt, h)
             if n_win:

@@ -67,8 +67,9 @@ __device__ __forceinline__ int row_index(const uint8_t* row, const DevCodec& c, 
     return static_cast<int>((w >> sh) & ((1u << b) - 1u));
 }
 
-__device__ __forceinline__ float row_norm(const uint8_t* row, const DevCodec& c) {
-    unsigned short h = static_cast<unsigned short>(row[c.index_bytes] | (row[c.index_bytes + 1] << 8));
+__device__ __forceinline__ float row_norm(const uint8_t* sub, const DevCodec& c, int block_size, int off) {
+    const uint8_t* n = sub + block_size * c.index_bytes + 2 * off;
+    unsigned short h = static_cast<unsigned short>(n[0] | (n[1] << 8));
     return __half2float(__ushort_as_half(h));
 }
 
@@ -164,9 +165,12 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
                 if (a.d_err && lane == 0) atomicOr(a.d_err, TQ_DERR_BLOCK);
                 blk = 0;
             }
-            const int64_t r = (blk * H + h) * bs + t % bs;
-            const uint8_t* krow = a.k_pages + r * a.kc.row_bytes;
-            const uint8_t* vrow = a.v_pages + r * a.vc.row_bytes;
+            const int64_t sp = (blk * H + h) * bs;
+            const int off = t % bs;
+            const uint8_t* ksub = a.k_pages + sp * a.kc.row_bytes;
+            const uint8_t* vsub = a.v_pages + sp * a.vc.row_bytes;
+            const uint8_t* krow = ksub + off * a.kc.index_bytes;
+            const uint8_t* vrow = vsub + off * a.vc.index_bytes;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 int g;
@@ -175,8 +179,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
                 ix = row_index(vrow, a.vc, 4 * lane + i, g);
                 vv[i] = a.vc.cent[g * 16 + ix];
             }
-            nk = row_norm(krow, a.kc);
-            nv = row_norm(vrow, a.vc);
+            nk = row_norm(ksub, a.kc, bs, off);
+            nv = row_norm(vsub, a.vc, bs, off);
         }
 #pragma unroll
         for (int g = 0; g < G; ++g) {

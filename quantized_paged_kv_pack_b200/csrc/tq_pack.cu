@@ -8,7 +8,9 @@
 //   z   = H (s * x)              Sylvester Walsh-Hadamard, signs s of the codec
 //   u   = z / (sqrt(128) n)      the rotated unit vector
 //   idx = #{boundaries of its group below u_j}, placed at packed position pos[h][j]
-//   row = [group-0 bitstream][group-1 bitstream][n16], LSB-first.
+//   row = [group-0 bitstream][group-1 bitstream][n16], LSB-first; in the
+//   sub-page of (block, head) the index bytes of the block_size rows come
+//   first, row after row, then the block_size norms.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -143,10 +145,10 @@ pack_rows_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__ k,
             }
         }
         const int64_t blk = slot / block_size, off = slot - blk * block_size;
-        uint8_t* pages = which ? v_pages : k_pages;
-        uint16_t* dst = reinterpret_cast<uint16_t*>(pages + ((blk * H + h) * block_size + off) * c.row_bytes);
+        uint8_t* sub = (which ? v_pages : k_pages) + (blk * H + h) * block_size * c.row_bytes;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(sub + off * c.index_bytes);
         if (lane < half_words) dst[lane] = static_cast<uint16_t>(word);
-        if (lane == 0) dst[half_words] = n16;
+        if (lane == 0) *reinterpret_cast<uint16_t*>(sub + block_size * c.index_bytes + 2 * off) = n16;
         __syncwarp();
     }
 }

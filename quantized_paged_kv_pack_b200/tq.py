@@ -215,23 +215,33 @@ def _need(t, dtype, shape, name):
 
 
 def page_pool(codec: Codec, num_blocks: int, block_size: int, device="cuda") -> torch.Tensor:
-    """Zeroed uint8 pool [num_blocks][H_kv][block_size][row_bytes]."""
-    return torch.zeros(num_blocks, codec.num_kv_heads, block_size, codec.row_bytes, dtype=torch.uint8, device=device)
+    """Zeroed uint8 pool [num_blocks][H_kv][block_size * row_bytes] (one sub-page per block and head)."""
+    return torch.zeros(num_blocks, codec.num_kv_heads, block_size * codec.row_bytes, dtype=torch.uint8,
+                       device=device)
+
+
+def _pools(kc, vc, k_pages, v_pages, block_size):
+    if k_pages.dim() != 3 or v_pages.dim() != 3:
+        raise ValueError("page pools must be [num_blocks][H_kv][block_size * row_bytes]")
+    if block_size < 1:
+        raise ValueError("block_size must be positive")
+    nb = k_pages.shape[0]
+    _need(k_pages, torch.uint8, (nb, kc.num_kv_heads, block_size * kc.row_bytes), "k_pages")
+    _need(v_pages, torch.uint8, (nb, vc.num_kv_heads, block_size * vc.row_bytes), "v_pages")
+    return nb
 
 
 def pack_kv(kc: Codec, vc: Codec, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
-            k_pages: torch.Tensor, v_pages: torch.Tensor, d_err: Optional[torch.Tensor] = None, stream=None):
+            k_pages: torch.Tensor, v_pages: torch.Tensor, block_size: int, d_err: Optional[torch.Tensor] = None,
+            stream=None):
     """Quantize and write K/V rows into the page pools (tq_pack_kv)."""
     T = k.shape[0] if k.dim() == 3 else -1
     H = kc.num_kv_heads
     _need(k, torch.bfloat16, (T, H, kc.head_dim), "k")
     _need(v, torch.bfloat16, (T, H, kc.head_dim), "v")
     _need(slot_mapping, torch.int64, (T,), "slot_mapping")
-    if k_pages.dim() != 4:
-        raise ValueError("page pools must be [num_blocks][H_kv][block_size][row_bytes]")
-    nb, _, bs, _ = k_pages.shape
-    _need(k_pages, torch.uint8, (nb, H, bs, kc.row_bytes), "k_pages")
-    _need(v_pages, torch.uint8, (nb, H, bs, vc.row_bytes), "v_pages")
+    nb = _pools(kc, vc, k_pages, v_pages, block_size)
+    bs = int(block_size)
     if d_err is not None:
         _need(d_err, torch.int32, (1,), "d_err")
     _check(lib().tq_pack_kv(kc.handle, vc.handle, _ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_pages),
@@ -248,7 +258,7 @@ def alloc_workspace(batch, num_q_heads, num_kv_heads, max_seq_len, block_size, d
 
 
 def decode_paged(kc: Codec, vc: Codec, q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
-                 block_tables: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
+                 block_size: int, block_tables: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
                  k_win: Optional[torch.Tensor], v_win: Optional[torch.Tensor], window: int,
                  softmax_scale: float, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                  d_err: Optional[torch.Tensor] = None, stream=None, phase: str = "all") -> torch.Tensor:
@@ -262,11 +272,8 @@ def decode_paged(kc: Codec, vc: Codec, q: torch.Tensor, k_pages: torch.Tensor, v
     B, Hq, d = q.shape
     H = kc.num_kv_heads
     _need(q, torch.bfloat16, (B, Hq, kc.head_dim), "q")
-    if k_pages.dim() != 4:
-        raise ValueError("page pools must be [num_blocks][H_kv][block_size][row_bytes]")
-    nb, _, bs, _ = k_pages.shape
-    _need(k_pages, torch.uint8, (nb, H, bs, kc.row_bytes), "k_pages")
-    _need(v_pages, torch.uint8, (nb, H, bs, vc.row_bytes), "v_pages")
+    nb = _pools(kc, vc, k_pages, v_pages, block_size)
+    bs = int(block_size)
     if block_tables.dim() != 2:
         raise ValueError("block_tables must be [batch][max_blocks_per_seq]")
     _need(block_tables, torch.int32, (B, block_tables.shape[1]), "block_tables")

@@ -78,7 +78,7 @@ class DecodeProblem:
                 slots = torch.as_tensor(bt[b, t // block_size].astype(np.int64) * block_size + t % block_size,
                                         device="cuda")
                 tq.pack_kv(self.kc, self.vc, k[:P].contiguous(), v[:P].contiguous(), slots, self.k_pages,
-                           self.v_pages)
+                           self.v_pages, block_size)
             if L > P:
                 self.k_win[b, :, :L - P] = k[P:].transpose(0, 1)
                 self.v_win[b, :, :L - P] = v[P:].transpose(0, 1)
@@ -89,7 +89,7 @@ class DecodeProblem:
         self.scale = 1.0 / math.sqrt(D)
 
     def run(self, **kw):
-        return tq.decode_paged(self.kc, self.vc, self.q, self.k_pages, self.v_pages, self.block_tables,
+        return tq.decode_paged(self.kc, self.vc, self.q, self.k_pages, self.v_pages, self.bs, self.block_tables,
                                self.seq_lens, self.max_seq_len, self.k_win if self.window else None,
                                self.v_win if self.window else None, self.window, self.scale, **kw)
 
@@ -104,8 +104,8 @@ class DecodeProblem:
             kp = self.k_pages[blocks][:, h:h + 1].cpu().numpy()
             vp = self.v_pages[blocks][:, h:h + 1].cpu().numpy()
         else:
-            kp = np.zeros((1, 1, self.bs, self.kc.row_bytes), np.uint8)
-            vp = np.zeros((1, 1, self.bs, self.vc.row_bytes), np.uint8)
+            kp = np.zeros((1, 1, self.bs * self.kc.row_bytes), np.uint8)
+            vp = np.zeros((1, 1, self.bs * self.vc.row_bytes), np.uint8)
         table = np.arange(max(nblk, 1))[None]
         q = self.q[b:b + 1, hq:hq + 1].float().cpu().numpy().astype(np.float64)
         kw = self.k_win[b:b + 1, h:h + 1].float().cpu().numpy().astype(np.float64)

@@ -68,11 +68,11 @@ def test_decode_full_small_workload():
     L = int(layout.seq_lens[0])
     k, v = W.sequence_kv(w, 0, 0, L, device="cuda")
     slots = W.slot_mapping(layout, 0, 0, L, w.block_size)
-    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp)
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, w.block_size)
     q = W.queries(w, device="cuda")
     bt = torch.as_tensor(layout.block_tables, device="cuda")
     sl = torch.as_tensor(layout.seq_lens.astype(np.int32), device="cuda")
-    out = tq.decode_paged(kc, vc, q, kp, vp, bt, sl, L, None, None, 0, 1 / math.sqrt(D))
+    out = tq.decode_paged(kc, vc, q, kp, vp, w.block_size, bt, sl, L, None, None, 0, 1 / math.sqrt(D))
     torch.cuda.synchronize()
     ref = O.decode_attention(q.float().cpu().numpy().astype(np.float64), kp.cpu().numpy(), vp.cpu().numpy(),
                              layout.block_tables, layout.seq_lens, None, None, 0, 1 / math.sqrt(D), kf, vf,
@@ -103,15 +103,16 @@ def test_decode_argument_errors():
     with pytest.raises(ValueError):
         prob.run(workspace=small)
     with pytest.raises(ValueError):
-        tq.decode_paged(prob.kc, prob.vc, prob.q, prob.k_pages, prob.v_pages, prob.block_tables, prob.seq_lens,
+        tq.decode_paged(prob.kc, prob.vc, prob.q, prob.k_pages, prob.v_pages, prob.bs, prob.block_tables, prob.seq_lens,
                         prob.max_seq_len, None, None, 4, prob.scale)
     q3 = torch.zeros(1, 3, D, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(tq.UnsupportedFormatError):  # 3 query heads per KV head
-        tq.decode_paged(prob.kc, prob.vc, q3, prob.k_pages, prob.v_pages, prob.block_tables, prob.seq_lens,
+        tq.decode_paged(prob.kc, prob.vc, q3, prob.k_pages, prob.v_pages, prob.bs, prob.block_tables, prob.seq_lens,
                         prob.max_seq_len, None, None, 0, prob.scale)
     prob2 = DecodeProblem([40], 2, 2, U4, U4, window=0, block_size=16, seed=4)
     with pytest.raises(ValueError):  # 3 query heads over 2 KV heads
-        tq.decode_paged(prob2.kc, prob2.vc, q3, prob2.k_pages, prob2.v_pages, prob2.block_tables, prob2.seq_lens,
+        tq.decode_paged(prob2.kc, prob2.vc, q3, prob2.k_pages, prob2.v_pages, prob2.bs, prob2.block_tables,
+                        prob2.seq_lens,
                         prob2.max_seq_len, None, None, 0, prob2.scale)
 
 
@@ -138,7 +139,7 @@ def _workload_problem(name, n_seq):
             t1 = min(P, t0 + 16384)
             k, v = W.sequence_kv(w, b, t0, t1, device="cuda")
             slots = W.slot_mapping(layout, b, t0, t1, w.block_size)
-            tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp)
+            tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, w.block_size)
     kw, vw = W.windows(w, layout, device="cuda")
     return w, kc, vc, kf, vf, layout, kp, vp, kw, vw
 
@@ -152,7 +153,8 @@ def test_decode_full_size_workloads_sampled(name):
     sl = torch.as_tensor(layout.seq_lens.astype(np.int32), device="cuda")
     maxL = int(layout.seq_lens.max())
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = tq.decode_paged(kc, vc, q, kp, vp, bt, sl, maxL, kw, vw, w.window, 1 / math.sqrt(D), d_err=err)
+    out = tq.decode_paged(kc, vc, q, kp, vp, w.block_size, bt, sl, maxL, kw, vw, w.window, 1 / math.sqrt(D),
+                          d_err=err)
     torch.cuda.synchronize()
     assert err.item() == 0
     got = out.cpu().numpy()

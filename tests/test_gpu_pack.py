@@ -22,6 +22,12 @@ FORMATS = [((4,), (128,)), ((3,), (128,)), ((2,), (128,)), ((4, 3), (64, 64)), (
            ((3, 2), (16, 112)), ((2, 4), (112, 16))]
 
 
+def rows_of(pages, slots, bs, fmt, H):
+    """Logical rows [n][H][row_bytes] of the given slots, read by the oracle's address formula."""
+    slots = np.asarray(slots, dtype=np.int64)
+    return np.stack([O.read_rows(pages, slots // bs, h, slots % bs, fmt, bs) for h in range(H)], axis=1)
+
+
 def compare_rows(gpu_rows, k_cpu, fmt, heads):
     """Compare GPU rows [N][H][row] with the oracle's quantization of k_cpu [N][H][d].
 
@@ -60,7 +66,7 @@ def test_pack_matches_oracle(kfmt, T, H, bs):
     slots[::7] = -1  # padding tokens
     kp, vp = tq.page_pool(kc, nb, bs), tq.page_pool(vc, nb, bs)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, d_err=err)
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, bs, d_err=err)
     torch.cuda.synchronize()
     assert err.item() == 0
     kcpu = k.float().cpu().numpy().astype(np.float64)
@@ -70,15 +76,16 @@ def test_pack_matches_oracle(kfmt, T, H, bs):
     gk, gv = kp.cpu().numpy(), vp.cpu().numpy()
     s = slots[live]
     for g, ref, src, f in ((gk, ref_kp, kcpu, kf), (gv, ref_vp, vcpu, vf)):
-        rows = g[s // bs, :, s % bs]
+        rows = rows_of(g, s, bs, f, H)
         compare_rows(rows, src[live], f, range(H))
         # bytes of slots nobody wrote stay zero, as in the oracle's pool
-        written = np.zeros((nb, bs), bool)
-        written[s // bs, s % bs] = True
-        assert not g.transpose(0, 2, 1, 3)[~written].any()
+        written = np.zeros(nb * bs, bool)
+        written[s] = True
+        free = np.nonzero(~written)[0]
+        assert not rows_of(g, free, bs, f, H).any()
         # where no index sits near a boundary the whole row is byte-identical
         if len(s):
-            same = (rows == ref[s // bs, :, s % bs]).all(axis=-1)
+            same = (rows == rows_of(ref, s, bs, f, H)).all(axis=-1)
             assert same.mean() > 0.99
             assert (rows[..., -2:] != 0).any(axis=-1).mean() > 0.99  # norms were written
 
@@ -91,11 +98,11 @@ def test_pack_reconstruction_mse_within_two_percent():
     gen.manual_seed(77)
     k, v = random_kv(T, H, gen)
     kp, vp = tq.page_pool(kc, T // 16, 16), tq.page_pool(vc, T // 16, 16)
-    tq.pack_kv(kc, vc, k, v, torch.arange(T, device="cuda"), kp, vp)
+    tq.pack_kv(kc, vc, k, v, torch.arange(T, device="cuda"), kp, vp, 16)
     torch.cuda.synchronize()
     for pages, src, f in ((kp, k, kf), (vp, v, vf)):
         x = src.float().cpu().numpy().astype(np.float64)
-        g = pages.cpu().numpy().reshape(T // 16, H, 16, -1).transpose(0, 2, 1, 3).reshape(T, H, -1)
+        g = rows_of(pages.cpu().numpy(), np.arange(T), 16, f, H)
         mse_gpu = mse_ref = 0.0
         for h in range(H):
             f1 = slice_format(f, h)
@@ -119,7 +126,7 @@ def test_pack_edge_values():
     k[5] = torch.linspace(-300, 300, D, device="cuda").to(torch.bfloat16)
     v = k.flip(0).contiguous()
     kp, vp = tq.page_pool(kc, 1, 8), tq.page_pool(vc, 1, 8)
-    tq.pack_kv(kc, vc, k, v, torch.arange(T, device="cuda"), kp, vp)
+    tq.pack_kv(kc, vc, k, v, torch.arange(T, device="cuda"), kp, vp, 8)
     torch.cuda.synchronize()
     rk, rv = O.pack_kv(k.float().cpu().numpy(), v.float().cpu().numpy(), np.arange(T), kf, vf, 1, 8)
     assert np.array_equal(kp.cpu().numpy(), rk)
@@ -131,9 +138,9 @@ def test_pack_empty_and_all_padding():
     vc, _ = codec_pair(2, (4,), (128,), 1)
     kp, vp = tq.page_pool(kc, 2, 16), tq.page_pool(vc, 2, 16)
     e = torch.empty(0, 2, D, dtype=torch.bfloat16, device="cuda")
-    tq.pack_kv(kc, vc, e, e, torch.empty(0, dtype=torch.int64, device="cuda"), kp, vp)
+    tq.pack_kv(kc, vc, e, e, torch.empty(0, dtype=torch.int64, device="cuda"), kp, vp, 16)
     k = torch.randn(5, 2, D, device="cuda").to(torch.bfloat16)
-    tq.pack_kv(kc, vc, k, k, torch.full((5,), -1, dtype=torch.int64, device="cuda"), kp, vp)
+    tq.pack_kv(kc, vc, k, k, torch.full((5,), -1, dtype=torch.int64, device="cuda"), kp, vp, 16)
     torch.cuda.synchronize()
     assert not kp.any() and not vp.any()
 
@@ -144,15 +151,17 @@ def test_pack_slot_outside_pool_sets_error_and_skips(monkeypatch):
     kp, vp = tq.page_pool(kc, 2, 4), tq.page_pool(vc, 2, 4)
     k = torch.randn(3, 1, D, device="cuda").to(torch.bfloat16)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    tq.pack_kv(kc, vc, k, k, torch.tensor([0, 8, 5], device="cuda"), kp, vp, d_err=err)
+    tq.pack_kv(kc, vc, k, k, torch.tensor([0, 8, 5], device="cuda"), kp, vp, 4, d_err=err)
     torch.cuda.synchronize()
     assert err.item() & tq.TQ_DERR_SLOT
-    assert kp[0, 0, 0].any() and kp[1, 0, 1].any()
-    assert not kp.view(-1, kp.shape[-1])[[1, 2, 3, 4, 6, 7]].any()
+    f = O.Format(D, 1, (4,), (128,), None, 0)
+    rows = rows_of(kp.cpu().numpy(), np.arange(8), 4, f, 1)
+    assert rows[0].any() and rows[5].any()
+    assert not rows[[1, 2, 3, 4, 6, 7]].any()
     monkeypatch.setenv("TQ_CHECKED", "1")
     err.zero_()
     with pytest.raises(IndexError):
-        tq.pack_kv(kc, vc, k, k, torch.tensor([0, 8, 5], device="cuda"), kp, vp, d_err=err)
+        tq.pack_kv(kc, vc, k, k, torch.tensor([0, 8, 5], device="cuda"), kp, vp, 4, d_err=err)
 
 
 def test_pack_argument_errors():
@@ -161,9 +170,11 @@ def test_pack_argument_errors():
     kp = tq.page_pool(kc, 2, 4)
     k = torch.randn(3, 2, D, device="cuda").to(torch.bfloat16)
     with pytest.raises(ValueError):
-        tq.pack_kv(kc, vc1, k, k, torch.arange(3, device="cuda"), kp, tq.page_pool(vc1, 2, 4))
+        tq.pack_kv(kc, vc1, k, k, torch.arange(3, device="cuda"), kp, tq.page_pool(vc1, 2, 4), 4)
     with pytest.raises(ValueError):
-        tq.pack_kv(kc, kc, k.float(), k, torch.arange(3, device="cuda"), kp, kp)
+        tq.pack_kv(kc, kc, k.float(), k, torch.arange(3, device="cuda"), kp, kp, 4)
+    with pytest.raises(ValueError):  # pool shaped for another block size
+        tq.pack_kv(kc, kc, k, k, torch.arange(3, device="cuda"), kp, kp, 8)
 
 
 def test_pack_workload_sample_full_size():
@@ -173,7 +184,7 @@ def test_pack_workload_sample_full_size():
     k, v, slots, layout = W.pack_batch(w, device="cuda")
     kp, vp = tq.page_pool(kc, layout.num_blocks, w.block_size), tq.page_pool(vc, layout.num_blocks, w.block_size)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, d_err=err)
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, w.block_size, d_err=err)
     torch.cuda.synchronize()
     assert err.item() == 0
     rng = np.random.default_rng(3)
@@ -181,8 +192,10 @@ def test_pack_workload_sample_full_size():
     s = slots[pick]
     flips = total = 0
     for pages, src, f in ((kp, k, kf), (vp, v, vf)):
-        rows = pages[torch.as_tensor(s // w.block_size, device="cuda"), :, torch.as_tensor(s % w.block_size, device="cuda")]
+        sub = pages[torch.as_tensor(s // w.block_size, device="cuda")].cpu().numpy()  # the touched sub-pages
+        rows = np.stack([O.read_rows(sub, np.arange(len(s)), h, s % w.block_size, f, w.block_size)
+                         for h in range(w.num_kv_heads)], axis=1)
         x = src[torch.as_tensor(pick, device="cuda")].float().cpu().numpy().astype(np.float64)
-        a, b = compare_rows(rows.cpu().numpy(), x, f, range(w.num_kv_heads))
+        a, b = compare_rows(rows, x, f, range(w.num_kv_heads))
         flips, total = flips + a, total + b
     assert flips <= MAX_FLIP_FRACTION * total

@@ -271,6 +271,12 @@ def test_reconstruction_error_matches_codebook_distortion(name):
 
 # --- pages, addressing --------------------------------------------------------
 
+def _hand_row(pages, blk, head, off, ib, bs):
+    """Row bytes read by hand from a (block, head) sub-page: index bytes, then the norm."""
+    sub = bytes(pages[blk, head])
+    return sub[off * ib:(off + 1) * ib] + sub[bs * ib + 2 * off: bs * ib + 2 * off + 2]
+
+
 def test_pack_addressing_by_formula():
     rng = np.random.default_rng(4)
     H, bs, nb, T = 2, 4, 6, 17
@@ -286,13 +292,18 @@ def test_pack_addressing_by_formula():
                 continue
             ki, kn, _ = O.quantize(k[t, h][None], kf, h)
             vi, vn, _ = O.quantize(v[t, h][None], vf, h)
-            assert np.array_equal(O.read_row(kp, slots[t], h, bs), O.encode_rows(ki, kn, kf)[0])
-            assert np.array_equal(O.read_row(vp, slots[t], h, bs), O.encode_rows(vi, vn, vf)[0])
+            assert np.array_equal(O.read_row(kp, slots[t], h, bs, kf), O.encode_rows(ki, kn, kf)[0])
+            assert np.array_equal(O.read_row(vp, slots[t], h, bs, vf), O.encode_rows(vi, vn, vf)[0])
+            # the same bytes, located by hand: index bytes at off*ib, the norm at bs*ib + 2*off
+            blk, off = divmod(int(slots[t]), bs)
+            row = _hand_row(kp, blk, h, off, O.index_bytes(kf), bs)
+            assert row == bytes(O.encode_rows(ki, kn, kf)[0])
     written = {(s // bs, s % bs) for s in slots if s >= 0}
     for blk in range(nb):
         for off in range(bs):
             if (blk, off) not in written:
-                assert not kp[blk, :, off].any()
+                for h in range(H):
+                    assert not any(_hand_row(kp, blk, h, off, O.index_bytes(kf), bs))
     with pytest.raises(IndexError):
         O.pack_kv(k, v, np.full(T, nb * bs), kf, vf, nb, bs)
 
@@ -317,7 +328,7 @@ def test_attention_single_token_returns_its_value():
     kp, vp, table = _pages_for(k, v, kf, vf, 16, rng)
     q = rng.standard_normal((1, 4, D))
     out = O.decode_attention(q, kp, vp, table[None], [1], None, None, 0, 0.1, kf, vf, 16)
-    vi, vn = O.decode_rows(vp[table[0], 0, 0][None], vf)
+    vi, vn = O.decode_rows(O.read_rows(vp, [table[0]], 0, [0], vf, 16), vf)
     vhat = O.dequantize_rows(vi, vn, vf, 0)[0]
     for g in range(4):
         assert np.allclose(out[0, g], vhat, atol=1e-13)
@@ -346,7 +357,7 @@ def test_attention_window_only_is_dense_softmax_by_hand():
     kw[0, 0, :L] = rng.standard_normal((L, d))
     vw[0, 0, :L] = rng.standard_normal((L, d))
     q = rng.standard_normal((1, 1, d))
-    pages = np.zeros((1, 1, 4, O.row_bytes(kf)), dtype=np.uint8)
+    pages = np.zeros((1, 1, 4 * O.row_bytes(kf)), dtype=np.uint8)
     out = O.decode_attention(q, pages, pages, np.zeros((1, 1), np.int64), [L], kw, vw, W, 0.2, kf, vf, 4)
     s = [0.2 * sum(q[0, 0, j] * kw[0, 0, t, j] for j in range(d)) for t in range(L)]
     m = max(s)
@@ -411,8 +422,8 @@ def test_attention_bruteforce_tiny():
     maxb = 2
     tables = np.array([[4, 1], [0, 3]])
     nb = 5
-    kp = np.zeros((nb, H, bs, O.row_bytes(kf)), np.uint8)
-    vp = np.zeros((nb, H, bs, O.row_bytes(vf)), np.uint8)
+    kp = np.zeros((nb, H, bs * O.row_bytes(kf)), np.uint8)
+    vp = np.zeros((nb, H, bs * O.row_bytes(vf)), np.uint8)
     kw = np.zeros((B, H, W, d))
     vw = np.zeros((B, H, W, d))
     hist_k, hist_v = {}, {}
@@ -450,8 +461,8 @@ def test_attention_bruteforce_tiny():
             keys, vals = [], []
             for t in range(P):
                 blk, off = tables[b][t // bs], t % bs
-                keys.append(hand_dequant(kp[blk, h, off], kf, h))
-                vals.append(hand_dequant(vp[blk, h, off], vf, h))
+                keys.append(hand_dequant(_hand_row(kp, blk, h, off, O.index_bytes(kf), bs), kf, h))
+                vals.append(hand_dequant(_hand_row(vp, blk, h, off, O.index_bytes(vf), bs), vf, h))
             for t in range(L - P):
                 keys.append(list(kw[b, h, t]))
                 vals.append(list(vw[b, h, t]))
