@@ -305,10 +305,10 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
         return false;
     const int G = num_q_heads / num_kv_heads;
     if (G > 16) return false;
-    // Aim for about 2048 packed work items per call, splits of 256..8192 tokens.
+    // Aim for about 4096 packed work items per call, splits of 512..8192 tokens.
     double total = static_cast<double>(std::max(max_seq_len, 1)) * std::max(batch, 1) * num_kv_heads;
-    int64_t s = static_cast<int64_t>(std::ceil(total / 2048.0));
-    s = std::min<int64_t>(std::max<int64_t>(s, 256), 8192);
+    int64_t s = static_cast<int64_t>(std::ceil(total / 4096.0));
+    s = std::min<int64_t>(std::max<int64_t>(s, 512), 8192);
     s = (s + 63) / 64 * 64;
     s = (s + block_size - 1) / block_size * block_size;
     plan->split_tokens = static_cast<int32_t>(s);

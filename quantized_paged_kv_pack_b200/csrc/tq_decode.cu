@@ -20,6 +20,8 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
+#include <string>
 
 #include "tq_internal.h"
 
@@ -29,26 +31,6 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kWarps = 4;
 constexpr float kLog2e = 1.4426950408889634f;
-
-struct DecodeArgs {
-    DevCodec kc, vc;
-    const __nv_bfloat16* q;
-    const uint8_t* k_pages;
-    const uint8_t* v_pages;
-    const int32_t* block_tables;
-    int32_t max_blocks;
-    const int32_t* seq_lens;
-    int32_t batch, num_q_heads, max_seq_len;
-    const __nv_bfloat16* k_win;
-    const __nv_bfloat16* v_win;
-    int32_t window;
-    float scale_log2;  // softmax_scale * log2(e)
-    int64_t num_blocks;
-    int32_t block_size;
-    int32_t split_tokens, max_splits, items_per_unit;
-    float* ws;
-    int* d_err;
-};
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -110,7 +92,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
     // Query prep: q_r = pi_K(H(s_K q)/sqrt(d)) * scale * log2(e) for packed items;
     // q * scale * log2(e) in the original domain for the window item.
     for (int g = warp; g < G; g += kWarps) {
-        const __nv_bfloat16* qp = a.q + (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
+        const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q) +
+                                  (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
         float z[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) z[i] = __bfloat162float(qp[4 * lane + i]);
@@ -156,8 +139,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
             const int64_t base = ((static_cast<int64_t>(b) * H + h) * a.window + t) * kHeadDim + 4 * lane;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                kv[i] = __bfloat162float(a.k_win[base + i]);
-                vv[i] = __bfloat162float(a.v_win[base + i]);
+                kv[i] = __bfloat162float(static_cast<const __nv_bfloat16*>(a.k_win)[base + i]);
+                vv[i] = __bfloat162float(static_cast<const __nv_bfloat16*>(a.v_win)[base + i]);
             }
         } else {
             int64_t blk = a.block_tables[static_cast<int64_t>(b) * a.max_blocks + t / bs];
@@ -331,12 +314,18 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
         return fail(TQ_ERR_VALUE, "null buffer");
     if (window > 0 && (!k_win || !v_win)) return fail(TQ_ERR_VALUE, "window > 0 needs k_win and v_win");
     if (num_blocks < 0 || max_blocks_per_seq < 0) return fail(TQ_ERR_VALUE, "negative size");
+    if (max_seq_len > window && num_blocks < 1) return fail(TQ_ERR_VALUE, "packed tokens need at least one block");
+    if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 15)
+        return fail(TQ_ERR_VALUE, "page pools must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(q) & 7) || (window > 0 && ((reinterpret_cast<uintptr_t>(k_win) |
+                                                                reinterpret_cast<uintptr_t>(v_win)) & 7)))
+        return fail(TQ_ERR_VALUE, "q and the windows must be 8-byte aligned");
     if (static_cast<int64_t>(max_blocks_per_seq) * block_size < static_cast<int64_t>(max_seq_len) - window)
         return fail(TQ_ERR_VALUE, "max_blocks_per_seq * block_size cannot hold max_seq_len - window tokens");
     DecodeArgs a;
     a.kc = kc->dev;
     a.vc = vc->dev;
-    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.q = q;
     a.k_pages = static_cast<const uint8_t*>(k_pages);
     a.v_pages = static_cast<const uint8_t*>(v_pages);
     a.block_tables = block_tables;
@@ -345,8 +334,8 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     a.batch = batch;
     a.num_q_heads = num_q_heads;
     a.max_seq_len = max_seq_len;
-    a.k_win = static_cast<const __nv_bfloat16*>(k_win);
-    a.v_win = static_cast<const __nv_bfloat16*>(v_win);
+    a.k_win = k_win;
+    a.v_win = v_win;
     a.window = window;
     a.scale_log2 = softmax_scale * kLog2e;
     a.num_blocks = num_blocks;
@@ -357,6 +346,16 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     a.ws = static_cast<float*>(workspace);
     a.d_err = d_err;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Tensor-core kernel for the formats it is instantiated for (block sizes a
+    // multiple of 16); the general kernel covers every other valid format.
+    // TQ_DECODE_KERNEL=general selects the general kernel (for cross-checks).
+    const char* force = std::getenv("TQ_DECODE_KERNEL");
+    if (!(force && std::string(force) == "general")) {
+        st = launch_decode_mma(a, kc, vc, plan.group, stream);
+        if (st == TQ_OK) return finish(s, d_err, "decode partials");
+        if (st != TQ_ERR_UNSUPPORTED) return st;
+        clear_error();
+    }
     dim3 grid(plan.items_per_unit, kc->desc.num_kv_heads, batch);
     switch (plan.group) {
         case 1: decode_partials_kernel<1><<<grid, kWarps * 32, 0, s>>>(a); break;

@@ -30,6 +30,27 @@ struct DevCodec {
     int32_t row_bytes;
 };
 
+// Arguments of the decode kernels (device pointers; see tq_decode_paged).
+struct DecodeArgs {
+    DevCodec kc, vc;
+    const void* q;                 // bf16 [B][H_q][128]
+    const uint8_t* k_pages;
+    const uint8_t* v_pages;
+    const int32_t* block_tables;
+    int32_t max_blocks;
+    const int32_t* seq_lens;
+    int32_t batch, num_q_heads, max_seq_len;
+    const void* k_win;             // bf16 [B][H_kv][window][128]
+    const void* v_win;
+    int32_t window;
+    float scale_log2;              // softmax_scale * log2(e)
+    int64_t num_blocks;
+    int32_t block_size;
+    int32_t split_tokens, max_splits, items_per_unit;
+    float* ws;
+    int* d_err;
+};
+
 }  // namespace tq
 
 struct tq_codec {
@@ -74,5 +95,11 @@ struct SplitPlan {
 };
 bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,
                      int32_t block_size, SplitPlan* plan);
+
+// Tensor-core decode partials. Returns TQ_ERR_UNSUPPORTED (without launching)
+// when the formats or the block size have no instantiation; the caller then
+// uses the general kernel.
+tq_status launch_decode_mma(const DecodeArgs& a, const tq_codec* kc, const tq_codec* vc, int group,
+                            void* stream);
 
 }  // namespace tq

@@ -175,3 +175,14 @@ def test_decode_full_size_workloads_sampled(name):
                                      slice_format(kf, h), slice_format(vf, h), w.block_size)[0, 0]
             assert np.abs(got[b, hq] - ref).max() <= ATOL
             assert np.abs(ref).max() > 0.5
+
+
+def test_tensor_core_and_general_kernels_agree(monkeypatch):
+    """Formats with a tensor-core instantiation against the general kernel on the same cache."""
+    prob = DecodeProblem([3000, 17, 260], 2, 8, M35, M35, window=32, block_size=16, seed=21)
+    fast = prob.run().clone()
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "general")
+    general = prob.run()
+    torch.cuda.synchronize()
+    assert (fast - general).abs().max().item() <= ATOL
+    check(prob)
