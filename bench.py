@@ -431,7 +431,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = WL.WORKLOADS[args.workload]
+    w = workload_of(args)
     kspec, vspec = WL.codec_specs(w)
     lay = WL.page_layout(w)
     from oracle import tq_oracle as O
@@ -456,13 +456,66 @@ def run_reference(args):
     return 0
 
 
+def workload_of(args):
+    w = WL.WORKLOADS[args.workload]
+    if args.batch:
+        w = WL.Workload(**{**w.__dict__, "batch": args.batch})
+    return w
+
+
+def run_pack(args, w, dist_ctx, rank, world):
+    """Headline on the pack workload: one step = tq_pack_kv over the whole batch."""
+    setup = PackSetup(w)
+    ms = measure_pack(setup, args.steps, args.warmup)
+    ms = max_over_ranks(ms, dist_ctx)
+    peak, peak_kind = peaks()
+    nbytes = setup.bytes()
+    hk, hv, hs = setup.k.cpu().pin_memory(), setup.v.cpu().pin_memory(), setup.slots.cpu().pin_memory()
+    herr = torch.zeros(1, dtype=torch.int32).pin_memory()
+
+    def e2e_step():
+        setup.k.copy_(hk, non_blocking=True)
+        setup.v.copy_(hv, non_blocking=True)
+        setup.slots.copy_(hs, non_blocking=True)
+        setup.step()
+        herr.copy_(setup.err, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    total, _ = time_steps([e2e_step], max(3, args.steps // 2), torch.cuda.current_stream())
+    e2e_ms = max_over_ranks(total / max(3, args.steps // 2), dist_ctx)
+    gbs = world * nbytes / (ms * 1e-3) / 1e9
+    line = {"metric": "TQ pack HBM GB/s (algorithmic bytes / step time)", "value": gbs, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+            "config": {"workload": w.name, "description": w.description, "batch": w.batch,
+                       "l2": f"no flush: {nbytes / 1e9:.2f} GB moved per step, L2 is 126 MB"},
+            "tokens_per_s": world * setup.k.shape[0] / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "kernel": "pack", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / peak,
+                         "traffic": stored_traffic(w.name, "tq_pack.cu")},
+            "e2e": {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": hk.numel() * 2 + hv.numel() * 2 + hs.numel() * 8,
+                    "d2h_bytes_per_step": 4},
+            "gpu_launches": args.steps}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args):
     dist_ctx = init_dist()
     rank = dist_ctx.get_rank() if dist_ctx else 0
     world = dist_ctx.get_world_size() if dist_ctx else 1
     if world == 1:
         torch.cuda.set_device(0)
-    w = WL.WORKLOADS[args.workload]
+    w = workload_of(args)
+    if w.kind == "pack":
+        rc = run_pack(args, w, dist_ctx, rank, world)
+        if dist_ctx is not None:
+            dist_ctx.barrier()
+            dist_ctx.destroy_process_group()
+        return rc
     setup = DecodeSetup(w, seed_offset=rank)
     step_ms, parts, clocks = measure_decode(setup, args.steps, args.warmup, dist_ctx)
     e2e_ms, h2d, d2h = measure_decode_e2e(setup, max(3, args.steps // 2), args.warmup)
@@ -541,6 +594,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(WL.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (small profiling cases)")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")

@@ -53,6 +53,7 @@ typedef enum {
 #define TQ_DERR_SLOT 1      /* tq_pack_kv: slot >= num_blocks * block_size (row skipped) */
 #define TQ_DERR_BLOCK 2     /* tq_decode_paged: block table entry outside [0, num_blocks) */
 #define TQ_DERR_TIMEOUT 4   /* a kernel's bounded wait expired; its results are invalid */
+#define TQ_DERR_LAUNCH 8    /* a kernel could not lay out its shared memory; its results are invalid */
 
 /*
  * One codec (format) for the keys or for the values of a layer.

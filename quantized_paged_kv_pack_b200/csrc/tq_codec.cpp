@@ -305,10 +305,11 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
         return false;
     const int G = num_q_heads / num_kv_heads;
     if (G > 16) return false;
-    // Aim for about 4096 packed work items per call, splits of 512..8192 tokens.
+    // Aim for about 4096 packed work items per call, splits of 512..4096 tokens
+    // (at most 32 tiles of 16 tokens for each of a CTA's 8 warps).
     double total = static_cast<double>(std::max(max_seq_len, 1)) * std::max(batch, 1) * num_kv_heads;
     int64_t s = static_cast<int64_t>(std::ceil(total / 4096.0));
-    s = std::min<int64_t>(std::max<int64_t>(s, 512), 8192);
+    s = std::min<int64_t>(std::max<int64_t>(s, 512), 4096);
     s = (s + 63) / 64 * 64;
     s = (s + block_size - 1) / block_size * block_size;
     plan->split_tokens = static_cast<int32_t>(s);
@@ -316,8 +317,11 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
     plan->items_per_unit = plan->max_splits + 1;
     plan->group = G;
     plan->record_floats = static_cast<size_t>(G) * (kHeadDim + 2);
-    plan->workspace_bytes = static_cast<size_t>(batch) * num_kv_heads * plan->items_per_unit *
-                            plan->record_floats * sizeof(float);
+    plan->record_bytes = static_cast<size_t>(batch) * num_kv_heads * plan->items_per_unit * plan->record_floats *
+                         sizeof(float);
+    plan->record_bytes = (plan->record_bytes + 255) / 256 * 256;
+    // then the rotated queries: [batch][num_q_heads][128] fp32
+    plan->workspace_bytes = plan->record_bytes + static_cast<size_t>(batch) * num_q_heads * kHeadDim * sizeof(float);
     return true;
 }
 

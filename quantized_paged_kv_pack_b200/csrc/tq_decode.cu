@@ -287,6 +287,7 @@ tq_status finish(cudaStream_t s, int32_t* d_err, const char* what) {
             if (cudaMemcpy(&h, d_err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
                 return fail(TQ_ERR_CUDA, "reading the device error word failed");
             if (h & TQ_DERR_TIMEOUT) return fail(TQ_ERR_TIMEOUT, "a bounded wait in the decode kernel expired");
+            if (h & TQ_DERR_LAUNCH) return fail(TQ_ERR_CUDA, "the decode kernel could not lay out shared memory");
             if (h & TQ_DERR_BLOCK) return fail(TQ_ERR_INDEX, "block table entry or length outside the pages");
         }
     }
@@ -344,6 +345,7 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     a.max_splits = plan.max_splits;
     a.items_per_unit = plan.items_per_unit;
     a.ws = static_cast<float*>(workspace);
+    a.qrot = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.record_bytes);
     a.d_err = d_err;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // Tensor-core kernel for the formats it is instantiated for (block sizes a

@@ -47,7 +47,8 @@ struct DecodeArgs {
     int64_t num_blocks;
     int32_t block_size;
     int32_t split_tokens, max_splits, items_per_unit;
-    float* ws;
+    float* ws;                     // records [B][H_kv][items_per_unit][G][2 + 128]
+    float* qrot;                   // rotated, scaled queries [B][H_q][128] in K packed order
     int* d_err;
 };
 
@@ -91,10 +92,19 @@ struct SplitPlan {
     int32_t items_per_unit; // max_splits + 1 (the last one is the window)
     int32_t group;          // query heads per KV head
     size_t record_floats;   // floats per work item record
+    size_t record_bytes;    // bytes of all records (256-byte multiple); rotated queries follow
     size_t workspace_bytes;
 };
 bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,
                      int32_t block_size, SplitPlan* plan);
+
+// Uniform 4-bit pack on the tensor cores; TQ_ERR_UNSUPPORTED (nothing
+// launched) for other formats or unaligned pools.
+tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
+                         const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
+                         int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream);
+// Launch-error check (and TQ_CHECKED synchronisation) after a pack launch.
+tq_status finish_pack(struct CUstream_st* stream, int32_t* d_err);
 
 // Tensor-core decode partials. Returns TQ_ERR_UNSUPPORTED (without launching)
 // when the formats or the block size have no instantiation; the caller then

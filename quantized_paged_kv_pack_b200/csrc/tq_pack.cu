@@ -17,6 +17,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
+#include <string>
 
 #include "tq_internal.h"
 
@@ -173,12 +175,27 @@ extern "C" tq_status tq_pack_kv(const tq_codec* kc, const tq_codec* vc, const vo
     if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 1)
         return fail(TQ_ERR_VALUE, "page pools must be 2-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Tensor-core path for uniform 4-bit codecs; the general kernel covers
+    // every other format. TQ_PACK_KERNEL=general selects the general kernel.
+    const char* force = std::getenv("TQ_PACK_KERNEL");
+    if (!(force && std::string(force) == "general")) {
+        tq_status st = launch_pack_u4(kc, vc, k, v, slot_mapping, num_tokens, k_pages, v_pages, num_blocks,
+                                      block_size, d_err, stream);
+        if (st != TQ_OK && st != TQ_ERR_UNSUPPORTED) return st;
+        if (st == TQ_OK) return finish_pack(s, d_err);
+        clear_error();
+    }
     const int64_t n_vec = num_tokens * kc->desc.num_kv_heads * 2;
     const int64_t blocks = std::min<int64_t>((n_vec + kPackWarps - 1) / kPackWarps, 148 * 32);
     pack_rows_kernel<<<static_cast<unsigned>(blocks), kPackWarps * 32, 0, s>>>(
         kc->dev, vc->dev, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
         slot_mapping, num_tokens, static_cast<uint8_t*>(k_pages), static_cast<uint8_t*>(v_pages), num_blocks,
         block_size, d_err);
+    return finish_pack(s, d_err);
+}
+
+namespace tq {
+tq_status finish_pack(cudaStream_t s, int32_t* d_err) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(TQ_ERR_CUDA, std::string("pack launch: ") + cudaGetErrorString(e));
     if (checked_mode()) {
@@ -193,3 +210,4 @@ extern "C" tq_status tq_pack_kv(const tq_codec* kc, const tq_codec* vc, const vo
     }
     return TQ_OK;
 }
+}  // namespace tq

@@ -22,7 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtq.so")
 
 TQ_OK, TQ_ERR_VALUE, TQ_ERR_INDEX, TQ_ERR_NOT_FOUND, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_TIMEOUT = range(7)
-TQ_DERR_SLOT, TQ_DERR_BLOCK, TQ_DERR_TIMEOUT = 1, 2, 4
+TQ_DERR_SLOT, TQ_DERR_BLOCK, TQ_DERR_TIMEOUT, TQ_DERR_LAUNCH = 1, 2, 4, 8
 HEAD_DIM = 128
 
 

@@ -199,3 +199,52 @@ def test_pack_workload_sample_full_size():
         a, b = compare_rows(rows, x, f, range(w.num_kv_heads))
         flips, total = flips + a, total + b
     assert flips <= MAX_FLIP_FRACTION * total
+
+
+def test_pack_edge_values_uniform_4bit_fast_path():
+    """Zero, tiny, huge and one-hot vectors through the tensor-core pack (uniform 4-bit K and V)."""
+    H = 2
+    kc, kf = codec_pair(H, (4,), (128,), 3)
+    vc, vf = codec_pair(H, (4,), (128,), 4)
+    T = 20
+    k = torch.zeros(T, H, D, dtype=torch.bfloat16, device="cuda")
+    k[1] = 1e-30
+    k[2, :, 0] = 70000.0
+    k[3] = 3.0e-3
+    k[4, :, 5] = -2.5
+    k[5] = torch.linspace(-300, 300, D, device="cuda").to(torch.bfloat16)
+    k[6:] = torch.randn(T - 6, H, D, device="cuda").to(torch.bfloat16) * 7
+    v = k.flip(0).contiguous()
+    slots = torch.tensor([5, 0, 17, 3, -1, 8, 9, 10, 11, 12, 13, 14, 15, 16, 1, 2, 4, 6, 7, 18], device="cuda")
+    kp, vp = tq.page_pool(kc, 3, 8), tq.page_pool(vc, 3, 8)
+    tq.pack_kv(kc, vc, k, v, slots, kp, vp, 8)
+    torch.cuda.synchronize()
+    rk, rv = O.pack_kv(k.float().cpu().numpy(), v.float().cpu().numpy(), slots.cpu().numpy(), kf, vf, 3, 8)
+    assert np.array_equal(kp.cpu().numpy(), rk)
+    assert np.array_equal(vp.cpu().numpy(), rv)
+
+
+def test_fast_and_general_pack_kernels_agree(monkeypatch):
+    H, T, bs = 4, 700, 16
+    kc, kf = codec_pair(H, (4,), (128,), 8)
+    vc, vf = codec_pair(H, (4,), (128,), 9)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    k, v = random_kv(T, H, gen)
+    nb = -(-T // bs) + 2
+    slots = torch.as_tensor(np.random.default_rng(1).permutation(nb * bs)[:T], device="cuda")
+    out = []
+    for mode in ("fast", "general"):
+        if mode == "general":
+            monkeypatch.setenv("TQ_PACK_KERNEL", "general")
+        kp, vp = tq.page_pool(kc, nb, bs), tq.page_pool(vc, nb, bs)
+        tq.pack_kv(kc, vc, k, v, slots, kp, vp, bs)
+        torch.cuda.synchronize()
+        out.append((kp.cpu().numpy(), vp.cpu().numpy()))
+    s = slots.cpu().numpy()
+    for i, (src, f) in enumerate(((k, kf), (v, vf))):
+        x = src.float().cpu().numpy().astype(np.float64)
+        for pages in (out[0][i], out[1][i]):
+            compare_rows(rows_of(pages, s, bs, f, H), x, f, range(H))
+        same = (out[0][i] == out[1][i]).mean()
+        assert same > 0.999
