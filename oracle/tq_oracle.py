@@ -515,7 +515,8 @@ def decode_attention(q, k_pages, v_pages, block_tables, seq_lens, k_win, v_win, 
     For each sequence b and query head g (KV head g // G), the keys and values
     are the dequantized packed tokens 0..P_b-1, read through the block table,
     followed by the bf16 window tokens (R7). out = softmax(scale q.k) @ v.
-    Returns out[B][H_q][d] for the sequences in ``batch`` (all by default).
+    A sequence with no tokens gets a zero output. Returns out[B][H_q][d] for
+    the sequences in ``batch`` (all by default).
     """
     q = np.asarray(q, dtype=np.float64)
     B, Hq, d = q.shape
@@ -537,6 +538,8 @@ def decode_attention(q, k_pages, v_pages, block_tables, seq_lens, k_win, v_win, 
             if n_win:
                 keys = np.concatenate((keys, np.asarray(k_win[b, h, :n_win], dtype=np.float64)))
                 vals = np.concatenate((vals, np.asarray(v_win[b, h, :n_win], dtype=np.float64)))
+            if L == 0:
+                continue  # an empty history attends to nothing: the output stays zero
             for g in range(G):
                 out[ob, h * G + g] = dense_attention(q[b, h * G + g], keys, vals, scale)
     return out

@@ -110,8 +110,6 @@ class DecodeProblem:
         q = self.q[b:b + 1, hq:hq + 1].float().cpu().numpy().astype(np.float64)
         kw = self.k_win[b:b + 1, h:h + 1].float().cpu().numpy().astype(np.float64)
         vw = self.v_win[b:b + 1, h:h + 1].float().cpu().numpy().astype(np.float64)
-        if L == 0:
-            return np.zeros(D)
         return O.decode_attention(q, kp, vp, table, [L], kw, vw, self.window, self.scale,
                                   slice_format(self.kf, h), slice_format(self.vf, h), self.bs)[0, 0]
 

@@ -515,3 +515,12 @@ def test_ledger_counts_what_the_oracle_allocates():
     assert led.workspace_bytes == 123
     assert led.metadata_bytes == led.norm_bytes + led.codebook_bytes + led.transform_bytes + led.window_bytes \
         + led.block_table_bytes + 123
+
+
+def test_attention_empty_history_is_zero():
+    kf, vf = fmt((4,), (128,)), fmt((4,), (128,))
+    pages = np.zeros((1, 1, 4 * O.row_bytes(kf)), dtype=np.uint8)
+    q = np.ones((2, 2, D))
+    win = np.ones((2, 1, 3, D))
+    out = O.decode_attention(q, pages, pages, np.zeros((2, 1), np.int64), [0, 1], win, win, 3, 0.1, kf, vf, 4)
+    assert np.all(out[0] == 0) and np.allclose(out[1], 1.0)
