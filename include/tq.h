@@ -212,6 +212,33 @@ tq_status tq_decode_combine(const tq_codec* vc, const int32_t* seq_lens, int32_t
                             const void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * tq_decode_paged_static - tq_decode_paged without a caller-provided workspace.
+ * The pages have no counterpart of this call. It is for callers that cannot
+ * call cudaMalloc: code running inside another runtime that owns all device
+ * memory (for instance a serving engine that reserves the whole GPU for its
+ * page pool up front), or code on a path where cudaMalloc's implicit
+ * device-wide synchronization is not allowed. It allocates nothing: the
+ * split-K scratch is a fixed array of TQ_STATIC_WORKSPACE_BYTES in the
+ * library's device image, which every GPU that loads the library holds
+ * until the process exits.
+ *
+ * Arguments mean what they mean for tq_decode_paged. The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current) and caches it, so make that first call before any
+ * stream capture. A call whose tq_decode_workspace_bytes(...) exceeds
+ * TQ_STATIC_WORKSPACE_BYTES returns TQ_ERR_VALUE before launching anything.
+ * All calls share the array and it keeps the last call's contents (nothing
+ * in it needs to start at zero); calls whose kernels overlap on the GPU, on
+ * different streams or from different threads, race on it.
+ */
+#define TQ_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+tq_status tq_decode_paged_static(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
+                                 const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                 const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t max_seq_len,
+                                 const void* k_win, const void* v_win, int32_t window, float softmax_scale,
+                                 int64_t num_blocks, int32_t block_size, float* out, int32_t* d_err, void* stream);
+
+/*
  * Byte ledger ([Design] "System Invariants": storage bytes and metadata bytes
  * are reported separately; the ratio includes norms, codebooks, transforms,
  * recent windows and workspace). Host arithmetic only.

@@ -9,7 +9,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtq.so")
-SOURCES = ["tq_codec.cpp", "tq_pack.cu", "tq_pack_mma.cu", "tq_decode.cu", "tq_decode_mma.cu"]
+SOURCES = ["tq_codec.cpp", "tq_pack.cu", "tq_pack_mma.cu", "tq_decode.cu", "tq_decode_mma.cu", "tq_decode_static.cu"]
 
 
 def nvcc():

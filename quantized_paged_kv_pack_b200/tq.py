@@ -77,10 +77,11 @@ def lib():
         L.tq_decode_paged.argtypes = dec + [_VP, _VP, _SZ, _VP, _VP]
         L.tq_decode_partials.argtypes = dec + [_VP, _SZ, _VP, _VP]
         L.tq_decode_combine.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _SZ, _VP]
+        L.tq_decode_paged_static.argtypes = dec + [_VP, _VP, _VP]
         L.tq_byte_ledger.argtypes = [P(_FormatDesc), P(_FormatDesc), _I32, _VP, _I32, _I32, _I32, _I64, _I32,
                                      P(_Ledger)]
         for name in ("tq_codec_host_tables", "tq_make_codec", "tq_pack_kv", "tq_decode_paged",
-                     "tq_decode_partials", "tq_decode_combine", "tq_byte_ledger"):
+                     "tq_decode_partials", "tq_decode_combine", "tq_byte_ledger", "tq_decode_paged_static"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -304,6 +305,50 @@ def decode_paged(kc: Codec, vc: Codec, q: torch.Tensor, k_pages: torch.Tensor, v
                                    *ws, s))
     else:
         raise ValueError(f"unknown phase {phase!r}")
+    return out
+
+
+STATIC_WORKSPACE_BYTES = 32 << 20
+
+
+def decode_paged_static(kc: Codec, vc: Codec, q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                        block_size: int, block_tables: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
+                        k_win: Optional[torch.Tensor], v_win: Optional[torch.Tensor], window: int,
+                        softmax_scale: float, out: Optional[torch.Tensor] = None,
+                        d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode attention that allocates no device memory in the library (tq_decode_paged_static).
+
+    For callers that cannot call cudaMalloc (another runtime owns the device
+    memory, or the path may not take cudaMalloc's implicit synchronization):
+    the split-K scratch is a fixed array of STATIC_WORKSPACE_BYTES inside the
+    library, shared by every call, so calls that overlap on the GPU race.
+    ``out`` should be preallocated by such callers; if it is None this
+    wrapper creates it with torch for convenience.
+    """
+    if q.dim() != 3:
+        raise ValueError("q must be [batch][num_q_heads][head_dim]")
+    B, Hq, d = q.shape
+    H = kc.num_kv_heads
+    _need(q, torch.bfloat16, (B, Hq, kc.head_dim), "q")
+    nb = _pools(kc, vc, k_pages, v_pages, block_size)
+    if block_tables.dim() != 2:
+        raise ValueError("block_tables must be [batch][max_blocks_per_seq]")
+    _need(block_tables, torch.int32, (B, block_tables.shape[1]), "block_tables")
+    _need(seq_lens, torch.int32, (B,), "seq_lens")
+    if window > 0:
+        _need(k_win, torch.bfloat16, (B, H, window, kc.head_dim), "k_win")
+        _need(v_win, torch.bfloat16, (B, H, window, kc.head_dim), "v_win")
+    else:
+        k_win = v_win = None
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, (B, Hq, d), "out")
+    if d_err is not None:
+        _need(d_err, torch.int32, (1,), "d_err")
+    _check(lib().tq_decode_paged_static(
+        kc.handle, vc.handle, _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), block_tables.shape[1],
+        _ptr(seq_lens), B, Hq, int(max_seq_len), _ptr(k_win), _ptr(v_win), int(window), float(softmax_scale), nb,
+        int(block_size), _ptr(out), _ptr(d_err), _stream(stream)))
     return out
 
 
