@@ -493,7 +493,7 @@ def run_pack(args, w, dist_ctx, rank, world):
             "tokens_per_s": world * setup.k.shape[0] / (ms * 1e-3),
             "roofline": {"bound": "hbm", "kernel": "pack", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / peak,
-                         "traffic": stored_traffic(w.name, "tq_pack.cu")},
+                         "traffic": stored_traffic(w.name, "tq_pack_mma.cu")},
             "e2e": {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": hk.numel() * 2 + hv.numel() * 2 + hs.numel() * 8,
                     "d2h_bytes_per_step": 4},
@@ -542,7 +542,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": "decode_partials", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "frac_of_8TBs": achieved / 8000.0,
-                     "traffic": stored_traffic(w.name, "tq_decode.cu")},
+                     "traffic": stored_traffic(w.name, "tq_decode_mma.cu")},
         "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,
@@ -568,7 +568,7 @@ def run_ours(args):
                                "kv_tokens_per_s": setup.kv_tokens() / (ms * 1e-3), "ms_per_step": ms,
                                "decode_partials_GB/s": sb / (p[1] * 1e-3) / 1e9,
                                "decode_partials_frac": sb / (p[1] * 1e-3) / 1e9 / peak,
-                               "traffic": stored_traffic(name, "tq_decode.cu")}
+                               "traffic": stored_traffic(name, "tq_decode_mma.cu")}
             else:
                 del setup
                 torch.cuda.empty_cache()
@@ -576,7 +576,7 @@ def run_ours(args):
                 ms = measure_pack(setup, max(5, args.steps // 2), args.warmup)
                 gbs = setup.bytes() / (ms * 1e-3) / 1e9
                 extra[name] = {"GB/s": gbs, "tokens_per_s": setup.k.shape[0] / (ms * 1e-3), "ms_per_step": ms,
-                               "frac": gbs / peak, "traffic": stored_traffic(name, "tq_pack.cu")}
+                               "frac": gbs / peak, "traffic": stored_traffic(name, "tq_pack_mma.cu")}
                 line["gpu_launches"] += max(5, args.steps // 2)
         line["per_workload"] = extra
     if rank == 0:
