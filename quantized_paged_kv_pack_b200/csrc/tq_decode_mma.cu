@@ -23,14 +23,23 @@
 // two indices of a pair come from two tokens at the same coordinate, so the
 // lane first interleaves two tokens' index bits.
 //
-// Data movement: each warp owns a ring of 4 tile slots in shared memory that
-// its lane 0 fills with cp.async.bulk copies (index rows of K and V, and their
-// norms) tracked by one mbarrier per slot, running up to 4 tiles ahead and
-// across the boundary into the CTA's next work item. Every wait is bounded;
-// on expiry the kernel sets TQ_DERR_TIMEOUT, drains its copies (bounded) and
-// stops. CTAs are persistent and take work items (sequence, KV head, split of
-// the packed tokens, query-head group) in a fixed stride; the 8 warps share an
-// item's tiles and merge their (max, sum, accumulator) states at its end.
+// Data movement: each compute warp owns a ring of tile slots in shared
+// memory. A ninth warp, the producer, fills them with 16-byte cp.async copies
+// from all its lanes (index rows of K and V, and their norms) in the order the
+// warps consume them, tracked by a "full" mbarrier per slot; a warp releases a
+// slot through its "empty" mbarrier. The producer runs ahead across work items
+// and keeps the next item's block ids in shared memory, so the compute warps
+// carry no address or block-table arithmetic. (Per-tile bulk copies cost the
+// copy engine a fixed overhead per operation that, at a few hundred bytes per
+// operation, capped the rate well below HBM speed.) Every wait is bounded; on
+// expiry the kernel sets TQ_DERR_TIMEOUT, waits for its copies and stops.
+// CTAs are persistent and take work items (sequence, KV head, split of the
+// packed tokens, query-head group) in a fixed stride; the compute warps share
+// an item's tiles and merge their (max, sum, accumulator) states at its end.
+//
+// Online softmax: each warp keeps a reference max per head that moves only
+// when a score exceeds it by more than 2^8, so weights stay below 2^8 and the
+// common tile needs one vote and no shuffles or rescale.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -46,9 +55,15 @@ namespace tq {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kNW = 8;              // warps per CTA
-constexpr int kStages = 4;          // ring slots per warp
-constexpr int kStageBytes = 2176;   // 16 rows of K and V (<= 64 index bytes each) + 2 x 32 norm bytes
+#ifndef TQ_DECODE_WARPS
+#define TQ_DECODE_WARPS 8
+#endif
+constexpr int kNW = TQ_DECODE_WARPS;  // compute warps per CTA (plus one producer warp)
+static_assert(kNW >= 1 && kNW <= 11, "11 compute warps fill the shared memory");
+#ifndef TQ_DECODE_STAGES
+#define TQ_DECODE_STAGES 4
+#endif
+constexpr int kStages = TQ_DECODE_STAGES;  // ring slots per compute warp
 constexpr int kLut = 65536;         // bytes of the dequantization table
 constexpr uint32_t kSpinLimit = 1u << 24;
 constexpr float kSlack = 8.0f;                 // log2 slack of the running max
@@ -72,6 +87,13 @@ using U4 = Fmt<4, 128, 0, 0>;
 using U3 = Fmt<3, 128, 0, 0>;
 using M43 = Fmt<4, 64, 3, 64>;
 using M42 = Fmt<4, 32, 2, 96>;
+
+// Bytes of one ring slot: 16 index rows of K and of V, each followed by the
+// 16 norms (32 bytes); a multiple of 16, the copy granule.
+template <class KF, class VF>
+__host__ __device__ constexpr uint32_t stage_bytes() {
+    return 16 * (KF::IB + VF::IB) + 64;
+}
 
 template <int B, int E, class F>
 __device__ __forceinline__ void static_for(F&& f) {
@@ -136,20 +158,26 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+__device__ __forceinline__ void upk(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t x, uint64_t y) {
+    uint64_t v;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(x), "l"(y));
+    return v;
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 
-__device__ __forceinline__ void mbar_init(uint32_t bar) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
-    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}" ::"r"(bar),
-                 "r"(bytes)
-                 : "memory");
-}
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -159,13 +187,6 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
 // Bounded wait for phase `parity` of `bar`; false when the limit expired.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     for (uint32_t i = 0; i < kSpinLimit; ++i)
@@ -279,19 +300,12 @@ __device__ __forceinline__ uint32_t lut_base(uint32_t lane_base) {
 // ---- work items -----------------------------------------------------------------
 
 struct Item {
-    int b, h, hg, split, t0, t1;
+    int b, h, hg, split, t0, t1;  // h: the KV head (per-head items) or the first of 8 (block items)
     bool win;
 };
 
-// Geometry of slot `slot`; false when the slot has no work.
-__device__ __forceinline__ bool item_of(const DecodeArgs& a, int64_t slot, int head_groups, Item& it) {
-    int64_t t = slot;
-    it.hg = static_cast<int>(t % head_groups);
-    t /= head_groups;
-    it.h = static_cast<int>(t % a.kc.num_heads);
-    t /= a.kc.num_heads;
-    it.b = static_cast<int>(t % a.batch);
-    it.split = static_cast<int>(t / a.batch);
+// Token range of item `split` of sequence it.b; false when it has no tokens.
+__device__ __forceinline__ bool item_range(const DecodeArgs& a, Item& it) {
     int L = __ldg(a.seq_lens + it.b);
     L = L < 0 ? 0 : (L > a.max_seq_len ? a.max_seq_len : L);
     const int n_win = min(a.window, L), P = L - n_win;
@@ -303,61 +317,105 @@ __device__ __forceinline__ bool item_of(const DecodeArgs& a, int64_t slot, int h
     return true;
 }
 
-// Number of this warp's tiles in a packed item.
-__device__ __forceinline__ int warp_tiles(const Item& it, int warp) {
-    if (it.win) return 0;
-    const int n = (it.t1 - it.t0 + 15) >> 4;
-    return n > warp ? (n - warp + kNW - 1) / kNW : 0;
+// Work slot -> item. Per-head items: (query-head group, KV head, sequence,
+// split). Block items (HB = 8): the KV heads are taken 8 at a time.
+template <int HB>
+__device__ __forceinline__ bool item_of(const DecodeArgs& a, int64_t slot, int head_groups, Item& it) {
+    const int hblocks = a.kc.num_heads / HB;
+    int64_t t = slot;
+    it.hg = static_cast<int>(t % head_groups);
+    t /= head_groups;
+    it.h = static_cast<int>(t % hblocks) * HB;
+    t /= hblocks;
+    it.b = static_cast<int>(t % a.batch);
+    it.split = static_cast<int>(t / a.batch);
+    return item_range(a, it);
 }
 
-// Block id of this warp's k-th tile of an item, lane k holding entry k (k < 32).
-__device__ __forceinline__ int load_block_ids(const DecodeArgs& a, const Item& it, int warp, int lane) {
-    const int n = warp_tiles(it, warp);
-    int blk = 0;
-    if (lane < n) {
-        const int tok = it.t0 + 16 * (warp + lane * kNW);
-        blk = __ldg(a.block_tables + static_cast<int64_t>(it.b) * a.max_blocks + tok / a.block_size);
-        if (blk < 0 || blk >= a.num_blocks) {
-            if (a.d_err) atomicOr(a.d_err, TQ_DERR_BLOCK);
-            blk = 0;
-        }
-    }
-    return blk;
+// Next packed item of this CTA at or after `slot`; false when none is left.
+template <int HB>
+__device__ __forceinline__ bool next_packed(const DecodeArgs& a, int64_t& slot, int head_groups, int64_t total_slots,
+                                            Item& it) {
+    for (; slot < total_slots; slot += gridDim.x)
+        if (item_of<HB>(a, slot, head_groups, it) && !it.win) return true;
+    return false;
 }
 
-struct Smem {
-    float red_o[kNW][8][kHeadDim];         // per-warp value accumulators (V packed order)
-    float red_m[kNW][8], red_l[kNW][8];
-    unsigned long long bar[kNW][kStages];
-    int abort_flag;
-};
+constexpr int kMaxItemTiles = 256;  // 16-token tiles of one work item (at most)
 
-constexpr int kRingBytes = kNW * kStages * kStageBytes;
-constexpr size_t kSmemHead = (sizeof(Smem) + 127) / 128 * 128;
-constexpr size_t kFrontBytes = kSmemHead + kRingBytes;
-// Layout: [Smem][rings][pad to a 64 KB boundary][table]. The table needs the
-// window offset of the dynamic area to be small; the kernel checks.
-constexpr size_t kSmemBytes = (kFrontBytes + kLut - 1) / kLut * kLut + kLut;
+// ---- synchronisation and copies ----------------------------------------------------
 
-template <class KF, class VF, int NH>
-__global__ void __launch_bounds__(kNW * 32, 1) decode_mma_kernel(DecodeArgs a, LutValues tv, int group,
-                                                                 int head_groups, int64_t total_slots) {
-    static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
-    constexpr int NJ = NH / 4;  // n-tiles: 4 heads x {hi, lo} each
-    extern __shared__ __align__(128) uint8_t dsm[];
-    Smem& sm = *reinterpret_cast<Smem*>(dsm);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = lane >> 2, c = lane & 3;
-
-    const uint32_t dsm_addr = static_cast<uint32_t>(__cvta_generic_to_shared(dsm));
-    const uint32_t ring_addr = dsm_addr + static_cast<uint32_t>(kSmemHead);
-    const uint32_t lut_addr = (dsm_addr + static_cast<uint32_t>(kFrontBytes) + (kLut - 1)) & ~uint32_t(kLut - 1);
-    if (lut_addr + kLut > dsm_addr + kSmemBytes) {
-        if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
-        return;
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init_count(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}" ::"r"(bar),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded, warp-uniform poll (every lane of the warp calls it).
+__device__ __forceinline__ bool mbar_poll_warp(uint32_t bar, uint32_t parity) {
+    bool ready = false;
+    for (uint32_t i = 0; i < kSpinLimit && !ready; ++i) ready = __any_sync(kFull, mbar_test(bar, parity));
+    return ready;
+}
+// Bounded wait by one thread that polls with short sleeps in between: it
+// reacts within about 100 ns and leaves the issue slots to the compute warps.
+__device__ __forceinline__ bool mbar_sleep_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_test(bar, parity)) return true;
+        __nanosleep(64);
     }
-    uint32_t* table = reinterpret_cast<uint32_t*>(dsm + (lut_addr - dsm_addr));
-    for (int i = threadIdx.x; i < kLut / 4; i += kNW * 32) {
+    return false;
+}
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+template <int NTHREADS>
+__device__ __forceinline__ void named_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NTHREADS) : "memory");
+}
+
+__device__ __forceinline__ uint64_t mul2(uint64_t x, uint64_t y) {
+    uint64_t v;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(x), "l"(y));
+    return v;
+}
+__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+// fp16 split of a float pair: hi = rn(x), lo = rn(x - hi) per element.
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __half2 h = __floats2half2_rn(x0, x1);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = half2_bits(x0 - __low2float(h), x1 - __high2float(h));
+}
+__device__ __forceinline__ float f16_at(uint32_t addr) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(lds16(addr))));
+}
+
+// Fills the per-lane dequantization table (see the top of the file).
+__device__ __forceinline__ void fill_table(uint32_t* table, const LutValues& tv, int tid, int nthreads) {
+    for (int i = tid; i < kLut / 4; i += nthreads) {
         const int e = i >> 6, half = (i >> 5) & 1;
         __half2 v = __floats2half2_rn(0.0f, 0.0f);
         if (half == 0) {
@@ -369,396 +427,805 @@ __global__ void __launch_bounds__(kNW * 32, 1) decode_mma_kernel(DecodeArgs a, L
         }
         table[i] = *reinterpret_cast<uint32_t*>(&v);
     }
+}
+
+// ---- one warp's attention state over packed tiles -------------------------------------
+
+// NH = 8: the 8 columns of every MMA are 8 query heads, and the fp16 hi and lo
+// halves of the fp32 operand (Q' or P') are two MMAs into the same
+// accumulator; a lane holds heads 2c and 2c + 1. NH = 4: columns 2h and 2h + 1
+// are the hi and lo halves of head h (4 heads), summed after the MMA; a lane
+// holds head c. Lane (r, c) = (lane / 4, lane % 4).
+template <class KF, class VF, int NH>
+struct WarpTiles {
+    static constexpr int HL = NH / 4;  // heads per lane
+    uint32_t bq[8][2 * HL];            // query B fragments per k-step
+    float o[8][4];                     // value accumulators: row tile q, rows r / r + 8, columns 2c / 2c + 1
+    float m_ref[HL], l_run[HL];
+
+    // Rotated, scaled queries of the item's query heads (rows of them), fp32
+    // [head][128] in the packed coordinate order.
+    __device__ __forceinline__ void begin(const float* qr, int rows, int r, int c) {
+        const int head = NH == 8 ? r : (r >> 1);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            // k-step s: B rows (2c, 2c+1) and (2c+8, 2c+9) are coordinates p..p+3 of lane c's chunk
+            const int p = s < KF::KS0 ? c * (KF::N0 / 4) + 4 * s : KF::N0 + c * (KF::N1 / 4) + 4 * (s - KF::KS0);
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (head < rows) x = __ldcg(reinterpret_cast<const float4*>(qr + head * kHeadDim + p));
+            uint32_t h01, l01, h23, l23;
+            split2(x.x, x.y, h01, l01);
+            split2(x.z, x.w, h23, l23);
+            if constexpr (NH == 8) {
+                bq[s][0] = h01;
+                bq[s][1] = h23;
+                bq[s][2] = l01;
+                bq[s][3] = l23;
+            } else {
+                bq[s][0] = (r & 1) ? l01 : h01;
+                bq[s][1] = (r & 1) ? l23 : h23;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) o[q][0] = o[q][1] = o[q][2] = o[q][3] = 0.0f;
+#pragma unroll
+        for (int e = 0; e < HL; ++e) {
+            m_ref[e] = -INFINITY;
+            l_run[e] = 0.0f;
+        }
+    }
+
+    // One 16-token tile: K index rows at kbase (norms at knorm), V index rows at
+    // vbase (norms at vnorm); tokens at or past nvalid are padding.
+    __device__ __forceinline__ void step(uint32_t kbase, uint32_t knorm, uint32_t vbase, uint32_t vnorm, int nvalid,
+                                         uint32_t lane_base, uint32_t psel, int lane, int r, int c) {
+        // ---- S^T = K^ Q'^T: rows tokens r, r + 8 ----
+        // Independent accumulator chains (k-step parity; hi / lo for NH = 8)
+        // keep the MMA dependency depth at 4.
+        constexpr int NC = NH == 8 ? 4 : 2;
+        float sacc[NC][4];
+#pragma unroll
+        for (int u = 0; u < NC; ++u) sacc[u][0] = sacc[u][1] = sacc[u][2] = sacc[u][3] = 0.0f;
+        auto score_step = [&](auto si, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+            constexpr int s_ = decltype(si)::value;
+            if constexpr (NH == 8) {
+                mma16816(sacc[s_ & 1], a0, a1, a2, a3, bq[s_][0], bq[s_][1]);
+                mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, bq[s_][2], bq[s_][3]);
+            } else {
+                mma16816(sacc[s_ & 1], a0, a1, a2, a3, bq[s_][0], bq[s_][1]);
+            }
+        };
+        {
+            constexpr int KW0 = (KF::KC0 + 3) / 4;
+            constexpr bool A0 = KF::KC0 % 4 == 0;
+            const Words<KW0> k0a = lds_span<KF::KC0, A0>(kbase + r * KF::IB + c * KF::KC0);
+            const Words<KW0> k0b = lds_span<KF::KC0, A0>(kbase + (r + 8) * KF::IB + c * KF::KC0);
+            const uint32_t base0 = lut_base<KF::B0>(lane_base);
+            static_for<0, KF::KS0>([&](auto si) {
+                constexpr int s_ = decltype(si)::value;
+                const uint32_t a0 = lut(pair_addr<KF::B0, 4 * s_ * KF::B0, KW0>(k0a.w, base0));
+                const uint32_t a1 = lut(pair_addr<KF::B0, 4 * s_ * KF::B0, KW0>(k0b.w, base0));
+                const uint32_t a2 = lut(pair_addr<KF::B0, (4 * s_ + 2) * KF::B0, KW0>(k0a.w, base0));
+                const uint32_t a3 = lut(pair_addr<KF::B0, (4 * s_ + 2) * KF::B0, KW0>(k0b.w, base0));
+                score_step(si, a0, a1, a2, a3);
+            });
+            if constexpr (KF::N1 > 0) {
+                constexpr int KW1 = (KF::KC1 + 3) / 4;
+                constexpr bool A1 = (KF::KC1 % 4 == 0) && (KF::BOFF1 % 4 == 0);
+                const uint32_t g1 = KF::BOFF1 + c * KF::KC1;
+                const Words<KW1> k1a = lds_span<KF::KC1, A1>(kbase + r * KF::IB + g1);
+                const Words<KW1> k1b = lds_span<KF::KC1, A1>(kbase + (r + 8) * KF::IB + g1);
+                const uint32_t base1 = lut_base<KF::B1>(lane_base);
+                static_for<0, KF::KS1>([&](auto si) {
+                    constexpr int s_ = decltype(si)::value;
+                    const uint32_t a0 = lut(pair_addr<KF::B1, 4 * s_ * KF::B1, KW1>(k1a.w, base1));
+                    const uint32_t a1 = lut(pair_addr<KF::B1, 4 * s_ * KF::B1, KW1>(k1b.w, base1));
+                    const uint32_t a2 = lut(pair_addr<KF::B1, (4 * s_ + 2) * KF::B1, KW1>(k1a.w, base1));
+                    const uint32_t a3 = lut(pair_addr<KF::B1, (4 * s_ + 2) * KF::B1, KW1>(k1b.w, base1));
+                    score_step(std::integral_constant<int, KF::KS0 + s_>{}, a0, a1, a2, a3);
+                });
+            }
+        }
+
+        // ---- online softmax over the lane's heads, tokens r and r + 8 ----
+        const float nk0 = f16_at(knorm + 2 * r), nk1 = f16_at(knorm + 2 * (r + 8));
+        const float nv0 = f16_at(vnorm + 2 * r), nv1 = f16_at(vnorm + 2 * (r + 8));
+        const bool ok0 = r < nvalid, ok1 = r + 8 < nvalid;
+        float sc[HL][2];  // head e of the lane, token r (0) or r + 8 (1)
+        if constexpr (NH == 8) {
+            float x0, x1, y0, y1;
+            upk(add2(add2(pk(sacc[0][0], sacc[0][1]), pk(sacc[1][0], sacc[1][1])),
+                     add2(pk(sacc[2][0], sacc[2][1]), pk(sacc[3][0], sacc[3][1]))),
+                x0, x1);
+            upk(add2(add2(pk(sacc[0][2], sacc[0][3]), pk(sacc[1][2], sacc[1][3])),
+                     add2(pk(sacc[2][2], sacc[2][3]), pk(sacc[3][2], sacc[3][3]))),
+                y0, y1);
+            upk(mul2(pk(x0, x1), pk(nk0, nk0)), x0, x1);
+            upk(mul2(pk(y0, y1), pk(nk1, nk1)), y0, y1);
+            sc[0][0] = ok0 ? x0 : -INFINITY;
+            sc[HL - 1][0] = ok0 ? x1 : -INFINITY;
+            sc[0][1] = ok1 ? y0 : -INFINITY;
+            sc[HL - 1][1] = ok1 ? y1 : -INFINITY;
+        } else {
+            float h0, l0, h1, l1;
+            upk(add2(pk(sacc[0][0], sacc[0][1]), pk(sacc[1][0], sacc[1][1])), h0, l0);
+            upk(add2(pk(sacc[0][2], sacc[0][3]), pk(sacc[1][2], sacc[1][3])), h1, l1);
+            sc[0][0] = ok0 ? (h0 + l0) * nk0 : -INFINITY;
+            sc[0][1] = ok1 ? (h1 + l1) * nk1 : -INFINITY;
+        }
+        // The reference max only moves when a score exceeds it by more than
+        // 2^kSlack; the shuffles and rescale run only then.
+        bool over = false;
+#pragma unroll
+        for (int e = 0; e < HL; ++e) over |= fmaxf(sc[e][0], sc[e][1]) > m_ref[e] + kSlack;
+        // The trip count is opaque to the compiler (0 or 1 at run time), so the
+        // rescale stays a branch instead of predicated straight-line code.
+        int rare = __any_sync(kFull, over) ? 1 : 0;
+        asm volatile("mov.b32 %0, %0;" : "+r"(rare));
+#pragma unroll 1
+        for (int t = 0; t < rare; ++t) {
+            float alpha[HL];
+#pragma unroll
+            for (int e = 0; e < HL; ++e) {
+                float mx = fmaxf(sc[e][0], sc[e][1]);
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+                const bool grow = mx > m_ref[e] + kSlack;
+                alpha[e] = grow ? ex2(m_ref[e] - mx) : 1.0f;
+                l_run[e] *= alpha[e];
+                if (grow) m_ref[e] = mx;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                o[q][0] *= alpha[0];
+                o[q][1] *= alpha[HL - 1];
+                o[q][2] *= alpha[0];
+                o[q][3] *= alpha[HL - 1];
+            }
+        }
+        // P' = p * n_V * 2^-kSlack (weight x norm stays within fp16).
+        float w[HL][2];
+#pragma unroll
+        for (int e = 0; e < HL; ++e) {
+            const float mref = m_ref[e] == -INFINITY ? 0.0f : m_ref[e];
+            const float p0 = ex2(sc[e][0] - mref), p1 = ex2(sc[e][1] - mref);
+            l_run[e] += p0 + p1;
+            w[e][0] = ok0 ? p0 * (nv0 * kSlackInv) : 0.0f;
+            w[e][1] = ok1 ? p1 * (nv1 * kSlackInv) : 0.0f;
+        }
+        // B fragments of P'^T: rows tokens (2c, 2c+1) and (2c+8, 2c+9), column r.
+        // Tokens 2c and 2c + 8 sit in lane 8c + (r >> 1), tokens 2c + 1 and
+        // 2c + 9 four lanes on.
+        const int srcA = 8 * c + (r >> 1), srcB = srcA + 4;
+        uint32_t bp[2 * HL];
+        if constexpr (NH == 8) {
+            // Per token: (head 2c, head 2c + 1) as hi and lo half2.
+            uint32_t th0, tl0, th1, tl1;
+            split2(w[0][0], w[1][0], th0, tl0);
+            split2(w[0][1], w[1][1], th1, tl1);
+            const uint32_t xa = __shfl_sync(kFull, th0, srcA), xb = __shfl_sync(kFull, th0, srcB);
+            const uint32_t ya = __shfl_sync(kFull, th1, srcA), yb = __shfl_sync(kFull, th1, srcB);
+            const uint32_t xla = __shfl_sync(kFull, tl0, srcA), xlb = __shfl_sync(kFull, tl0, srcB);
+            const uint32_t yla = __shfl_sync(kFull, tl1, srcA), ylb = __shfl_sync(kFull, tl1, srcB);
+            bp[0] = prmt(xa, xb, psel);
+            bp[1] = prmt(ya, yb, psel);
+            bp[2] = prmt(xla, xlb, psel);
+            bp[3] = prmt(yla, ylb, psel);
+        } else {
+            // Per lane: (token r, token r + 8) as hi and lo half2.
+            uint32_t xh, xl;
+            split2(w[0][0], w[0][1], xh, xl);
+            const uint32_t xa = __shfl_sync(kFull, xh, srcA), ya = __shfl_sync(kFull, xl, srcA);
+            const uint32_t xb = __shfl_sync(kFull, xh, srcB), yb = __shfl_sync(kFull, xl, srcB);
+            const uint32_t pa = (r & 1) ? ya : xa, pb = (r & 1) ? yb : xb;
+            bp[0] = prmt(pa, pb, 0x5410u);
+            bp[1] = prmt(pa, pb, 0x7632u);
+        }
+        auto value_step = [&](auto qi, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+            constexpr int q = decltype(qi)::value;
+            mma16816(o[q], a0, a1, a2, a3, bp[0], bp[1]);
+            if constexpr (NH == 8) mma16816(o[q], a0, a1, a2, a3, bp[2], bp[3]);
+        };
+
+        // ---- O^T += V^T P'^T over 8 coordinate row tiles ----
+        const uint32_t r0 = vbase + (2 * c) * VF::IB, r1 = r0 + VF::IB;
+        const uint32_t r8 = vbase + (2 * c + 8) * VF::IB, r9 = r8 + VF::IB;
+        {
+            constexpr int NW0 = (VF::VC0 + 3) / 4;
+            constexpr bool A0 = VF::VC0 % 4 == 0;
+            const Words<NW0> t0 = lds_span<VF::VC0, A0>(r0 + r * VF::VC0);
+            const Words<NW0> t1 = lds_span<VF::VC0, A0>(r1 + r * VF::VC0);
+            const Words<NW0> t8 = lds_span<VF::VC0, A0>(r8 + r * VF::VC0);
+            const Words<NW0> t9 = lds_span<VF::VC0, A0>(r9 + r * VF::VC0);
+            uint32_t e01[NW0], o01[NW0], e89[NW0], o89[NW0];
+            interleave<VF::B0, NW0>(t0.w, t1.w, e01, o01);
+            interleave<VF::B0, NW0>(t8.w, t9.w, e89, o89);
+            const uint32_t base0 = lut_base<VF::B0>(lane_base);
+            static_for<0, VF::MT0>([&](auto qi) {
+                constexpr int q = decltype(qi)::value;
+                const uint32_t a0 = lut(vpair_addr<VF::B0, 2 * q, NW0>(e01, o01, base0));
+                const uint32_t a1 = lut(vpair_addr<VF::B0, 2 * q + 1, NW0>(e01, o01, base0));
+                const uint32_t a2 = lut(vpair_addr<VF::B0, 2 * q, NW0>(e89, o89, base0));
+                const uint32_t a3 = lut(vpair_addr<VF::B0, 2 * q + 1, NW0>(e89, o89, base0));
+                value_step(qi, a0, a1, a2, a3);
+            });
+        }
+        if constexpr (VF::N1 > 0) {
+            constexpr int NW1 = (VF::VC1 + 3) / 4;
+            constexpr bool A1 = (VF::VC1 % 4 == 0) && (VF::BOFF1 % 4 == 0);
+            const uint32_t g1 = VF::BOFF1 + r * VF::VC1;
+            const Words<NW1> t0 = lds_span<VF::VC1, A1>(r0 + g1);
+            const Words<NW1> t1 = lds_span<VF::VC1, A1>(r1 + g1);
+            const Words<NW1> t8 = lds_span<VF::VC1, A1>(r8 + g1);
+            const Words<NW1> t9 = lds_span<VF::VC1, A1>(r9 + g1);
+            uint32_t e01[NW1], o01[NW1], e89[NW1], o89[NW1];
+            interleave<VF::B1, NW1>(t0.w, t1.w, e01, o01);
+            interleave<VF::B1, NW1>(t8.w, t9.w, e89, o89);
+            const uint32_t base1 = lut_base<VF::B1>(lane_base);
+            static_for<0, VF::MT1>([&](auto qi) {
+                constexpr int q = decltype(qi)::value;
+                const uint32_t a0 = lut(vpair_addr<VF::B1, 2 * q, NW1>(e01, o01, base1));
+                const uint32_t a1 = lut(vpair_addr<VF::B1, 2 * q + 1, NW1>(e01, o01, base1));
+                const uint32_t a2 = lut(vpair_addr<VF::B1, 2 * q, NW1>(e89, o89, base1));
+                const uint32_t a3 = lut(vpair_addr<VF::B1, 2 * q + 1, NW1>(e89, o89, base1));
+                value_step(std::integral_constant<int, VF::MT0 + q>{}, a0, a1, a2, a3);
+            });
+        }
+    }
+
+    // Writes (max, sum, accumulator x 2^kSlack) of each of the lane's heads:
+    // m[head * ml_stride], l[head * ml_stride] and acc[head * acc_stride +
+    // packed coordinate]. Row r of value tile q is packed coordinate p0, row
+    // r + 8 is p0 + 1.
+    __device__ __forceinline__ void finish(float* m, float* l, float* acc, int ml_stride, int acc_stride, int rows,
+                                           int r, int c) {
+#pragma unroll
+        for (int e = 0; e < HL; ++e) {
+            float lsum = l_run[e];
+            lsum += __shfl_xor_sync(kFull, lsum, 4);
+            lsum += __shfl_xor_sync(kFull, lsum, 8);
+            lsum += __shfl_xor_sync(kFull, lsum, 16);
+            const int head = NH == 8 ? 2 * c + e : c;
+            if (head < rows) {
+                if (r == 0) {
+                    m[head * ml_stride] = m_ref[e];
+                    l[head * ml_stride] = lsum;
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const bool g1 = q >= VF::MT0;
+                    const int ql = g1 ? q - VF::MT0 : q;
+                    const int per = g1 ? VF::N1 / 8 : VF::N0 / 8;
+                    const int p0 = (g1 ? VF::N0 : 0) + r * per + 2 * ql;
+                    float2 val;
+                    if constexpr (NH == 8) {
+                        val = e == 0 ? make_float2(o[q][0], o[q][2]) : make_float2(o[q][1], o[q][3]);
+                    } else {
+                        val = make_float2(o[q][0] + o[q][1], o[q][2] + o[q][3]);
+                    }
+                    *reinterpret_cast<float2*>(acc + head * acc_stride + p0) =
+                        make_float2(val.x * 256.0f, val.y * 256.0f);
+                }
+            }
+        }
+    }
+};
+
+// Dense bf16 window of KV head h for the item's query heads: tokens
+// t_first, t_first + t_step, ... < it.t1, on CUDA cores (lane: 4 coordinates).
+// Writes (max, sum, accumulator) per query head g < rows: m[g * ml_stride],
+// l[g * ml_stride], acc[g * acc_stride + coordinate] (acc 8-byte aligned).
+__device__ __forceinline__ void window_state(const DecodeArgs& a, const Item& it, int h, int head0, int rows,
+                                             int t_first, int t_step, int lane, float* m_out, float* l_out,
+                                             float* acc_out, int ml_stride, int acc_stride) {
+    const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
+    const int H = a.kc.num_heads;
+    float qv[8][4], m[8], l[8], acc[8][4];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        m[g] = -INFINITY;
+        l[g] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[g][i] = 0.0f;
+            qv[g][i] = 0.0f;
+        }
+        if (g < rows) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(
+                qg + (static_cast<int64_t>(it.b) * a.num_q_heads + head0 + g) * kHeadDim + 4 * lane);
+            qv[g][0] = __uint_as_float(raw.x << 16) * a.scale_log2;
+            qv[g][1] = __uint_as_float(raw.x & 0xffff0000u) * a.scale_log2;
+            qv[g][2] = __uint_as_float(raw.y << 16) * a.scale_log2;
+            qv[g][3] = __uint_as_float(raw.y & 0xffff0000u) * a.scale_log2;
+        }
+    }
+    const __nv_bfloat16* kw = static_cast<const __nv_bfloat16*>(a.k_win);
+    const __nv_bfloat16* vw = static_cast<const __nv_bfloat16*>(a.v_win);
+    for (int tk = t_first; tk < it.t1; tk += t_step) {
+        const int64_t base = ((static_cast<int64_t>(it.b) * H + h) * a.window + tk) * kHeadDim + 4 * lane;
+        const uint2 kr = *reinterpret_cast<const uint2*>(kw + base);
+        const uint2 vr = *reinterpret_cast<const uint2*>(vw + base);
+        const float kx[4] = {__uint_as_float(kr.x << 16), __uint_as_float(kr.x & 0xffff0000u),
+                             __uint_as_float(kr.y << 16), __uint_as_float(kr.y & 0xffff0000u)};
+        const float vx[4] = {__uint_as_float(vr.x << 16), __uint_as_float(vr.x & 0xffff0000u),
+                             __uint_as_float(vr.y << 16), __uint_as_float(vr.y & 0xffff0000u)};
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            if (g < rows) {
+                float sc = qv[g][0] * kx[0] + qv[g][1] * kx[1] + qv[g][2] * kx[2] + qv[g][3] * kx[3];
+#pragma unroll
+                for (int mm = 16; mm; mm >>= 1) sc += __shfl_xor_sync(kFull, sc, mm);
+                const float mn = fmaxf(m[g], sc);
+                const float alpha = ex2(m[g] - mn);
+                const float p = ex2(sc - mn);
+                l[g] = l[g] * alpha + p;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[g][i] = acc[g][i] * alpha + p * vx[i];
+                m[g] = mn;
+            }
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        if (g < rows) {
+            if (lane == 0) {
+                m_out[g * ml_stride] = m[g];
+                l_out[g * ml_stride] = l[g];
+            }
+            float2* dst = reinterpret_cast<float2*>(acc_out + g * acc_stride + 4 * lane);
+            dst[0] = make_float2(acc[g][0], acc[g][1]);
+            dst[1] = make_float2(acc[g][2], acc[g][3]);
+        }
+    }
+}
+
+// Record of item (b, KV head h, split): [group][2 + 128] floats.
+__device__ __forceinline__ float* record_of(const DecodeArgs& a, int b, int h, int split, int group) {
+    return a.ws + ((static_cast<int64_t>(b) * a.kc.num_heads + h) * a.items_per_unit + split) *
+                      static_cast<int64_t>(group) * (kHeadDim + 2);
+}
+
+// ==== block kernel: one page block of 8 KV heads per ring slot ========================
+//
+// A work item is (query-head group, 8 consecutive KV heads, sequence, split).
+// A ring slot holds one page block of the 8 heads in both pools: [K: 8 x
+// (bs index rows, bs norms)][V: the same]. The sub-pages of consecutive heads
+// are adjacent in a pool, so a slot takes two bulk copies whatever the block
+// size. Compute warp w reads KV head w of every slot, 16 tokens at a time,
+// and writes its records itself: nothing is merged across warps.
+
+constexpr int kBlkWarps = 8;        // compute warps = KV heads per slot
+constexpr int kBlkMaxSlots = 16;
+constexpr int kBlkMinSlots = 4;     // fewer slots of a larger block: the per-head kernel instead
+
+struct BlkSmem {
+    unsigned long long full[kBlkMaxSlots];   // producer -> warps: slot filled (tx bytes)
+    unsigned long long empty[kBlkMaxSlots];  // warps -> producer: 8 releases free a slot
+    int ids[2][kMaxItemTiles];               // producer: block ids of the current and next item
+};
+
+// Ring placement around the 64 KB table: n_low slots between the header and
+// the table, the rest after it.
+struct BlkRing {
+    uint32_t low, high;
+    int n_low, n;
+    uint32_t stride;
+    __device__ __forceinline__ uint32_t slot(int s) const {
+        return s < n_low ? low + s * stride : high + (s - n_low) * stride;
+    }
+};
+
+// Bytes of a ring slot: one block of 8 heads in both pools.
+template <class KF, class VF>
+__host__ __device__ constexpr uint32_t blk_slot_bytes(int bs) {
+    return static_cast<uint32_t>(kBlkWarps * bs * (KF::IB + 2 + VF::IB + 2));
+}
+
+template <class KF, class VF>
+__device__ void produce_blk(const DecodeArgs& a, BlkSmem& sm, const BlkRing& ring, int head_groups,
+                            int64_t total_slots, int lane) {
+    constexpr int kPer = kMaxItemTiles / 32;
+    const int H = a.kc.num_heads, bs = a.block_size;
+    const uint32_t k_bytes = kBlkWarps * bs * (KF::IB + 2), v_bytes = kBlkWarps * bs * (VF::IB + 2);
+    auto read_ids = [&](const Item& it, int (&v)[kPer]) {
+        const int nblk = (it.t1 - it.t0 + bs - 1) / bs;
+        const int32_t* bt = a.block_tables + static_cast<int64_t>(it.b) * a.max_blocks + it.t0 / bs;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int i = lane + 32 * k;
+            v[k] = i < nblk ? __ldg(bt + i) : 0;
+        }
+    };
+    uint32_t fill = 0;
+    int buf = 0;
+    int64_t slot = blockIdx.x;
+    Item cur;
+    bool have = next_packed<kBlkWarps>(a, slot, head_groups, total_slots, cur);
+    if (have) {
+        int v[kPer];
+        read_ids(cur, v);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) sm.ids[0][lane + 32 * k] = v[k];
+    }
+    __syncwarp();
+    bool stop = false;
+    while (have && !stop) {
+        int64_t slot_n = slot + gridDim.x;
+        Item nxt;
+        const bool have_n = next_packed<kBlkWarps>(a, slot_n, head_groups, total_slots, nxt);
+        int v[kPer];
+        if (have_n) read_ids(nxt, v);
+        if (lane == 0) {
+            const int nblk = (cur.t1 - cur.t0 + bs - 1) / bs;
+#pragma unroll 1
+            for (int i = 0; i < nblk; ++i, ++fill) {
+                const int s = static_cast<int>(fill % ring.n);
+                const uint32_t use = fill / ring.n;
+                const uint32_t full = smem_addr(&sm.full[s]);
+                if (use > 0 && !mbar_sleep_wait(smem_addr(&sm.empty[s]), (use - 1) & 1u)) {
+                    // The compute warps stop on their own bounded waits.
+                    if (a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
+                    stop = true;
+                    break;
+                }
+                int blk = sm.ids[buf][i];
+                if (blk < 0 || blk >= a.num_blocks) {
+                    if (a.d_err) atomicOr(a.d_err, TQ_DERR_BLOCK);
+                    blk = 0;
+                }
+                const int64_t sp = (static_cast<int64_t>(blk) * H + cur.h) * bs;  // first of 8 sub-pages
+                const uint32_t dst = ring.slot(s);
+                mbar_expect(full, k_bytes + v_bytes);
+                bulk_copy(dst, a.k_pages + sp * (KF::IB + 2), k_bytes, full);
+                bulk_copy(dst + k_bytes, a.v_pages + sp * (VF::IB + 2), v_bytes, full);
+            }
+        }
+        stop = __shfl_sync(kFull, stop, 0);
+        buf ^= 1;
+        if (have_n && !stop) {
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) sm.ids[buf][lane + 32 * k] = v[k];
+        }
+        __syncwarp();
+        cur = nxt;
+        have = have_n;
+        slot = slot_n;
+    }
+    // Wait (bounded) for the copies in flight before the CTA can retire.
+    fill = __shfl_sync(kFull, fill, 0);
     if (lane == 0)
-        for (int s = 0; s < kStages; ++s)
-            mbar_init(static_cast<uint32_t>(__cvta_generic_to_shared(&sm.bar[warp][s])));
-    if (threadIdx.x == 0) sm.abort_flag = 0;
+        for (uint32_t f = fill > static_cast<uint32_t>(ring.n) ? fill - ring.n : 0; f < fill; ++f)
+            if (!mbar_wait(smem_addr(&sm.full[f % ring.n]), (f / ring.n) & 1u)) break;
+}
+
+// B16: the block size is 16 (one tile per slot; a simpler consumer loop that
+// measured markedly faster than the general one).
+template <class KF, class VF, int NH, bool B16>
+__global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(DecodeArgs a, LutValues tv, int group,
+                                                                             int head_groups, int64_t total_slots) {
+    static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
+    extern __shared__ __align__(128) uint8_t dsm[];
+    BlkSmem& sm = *reinterpret_cast<BlkSmem*>(dsm);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, c = lane & 3;
+    const int bs = a.block_size;
+
+    // Shared memory: [BlkSmem][slots][64 KB table at a 64 KB boundary][slots].
+    uint32_t dyn_bytes;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_bytes));
+    const uint32_t dsm_addr = smem_addr(dsm), dsm_end = dsm_addr + dyn_bytes;
+    BlkRing ring;
+    ring.stride = blk_slot_bytes<KF, VF>(bs);
+    ring.low = (dsm_addr + static_cast<uint32_t>(sizeof(BlkSmem)) + 127) & ~127u;
+    const uint32_t lut_addr = (ring.low + (kLut - 1)) & ~uint32_t(kLut - 1);
+    ring.n_low = static_cast<int>((lut_addr - ring.low) / ring.stride);
+    ring.high = lut_addr + kLut;
+    const int n_high = ring.high < dsm_end ? static_cast<int>((dsm_end - ring.high) / ring.stride) : 0;
+    ring.n = min(ring.n_low + n_high, kBlkMaxSlots);
+    if (lut_addr + kLut > dsm_end || ring.n < 2) {
+        if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
+        return;
+    }
+    fill_table(reinterpret_cast<uint32_t*>(dsm + (lut_addr - dsm_addr)), tv, threadIdx.x, (kBlkWarps + 1) * 32);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kBlkMaxSlots; ++s) {
+            mbar_init_count(smem_addr(&sm.full[s]), 1);
+            mbar_init_count(smem_addr(&sm.empty[s]), kBlkWarps);
+        }
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
+    if (warp == kBlkWarps) {
+        produce_blk<KF, VF>(a, sm, ring, head_groups, total_slots, lane);
+        return;
+    }
     uint32_t lane_base;
     asm volatile("or.b32 %0, %1, %2;" : "=r"(lane_base) : "r"(lut_addr), "r"(static_cast<uint32_t>(lane) << 2));
-
-    const int H = a.kc.num_heads, bs = a.block_size;
-    const uint8_t* const k_pages = a.k_pages;
-    const uint8_t* const v_pages = a.v_pages;
-    const bool bs_pow2 = (bs & (bs - 1)) == 0;
+    const uint32_t psel = (r & 1) ? 0x7632u : 0x5410u;
     const int rows = group < NH ? group : NH;
-    const uint32_t my_ring = ring_addr + static_cast<uint32_t>(warp * kStages * kStageBytes);
-    const uint32_t bar0 = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.bar[warp][0]));
-    constexpr uint32_t kKBytes = 16 * KF::IB, kVBytes = 16 * VF::IB;
-    constexpr uint32_t kTileBytes = kKBytes + kVBytes + 64;
+    // This warp's head within a slot: K sub-page at k_off, V sub-page at v_off.
+    const uint32_t k_sub = bs * (KF::IB + 2), v_sub = bs * (VF::IB + 2);
+    const uint32_t k_off = warp * k_sub, v_off = kBlkWarps * k_sub + warp * v_sub;
+    uint32_t consumed = 0;
+    WarpTiles<KF, VF, NH> wt;
 
-    // ---- producer (lane 0 issues; every lane tracks the cursor) ----
-    // The producer feeds this warp's tiles in consumption order, one tile per
-    // consumed tile after an initial fill of the ring. It keeps the block ids of
-    // its current item and, loaded one item earlier, of the next one.
-    struct Cursor {
-        int64_t slot;
-        Item it;
-        int n;    // this warp's tiles in the item (0: no item)
-        int ids;  // lane k: block id of the warp's k-th tile
-    };
-    auto find_from = [&](int64_t slot, Cursor& cur) {
-        cur.n = 0;
-        for (; slot < total_slots; slot += gridDim.x) {
-            if (!item_of(a, slot, head_groups, cur.it)) continue;
-            const int n = warp_tiles(cur.it, warp);
-            if (n > 0) {
-                cur.slot = slot;
-                cur.n = n;
-                cur.ids = load_block_ids(a, cur.it, warp, lane);
-                return;
-            }
-        }
-        cur.slot = total_slots;
-    };
-    Cursor pc, nc;
-    find_from(blockIdx.x, pc);
-    find_from(pc.n ? pc.slot + gridDim.x : total_slots, nc);
-    int p_k = 0;
-    uint32_t issued = 0, consumed = 0, phase_bits = 0;
-    bool timed_out = false;
-    const uint32_t k_row_bytes = KF::IB + 2, v_row_bytes = VF::IB + 2;
-
-    auto issue_one = [&]() {
-        if (pc.n == 0) return;
-        const int blk = __shfl_sync(kFull, pc.ids, p_k);
-        if (lane == 0) {
-            const int tok = pc.it.t0 + 16 * (warp + p_k * kNW);
-            const int64_t sp = (static_cast<int64_t>(blk) * H + pc.it.h) * bs;
-            const uint8_t* ks = k_pages + sp * k_row_bytes;
-            const uint8_t* vs = v_pages + sp * v_row_bytes;
-            const int off = bs_pow2 ? (tok & (bs - 1)) : tok % bs;
-            const uint32_t s = issued % kStages;
-            const uint32_t dst = my_ring + s * kStageBytes, bar = bar0 + 8 * s;
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_expect(bar, kTileBytes);
-            bulk_copy(dst, ks + off * KF::IB, kKBytes, bar);
-            bulk_copy(dst + kKBytes, vs + off * VF::IB, kVBytes, bar);
-            bulk_copy(dst + kKBytes + kVBytes, ks + bs * KF::IB + 2 * off, 32, bar);
-            bulk_copy(dst + kKBytes + kVBytes + 32, vs + bs * VF::IB + 2 * off, 32, bar);
-        }
-        ++issued;
-        if (++p_k == pc.n) {
-            pc = nc;
-            p_k = 0;
-            find_from(pc.n ? pc.slot + gridDim.x : total_slots, nc);
-        }
-    };
-    for (int i = 0; i < kStages; ++i) issue_one();
-
-    const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
     for (int64_t slot = blockIdx.x; slot < total_slots; slot += gridDim.x) {
         Item it;
-        if (!item_of(a, slot, head_groups, it)) continue;
-        const int head0 = it.h * group + it.hg * 8;  // first query head of the item
-
+        if (!item_of<kBlkWarps>(a, slot, head_groups, it)) continue;
+        const int h = it.h + warp;                    // this warp's KV head
+        const int head0 = h * group + it.hg * 8;      // its first query head of the item
+        float* rec = record_of(a, it.b, h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
         if (it.win) {
-            // Dense bf16 window on CUDA cores: tokens spread over the warps.
-            float qv[8][4], m[8], l[8], acc[8][4];
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-                m[g] = -INFINITY;
-                l[g] = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    acc[g][i] = 0.0f;
-                    qv[g][i] = 0.0f;
-                }
-                if (g < rows) {
-                    const uint2 raw = *reinterpret_cast<const uint2*>(
-                        qg + (static_cast<int64_t>(it.b) * a.num_q_heads + head0 + g) * kHeadDim + 4 * lane);
-                    qv[g][0] = __uint_as_float(raw.x << 16) * a.scale_log2;
-                    qv[g][1] = __uint_as_float(raw.x & 0xffff0000u) * a.scale_log2;
-                    qv[g][2] = __uint_as_float(raw.y << 16) * a.scale_log2;
-                    qv[g][3] = __uint_as_float(raw.y & 0xffff0000u) * a.scale_log2;
-                }
-            }
-            const __nv_bfloat16* kw = static_cast<const __nv_bfloat16*>(a.k_win);
-            const __nv_bfloat16* vw = static_cast<const __nv_bfloat16*>(a.v_win);
-            for (int tk = it.t0 + warp; tk < it.t1; tk += kNW) {
-                const int64_t base = ((static_cast<int64_t>(it.b) * H + it.h) * a.window + tk) * kHeadDim + 4 * lane;
-                const uint2 kr = *reinterpret_cast<const uint2*>(kw + base);
-                const uint2 vr = *reinterpret_cast<const uint2*>(vw + base);
-                const float kx[4] = {__uint_as_float(kr.x << 16), __uint_as_float(kr.x & 0xffff0000u),
-                                     __uint_as_float(kr.y << 16), __uint_as_float(kr.y & 0xffff0000u)};
-                const float vx[4] = {__uint_as_float(vr.x << 16), __uint_as_float(vr.x & 0xffff0000u),
-                                     __uint_as_float(vr.y << 16), __uint_as_float(vr.y & 0xffff0000u)};
-#pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    if (g < rows) {
-                        float s = qv[g][0] * kx[0] + qv[g][1] * kx[1] + qv[g][2] * kx[2] + qv[g][3] * kx[3];
-#pragma unroll
-                        for (int mm = 16; mm; mm >>= 1) s += __shfl_xor_sync(kFull, s, mm);
-                        const float mn = fmaxf(m[g], s);
-                        const float alpha = ex2(m[g] - mn);
-                        const float p = ex2(s - mn);
-                        l[g] = l[g] * alpha + p;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) acc[g][i] = acc[g][i] * alpha + p * vx[i];
-                        m[g] = mn;
-                    }
-                }
-            }
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-                if (g < rows) {
-                    if (lane == 0) {
-                        sm.red_m[warp][g] = m[g];
-                        sm.red_l[warp][g] = l[g];
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) sm.red_o[warp][g][4 * lane + i] = acc[g][i];
-                }
-            }
-        } else {
-            const int n_mine = warp_tiles(it, warp);
-            // Query-side B fragments: column r of n-tile j is head 4j + r/2, half r%2.
-            uint32_t bq[8][NJ][2];
-            {
-                const float* qr = a.qrot + (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim;
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const int p = s < KF::KS0 ? c * (KF::N0 / 4) + 4 * s
-                                              : KF::N0 + c * (KF::N1 / 4) + 4 * (s - KF::KS0);
-#pragma unroll
-                    for (int j = 0; j < NJ; ++j) {
-                        const int head = 4 * j + (r >> 1);
-                        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (head < rows) x = __ldcg(reinterpret_cast<const float4*>(qr + head * kHeadDim + p));
-                        const __half2 h01 = __floats2half2_rn(x.x, x.y), h23 = __floats2half2_rn(x.z, x.w);
-                        __half2 v01 = h01, v23 = h23;
-                        if (r & 1) {
-                            v01 = __floats2half2_rn(x.x - __low2float(h01), x.y - __high2float(h01));
-                            v23 = __floats2half2_rn(x.z - __low2float(h23), x.w - __high2float(h23));
-                        }
-                        bq[s][j][0] = *reinterpret_cast<const uint32_t*>(&v01);
-                        bq[s][j][1] = *reinterpret_cast<const uint32_t*>(&v23);
-                    }
-                }
-            }
-            float o[8][NJ][4];
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) o[q][j][0] = o[q][j][1] = o[q][j][2] = o[q][j][3] = 0.0f;
-            float m_run[NJ], l_run[NJ];
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-                m_run[j] = -INFINITY;
-                l_run[j] = 0.0f;
-            }
-            // The producer runs ahead into this item's tiles and then the next item's.
-            for (int k = 0; k < n_mine && !timed_out; ++k) {
-                const uint32_t s = consumed % kStages;
-                if (!mbar_wait(bar0 + 8 * s, (phase_bits >> s) & 1u)) {
+            window_state(a, it, h, head0, rows, it.t0, 1, lane, rec, rec + 1, rec + 2, kHeadDim + 2, kHeadDim + 2);
+            continue;
+        }
+        wt.begin(a.qrot + (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim, rows, r, c);
+        bool timed_out = false;
+        const int ntiles = (it.t1 - it.t0 + 15) >> 4;
+        if constexpr (B16) {
+            for (int k = 0; k < ntiles; ++k, ++consumed) {
+                const int s = static_cast<int>(consumed % ring.n);
+                if (!mbar_wait(smem_addr(&sm.full[s]), (consumed / ring.n) & 1u)) {
                     timed_out = true;
                     break;
                 }
-                phase_bits ^= 1u << s;
-                const uint32_t slot_a = my_ring + s * kStageBytes;
-                const uint32_t kbase = slot_a, vbase = slot_a + kKBytes, nbase = slot_a + kKBytes + kVBytes;
-                const int nvalid = min(16, it.t1 - (it.t0 + 16 * (warp + k * kNW)));
-
-                // ---- S^T = K^ Q'^T: rows tokens r, r + 8 ----
-                // Two accumulator chains (even / odd k-steps) halve the MMA dependency depth.
-                float sacc[2][NJ][4];
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int j = 0; j < NJ; ++j) sacc[u][j][0] = sacc[u][j][1] = sacc[u][j][2] = sacc[u][j][3] = 0.0f;
-                {
-                    constexpr int KW0 = (KF::KC0 + 3) / 4;
-                    constexpr bool A0 = KF::KC0 % 4 == 0;
-                    const Words<KW0> k0a = lds_span<KF::KC0, A0>(kbase + r * KF::IB + c * KF::KC0);
-                    const Words<KW0> k0b = lds_span<KF::KC0, A0>(kbase + (r + 8) * KF::IB + c * KF::KC0);
-                    const uint32_t base0 = lut_base<KF::B0>(lane_base);
-                    static_for<0, KF::KS0>([&](auto si) {
-                        constexpr int s_ = decltype(si)::value;
-                        const uint32_t a0 = lut(pair_addr<KF::B0, 4 * s_ * KF::B0, KW0>(k0a.w, base0));
-                        const uint32_t a1 = lut(pair_addr<KF::B0, 4 * s_ * KF::B0, KW0>(k0b.w, base0));
-                        const uint32_t a2 = lut(pair_addr<KF::B0, (4 * s_ + 2) * KF::B0, KW0>(k0a.w, base0));
-                        const uint32_t a3 = lut(pair_addr<KF::B0, (4 * s_ + 2) * KF::B0, KW0>(k0b.w, base0));
-#pragma unroll
-                        for (int j = 0; j < NJ; ++j)
-                            mma16816(sacc[s_ & 1][j], a0, a1, a2, a3, bq[s_][j][0], bq[s_][j][1]);
-                    });
-                    if constexpr (KF::N1 > 0) {
-                        constexpr int KW1 = (KF::KC1 + 3) / 4;
-                        constexpr bool A1 = (KF::KC1 % 4 == 0) && (KF::BOFF1 % 4 == 0);
-                        const uint32_t g1 = KF::BOFF1 + c * KF::KC1;
-                        const Words<KW1> k1a = lds_span<KF::KC1, A1>(kbase + r * KF::IB + g1);
-                        const Words<KW1> k1b = lds_span<KF::KC1, A1>(kbase + (r + 8) * KF::IB + g1);
-                        const uint32_t base1 = lut_base<KF::B1>(lane_base);
-                        static_for<0, KF::KS1>([&](auto si) {
-                            constexpr int s_ = decltype(si)::value;
-                            const uint32_t a0 = lut(pair_addr<KF::B1, 4 * s_ * KF::B1, KW1>(k1a.w, base1));
-                            const uint32_t a1 = lut(pair_addr<KF::B1, 4 * s_ * KF::B1, KW1>(k1b.w, base1));
-                            const uint32_t a2 = lut(pair_addr<KF::B1, (4 * s_ + 2) * KF::B1, KW1>(k1a.w, base1));
-                            const uint32_t a3 = lut(pair_addr<KF::B1, (4 * s_ + 2) * KF::B1, KW1>(k1b.w, base1));
-#pragma unroll
-                            for (int j = 0; j < NJ; ++j)
-                                mma16816(sacc[(KF::KS0 + s_) & 1][j], a0, a1, a2, a3, bq[KF::KS0 + s_][j][0],
-                                         bq[KF::KS0 + s_][j][1]);
-                        });
-                    }
-                }
-
-                // ---- online softmax: head 4j + c, tokens r and r + 8 ----
-                const float nk0 = __half2float(__ushort_as_half(static_cast<unsigned short>(lds16(nbase + 2 * r))));
-                const float nk1 =
-                    __half2float(__ushort_as_half(static_cast<unsigned short>(lds16(nbase + 2 * (r + 8)))));
-                const float nv0 =
-                    __half2float(__ushort_as_half(static_cast<unsigned short>(lds16(nbase + 32 + 2 * r))));
-                const float nv1 =
-                    __half2float(__ushort_as_half(static_cast<unsigned short>(lds16(nbase + 32 + 2 * (r + 8)))));
-                const bool ok0 = r < nvalid, ok1 = r + 8 < nvalid;
-                const float nv0s = nv0 * kSlackInv, nv1s = nv1 * kSlackInv;
-                uint32_t bp[NJ][2];
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    const float s0 =
-                        ok0 ? ((sacc[0][j][0] + sacc[1][j][0]) + (sacc[0][j][1] + sacc[1][j][1])) * nk0 : -INFINITY;
-                    const float s1 =
-                        ok1 ? ((sacc[0][j][2] + sacc[1][j][2]) + (sacc[0][j][3] + sacc[1][j][3])) * nk1 : -INFINITY;
-                    float mx = fmaxf(s0, s1);
-                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-                    // The reference max only moves when a score exceeds it by more
-                    // than 2^kSlack, so weights stay below 2^kSlack and the
-                    // accumulators are rescaled rarely.
-                    const bool grow = mx > m_run[j] + kSlack;
-                    // A loop with a data-dependent trip count keeps this rare path a branch.
-                    const int rescale = __any_sync(kFull, grow) ? 1 : 0;
-#pragma unroll 1
-                    for (int t = 0; t < rescale; ++t) {
-                        const float m_new = grow ? mx : m_run[j];
-                        const float alpha = grow ? ex2(m_run[j] - m_new) : 1.0f;
-                        l_run[j] *= alpha;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            o[q][j][0] *= alpha;
-                            o[q][j][1] *= alpha;
-                            o[q][j][2] *= alpha;
-                            o[q][j][3] *= alpha;
-                        }
-                        m_run[j] = m_new;
-                    }
-                    const float mref = m_run[j] == -INFINITY ? 0.0f : m_run[j];
-                    const float p0 = ex2(s0 - mref), p1 = ex2(s1 - mref);
-                    l_run[j] += p0 + p1;
-                    // P' carries 2^-kSlack so that weight x norm stays within fp16.
-                    const float w0 = ok0 ? p0 * nv0s : 0.0f, w1 = ok1 ? p1 * nv1s : 0.0f;
-                    const __half2 X = __floats2half2_rn(w0, w1);
-                    const __half2 Y = __floats2half2_rn(w0 - __low2float(X), w1 - __high2float(X));
-                    const uint32_t xu = *reinterpret_cast<const uint32_t*>(&X);
-                    const uint32_t yu = *reinterpret_cast<const uint32_t*>(&Y);
-                    // B fragment of P'^T: tokens (2c, 2c+1) and (2c+8, 2c+9), column r.
-                    const int srcA = 8 * c + (r >> 1), srcB = srcA + 4;
-                    const uint32_t xa = __shfl_sync(kFull, xu, srcA), ya = __shfl_sync(kFull, yu, srcA);
-                    const uint32_t xb = __shfl_sync(kFull, xu, srcB), yb = __shfl_sync(kFull, yu, srcB);
-                    const uint32_t pa = (r & 1) ? ya : xa, pb = (r & 1) ? yb : xb;
-                    bp[j][0] = prmt(pa, pb, 0x5410u);
-                    bp[j][1] = prmt(pa, pb, 0x7632u);
-                }
-
-                // ---- O^T += V^T P'^T over 8 coordinate row tiles ----
-                {
-                    const uint32_t r0 = vbase + (2 * c) * VF::IB, r1 = r0 + VF::IB;
-                    const uint32_t r8 = vbase + (2 * c + 8) * VF::IB, r9 = r8 + VF::IB;
-                    {
-                        constexpr int NW0 = (VF::VC0 + 3) / 4;
-                        constexpr bool A0 = VF::VC0 % 4 == 0;
-                        const Words<NW0> t0 = lds_span<VF::VC0, A0>(r0 + r * VF::VC0);
-                        const Words<NW0> t1 = lds_span<VF::VC0, A0>(r1 + r * VF::VC0);
-                        const Words<NW0> t8 = lds_span<VF::VC0, A0>(r8 + r * VF::VC0);
-                        const Words<NW0> t9 = lds_span<VF::VC0, A0>(r9 + r * VF::VC0);
-                        uint32_t e01[NW0], o01[NW0], e89[NW0], o89[NW0];
-                        interleave<VF::B0, NW0>(t0.w, t1.w, e01, o01);
-                        interleave<VF::B0, NW0>(t8.w, t9.w, e89, o89);
-                        const uint32_t base0 = lut_base<VF::B0>(lane_base);
-                        static_for<0, VF::MT0>([&](auto qi) {
-                            constexpr int q = decltype(qi)::value;
-                            const uint32_t a0 = lut(vpair_addr<VF::B0, 2 * q, NW0>(e01, o01, base0));
-                            const uint32_t a1 = lut(vpair_addr<VF::B0, 2 * q + 1, NW0>(e01, o01, base0));
-                            const uint32_t a2 = lut(vpair_addr<VF::B0, 2 * q, NW0>(e89, o89, base0));
-                            const uint32_t a3 = lut(vpair_addr<VF::B0, 2 * q + 1, NW0>(e89, o89, base0));
-#pragma unroll
-                            for (int j = 0; j < NJ; ++j) mma16816(o[q][j], a0, a1, a2, a3, bp[j][0], bp[j][1]);
-                        });
-                    }
-                    if constexpr (VF::N1 > 0) {
-                        constexpr int NW1 = (VF::VC1 + 3) / 4;
-                        constexpr bool A1 = (VF::VC1 % 4 == 0) && (VF::BOFF1 % 4 == 0);
-                        const uint32_t g1 = VF::BOFF1 + r * VF::VC1;
-                        const Words<NW1> t0 = lds_span<VF::VC1, A1>(r0 + g1);
-                        const Words<NW1> t1 = lds_span<VF::VC1, A1>(r1 + g1);
-                        const Words<NW1> t8 = lds_span<VF::VC1, A1>(r8 + g1);
-                        const Words<NW1> t9 = lds_span<VF::VC1, A1>(r9 + g1);
-                        uint32_t e01[NW1], o01[NW1], e89[NW1], o89[NW1];
-                        interleave<VF::B1, NW1>(t0.w, t1.w, e01, o01);
-                        interleave<VF::B1, NW1>(t8.w, t9.w, e89, o89);
-                        const uint32_t base1 = lut_base<VF::B1>(lane_base);
-                        static_for<0, VF::MT1>([&](auto qi) {
-                            constexpr int q = decltype(qi)::value;
-                            const uint32_t a0 = lut(vpair_addr<VF::B1, 2 * q, NW1>(e01, o01, base1));
-                            const uint32_t a1 = lut(vpair_addr<VF::B1, 2 * q + 1, NW1>(e01, o01, base1));
-                            const uint32_t a2 = lut(vpair_addr<VF::B1, 2 * q, NW1>(e89, o89, base1));
-                            const uint32_t a3 = lut(vpair_addr<VF::B1, 2 * q + 1, NW1>(e89, o89, base1));
-#pragma unroll
-                            for (int j = 0; j < NJ; ++j)
-                                mma16816(o[VF::MT0 + q][j], a0, a1, a2, a3, bp[j][0], bp[j][1]);
-                        });
-                    }
-                }
+                const uint32_t kb = ring.slot(s) + k_off, vb = ring.slot(s) + v_off;
+                wt.step(kb, kb + 16 * KF::IB, vb, vb + 16 * VF::IB, min(16, it.t1 - (it.t0 + 16 * k)), lane_base,
+                        psel, lane, r, c);
                 __syncwarp();
-                ++consumed;
-                issue_one();  // refill the slot just freed
+                if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with the slot
             }
-            // Publish this warp's state (head 4j + c; positions of rows r and r + 8).
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-                float lsum = l_run[j];
-                lsum += __shfl_xor_sync(kFull, lsum, 4);
-                lsum += __shfl_xor_sync(kFull, lsum, 8);
-                lsum += __shfl_xor_sync(kFull, lsum, 16);
-                const int head = 4 * j + c;
-                if (head < rows) {
-                    if (r == 0) {
-                        sm.red_m[warp][head] = m_run[j];
-                        sm.red_l[warp][head] = lsum;
+        } else {
+            // 16-token tiles; a slot (one block) holds bs / 16 of them.
+            const int tpb = bs >> 4;
+            uint32_t kb = 0, vb = 0;
+            for (int k = 0, j = 0; k < ntiles; ++k) {
+                const int s = static_cast<int>(consumed % ring.n);
+                if (j == 0) {
+                    if (!mbar_wait(smem_addr(&sm.full[s]), (consumed / ring.n) & 1u)) {
+                        timed_out = true;
+                        break;
                     }
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const bool g1 = q >= VF::MT0;
-                        const int ql = g1 ? q - VF::MT0 : q;
-                        const int per = g1 ? VF::N1 / 8 : VF::N0 / 8;
-                        const int p0 = (g1 ? VF::N0 : 0) + r * per + 2 * ql;
-                        *reinterpret_cast<float2*>(&sm.red_o[warp][head][p0]) =
-                            make_float2((o[q][j][0] + o[q][j][1]) * 256.0f, (o[q][j][2] + o[q][j][3]) * 256.0f);
-                    }
+                    kb = ring.slot(s) + k_off;
+                    vb = ring.slot(s) + v_off;
+                }
+                wt.step(kb + 16 * j * KF::IB, kb + bs * KF::IB + 32 * j, vb + 16 * j * VF::IB,
+                        vb + bs * VF::IB + 32 * j, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, psel, lane, r, c);
+                if (++j == tpb || k + 1 == ntiles) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with the slot
+                    ++consumed;
+                    j = 0;
                 }
             }
+        }
+        if (timed_out) {
+            if (lane == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
+            break;
+        }
+        wt.finish(rec, rec + 1, rec + 2, kHeadDim + 2, kHeadDim + 2, rows, r, c);
+    }
+}
+
+// ==== per-head kernel: one KV head per work item, tiles spread over the warps =========
+//
+// For KV head counts that are not a multiple of 8. A work item is (query-head
+// group, KV head, sequence, split); tile t of an item goes to compute warp t %
+// NW, which keeps its own ring of slots; the warps merge their states through
+// shared memory at the end of the item.
+
+template <int NW>
+struct Smem {
+    float red_o[NW][8][kHeadDim];         // per-warp value accumulators (V packed order)
+    float red_m[NW][8], red_l[NW][8];
+    unsigned long long full[NW][kStages];   // producer -> warp: slot filled (tx bytes)
+    unsigned long long empty[NW][kStages];  // warp -> producer: slot free again
+    int ids[2][kMaxItemTiles];              // producer: block ids of the current and next item
+    int abort_flag;
+};
+
+// Dynamic shared memory: [Smem][pad to a 64 KB boundary][table][rings]. The
+// size assumes the Smem block plus the window offset of the dynamic area stays
+// within the first 64 KB; the kernel checks the layout before using it.
+template <int NW>
+__host__ __device__ constexpr size_t smem_head_bytes() {
+    return (sizeof(Smem<NW>) + 127) / 128 * 128;
+}
+template <int NW, uint32_t SB>
+__host__ __device__ constexpr size_t smem_bytes() {
+    return 2 * static_cast<size_t>(kLut) + static_cast<size_t>(NW) * kStages * SB;
+}
+
+// Producer warp. Lane w (w < NW) feeds compute warp w: in each packed work
+// item (in the compute warps' order) warp w consumes tiles w, w + NW, ...; for
+// each, the lane waits for the ring slot's release and copies the tile in. A
+// slot is [K rows][K norms][V rows][V norms]; with 16-token blocks each half is
+// one whole sub-page (rows then norms) and takes one bulk copy. While the
+// lanes stream an item, all 32 lanes read the next item's block ids into a
+// shared-memory buffer, so table reads never sit between consecutive copies.
+template <class KF, class VF, int NW>
+__device__ void produce_head(const DecodeArgs& a, Smem<NW>& sm, uint32_t ring_addr, int head_groups,
+                             int64_t total_slots, int lane) {
+    constexpr uint32_t kKRows = 16 * KF::IB, kVRows = 16 * VF::IB;
+    constexpr uint32_t kKTile = kKRows + 32, kTileBytes = kKTile + kVRows + 32;
+    constexpr uint32_t kStageBytes = stage_bytes<KF, VF>();
+    constexpr int kPer = kMaxItemTiles / 32;
+    const int H = a.kc.num_heads, bs = a.block_size;
+    const bool bs_pow2 = (bs & (bs - 1)) == 0, whole = bs == 16;
+    const uint32_t my_ring = ring_addr + static_cast<uint32_t>(lane * kStages * kStageBytes);
+    auto read_ids = [&](const Item& it, int (&v)[kPer]) {
+        const int ntiles = (it.t1 - it.t0 + 15) >> 4;
+        const int32_t* bt = a.block_tables + static_cast<int64_t>(it.b) * a.max_blocks;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int tl = lane + 32 * k;
+            v[k] = tl < ntiles ? __ldg(bt + (it.t0 + 16 * tl) / bs) : 0;
+        }
+    };
+    uint32_t fill = 0;
+    int buf = 0;
+    int64_t slot = blockIdx.x;
+    Item cur;
+    bool have = next_packed<1>(a, slot, head_groups, total_slots, cur);
+    if (have) {
+        int v[kPer];
+        read_ids(cur, v);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) sm.ids[0][lane + 32 * k] = v[k];
+    }
+    __syncwarp();
+    bool stop = false;
+    while (have) {
+        int64_t slot_n = slot + gridDim.x;
+        Item nxt;
+        const bool have_n = next_packed<1>(a, slot_n, head_groups, total_slots, nxt);
+        int v[kPer];
+        if (have_n) read_ids(nxt, v);
+        const int ntiles = (cur.t1 - cur.t0 + 15) >> 4;
+        if (lane < NW) {
+            const uint32_t full0 = smem_addr(&sm.full[lane][0]), empty0 = smem_addr(&sm.empty[lane][0]);
+#pragma unroll 1
+            for (int tl = lane; tl < ntiles; tl += NW) {
+                const uint32_t st = fill % kStages, use = fill / kStages;
+                const uint32_t full = full0 + 8 * st;
+                if (use > 0) {
+                    bool ready = false;
+                    for (uint32_t i = 0; i < kSpinLimit && !ready; ++i) ready = mbar_test(empty0 + 8 * st, (use - 1) & 1u);
+                    if (!ready) {
+                        // The compute warps stop on their own bounded waits.
+                        if (a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
+                        stop = true;
+                        break;
+                    }
+                }
+                int blk = sm.ids[buf][tl];
+                if (blk < 0 || blk >= a.num_blocks) {
+                    if (a.d_err) atomicOr(a.d_err, TQ_DERR_BLOCK);
+                    blk = 0;
+                }
+                const int tok = cur.t0 + 16 * tl;
+                const int off = bs_pow2 ? (tok & (bs - 1)) : tok % bs;
+                const int64_t sp = (static_cast<int64_t>(blk) * H + cur.h) * bs;
+                const uint8_t* ks = a.k_pages + sp * (KF::IB + 2);
+                const uint8_t* vs = a.v_pages + sp * (VF::IB + 2);
+                const uint32_t dst = my_ring + st * kStageBytes;
+                mbar_expect(full, kTileBytes);
+                if (whole) {
+                    bulk_copy(dst, ks, kKTile, full);
+                    bulk_copy(dst + kKTile, vs, kVRows + 32, full);
+                } else {
+                    bulk_copy(dst, ks + off * KF::IB, kKRows, full);
+                    bulk_copy(dst + kKRows, ks + bs * KF::IB + 2 * off, 32, full);
+                    bulk_copy(dst + kKTile, vs + off * VF::IB, kVRows, full);
+                    bulk_copy(dst + kKTile + kVRows, vs + bs * VF::IB + 2 * off, 32, full);
+                }
+                ++fill;
+            }
+        }
+        if (__any_sync(kFull, stop)) break;
+        buf ^= 1;
+        if (have_n) {
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) sm.ids[buf][lane + 32 * k] = v[k];
+        }
+        __syncwarp();
+        cur = nxt;
+        have = have_n;
+        slot = slot_n;
+    }
+    // Wait (bounded) for this lane's copies in flight before the CTA can retire.
+    if (lane < NW)
+        for (uint32_t f = fill > kStages ? fill - kStages : 0; f < fill; ++f)
+            if (!mbar_wait(smem_addr(&sm.full[lane][f % kStages]), (f / kStages) & 1u)) break;
+}
+
+template <class KF, class VF, int NH, int NW>
+__global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs a, LutValues tv, int group,
+                                                                      int head_groups, int64_t total_slots) {
+    static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
+    extern __shared__ __align__(128) uint8_t dsm[];
+    Smem<NW>& sm = *reinterpret_cast<Smem<NW>*>(dsm);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, c = lane & 3;
+    constexpr uint32_t kStageBytes = stage_bytes<KF, VF>();
+
+    const uint32_t dsm_addr = smem_addr(dsm);
+    const uint32_t lut_addr =
+        (dsm_addr + static_cast<uint32_t>(smem_head_bytes<NW>()) + (kLut - 1)) & ~uint32_t(kLut - 1);
+    const uint32_t ring_addr = lut_addr + kLut;
+    if (ring_addr + NW * kStages * kStageBytes > dsm_addr + smem_bytes<NW, kStageBytes>()) {
+        if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
+        return;
+    }
+    fill_table(reinterpret_cast<uint32_t*>(dsm + (lut_addr - dsm_addr)), tv, threadIdx.x, (NW + 1) * 32);
+    if (threadIdx.x == 0) {
+        for (int w = 0; w < NW; ++w)
+            for (int s = 0; s < kStages; ++s) {
+                mbar_init_count(smem_addr(&sm.full[w][s]), 1);
+                mbar_init_count(smem_addr(&sm.empty[w][s]), 1);
+            }
+        sm.abort_flag = 0;
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    if (warp == NW) {
+        produce_head<KF, VF, NW>(a, sm, ring_addr, head_groups, total_slots, lane);
+        return;
+    }
+    uint32_t lane_base;
+    asm volatile("or.b32 %0, %1, %2;" : "=r"(lane_base) : "r"(lut_addr), "r"(static_cast<uint32_t>(lane) << 2));
+    const uint32_t psel = (r & 1) ? 0x7632u : 0x5410u;
+    const int rows = group < NH ? group : NH;
+    const uint32_t my_ring = ring_addr + static_cast<uint32_t>(warp * kStages * kStageBytes);
+    uint32_t consumed = 0;
+    bool timed_out = false;
+    WarpTiles<KF, VF, NH> wt;
+
+    for (int64_t slot = blockIdx.x; slot < total_slots; slot += gridDim.x) {
+        Item it;
+        if (!item_of<1>(a, slot, head_groups, it)) continue;
+        const int head0 = it.h * group + it.hg * 8;  // first query head of the item
+        if (it.win) {
+            window_state(a, it, it.h, head0, rows, it.t0 + warp, NW, lane, &sm.red_m[warp][0], &sm.red_l[warp][0],
+                         &sm.red_o[warp][0][0], 1, kHeadDim);
+        } else {
+            wt.begin(a.qrot + (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim, rows, r, c);
+            const int ntiles = (it.t1 - it.t0 + 15) >> 4;
+            const int n_mine = ntiles > warp ? (ntiles - warp + NW - 1) / NW : 0;
+            for (int k = 0; k < n_mine; ++k) {
+                const uint32_t st = consumed % kStages;
+                if (!mbar_wait(smem_addr(&sm.full[warp][st]), (consumed / kStages) & 1u)) {
+                    timed_out = true;
+                    break;
+                }
+                // Slot layout: [K rows][K norms][V rows][V norms].
+                const uint32_t kbase = my_ring + st * kStageBytes, vbase = kbase + 16 * KF::IB + 32;
+                wt.step(kbase, kbase + 16 * KF::IB, vbase, vbase + 16 * VF::IB,
+                        min(16, it.t1 - (it.t0 + 16 * (warp + k * NW))), lane_base, psel, lane, r, c);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&sm.empty[warp][st]));  // slot free for the producer
+                ++consumed;
+            }
+            wt.finish(&sm.red_m[warp][0], &sm.red_l[warp][0], &sm.red_o[warp][0][0], 1, kHeadDim, rows, r, c);
         }
         if (timed_out && lane == 0) {
             atomicOr(&sm.abort_flag, 1);
             if (a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
         }
-        __syncthreads();
-        if (sm.abort_flag) break;
+        named_sync<NW * 32>();
+        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) break;
         // Merge the warps and write one record per query head.
-        float* rec = a.ws + ((static_cast<int64_t>(it.b) * H + it.h) * a.items_per_unit + it.split) *
-                                static_cast<int64_t>(group) * (kHeadDim + 2);
-        for (int e = threadIdx.x; e < rows * kHeadDim; e += kNW * 32) {
+        float* rec = record_of(a, it.b, it.h, it.split, group);
+        for (int e = threadIdx.x; e < rows * kHeadDim; e += NW * 32) {
             const int g = e / kHeadDim, jj = e - g * kHeadDim;
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kNW; ++w) M = fmaxf(M, sm.red_m[w][g]);
+            for (int w = 0; w < NW; ++w) M = fmaxf(M, sm.red_m[w][g]);
             float Ls = 0.0f, A = 0.0f;
             if (M != -INFINITY) {
 #pragma unroll
-                for (int w = 0; w < kNW; ++w) {
+                for (int w = 0; w < NW; ++w) {
                     const float mw = sm.red_m[w][g];
                     if (mw != -INFINITY) {
                         const float f = ex2(mw - M);
@@ -774,16 +1241,7 @@ __global__ void __launch_bounds__(kNW * 32, 1) decode_mma_kernel(DecodeArgs a, L
                 rg[1] = Ls;
             }
         }
-        __syncthreads();
-    }
-    // Drain this warp's copies still in flight (bounded) before the CTA exits.
-    for (; consumed < issued; ++consumed) {
-        const uint32_t s = consumed % kStages;
-        if (!mbar_wait(bar0 + 8 * s, (phase_bits >> s) & 1u)) {
-            if (lane == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
-            break;
-        }
-        phase_bits ^= 1u << s;
+        named_sync<NW * 32>();
     }
 }
 
@@ -818,13 +1276,28 @@ __global__ void __launch_bounds__(128) rotate_queries_kernel(DevCodec kc, const 
     for (int i = 0; i < 4; ++i) out[row * kHeadDim + kc.pos[h * kHeadDim + 4 * lane + i]] = z[i] * sc;
 }
 
+constexpr int kMaxDynSmem = 227 * 1024;
+
 template <class KF, class VF, int NH>
 tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaStream_t s) {
+    constexpr int NW = kNW;
+    constexpr size_t head_bytes = smem_bytes<NW, stage_bytes<KF, VF>()>();
+    static_assert(head_bytes <= kMaxDynSmem, "shared memory of the per-head decode kernel");
+    // The block kernel wants at least kBlkMinSlots slots beside the table.
+    const bool blk = a.kc.num_heads % kBlkWarps == 0 &&
+                     static_cast<size_t>(blk_slot_bytes<KF, VF>(a.block_size)) * kBlkMinSlots <=
+                         static_cast<size_t>(kMaxDynSmem) - kLut - 4096;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(decode_mma_kernel<KF, VF, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(kSmemBytes));
+        attr_err = cudaFuncSetAttribute(decode_mma_kernel<KF, VF, NH, NW>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(head_bytes));
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(decode_blk_kernel<KF, VF, NH, true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(decode_blk_kernel<KF, VF, NH, false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     });
     if (attr_err != cudaSuccess) return fail(TQ_ERR_CUDA, "cannot reserve shared memory for the decode kernel");
     int dev = 0, sms = 148;
@@ -834,10 +1307,20 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     const int64_t rows = static_cast<int64_t>(a.batch) * a.num_q_heads;
     rotate_queries_kernel<<<static_cast<unsigned>((rows + 3) / 4), 128, 0, s>>>(
         a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads, group, rows, a.scale_log2, a.qrot);
-    const int64_t slots = static_cast<int64_t>(a.items_per_unit) * a.batch * a.kc.num_heads * head_groups;
-    const int grid = static_cast<int>(slots < sms ? slots : sms);
-    if (grid > 0)
-        decode_mma_kernel<KF, VF, NH><<<grid, kNW * 32, kSmemBytes, s>>>(a, tv, group, head_groups, slots);
+    const int64_t units = static_cast<int64_t>(a.items_per_unit) * a.batch * head_groups *
+                          (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);
+    const int grid = static_cast<int>(units < sms ? units : sms);
+    if (grid > 0) {
+        if (blk && a.block_size == 16)
+            decode_blk_kernel<KF, VF, NH, true><<<grid, (kBlkWarps + 1) * 32, kMaxDynSmem, s>>>(a, tv, group,
+                                                                                                head_groups, units);
+        else if (blk)
+            decode_blk_kernel<KF, VF, NH, false><<<grid, (kBlkWarps + 1) * 32, kMaxDynSmem, s>>>(a, tv, group,
+                                                                                                 head_groups, units);
+        else
+            decode_mma_kernel<KF, VF, NH, NW><<<grid, (NW + 1) * 32, head_bytes, s>>>(a, tv, group, head_groups,
+                                                                                      units);
+    }
     return TQ_OK;
 }
 
@@ -866,8 +1349,8 @@ tq_status dispatch_v(const DecodeArgs& a, const tq_codec* vc, const LutValues& t
 
 tq_status launch_decode_mma(const DecodeArgs& a, const tq_codec* kc, const tq_codec* vc, int group, void* stream) {
     if (a.block_size % 16 != 0) return TQ_ERR_UNSUPPORTED;
+    if (a.split_tokens > 16 * kMaxItemTiles) return TQ_ERR_UNSUPPORTED;  // the producer's id buffer
     if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return TQ_ERR_UNSUPPORTED;
-    if (a.split_tokens > 16 * kNW * 32) return TQ_ERR_UNSUPPORTED;  // at most 32 tiles per warp and item
     LutValues tv{};
     for (const tq_codec* c : {kc, vc})
         for (int g = 0; g < c->desc.n_groups; ++g) {

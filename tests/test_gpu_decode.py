@@ -186,3 +186,48 @@ def test_tensor_core_and_general_kernels_agree(monkeypatch):
     torch.cuda.synchronize()
     assert (fast - general).abs().max().item() <= ATOL
     check(prob)
+
+
+# ---- KV head counts that are multiples of 8: the kernel that stages one
+# 16-token tile of 8 KV heads per ring slot and gives each warp one KV head.
+
+@pytest.mark.parametrize("kspec,vspec", [(U4, U4), (M35, M35), (M25, U3), (U2, M35), (U3, U2)])
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_decode_eight_kv_heads_matches_oracle(kspec, vspec, G):
+    lens = [1, 16, 17, 300, 1100]
+    prob = DecodeProblem(lens, 8, G, kspec, (vspec[0], vspec[1], vspec[2] + 10), window=0, block_size=16,
+                         seed=100 + G)
+    rng = np.random.default_rng(G)
+    pairs = [(b, int(hq)) for b in range(prob.B) for hq in rng.choice(prob.Hq, min(prob.Hq, 12), replace=False)]
+    check(prob, pairs)
+
+
+@pytest.mark.parametrize("window,bs", [(8, 16), (64, 32), (128, 48)])
+def test_decode_eight_kv_heads_windows_and_block_sizes(window, bs):
+    """Block sizes above 16 take the per-head copies of a slot; windows go to the warps directly."""
+    lens = [0, 1, window, window + 1, 3 * window + 5, 2100]
+    prob = DecodeProblem(lens, 8, 4, M25, U3, window=window, block_size=bs, seed=window + bs)
+    pairs = [(b, hq) for b in range(prob.B) for hq in (0, 5, 13, 31)]
+    check(prob, pairs)
+
+
+def test_decode_sixteen_kv_heads_gqa16():
+    """Two groups of 8 KV heads, two query-head groups per KV head."""
+    prob = DecodeProblem([5000, 700], 16, 16, U4, M35, window=16, block_size=16, seed=31)
+    pairs = [(b, hq) for b in range(prob.B) for hq in (0, 7, 8, 15, 130, 255)]
+    check(prob, pairs)
+
+
+def test_decode_eight_kv_heads_all_heads():
+    """Every query head of a GQA-8 cache with 8 KV heads (each warp's records)."""
+    prob = DecodeProblem([2500, 40], 8, 8, M35, M35, window=32, block_size=16, seed=41)
+    check(prob)
+
+
+def test_decode_eight_kv_heads_bad_block_id_sets_error_without_fault():
+    prob = DecodeProblem([200], 8, 2, U4, U4, window=0, block_size=16, seed=42)
+    prob.block_tables[0, 3] = -7
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    prob.run(d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() & tq.TQ_DERR_BLOCK
