@@ -65,7 +65,9 @@ static_assert(kNW >= 1 && kNW <= 11, "11 compute warps fill the shared memory");
 #endif
 constexpr int kStages = TQ_DECODE_STAGES;  // ring slots per compute warp
 constexpr int kLut = 65536;         // bytes of the dequantization table
-constexpr uint32_t kSpinLimit = 1u << 24;
+constexpr uint32_t kSpinLimit = 1u << 24;   // polls of a spinning wait
+constexpr uint32_t kWaitHintNs = 16384;     // sleep bound of one blocking wait attempt
+constexpr uint32_t kWaitRounds = 1u << 16;  // blocking wait attempts (about a second)
 constexpr float kSlack = 8.0f;                 // log2 slack of the running max
 constexpr float kSlackInv = 1.0f / 256.0f;     // 2^-kSlack, folded into P'
 
@@ -178,18 +180,21 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// One wait attempt: the thread sleeps until phase `parity` of `bar` completes
+// or about kWaitHintNs pass; true when the phase completed.
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "n"(kWaitHintNs)
         : "memory");
     return ok != 0;
 }
-// Bounded wait for phase `parity` of `bar`; false when the limit expired.
+// Bounded wait for phase `parity` of `bar` (about a second at most); false
+// when the limit expired.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
+    for (uint32_t i = 0; i < kWaitRounds; ++i)
         if (mbar_try(bar, parity)) return true;
     return false;
 }
@@ -368,21 +373,6 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded, warp-uniform poll (every lane of the warp calls it).
-__device__ __forceinline__ bool mbar_poll_warp(uint32_t bar, uint32_t parity) {
-    bool ready = false;
-    for (uint32_t i = 0; i < kSpinLimit && !ready; ++i) ready = __any_sync(kFull, mbar_test(bar, parity));
-    return ready;
-}
-// Bounded wait by one thread that polls with short sleeps in between: it
-// reacts within about 100 ns and leaves the issue slots to the compute warps.
-__device__ __forceinline__ bool mbar_sleep_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (mbar_test(bar, parity)) return true;
-        __nanosleep(64);
-    }
-    return false;
-}
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -440,6 +430,7 @@ template <class KF, class VF, int NH>
 struct WarpTiles {
     static constexpr int HL = NH / 4;  // heads per lane
     uint32_t bq[8][2 * HL];            // query B fragments per k-step
+    uint32_t bp[2 * HL];               // P' B fragments of the last scored tile
     float o[8][4];                     // value accumulators: row tile q, rows r / r + 8, columns 2c / 2c + 1
     float m_ref[HL], l_run[HL];
 
@@ -475,10 +466,11 @@ struct WarpTiles {
         }
     }
 
-    // One 16-token tile: K index rows at kbase (norms at knorm), V index rows at
-    // vbase (norms at vnorm); tokens at or past nvalid are padding.
-    __device__ __forceinline__ void step(uint32_t kbase, uint32_t knorm, uint32_t vbase, uint32_t vnorm, int nvalid,
-                                         uint32_t lane_base, uint32_t psel, int lane, int r, int c) {
+    // Scores of one 16-token tile (K index rows at kbase, norms at knorm) and
+    // the online-softmax update; leaves the tile's P' (V norms at vnorm) in bp
+    // for values(). Tokens at or past nvalid are padding.
+    __device__ __forceinline__ void scores(uint32_t kbase, uint32_t knorm, uint32_t vnorm, int nvalid,
+                                           uint32_t lane_base, uint32_t psel, int r, int c) {
         // ---- S^T = K^ Q'^T: rows tokens r, r + 8 ----
         // Independent accumulator chains (k-step parity; hi / lo for NH = 8)
         // keep the MMA dependency depth at 4.
@@ -598,7 +590,6 @@ struct WarpTiles {
         // Tokens 2c and 2c + 8 sit in lane 8c + (r >> 1), tokens 2c + 1 and
         // 2c + 9 four lanes on.
         const int srcA = 8 * c + (r >> 1), srcB = srcA + 4;
-        uint32_t bp[2 * HL];
         if constexpr (NH == 8) {
             // Per token: (head 2c, head 2c + 1) as hi and lo half2.
             uint32_t th0, tl0, th1, tl1;
@@ -622,6 +613,18 @@ struct WarpTiles {
             bp[0] = prmt(pa, pb, 0x5410u);
             bp[1] = prmt(pa, pb, 0x7632u);
         }
+    }
+
+    // One 16-token tile: K index rows at kbase (norms at knorm), V index rows at
+    // vbase (norms at vnorm); tokens at or past nvalid are padding.
+    __device__ __forceinline__ void step(uint32_t kbase, uint32_t knorm, uint32_t vbase, uint32_t vnorm, int nvalid,
+                                         uint32_t lane_base, uint32_t psel, int r, int c) {
+        scores(kbase, knorm, vnorm, nvalid, lane_base, psel, r, c);
+        values(vbase, lane_base, r, c);
+    }
+
+    // O^T += V^T P'^T for the tile last passed to scores(): V index rows at vbase.
+    __device__ __forceinline__ void values(uint32_t vbase, uint32_t lane_base, int r, int c) {
         auto value_step = [&](auto qi, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
             constexpr int q = decltype(qi)::value;
             mma16816(o[q], a0, a1, a2, a3, bp[0], bp[1]);
@@ -863,7 +866,7 @@ __device__ void produce_blk(const DecodeArgs& a, BlkSmem& sm, const BlkRing& rin
                 const int s = static_cast<int>(fill % ring.n);
                 const uint32_t use = fill / ring.n;
                 const uint32_t full = smem_addr(&sm.full[s]);
-                if (use > 0 && !mbar_sleep_wait(smem_addr(&sm.empty[s]), (use - 1) & 1u)) {
+                if (use > 0 && !mbar_wait(smem_addr(&sm.empty[s]), (use - 1) & 1u)) {
                     // The compute warps stop on their own bounded waits.
                     if (a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
                     stop = true;
@@ -899,9 +902,10 @@ __device__ void produce_blk(const DecodeArgs& a, BlkSmem& sm, const BlkRing& rin
             if (!mbar_wait(smem_addr(&sm.full[f % ring.n]), (f / ring.n) & 1u)) break;
 }
 
-// B16: the block size is 16 (one tile per slot; a simpler consumer loop that
-// measured markedly faster than the general one).
-template <class KF, class VF, int NH, bool B16>
+// TPB: 16-token tiles per block when the block size is 16 or 32 (a consumer
+// loop with fixed offsets, which measured markedly faster), else 0 (any
+// multiple of 16).
+template <class KF, class VF, int NH, int TPB>
 __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(DecodeArgs a, LutValues tv, int group,
                                                                              int head_groups, int64_t total_slots) {
     static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
@@ -963,16 +967,20 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
         wt.begin(a.qrot + (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim, rows, r, c);
         bool timed_out = false;
         const int ntiles = (it.t1 - it.t0 + 15) >> 4;
-        if constexpr (B16) {
-            for (int k = 0; k < ntiles; ++k, ++consumed) {
+        if constexpr (TPB > 0) {
+            constexpr int kBs = 16 * TPB;
+            for (int k = 0; k < ntiles; k += TPB, ++consumed) {
                 const int s = static_cast<int>(consumed % ring.n);
                 if (!mbar_wait(smem_addr(&sm.full[s]), (consumed / ring.n) & 1u)) {
                     timed_out = true;
                     break;
                 }
                 const uint32_t kb = ring.slot(s) + k_off, vb = ring.slot(s) + v_off;
-                wt.step(kb, kb + 16 * KF::IB, vb, vb + 16 * VF::IB, min(16, it.t1 - (it.t0 + 16 * k)), lane_base,
-                        psel, lane, r, c);
+#pragma unroll 1
+                for (int j = 0; j < TPB && k + j < ntiles; ++j)
+                    wt.step(kb + 16 * j * KF::IB, kb + kBs * KF::IB + 32 * j, vb + 16 * j * VF::IB,
+                            vb + kBs * VF::IB + 32 * j, min(16, it.t1 - (it.t0 + 16 * (k + j))), lane_base, psel, r,
+                            c);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with the slot
             }
@@ -991,7 +999,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
                     vb = ring.slot(s) + v_off;
                 }
                 wt.step(kb + 16 * j * KF::IB, kb + bs * KF::IB + 32 * j, vb + 16 * j * VF::IB,
-                        vb + bs * VF::IB + 32 * j, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, psel, lane, r, c);
+                        vb + bs * VF::IB + 32 * j, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, psel, r, c);
                 if (++j == tpb || k + 1 == ntiles) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with the slot
@@ -1202,7 +1210,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
                 // Slot layout: [K rows][K norms][V rows][V norms].
                 const uint32_t kbase = my_ring + st * kStageBytes, vbase = kbase + 16 * KF::IB + 32;
                 wt.step(kbase, kbase + 16 * KF::IB, vbase, vbase + 16 * VF::IB,
-                        min(16, it.t1 - (it.t0 + 16 * (warp + k * NW))), lane_base, psel, lane, r, c);
+                        min(16, it.t1 - (it.t0 + 16 * (warp + k * NW))), lane_base, psel, r, c);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&sm.empty[warp][st]));  // slot free for the producer
                 ++consumed;
@@ -1293,10 +1301,13 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
         attr_err = cudaFuncSetAttribute(decode_mma_kernel<KF, VF, NH, NW>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(head_bytes));
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(decode_blk_kernel<KF, VF, NH, true>,
+            attr_err = cudaFuncSetAttribute(decode_blk_kernel<KF, VF, NH, 1>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(decode_blk_kernel<KF, VF, NH, false>,
+            attr_err = cudaFuncSetAttribute(decode_blk_kernel<KF, VF, NH, 2>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(decode_blk_kernel<KF, VF, NH, 0>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     });
     if (attr_err != cudaSuccess) return fail(TQ_ERR_CUDA, "cannot reserve shared memory for the decode kernel");
@@ -1311,12 +1322,13 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
                           (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);
     const int grid = static_cast<int>(units < sms ? units : sms);
     if (grid > 0) {
+        const dim3 threads((kBlkWarps + 1) * 32);
         if (blk && a.block_size == 16)
-            decode_blk_kernel<KF, VF, NH, true><<<grid, (kBlkWarps + 1) * 32, kMaxDynSmem, s>>>(a, tv, group,
-                                                                                                head_groups, units);
+            decode_blk_kernel<KF, VF, NH, 1><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
+        else if (blk && a.block_size == 32)
+            decode_blk_kernel<KF, VF, NH, 2><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
         else if (blk)
-            decode_blk_kernel<KF, VF, NH, false><<<grid, (kBlkWarps + 1) * 32, kMaxDynSmem, s>>>(a, tv, group,
-                                                                                                 head_groups, units);
+            decode_blk_kernel<KF, VF, NH, 0><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
         else
             decode_mma_kernel<KF, VF, NH, NW><<<grid, (NW + 1) * 32, head_bytes, s>>>(a, tv, group, head_groups,
                                                                                       units);
