@@ -22,6 +22,10 @@
 //    idx = below + (v > boundary) with one compare.
 //  * Rows are staged in shared memory and written with 16-byte stores; norms
 //    go to the sub-page's norm array.
+//  * Loads. Each warp copies its next unit's 16 input rows into a shared
+//    buffer with cp.async while it computes the current one (double
+//    buffering); ldmatrix reads the MMA A fragments from rows padded to 272
+//    bytes, free of bank conflicts.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -30,6 +34,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "tq_internal.h"
 
@@ -37,7 +42,8 @@ namespace tq {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kPW = 8;               // warps per CTA
+constexpr int kPW = 16;              // warps per CTA (one CTA per SM)
+constexpr int kRowPad = 272;         // bytes per staged input row (256 + 16: 8 rows hit 8 bank quads)
 constexpr int kCells = 129;          // v = 64 u in [-64, 64], cells round(v) + 64
 constexpr float kCellScale = 64.0f;
 
@@ -51,6 +57,7 @@ struct PackSmem {
     uint32_t bfrag[2][8][2][32][2];  // [K/V][a][n-tile][lane][reg]: B operands (+-1 bf16 pairs)
     uint8_t rows[kPW][16][64];       // staged index rows of a warp's 16 tokens
     unsigned short norms[kPW][16];
+    uint8_t xbuf[kPW][2][16][kRowPad];  // double-buffered input rows (bf16) of a warp's units
 };
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -85,11 +92,40 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+// The two bf16 of a word as an fp32 pair (exact).
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+    return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     uint2 v;
     asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
     return v;
+}
+
+template <int I = 0, class F>
+__device__ __forceinline__ void static_for8(F&& f) {
+    if constexpr (I < 8) {
+        f(std::integral_constant<int, I>{});
+        static_for8<I + 1>(f);
+    }
+}
+
+// Byte store to shared address base + OFF (OFF a compile-time offset).
+template <int OFF>
+__device__ __forceinline__ void sts8(uint32_t base, uint32_t v) {
+    asm volatile("st.shared.u8 [%0+%1], %2;" ::"r"(base), "n"(OFF), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& d0, uint32_t& d1, uint32_t& d2, uint32_t& d3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(d0), "=r"(d1), "=r"(d2), "=r"(d3)
+                 : "r"(addr));
 }
 
 __device__ __forceinline__ double warp4_sum_d(double v) {
@@ -98,12 +134,17 @@ __device__ __forceinline__ double warp4_sum_d(double v) {
     return v;
 }
 
-__global__ void __launch_bounds__(kPW * 32, 2) pack_u4_kernel(DevCodec kc, DevCodec vc, QuantCell* __restrict__ g_cells,
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__global__ void __launch_bounds__(kPW * 32, 1) pack_u4_kernel(DevCodec kc, DevCodec vc, QuantCell* __restrict__ g_cells,
                                                           const __nv_bfloat16* __restrict__ k,
                                                           const __nv_bfloat16* __restrict__ v,
-                                                          const int64_t* __restrict__ slots, int64_t num_tokens,
+                                                          const int64_t* __restrict__ slots, int num_tokens,
                                                           uint8_t* __restrict__ k_pages, uint8_t* __restrict__ v_pages,
-                                                          int64_t num_blocks, int block_size, int* __restrict__ d_err) {
+                                                          int capacity, int block_size, int bs_log2,
+                                                          int* __restrict__ d_err) {
     extern __shared__ __align__(16) uint8_t psm_raw[];
     PackSmem& sm = *reinterpret_cast<PackSmem*>(psm_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -115,12 +156,12 @@ __global__ void __launch_bounds__(kPW * 32, 2) pack_u4_kernel(DevCodec kc, DevCo
         const int ln = i & 31, t = (i >> 5) & 1, a = (i >> 6) & 7, which = i >> 9;
         const float* sign = which ? vc.sign : kc.sign;
         const int rr = ln >> 2, cc = ln & 3;
-        const int bp = 4 * (rr >> 1) + 2 * t + (rr & 1);  // output column b' of lane rr in n-tile t
+        const int bp = 8 * t + rr;  // output column b' of lane rr in n-tile t
         uint32_t regs[2];
         for (int q = 0; q < 2; ++q) {
             unsigned short h[2];
             for (int e = 0; e < 2; ++e) {
-                const int b = 4 * cc + 2 * q + e;          // input coordinate b of this k-slot
+                const int b = 2 * cc + 8 * q + e;          // input coordinate b of this k-slot
                 const float val = sign[16 * a + b] * ((__popc(bp & b) & 1) ? -1.0f : 1.0f);
                 h[e] = val > 0 ? 0x3F80 : 0xBF80;
             }
@@ -131,148 +172,175 @@ __global__ void __launch_bounds__(kPW * 32, 2) pack_u4_kernel(DevCodec kc, DevCo
     }
     __syncthreads();
 
-    const int64_t H = kc.num_heads;
-    const int64_t groups = (num_tokens + 15) / 16;
-    const int64_t units = groups * H * 2;
-    const int64_t capacity = num_blocks * block_size;
+    // 32-bit index arithmetic throughout: the host checks that tokens, units and
+    // slots fit (a 64-bit division is a long software routine on the GPU).
+    const int H = kc.num_heads;
+    const int units = (num_tokens + 15) / 16 * H * 2;
     const uint32_t cell_lane = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.cells[0][lane]));
     // address of cell e for this lane = cell_lane + e * 256; e = bits(v + 1.5*2^23) - 0x4B400000 + 64
     const uint32_t cell_adj = cell_lane + 64u * 256u - 0x40000000u;
 
-    for (int64_t u = static_cast<int64_t>(blockIdx.x) * kPW + warp; u < units;
-         u += static_cast<int64_t>(gridDim.x) * kPW) {
-        const int which = static_cast<int>(u & 1);
-        const int64_t gh = u >> 1;
-        const int h = static_cast<int>(gh % H);
-        const int64_t t0 = (gh / H) * 16;
-        const __nv_bfloat16* src = which ? v : k;
+    // Unit u = (16-token group, KV head, K or V). The warp's 16 input rows of a
+    // unit are 16 x 256 contiguous bytes at a stride of H x 256: lane l copies
+    // 16-byte pieces l, l + 32, ... (token = piece / 16); rows past the end are
+    // zero-filled without reading.
+    const uint32_t xbuf0 = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.xbuf[warp][0][0][0]));
+    auto issue = [&](int uu, int buf) {
+        const int which_ = uu & 1, gh_ = uu >> 1;
+        const int tg_ = gh_ / H, h_ = gh_ - tg_ * H;
+        const __nv_bfloat16* src_ = which_ ? v : k;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int piece = lane + 32 * i, tok = piece >> 4, part = piece & 15;
+            const int t = tg_ * 16 + tok;
+            const bool live = t < num_tokens;
+            // A row past the end is zero-filled (no bytes read; the address stays in the tensor).
+            const __nv_bfloat16* g = src_ + (static_cast<int64_t>(live ? t : 0) * H + h_) * kHeadDim + 8 * part;
+            cp_async16(xbuf0 + (buf * 16 + tok) * kRowPad + 16 * part, g, live ? 16u : 0u);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    const int stride = gridDim.x * kPW;
+    int u = blockIdx.x * kPW + warp;
+    if (u < units) issue(u, 0);
+    for (int it = 0; u < units; u += stride, ++it) {
+        const int cur = it & 1;
+        const int which = u & 1;
+        const int gh = u >> 1;
+        const int tg = gh / H, h = gh - tg * H;
+        const int t0 = tg * 16;
 
         // Slots of the 16 tokens (lane i < 16 holds token t0 + i).
         int64_t my_slot = -1;
         if (lane < 16 && t0 + lane < num_tokens) my_slot = __ldg(slots + t0 + lane);
-        const bool live_lo = t0 + r < num_tokens, live_hi = t0 + r + 8 < num_tokens;
 
-        // A operands: tokens r and r + 8, coordinates 16a + 4c .. 16a + 4c + 3.
-        uint2 xa[8], xb[8];
-        const __nv_bfloat16* p_lo = src + ((t0 + r) * H + h) * kHeadDim + 4 * c;
-        const __nv_bfloat16* p_hi = src + ((t0 + r + 8) * H + h) * kHeadDim + 4 * c;
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-            xa[a] = live_lo ? __ldg(reinterpret_cast<const uint2*>(p_lo + 16 * a)) : make_uint2(0, 0);
-            xb[a] = live_hi ? __ldg(reinterpret_cast<const uint2*>(p_hi + 16 * a)) : make_uint2(0, 0);
+        // The next unit's rows go to the other buffer while this one is computed.
+        if (u + stride < units) {
+            issue(u + stride, cur ^ 1);
+        } else {
+            asm volatile("cp.async.commit_group;" ::: "memory");
         }
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncwarp();
 
-        // z = (H_16 D_s) per a on the tensor cores: zc[a][t] holds columns b' = 4c + 2t + {0,1}.
-        float zc[8][2][4];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const uint2 bf = *reinterpret_cast<const uint2*>(&sm.bfrag[which][a][t][lane][0]);
-                mma_bf16(zc[a][t], xa[a].x, xb[a].x, xa[a].y, xb[a].y, bf.x, bf.y);
-            }
-        }
-
-        // Sum of exact squares (fp32), per token, over this lane's 32 coordinates then the 4 lanes.
-        float ss_lo = 0.0f, ss_hi = 0.0f;
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-            const float l0 = __uint_as_float(xa[a].x << 16), l1 = __uint_as_float(xa[a].x & 0xffff0000u);
-            const float l2 = __uint_as_float(xa[a].y << 16), l3 = __uint_as_float(xa[a].y & 0xffff0000u);
-            const float h0 = __uint_as_float(xb[a].x << 16), h1 = __uint_as_float(xb[a].x & 0xffff0000u);
-            const float h2 = __uint_as_float(xb[a].y << 16), h3 = __uint_as_float(xb[a].y & 0xffff0000u);
-            ss_lo = fmaf(l0, l0, fmaf(l1, l1, fmaf(l2, l2, fmaf(l3, l3, ss_lo))));
-            ss_hi = fmaf(h0, h0, fmaf(h1, h1, fmaf(h2, h2, fmaf(h3, h3, ss_hi))));
-        }
-        ss_lo += __shfl_xor_sync(kFull, ss_lo, 1);
-        ss_lo += __shfl_xor_sync(kFull, ss_lo, 2);
-        ss_hi += __shfl_xor_sync(kFull, ss_hi, 1);
-        ss_hi += __shfl_xor_sync(kFull, ss_hi, 2);
-
-        // fp16 norm, correctly rounded; fp64 when the fp32 value is too close to call.
+        // A operands of group a (ldmatrix.x4, once per half below to keep registers
+        // low): xa[a] = token r, coordinates 16a + 2c + {0,1} and 16a + 2c + 8 + {0,1};
+        // xb[a] the same for token r + 8. Lane l addresses row l % 8 of matrix l / 8.
+        const uint32_t frag_row = xbuf0 + (cur * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)) * kRowPad +
+                                  ((lane >> 4) & 1) * 16;
         float n_tok[2];
         unsigned short n16[2];
-        bool risky[2];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float ss = i ? ss_hi : ss_lo;
-            const float n32 = sqrtf(ss);
-            bool rk = !(ss > 1e-30f && ss < 1e30f) || n32 > 60000.0f;
-            const __half hh = __float2half_rn(n32);
-            const unsigned short hb = __half_as_ushort(hh);
-            if (!rk) {
-                const float hf = __half2float(hh);
-                const float up = __half2float(__ushort_as_half(static_cast<unsigned short>(hb + 1)));
-                const float dn = __half2float(__ushort_as_half(static_cast<unsigned short>(hb - 1)));
-                const float tol = 1e-6f * n32;
-                rk = fabsf(n32 - 0.5f * (hf + up)) <= tol || fabsf(n32 - 0.5f * (hf + dn)) <= tol;
-            }
-            risky[i] = rk;
-            n_tok[i] = n32;
-            n16[i] = hb;
-        }
-        if (__any_sync(kFull, risky[0] || risky[1])) {
-            // Rare: exact-enough fp64 sums for the tokens that need them (all lanes join the shuffles).
-            double d_lo = 0.0, d_hi = 0.0;
+        for (int t = 0; t < 2; ++t) {
+            uint2 xa[8], xb[8];
 #pragma unroll
-            for (int a = 0; a < 8; ++a) {
-                const double l0 = __uint_as_float(xa[a].x << 16), l1 = __uint_as_float(xa[a].x & 0xffff0000u);
-                const double l2 = __uint_as_float(xa[a].y << 16), l3 = __uint_as_float(xa[a].y & 0xffff0000u);
-                const double h0 = __uint_as_float(xb[a].x << 16), h1 = __uint_as_float(xb[a].x & 0xffff0000u);
-                const double h2 = __uint_as_float(xb[a].y << 16), h3 = __uint_as_float(xb[a].y & 0xffff0000u);
-                d_lo += l0 * l0 + l1 * l1 + l2 * l2 + l3 * l3;
-                d_hi += h0 * h0 + h1 * h1 + h2 * h2 + h3 * h3;
-            }
-            d_lo = warp4_sum_d(d_lo);
-            d_hi = warp4_sum_d(d_hi);
+            for (int a = 0; a < 8; ++a) ldsm_x4(frag_row + 32 * a, xa[a].x, xb[a].x, xa[a].y, xb[a].y);
+            if (t == 0) {
+                // Sum of exact squares (fp32), per token, over this lane's 32 coordinates
+                // (two interleaved partial sums in a packed pair) then the 4 lanes.
+                float ss_lo, ss_hi;
+                {
+                    uint64_t acc_lo = 0, acc_hi = 0;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                if (risky[i]) {
-                    const double nd = sqrt(i ? d_hi : d_lo);
-                    n16[i] = __half_as_ushort(__double2half(nd));
-                    n_tok[i] = static_cast<float>(nd);
+                    for (int a = 0; a < 8; ++a) {
+                        const uint64_t l01 = bf16x2_to_f32x2(xa[a].x), l23 = bf16x2_to_f32x2(xa[a].y);
+                        const uint64_t h01 = bf16x2_to_f32x2(xb[a].x), h23 = bf16x2_to_f32x2(xb[a].y);
+                        acc_lo = fma2(l01, l01, fma2(l23, l23, acc_lo));
+                        acc_hi = fma2(h01, h01, fma2(h23, h23, acc_hi));
+                    }
+                    float p, q;
+                    upk(acc_lo, p, q);
+                    ss_lo = p + q;
+                    upk(acc_hi, p, q);
+                    ss_hi = p + q;
+                }
+                ss_lo += __shfl_xor_sync(kFull, ss_lo, 1);
+                ss_lo += __shfl_xor_sync(kFull, ss_lo, 2);
+                ss_hi += __shfl_xor_sync(kFull, ss_hi, 1);
+                ss_hi += __shfl_xor_sync(kFull, ss_hi, 2);
+
+                // fp16 norm, correctly rounded; fp64 when the fp32 value is too close to call.
+                bool risky[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float ss = i ? ss_hi : ss_lo;
+                    const float n32 = sqrtf(ss);
+                    bool rk = !(ss > 1e-30f && ss < 1e30f) || n32 > 60000.0f;
+                    const __half hh = __float2half_rn(n32);
+                    const unsigned short hb = __half_as_ushort(hh);
+                    if (!rk) {
+                        const float hf = __half2float(hh);
+                        const float up = __half2float(__ushort_as_half(static_cast<unsigned short>(hb + 1)));
+                        const float dn = __half2float(__ushort_as_half(static_cast<unsigned short>(hb - 1)));
+                        const float tol = 1e-6f * n32;
+                        rk = fabsf(n32 - 0.5f * (hf + up)) <= tol || fabsf(n32 - 0.5f * (hf + dn)) <= tol;
+                    }
+                    risky[i] = rk;
+                    n_tok[i] = n32;
+                    n16[i] = hb;
+                }
+                if (__any_sync(kFull, risky[0] || risky[1])) {
+                    // Rare: exact-enough fp64 sums for the tokens that need them (all lanes join the shuffles).
+                    double d_lo = 0.0, d_hi = 0.0;
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) {
+                        const double l0 = __uint_as_float(xa[a].x << 16), l1 = __uint_as_float(xa[a].x & 0xffff0000u);
+                        const double l2 = __uint_as_float(xa[a].y << 16), l3 = __uint_as_float(xa[a].y & 0xffff0000u);
+                        const double h0 = __uint_as_float(xb[a].x << 16), h1 = __uint_as_float(xb[a].x & 0xffff0000u);
+                        const double h2 = __uint_as_float(xb[a].y << 16), h3 = __uint_as_float(xb[a].y & 0xffff0000u);
+                        d_lo += l0 * l0 + l1 * l1 + l2 * l2 + l3 * l3;
+                        d_hi += h0 * h0 + h1 * h1 + h2 * h2 + h3 * h3;
+                    }
+                    d_lo = warp4_sum_d(d_lo);
+                    d_hi = warp4_sum_d(d_hi);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        if (risky[i]) {
+                            const double nd = sqrt(i ? d_hi : d_lo);
+                            n16[i] = __half_as_ushort(__double2half(nd));
+                            n_tok[i] = static_cast<float>(nd);
+                        }
+                    }
                 }
             }
-        }
 
-        // H_8 across a (three butterfly stages on packed pairs).
-        uint64_t zp[8][2][2];  // [a][t][token]: (columns 2c, 2c+1 of n-tile t)
-#pragma unroll
-        for (int a = 0; a < 8; ++a)
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                zp[a][t][0] = pk(zc[a][t][0], zc[a][t][1]);
-                zp[a][t][1] = pk(zc[a][t][2], zc[a][t][3]);
-            }
-#pragma unroll
-        for (int m = 1; m < 8; m <<= 1)
-#pragma unroll
-            for (int a = 0; a < 8; ++a)
-                if (!(a & m))
-#pragma unroll
-                    for (int t = 0; t < 2; ++t)
-#pragma unroll
-                        for (int i = 0; i < 2; ++i) {
-                            const uint64_t x0 = zp[a][t][i], x1 = zp[a | m][t][i];
-                            zp[a][t][i] = add2(x0, x1);
-                            zp[a | m][t][i] = sub2(x0, x1);
-                        }
-
-        // Quantize: v = z * 64 / (sqrt(128) n); cell lookup; pack 4 nibbles per (token, a').
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float n = n_tok[i];
-            float kq = n > 0.0f ? kCellScale / (n * 11.313708498984761f) : 0.0f;
-            if (!(kq < 3.0e38f)) kq = 0.0f;  // norms too small to scale: treat as the zero vector
-            const uint64_t kq2 = pk(kq, kq);
-            const uint64_t magic2 = pk(12582912.0f, 12582912.0f);
-            unsigned short* row = reinterpret_cast<unsigned short*>(&sm.rows[warp][r + 8 * i][0]);
+            // z = (H_16 D_s) per a on the tensor cores: columns b' = 8t + 2c + {0,1} of n-tile t.
+            uint64_t zp[8][2];  // [a][token]: (columns 2c, 2c+1 of n-tile t)
 #pragma unroll
             for (int a = 0; a < 8; ++a) {
-                uint32_t word = 0;
+                const uint2 bf = *reinterpret_cast<const uint2*>(&sm.bfrag[which][a][t][lane][0]);
+                float zc[4];
+                mma_bf16(zc, xa[a].x, xb[a].x, xa[a].y, xb[a].y, bf.x, bf.y);
+                zp[a][0] = pk(zc[0], zc[1]);
+                zp[a][1] = pk(zc[2], zc[3]);
+            }
+            // H_8 across a (three butterfly stages on packed pairs).
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    const uint64_t vv = mul2(zp[a][t][i], kq2);
+            for (int m = 1; m < 8; m <<= 1)
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+                    if (!(a & m))
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const uint64_t x0 = zp[a][i], x1 = zp[a | m][i];
+                            zp[a][i] = add2(x0, x1);
+                            zp[a | m][i] = sub2(x0, x1);
+                        }
+
+            // Quantize: v = z * 64 / (sqrt(128) n); cell lookup; one byte (2 nibbles,
+            // coordinates 16a' + 8t + 2c and the next) per (token, a').
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float n = n_tok[i];
+                float kq = n > 0.0f ? kCellScale / (n * 11.313708498984761f) : 0.0f;
+                if (!(kq < 3.0e38f)) kq = 0.0f;  // norms too small to scale: treat as the zero vector
+                const uint64_t kq2 = pk(kq, kq);
+                const uint64_t magic2 = pk(12582912.0f, 12582912.0f);
+                const uint32_t row =
+                    static_cast<uint32_t>(__cvta_generic_to_shared(&sm.rows[warp][r + 8 * i][c])) + 4 * t;
+                static_for8([&](auto ai) {
+                    constexpr int a = decltype(ai)::value;
+                    const uint64_t vv = mul2(zp[a][i], kq2);
                     const uint64_t mm = add2(vv, magic2);
                     float v0, v1, m0, m1;
                     upk(vv, v0, v1);
@@ -281,11 +349,10 @@ __global__ void __launch_bounds__(kPW * 32, 2) pack_u4_kernel(DevCodec kc, DevCo
                     const uint2 e1 = lds64(__float_as_uint(m1) * 256u + cell_adj);
                     const uint32_t i0 = e0.y + (v0 > __uint_as_float(e0.x) ? 1u : 0u);
                     const uint32_t i1 = e1.y + (v1 > __uint_as_float(e1.x) ? 1u : 0u);
-                    word |= (i0 | (i1 << 4)) << (8 * t);
-                }
-                row[4 * a + c] = static_cast<unsigned short>(word);  // bytes 8a + 2c, 8a + 2c + 1
+                    sts8<8 * a>(row, i0 | (i1 << 4));
+                });
+                if (t == 0 && c == 0) sm.norms[warp][r + 8 * i] = n16[i];
             }
-            if (c == 0) sm.norms[warp][r + 8 * i] = n16[i];
         }
         __syncwarp();
 
@@ -297,8 +364,10 @@ __global__ void __launch_bounds__(kPW * 32, 2) pack_u4_kernel(DevCodec kc, DevCo
             const int chunk = lane + 32 * q, row = chunk >> 2, part = chunk & 3;
             const int64_t slot = __shfl_sync(kFull, my_slot, row);
             if (slot >= 0 && slot < capacity) {
-                const int64_t blk = slot / block_size, off = slot - blk * block_size;
-                uint8_t* sub = pages + (blk * H + h) * block_size * rb;
+                const int s32 = static_cast<int>(slot);
+                const int blk = bs_log2 >= 0 ? s32 >> bs_log2 : s32 / block_size;
+                const int off = s32 - blk * block_size;
+                uint8_t* sub = pages + (static_cast<int64_t>(blk) * H + h) * block_size * rb;
                 *reinterpret_cast<uint4*>(sub + off * 64 + 16 * part) =
                     *reinterpret_cast<const uint4*>(&sm.rows[warp][row][16 * part]);
                 if (part == 0)
@@ -336,6 +405,11 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
         if (c->desc.n_groups != 1 || c->desc.group_bits[0] != 4) return TQ_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 15) return TQ_ERR_UNSUPPORTED;
     if (block_size % 8 != 0) return TQ_ERR_UNSUPPORTED;  // 16-byte aligned rows and norm arrays
+    // 32-bit index arithmetic in the kernel: slots, tokens and work units must fit.
+    const int64_t capacity = num_blocks * block_size;
+    const int64_t n_units = (num_tokens + 15) / 16 * kc->desc.num_kv_heads * 2;
+    if (capacity > INT32_MAX || n_units > INT32_MAX || num_tokens > INT32_MAX - 16) return TQ_ERR_UNSUPPORTED;
+    const int bs_log2 = (block_size & (block_size - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(block_size)) : -1;
     // The cell table depends only on the 4-bit codebook, the same for every codec.
     static std::once_flag once;
     static QuantCell* d_cells = nullptr;
@@ -353,13 +427,12 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t units = (num_tokens + 15) / 16 * kc->desc.num_kv_heads * 2;
-    const int64_t want = (units + kPW - 1) / kPW;
-    const int grid = static_cast<int>(want < 4LL * sms ? want : 4LL * sms);
+    const int64_t want = (n_units + kPW - 1) / kPW;
+    const int grid = static_cast<int>(want < sms ? want : sms);
     pack_u4_kernel<<<grid, kPW * 32, sizeof(PackSmem), static_cast<cudaStream_t>(stream)>>>(
         kc->dev, vc->dev, d_cells, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-        slot_mapping, num_tokens, static_cast<uint8_t*>(k_pages), static_cast<uint8_t*>(v_pages), num_blocks,
-        block_size, d_err);
+        slot_mapping, static_cast<int>(num_tokens), static_cast<uint8_t*>(k_pages), static_cast<uint8_t*>(v_pages),
+        static_cast<int>(capacity), block_size, bs_log2, d_err);
     return TQ_OK;
 }
 
