@@ -347,6 +347,8 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     a.ws = static_cast<float*>(workspace);
     a.qrot = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.record_bytes);
     a.d_err = d_err;
+    const char* withhold = std::getenv("TQ_TEST_WITHHOLD_COPIES");
+    a.withhold_copies = withhold && std::string(withhold) == "1";
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // Tensor-core kernel for the formats it is instantiated for (block sizes a
     // multiple of 16); the general kernel covers every other valid format.

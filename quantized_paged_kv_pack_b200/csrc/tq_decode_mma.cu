@@ -69,7 +69,6 @@ constexpr uint32_t kSpinLimit = 1u << 24;   // polls of a spinning wait
 constexpr uint32_t kWaitHintNs = 16384;     // sleep bound of one blocking wait attempt
 constexpr uint32_t kWaitRounds = 1u << 16;  // blocking wait attempts (about a second)
 constexpr float kSlack = 8.0f;                 // log2 slack of the running max
-constexpr float kSlackInv = 1.0f / 256.0f;     // 2^-kSlack, folded into P'
 
 template <int B0_, int N0_, int B1_, int N1_>
 struct Fmt {
@@ -576,15 +575,19 @@ struct WarpTiles {
                 o[q][3] *= alpha[HL - 1];
             }
         }
-        // P' = p * n_V * 2^-kSlack (weight x norm stays within fp16).
+        // P' = p 2^-kSlack n_V (weight x norm stays within fp16); the sums l_run
+        // are kept in the same 2^-kSlack units. m_ref is finite here: the first
+        // tile of an item always takes the branch above (a valid score exceeds
+        // -inf + kSlack), which sets it.
+        const float nv0m = ok0 ? nv0 : 0.0f, nv1m = ok1 ? nv1 : 0.0f;  // padding rows may hold anything
         float w[HL][2];
 #pragma unroll
         for (int e = 0; e < HL; ++e) {
-            const float mref = m_ref[e] == -INFINITY ? 0.0f : m_ref[e];
-            const float p0 = ex2(sc[e][0] - mref), p1 = ex2(sc[e][1] - mref);
+            const float mb = m_ref[e] + kSlack;
+            const float p0 = ex2(sc[e][0] - mb), p1 = ex2(sc[e][1] - mb);
             l_run[e] += p0 + p1;
-            w[e][0] = ok0 ? p0 * (nv0 * kSlackInv) : 0.0f;
-            w[e][1] = ok1 ? p1 * (nv1 * kSlackInv) : 0.0f;
+            w[e][0] = p0 * nv0m;
+            w[e][1] = p1 * nv1m;
         }
         // B fragments of P'^T: rows tokens (2c, 2c+1) and (2c+8, 2c+9), column r.
         // Tokens 2c and 2c + 8 sit in lane 8c + (r >> 1), tokens 2c + 1 and
@@ -689,6 +692,7 @@ struct WarpTiles {
             lsum += __shfl_xor_sync(kFull, lsum, 4);
             lsum += __shfl_xor_sync(kFull, lsum, 8);
             lsum += __shfl_xor_sync(kFull, lsum, 16);
+            lsum *= 256.0f;  // back from 2^-kSlack units
             const int head = NH == 8 ? 2 * c + e : c;
             if (head < rows) {
                 if (r == 0) {
@@ -828,6 +832,7 @@ __host__ __device__ constexpr uint32_t blk_slot_bytes(int bs) {
 template <class KF, class VF>
 __device__ void produce_blk(const DecodeArgs& a, BlkSmem& sm, const BlkRing& ring, int head_groups,
                             int64_t total_slots, int lane) {
+    if (a.withhold_copies) return;  // test hook: the compute warps' waits expire
     constexpr int kPer = kMaxItemTiles / 32;
     const int H = a.kc.num_heads, bs = a.block_size;
     const uint32_t k_bytes = kBlkWarps * bs * (KF::IB + 2), v_bytes = kBlkWarps * bs * (VF::IB + 2);
@@ -1055,6 +1060,7 @@ __host__ __device__ constexpr size_t smem_bytes() {
 template <class KF, class VF, int NW>
 __device__ void produce_head(const DecodeArgs& a, Smem<NW>& sm, uint32_t ring_addr, int head_groups,
                              int64_t total_slots, int lane) {
+    if (a.withhold_copies) return;  // test hook: the compute warps' waits expire
     constexpr uint32_t kKRows = 16 * KF::IB, kVRows = 16 * VF::IB;
     constexpr uint32_t kKTile = kKRows + 32, kTileBytes = kKTile + kVRows + 32;
     constexpr uint32_t kStageBytes = stage_bytes<KF, VF>();

@@ -50,6 +50,10 @@ struct DecodeArgs {
     float* ws;                     // records [B][H_kv][items_per_unit][G][2 + 128]
     float* qrot;                   // rotated, scaled queries [B][H_q][128] in K packed order
     int* d_err;
+    // Test hook (TQ_TEST_WITHHOLD_COPIES=1): the tensor-core kernels' producer
+    // issues no copies, so the compute warps' bounded waits expire and report
+    // TQ_DERR_TIMEOUT. Nothing sets it in normal use.
+    int32_t withhold_copies;
 };
 
 }  // namespace tq
