@@ -54,6 +54,10 @@ R7  The last min(W, L_b) tokens of a sequence live only in the dense bf16
     window; the first P_b = L_b - min(W, L_b) tokens are packed.
 R8  slot < 0 is a padding token and is skipped; slot >= num_blocks*block_size
     raises IndexError.
+R14 Boundary-token preservation: the first S and the last W tokens of a
+    sequence stay dense, the ones between are packed (boundary_dense_tokens).
+    Attention is a sum over keys, so the dense ones may sit in one buffer in
+    any order; the decode treats them as its window.
 """
 
 from __future__ import annotations
@@ -68,7 +72,7 @@ from scipy.special import betainc, betaincinv, gammaln
 
 __all__ = [
     "Format", "coord_density_const", "coord_cdf", "coord_tail", "cell_mass",
-    "cell_first_moment", "cell_second_moment", "lloyd_max", "codebook",
+    "cell_first_moment", "cell_second_moment", "lloyd_max", "codebook", "boundary_dense_tokens",
     "splitmix64", "hadamard_signs", "hadamard_matrix", "rotate", "unrotate",
     "permutation", "position_bits", "row_bytes", "index_bytes",
     "quantize", "encode_rows", "decode_rows", "dequantize_rows",
@@ -543,6 +547,24 @@ def decode_attention(q, k_pages, v_pages, block_tables, seq_lens, k_win, v_win, 
             for g in range(G):
                 out[ob, h * G + g] = dense_attention(q[b, h * G + g], keys, vals, scale)
     return out
+
+
+def boundary_dense_tokens(L: int, sinks: int, window: int):
+    """Token positions kept dense under boundary-token preservation (R14).
+
+    The policy keeps some boundary tokens dense next to the recent window
+    (TurboQuant "Design" page, "Format Strategy"); which tokens is not stated.
+    Reading: the first min(sinks, L) tokens and the last min(window, L - that)
+    tokens stay dense bf16; the tokens between them are packed. Returns
+    (dense positions in order, first packed position, packed count). The dense
+    positions are what the decode call's window buffer holds, in this order,
+    with window = sinks + window.
+    """
+    s = min(sinks, L)
+    w = min(window, L - s)
+    P = L - s - w
+    dense = list(range(s)) + list(range(s + P, L))
+    return dense, s, P
 
 
 def dense_attention(q, keys, vals, scale: float):

@@ -43,11 +43,19 @@ def random_kv(T, H, gen, scale_outliers=True):
 
 
 class DecodeProblem:
-    """A paged cache written by the GPU pack kernel, plus queries and windows."""
+    """A paged cache written by the GPU pack kernel, plus queries and windows.
 
-    def __init__(self, lens, H, G, kspec, vspec, window, block_size, seed, slack=1.3):
+    With ``sinks`` = S > 0 (boundary-token preservation) the first min(S, L)
+    tokens of a sequence stay dense too: the dense buffer holds them followed by
+    the last ``window`` tokens, the pages hold the tokens in between, and the
+    decode call's window is S + window.
+    """
+
+    def __init__(self, lens, H, G, kspec, vspec, window, block_size, seed, slack=1.3, sinks=0):
         self.lens = np.asarray(lens, dtype=np.int64)
         self.B, self.H, self.G, self.Hq = len(lens), H, G, H * G
+        self.sinks = sinks
+        window = window + sinks  # dense tokens per sequence (at most)
         self.window, self.bs = window, block_size
         gen = torch.Generator(device="cuda")
         gen.manual_seed(seed)
@@ -70,18 +78,22 @@ class DecodeProblem:
         Wn = max(window, 1)
         self.k_win = torch.zeros(self.B, H, Wn, D, dtype=torch.bfloat16, device="cuda")
         self.v_win = torch.zeros_like(self.k_win)
+        self.kv = []  # the original tokens, in order (for order-independent checks)
         for b in range(self.B):
             L, P = int(self.lens[b]), int(packed[b])
             k, v = random_kv(L, H, gen)
+            self.kv.append((k, v))
+            s0 = min(sinks, L)  # packed tokens are s0 .. s0 + P - 1
             if P:
                 t = np.arange(P)
                 slots = torch.as_tensor(bt[b, t // block_size].astype(np.int64) * block_size + t % block_size,
                                         device="cuda")
-                tq.pack_kv(self.kc, self.vc, k[:P].contiguous(), v[:P].contiguous(), slots, self.k_pages,
-                           self.v_pages, block_size)
+                tq.pack_kv(self.kc, self.vc, k[s0:s0 + P].contiguous(), v[s0:s0 + P].contiguous(), slots,
+                           self.k_pages, self.v_pages, block_size)
             if L > P:
-                self.k_win[b, :, :L - P] = k[P:].transpose(0, 1)
-                self.v_win[b, :, :L - P] = v[P:].transpose(0, 1)
+                dense = torch.cat((torch.arange(0, s0), torch.arange(s0 + P, L))).to(k.device)
+                self.k_win[b, :, :L - P] = k[dense].transpose(0, 1)
+                self.v_win[b, :, :L - P] = v[dense].transpose(0, 1)
         self.q = torch.randn(self.B, self.Hq, D, generator=gen, device="cuda").to(torch.bfloat16)
         self.block_tables = torch.as_tensor(bt, device="cuda")
         self.seq_lens = torch.as_tensor(self.lens.astype(np.int32), device="cuda")

@@ -231,3 +231,14 @@ def test_decode_eight_kv_heads_bad_block_id_sets_error_without_fault():
     prob.run(d_err=err)
     torch.cuda.synchronize()
     assert err.item() & tq.TQ_DERR_BLOCK
+
+
+@pytest.mark.parametrize("H,bs", [(8, 16), (2, 32)])  # the block kernel and the per-head kernel
+def test_decode_boundary_tokens_dense(H, bs):
+    """Boundary-token preservation: first S and last W tokens dense, the middle packed (one window buffer)."""
+    lens = [0, 3, 4, 11, 12, 700, 3000]
+    prob = DecodeProblem(lens, H, 4, M35, U3, window=8, block_size=bs, seed=80 + H, sinks=4)
+    assert prob.window == 12
+    rng = np.random.default_rng(H)
+    pairs = [(b, int(hq)) for b in range(prob.B) for hq in rng.choice(prob.Hq, min(prob.Hq, 6), replace=False)]
+    check(prob, pairs)

@@ -524,3 +524,59 @@ def test_attention_empty_history_is_zero():
     win = np.ones((2, 1, 3, D))
     out = O.decode_attention(q, pages, pages, np.zeros((2, 1), np.int64), [0, 1], win, win, 3, 0.1, kf, vf, 4)
     assert np.all(out[0] == 0) and np.allclose(out[1], 1.0)
+
+
+def test_boundary_dense_tokens_counts():
+    """First S and last W tokens dense, the middle packed; short sequences are all dense."""
+    for L in range(0, 30):
+        for S in (0, 1, 4):
+            for W in (0, 3, 8):
+                dense, s0, P = O.boundary_dense_tokens(L, S, W)
+                assert s0 == min(S, L) and P == max(0, L - S - W)
+                packed = list(range(s0, s0 + P))
+                assert sorted(dense + packed) == list(range(L))  # a partition of the tokens
+                assert dense[:s0] == list(range(s0))             # the sinks lead the dense buffer
+                assert all(t >= s0 + P for t in dense[s0:])      # then the most recent tokens
+
+
+def test_boundary_tokens_as_window_equal_attention_in_token_order():
+    """Sinks and recent tokens passed as one window give attention over the original token order."""
+    rng = np.random.default_rng(44)
+    d, H, G, bs = 16, 2, 2, 4
+    kf = O.Format(d, H, (4,), (d,), None, 5)
+    vf = O.Format(d, H, (3,), (d,), None, 6)
+    S, W = 3, 5
+    lens = [2, 7, 30]
+    B = len(lens)
+    nb = 16
+    kp = np.zeros((nb, H, bs * O.row_bytes(kf)), np.uint8)
+    vp = np.zeros((nb, H, bs * O.row_bytes(vf)), np.uint8)
+    kw = np.zeros((B, H, S + W, d))
+    vw = np.zeros((B, H, S + W, d))
+    tables = np.zeros((B, 8), np.int64)
+    free = list(rng.permutation(nb))
+    hist = []
+    for b, L in enumerate(lens):
+        kk = O.bf16_round(rng.standard_normal((L, H, d)) * 2).astype(np.float64)
+        vv = O.bf16_round(rng.standard_normal((L, H, d)) * 2).astype(np.float64)
+        dense, s0, P = O.boundary_dense_tokens(L, S, W)
+        nblk = -(-P // bs)
+        tables[b, :nblk] = [free.pop() for _ in range(nblk)]
+        slots = tables[b, np.arange(P) // bs] * bs + np.arange(P) % bs
+        O.pack_kv(kk[s0:s0 + P], vv[s0:s0 + P], slots, kf, vf, nb, bs, kp, vp)
+        kw[b, :, :len(dense)] = kk[dense].transpose(1, 0, 2)
+        vw[b, :, :len(dense)] = vv[dense].transpose(1, 0, 2)
+        hist.append((kk, vv, s0, P))
+    q = rng.standard_normal((B, H * G, d))
+    out = O.decode_attention(q, kp, vp, tables, lens, kw, vw, S + W, 0.3, kf, vf, bs)
+    for b, L in enumerate(lens):
+        kk, vv, s0, P = hist[b]
+        for h in range(H):
+            # keys in token order: dense sinks, the packed middle as stored, dense recent tokens
+            ki, kn = O.decode_rows(O.read_rows(kp, tables[b, np.arange(P) // bs], h, np.arange(P) % bs, kf, bs), kf)
+            vi, vn = O.decode_rows(O.read_rows(vp, tables[b, np.arange(P) // bs], h, np.arange(P) % bs, vf, bs), vf)
+            keys = np.concatenate((kk[:s0, h], O.dequantize_rows(ki, kn, kf, h), kk[s0 + P:, h]))
+            vals = np.concatenate((vv[:s0, h], O.dequantize_rows(vi, vn, vf, h), vv[s0 + P:, h]))
+            for g in range(G):
+                ref = O.dense_attention(q[b, h * G + g], keys, vals, 0.3)
+                assert np.abs(out[b, h * G + g] - ref).max() < 1e-12
