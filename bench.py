@@ -83,7 +83,8 @@ class DecodeSetup:
         self.vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed)
         lay = WL.page_layout(w)
         B = len(lay.seq_lens)
-        # one spare block per sequence takes the step's appended row
+        # one spare block per sequence, next in its block table, takes the rows the
+        # step's window eviction packs when the packed length ends on a block boundary
         self.num_blocks = lay.num_blocks + B
         self.append_block = np.arange(lay.num_blocks, lay.num_blocks + B)
         self.layout = lay
@@ -98,20 +99,30 @@ class DecodeSetup:
                 slots = torch.as_tensor(WL.slot_mapping(lay, b, t0, t1, bs), device="cuda")
                 tq.pack_kv(self.kc, self.vc, k, v, slots, self.kp, self.vp, bs)
         self.kw, self.vw = WL.windows(w, lay, device="cuda")
+        if w.window:
+            # ring order for tq_window_append: token t of the window in slot t % W
+            for b in range(B):
+                shift = int(lay.packed_lens[b]) % w.window
+                n = int(min(w.window, lay.seq_lens[b]))
+                if shift and n == w.window:
+                    self.kw[b] = torch.roll(self.kw[b], shifts=shift, dims=1)
+                    self.vw[b] = torch.roll(self.vw[b], shifts=shift, dims=1)
         self.q = WL.queries(w, device="cuda")
-        self.bt = torch.as_tensor(lay.block_tables, device="cuda")
+        nblk = -(-lay.packed_lens // bs)
+        bt = np.concatenate((lay.block_tables, np.zeros((B, 1), lay.block_tables.dtype)), axis=1)
+        bt[np.arange(B), nblk] = self.append_block
+        self.bt = torch.as_tensor(bt.astype(np.int32), device="cuda")
         self.sl = torch.as_tensor(lay.seq_lens.astype(np.int32), device="cuda")
         self.max_len = int(lay.seq_lens.max())
         self.scale = 1.0 / math.sqrt(D)
         self.ws = tq.alloc_workspace(B, w.num_q_heads, w.num_kv_heads, self.max_len, bs)
         self.out = torch.empty(B, w.num_q_heads, D, dtype=torch.float32, device="cuda")
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
-        # the step's appended vector per (sequence, head): the token leaving the window
+        # the step's new token per (sequence, head); the token it replaces in the window is packed
         g = torch.Generator(device="cuda")
         g.manual_seed(w.seed + 99)
         self.new_k = (torch.randn(B, w.num_kv_heads, D, generator=g, device="cuda") * 2).to(torch.bfloat16)
         self.new_v = (torch.randn(B, w.num_kv_heads, D, generator=g, device="cuda") * 2).to(torch.bfloat16)
-        self.new_slots = torch.as_tensor(self.append_block.astype(np.int64) * bs, device="cuda")
         torch.cuda.synchronize()
 
     # algorithmic bytes -----------------------------------------------------
@@ -127,8 +138,10 @@ class DecodeSetup:
         return len(self.layout.seq_lens) * self.w.num_q_heads * D * 4
 
     def pack_bytes(self):
+        """Window eviction with append: new K/V read, evicted K/V read, window slot written, rows written."""
         B, H = len(self.layout.seq_lens), self.w.num_kv_heads
-        return B * H * D * 2 * 2 + B * H * (self.kc.row_bytes + self.vc.row_bytes) + B * 8
+        win = 2 * (B * H * D * 2 * 2) if self.w.window else 0
+        return B * H * D * 2 * 2 + win + B * H * (self.kc.row_bytes + self.vc.row_bytes) + B * 8
 
     def step_bytes(self):
         return self.decode_split_bytes() + self.out_bytes() + self.pack_bytes()
@@ -137,9 +150,16 @@ class DecodeSetup:
         return int(self.layout.seq_lens.sum())
 
     # the step ---------------------------------------------------------------
-    def pack(self, k=None, v=None, slots=None):
-        tq.pack_kv(self.kc, self.vc, self.new_k if k is None else k, self.new_v if v is None else v,
-                   self.new_slots if slots is None else slots, self.kp, self.vp, self.w.block_size, d_err=self.err)
+    def pack(self, k=None, v=None):
+        """The step's write side: tq_window_append of one new token per sequence.
+
+        The lengths are not advanced, so every step evicts into the same packed
+        position and each timed step does the same work over the same history.
+        """
+        w = self.w
+        tq.window_append(self.kc, self.vc, self.new_k if k is None else k, self.new_v if v is None else v,
+                         self.kw if w.window else None, self.vw if w.window else None, w.window, 0, self.sl,
+                         self.bt, self.kp, self.vp, w.block_size, d_err=self.err)
 
     def decode(self, phase="all", q=None, out=None):
         w = self.w
@@ -278,18 +298,15 @@ def measure_decode_e2e(setup: DecodeSetup, steps, warmup):
     hq = setup.q.cpu().pin_memory()
     hk = setup.new_k.cpu().pin_memory()
     hv = setup.new_v.cpu().pin_memory()
-    hs = setup.new_slots.cpu().pin_memory()
     hout = torch.empty(B, Hq, D, dtype=torch.float32).pin_memory()
-    dq, dk, dv, ds = torch.empty_like(setup.q), torch.empty_like(setup.new_k), torch.empty_like(setup.new_v), \
-        torch.empty_like(setup.new_slots)
+    dq, dk, dv = torch.empty_like(setup.q), torch.empty_like(setup.new_k), torch.empty_like(setup.new_v)
     dout = torch.empty_like(setup.out)
 
     def step():
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
-        ds.copy_(hs, non_blocking=True)
-        setup.pack(dk, dv, ds)
+        setup.pack(dk, dv)
         setup.decode("all", q=dq, out=dout)
         hout.copy_(dout, non_blocking=True)
 
@@ -297,7 +314,7 @@ def measure_decode_e2e(setup: DecodeSetup, steps, warmup):
         step()
     torch.cuda.synchronize()
     total, _ = time_steps([step], steps, torch.cuda.current_stream())
-    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + hs.numel() * 8
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
     d2h = hout.numel() * 4
     return total / steps, h2d, d2h
 
@@ -537,7 +554,7 @@ def run_ours(args):
                    "parallelism": f"{world} independent replicas (no collective)",
                    "l2": f"no flush: {split_bytes / 1e9:.2f} GB of pages read per step, L2 is 126 MB"},
         "kv_tokens_per_s": world * setup.kv_tokens() / (step_ms * 1e-3),
-        "step_breakdown_ms": {"pack": parts[0], "decode_partials": parts[1], "decode_combine": parts[2]},
+        "step_breakdown_ms": {"window_append": parts[0], "decode_partials": parts[1], "decode_combine": parts[2]},
         "algorithmic_bytes_per_step": step_bytes,
         "roofline": {"bound": "hbm", "kernel": "decode_partials", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
@@ -545,7 +562,7 @@ def run_ours(args):
                      "traffic": stored_traffic(w.name, "tq_decode_mma.cu")},
         "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 4 * args.steps,  # window append, query rotation, decode partials, combine
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline:

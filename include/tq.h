@@ -51,7 +51,7 @@ typedef enum {
 
 /* Bits of the device error word. */
 #define TQ_DERR_SLOT 1      /* tq_pack_kv: slot >= num_blocks * block_size (row skipped) */
-#define TQ_DERR_BLOCK 2     /* tq_decode_paged: block table entry outside [0, num_blocks) */
+#define TQ_DERR_BLOCK 2     /* tq_decode_paged, tq_window_append: block table entry outside [0, num_blocks) */
 #define TQ_DERR_TIMEOUT 4   /* a kernel's bounded wait expired; its results are invalid */
 #define TQ_DERR_LAUNCH 8    /* a kernel could not lay out its shared memory; its results are invalid */
 
@@ -142,6 +142,41 @@ int32_t tq_codec_row_bytes(const tq_codec* codec);
 tq_status tq_pack_kv(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
                      const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
                      int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream);
+
+/*
+ * tq_window_append - window eviction with append, the write side of a decode
+ * step. [Design] "Data Ownership": CompressedKVCache owns sequence-level
+ * compressed blocks and recent windows; [Design] "Format Strategy": recent
+ * dense window, boundary tokens kept dense; "Serving Route Design": packed
+ * rows are written into persistent pages through block tables.
+ *
+ * Appends one token per sequence. With L = seq_lens[b] tokens before the
+ * call, the dense buffer of (b, head) has sinks + window slots: the first
+ * min(sinks, L) tokens in slots 0 .. sinks-1, and token t >= sinks in slot
+ * sinks + (t - sinks) % window while it is among the last `window` tokens.
+ * The new token L goes to slot L when L < sinks, else to its ring slot; when
+ * that slot still holds token L - window, that token is first packed (as
+ * tq_pack_kv would) at packed position L - sinks - window of the sequence:
+ * block block_tables[b][p / block_size], offset p % block_size. With
+ * window = 0 the new token itself is packed, at position L - sinks. The
+ * buffers then match what tq_decode_paged reads with window' = sinks + window
+ * and seq_lens[b] = L + 1; the caller advances seq_lens.
+ *
+ * k_new, v_new   device bf16 [batch][num_kv_heads][head_dim]
+ * k_win, v_win   device bf16 [batch][num_kv_heads][sinks + window][head_dim],
+ *                updated in place (may be NULL when sinks + window == 0)
+ * seq_lens       device int32 [batch], lengths before the append (read only)
+ * block_tables   device int32 [batch][max_blocks_per_seq]
+ * k_pages, v_pages as for tq_pack_kv.
+ * Errors: TQ_ERR_VALUE for inconsistent arguments. A packed position past the
+ * block table, or a block id outside [0, num_blocks), sets TQ_DERR_BLOCK and
+ * that row is not written (the new token still enters the dense buffer).
+ * This library's own extension: the pages name the ownership, not the call.
+ */
+tq_status tq_window_append(const tq_codec* kc, const tq_codec* vc, const void* k_new, const void* v_new,
+                           void* k_win, void* v_win, int32_t window, int32_t sinks, const int32_t* seq_lens,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq, void* k_pages, void* v_pages,
+                           int64_t num_blocks, int32_t block_size, int32_t batch, int32_t* d_err, void* stream);
 
 /*
  * Workspace bytes that tq_decode_paged needs for these sizes; bounded by the

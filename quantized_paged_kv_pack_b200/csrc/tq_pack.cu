@@ -68,6 +68,72 @@ __device__ __forceinline__ unsigned short norm_fp16_bits(const float (&x)[4], fl
     return hb;
 }
 
+// One warp quantizes the vector x (lane l holds elements 4l .. 4l+3) of KV
+// head h and writes its row at `offset` of the sub-page `sub` (block_size
+// rows). idx_buf: 128 bytes of shared scratch owned by the warp.
+__device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8_t* sub, int64_t offset,
+                            int block_size, uint8_t* idx_buf, int lane) {
+    float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
+    float n32 = sqrtf(ss);
+    const unsigned short n16 = norm_fp16_bits(x, ss, n32);
+
+    float z[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) z[i] = x[i] * c.sign[4 * lane + i];
+    {
+        float a = z[0] + z[1], b = z[0] - z[1], cc = z[2] + z[3], d = z[2] - z[3];
+        z[0] = a + cc;
+        z[2] = a - cc;
+        z[1] = b + d;
+        z[3] = b - d;
+    }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float p = __shfl_xor_sync(kFull, z[i], m);
+            z[i] = (lane & m) ? (p - z[i]) : (z[i] + p);
+        }
+    }
+    const float inv = n32 > 0.0f ? 1.0f / (n32 * 11.313708498984761f) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int j = 4 * lane + i;
+        const int p = c.pos[h * kHeadDim + j];
+        const int g = (c.n_groups == 2 && p >= c.pos0[1]) ? 1 : 0;
+        const float u = z[i] * inv;
+        const int levels = 1 << c.bits[g];
+        int idx = 0;
+        for (int q = 0; q < levels - 1; ++q) idx += (c.bound[g * 16 + q] < u) ? 1 : 0;
+        idx_buf[p] = static_cast<uint8_t>(idx);
+    }
+    __syncwarp();
+    const int half_words = c.index_bytes / 2;
+    unsigned word = 0;
+    if (lane < half_words) {
+        for (int i = 0; i < 16; ++i) {
+            const int B = 16 * lane + i;
+            const int g = (c.n_groups == 2 && B >= 8 * c.byte_off[1]) ? 1 : 0;
+            const int lb = B - 8 * c.byte_off[g];
+            const int b = c.bits[g];
+            const int q = lb / b, r = lb - q * b;
+            word |= ((idx_buf[c.pos0[g] + q] >> r) & 1u) << i;
+        }
+    }
+    uint16_t* dst = reinterpret_cast<uint16_t*>(sub + offset * c.index_bytes);
+    if (lane < half_words) dst[lane] = static_cast<uint16_t>(word);
+    if (lane == 0) *reinterpret_cast<uint16_t*>(sub + block_size * c.index_bytes + 2 * offset) = n16;
+    __syncwarp();
+}
+
+__device__ __forceinline__ void load_bf16x4(const __nv_bfloat16* src, float (&x)[4]) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(src);
+    x[0] = __uint_as_float(raw.x << 16);
+    x[1] = __uint_as_float(raw.x & 0xffff0000u);
+    x[2] = __uint_as_float(raw.y << 16);
+    x[3] = __uint_as_float(raw.y & 0xffff0000u);
+}
+
 __global__ void __launch_bounds__(kPackWarps * 32)
 pack_rows_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__ k,
                  const __nv_bfloat16* __restrict__ v, const int64_t* __restrict__ slots, int64_t num_tokens,
@@ -91,67 +157,70 @@ pack_rows_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__ k,
             continue;
         }
         const DevCodec& c = which ? vc : kc;
-        const __nv_bfloat16* src = (which ? v : k) + th * kHeadDim + 4 * lane;
-        uint2 raw = *reinterpret_cast<const uint2*>(src);
         float x[4];
-        x[0] = __uint_as_float(raw.x << 16);
-        x[1] = __uint_as_float(raw.x & 0xffff0000u);
-        x[2] = __uint_as_float(raw.y << 16);
-        x[3] = __uint_as_float(raw.y & 0xffff0000u);
-
-        float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
-        float n32 = sqrtf(ss);
-        unsigned short n16 = norm_fp16_bits(x, ss, n32);
-
-        float z[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) z[i] = x[i] * c.sign[4 * lane + i];
-        {
-            float a = z[0] + z[1], b = z[0] - z[1], cc = z[2] + z[3], d = z[2] - z[3];
-            z[0] = a + cc;
-            z[2] = a - cc;
-            z[1] = b + d;
-            z[3] = b - d;
-        }
-#pragma unroll
-        for (int m = 1; m < 32; m <<= 1) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float p = __shfl_xor_sync(kFull, z[i], m);
-                z[i] = (lane & m) ? (p - z[i]) : (z[i] + p);
-            }
-        }
-        const float inv = n32 > 0.0f ? 1.0f / (n32 * 11.313708498984761f) : 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = 4 * lane + i;
-            const int p = c.pos[h * kHeadDim + j];
-            const int g = (c.n_groups == 2 && p >= c.pos0[1]) ? 1 : 0;
-            const float u = z[i] * inv;
-            const int levels = 1 << c.bits[g];
-            int idx = 0;
-            for (int q = 0; q < levels - 1; ++q) idx += (c.bound[g * 16 + q] < u) ? 1 : 0;
-            idx_buf[warp][p] = static_cast<uint8_t>(idx);
-        }
-        __syncwarp();
-        const int half_words = c.index_bytes / 2;
-        unsigned word = 0;
-        if (lane < half_words) {
-            for (int i = 0; i < 16; ++i) {
-                const int B = 16 * lane + i;
-                const int g = (c.n_groups == 2 && B >= 8 * c.byte_off[1]) ? 1 : 0;
-                const int lb = B - 8 * c.byte_off[g];
-                const int b = c.bits[g];
-                const int q = lb / b, r = lb - q * b;
-                word |= ((idx_buf[warp][c.pos0[g] + q] >> r) & 1u) << i;
-            }
-        }
+        load_bf16x4((which ? v : k) + th * kHeadDim + 4 * lane, x);
         const int64_t blk = slot / block_size, off = slot - blk * block_size;
         uint8_t* sub = (which ? v_pages : k_pages) + (blk * H + h) * block_size * c.row_bytes;
-        uint16_t* dst = reinterpret_cast<uint16_t*>(sub + off * c.index_bytes);
-        if (lane < half_words) dst[lane] = static_cast<uint16_t>(word);
-        if (lane == 0) *reinterpret_cast<uint16_t*>(sub + block_size * c.index_bytes + 2 * off) = n16;
-        __syncwarp();
+        pack_vector(c, x, h, sub, off, block_size, idx_buf[warp], lane);
+    }
+}
+
+// Window eviction with append. One warp per (sequence, KV head, K or V). With
+// L = seq_lens[b] tokens before the append, the dense buffer holds the first
+// min(S, L) tokens in slots 0 .. S-1 and the recent ones in a ring: token
+// t >= S in slot S + (t - S) % W. The new token L takes slot L (L < S) or its
+// ring slot; when the ring is full, the token it replaces, L - W, is packed
+// first, at packed position L - S - W of the sequence's block table. With
+// W = 0 the new token itself is packed (at position L - S).
+__global__ void __launch_bounds__(kPackWarps * 32)
+window_append_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__ k_new,
+                     const __nv_bfloat16* __restrict__ v_new, __nv_bfloat16* __restrict__ k_win,
+                     __nv_bfloat16* __restrict__ v_win, int window, int sinks, const int32_t* __restrict__ seq_lens,
+                     const int32_t* __restrict__ block_tables, int max_blocks, uint8_t* __restrict__ k_pages,
+                     uint8_t* __restrict__ v_pages, int64_t num_blocks, int block_size, int batch,
+                     int* __restrict__ d_err) {
+    __shared__ uint8_t idx_buf[kPackWarps][kHeadDim];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = kc.num_heads;
+    const int64_t n_vec = static_cast<int64_t>(batch) * H * 2;
+    const int dense = sinks + window;  // slots per (sequence, head) in the dense buffer
+    for (int64_t vec = static_cast<int64_t>(blockIdx.x) * kPackWarps + warp; vec < n_vec;
+         vec += static_cast<int64_t>(gridDim.x) * kPackWarps) {
+        const int which = static_cast<int>(vec & 1);
+        const int64_t bh = vec >> 1;
+        const int b = static_cast<int>(bh / H), h = static_cast<int>(bh - static_cast<int64_t>(b) * H);
+        const DevCodec& c = which ? vc : kc;
+        const int L = max(__ldg(seq_lens + b), 0);
+        const __nv_bfloat16* src_new = (which ? v_new : k_new) + bh * kHeadDim + 4 * lane;
+        __nv_bfloat16* wbuf = (which ? v_win : k_win) + bh * static_cast<int64_t>(dense) * kHeadDim;
+        int slot_w = -1;      // dense slot the new token goes to (-1: none)
+        int64_t packed = -1;  // packed position of the vector to pack (-1: none)
+        bool pack_new = false;
+        if (L < sinks) {
+            slot_w = L;
+        } else if (window == 0) {
+            packed = L - sinks;
+            pack_new = true;
+        } else {
+            const int r = L - sinks;
+            slot_w = sinks + r % window;
+            if (r >= window) packed = r - window;
+        }
+        if (packed >= 0) {
+            const int64_t bi = packed / block_size, off = packed - bi * block_size;
+            const int blk = bi < max_blocks ? __ldg(block_tables + static_cast<int64_t>(b) * max_blocks + bi) : -1;
+            if (blk < 0 || blk >= num_blocks) {
+                if (lane == 0 && d_err) atomicOr(d_err, TQ_DERR_BLOCK);
+            } else {
+                float x[4];
+                load_bf16x4(pack_new ? src_new : wbuf + static_cast<int64_t>(slot_w) * kHeadDim + 4 * lane, x);
+                uint8_t* sub = (which ? v_pages : k_pages) + (static_cast<int64_t>(blk) * H + h) * block_size * c.row_bytes;
+                pack_vector(c, x, h, sub, off, block_size, idx_buf[warp], lane);  // reads x before the slot is reused
+            }
+        }
+        if (slot_w >= 0)
+            *reinterpret_cast<uint2*>(wbuf + static_cast<int64_t>(slot_w) * kHeadDim + 4 * lane) =
+                *reinterpret_cast<const uint2*>(src_new);
     }
 }
 
@@ -194,6 +263,37 @@ extern "C" tq_status tq_pack_kv(const tq_codec* kc, const tq_codec* vc, const vo
     return finish_pack(s, d_err);
 }
 
+extern "C" tq_status tq_window_append(const tq_codec* kc, const tq_codec* vc, const void* k_new, const void* v_new,
+                                      void* k_win, void* v_win, int32_t window, int32_t sinks,
+                                      const int32_t* seq_lens, const int32_t* block_tables,
+                                      int32_t max_blocks_per_seq, void* k_pages, void* v_pages, int64_t num_blocks,
+                                      int32_t block_size, int32_t batch, int32_t* d_err, void* stream) {
+    clear_error();
+    if (!kc || !vc) return fail(TQ_ERR_VALUE, "null codec");
+    if (kc->desc.num_kv_heads != vc->desc.num_kv_heads || kc->desc.head_dim != vc->desc.head_dim)
+        return fail(TQ_ERR_VALUE, "K and V codecs disagree on num_kv_heads or head_dim");
+    if (batch < 0 || window < 0 || sinks < 0 || block_size < 1 || num_blocks < 0 || max_blocks_per_seq < 0)
+        return fail(TQ_ERR_VALUE, "negative size");
+    if (batch == 0) return TQ_OK;
+    if (!k_new || !v_new || !seq_lens || !k_pages || !v_pages || (max_blocks_per_seq > 0 && !block_tables))
+        return fail(TQ_ERR_VALUE, "null buffer");
+    if (window + sinks > 0 && (!k_win || !v_win)) return fail(TQ_ERR_VALUE, "null dense buffer");
+    if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new) |
+         reinterpret_cast<uintptr_t>(k_win) | reinterpret_cast<uintptr_t>(v_win)) & 7)
+        return fail(TQ_ERR_VALUE, "k_new, v_new and the dense buffers must be 8-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 1)
+        return fail(TQ_ERR_VALUE, "page pools must be 2-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t n_vec = static_cast<int64_t>(batch) * kc->desc.num_kv_heads * 2;
+    const int64_t blocks = std::min<int64_t>((n_vec + kPackWarps - 1) / kPackWarps, 148 * 32);
+    window_append_kernel<<<static_cast<unsigned>(blocks), kPackWarps * 32, 0, s>>>(
+        kc->dev, vc->dev, static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
+        static_cast<__nv_bfloat16*>(k_win), static_cast<__nv_bfloat16*>(v_win), window, sinks, seq_lens,
+        block_tables, max_blocks_per_seq, static_cast<uint8_t*>(k_pages), static_cast<uint8_t*>(v_pages),
+        num_blocks, block_size, batch, d_err);
+    return finish_pack(s, d_err);
+}
+
 namespace tq {
 tq_status finish_pack(cudaStream_t s, int32_t* d_err) {
     cudaError_t e = cudaGetLastError();
@@ -206,6 +306,7 @@ tq_status finish_pack(cudaStream_t s, int32_t* d_err) {
             if (cudaMemcpy(&h, d_err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
                 return fail(TQ_ERR_CUDA, "reading the device error word failed");
             if (h & TQ_DERR_SLOT) return fail(TQ_ERR_INDEX, "slot mapping points outside the allocated pages");
+            if (h & TQ_DERR_BLOCK) return fail(TQ_ERR_INDEX, "block table entry outside the allocated pages");
         }
     }
     return TQ_OK;

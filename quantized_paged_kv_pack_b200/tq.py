@@ -78,10 +78,13 @@ def lib():
         L.tq_decode_partials.argtypes = dec + [_VP, _SZ, _VP, _VP]
         L.tq_decode_combine.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _SZ, _VP]
         L.tq_decode_paged_static.argtypes = dec + [_VP, _VP, _VP]
+        L.tq_window_append.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP, _I64,
+                                       _I32, _I32, _VP, _VP]
         L.tq_byte_ledger.argtypes = [P(_FormatDesc), P(_FormatDesc), _I32, _VP, _I32, _I32, _I32, _I64, _I32,
                                      P(_Ledger)]
         for name in ("tq_codec_host_tables", "tq_make_codec", "tq_pack_kv", "tq_decode_paged",
-                     "tq_decode_partials", "tq_decode_combine", "tq_byte_ledger", "tq_decode_paged_static"):
+                     "tq_decode_partials", "tq_decode_combine", "tq_byte_ledger", "tq_decode_paged_static",
+                     "tq_window_append"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -247,6 +250,38 @@ def pack_kv(kc: Codec, vc: Codec, k: torch.Tensor, v: torch.Tensor, slot_mapping
         _need(d_err, torch.int32, (1,), "d_err")
     _check(lib().tq_pack_kv(kc.handle, vc.handle, _ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_pages),
                             _ptr(v_pages), nb, bs, _ptr(d_err), _stream(stream)))
+
+
+def window_append(kc: Codec, vc: Codec, k_new: torch.Tensor, v_new: torch.Tensor, k_win: Optional[torch.Tensor],
+                  v_win: Optional[torch.Tensor], window: int, sinks: int, seq_lens: torch.Tensor,
+                  block_tables: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_size: int,
+                  d_err: Optional[torch.Tensor] = None, stream=None):
+    """Append one token per sequence, evicting the oldest window token into the pages (tq_window_append).
+
+    ``k_win``/``v_win`` are [B][H][sinks + window][d] dense buffers (updated in
+    place); ``seq_lens`` holds the lengths before the append and is not changed.
+    """
+    B = k_new.shape[0] if k_new.dim() == 3 else -1
+    H = kc.num_kv_heads
+    _need(k_new, torch.bfloat16, (B, H, kc.head_dim), "k_new")
+    _need(v_new, torch.bfloat16, (B, H, kc.head_dim), "v_new")
+    dense = int(window) + int(sinks)
+    if dense > 0:
+        if k_win is None or v_win is None:
+            raise ValueError("sinks + window > 0 needs the dense buffers")
+        _need(k_win, torch.bfloat16, (B, H, dense, kc.head_dim), "k_win")
+        _need(v_win, torch.bfloat16, (B, H, dense, kc.head_dim), "v_win")
+    _need(seq_lens, torch.int32, (B,), "seq_lens")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be [batch][max_blocks_per_seq]")
+    _need(block_tables, torch.int32, (B, block_tables.shape[1]), "block_tables")
+    nb = _pools(kc, vc, k_pages, v_pages, block_size)
+    if d_err is not None:
+        _need(d_err, torch.int32, (1,), "d_err")
+    _check(lib().tq_window_append(kc.handle, vc.handle, _ptr(k_new), _ptr(v_new), _ptr(k_win), _ptr(v_win),
+                                  int(window), int(sinks), _ptr(seq_lens), _ptr(block_tables),
+                                  int(block_tables.shape[1]), _ptr(k_pages), _ptr(v_pages), nb, int(block_size), B,
+                                  _ptr(d_err), _stream(stream)))
 
 
 def decode_workspace_bytes(batch: int, num_q_heads: int, num_kv_heads: int, max_seq_len: int, block_size: int) -> int:
