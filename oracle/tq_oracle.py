@@ -54,6 +54,17 @@ R7  The last min(W, L_b) tokens of a sequence live only in the dense bf16
     window; the first P_b = L_b - min(W, L_b) tokens are packed.
 R8  slot < 0 is a padding token and is skipped; slot >= num_blocks*block_size
     raises IndexError.
+R16 QJL residual stage (TurboQuant "Design" page, "Recipe Strategy": row
+    [MSE indices][QJL signs][vector norm][residual norm]). With qjl set, the
+    MSE part is the format's groups as above; r = u - c[idx] is the residual
+    of the unit rotated vector (rotated coordinate order), g = ||r|| is
+    stored as fp16 after the norm, and bit i of the d sign bits (LSB-first)
+    is 1 when (S r)_i >= 0. S is d x d with iid N(0, 1) entries held in fp32
+    (qjl_matrix). The key a row stands for is the unbiased inner-product
+    estimate n R^T (c[idx] + sqrt(pi/2) / d * g * S^T z), z = 2 bits - 1:
+    E over S of its product with q equals q . x when g is exact. In a
+    sub-page the sign bytes follow the index bytes of each row and the norm
+    area holds (norm, residual norm) per row.
 R14 Boundary-token preservation: the first S and the last W tokens of a
     sequence stay dense, the ones between are packed (boundary_dense_tokens).
     Attention is a sum over keys, so the dense ones may sit in one buffer in
@@ -73,6 +84,7 @@ from scipy.special import betainc, betaincinv, gammaln
 __all__ = [
     "Format", "coord_density_const", "coord_cdf", "coord_tail", "cell_mass",
     "cell_first_moment", "cell_second_moment", "lloyd_max", "codebook", "boundary_dense_tokens",
+    "qjl_matrix", "quantize_qjl", "norm_bytes", "mse_index_bytes",
     "splitmix64", "hadamard_signs", "hadamard_matrix", "rotate", "unrotate",
     "permutation", "position_bits", "row_bytes", "index_bytes",
     "quantize", "encode_rows", "decode_rows", "dequantize_rows",
@@ -100,6 +112,7 @@ class Format:
     group_size: tuple
     high_coords: Optional[np.ndarray] = field(default=None, compare=False)
     seed: int = 0
+    qjl: bool = False
 
     def __post_init__(self):
         d = self.head_dim
@@ -324,7 +337,8 @@ def position_bits(fmt: Format) -> np.ndarray:
     return np.concatenate([np.full(n, b) for b, n in zip(fmt.group_bits, fmt.group_size)])
 
 
-def index_bytes(fmt: Format) -> int:
+def mse_index_bytes(fmt: Format) -> int:
+    """Bytes of the groups' index bitstreams."""
     total = 0
     for b, n in zip(fmt.group_bits, fmt.group_size):
         if (b * n) % 8:
@@ -333,9 +347,19 @@ def index_bytes(fmt: Format) -> int:
     return total
 
 
+def index_bytes(fmt: Format) -> int:
+    """Bytes of a row before its norms: the index bitstreams, then the QJL signs (R16)."""
+    return mse_index_bytes(fmt) + (fmt.head_dim // 8 if fmt.qjl else 0)
+
+
+def norm_bytes(fmt: Format) -> int:
+    """fp16 norm, then the fp16 residual norm with QJL (R16)."""
+    return 4 if fmt.qjl else 2
+
+
 def row_bytes(fmt: Format) -> int:
-    """Index bytes of every group plus the 2-byte fp16 norm."""
-    return index_bytes(fmt) + 2
+    """Index bytes (and QJL signs) of a row plus its fp16 norm(s)."""
+    return index_bytes(fmt) + norm_bytes(fmt)
 
 
 def quantize(x, fmt: Format, head: int):
@@ -362,6 +386,49 @@ def quantize(x, fmt: Format, head: int):
     return idx, n16, u
 
 
+QJL_SEED_XOR = 0x51534A4C00000001  # "QSJL": the S stream is independent of the sign stream
+
+
+@functools.lru_cache(maxsize=None)
+def _qjl_matrix_cached(seed: int, d: int) -> np.ndarray:
+    x = splitmix64(seed ^ QJL_SEED_XOR, 2 * d * d)
+    a = np.array(x[0::2], dtype=np.uint64)
+    b = np.array(x[1::2], dtype=np.uint64)
+    u1 = ((a >> np.uint64(11)).astype(np.float64) + 1.0) * 2.0 ** -53  # (0, 1]
+    u2 = (b >> np.uint64(11)).astype(np.float64) * 2.0 ** -53          # [0, 1)
+    z = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)         # Box-Muller, cosine branch
+    return z.astype(np.float32).astype(np.float64).reshape(d, d)
+
+
+def qjl_matrix(fmt: Format) -> np.ndarray:
+    """S of R16: S[i][j] = N(0, 1) drawn from SplitMix64(seed ^ QJL_SEED_XOR) outputs 2k, 2k+1
+    (k = i d + j) by the Box-Muller cosine branch, then rounded to fp32."""
+    return _qjl_matrix_cached(int(fmt.seed), int(fmt.head_dim)).copy()
+
+
+def quantize_qjl(x, fmt: Format, head: int):
+    """quantize() plus the QJL stage (R16): returns (idx, n16, u, signs, g16).
+
+    signs[..., i] in {0, 1} (1: (S r)_i >= 0), g16 = fp16(||r||), r the
+    residual of u in rotated coordinate order.
+    """
+    idx, n16, u = quantize(x, fmt, head)
+    d = fmt.head_dim
+    c_hat = np.empty(idx.shape, dtype=np.float64)
+    start = 0
+    for b, size in zip(fmt.group_bits, fmt.group_size):
+        c, _ = codebook(b, d)
+        c_hat[..., start:start + size] = c[idx[..., start:start + size]]
+        start += size
+    perm = permutation(fmt, head)
+    r = np.empty(u.shape, dtype=np.float64)
+    r[..., perm] = u - c_hat                       # back to rotated coordinate order
+    g16 = fp16_round(np.sqrt(np.sum(r * r, axis=-1)))
+    proj = r @ qjl_matrix(fmt).T                    # (S r)_i
+    signs = (proj >= 0).astype(np.int64)
+    return idx, n16, u, signs, g16
+
+
 def boundary_margin(u, fmt: Format):
     """Per position: |u - nearest boundary| / max(|boundary|, 1/sqrt(d)).
 
@@ -385,8 +452,8 @@ def _fp16_bytes(n16):
     return np.asarray(n16, dtype=np.float64).astype(np.float16).view(np.uint8).reshape(np.shape(n16) + (2,))
 
 
-def encode_rows(idx, n16, fmt: Format) -> np.ndarray:
-    """Pack indices (packed order) and fp16 norms into rows of ``row_bytes`` (R6)."""
+def encode_rows(idx, n16, fmt: Format, signs=None, g16=None) -> np.ndarray:
+    """Pack indices (packed order) and fp16 norms into rows of ``row_bytes`` (R6; R16 with QJL)."""
     idx = np.asarray(idx, dtype=np.int64)
     lead = idx.shape[:-1]
     parts = []
@@ -400,12 +467,19 @@ def encode_rows(idx, n16, fmt: Format) -> np.ndarray:
         bits = (seg[..., :, None] >> np.arange(b)) & 1  # LSB-first within each index
         parts.append(np.packbits(bits.reshape(lead + (size * b,)).astype(np.uint8), axis=-1, bitorder="little"))
         start += size
+    if fmt.qjl:
+        if signs is None or g16 is None:
+            raise ValueError("a QJL format needs the signs and the residual norm")
+        parts.append(np.packbits(np.asarray(signs, dtype=np.uint8), axis=-1, bitorder="little"))
     parts.append(_fp16_bytes(n16))
+    if fmt.qjl:
+        parts.append(_fp16_bytes(g16))
     return np.concatenate(parts, axis=-1)
 
 
 def decode_rows(rows, fmt: Format):
-    """Inverse of ``encode_rows``: (idx in packed order, n16 as fp64)."""
+    """Inverse of ``encode_rows``: (idx in packed order, n16 as fp64), and with QJL
+    also (signs in {0, 1}, g16 as fp64)."""
     rows = np.asarray(rows, dtype=np.uint8)
     lead = rows.shape[:-1]
     if rows.shape[-1] != row_bytes(fmt):
@@ -417,12 +491,23 @@ def decode_rows(rows, fmt: Format):
         bits = np.unpackbits(rows[..., off:off + nbytes], axis=-1, bitorder="little").reshape(lead + (size, b))
         idx.append((bits.astype(np.int64) << np.arange(b)).sum(axis=-1))
         off += nbytes
+    if fmt.qjl:
+        nb = fmt.head_dim // 8
+        signs = np.unpackbits(rows[..., off:off + nb], axis=-1, bitorder="little").astype(np.int64)
+        off += nb
     n16 = rows[..., off:off + 2].copy().view(np.float16).reshape(lead).astype(np.float64)
+    if fmt.qjl:
+        g16 = rows[..., off + 2:off + 4].copy().view(np.float16).reshape(lead).astype(np.float64)
+        return np.concatenate(idx, axis=-1), n16, signs, g16
     return np.concatenate(idx, axis=-1), n16
 
 
-def dequantize_rows(idx, n16, fmt: Format, head: int):
-    """x_hat = n16 * s * (H c_hat) / sqrt(d), c_hat placed back at the rotated coordinates."""
+def dequantize_rows(idx, n16, fmt: Format, head: int, signs=None, g16=None):
+    """x_hat = n16 * s * (H c_hat) / sqrt(d), c_hat placed back at the rotated coordinates.
+
+    With QJL (R16) c_hat gains sqrt(pi/2) / d * g16 * S^T z: the vector whose
+    product with any q is the unbiased estimate of q . x.
+    """
     idx = np.asarray(idx, dtype=np.int64)
     d = fmt.head_dim
     vals = np.empty(idx.shape, dtype=np.float64)
@@ -433,6 +518,12 @@ def dequantize_rows(idx, n16, fmt: Format, head: int):
         start += size
     rot = np.empty_like(vals)
     rot[..., permutation(fmt, head)] = vals
+    if fmt.qjl:
+        if signs is None or g16 is None:
+            raise ValueError("a QJL format needs the signs and the residual norm")
+        z = 2.0 * np.asarray(signs, dtype=np.float64) - 1.0
+        rot = rot + (math.sqrt(math.pi / 2.0) / d) * np.asarray(g16, dtype=np.float64)[..., None] * (
+            z @ qjl_matrix(fmt))
     return np.asarray(n16, dtype=np.float64)[..., None] * unrotate(rot, hadamard_signs(fmt.seed, d))
 
 
@@ -446,23 +537,23 @@ def subpage_bytes(fmt: Format, block_size: int) -> int:
 
 def write_rows(pages, blocks, head: int, offsets, rows, fmt: Format, block_size: int):
     """Store logical rows at (block, offset) of one head's sub-pages (R6 layout)."""
-    ib = index_bytes(fmt)
+    ib, nb = index_bytes(fmt), norm_bytes(fmt)
     blocks = np.asarray(blocks, dtype=np.int64)
     offsets = np.asarray(offsets, dtype=np.int64)
     rows = np.asarray(rows, dtype=np.uint8)
     cols = offsets[:, None] * ib + np.arange(ib)[None, :]
     pages[blocks[:, None], head, cols] = rows[:, :ib]
-    ncols = block_size * ib + 2 * offsets[:, None] + np.arange(2)[None, :]
+    ncols = block_size * ib + nb * offsets[:, None] + np.arange(nb)[None, :]
     pages[blocks[:, None], head, ncols] = rows[:, ib:]
 
 
 def read_rows(pages, blocks, head: int, offsets, fmt: Format, block_size: int):
     """Logical rows [n][row_bytes] at (block, offset) of one head's sub-pages."""
-    ib = index_bytes(fmt)
+    ib, nb = index_bytes(fmt), norm_bytes(fmt)
     blocks = np.asarray(blocks, dtype=np.int64)
     offsets = np.asarray(offsets, dtype=np.int64)
     cols = offsets[:, None] * ib + np.arange(ib)[None, :]
-    ncols = block_size * ib + 2 * offsets[:, None] + np.arange(2)[None, :]
+    ncols = block_size * ib + nb * offsets[:, None] + np.arange(nb)[None, :]
     return np.concatenate((pages[blocks[:, None], head, cols], pages[blocks[:, None], head, ncols]), axis=-1)
 
 
@@ -492,8 +583,13 @@ def pack_kv(k, v, slot_mapping, kfmt: Format, vfmt: Format, num_blocks: int, blo
     off = slots[live] % block_size
     for h in range(H):
         for src, fmt, pages in ((k, kfmt, k_pages), (v, vfmt, v_pages)):
-            idx, n16, _ = quantize(src[live, h, :], fmt, h)
-            write_rows(pages, blk, h, off, encode_rows(idx, n16, fmt), fmt, block_size)
+            if fmt.qjl:
+                idx, n16, _, signs, g16 = quantize_qjl(src[live, h, :], fmt, h)
+                rows = encode_rows(idx, n16, fmt, signs, g16)
+            else:
+                idx, n16, _ = quantize(src[live, h, :], fmt, h)
+                rows = encode_rows(idx, n16, fmt)
+            write_rows(pages, blk, h, off, rows, fmt, block_size)
     return k_pages, v_pages
 
 
@@ -535,10 +631,10 @@ def decode_attention(q, k_pages, v_pages, block_tables, seq_lens, k_win, v_win, 
         n_win = min(window, L)
         P = L - n_win
         for h in range(H):
-            ki, kn = decode_rows(_gather_rows(k_pages, block_tables[b], P, h, block_size, kfmt), kfmt)
-            vi, vn = decode_rows(_gather_rows(v_pages, block_tables[b], P, h, block_size, vfmt), vfmt)
-            keys = dequantize_rows(ki, kn, kfmt, h)
-            vals = dequantize_rows(vi, vn, vfmt, h)
+            kd = decode_rows(_gather_rows(k_pages, block_tables[b], P, h, block_size, kfmt), kfmt)
+            vd = decode_rows(_gather_rows(v_pages, block_tables[b], P, h, block_size, vfmt), vfmt)
+            keys = dequantize_rows(kd[0], kd[1], kfmt, h, *kd[2:])  # (signs, g16) follow with QJL
+            vals = dequantize_rows(vd[0], vd[1], vfmt, h, *vd[2:])
             if n_win:
                 keys = np.concatenate((keys, np.asarray(k_win[b, h, :n_win], dtype=np.float64)))
                 vals = np.concatenate((vals, np.asarray(v_win[b, h, :n_win], dtype=np.float64)))
@@ -606,11 +702,13 @@ def byte_ledger(kfmt: Format, vfmt: Format, seq_lens: Sequence[int], window: int
                 num_blocks: int, workspace_bytes: int = 0) -> Ledger:
     """Plain byte arithmetic for one layer's cache.
 
-    dense: bf16 K and V of every token. index: packed index bytes of the packed
-    tokens. norms: 2 bytes per packed row, K and V. codebooks: fp16 centroids
+    dense: bf16 K and V of every token. index: packed index bytes (with QJL
+    also the sign bytes) of the packed tokens. norms: 2 bytes per packed row
+    (4 with QJL: the residual norm too), K and V. codebooks: fp16 centroids
     and fp32 boundaries of every group of both codecs. transforms: d int8 signs
-    and H_kv*d int16 permutation entries per codec. window: the allocated bf16
-    window, K and V. block tables: one int32 per used block.
+    and H_kv*d int16 permutation entries per codec, plus the fp32 d x d QJL
+    matrix of a QJL codec. window: the allocated bf16 window, K and V. block
+    tables: one int32 per used block.
     """
     H, d = kfmt.num_kv_heads, kfmt.head_dim
     lens = [int(x) for x in seq_lens]
@@ -618,12 +716,12 @@ def byte_ledger(kfmt: Format, vfmt: Format, seq_lens: Sequence[int], window: int
     P = sum(packed)
     dense = 2 * 2 * H * d * sum(lens)
     idx = P * H * (index_bytes(kfmt) + index_bytes(vfmt))
-    norms = P * H * 2 * 2
+    norms = P * H * (norm_bytes(kfmt) + norm_bytes(vfmt))
     cb = 0
     for fmt in (kfmt, vfmt):
         for b in fmt.group_bits:
             cb += (1 << b) * 2 + ((1 << b) - 1) * 4
-    transforms = 2 * (d + H * d * 2)
+    transforms = 2 * (d + H * d * 2) + sum(4 * d * d for fmt in (kfmt, vfmt) if fmt.qjl)
     win = 2 * 2 * len(lens) * H * window * d
     bt = 4 * sum(-(-p // block_size) for p in packed)
     pool = num_blocks * H * block_size * (row_bytes(kfmt) + row_bytes(vfmt))

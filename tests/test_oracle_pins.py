@@ -580,3 +580,109 @@ def test_boundary_tokens_as_window_equal_attention_in_token_order():
             for g in range(G):
                 ref = O.dense_attention(q[b, h * G + g], keys, vals, 0.3)
                 assert np.abs(out[b, h * G + g] - ref).max() < 1e-12
+
+
+# ---- QJL residual stage (R16) ----------------------------------------------------------
+
+def test_qjl_estimator_is_unbiased_over_the_projection():
+    """E_S[q . (c + sqrt(pi/2)/d g S^T sign(S r))] = q . u for Gaussian S (the QJL identity).
+
+    Averaged over many independent S, the estimate converges to the exact
+    product; a wrong constant or an inverted sign convention is far outside
+    the bound (the mean of S^T sign(S r) is sqrt(2/pi) d r / |r| exactly).
+    """
+    rng = np.random.default_rng(7)
+    d = 64
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    c_hat = np.round(u * 4) / 4  # any fixed approximation; r is its residual
+    r = u - c_hat
+    g = np.linalg.norm(r)
+    q = rng.standard_normal(d) + 5 * r / g  # a clear component along the residual
+    n_draw = 4000
+    est = np.empty(n_draw)
+    for i in range(n_draw):
+        S = rng.standard_normal((d, d))
+        z = np.where(S @ r >= 0, 1.0, -1.0)
+        est[i] = q @ (c_hat + math.sqrt(math.pi / 2) / d * g * (S.T @ z))
+    exact = q @ u
+    sem = est.std(ddof=1) / math.sqrt(n_draw)
+    assert abs(est.mean() - exact) < 4.5 * sem
+    # the QJL variance bound: Var <= pi/(2d) |q|^2 g^2
+    assert est.var() <= 1.05 * math.pi / (2 * d) * (q @ q) * g * g
+    # and the constant matters: the same draws with 1/d instead of sqrt(pi/2)/d are biased
+    biased = (est - q @ c_hat) / math.sqrt(math.pi / 2) + q @ c_hat
+    assert abs(biased.mean() - exact) > 10 * sem
+
+
+def test_qjl_matrix_is_standard_normal():
+    """S entries (Box-Muller over SplitMix64) pass a Kolmogorov-Smirnov test against N(0, 1)."""
+    import scipy.stats
+    fmt = O.Format(128, 1, (3,), (128,), None, 5, qjl=True)
+    S = O.qjl_matrix(fmt)
+    assert S.shape == (128, 128)
+    assert np.all(S == S.astype(np.float32))  # held in fp32
+    p = scipy.stats.kstest(S.ravel(), "norm").pvalue
+    assert p > 1e-3
+    assert abs(S.mean()) < 0.03 and abs(S.std() - 1) < 0.02
+    # independent of the sign stream: another seed gives another matrix
+    S2 = O.qjl_matrix(O.Format(128, 1, (3,), (128,), None, 6, qjl=True))
+    assert abs(np.corrcoef(S.ravel(), S2.ravel())[0, 1]) < 0.03
+
+
+def test_qjl_row_layout_by_hand():
+    """[MSE indices][d sign bits LSB-first][fp16 norm][fp16 residual norm], decoded bit by bit."""
+    rng = np.random.default_rng(12)
+    d, H = 16, 1
+    high = np.array([[0, 3, 5, 6, 9, 10, 12, 15]])
+    fmt = O.Format(d, H, (3, 2), (8, 8), high, 4, qjl=True)
+    assert O.row_bytes(fmt) == 3 + 2 + d // 8 + 4
+    x = O.bf16_round(rng.standard_normal((5, d)) * 3)
+    idx, n16, u, signs, g16 = O.quantize_qjl(x, fmt, 0)
+    rows = O.encode_rows(idx, n16, fmt, signs, g16)
+    for t in range(5):
+        row = rows[t]
+        bit = lambda k: (int(row[k // 8]) >> (k % 8)) & 1
+        pos = 0
+        for p in range(16):
+            b = 3 if p < 8 else 2
+            assert sum(bit(pos + j) << j for j in range(b)) == idx[t, p]
+            pos += b
+        assert pos == 40
+        for i in range(d):
+            assert bit(pos + i) == signs[t, i]
+        nb = 40 // 8 + d // 8
+        assert struct.unpack("<e", bytes(row[nb:nb + 2]))[0] == n16[t]
+        assert struct.unpack("<e", bytes(row[nb + 2:nb + 4]))[0] == g16[t]
+    back = O.decode_rows(rows, fmt)
+    assert np.array_equal(back[0], idx) and np.array_equal(back[2], signs)
+    assert np.array_equal(back[1], n16) and np.array_equal(back[3], g16)
+
+
+def test_qjl_residual_and_signs_follow_the_definitions():
+    """r = u - c[idx] in rotated order, g = |r|, bit i = [(S r)_i >= 0]; keys from rows agree."""
+    rng = np.random.default_rng(13)
+    d, H = 128, 2
+    fmt = O.Format(d, H, (3,), (d,), None, 21, qjl=True)
+    x = O.bf16_round(rng.standard_normal((6, d)) * 2)
+    idx, n16, u, signs, g16 = O.quantize_qjl(x, fmt, 1)
+    c, _ = O.codebook(3, d)
+    r = u - c[idx]  # one group: packed order is rotated order
+    assert np.allclose(g16, O.fp16_round(np.linalg.norm(r, axis=-1)))
+    proj = r @ O.qjl_matrix(fmt).T
+    assert np.array_equal(signs, (proj >= 0).astype(np.int64))
+    # the key a row stands for: n R^T (c[idx] + sqrt(pi/2)/d g S^T z)
+    key = O.dequantize_rows(idx, n16, fmt, 1, signs, g16)
+    z = 2.0 * signs - 1.0
+    rot = c[idx] + math.sqrt(math.pi / 2) / d * g16[:, None] * (z @ O.qjl_matrix(fmt))
+    H128 = O.hadamard_matrix(d)
+    s = O.hadamard_signs(fmt.seed, d)
+    expect = n16[:, None] * (rot @ H128.T) * s / math.sqrt(d)
+    assert np.allclose(key, expect, atol=1e-12)
+    # q . key estimates q . x: over many vectors the mean error is small against the spread
+    q = rng.standard_normal(d)
+    xs = O.bf16_round(rng.standard_normal((400, d)))
+    i2, n2, _, s2, g2 = O.quantize_qjl(xs, fmt, 0)
+    est = O.dequantize_rows(i2, n2, fmt, 0, s2, g2) @ q
+    err = est - xs @ q
+    assert abs(err.mean()) < 4 * err.std(ddof=1) / math.sqrt(len(err))
