@@ -71,6 +71,18 @@ typedef enum {
  *                the rotated coordinates of group 0, strictly ascending.
  *                NULL when n_groups == 1. Copied by tq_make_codec.
  * hadamard_seed  SplitMix64 seed of the sign vector of the rotation.
+ * qjl            0, or 1 for the QJL residual stage ([Design] "Recipe
+ *                Strategy": row [MSE indices][QJL signs][vector norm]
+ *                [residual norm]). The groups above are the MSE part; the row
+ *                then carries head_dim sign bits of S r (r = u - c[idx], the
+ *                residual of the unit rotated vector in rotated coordinate
+ *                order; bit i = 1 when (S r)_i >= 0, LSB-first) and the fp16
+ *                residual norm |r| after the norm. S = tq_codec_qjl_matrix.
+ *                In a sub-page the sign bytes follow each row's index bytes and
+ *                the norm area holds (norm, residual norm) per row. The key a
+ *                row stands for is n R^T (c + sqrt(pi/2)/d |r| S^T z), z = 2 bits
+ *                - 1: its product with q is the unbiased QJL estimate of q.x.
+ *                Decode accepts QJL for K only.
  */
 typedef struct {
     int32_t head_dim;
@@ -80,6 +92,7 @@ typedef struct {
     int32_t group_size[2];
     const int16_t* high_coords;
     uint64_t hadamard_seed;
+    int32_t qjl;
 } tq_format_desc;
 
 typedef struct tq_codec tq_codec; /* opaque, immutable after tq_make_codec */
@@ -103,6 +116,16 @@ typedef struct tq_codec tq_codec; /* opaque, immutable after tq_make_codec */
  */
 tq_status tq_codec_host_tables(const tq_format_desc* desc, uint16_t* centroids_f16, float* boundaries,
                                int8_t* signs, int16_t* perm, int32_t* row_bytes);
+
+/*
+ * The QJL matrix S of a codec: out, float [head_dim][head_dim], row-major.
+ * S[i][j] is the cosine branch of the Box-Muller transform of two uniforms
+ * from SplitMix64 seeded with hadamard_seed ^ 0x51534A4C00000001: outputs
+ * 2k and 2k + 1 (k = i * head_dim + j) give u1 = ((x >> 11) + 1) 2^-53 and
+ * u2 = (x >> 11) 2^-53, S = sqrt(-2 ln u1) cos(2 pi u2) in double, rounded to
+ * float. Host only; TQ_ERR_VALUE for an invalid descriptor.
+ */
+tq_status tq_codec_qjl_matrix(const tq_format_desc* desc, float* out);
 
 /*
  * Validate `desc`, build the codec tables on the host and copy them to the

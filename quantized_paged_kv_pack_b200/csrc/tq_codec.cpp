@@ -184,6 +184,18 @@ uint64_t splitmix64_next(uint64_t& state) {
     return z ^ (z >> 31);
 }
 
+// S of the QJL stage, row-major [d][d] (see tq_codec_qjl_matrix in tq.h).
+void qjl_matrix(uint64_t seed, int d, std::vector<float>& out) {
+    out.resize(static_cast<size_t>(d) * d);
+    uint64_t state = seed ^ 0x51534A4C00000001ull;
+    for (size_t k = 0; k < out.size(); ++k) {
+        const uint64_t a = splitmix64_next(state), b = splitmix64_next(state);
+        const double u1 = (static_cast<double>(a >> 11) + 1.0) * 0x1p-53;  // (0, 1]
+        const double u2 = static_cast<double>(b >> 11) * 0x1p-53;          // [0, 1)
+        out[k] = static_cast<float>(std::sqrt(-2.0 * std::log(u1)) * std::cos(2.0 * M_PI * u2));
+    }
+}
+
 }  // namespace
 
 tq_status fail(tq_status st, const std::string& msg) {
@@ -216,6 +228,7 @@ tq_status validate_desc(const tq_format_desc* d) {
         total += n;
     }
     if (total != d->head_dim) return fail(TQ_ERR_VALUE, "group sizes must sum to head_dim");
+    if (d->qjl != 0 && d->qjl != 1) return fail(TQ_ERR_VALUE, "qjl must be 0 or 1");
     if (d->n_groups == 1) {
         if (d->high_coords) return fail(TQ_ERR_VALUE, "high_coords given for a one-group format");
     } else {
@@ -278,8 +291,11 @@ tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c) {
     }
     int bytes = 0;
     for (int g = 0; g < desc->n_groups; ++g) bytes += desc->group_bits[g] * desc->group_size[g] / 8;
-    c->index_bytes = bytes;
-    c->row_bytes = bytes + 2;
+    const int sign_bytes = desc->qjl ? d / 8 : 0, norm_bytes = desc->qjl ? 4 : 2;
+    c->index_bytes = bytes + sign_bytes;
+    c->row_bytes = c->index_bytes + norm_bytes;
+    c->qjl_s.clear();
+    if (desc->qjl) qjl_matrix(desc->hadamard_seed, d, c->qjl_s);
     DevCodec& v = c->dev;
     v.num_heads = H;
     v.n_groups = desc->n_groups;
@@ -295,6 +311,10 @@ tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c) {
     }
     v.index_bytes = c->index_bytes;
     v.row_bytes = c->row_bytes;
+    v.qjl = desc->qjl;
+    v.mse_bytes = bytes;
+    v.norm_bytes = norm_bytes;
+    v.qjl_st = nullptr;  // set by tq_make_codec
     return TQ_OK;
 }
 
@@ -351,6 +371,17 @@ tq_status tq_codec_host_tables(const tq_format_desc* desc, uint16_t* centroids_f
     return TQ_OK;
 }
 
+tq_status tq_codec_qjl_matrix(const tq_format_desc* desc, float* out) {
+    clear_error();
+    tq_status st = validate_desc(desc);
+    if (st != TQ_OK) return st;
+    if (!out) return fail(TQ_ERR_VALUE, "null output pointer");
+    std::vector<float> s;
+    qjl_matrix(desc->hadamard_seed, desc->head_dim, s);
+    std::memcpy(out, s.data(), s.size() * sizeof(float));
+    return TQ_OK;
+}
+
 tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     clear_error();
     if (!out) return fail(TQ_ERR_VALUE, "null output pointer");
@@ -364,7 +395,9 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     const int d = desc->head_dim, H = desc->num_kv_heads;
     const size_t n_sign = d * sizeof(float), n_cent = 2 * kMaxLevels * sizeof(float);
     const size_t n_perm = static_cast<size_t>(H) * d * sizeof(int16_t);
-    const size_t total = n_sign + 2 * n_cent + 2 * n_perm;
+    const size_t off_s = (n_sign + 2 * n_cent + 2 * n_perm + 15) / 16 * 16;
+    const size_t n_s = c->qjl_s.size() * sizeof(float);
+    const size_t total = off_s + n_s;
     std::vector<char> host(total);
     char* p = host.data();
     std::memcpy(p, c->sign, n_sign);
@@ -372,6 +405,11 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     std::memcpy(p + n_sign + n_cent, c->bound, n_cent);
     std::memcpy(p + n_sign + 2 * n_cent, c->perm.data(), n_perm);
     std::memcpy(p + n_sign + 2 * n_cent + n_perm, c->pos.data(), n_perm);
+    if (n_s) {  // QJL: S transposed, so that a warp reads one row of S^T per coordinate j
+        float* st = reinterpret_cast<float*>(p + off_s);
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) st[static_cast<size_t>(j) * d + i] = c->qjl_s[static_cast<size_t>(i) * d + j];
+    }
     if (cudaGetDevice(&c->device) != cudaSuccess || cudaMalloc(&c->d_tables, total) != cudaSuccess) {
         cudaGetLastError();
         delete c;
@@ -389,6 +427,7 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     c->dev.bound = reinterpret_cast<const float*>(base + n_sign + n_cent);
     c->dev.perm = reinterpret_cast<const int16_t*>(base + n_sign + 2 * n_cent);
     c->dev.pos = reinterpret_cast<const int16_t*>(base + n_sign + 2 * n_cent + n_perm);
+    c->dev.qjl_st = n_s ? reinterpret_cast<const float*>(base + off_s) : nullptr;
     *out = c;
     return TQ_OK;
 }
@@ -435,13 +474,13 @@ tq_status tq_byte_ledger(const tq_format_desc* kdesc, const tq_format_desc* vdes
     tq_ledger r{};
     r.dense_bytes = 2 * 2 * H * d * total;
     r.index_bytes = packed * H * (kc.index_bytes + vc.index_bytes);
-    r.norm_bytes = packed * H * 2 * 2;
+    r.norm_bytes = packed * H * ((kdesc->qjl ? 4 : 2) + (vdesc->qjl ? 4 : 2));
     for (const tq_format_desc* desc : {kdesc, vdesc})
         for (int g = 0; g < desc->n_groups; ++g) {
             int64_t L = int64_t(1) << desc->group_bits[g];
             r.codebook_bytes += L * 2 + (L - 1) * 4;
         }
-    r.transform_bytes = 2 * (d + H * d * 2);
+    r.transform_bytes = 2 * (d + H * d * 2) + 4 * d * d * ((kdesc->qjl ? 1 : 0) + (vdesc->qjl ? 1 : 0));
     r.window_bytes = 2 * 2 * static_cast<int64_t>(batch) * H * window * d;
     r.block_table_bytes = 4 * blocks;
     r.workspace_bytes = static_cast<int64_t>(

@@ -49,8 +49,10 @@ __device__ __forceinline__ int row_index(const uint8_t* row, const DevCodec& c, 
     return static_cast<int>((w >> sh) & ((1u << b) - 1u));
 }
 
-__device__ __forceinline__ float row_norm(const uint8_t* sub, const DevCodec& c, int block_size, int off) {
-    const uint8_t* n = sub + block_size * c.index_bytes + 2 * off;
+// The fp16 norm (which = 0) or, with QJL, the residual norm (which = 1) of row `off`.
+__device__ __forceinline__ float row_norm(const uint8_t* sub, const DevCodec& c, int block_size, int off,
+                                          int which = 0) {
+    const uint8_t* n = sub + block_size * c.index_bytes + c.norm_bytes * off + 2 * which;
     unsigned short h = static_cast<unsigned short>(n[0] | (n[1] << 8));
     return __half2float(__ushort_as_half(h));
 }
@@ -82,6 +84,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
     __shared__ float qs[G][kHeadDim];
     __shared__ float red_m[kWarps][G], red_l[kWarps][G];
     __shared__ float red_acc[kWarps][G][kHeadDim];
+    // QJL keys: (S q_r)_i (q_r in rotated coordinate order) during the token loop,
+    // in the space of the per-warp accumulators, which are written only after it.
+    float (*sq)[kHeadDim] = red_acc[0];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     int t0, t1;
@@ -123,6 +128,18 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
         for (int i = 0; i < 4; ++i) qs[g][a.kc.pos[h * kHeadDim + 4 * lane + i]] = z[i] * sc;
     }
     __syncthreads();
+    const bool qjl = a.kc.qjl && !is_win;
+    if (qjl) {
+        // (S q_r)_i = sum_j S^T[j][i] q_r[j], q_r[j] = qs[pos(j)]; times sqrt(pi/2)/d, the estimator's constant.
+        for (int e = threadIdx.x; e < G * kHeadDim; e += kWarps * 32) {
+            const int g = e / kHeadDim, i = e - g * kHeadDim;
+            float acc = 0.0f;
+            for (int j = 0; j < kHeadDim; ++j)
+                acc = fmaf(__ldg(a.kc.qjl_st + j * kHeadDim + i), qs[g][a.kc.pos[h * kHeadDim + j]], acc);
+            sq[g][i] = acc * (1.2533141373155003f / kHeadDim);  // sqrt(pi/2) / d
+        }
+        __syncthreads();
+    }
 
     float m[G], l[G], acc[G][4];
 #pragma unroll
@@ -134,7 +151,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
     }
     const int bs = a.block_size;
     for (int t = t0 + warp; t < t1; t += kWarps) {
-        float kv[4], vv[4], nk = 1.0f, nv = 1.0f;
+        float kv[4], vv[4], nk = 1.0f, nv = 1.0f, gk = 0.0f, zk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         if (is_win) {
             const int64_t base = ((static_cast<int64_t>(b) * H + h) * a.window + t) * kHeadDim + 4 * lane;
 #pragma unroll
@@ -164,12 +181,25 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
             }
             nk = row_norm(ksub, a.kc, bs, off);
             nv = row_norm(vsub, a.vc, bs, off);
+            if (qjl) {
+                // sign bits 4l .. 4l+3 of the QJL stream (after the index bitstreams)
+                const unsigned bits = (krow[a.kc.mse_bytes + (lane >> 1)] >> (4 * (lane & 1))) & 0xFu;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) zk[i] = ((bits >> i) & 1u) ? 1.0f : -1.0f;
+                gk = row_norm(ksub, a.kc, bs, off, 1);
+            }
         }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             float s = 0.0f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) s += qs[g][4 * lane + i] * kv[i];
+            if (qjl) {
+                float t = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) t += sq[g][4 * lane + i] * zk[i];
+                s += gk * t;  // q_r . (c + sqrt(pi/2)/d g S^T z), summed over the warp below
+            }
             s = warp_sum(s) * nk;
             const float mn = fmaxf(m[g], s);
             const float alpha = exp2f(m[g] - mn);
@@ -181,6 +211,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
             m[g] = mn;
         }
     }
+    if (qjl) __syncthreads();  // every warp is done with sq before red_acc is written
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         if (lane == 0) {
@@ -268,6 +299,7 @@ tq_status check_decode_args(const tq_codec* kc, const tq_codec* vc, int32_t batc
     const int G = num_q_heads / H;
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
         return fail(TQ_ERR_UNSUPPORTED, "query heads per KV head must be 1, 2, 4, 8 or 16");
+    if (vc->desc.qjl) return fail(TQ_ERR_UNSUPPORTED, "decode implements the QJL stage for keys only");
     if (!make_split_plan(batch, num_q_heads, H, max_seq_len, block_size, plan))
         return fail(TQ_ERR_VALUE, "invalid decode sizes");
     if (workspace_bytes < plan->workspace_bytes) return fail(TQ_ERR_VALUE, "workspace smaller than tq_decode_workspace_bytes");
@@ -353,8 +385,9 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     // Tensor-core kernel for the formats it is instantiated for (block sizes a
     // multiple of 16); the general kernel covers every other valid format.
     // TQ_DECODE_KERNEL=general selects the general kernel (for cross-checks).
+    // QJL keys (the sign-bit score term) run on the general kernel.
     const char* force = std::getenv("TQ_DECODE_KERNEL");
-    if (!(force && std::string(force) == "general")) {
+    if (!(force && std::string(force) == "general") && !kc->desc.qjl) {
         st = launch_decode_mma(a, kc, vc, plan.group, stream);
         if (st == TQ_OK) return finish(s, d_err, "decode partials");
         if (st != TQ_ERR_UNSUPPORTED) return st;

@@ -26,8 +26,12 @@ struct DevCodec {
     int32_t size[2];
     int32_t pos0[2];        // first packed position of each group
     int32_t byte_off[2];    // byte offset of each group's bitstream in the row
-    int32_t index_bytes;
+    int32_t index_bytes;    // bytes before the norms: the index bitstreams, then the QJL signs
     int32_t row_bytes;
+    int32_t qjl;            // 1: QJL residual stage
+    int32_t mse_bytes;      // bytes of the index bitstreams
+    int32_t norm_bytes;     // 2, or 4 with QJL (norm, residual norm)
+    const float* qjl_st;    // QJL: S transposed, [128][128] (entry j * 128 + i = S[i][j])
 };
 
 // Arguments of the decode kernels (device pointers; see tq_decode_paged).
@@ -67,6 +71,7 @@ struct tq_codec {
     float sign[tq::kHeadDim];
     std::vector<int16_t> perm;     // [H][d]
     std::vector<int16_t> pos;      // [H][d]
+    std::vector<float> qjl_s;      // QJL: S, [d][d] row-major
     int32_t row_bytes = 0;
     int32_t index_bytes = 0;
     int device = 0;

@@ -70,9 +70,10 @@ __device__ __forceinline__ unsigned short norm_fp16_bits(const float (&x)[4], fl
 
 // One warp quantizes the vector x (lane l holds elements 4l .. 4l+3) of KV
 // head h and writes its row at `offset` of the sub-page `sub` (block_size
-// rows). idx_buf: 128 bytes of shared scratch owned by the warp.
+// rows). idx_buf: 128 bytes, r_buf: 128 floats of shared scratch owned by the
+// warp (r_buf is used by the QJL stage only).
 __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8_t* sub, int64_t offset,
-                            int block_size, uint8_t* idx_buf, int lane) {
+                            int block_size, uint8_t* idx_buf, float* r_buf, int lane) {
     float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
     float n32 = sqrtf(ss);
     const unsigned short n16 = norm_fp16_bits(x, ss, n32);
@@ -96,6 +97,7 @@ __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8
         }
     }
     const float inv = n32 > 0.0f ? 1.0f / (n32 * 11.313708498984761f) : 0.0f;
+    float rr = 0.0f;  // QJL: sum of squared residuals of this lane's coordinates
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int j = 4 * lane + i;
@@ -106,9 +108,29 @@ __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8
         int idx = 0;
         for (int q = 0; q < levels - 1; ++q) idx += (c.bound[g * 16 + q] < u) ? 1 : 0;
         idx_buf[p] = static_cast<uint8_t>(idx);
+        if (c.qjl) {
+            const float r = u - c.cent[g * 16 + idx];  // residual, rotated coordinate j
+            r_buf[j] = r;
+            rr += r * r;
+        }
     }
     __syncwarp();
-    const int half_words = c.index_bytes / 2;
+    // QJL stage: (S r)_i for i = lane + 32k from S^T rows (coalesced), sign bits by ballot.
+    uint32_t sign_word[4] = {0u, 0u, 0u, 0u};
+    unsigned short g16 = 0;
+    if (c.qjl) {
+        g16 = __half_as_ushort(__float2half_rn(sqrtf(warp_sum(rr))));
+        float proj[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int j = 0; j < kHeadDim; ++j) {
+            const float r = r_buf[j];
+            const float* st = c.qjl_st + j * kHeadDim + lane;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) proj[k] = fmaf(__ldg(st + 32 * k), r, proj[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sign_word[k] = __ballot_sync(kFull, proj[k] >= 0.0f);
+    }
+    const int half_words = c.mse_bytes / 2;
     unsigned word = 0;
     if (lane < half_words) {
         for (int i = 0; i < 16; ++i) {
@@ -122,7 +144,13 @@ __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8
     }
     uint16_t* dst = reinterpret_cast<uint16_t*>(sub + offset * c.index_bytes);
     if (lane < half_words) dst[lane] = static_cast<uint16_t>(word);
-    if (lane == 0) *reinterpret_cast<uint16_t*>(sub + block_size * c.index_bytes + 2 * offset) = n16;
+    uint16_t* nrm = reinterpret_cast<uint16_t*>(sub + block_size * c.index_bytes + c.norm_bytes * offset);
+    if (c.qjl) {
+        // sign bits after the index bitstreams, LSB-first: half-word m holds bits 16m .. 16m+15
+        if (lane < kHeadDim / 16) dst[half_words + lane] = static_cast<uint16_t>(sign_word[lane >> 1] >> (16 * (lane & 1)));
+        if (lane == 0) nrm[1] = g16;
+    }
+    if (lane == 0) nrm[0] = n16;
     __syncwarp();
 }
 
@@ -140,6 +168,7 @@ pack_rows_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__ k,
                  uint8_t* __restrict__ k_pages, uint8_t* __restrict__ v_pages, int64_t num_blocks,
                  int block_size, int* __restrict__ d_err) {
     __shared__ uint8_t idx_buf[kPackWarps][kHeadDim];
+    __shared__ float r_buf[kPackWarps][kHeadDim];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t H = kc.num_heads;
     const int64_t n_vec = num_tokens * H * 2;
@@ -161,7 +190,7 @@ pack_rows_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__ k,
         load_bf16x4((which ? v : k) + th * kHeadDim + 4 * lane, x);
         const int64_t blk = slot / block_size, off = slot - blk * block_size;
         uint8_t* sub = (which ? v_pages : k_pages) + (blk * H + h) * block_size * c.row_bytes;
-        pack_vector(c, x, h, sub, off, block_size, idx_buf[warp], lane);
+        pack_vector(c, x, h, sub, off, block_size, idx_buf[warp], r_buf[warp], lane);
     }
 }
 
@@ -180,6 +209,7 @@ window_append_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__
                      uint8_t* __restrict__ v_pages, int64_t num_blocks, int block_size, int batch,
                      int* __restrict__ d_err) {
     __shared__ uint8_t idx_buf[kPackWarps][kHeadDim];
+    __shared__ float r_buf[kPackWarps][kHeadDim];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = kc.num_heads;
     const int64_t n_vec = static_cast<int64_t>(batch) * H * 2;
@@ -215,7 +245,7 @@ window_append_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__
                 float x[4];
                 load_bf16x4(pack_new ? src_new : wbuf + static_cast<int64_t>(slot_w) * kHeadDim + 4 * lane, x);
                 uint8_t* sub = (which ? v_pages : k_pages) + (static_cast<int64_t>(blk) * H + h) * block_size * c.row_bytes;
-                pack_vector(c, x, h, sub, off, block_size, idx_buf[warp], lane);  // reads x before the slot is reused
+                pack_vector(c, x, h, sub, off, block_size, idx_buf[warp], r_buf[warp], lane);  // x read before the slot is reused
             }
         }
         if (slot_w >= 0)

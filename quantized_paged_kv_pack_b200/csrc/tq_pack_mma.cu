@@ -402,7 +402,7 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
                          const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
                          int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream) {
     for (const tq_codec* c : {kc, vc})
-        if (c->desc.n_groups != 1 || c->desc.group_bits[0] != 4) return TQ_ERR_UNSUPPORTED;
+        if (c->desc.n_groups != 1 || c->desc.group_bits[0] != 4 || c->desc.qjl) return TQ_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 15) return TQ_ERR_UNSUPPORTED;
     if (block_size % 8 != 0) return TQ_ERR_UNSUPPORTED;  // 16-byte aligned rows and norm arrays
     // 32-bit index arithmetic in the kernel: slots, tokens and work units must fit.

@@ -41,7 +41,8 @@ class TQCudaError(RuntimeError):
 class _FormatDesc(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("n_groups", ctypes.c_int32),
                 ("group_bits", ctypes.c_int32 * 2), ("group_size", ctypes.c_int32 * 2),
-                ("high_coords", ctypes.POINTER(ctypes.c_int16)), ("hadamard_seed", ctypes.c_uint64)]
+                ("high_coords", ctypes.POINTER(ctypes.c_int16)), ("hadamard_seed", ctypes.c_uint64),
+                ("qjl", ctypes.c_int32)]
 
 
 class _Ledger(ctypes.Structure):
@@ -65,6 +66,7 @@ def lib():
         P = ctypes.POINTER
         L.tq_last_error.restype = ctypes.c_char_p
         L.tq_codec_host_tables.argtypes = [P(_FormatDesc), _VP, _VP, _VP, _VP, _VP]
+        L.tq_codec_qjl_matrix.argtypes = [P(_FormatDesc), _VP]
         L.tq_make_codec.argtypes = [P(_FormatDesc), P(_VP)]
         L.tq_free_codec.argtypes = [_VP]
         L.tq_free_codec.restype = None
@@ -82,7 +84,7 @@ def lib():
                                        _I32, _I32, _VP, _VP]
         L.tq_byte_ledger.argtypes = [P(_FormatDesc), P(_FormatDesc), _I32, _VP, _I32, _I32, _I32, _I64, _I32,
                                      P(_Ledger)]
-        for name in ("tq_codec_host_tables", "tq_make_codec", "tq_pack_kv", "tq_decode_paged",
+        for name in ("tq_codec_host_tables", "tq_codec_qjl_matrix", "tq_make_codec", "tq_pack_kv", "tq_decode_paged",
                      "tq_decode_partials", "tq_decode_combine", "tq_byte_ledger", "tq_decode_paged_static",
                      "tq_window_append"):
             getattr(L, name).restype = ctypes.c_int
@@ -107,7 +109,7 @@ def _check(status: int):
     raise TQCudaError(msg or f"tq status {status}")
 
 
-def _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed):
+def _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl=False):
     bits, sizes = tuple(group_bits), tuple(group_size)
     d = _FormatDesc()
     d.head_dim, d.num_kv_heads, d.n_groups = head_dim, num_kv_heads, len(bits)
@@ -120,12 +122,13 @@ def _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed):
         keep = np.ascontiguousarray(np.asarray(high_coords, dtype=np.int16))
         d.high_coords = keep.ctypes.data_as(ctypes.POINTER(ctypes.c_int16))
     d.hadamard_seed = int(seed) & ((1 << 64) - 1)
+    d.qjl = 1 if qjl else 0
     return d, keep
 
 
-def codec_host_tables(head_dim, num_kv_heads, group_bits, group_size, high_coords=None, seed=0):
+def codec_host_tables(head_dim, num_kv_heads, group_bits, group_size, high_coords=None, seed=0, qjl=False):
     """Host-side codec tables (no CUDA call): codebooks, signs, permutation, row bytes."""
-    d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed)
+    d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl)
     c16 = np.zeros((2, 16), np.uint16)
     bnd = np.zeros((2, 15), np.float32)
     sg = np.zeros(head_dim, np.int8)
@@ -137,15 +140,25 @@ def codec_host_tables(head_dim, num_kv_heads, group_bits, group_size, high_coord
     return {"centroids_f16": c16, "boundaries": bnd, "signs": sg, "perm": perm, "row_bytes": rb.value}
 
 
+def qjl_matrix(head_dim, num_kv_heads, group_bits, group_size, high_coords=None, seed=0) -> np.ndarray:
+    """The QJL matrix S of a codec (tq_codec_qjl_matrix), float32 [head_dim][head_dim]; host only."""
+    d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, True)
+    out = np.zeros((head_dim, head_dim), np.float32)
+    _check(lib().tq_codec_qjl_matrix(ctypes.byref(d), out.ctypes.data))
+    del keep
+    return out
+
+
 class Codec:
     """A device codec (tq_make_codec); immutable, freed on close()."""
 
     def __init__(self, num_kv_heads: int, group_bits: Sequence[int], group_size: Sequence[int],
-                 high_coords=None, seed: int = 0, head_dim: int = HEAD_DIM):
+                 high_coords=None, seed: int = 0, head_dim: int = HEAD_DIM, qjl: bool = False):
         self.head_dim, self.num_kv_heads = head_dim, num_kv_heads
         self.group_bits, self.group_size, self.seed = tuple(group_bits), tuple(group_size), seed
+        self.qjl = bool(qjl)
         self.high_coords = None if high_coords is None else np.asarray(high_coords, dtype=np.int16)
-        d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed)
+        d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl)
         h = _VP()
         _check(lib().tq_make_codec(ctypes.byref(d), ctypes.byref(h)))
         del keep
@@ -159,7 +172,8 @@ class Codec:
         return self._h
 
     def desc(self):
-        return _desc(self.head_dim, self.num_kv_heads, self.group_bits, self.group_size, self.high_coords, self.seed)
+        return _desc(self.head_dim, self.num_kv_heads, self.group_bits, self.group_size, self.high_coords, self.seed,
+                     self.qjl)
 
     def close(self):
         if getattr(self, "_h", None) is not None:
@@ -407,9 +421,9 @@ def host_ledger(num_kv_heads, kspec: dict, vspec: dict, seq_lens, window, num_q_
     lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
     max_seq_len = int(lens.max()) if max_seq_len is None and len(lens) else int(max_seq_len or 0)
     kd, kkeep = _desc(HEAD_DIM, num_kv_heads, kspec["group_bits"], kspec["group_size"], kspec.get("high_coords"),
-                      kspec.get("seed", 0))
+                      kspec.get("seed", 0), kspec.get("qjl", False))
     vd, vkeep = _desc(HEAD_DIM, num_kv_heads, vspec["group_bits"], vspec["group_size"], vspec.get("high_coords"),
-                      vspec.get("seed", 0))
+                      vspec.get("seed", 0), vspec.get("qjl", False))
     r = _Ledger()
     _check(lib().tq_byte_ledger(ctypes.byref(kd), ctypes.byref(vd), len(lens), lens.ctypes.data, window, num_q_heads,
                                 block_size, num_blocks, max_seq_len, ctypes.byref(r)))

@@ -17,17 +17,18 @@ def random_high(H, n, seed):
     return np.stack([np.sort(rng.choice(D, n, replace=False)) for _ in range(H)]).astype(np.int16)
 
 
-def codec_pair(H, bits, sizes, seed, high=None):
+def codec_pair(H, bits, sizes, seed, high=None, qjl=False):
     """(device Codec, oracle Format) for the same plain parameters."""
     if len(bits) == 2 and high is None:
         high = random_high(H, sizes[0], seed + 17)
-    return tq.Codec(H, bits, sizes, high, seed), O.Format(D, H, tuple(bits), tuple(sizes), high, seed)
+    return (tq.Codec(H, bits, sizes, high, seed, qjl=qjl),
+            O.Format(D, H, tuple(bits), tuple(sizes), high, seed, qjl=qjl))
 
 
 def slice_format(f: O.Format, h: int) -> O.Format:
     """The oracle format of KV head h alone (metadata sliced to one head)."""
     hc = None if f.high_coords is None else np.asarray(f.high_coords)[h:h + 1]
-    return O.Format(f.head_dim, 1, f.group_bits, f.group_size, hc, f.seed)
+    return O.Format(f.head_dim, 1, f.group_bits, f.group_size, hc, f.seed, qjl=f.qjl)
 
 
 def random_kv(T, H, gen, scale_outliers=True):
@@ -51,7 +52,8 @@ class DecodeProblem:
     decode call's window is S + window.
     """
 
-    def __init__(self, lens, H, G, kspec, vspec, window, block_size, seed, slack=1.3, sinks=0):
+    def __init__(self, lens, H, G, kspec, vspec, window, block_size, seed, slack=1.3, sinks=0, kqjl=False,
+                 vqjl=False):
         self.lens = np.asarray(lens, dtype=np.int64)
         self.B, self.H, self.G, self.Hq = len(lens), H, G, H * G
         self.sinks = sinks
@@ -60,8 +62,8 @@ class DecodeProblem:
         gen = torch.Generator(device="cuda")
         gen.manual_seed(seed)
         rng = np.random.default_rng(seed)
-        self.kc, self.kf = codec_pair(H, *kspec)
-        self.vc, self.vf = codec_pair(H, *vspec)
+        self.kc, self.kf = codec_pair(H, *kspec, qjl=kqjl)
+        self.vc, self.vf = codec_pair(H, *vspec, qjl=vqjl)
         packed = self.lens - np.minimum(window, self.lens)
         nblk = -(-packed // block_size)
         self.num_blocks = max(1, int(math.ceil(slack * nblk.sum())) + 1)

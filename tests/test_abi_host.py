@@ -134,3 +134,33 @@ def test_recipe_metadata_loader(tmp_path):
     with pytest.raises(ValueError):
         bad.write_text(json.dumps({"head_dim": 128}))
         tq.load_recipe_metadata(str(bad))
+
+
+
+# ---- QJL codecs (host side) ------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", [0, 5, 2**63 + 11])
+def test_qjl_matrix_equals_oracle(seed):
+    """The library's S (C++ double math, rounded to float) equals the oracle's (NumPy) entry for entry."""
+    got = tq.qjl_matrix(D, 2, (3,), (128,), None, seed)
+    ref = O.qjl_matrix(O.Format(D, 2, (3,), (128,), None, seed, qjl=True))
+    assert got.dtype == np.float32 and got.shape == (D, D)
+    mismatch = np.count_nonzero(got.astype(np.float64) != ref)
+    assert mismatch == 0  # an fp64 last-ulp difference could flip one fp32 rounding; none seen at these seeds
+
+
+def test_qjl_row_bytes_and_ledger():
+    H, Hq, W, bs = 8, 32, 64, 16
+    hc = _high(H, 64, 5)
+    t = tq.codec_host_tables(D, H, (3, 2), (64, 64), hc, 7, qjl=True)
+    f = O.Format(D, H, (3, 2), (64, 64), hc, 7, qjl=True)
+    assert t["row_bytes"] == O.row_bytes(f) == 40 + 16 + 4
+    lens = [0, 5, 64, 65, 1000, 4097]
+    ksp = {"group_bits": (3, 2), "group_size": (64, 64), "seed": 7, "high_coords": hc, "qjl": True}
+    vsp = {"group_bits": (3,), "group_size": (128,), "seed": 1, "high_coords": None}
+    nb = sum(-(-(L - min(W, L)) // bs) for L in lens) + 3
+    got = tq.host_ledger(H, ksp, vsp, lens, W, Hq, bs, nb)
+    ws = tq.decode_workspace_bytes(len(lens), Hq, H, max(lens), bs)
+    ref = O.byte_ledger(f, O.Format(D, H, (3,), (128,), None, 1), lens, W, bs, nb, workspace_bytes=ws)
+    for key in ("index_bytes", "norm_bytes", "transform_bytes", "page_pool_bytes", "metadata_bytes"):
+        assert got[key] == getattr(ref, key), key

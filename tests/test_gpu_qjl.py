@@ -1,0 +1,105 @@
+"""GPU parity of the QJL residual stage: pack rows and decode scores against the oracle."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import tq_oracle as O
+from quantized_paged_kv_pack_b200 import tq
+
+from helpers import D, DecodeProblem, codec_pair, random_kv, slice_format
+
+pytestmark = pytest.mark.gpu
+
+BOUNDARY_REL = 1e-5
+SIGN_REL = 1e-4  # a sign may differ only where |(S r)_i| is this small against |r| sqrt(d)
+
+
+def check_qjl_rows(rows, x, fmt, heads):
+    """GPU rows [N][H][row] against the oracle's QJL quantization of x [N][H][d]."""
+    compared = 0
+    for h in heads:
+        f1 = slice_format(fmt, h)
+        idx, n16, u, signs, g16 = O.quantize_qjl(x[:, h], f1, 0)
+        gidx, gn16, gsigns, gg16 = O.decode_rows(rows[:, h], f1)
+        assert np.array_equal(gn16.astype(np.float16).view(np.uint16), n16.astype(np.float16).view(np.uint16))
+        bad = np.any(gidx != idx, axis=-1)  # vectors with an index flip at a boundary
+        if bad.any():
+            margin = O.boundary_margin(u, f1)
+            flips = gidx != idx
+            assert np.all(margin[flips] <= BOUNDARY_REL), "index mismatch away from a codebook boundary"
+        ok = ~bad
+        # residual norms: fp16 of |r|, equal unless |r| sits at an fp16 rounding midpoint
+        gd = gg16[ok] != g16[ok]
+        if gd.any():
+            rel = np.abs(gg16[ok][gd] - g16[ok][gd]) / np.maximum(g16[ok][gd], 1e-30)
+            assert np.all(rel < 2e-3), "residual norm differs by more than one fp16 step"
+            assert gd.sum() <= max(2, 0.002 * ok.sum())
+        # signs: equal except where the projection is negligibly small
+        r = np.empty(u.shape)
+        perm = O.permutation(f1, 0)
+        start = 0
+        chat = np.empty(u.shape)
+        for b, size in zip(f1.group_bits, f1.group_size):
+            cb, _ = O.codebook(b, D)
+            chat[:, start:start + size] = cb[idx[:, start:start + size]]
+            start += size
+        r[:, perm] = u - chat
+        proj = r @ O.qjl_matrix(f1).T
+        scale = np.linalg.norm(r, axis=-1, keepdims=True) * math.sqrt(D)
+        diff = (gsigns != signs) & ok[:, None]
+        assert np.all(np.abs(proj[diff]) <= SIGN_REL * np.broadcast_to(scale, proj.shape)[diff]), \
+            "QJL sign mismatch away from zero"
+        compared += int(ok.sum())
+    return compared
+
+
+@pytest.mark.parametrize("kfmt", [((3,), (128,)), ((3, 2), (64, 64)), ((2,), (128,)), ((4, 3), (64, 64))])
+@pytest.mark.parametrize("T,H,bs", [(37, 2, 16), (300, 8, 32)])
+def test_qjl_pack_matches_oracle(kfmt, T, H, bs):
+    kc, kf = codec_pair(H, *kfmt, 31, qjl=True)
+    vc, vf = codec_pair(H, (3,), (128,), 32, qjl=True)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(T + H)
+    k, v = random_kv(T, H, gen)
+    nb = -(-T // bs) + 2
+    rng = np.random.default_rng(T)
+    slots = rng.permutation(nb * bs)[:T].astype(np.int64)
+    kp, vp = tq.page_pool(kc, nb, bs), tq.page_pool(vc, nb, bs)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, bs, d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    for pages, src, f in ((kp, k, kf), (vp, v, vf)):
+        x = src.float().cpu().numpy().astype(np.float64)
+        rows = np.stack([O.read_rows(pages.cpu().numpy(), slots // bs, h, slots % bs, f, bs) for h in range(H)], 1)
+        assert check_qjl_rows(rows, x, f, range(H)) > 0.9 * T * H
+
+
+@pytest.mark.parametrize("H,G,kfmt,vfmt", [(2, 4, ((3,), (128,)), ((3,), (128,))),
+                                           (8, 8, ((3, 2), (64, 64)), ((4, 3), (64, 64)))])
+def test_qjl_decode_matches_oracle(H, G, kfmt, vfmt):
+    """Decode with QJL keys (general kernel) against the oracle on the same GPU-written pages."""
+    lens = [1, 17, 300, 2100]
+    prob = DecodeProblem(lens, H, G, (kfmt[0], kfmt[1], 41), (vfmt[0], vfmt[1], 42), window=8, block_size=16,
+                         seed=H, kqjl=True)
+    out = prob.run()
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    rng = np.random.default_rng(G)
+    worst = 0.0
+    for b in range(prob.B):
+        for hq in rng.choice(prob.Hq, 4, replace=False):
+            ref = prob.oracle(b, int(hq))
+            worst = max(worst, float(np.abs(got[b, hq] - ref).max()))
+            assert np.abs(ref).max() > 0.3
+    assert worst <= 2e-3, worst
+
+
+def test_qjl_value_codec_is_rejected_by_decode():
+    prob = DecodeProblem([40], 2, 2, ((3,), (128,), 1), ((3,), (128,), 2), window=0, block_size=16, seed=3,
+                         vqjl=True)
+    with pytest.raises(tq.UnsupportedFormatError):
+        prob.run()
