@@ -42,6 +42,7 @@ class CodecSpec:
     group_size: tuple
     seed: int
     high_coords: Optional[np.ndarray] = None  # [H_kv][group_size[0]] int16, sorted
+    qjl: bool = False                         # QJL residual stage after the MSE groups
 
 
 @dataclass(frozen=True)
@@ -66,6 +67,7 @@ class Workload:
     lengths: str            # "fixed:N", "uniform:lo:hi", "loguniform:lo:hi"
     pool_slack: float = 1.0  # page pool = ceil(slack * needed) blocks, free blocks interleaved
     description: str = ""
+    k_qjl: bool = False      # keys carry the QJL residual stage
 
 
 WORKLOADS = {
@@ -96,6 +98,13 @@ WORKLOADS = {
         description="decode batch 256, 32 query / 8 KV heads, context log-uniform [512, 65536], "
                     "block 32, K 2.5-bit (32 channels at 4 bits + 96 at 2 bits), V uniform 3-bit, "
                     "128-token bf16 window, fragmented page pool"),
+    "decode_llama8b_3p5bit_qjl": Workload(
+        "decode_llama8b_3p5bit_qjl", "decode", 1006, 16, 32, 8, 128, 16, 128,
+        (3, 2), (64, 64), (4, 3), (64, 64), 61, 62, 8, True, "fixed:16384", k_qjl=True,
+        description="decode batch 16, 32 query / 8 KV heads (Llama-3.1-8B), context 16384, block 16, "
+                    "K 2.5-bit MSE (64 channels at 3 bits + 64 at 2) plus the 1-bit QJL residual stage "
+                    "(3.5 bits per channel), V 3.5-bit, 128-token bf16 window; QJL keys run on the general "
+                    "CUDA-core kernel")
 }
 
 
@@ -107,12 +116,12 @@ def codec_specs(w: Workload):
     """(K spec, V spec). High channel sets are seeded, sorted, independent for K and V."""
     rng = _rng(w.seed * 7 + 3)
     specs = []
-    for bits, sizes, seed in ((w.k_bits, w.k_sizes, w.k_seed), (w.v_bits, w.v_sizes, w.v_seed)):
+    for bits, sizes, seed, qjl in ((w.k_bits, w.k_sizes, w.k_seed, w.k_qjl), (w.v_bits, w.v_sizes, w.v_seed, False)):
         high = None
         if len(bits) == 2:
             high = np.stack([np.sort(rng.choice(w.head_dim, sizes[0], replace=False))
                              for _ in range(w.num_kv_heads)]).astype(np.int16)
-        specs.append(CodecSpec(tuple(bits), tuple(sizes), seed, high))
+        specs.append(CodecSpec(tuple(bits), tuple(sizes), seed, high, qjl))
     return specs[0], specs[1]
 
 
