@@ -65,6 +65,17 @@ R16 QJL residual stage (TurboQuant "Design" page, "Recipe Strategy": row
     E over S of its product with q equals q . x when g is exact. In a
     sub-page the sign bytes follow the index bytes of each row and the norm
     area holds (norm, residual norm) per row.
+R17 Group-wise rotation (SURVEY's original-domain reading of the high/low
+    recipe; "Recipe Strategy": the high channel set comes from calibration
+    metadata). With groupwise set, group 0 is the set of ORIGINAL channels
+    high_coords[h] (ascending) and group 1 the other channels (ascending).
+    Each group is rotated on its own: y_g = B_g (s[ch_g] * x[ch_g]), B_g the
+    block-diagonal of orthonormal natural-order Hadamard blocks of the
+    power-of-two sizes that make up |g|, largest first (96 = 64 + 32), s the
+    codec's sign vector indexed by channel. Each group has its own norm
+    n_g = |x[ch_g]| (fp16) and codebook (Lloyd-Max for dimension |g|);
+    u_g = y_g / n_g. Row = [group-0 indices][group-1 indices][n_0][n_1];
+    the norm area of a sub-page holds (n_0, n_1) per row.
 R14 Boundary-token preservation: the first S and the last W tokens of a
     sequence stay dense, the ones between are packed (boundary_dense_tokens).
     Attention is a sum over keys, so the dense ones may sit in one buffer in
@@ -84,7 +95,8 @@ from scipy.special import betainc, betaincinv, gammaln
 __all__ = [
     "Format", "coord_density_const", "coord_cdf", "coord_tail", "cell_mass",
     "cell_first_moment", "cell_second_moment", "lloyd_max", "codebook", "boundary_dense_tokens",
-    "qjl_matrix", "quantize_qjl", "norm_bytes", "mse_index_bytes",
+    "qjl_matrix", "quantize_qjl", "norm_bytes", "mse_index_bytes", "group_rotation", "group_channels",
+    "pow2_blocks",
     "splitmix64", "hadamard_signs", "hadamard_matrix", "rotate", "unrotate",
     "permutation", "position_bits", "row_bytes", "index_bytes",
     "quantize", "encode_rows", "decode_rows", "dequantize_rows",
@@ -113,9 +125,12 @@ class Format:
     high_coords: Optional[np.ndarray] = field(default=None, compare=False)
     seed: int = 0
     qjl: bool = False
+    groupwise: bool = False
 
     def __post_init__(self):
         d = self.head_dim
+        if self.groupwise and (len(self.group_bits) != 2 or self.qjl):
+            raise ValueError("group-wise rotation needs two groups and no QJL stage")
         if len(self.group_bits) != len(self.group_size) or len(self.group_bits) not in (1, 2):
             raise ValueError("one or two channel groups")
         if sum(self.group_size) != d:
@@ -353,8 +368,41 @@ def index_bytes(fmt: Format) -> int:
 
 
 def norm_bytes(fmt: Format) -> int:
-    """fp16 norm, then the fp16 residual norm with QJL (R16)."""
-    return 4 if fmt.qjl else 2
+    """fp16 norm, then the fp16 residual norm with QJL (R16) or the group-1 norm (R17)."""
+    return 4 if (fmt.qjl or fmt.groupwise) else 2
+
+
+def pow2_blocks(n: int):
+    """The power-of-two sizes that make up n, largest first (R17)."""
+    return [1 << k for k in range(n.bit_length() - 1, -1, -1) if n >> k & 1]
+
+
+def group_channels(fmt: Format, head: int):
+    """(channels of group 0, channels of group 1), ascending (R17)."""
+    d = fmt.head_dim
+    high = np.asarray(fmt.high_coords[head], dtype=np.int64)
+    return high, np.setdiff1d(np.arange(d), high)
+
+
+def group_rotation(fmt: Format, head: int) -> np.ndarray:
+    """R (d x d) with (R x)[p] = the rotated coordinate at packed position p (R17).
+
+    Rows 0 .. n0-1 are group 0's B_0 diag(s[ch_0]) applied to x[ch_0], rows n0 ..
+    d-1 group 1's; R is orthogonal.
+    """
+    d = fmt.head_dim
+    s = hadamard_signs(fmt.seed, d)
+    R = np.zeros((d, d))
+    row = 0
+    for ch in group_channels(fmt, head):
+        col = 0
+        for m in pow2_blocks(len(ch)):
+            blk = hadamard_matrix(m) / math.sqrt(m)
+            cols = ch[col:col + m]
+            R[row:row + m, cols] = blk * s[cols][None, :]
+            row += m
+            col += m
+    return R
 
 
 def row_bytes(fmt: Format) -> int:
@@ -371,6 +419,8 @@ def quantize(x, fmt: Format, head: int):
     """
     x = np.asarray(x, dtype=np.float64)
     d = fmt.head_dim
+    if fmt.groupwise:
+        return _quantize_groupwise(x, fmt, head)
     n = np.sqrt(np.sum(x * x, axis=-1))
     y = rotate(x, hadamard_signs(fmt.seed, d))
     safe = np.where(n > 0, n, 1.0)
@@ -384,6 +434,26 @@ def quantize(x, fmt: Format, head: int):
         start += size
     n16 = n if 16 in fmt.group_bits else fp16_round(n)
     return idx, n16, u
+
+
+def _quantize_groupwise(x, fmt: Format, head: int):
+    """quantize() under R17: n16 is [..., 2] (the two group norms, fp16-rounded)."""
+    d = fmt.head_dim
+    y = x @ group_rotation(fmt, head).T          # packed order
+    idx = np.empty(y.shape, dtype=np.int64)
+    u = np.empty(y.shape)
+    norms = []
+    start = 0
+    for (b, size), ch in zip(zip(fmt.group_bits, fmt.group_size), group_channels(fmt, head)):
+        n = np.sqrt(np.sum(x[..., ch] ** 2, axis=-1))
+        safe = np.where(n > 0, n, 1.0)
+        seg = np.where(n[..., None] > 0, y[..., start:start + size] / safe[..., None], 0.0)
+        _, beta = codebook(b, size)
+        idx[..., start:start + size] = np.searchsorted(beta, seg, side="left")
+        u[..., start:start + size] = seg
+        norms.append(fp16_round(n))
+        start += size
+    return idx, np.stack(norms, axis=-1), u
 
 
 QJL_SEED_XOR = 0x51534A4C00000001  # "QSJL": the S stream is independent of the sign stream
@@ -440,7 +510,7 @@ def boundary_margin(u, fmt: Format):
     out = np.empty(u.shape)
     start = 0
     for b, size in zip(fmt.group_bits, fmt.group_size):
-        _, beta = codebook(b, d)
+        _, beta = codebook(b, size if fmt.groupwise else d)
         seg = u[..., start:start + size, None]
         dist = np.abs(seg - beta) / np.maximum(np.abs(beta), 1.0 / math.sqrt(d))
         out[..., start:start + size] = dist.min(axis=-1)
@@ -471,6 +541,10 @@ def encode_rows(idx, n16, fmt: Format, signs=None, g16=None) -> np.ndarray:
         if signs is None or g16 is None:
             raise ValueError("a QJL format needs the signs and the residual norm")
         parts.append(np.packbits(np.asarray(signs, dtype=np.uint8), axis=-1, bitorder="little"))
+    if fmt.groupwise:
+        n16 = np.asarray(n16, dtype=np.float64)
+        parts += [_fp16_bytes(n16[..., 0]), _fp16_bytes(n16[..., 1])]
+        return np.concatenate(parts, axis=-1)
     parts.append(_fp16_bytes(n16))
     if fmt.qjl:
         parts.append(_fp16_bytes(g16))
@@ -495,6 +569,9 @@ def decode_rows(rows, fmt: Format):
         nb = fmt.head_dim // 8
         signs = np.unpackbits(rows[..., off:off + nb], axis=-1, bitorder="little").astype(np.int64)
         off += nb
+    if fmt.groupwise:
+        n16 = rows[..., off:off + 4].copy().view(np.float16).reshape(lead + (2,)).astype(np.float64)
+        return np.concatenate(idx, axis=-1), n16
     n16 = rows[..., off:off + 2].copy().view(np.float16).reshape(lead).astype(np.float64)
     if fmt.qjl:
         g16 = rows[..., off + 2:off + 4].copy().view(np.float16).reshape(lead).astype(np.float64)
@@ -513,9 +590,14 @@ def dequantize_rows(idx, n16, fmt: Format, head: int, signs=None, g16=None):
     vals = np.empty(idx.shape, dtype=np.float64)
     start = 0
     for b, size in zip(fmt.group_bits, fmt.group_size):
-        c, _ = codebook(b, d)
+        c, _ = codebook(b, size if fmt.groupwise else d)
         vals[..., start:start + size] = c[idx[..., start:start + size]]
+        if fmt.groupwise:  # R17: each group scaled by its own norm, then R^T back to the channels
+            gi = 0 if start == 0 else 1
+            vals[..., start:start + size] *= np.asarray(n16, dtype=np.float64)[..., gi:gi + 1]
         start += size
+    if fmt.groupwise:
+        return vals @ group_rotation(fmt, head)
     rot = np.empty_like(vals)
     rot[..., permutation(fmt, head)] = vals
     if fmt.qjl:

@@ -686,3 +686,86 @@ def test_qjl_residual_and_signs_follow_the_definitions():
     est = O.dequantize_rows(i2, n2, fmt, 0, s2, g2) @ q
     err = est - xs @ q
     assert abs(err.mean()) < 4 * err.std(ddof=1) / math.sqrt(len(err))
+
+
+# ---- group-wise rotation (R17) ------------------------------------------------------------
+
+def _gw_format(bits=(4, 2), sizes=(32, 96), H=2, seed=9):
+    rng = np.random.default_rng(seed)
+    high = np.stack([np.sort(rng.choice(D, sizes[0], replace=False)) for _ in range(H)])
+    return O.Format(D, H, bits, sizes, high, seed, groupwise=True)
+
+
+def test_groupwise_rotation_is_blockwise_orthogonal():
+    """R is orthogonal, keeps each group's channels inside its own rows, and its
+    power-of-two blocks are the textbook Sylvester matrices (scipy) with signs."""
+    f = _gw_format()
+    R = O.group_rotation(f, 1)
+    assert np.allclose(R @ R.T, np.eye(D), atol=1e-14)
+    g0, g1 = O.group_channels(f, 1)
+    assert np.all(R[:32][:, g1] == 0) and np.all(R[32:][:, g0] == 0)
+    s = O.hadamard_signs(f.seed, D)
+    blocks = [(0, g0[:32], 32), (32, g1[:64], 64), (96, g1[64:], 32)]  # 96 = 64 + 32
+    for row, cols, m in blocks:
+        ref = scipy.linalg.hadamard(m) / math.sqrt(m) * s[cols][None, :]
+        assert np.allclose(R[row:row + m][:, cols], ref, atol=1e-15)
+    assert O.pow2_blocks(112) == [64, 32, 16] and O.pow2_blocks(48) == [32, 16]
+
+
+def test_groupwise_per_group_distortion_matches_dimension_n_g():
+    """For Gaussian x each group's unit vector is uniform on its own sphere, so the
+    coordinate error equals the Lloyd-Max distortion for dimension |g| (not d)."""
+    f = _gw_format((4, 2), (32, 96), H=1, seed=3)
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((20000, D))
+    idx, n16, u = O.quantize(x, f, 0)
+    start = 0
+    for b, n in zip(f.group_bits, f.group_size):
+        c, beta = O.codebook(b, n)
+        e = np.concatenate(([-1.0], beta, [1.0]))
+        per = (O.cell_second_moment(e[:-1], e[1:], n) - 2 * c * O.cell_first_moment(e[:-1], e[1:], n)
+               + c * c * O.cell_mass(e[:-1], e[1:], n)).sum()
+        err = ((u[:, start:start + n] - c[idx[:, start:start + n]]) ** 2).sum(axis=1)
+        sigma = err.std() / math.sqrt(len(err))
+        assert abs(err.mean() - n * per) < 4 * sigma
+        # the same codebook for dimension d would be measurably off for the small group
+        if n == 32:
+            c128, beta128 = O.codebook(b, D)
+            e128 = np.concatenate(([-1.0], beta128, [1.0]))
+            per128 = (O.cell_second_moment(e128[:-1], e128[1:], n) - 2 * c128 * O.cell_first_moment(e128[:-1], e128[1:], n)
+                      + c128 * c128 * O.cell_mass(e128[:-1], e128[1:], n)).sum()
+            assert per128 > per * 1.01
+        start += n
+    # norms: one fp16 norm per group, of that group's channels
+    g0, g1 = O.group_channels(f, 0)
+    assert np.array_equal(n16[:, 0], O.fp16_round(np.linalg.norm(x[:, g0], axis=1)))
+    assert np.array_equal(n16[:, 1], O.fp16_round(np.linalg.norm(x[:, g1], axis=1)))
+
+
+def test_groupwise_row_layout_and_reconstruction():
+    """Row = [group-0 indices][group-1 indices][n_0][n_1]; keys rebuild from the rows as
+    each group's norm times R^T of its centroids."""
+    f = _gw_format((3, 2), (64, 64), H=1, seed=8)
+    rng = np.random.default_rng(6)
+    x = O.bf16_round(rng.standard_normal((7, D)) * 2)
+    idx, n16, u = O.quantize(x, f, 0)
+    rows = O.encode_rows(idx, n16, f)
+    assert rows.shape[-1] == O.row_bytes(f) == 24 + 16 + 4
+    for t in range(7):
+        assert struct.unpack("<e", bytes(rows[t, 40:42]))[0] == n16[t, 0]
+        assert struct.unpack("<e", bytes(rows[t, 42:44]))[0] == n16[t, 1]
+        bit = lambda k: (int(rows[t, k // 8]) >> (k % 8)) & 1
+        pos = 0
+        for p in range(D):
+            b = 3 if p < 64 else 2
+            assert sum(bit(pos + j) << j for j in range(b)) == idx[t, p]
+            pos += b
+    back_idx, back_n = O.decode_rows(rows, f)
+    xr = O.dequantize_rows(back_idx, back_n, f, 0)
+    c0, _ = O.codebook(3, 64)
+    c1, _ = O.codebook(2, 64)
+    chat = np.concatenate((c0[idx[:, :64]] * n16[:, :1], c1[idx[:, 64:]] * n16[:, 1:]), axis=1)
+    assert np.allclose(xr, chat @ O.group_rotation(f, 0), atol=1e-12)
+    # and close to x: each group within its codebook's error
+    rel = np.linalg.norm(xr - x, axis=1) / np.linalg.norm(x, axis=1)
+    assert np.all(rel < 0.5)
