@@ -83,6 +83,16 @@ typedef enum {
  *                row stands for is n R^T (c + sqrt(pi/2)/d |r| S^T z), z = 2 bits
  *                - 1: its product with q is the unbiased QJL estimate of q.x.
  *                Decode accepts QJL for K only.
+ * groupwise      0, or 1 for group-wise rotation with per-group norms (two
+ *                groups, no QJL): group 0 is the set of ORIGINAL channels
+ *                high_coords[h] and group 1 the other channels, each ascending;
+ *                each group is rotated on its own, y_g = B_g (s[ch] * x[ch]),
+ *                B_g the block-diagonal of orthonormal natural-order Hadamard
+ *                blocks of the power-of-two sizes that make up the group size,
+ *                largest first (96 = 64 + 32); each group has its own fp16 norm
+ *                and a Lloyd-Max codebook for its own dimension. Row: the two
+ *                index bitstreams, then the two norms (norm area: 4 bytes per
+ *                row). Pack and decode run it on the general kernels.
  */
 typedef struct {
     int32_t head_dim;
@@ -93,6 +103,7 @@ typedef struct {
     const int16_t* high_coords;
     uint64_t hadamard_seed;
     int32_t qjl;
+    int32_t groupwise;
 } tq_format_desc;
 
 typedef struct tq_codec tq_codec; /* opaque, immutable after tq_make_codec */

@@ -229,6 +229,9 @@ tq_status validate_desc(const tq_format_desc* d) {
     }
     if (total != d->head_dim) return fail(TQ_ERR_VALUE, "group sizes must sum to head_dim");
     if (d->qjl != 0 && d->qjl != 1) return fail(TQ_ERR_VALUE, "qjl must be 0 or 1");
+    if (d->groupwise != 0 && d->groupwise != 1) return fail(TQ_ERR_VALUE, "groupwise must be 0 or 1");
+    if (d->groupwise && (d->n_groups != 2 || d->qjl))
+        return fail(TQ_ERR_VALUE, "group-wise rotation needs two groups and no QJL stage");
     if (d->n_groups == 1) {
         if (d->high_coords) return fail(TQ_ERR_VALUE, "high_coords given for a one-group format");
     } else {
@@ -258,7 +261,8 @@ tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c) {
     }
     for (int g = 0; g < 2; ++g) {
         if (g < desc->n_groups) {
-            const Codebook& cb = codebook(desc->group_bits[g], d);
+            // group-wise: the Lloyd-Max codebook of the group's own dimension
+            const Codebook& cb = codebook(desc->group_bits[g], desc->groupwise ? desc->group_size[g] : d);
             std::memcpy(c->cent16[g], cb.c16, sizeof(cb.c16));
             std::memcpy(c->cent[g], cb.c, sizeof(cb.c));
             std::memcpy(c->bound[g], cb.b, sizeof(cb.b));
@@ -291,11 +295,40 @@ tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c) {
     }
     int bytes = 0;
     for (int g = 0; g < desc->n_groups; ++g) bytes += desc->group_bits[g] * desc->group_size[g] / 8;
-    const int sign_bytes = desc->qjl ? d / 8 : 0, norm_bytes = desc->qjl ? 4 : 2;
+    const int sign_bytes = desc->qjl ? d / 8 : 0, norm_bytes = (desc->qjl || desc->groupwise) ? 4 : 2;
     c->index_bytes = bytes + sign_bytes;
     c->row_bytes = c->index_bytes + norm_bytes;
     c->qjl_s.clear();
     if (desc->qjl) qjl_matrix(desc->hadamard_seed, d, c->qjl_s);
+    c->rot_t.clear();
+    if (desc->groupwise) {
+        // R_h: rows = packed positions, columns = channels; perm[h] lists group 0's
+        // channels then group 1's, and each group's rows are its Hadamard blocks.
+        c->rot_t.assign(static_cast<size_t>(H) * d * d, 0.0f);
+        for (int h = 0; h < H; ++h) {
+            const int16_t* ch = c->perm.data() + static_cast<size_t>(h) * d;
+            float* rt = c->rot_t.data() + static_cast<size_t>(h) * d * d;
+            int row = 0;
+            for (int g = 0; g < 2; ++g) {
+                const int n = desc->group_size[g];
+                const int16_t* cg = ch + (g ? desc->group_size[0] : 0);
+                int col = 0;
+                for (int k = 30; k >= 0; --k) {
+                    const int m = 1 << k;
+                    if (!(n & m)) continue;
+                    const double inv = 1.0 / std::sqrt(static_cast<double>(m));
+                    for (int a = 0; a < m; ++a)
+                        for (int b = 0; b < m; ++b) {
+                            const int j = cg[col + b];
+                            const double hv = (__builtin_popcount(static_cast<unsigned>(a & b)) & 1) ? -inv : inv;
+                            rt[static_cast<size_t>(j) * d + row + a] = static_cast<float>(hv * c->sign[j]);
+                        }
+                    row += m;
+                    col += m;
+                }
+            }
+        }
+    }
     DevCodec& v = c->dev;
     v.num_heads = H;
     v.n_groups = desc->n_groups;
@@ -315,6 +348,8 @@ tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c) {
     v.mse_bytes = bytes;
     v.norm_bytes = norm_bytes;
     v.qjl_st = nullptr;  // set by tq_make_codec
+    v.groupwise = desc->groupwise;
+    v.rot_t = nullptr;   // set by tq_make_codec
     return TQ_OK;
 }
 
@@ -397,7 +432,8 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     const size_t n_perm = static_cast<size_t>(H) * d * sizeof(int16_t);
     const size_t off_s = (n_sign + 2 * n_cent + 2 * n_perm + 15) / 16 * 16;
     const size_t n_s = c->qjl_s.size() * sizeof(float);
-    const size_t total = off_s + n_s;
+    const size_t off_r = (off_s + n_s + 15) / 16 * 16, n_r = c->rot_t.size() * sizeof(float);
+    const size_t total = off_r + n_r;
     std::vector<char> host(total);
     char* p = host.data();
     std::memcpy(p, c->sign, n_sign);
@@ -410,6 +446,7 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
         for (int i = 0; i < d; ++i)
             for (int j = 0; j < d; ++j) st[static_cast<size_t>(j) * d + i] = c->qjl_s[static_cast<size_t>(i) * d + j];
     }
+    if (n_r) std::memcpy(p + off_r, c->rot_t.data(), n_r);
     if (cudaGetDevice(&c->device) != cudaSuccess || cudaMalloc(&c->d_tables, total) != cudaSuccess) {
         cudaGetLastError();
         delete c;
@@ -428,6 +465,7 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     c->dev.perm = reinterpret_cast<const int16_t*>(base + n_sign + 2 * n_cent);
     c->dev.pos = reinterpret_cast<const int16_t*>(base + n_sign + 2 * n_cent + n_perm);
     c->dev.qjl_st = n_s ? reinterpret_cast<const float*>(base + off_s) : nullptr;
+    c->dev.rot_t = n_r ? reinterpret_cast<const float*>(base + off_r) : nullptr;
     *out = c;
     return TQ_OK;
 }
@@ -474,7 +512,7 @@ tq_status tq_byte_ledger(const tq_format_desc* kdesc, const tq_format_desc* vdes
     tq_ledger r{};
     r.dense_bytes = 2 * 2 * H * d * total;
     r.index_bytes = packed * H * (kc.index_bytes + vc.index_bytes);
-    r.norm_bytes = packed * H * ((kdesc->qjl ? 4 : 2) + (vdesc->qjl ? 4 : 2));
+    r.norm_bytes = packed * H * ((kdesc->qjl || kdesc->groupwise ? 4 : 2) + (vdesc->qjl || vdesc->groupwise ? 4 : 2));
     for (const tq_format_desc* desc : {kdesc, vdesc})
         for (int g = 0; g < desc->n_groups; ++g) {
             int64_t L = int64_t(1) << desc->group_bits[g];

@@ -107,6 +107,19 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
             for (int i = 0; i < 4; ++i) qs[g][4 * lane + i] = z[i] * a.scale_log2;
             continue;
         }
+        if (a.kc.groupwise) {
+            // q_r = R_h q (packed positions; R_h orthonormal), lane l: positions l + 32k
+            float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const float* rt = a.kc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim + lane;
+            for (int j = 0; j < kHeadDim; ++j) {
+                const float qj = __shfl_sync(kFull, z[j & 3], j >> 2);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) y[k] = fmaf(__ldg(rt + j * kHeadDim + 32 * k), qj, y[k]);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) qs[g][lane + 32 * k] = y[k] * a.scale_log2;
+            continue;
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) z[i] *= a.kc.sign[4 * lane + i];
         {
@@ -181,6 +194,18 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
             }
             nk = row_norm(ksub, a.kc, bs, off);
             nv = row_norm(vsub, a.vc, bs, off);
+            if (a.kc.groupwise) {  // per-group norms: fold each position's norm into its centroid
+                const float nk1 = row_norm(ksub, a.kc, bs, off, 1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) kv[i] *= (4 * lane + i >= a.kc.pos0[1]) ? nk1 : nk;
+                nk = 1.0f;
+            }
+            if (a.vc.groupwise) {
+                const float nv1 = row_norm(vsub, a.vc, bs, off, 1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) vv[i] *= (4 * lane + i >= a.vc.pos0[1]) ? nv1 : nv;
+                nv = 1.0f;
+            }
             if (qjl) {
                 // sign bits 4l .. 4l+3 of the QJL stream (after the index bitstreams)
                 const unsigned bits = (krow[a.kc.mse_bytes + (lane >> 1)] >> (4 * (lane & 1))) & 0xFu;
@@ -274,15 +299,24 @@ __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, c
             win = rec(max_splits)[2 + j] * f;
         }
     }
-    y[vc.perm[h * kHeadDim + j]] = rot;  // back to rotated coordinate order
-    __syncthreads();
-    for (int len = 1; len < kHeadDim; len <<= 1) {  // Walsh-Hadamard, natural order
-        float mine = y[j], other = y[j ^ len];
+    float x;
+    if (vc.groupwise) {
+        y[j] = rot;  // packed positions
         __syncthreads();
-        y[j] = (j & len) ? (other - mine) : (mine + other);
+        const float* rt = vc.rot_t + (static_cast<int64_t>(h) * kHeadDim + j) * kHeadDim;  // R_h^T row j
+        x = 0.0f;
+        for (int p = 0; p < kHeadDim; ++p) x = fmaf(rt[p], y[p], x);
+    } else {
+        y[vc.perm[h * kHeadDim + j]] = rot;  // back to rotated coordinate order
         __syncthreads();
+        for (int len = 1; len < kHeadDim; len <<= 1) {  // Walsh-Hadamard, natural order
+            float mine = y[j], other = y[j ^ len];
+            __syncthreads();
+            y[j] = (j & len) ? (other - mine) : (mine + other);
+            __syncthreads();
+        }
+        x = vc.sign[j] * y[j] * 0.08838834764831845f;
     }
-    const float x = vc.sign[j] * y[j] * 0.08838834764831845f;
     out[(static_cast<int64_t>(b) * num_q_heads + hq) * kHeadDim + j] = Ls > 0.0f ? (x + win) / Ls : 0.0f;
 }
 
@@ -385,9 +419,9 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     // Tensor-core kernel for the formats it is instantiated for (block sizes a
     // multiple of 16); the general kernel covers every other valid format.
     // TQ_DECODE_KERNEL=general selects the general kernel (for cross-checks).
-    // QJL keys (the sign-bit score term) run on the general kernel.
+    // QJL keys (the sign-bit score term) and group-wise codecs run on the general kernel.
     const char* force = std::getenv("TQ_DECODE_KERNEL");
-    if (!(force && std::string(force) == "general") && !kc->desc.qjl) {
+    if (!(force && std::string(force) == "general") && !kc->desc.qjl && !kc->desc.groupwise && !vc->desc.groupwise) {
         st = launch_decode_mma(a, kc, vc, plan.group, stream);
         if (st == TQ_OK) return finish(s, d_err, "decode partials");
         if (st != TQ_ERR_UNSUPPORTED) return st;

@@ -32,6 +32,8 @@ struct DevCodec {
     int32_t mse_bytes;      // bytes of the index bitstreams
     int32_t norm_bytes;     // 2, or 4 with QJL (norm, residual norm)
     const float* qjl_st;    // QJL: S transposed, [128][128] (entry j * 128 + i = S[i][j])
+    int32_t groupwise;      // 1: group-wise rotation with per-group norms
+    const float* rot_t;     // group-wise: R transposed per head, [H][128][128] (entry (h, j, p) = R_h[p][j])
 };
 
 // Arguments of the decode kernels (device pointers; see tq_decode_paged).
@@ -72,6 +74,7 @@ struct tq_codec {
     std::vector<int16_t> perm;     // [H][d]
     std::vector<int16_t> pos;      // [H][d]
     std::vector<float> qjl_s;      // QJL: S, [d][d] row-major
+    std::vector<float> rot_t;      // group-wise: R transposed per head, [H][d][d]
     int32_t row_bytes = 0;
     int32_t index_bytes = 0;
     int device = 0;

@@ -72,8 +72,15 @@ __device__ __forceinline__ unsigned short norm_fp16_bits(const float (&x)[4], fl
 // head h and writes its row at `offset` of the sub-page `sub` (block_size
 // rows). idx_buf: 128 bytes, r_buf: 128 floats of shared scratch owned by the
 // warp (r_buf is used by the QJL stage only).
+__device__ void pack_vector_groupwise(const DevCodec& c, const float (&x)[4], int h, uint8_t* sub, int64_t offset,
+                                      int block_size, uint8_t* idx_buf, float* x_buf, int lane);
+
 __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8_t* sub, int64_t offset,
                             int block_size, uint8_t* idx_buf, float* r_buf, int lane) {
+    if (c.groupwise) {
+        pack_vector_groupwise(c, x, h, sub, offset, block_size, idx_buf, r_buf, lane);
+        return;
+    }
     float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
     float n32 = sqrtf(ss);
     const unsigned short n16 = norm_fp16_bits(x, ss, n32);
@@ -151,6 +158,71 @@ __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8
         if (lane == 0) nrm[1] = g16;
     }
     if (lane == 0) nrm[0] = n16;
+    __syncwarp();
+}
+
+// Group-wise rotation (two groups of original channels, each rotated on its
+// own by the per-head matrix R_h, rows = packed positions): y = R_h x, one fp16
+// norm per group from the exact squares of its channels, u_p = y_p / n_g(p).
+// Lane l handles packed positions l, l+32, l+64, l+96.
+__device__ void pack_vector_groupwise(const DevCodec& c, const float (&x)[4], int h, uint8_t* sub, int64_t offset,
+                                      int block_size, uint8_t* idx_buf, float* x_buf, int lane) {
+    const int n0 = c.pos0[1];  // group 0 occupies packed positions [0, n0)
+    float xm[2][4];            // the lane's channels, masked to each group
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int j = 4 * lane + i;
+        x_buf[j] = x[i];
+        const bool in0 = c.pos[h * kHeadDim + j] < n0;
+        xm[0][i] = in0 ? x[i] : 0.0f;
+        xm[1][i] = in0 ? 0.0f : x[i];
+    }
+    unsigned short n16[2];
+    float n32[2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        const float ss = warp_sum(xm[g][0] * xm[g][0] + xm[g][1] * xm[g][1] + xm[g][2] * xm[g][2] + xm[g][3] * xm[g][3]);
+        n32[g] = sqrtf(ss);
+        n16[g] = norm_fp16_bits(xm[g], ss, n32[g]);
+    }
+    __syncwarp();
+    float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const float* rt = c.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim + lane;
+    for (int j = 0; j < kHeadDim; ++j) {
+        const float xj = x_buf[j];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) y[k] = fmaf(__ldg(rt + j * kHeadDim + 32 * k), xj, y[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int p = lane + 32 * k;
+        const int g = p >= n0 ? 1 : 0;
+        const float u = n32[g] > 0.0f ? y[k] / n32[g] : 0.0f;
+        const int levels = 1 << c.bits[g];
+        int idx = 0;
+        for (int q = 0; q < levels - 1; ++q) idx += (c.bound[g * 16 + q] < u) ? 1 : 0;
+        idx_buf[p] = static_cast<uint8_t>(idx);
+    }
+    __syncwarp();
+    const int half_words = c.mse_bytes / 2;
+    unsigned word = 0;
+    if (lane < half_words) {
+        for (int i = 0; i < 16; ++i) {
+            const int B = 16 * lane + i;
+            const int g = B >= 8 * c.byte_off[1] ? 1 : 0;
+            const int lb = B - 8 * c.byte_off[g];
+            const int b = c.bits[g];
+            const int q = lb / b, r = lb - q * b;
+            word |= ((idx_buf[c.pos0[g] + q] >> r) & 1u) << i;
+        }
+    }
+    uint16_t* dst = reinterpret_cast<uint16_t*>(sub + offset * c.index_bytes);
+    if (lane < half_words) dst[lane] = static_cast<uint16_t>(word);
+    uint16_t* nrm = reinterpret_cast<uint16_t*>(sub + block_size * c.index_bytes + c.norm_bytes * offset);
+    if (lane == 0) {
+        nrm[0] = n16[0];
+        nrm[1] = n16[1];
+    }
     __syncwarp();
 }
 

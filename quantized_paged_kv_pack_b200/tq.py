@@ -42,7 +42,7 @@ class _FormatDesc(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("n_groups", ctypes.c_int32),
                 ("group_bits", ctypes.c_int32 * 2), ("group_size", ctypes.c_int32 * 2),
                 ("high_coords", ctypes.POINTER(ctypes.c_int16)), ("hadamard_seed", ctypes.c_uint64),
-                ("qjl", ctypes.c_int32)]
+                ("qjl", ctypes.c_int32), ("groupwise", ctypes.c_int32)]
 
 
 class _Ledger(ctypes.Structure):
@@ -109,7 +109,7 @@ def _check(status: int):
     raise TQCudaError(msg or f"tq status {status}")
 
 
-def _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl=False):
+def _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl=False, groupwise=False):
     bits, sizes = tuple(group_bits), tuple(group_size)
     d = _FormatDesc()
     d.head_dim, d.num_kv_heads, d.n_groups = head_dim, num_kv_heads, len(bits)
@@ -123,12 +123,14 @@ def _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl
         d.high_coords = keep.ctypes.data_as(ctypes.POINTER(ctypes.c_int16))
     d.hadamard_seed = int(seed) & ((1 << 64) - 1)
     d.qjl = 1 if qjl else 0
+    d.groupwise = 1 if groupwise else 0
     return d, keep
 
 
-def codec_host_tables(head_dim, num_kv_heads, group_bits, group_size, high_coords=None, seed=0, qjl=False):
+def codec_host_tables(head_dim, num_kv_heads, group_bits, group_size, high_coords=None, seed=0, qjl=False,
+                      groupwise=False):
     """Host-side codec tables (no CUDA call): codebooks, signs, permutation, row bytes."""
-    d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl)
+    d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl, groupwise)
     c16 = np.zeros((2, 16), np.uint16)
     bnd = np.zeros((2, 15), np.float32)
     sg = np.zeros(head_dim, np.int8)
@@ -153,12 +155,13 @@ class Codec:
     """A device codec (tq_make_codec); immutable, freed on close()."""
 
     def __init__(self, num_kv_heads: int, group_bits: Sequence[int], group_size: Sequence[int],
-                 high_coords=None, seed: int = 0, head_dim: int = HEAD_DIM, qjl: bool = False):
+                 high_coords=None, seed: int = 0, head_dim: int = HEAD_DIM, qjl: bool = False,
+                 groupwise: bool = False):
         self.head_dim, self.num_kv_heads = head_dim, num_kv_heads
         self.group_bits, self.group_size, self.seed = tuple(group_bits), tuple(group_size), seed
-        self.qjl = bool(qjl)
+        self.qjl, self.groupwise = bool(qjl), bool(groupwise)
         self.high_coords = None if high_coords is None else np.asarray(high_coords, dtype=np.int16)
-        d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl)
+        d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, qjl, groupwise)
         h = _VP()
         _check(lib().tq_make_codec(ctypes.byref(d), ctypes.byref(h)))
         del keep
@@ -173,7 +176,7 @@ class Codec:
 
     def desc(self):
         return _desc(self.head_dim, self.num_kv_heads, self.group_bits, self.group_size, self.high_coords, self.seed,
-                     self.qjl)
+                     self.qjl, self.groupwise)
 
     def close(self):
         if getattr(self, "_h", None) is not None:
@@ -421,9 +424,9 @@ def host_ledger(num_kv_heads, kspec: dict, vspec: dict, seq_lens, window, num_q_
     lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
     max_seq_len = int(lens.max()) if max_seq_len is None and len(lens) else int(max_seq_len or 0)
     kd, kkeep = _desc(HEAD_DIM, num_kv_heads, kspec["group_bits"], kspec["group_size"], kspec.get("high_coords"),
-                      kspec.get("seed", 0), kspec.get("qjl", False))
+                      kspec.get("seed", 0), kspec.get("qjl", False), kspec.get("groupwise", False))
     vd, vkeep = _desc(HEAD_DIM, num_kv_heads, vspec["group_bits"], vspec["group_size"], vspec.get("high_coords"),
-                      vspec.get("seed", 0), vspec.get("qjl", False))
+                      vspec.get("seed", 0), vspec.get("qjl", False), vspec.get("groupwise", False))
     r = _Ledger()
     _check(lib().tq_byte_ledger(ctypes.byref(kd), ctypes.byref(vd), len(lens), lens.ctypes.data, window, num_q_heads,
                                 block_size, num_blocks, max_seq_len, ctypes.byref(r)))

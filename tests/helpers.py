@@ -17,18 +17,18 @@ def random_high(H, n, seed):
     return np.stack([np.sort(rng.choice(D, n, replace=False)) for _ in range(H)]).astype(np.int16)
 
 
-def codec_pair(H, bits, sizes, seed, high=None, qjl=False):
+def codec_pair(H, bits, sizes, seed, high=None, qjl=False, groupwise=False):
     """(device Codec, oracle Format) for the same plain parameters."""
     if len(bits) == 2 and high is None:
         high = random_high(H, sizes[0], seed + 17)
-    return (tq.Codec(H, bits, sizes, high, seed, qjl=qjl),
-            O.Format(D, H, tuple(bits), tuple(sizes), high, seed, qjl=qjl))
+    return (tq.Codec(H, bits, sizes, high, seed, qjl=qjl, groupwise=groupwise),
+            O.Format(D, H, tuple(bits), tuple(sizes), high, seed, qjl=qjl, groupwise=groupwise))
 
 
 def slice_format(f: O.Format, h: int) -> O.Format:
     """The oracle format of KV head h alone (metadata sliced to one head)."""
     hc = None if f.high_coords is None else np.asarray(f.high_coords)[h:h + 1]
-    return O.Format(f.head_dim, 1, f.group_bits, f.group_size, hc, f.seed, qjl=f.qjl)
+    return O.Format(f.head_dim, 1, f.group_bits, f.group_size, hc, f.seed, qjl=f.qjl, groupwise=f.groupwise)
 
 
 def random_kv(T, H, gen, scale_outliers=True):
@@ -53,7 +53,7 @@ class DecodeProblem:
     """
 
     def __init__(self, lens, H, G, kspec, vspec, window, block_size, seed, slack=1.3, sinks=0, kqjl=False,
-                 vqjl=False):
+                 vqjl=False, kgw=False, vgw=False):
         self.lens = np.asarray(lens, dtype=np.int64)
         self.B, self.H, self.G, self.Hq = len(lens), H, G, H * G
         self.sinks = sinks
@@ -62,8 +62,8 @@ class DecodeProblem:
         gen = torch.Generator(device="cuda")
         gen.manual_seed(seed)
         rng = np.random.default_rng(seed)
-        self.kc, self.kf = codec_pair(H, *kspec, qjl=kqjl)
-        self.vc, self.vf = codec_pair(H, *vspec, qjl=vqjl)
+        self.kc, self.kf = codec_pair(H, *kspec, qjl=kqjl, groupwise=kgw)
+        self.vc, self.vf = codec_pair(H, *vspec, qjl=vqjl, groupwise=vgw)
         packed = self.lens - np.minimum(window, self.lens)
         nblk = -(-packed // block_size)
         self.num_blocks = max(1, int(math.ceil(slack * nblk.sum())) + 1)

@@ -164,3 +164,30 @@ def test_qjl_row_bytes_and_ledger():
     ref = O.byte_ledger(f, O.Format(D, H, (3,), (128,), None, 1), lens, W, bs, nb, workspace_bytes=ws)
     for key in ("index_bytes", "norm_bytes", "transform_bytes", "page_pool_bytes", "metadata_bytes"):
         assert got[key] == getattr(ref, key), key
+
+
+
+def test_groupwise_row_bytes_ledger_and_validation():
+    H, Hq, W, bs = 4, 16, 32, 16
+    hc = _high(H, 32, 4)
+    t = tq.codec_host_tables(D, H, (4, 2), (32, 96), hc, 3, groupwise=True)
+    f = O.Format(D, H, (4, 2), (32, 96), hc, 3, groupwise=True)
+    assert t["row_bytes"] == O.row_bytes(f) == 16 + 24 + 4
+    # codebooks of the groups' own dimensions (32 and 96)
+    for g, (b, n) in enumerate(((4, 32), (2, 96))):
+        c, beta = O.codebook(b, n)
+        assert np.array_equal(t["centroids_f16"][g][:1 << b], c.astype(np.float16).view(np.uint16))
+        assert np.array_equal(t["boundaries"][g][:(1 << b) - 1], beta.astype(np.float32))
+    lens = [0, 9, 32, 33, 700]
+    ksp = {"group_bits": (4, 2), "group_size": (32, 96), "seed": 3, "high_coords": hc, "groupwise": True}
+    vsp = {"group_bits": (3,), "group_size": (128,), "seed": 1, "high_coords": None}
+    nb = sum(-(-(L - min(W, L)) // bs) for L in lens) + 2
+    got = tq.host_ledger(H, ksp, vsp, lens, W, Hq, bs, nb)
+    ws = tq.decode_workspace_bytes(len(lens), Hq, H, max(lens), bs)
+    ref = O.byte_ledger(f, O.Format(D, H, (3,), (128,), None, 1), lens, W, bs, nb, workspace_bytes=ws)
+    for key in ("index_bytes", "norm_bytes", "transform_bytes", "page_pool_bytes", "metadata_bytes"):
+        assert got[key] == getattr(ref, key), key
+    with pytest.raises(ValueError):  # group-wise needs two groups
+        tq.codec_host_tables(D, H, (3,), (128,), None, 3, groupwise=True)
+    with pytest.raises(ValueError):  # and no QJL stage
+        tq.codec_host_tables(D, H, (4, 2), (32, 96), hc, 3, qjl=True, groupwise=True)
