@@ -65,7 +65,7 @@ R16 QJL residual stage (TurboQuant "Design" page, "Recipe Strategy": row
     E over S of its product with q equals q . x when g is exact. In a
     sub-page the sign bytes follow the index bytes of each row and the norm
     area holds (norm, residual norm) per row.
-R17 Group-wise rotation (SURVEY's original-domain reading of the high/low
+R17 Group-wise rotation (the original-channel reading of the high/low
     recipe; "Recipe Strategy": the high channel set comes from calibration
     metadata). With groupwise set, group 0 is the set of ORIGINAL channels
     high_coords[h] (ascending) and group 1 the other channels (ascending).

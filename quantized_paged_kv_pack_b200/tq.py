@@ -196,7 +196,8 @@ def load_recipe_metadata(path: str) -> dict:
     TurboQuant "Design" page, "Recipe Strategy": activation energy -> sorted
     high-precision indices -> metadata JSON; runtime loads and validates it.
     "Error Model": a missing file raises FileNotFoundError. The keys are
-    head_dim, num_kv_heads, group_bits, group_size, high_coords, hadamard_seed.
+    head_dim, num_kv_heads, group_bits, group_size, high_coords, hadamard_seed,
+    and optionally qjl and groupwise (booleans).
     """
     if not os.path.exists(path):
         raise FileNotFoundError(f"recipe metadata not found: {path}")
@@ -206,12 +207,37 @@ def load_recipe_metadata(path: str) -> dict:
         spec = dict(head_dim=int(meta["head_dim"]), num_kv_heads=int(meta["num_kv_heads"]),
                     group_bits=tuple(meta["group_bits"]), group_size=tuple(meta["group_size"]),
                     high_coords=None if meta.get("high_coords") is None else np.asarray(meta["high_coords"], np.int16),
-                    seed=int(meta.get("hadamard_seed", 0)))
+                    seed=int(meta.get("hadamard_seed", 0)), qjl=bool(meta.get("qjl", False)),
+                    groupwise=bool(meta.get("groupwise", False)))
     except (KeyError, TypeError) as e:
         raise ValueError(f"malformed recipe metadata: {e}") from e
     codec_host_tables(spec["head_dim"], spec["num_kv_heads"], spec["group_bits"], spec["group_size"],
-                      spec["high_coords"], spec["seed"])  # validates
+                      spec["high_coords"], spec["seed"], spec["qjl"], spec["groupwise"])  # validates
     return spec
+
+
+def slice_recipe(spec: dict, rank: int, world: int) -> dict:
+    """The recipe of one tensor-parallel partition of the KV heads.
+
+    TurboQuant "Design" page, "Recipe Strategy": the runtime slices the
+    metadata by tensor-parallel partition. KV heads are split into `world`
+    contiguous ranges; partition `rank` keeps heads [rank H/world, (rank+1)
+    H/world) and their rows of high_coords. The sign seed is shared, so every
+    partition rotates as the whole model does.
+    """
+    H = int(spec["num_kv_heads"])
+    if world < 1 or H % world:
+        raise ValueError(f"num_kv_heads {H} does not split into {world} partitions")
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside [0, {world})")
+    n = H // world
+    out = dict(spec)
+    out["num_kv_heads"] = n
+    if spec.get("high_coords") is not None:
+        out["high_coords"] = np.ascontiguousarray(np.asarray(spec["high_coords"])[rank * n:(rank + 1) * n])
+    codec_host_tables(spec["head_dim"], n, spec["group_bits"], spec["group_size"], out.get("high_coords"),
+                      spec.get("seed", 0), spec.get("qjl", False), spec.get("groupwise", False))  # validates
+    return out
 
 
 def _stream(stream):

@@ -191,3 +191,24 @@ def test_groupwise_row_bytes_ledger_and_validation():
         tq.codec_host_tables(D, H, (3,), (128,), None, 3, groupwise=True)
     with pytest.raises(ValueError):  # and no QJL stage
         tq.codec_host_tables(D, H, (4, 2), (32, 96), hc, 3, qjl=True, groupwise=True)
+
+
+
+def test_recipe_slicing_by_tensor_parallel_partition(tmp_path):
+    hc = _high(8, 32, 12)
+    p = tmp_path / "recipe.json"
+    p.write_text(json.dumps({"head_dim": 128, "num_kv_heads": 8, "group_bits": [4, 2], "group_size": [32, 96],
+                             "high_coords": hc.tolist(), "hadamard_seed": 5, "groupwise": True}))
+    spec = tq.load_recipe_metadata(str(p))
+    assert spec["groupwise"] and not spec["qjl"]
+    parts = [tq.slice_recipe(spec, r, 4) for r in range(4)]
+    assert all(q["num_kv_heads"] == 2 for q in parts)
+    assert np.array_equal(np.concatenate([q["high_coords"] for q in parts]), hc)
+    # a partition's codec tables equal the corresponding heads of the whole model's
+    whole = tq.codec_host_tables(128, 8, (4, 2), (32, 96), hc, 5, groupwise=True)
+    part = tq.codec_host_tables(128, 2, (4, 2), (32, 96), parts[3]["high_coords"], 5, groupwise=True)
+    assert np.array_equal(part["perm"], whole["perm"][6:8]) and np.array_equal(part["signs"], whole["signs"])
+    with pytest.raises(ValueError):
+        tq.slice_recipe(spec, 0, 3)
+    with pytest.raises(ValueError):
+        tq.slice_recipe(spec, 4, 4)
