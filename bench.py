@@ -36,7 +36,9 @@ from quantized_paged_kv_pack_b200 import tq  # noqa: E402
 from quantized_paged_kv_pack_b200 import workloads as WL  # noqa: E402
 
 HEADLINE = "decode_llama70b_3p5bit"
-EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl", "pack_llama8b_4bit"]
+EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl",
+         "decode_llama8b_3p5bit_groupwise",
+         "pack_llama8b_4bit"]
 D = 128
 METRIC = "paged TQ decode HBM GB/s (algorithmic bytes / step time)"
 
@@ -79,8 +81,10 @@ class DecodeSetup:
         self.w = w
         ks, vs = WL.codec_specs(w)
         self.kspec, self.vspec = ks, vs
-        self.kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed, qjl=ks.qjl)
-        self.vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed, qjl=vs.qjl)
+        self.kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed,
+                           qjl=ks.qjl, groupwise=ks.groupwise)
+        self.vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed,
+                           qjl=vs.qjl, groupwise=vs.groupwise)
         lay = WL.page_layout(w)
         B = len(lay.seq_lens)
         # one spare block per sequence, next in its block table, takes the rows the
@@ -174,8 +178,10 @@ class PackSetup:
     def __init__(self, w: WL.Workload):
         self.w = w
         ks, vs = WL.codec_specs(w)
-        self.kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed, qjl=ks.qjl)
-        self.vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed, qjl=vs.qjl)
+        self.kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed,
+                           qjl=ks.qjl, groupwise=ks.groupwise)
+        self.vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed,
+                           qjl=vs.qjl, groupwise=vs.groupwise)
         self.k, self.v, slots, lay = WL.pack_batch(w, device="cuda")
         self.slots = torch.as_tensor(slots, device="cuda")
         self.kp = tq.page_pool(self.kc, lay.num_blocks, w.block_size)
@@ -365,8 +371,10 @@ def _oracle_formats(w, kspec, vspec, h):
 
     hk = None if kspec.high_coords is None else kspec.high_coords[h:h + 1]
     hv = None if vspec.high_coords is None else vspec.high_coords[h:h + 1]
-    return (O.Format(D, 1, kspec.group_bits, kspec.group_size, hk, kspec.seed, qjl=kspec.qjl),
-            O.Format(D, 1, vspec.group_bits, vspec.group_size, hv, vspec.seed, qjl=vspec.qjl))
+    return (O.Format(D, 1, kspec.group_bits, kspec.group_size, hk, kspec.seed, qjl=kspec.qjl,
+                     groupwise=kspec.groupwise),
+            O.Format(D, 1, vspec.group_bits, vspec.group_size, hv, vspec.seed, qjl=vspec.qjl,
+                     groupwise=vspec.groupwise))
 
 
 def _median_sequence(lay):
@@ -454,7 +462,8 @@ def run_reference(args):
     from oracle import tq_oracle as O
 
     rb = sum(O.row_bytes(O.Format(D, 1, s.group_bits, s.group_size,
-                                  None if s.high_coords is None else s.high_coords[:1], s.seed, qjl=s.qjl))
+                                  None if s.high_coords is None else s.high_coords[:1], s.seed, qjl=s.qjl,
+                                  groupwise=s.groupwise))
              for s in (kspec, vspec))
     src = lambda b, h: oracle_pages_unit(w, kspec, vspec, lay, b, h)  # noqa: E731
     for _ in range(args.warmup):

@@ -43,6 +43,7 @@ class CodecSpec:
     seed: int
     high_coords: Optional[np.ndarray] = None  # [H_kv][group_size[0]] int16, sorted
     qjl: bool = False                         # QJL residual stage after the MSE groups
+    groupwise: bool = False                   # high_coords name original channels, per-group rotation
 
 
 @dataclass(frozen=True)
@@ -68,6 +69,7 @@ class Workload:
     pool_slack: float = 1.0  # page pool = ceil(slack * needed) blocks, free blocks interleaved
     description: str = ""
     k_qjl: bool = False      # keys carry the QJL residual stage
+    groupwise: bool = False  # K and V: group-wise rotation with per-group norms
 
 
 WORKLOADS = {
@@ -104,7 +106,14 @@ WORKLOADS = {
         description="decode batch 16, 32 query / 8 KV heads (Llama-3.1-8B), context 16384, block 16, "
                     "K 2.5-bit MSE (64 channels at 3 bits + 64 at 2) plus the 1-bit QJL residual stage "
                     "(3.5 bits per channel), V 3.5-bit, 128-token bf16 window; QJL keys run on the general "
-                    "CUDA-core kernel")
+                    "CUDA-core kernel"),
+    "decode_llama8b_3p5bit_groupwise": Workload(
+        "decode_llama8b_3p5bit_groupwise", "decode", 1007, 16, 32, 8, 128, 16, 128,
+        (4, 3), (64, 64), (4, 3), (64, 64), 71, 72, 8, True, "fixed:16384", groupwise=True,
+        description="decode batch 16, 32 query / 8 KV heads (Llama-3.1-8B), context 16384, block 16, "
+                    "K and V 3.5-bit group-wise: 64 original channels (the outlier channels among them) "
+                    "at 4 bits and the other 64 at 3 bits, each group rotated on its own with its own norm, "
+                    "128-token bf16 window; group-wise formats run on the general CUDA-core kernel"),
 }
 
 
@@ -113,15 +122,28 @@ def _rng(seed: int) -> np.random.Generator:
 
 
 def codec_specs(w: Workload):
-    """(K spec, V spec). High channel sets are seeded, sorted, independent for K and V."""
+    """(K spec, V spec). High channel sets are seeded, sorted, independent for K and V.
+
+    A group-wise workload stands in for calibration: its high set of original
+    channels holds that head's outlier channels plus seeded others.
+    """
     rng = _rng(w.seed * 7 + 3)
     specs = []
-    for bits, sizes, seed, qjl in ((w.k_bits, w.k_sizes, w.k_seed, w.k_qjl), (w.v_bits, w.v_sizes, w.v_seed, False)):
+    for which, (bits, sizes, seed, qjl) in enumerate(((w.k_bits, w.k_sizes, w.k_seed, w.k_qjl),
+                                                       (w.v_bits, w.v_sizes, w.v_seed, False))):
         high = None
-        if len(bits) == 2:
+        if len(bits) == 2 and w.groupwise:
+            out = _outlier_channels(w, which)
+            rows = []
+            for h in range(w.num_kv_heads):
+                rest = np.setdiff1d(np.arange(w.head_dim), out[h])
+                extra = rng.choice(rest, sizes[0] - len(out[h]), replace=False)
+                rows.append(np.sort(np.concatenate([out[h], extra])))
+            high = np.stack(rows).astype(np.int16)
+        elif len(bits) == 2:
             high = np.stack([np.sort(rng.choice(w.head_dim, sizes[0], replace=False))
                              for _ in range(w.num_kv_heads)]).astype(np.int16)
-        specs.append(CodecSpec(tuple(bits), tuple(sizes), seed, high, qjl))
+        specs.append(CodecSpec(tuple(bits), tuple(sizes), seed, high, qjl, w.groupwise))
     return specs[0], specs[1]
 
 

@@ -131,8 +131,12 @@ class DecodeProblem:
 def workload_codecs(w):
     """(device K codec, device V codec, oracle K format, oracle V format) of a named workload."""
     ks, vs = W.codec_specs(w)
-    kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed, qjl=ks.qjl)
-    vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed, qjl=vs.qjl)
-    kf = O.Format(D, w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed, qjl=ks.qjl)
-    vf = O.Format(D, w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed, qjl=vs.qjl)
+    kc = tq.Codec(w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed, qjl=ks.qjl,
+                  groupwise=ks.groupwise)
+    vc = tq.Codec(w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed, qjl=vs.qjl,
+                  groupwise=vs.groupwise)
+    kf = O.Format(D, w.num_kv_heads, ks.group_bits, ks.group_size, ks.high_coords, ks.seed, qjl=ks.qjl,
+                  groupwise=ks.groupwise)
+    vf = O.Format(D, w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed, qjl=vs.qjl,
+                  groupwise=vs.groupwise)
     return kc, vc, kf, vf

@@ -145,7 +145,7 @@ def _workload_problem(name, n_seq):
 
 
 @pytest.mark.parametrize("name", ["decode_llama8b_4bit", "decode_llama70b_3p5bit", "decode_llama8b_2p5bit",
-                                  "decode_llama8b_3p5bit_qjl"])
+                                  "decode_llama8b_3p5bit_qjl", "decode_llama8b_3p5bit_groupwise"])
 def test_decode_full_size_workloads_sampled(name):
     """Full-size workloads in the benchmark's launch; the oracle checks sampled outputs."""
     w, kc, vc, kf, vf, layout, kp, vp, kw, vw = _workload_problem(name, None)
