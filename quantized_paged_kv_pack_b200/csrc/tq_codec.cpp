@@ -375,8 +375,9 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
     plan->record_bytes = static_cast<size_t>(batch) * num_kv_heads * plan->items_per_unit * plan->record_floats *
                          sizeof(float);
     plan->record_bytes = (plan->record_bytes + 255) / 256 * 256;
-    // then the rotated queries: [batch][num_q_heads][128] fp32
-    plan->workspace_bytes = plan->record_bytes + static_cast<size_t>(batch) * num_q_heads * kHeadDim * sizeof(float);
+    // then the rotated queries and their QJL projections: 2 x [batch][num_q_heads][128] fp32
+    plan->workspace_bytes =
+        plan->record_bytes + 2 * static_cast<size_t>(batch) * num_q_heads * kHeadDim * sizeof(float);
     return true;
 }
 

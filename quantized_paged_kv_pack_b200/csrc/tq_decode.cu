@@ -412,19 +412,22 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     a.items_per_unit = plan.items_per_unit;
     a.ws = static_cast<float*>(workspace);
     a.qrot = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.record_bytes);
+    a.qjl_q = a.qrot + static_cast<size_t>(batch) * num_q_heads * kHeadDim;
     a.d_err = d_err;
     const char* withhold = std::getenv("TQ_TEST_WITHHOLD_COPIES");
     a.withhold_copies = withhold && std::string(withhold) == "1";
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // Tensor-core kernel for the formats it is instantiated for (block sizes a
     // multiple of 16); the general kernel covers every other valid format.
-    // TQ_DECODE_KERNEL=general selects the general kernel (for cross-checks).
-    // QJL keys (the sign-bit score term) and group-wise codecs run on the general kernel.
+    // TQ_DECODE_KERNEL=general selects the general kernel and =tensor the
+    // tensor-core one (unsupported formats then fail), for cross-checks.
     const char* force = std::getenv("TQ_DECODE_KERNEL");
-    if (!(force && std::string(force) == "general") && !kc->desc.qjl && !kc->desc.groupwise && !vc->desc.groupwise) {
+    const std::string forced = force ? force : "";
+    if (forced != "general") {
         st = launch_decode_mma(a, kc, vc, plan.group, stream);
         if (st == TQ_OK) return finish(s, d_err, "decode partials");
         if (st != TQ_ERR_UNSUPPORTED) return st;
+        if (forced == "tensor") return fail(TQ_ERR_UNSUPPORTED, "no tensor-core decode for these formats");
         clear_error();
     }
     dim3 grid(plan.items_per_unit, kc->desc.num_kv_heads, batch);

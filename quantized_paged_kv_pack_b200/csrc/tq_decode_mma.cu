@@ -23,19 +23,20 @@
 // two indices of a pair come from two tokens at the same coordinate, so the
 // lane first interleaves two tokens' index bits.
 //
-// Data movement: each compute warp owns a ring of tile slots in shared
-// memory. A ninth warp, the producer, fills them with 16-byte cp.async copies
-// from all its lanes (index rows of K and V, and their norms) in the order the
-// warps consume them, tracked by a "full" mbarrier per slot; a warp releases a
-// slot through its "empty" mbarrier. The producer runs ahead across work items
-// and keeps the next item's block ids in shared memory, so the compute warps
-// carry no address or block-table arithmetic. (Per-tile bulk copies cost the
-// copy engine a fixed overhead per operation that, at a few hundred bytes per
-// operation, capped the rate well below HBM speed.) Every wait is bounded; on
-// expiry the kernel sets TQ_DERR_TIMEOUT, waits for its copies and stops.
-// CTAs are persistent and take work items (sequence, KV head, split of the
-// packed tokens, query-head group) in a fixed stride; the compute warps share
-// an item's tiles and merge their (max, sum, accumulator) states at its end.
+// Data movement: a ninth warp, the producer, fills ring slots in shared memory
+// with bulk copies (cp.async.bulk, completion counted on a "full" mbarrier per
+// slot) in the order the compute warps consume them; a warp releases a slot
+// through an "empty" mbarrier. The producer runs ahead across work items and
+// keeps the next item's block ids in shared memory, so the compute warps carry
+// no address or block-table arithmetic. Two layouts: with a multiple of 8 KV
+// heads a slot is one page block of 8 consecutive heads in both pools (two
+// copies of several KB; warp w takes head w), otherwise each warp owns a ring
+// of 16-token tiles of one head. (Copies of a few hundred bytes each cost the
+// copy engine a fixed overhead per operation that capped the rate well below
+// HBM speed; the 8-head slots make every copy large.) Every wait is bounded;
+// on expiry the kernel sets TQ_DERR_TIMEOUT, waits for its copies and stops.
+// CTAs are persistent and take work items (sequence, KV head or 8 of them,
+// split of the packed tokens, query-head group) in a fixed stride.
 //
 // Online softmax: each warp keeps a reference max per head that moves only
 // when a score exceeds it by more than 2^8, so weights stay below 2^8 and the
@@ -70,6 +71,7 @@ constexpr uint32_t kWaitHintNs = 16384;     // sleep bound of one blocking wait 
 constexpr uint32_t kWaitRounds = 1u << 16;  // blocking wait attempts (about a second)
 constexpr float kSlack = 8.0f;                 // log2 slack of the running max
 
+#pragma nv_diag_suppress 177  // not every format constant is used by every instantiation
 template <int B0_, int N0_, int B1_, int N1_>
 struct Fmt {
     static constexpr int B0 = B0_, N0 = N0_, B1 = B1_, N1 = N1_;
@@ -82,18 +84,33 @@ struct Fmt {
     static constexpr int VC0 = N0 / 8 * B0 / 8;         // value side: bytes of group 0 per lane
     static constexpr int VC1 = N1 / 8 * B1 / 8;
     static_assert(KS0 + KS1 == 8 && MT0 + MT1 == 8, "head_dim 128");
-    static_assert(IB <= 64, "tile slot holds rows of at most 64 index bytes");
+    static_assert(IB % 4 == 0 && IB <= 64, "index groups of whole words, at most 64 bytes");
 };
-using U4 = Fmt<4, 128, 0, 0>;
-using U3 = Fmt<3, 128, 0, 0>;
-using M43 = Fmt<4, 64, 3, 64>;
-using M42 = Fmt<4, 32, 2, 96>;
 
-// Bytes of one ring slot: 16 index rows of K and of V, each followed by the
-// 16 norms (32 bytes); a multiple of 16, the copy granule.
+// What a row holds besides its index groups. Plain: one fp16 norm. Group-wise
+// (the high channels are original channels, each group rotated on its own):
+// one fp16 norm per group. QJL keys: the 128 residual sign bits after the
+// index groups, and the norm followed by the residual norm.
+constexpr int kPlain = 0, kGroupwise = 1, kQjl = 2;
+template <class F, int MODE_>
+struct Row : F {
+    static constexpr int MODE = MODE_;
+    static constexpr int RB = F::IB + (MODE_ == kQjl ? kHeadDim / 8 : 0);  // bytes of an index row
+    static constexpr int NB = MODE_ == kPlain ? 2 : 4;                     // bytes of a row's norms
+};
+using U4 = Row<Fmt<4, 128, 0, 0>, kPlain>;
+using U3 = Row<Fmt<3, 128, 0, 0>, kPlain>;
+using M43 = Row<Fmt<4, 64, 3, 64>, kPlain>;
+using M42 = Row<Fmt<4, 32, 2, 96>, kPlain>;
+using M32Q = Row<Fmt<3, 64, 2, 64>, kQjl>;
+using M43Q = Row<Fmt<4, 64, 3, 64>, kQjl>;
+using M43G = Row<Fmt<4, 64, 3, 64>, kGroupwise>;
+
+// Bytes of one ring slot: 16 index rows of K followed by their 16 norms, then
+// the same for V; a multiple of 16, the copy granule.
 template <class KF, class VF>
 __host__ __device__ constexpr uint32_t stage_bytes() {
-    return 16 * (KF::IB + VF::IB) + 64;
+    return 16 * (KF::RB + KF::NB + VF::RB + VF::NB);
 }
 
 template <int B, int E, class F>
@@ -425,18 +442,56 @@ __device__ __forceinline__ void fill_table(uint32_t* table, const LutValues& tv,
 // accumulator; a lane holds heads 2c and 2c + 1. NH = 4: columns 2h and 2h + 1
 // are the hi and lo halves of head h (4 heads), summed after the MMA; a lane
 // holds head c. Lane (r, c) = (lane / 4, lane % 4).
+//
+// Group-wise K: the score k-steps of each group accumulate apart and take that
+// group's norm. Group-wise V: the value row tiles of group 1 take P' built with
+// the group-1 norms. QJL keys: 8 more k-steps per tile score the sign bits
+// against the projected query (the A operand is +-|r| per token, exact in
+// fp16); they land in the same accumulators as the index groups, so the
+// token's score is n (q'.c + sqrt(pi/2)/128 |r| (S q').z) before the norm.
 template <class KF, class VF, int NH>
 struct WarpTiles {
     static constexpr int HL = NH / 4;  // heads per lane
+    static constexpr bool KQ = KF::MODE == kQjl, KG = KF::MODE == kGroupwise, VG = VF::MODE == kGroupwise;
     uint32_t bq[8][2 * HL];            // query B fragments per k-step
-    uint32_t bp[2 * HL];               // P' B fragments of the last scored tile
+    uint32_t bz[KQ ? 8 : 1][2 * HL];   // QJL: projected-query B fragments per sign k-step
+    uint32_t bp[2 * HL];               // P' B fragments of the last scored tile (group 0 norms when VG)
+    uint32_t bp1[VG ? 2 * HL : 1];     // VG: P' B fragments with the group-1 norms
     float o[8][4];                     // value accumulators: row tile q, rows r / r + 8, columns 2c / 2c + 1
     float m_ref[HL], l_run[HL];
 
     // Rotated, scaled queries of the item's query heads (rows of them), fp32
-    // [head][128] in the packed coordinate order.
-    __device__ __forceinline__ void begin(const float* qr, int rows, int r, int c) {
+    // [head][128] in the packed coordinate order; for QJL keys also their
+    // projections qz, [head][128] in projection order.
+    __device__ __forceinline__ void begin(const float* qr, const float* qz, int rows, int r, int c) {
         const int head = NH == 8 ? r : (r >> 1);
+        if constexpr (KQ) {
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                // sign k-step s: B rows (2c, 2c+1) and (2c+8, 2c+9) are projections
+                // 32c + s + (0, 8) and 32c + s + (16, 24)
+                float x0 = 0.0f, x1 = 0.0f, x2 = 0.0f, x3 = 0.0f;
+                if (head < rows) {
+                    const float* z = qz + head * kHeadDim + 32 * c + s;
+                    x0 = __ldcg(z);
+                    x1 = __ldcg(z + 8);
+                    x2 = __ldcg(z + 16);
+                    x3 = __ldcg(z + 24);
+                }
+                uint32_t h01, l01, h23, l23;
+                split2(x0, x1, h01, l01);
+                split2(x2, x3, h23, l23);
+                if constexpr (NH == 8) {
+                    bz[s][0] = h01;
+                    bz[s][1] = h23;
+                    bz[s][2] = l01;
+                    bz[s][3] = l23;
+                } else {
+                    bz[s][0] = (r & 1) ? l01 : h01;
+                    bz[s][1] = (r & 1) ? l23 : h23;
+                }
+            }
+        }
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
             // k-step s: B rows (2c, 2c+1) and (2c+8, 2c+9) are coordinates p..p+3 of lane c's chunk
@@ -471,26 +526,51 @@ struct WarpTiles {
     __device__ __forceinline__ void scores(uint32_t kbase, uint32_t knorm, uint32_t vnorm, int nvalid,
                                            uint32_t lane_base, uint32_t psel, int r, int c) {
         // ---- S^T = K^ Q'^T: rows tokens r, r + 8 ----
-        // Independent accumulator chains (k-step parity; hi / lo for NH = 8)
-        // keep the MMA dependency depth at 4.
+        // Independent accumulator chains (k-step parity, or the group when K is
+        // group-wise; hi / lo for NH = 8) keep the MMA dependency depth at 4.
         constexpr int NC = NH == 8 ? 4 : 2;
         float sacc[NC][4];
 #pragma unroll
         for (int u = 0; u < NC; ++u) sacc[u][0] = sacc[u][1] = sacc[u][2] = sacc[u][3] = 0.0f;
         auto score_step = [&](auto si, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
             constexpr int s_ = decltype(si)::value;
+            constexpr int u = KG ? (s_ < KF::KS0 ? 0 : 1) : (s_ & 1);
             if constexpr (NH == 8) {
-                mma16816(sacc[s_ & 1], a0, a1, a2, a3, bq[s_][0], bq[s_][1]);
-                mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, bq[s_][2], bq[s_][3]);
+                mma16816(sacc[u], a0, a1, a2, a3, bq[s_][0], bq[s_][1]);
+                mma16816(sacc[2 + u], a0, a1, a2, a3, bq[s_][2], bq[s_][3]);
             } else {
-                mma16816(sacc[s_ & 1], a0, a1, a2, a3, bq[s_][0], bq[s_][1]);
+                mma16816(sacc[u], a0, a1, a2, a3, bq[s_][0], bq[s_][1]);
             }
         };
+        if constexpr (KQ) {
+            // Sign k-step s takes bits s, s + 8, s + 16, s + 24 of the lane's word
+            // (projections 32c + ...): shifted to the top of bytes 0..3, prmt
+            // turns each into an all-ones or all-zero byte in the high byte of
+            // a half, which becomes the sign of +-|r|.
+            const uint32_t wa = lds32(kbase + r * KF::RB + KF::IB + 4 * c);
+            const uint32_t wb = lds32(kbase + (r + 8) * KF::RB + KF::IB + 4 * c);
+            const uint32_t ga = lds16(knorm + KF::NB * r + 2), gb = lds16(knorm + KF::NB * (r + 8) + 2);
+            const uint32_t rn_a = ga | (ga << 16), rn_b = gb | (gb << 16);
+            static_for<0, 8>([&](auto si) {
+                constexpr int s_ = decltype(si)::value;
+                const uint32_t ya = wa << (7 - s_), yb = wb << (7 - s_);
+                const uint32_t a0 = rn_a | (~prmt(ya, 0u, 0x9484u) & 0x80008000u);
+                const uint32_t a1 = rn_b | (~prmt(yb, 0u, 0x9484u) & 0x80008000u);
+                const uint32_t a2 = rn_a | (~prmt(ya, 0u, 0xB4A4u) & 0x80008000u);
+                const uint32_t a3 = rn_b | (~prmt(yb, 0u, 0xB4A4u) & 0x80008000u);
+                if constexpr (NH == 8) {
+                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, bz[s_][0], bz[s_][1]);
+                    mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, bz[s_][2], bz[s_][3]);
+                } else {
+                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, bz[s_][0], bz[s_][1]);
+                }
+            });
+        }
         {
             constexpr int KW0 = (KF::KC0 + 3) / 4;
             constexpr bool A0 = KF::KC0 % 4 == 0;
-            const Words<KW0> k0a = lds_span<KF::KC0, A0>(kbase + r * KF::IB + c * KF::KC0);
-            const Words<KW0> k0b = lds_span<KF::KC0, A0>(kbase + (r + 8) * KF::IB + c * KF::KC0);
+            const Words<KW0> k0a = lds_span<KF::KC0, A0>(kbase + r * KF::RB + c * KF::KC0);
+            const Words<KW0> k0b = lds_span<KF::KC0, A0>(kbase + (r + 8) * KF::RB + c * KF::KC0);
             const uint32_t base0 = lut_base<KF::B0>(lane_base);
             static_for<0, KF::KS0>([&](auto si) {
                 constexpr int s_ = decltype(si)::value;
@@ -504,8 +584,8 @@ struct WarpTiles {
                 constexpr int KW1 = (KF::KC1 + 3) / 4;
                 constexpr bool A1 = (KF::KC1 % 4 == 0) && (KF::BOFF1 % 4 == 0);
                 const uint32_t g1 = KF::BOFF1 + c * KF::KC1;
-                const Words<KW1> k1a = lds_span<KF::KC1, A1>(kbase + r * KF::IB + g1);
-                const Words<KW1> k1b = lds_span<KF::KC1, A1>(kbase + (r + 8) * KF::IB + g1);
+                const Words<KW1> k1a = lds_span<KF::KC1, A1>(kbase + r * KF::RB + g1);
+                const Words<KW1> k1b = lds_span<KF::KC1, A1>(kbase + (r + 8) * KF::RB + g1);
                 const uint32_t base1 = lut_base<KF::B1>(lane_base);
                 static_for<0, KF::KS1>([&](auto si) {
                     constexpr int s_ = decltype(si)::value;
@@ -519,11 +599,25 @@ struct WarpTiles {
         }
 
         // ---- online softmax over the lane's heads, tokens r and r + 8 ----
-        const float nk0 = f16_at(knorm + 2 * r), nk1 = f16_at(knorm + 2 * (r + 8));
-        const float nv0 = f16_at(vnorm + 2 * r), nv1 = f16_at(vnorm + 2 * (r + 8));
+        const float nk0 = f16_at(knorm + KF::NB * r), nk1 = f16_at(knorm + KF::NB * (r + 8));
+        const float nv0 = f16_at(vnorm + VF::NB * r), nv1 = f16_at(vnorm + VF::NB * (r + 8));
         const bool ok0 = r < nvalid, ok1 = r + 8 < nvalid;
         float sc[HL][2];  // head e of the lane, token r (0) or r + 8 (1)
-        if constexpr (NH == 8) {
+        if constexpr (NH == 8 && KG) {
+            // chains 0 / 2: group 0 hi / lo; chains 1 / 3: group 1
+            const float mk0 = f16_at(knorm + KF::NB * r + 2), mk1 = f16_at(knorm + KF::NB * (r + 8) + 2);
+            float x0, x1, y0, y1;
+            upk(add2(mul2(add2(pk(sacc[0][0], sacc[0][1]), pk(sacc[2][0], sacc[2][1])), pk(nk0, nk0)),
+                     mul2(add2(pk(sacc[1][0], sacc[1][1]), pk(sacc[3][0], sacc[3][1])), pk(mk0, mk0))),
+                x0, x1);
+            upk(add2(mul2(add2(pk(sacc[0][2], sacc[0][3]), pk(sacc[2][2], sacc[2][3])), pk(nk1, nk1)),
+                     mul2(add2(pk(sacc[1][2], sacc[1][3]), pk(sacc[3][2], sacc[3][3])), pk(mk1, mk1))),
+                y0, y1);
+            sc[0][0] = ok0 ? x0 : -INFINITY;
+            sc[HL - 1][0] = ok0 ? x1 : -INFINITY;
+            sc[0][1] = ok1 ? y0 : -INFINITY;
+            sc[HL - 1][1] = ok1 ? y1 : -INFINITY;
+        } else if constexpr (NH == 8) {
             float x0, x1, y0, y1;
             upk(add2(add2(pk(sacc[0][0], sacc[0][1]), pk(sacc[1][0], sacc[1][1])),
                      add2(pk(sacc[2][0], sacc[2][1]), pk(sacc[3][0], sacc[3][1]))),
@@ -537,6 +631,11 @@ struct WarpTiles {
             sc[HL - 1][0] = ok0 ? x1 : -INFINITY;
             sc[0][1] = ok1 ? y0 : -INFINITY;
             sc[HL - 1][1] = ok1 ? y1 : -INFINITY;
+        } else if constexpr (KG) {
+            // chain 0: group 0 (hi, lo columns); chain 1: group 1
+            const float mk0 = f16_at(knorm + KF::NB * r + 2), mk1 = f16_at(knorm + KF::NB * (r + 8) + 2);
+            sc[0][0] = ok0 ? (sacc[0][0] + sacc[0][1]) * nk0 + (sacc[1][0] + sacc[1][1]) * mk0 : -INFINITY;
+            sc[0][1] = ok1 ? (sacc[0][2] + sacc[0][3]) * nk1 + (sacc[1][2] + sacc[1][3]) * mk1 : -INFINITY;
         } else {
             float h0, l0, h1, l1;
             upk(add2(pk(sacc[0][0], sacc[0][1]), pk(sacc[1][0], sacc[1][1])), h0, l0);
@@ -580,41 +679,51 @@ struct WarpTiles {
         // tile of an item always takes the branch above (a valid score exceeds
         // -inf + kSlack), which sets it.
         const float nv0m = ok0 ? nv0 : 0.0f, nv1m = ok1 ? nv1 : 0.0f;  // padding rows may hold anything
-        float w[HL][2];
+        float p[HL][2];
 #pragma unroll
         for (int e = 0; e < HL; ++e) {
             const float mb = m_ref[e] + kSlack;
-            const float p0 = ex2(sc[e][0] - mb), p1 = ex2(sc[e][1] - mb);
-            l_run[e] += p0 + p1;
-            w[e][0] = p0 * nv0m;
-            w[e][1] = p1 * nv1m;
+            p[e][0] = ex2(sc[e][0] - mb);
+            p[e][1] = ex2(sc[e][1] - mb);
+            l_run[e] += p[e][0] + p[e][1];
         }
-        // B fragments of P'^T: rows tokens (2c, 2c+1) and (2c+8, 2c+9), column r.
-        // Tokens 2c and 2c + 8 sit in lane 8c + (r >> 1), tokens 2c + 1 and
-        // 2c + 9 four lanes on.
+        weights(p, nv0m, nv1m, psel, r, c, bp);
+        if constexpr (VG) {
+            const float mv0 = ok0 ? f16_at(vnorm + VF::NB * r + 2) : 0.0f;
+            const float mv1 = ok1 ? f16_at(vnorm + VF::NB * (r + 8) + 2) : 0.0f;
+            weights(p, mv0, mv1, psel, r, c, bp1);
+        }
+    }
+
+    // B fragments of P'^T (P' = p n_V for the V norms n0 of token r and n1 of
+    // token r + 8): rows tokens (2c, 2c+1) and (2c+8, 2c+9), column r. Tokens
+    // 2c and 2c + 8 sit in lane 8c + (r >> 1), tokens 2c + 1 and 2c + 9 four
+    // lanes on.
+    __device__ __forceinline__ static void weights(const float (&p)[HL][2], float n0, float n1, uint32_t psel, int r,
+                                                   int c, uint32_t (&out)[2 * HL]) {
         const int srcA = 8 * c + (r >> 1), srcB = srcA + 4;
         if constexpr (NH == 8) {
             // Per token: (head 2c, head 2c + 1) as hi and lo half2.
             uint32_t th0, tl0, th1, tl1;
-            split2(w[0][0], w[1][0], th0, tl0);
-            split2(w[0][1], w[1][1], th1, tl1);
+            split2(p[0][0] * n0, p[1][0] * n0, th0, tl0);
+            split2(p[0][1] * n1, p[1][1] * n1, th1, tl1);
             const uint32_t xa = __shfl_sync(kFull, th0, srcA), xb = __shfl_sync(kFull, th0, srcB);
             const uint32_t ya = __shfl_sync(kFull, th1, srcA), yb = __shfl_sync(kFull, th1, srcB);
             const uint32_t xla = __shfl_sync(kFull, tl0, srcA), xlb = __shfl_sync(kFull, tl0, srcB);
             const uint32_t yla = __shfl_sync(kFull, tl1, srcA), ylb = __shfl_sync(kFull, tl1, srcB);
-            bp[0] = prmt(xa, xb, psel);
-            bp[1] = prmt(ya, yb, psel);
-            bp[2] = prmt(xla, xlb, psel);
-            bp[3] = prmt(yla, ylb, psel);
+            out[0] = prmt(xa, xb, psel);
+            out[1] = prmt(ya, yb, psel);
+            out[2] = prmt(xla, xlb, psel);
+            out[3] = prmt(yla, ylb, psel);
         } else {
             // Per lane: (token r, token r + 8) as hi and lo half2.
             uint32_t xh, xl;
-            split2(w[0][0], w[0][1], xh, xl);
+            split2(p[0][0] * n0, p[0][1] * n1, xh, xl);
             const uint32_t xa = __shfl_sync(kFull, xh, srcA), ya = __shfl_sync(kFull, xl, srcA);
             const uint32_t xb = __shfl_sync(kFull, xh, srcB), yb = __shfl_sync(kFull, xl, srcB);
             const uint32_t pa = (r & 1) ? ya : xa, pb = (r & 1) ? yb : xb;
-            bp[0] = prmt(pa, pb, 0x5410u);
-            bp[1] = prmt(pa, pb, 0x7632u);
+            out[0] = prmt(pa, pb, 0x5410u);
+            out[1] = prmt(pa, pb, 0x7632u);
         }
     }
 
@@ -630,13 +739,18 @@ struct WarpTiles {
     __device__ __forceinline__ void values(uint32_t vbase, uint32_t lane_base, int r, int c) {
         auto value_step = [&](auto qi, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
             constexpr int q = decltype(qi)::value;
-            mma16816(o[q], a0, a1, a2, a3, bp[0], bp[1]);
-            if constexpr (NH == 8) mma16816(o[q], a0, a1, a2, a3, bp[2], bp[3]);
+            if constexpr (VG && q >= VF::MT0) {
+                mma16816(o[q], a0, a1, a2, a3, bp1[0], bp1[1]);
+                if constexpr (NH == 8) mma16816(o[q], a0, a1, a2, a3, bp1[2], bp1[3]);
+            } else {
+                mma16816(o[q], a0, a1, a2, a3, bp[0], bp[1]);
+                if constexpr (NH == 8) mma16816(o[q], a0, a1, a2, a3, bp[2], bp[3]);
+            }
         };
 
         // ---- O^T += V^T P'^T over 8 coordinate row tiles ----
-        const uint32_t r0 = vbase + (2 * c) * VF::IB, r1 = r0 + VF::IB;
-        const uint32_t r8 = vbase + (2 * c + 8) * VF::IB, r9 = r8 + VF::IB;
+        const uint32_t r0 = vbase + (2 * c) * VF::RB, r1 = r0 + VF::RB;
+        const uint32_t r8 = vbase + (2 * c + 8) * VF::RB, r9 = r8 + VF::RB;
         {
             constexpr int NW0 = (VF::VC0 + 3) / 4;
             constexpr bool A0 = VF::VC0 % 4 == 0;
@@ -826,7 +940,7 @@ struct BlkRing {
 // Bytes of a ring slot: one block of 8 heads in both pools.
 template <class KF, class VF>
 __host__ __device__ constexpr uint32_t blk_slot_bytes(int bs) {
-    return static_cast<uint32_t>(kBlkWarps * bs * (KF::IB + 2 + VF::IB + 2));
+    return static_cast<uint32_t>(kBlkWarps * bs * (KF::RB + KF::NB + VF::RB + VF::NB));
 }
 
 template <class KF, class VF>
@@ -835,7 +949,7 @@ __device__ void produce_blk(const DecodeArgs& a, BlkSmem& sm, const BlkRing& rin
     if (a.withhold_copies) return;  // test hook: the compute warps' waits expire
     constexpr int kPer = kMaxItemTiles / 32;
     const int H = a.kc.num_heads, bs = a.block_size;
-    const uint32_t k_bytes = kBlkWarps * bs * (KF::IB + 2), v_bytes = kBlkWarps * bs * (VF::IB + 2);
+    const uint32_t k_bytes = kBlkWarps * bs * (KF::RB + KF::NB), v_bytes = kBlkWarps * bs * (VF::RB + VF::NB);
     auto read_ids = [&](const Item& it, int (&v)[kPer]) {
         const int nblk = (it.t1 - it.t0 + bs - 1) / bs;
         const int32_t* bt = a.block_tables + static_cast<int64_t>(it.b) * a.max_blocks + it.t0 / bs;
@@ -885,8 +999,8 @@ __device__ void produce_blk(const DecodeArgs& a, BlkSmem& sm, const BlkRing& rin
                 const int64_t sp = (static_cast<int64_t>(blk) * H + cur.h) * bs;  // first of 8 sub-pages
                 const uint32_t dst = ring.slot(s);
                 mbar_expect(full, k_bytes + v_bytes);
-                bulk_copy(dst, a.k_pages + sp * (KF::IB + 2), k_bytes, full);
-                bulk_copy(dst + k_bytes, a.v_pages + sp * (VF::IB + 2), v_bytes, full);
+                bulk_copy(dst, a.k_pages + sp * (KF::RB + KF::NB), k_bytes, full);
+                bulk_copy(dst + k_bytes, a.v_pages + sp * (VF::RB + VF::NB), v_bytes, full);
             }
         }
         stop = __shfl_sync(kFull, stop, 0);
@@ -954,7 +1068,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
     const uint32_t psel = (r & 1) ? 0x7632u : 0x5410u;
     const int rows = group < NH ? group : NH;
     // This warp's head within a slot: K sub-page at k_off, V sub-page at v_off.
-    const uint32_t k_sub = bs * (KF::IB + 2), v_sub = bs * (VF::IB + 2);
+    const uint32_t k_sub = bs * (KF::RB + KF::NB), v_sub = bs * (VF::RB + VF::NB);
     const uint32_t k_off = warp * k_sub, v_off = kBlkWarps * k_sub + warp * v_sub;
     uint32_t consumed = 0;
     WarpTiles<KF, VF, NH> wt;
@@ -969,7 +1083,8 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
             window_state(a, it, h, head0, rows, it.t0, 1, lane, rec, rec + 1, rec + 2, kHeadDim + 2, kHeadDim + 2);
             continue;
         }
-        wt.begin(a.qrot + (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim, rows, r, c);
+        const int64_t q_off = (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim;
+        wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
         bool timed_out = false;
         const int ntiles = (it.t1 - it.t0 + 15) >> 4;
         if constexpr (TPB > 0) {
@@ -983,9 +1098,9 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
                 const uint32_t kb = ring.slot(s) + k_off, vb = ring.slot(s) + v_off;
 #pragma unroll 1
                 for (int j = 0; j < TPB && k + j < ntiles; ++j)
-                    wt.step(kb + 16 * j * KF::IB, kb + kBs * KF::IB + 32 * j, vb + 16 * j * VF::IB,
-                            vb + kBs * VF::IB + 32 * j, min(16, it.t1 - (it.t0 + 16 * (k + j))), lane_base, psel, r,
-                            c);
+                    wt.step(kb + 16 * j * KF::RB, kb + kBs * KF::RB + 16 * KF::NB * j, vb + 16 * j * VF::RB,
+                            vb + kBs * VF::RB + 16 * VF::NB * j, min(16, it.t1 - (it.t0 + 16 * (k + j))), lane_base,
+                            psel, r, c);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with the slot
             }
@@ -1003,8 +1118,8 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
                     kb = ring.slot(s) + k_off;
                     vb = ring.slot(s) + v_off;
                 }
-                wt.step(kb + 16 * j * KF::IB, kb + bs * KF::IB + 32 * j, vb + 16 * j * VF::IB,
-                        vb + bs * VF::IB + 32 * j, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, psel, r, c);
+                wt.step(kb + 16 * j * KF::RB, kb + bs * KF::RB + 16 * KF::NB * j, vb + 16 * j * VF::RB,
+                        vb + bs * VF::RB + 16 * VF::NB * j, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, psel, r, c);
                 if (++j == tpb || k + 1 == ntiles) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with the slot
@@ -1061,8 +1176,9 @@ template <class KF, class VF, int NW>
 __device__ void produce_head(const DecodeArgs& a, Smem<NW>& sm, uint32_t ring_addr, int head_groups,
                              int64_t total_slots, int lane) {
     if (a.withhold_copies) return;  // test hook: the compute warps' waits expire
-    constexpr uint32_t kKRows = 16 * KF::IB, kVRows = 16 * VF::IB;
-    constexpr uint32_t kKTile = kKRows + 32, kTileBytes = kKTile + kVRows + 32;
+    constexpr uint32_t kKRows = 16 * KF::RB, kVRows = 16 * VF::RB;
+    constexpr uint32_t kKNorms = 16 * KF::NB, kVNorms = 16 * VF::NB;
+    constexpr uint32_t kKTile = kKRows + kKNorms, kTileBytes = kKTile + kVRows + kVNorms;
     constexpr uint32_t kStageBytes = stage_bytes<KF, VF>();
     constexpr int kPer = kMaxItemTiles / 32;
     const int H = a.kc.num_heads, bs = a.block_size;
@@ -1121,18 +1237,18 @@ __device__ void produce_head(const DecodeArgs& a, Smem<NW>& sm, uint32_t ring_ad
                 const int tok = cur.t0 + 16 * tl;
                 const int off = bs_pow2 ? (tok & (bs - 1)) : tok % bs;
                 const int64_t sp = (static_cast<int64_t>(blk) * H + cur.h) * bs;
-                const uint8_t* ks = a.k_pages + sp * (KF::IB + 2);
-                const uint8_t* vs = a.v_pages + sp * (VF::IB + 2);
+                const uint8_t* ks = a.k_pages + sp * (KF::RB + KF::NB);
+                const uint8_t* vs = a.v_pages + sp * (VF::RB + VF::NB);
                 const uint32_t dst = my_ring + st * kStageBytes;
                 mbar_expect(full, kTileBytes);
                 if (whole) {
                     bulk_copy(dst, ks, kKTile, full);
-                    bulk_copy(dst + kKTile, vs, kVRows + 32, full);
+                    bulk_copy(dst + kKTile, vs, kVRows + kVNorms, full);
                 } else {
-                    bulk_copy(dst, ks + off * KF::IB, kKRows, full);
-                    bulk_copy(dst + kKRows, ks + bs * KF::IB + 2 * off, 32, full);
-                    bulk_copy(dst + kKTile, vs + off * VF::IB, kVRows, full);
-                    bulk_copy(dst + kKTile + kVRows, vs + bs * VF::IB + 2 * off, 32, full);
+                    bulk_copy(dst, ks + off * KF::RB, kKRows, full);
+                    bulk_copy(dst + kKRows, ks + bs * KF::RB + KF::NB * off, kKNorms, full);
+                    bulk_copy(dst + kKTile, vs + off * VF::RB, kVRows, full);
+                    bulk_copy(dst + kKTile + kVRows, vs + bs * VF::RB + VF::NB * off, kVNorms, full);
                 }
                 ++fill;
             }
@@ -1204,7 +1320,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
             window_state(a, it, it.h, head0, rows, it.t0 + warp, NW, lane, &sm.red_m[warp][0], &sm.red_l[warp][0],
                          &sm.red_o[warp][0][0], 1, kHeadDim);
         } else {
-            wt.begin(a.qrot + (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim, rows, r, c);
+            const int64_t q_off = (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim;
+            wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
             const int ntiles = (it.t1 - it.t0 + 15) >> 4;
             const int n_mine = ntiles > warp ? (ntiles - warp + NW - 1) / NW : 0;
             for (int k = 0; k < n_mine; ++k) {
@@ -1214,8 +1331,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
                     break;
                 }
                 // Slot layout: [K rows][K norms][V rows][V norms].
-                const uint32_t kbase = my_ring + st * kStageBytes, vbase = kbase + 16 * KF::IB + 32;
-                wt.step(kbase, kbase + 16 * KF::IB, vbase, vbase + 16 * VF::IB,
+                const uint32_t kbase = my_ring + st * kStageBytes, vbase = kbase + 16 * (KF::RB + KF::NB);
+                wt.step(kbase, kbase + 16 * KF::RB, vbase, vbase + 16 * VF::RB,
                         min(16, it.t1 - (it.t0 + 16 * (warp + k * NW))), lane_base, psel, r, c);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&sm.empty[warp][st]));  // slot free for the producer
@@ -1260,8 +1377,11 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
 }
 
 // Rotated queries: q_r = pi_K(H(s_K * q) / sqrt(128)) * scale * log2(e), one warp per (b, query head).
+// With QJL keys also qjl_out = sqrt(pi/2)/128 * S q_r, S applied in rotated
+// (not packed) coordinate order, as the residual it projected.
 __global__ void __launch_bounds__(128) rotate_queries_kernel(DevCodec kc, const __nv_bfloat16* q, int num_q_heads,
-                                                              int group, int64_t total, float scale_log2, float* out) {
+                                                              int group, int64_t total, float scale_log2, float* out,
+                                                              float* qjl_out) {
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
     if (row >= total) return;
@@ -1287,7 +1407,60 @@ __global__ void __launch_bounds__(128) rotate_queries_kernel(DevCodec kc, const 
         }
     const float sc = scale_log2 * 0.08838834764831845f;  // 1/sqrt(128)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) out[row * kHeadDim + kc.pos[h * kHeadDim + 4 * lane + i]] = z[i] * sc;
+    for (int i = 0; i < 4; ++i) {
+        z[i] *= sc;
+        out[row * kHeadDim + kc.pos[h * kHeadDim + 4 * lane + i]] = z[i];
+    }
+    if (qjl_out != nullptr) {
+        // (S q_r)_i = sum_j S[i][j] q_r[j]; lane: outputs 4 lane .. 4 lane + 3
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
+        for (int j0 = 0; j0 < kHeadDim; j0 += 4) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const float qj = __shfl_sync(kFull, z[jj], j0 >> 2);
+                const float4 s4 = __ldg(reinterpret_cast<const float4*>(kc.qjl_st + (j0 + jj) * kHeadDim) + lane);
+                acc[0] = fmaf(s4.x, qj, acc[0]);
+                acc[1] = fmaf(s4.y, qj, acc[1]);
+                acc[2] = fmaf(s4.z, qj, acc[2]);
+                acc[3] = fmaf(s4.w, qj, acc[3]);
+            }
+        }
+        constexpr float kappa = 1.2533141373155003f / kHeadDim;  // sqrt(pi/2) / d, the estimator's constant
+        reinterpret_cast<float4*>(qjl_out + row * kHeadDim)[lane] =
+            make_float4(acc[0] * kappa, acc[1] * kappa, acc[2] * kappa, acc[3] * kappa);
+    }
+}
+
+// Group-wise K: q_r = R_h q * scale * log2(e) in packed order (R_h from the
+// codec: rot_t entry (h, j, p) = R_h[p][j]); one warp per (b, query head),
+// lane: packed positions 4 lane .. 4 lane + 3.
+__global__ void __launch_bounds__(128) rotate_queries_dense_kernel(DevCodec kc, const __nv_bfloat16* q,
+                                                                    int num_q_heads, int group, int64_t total,
+                                                                    float scale_log2, float* out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+    if (row >= total) return;
+    const int hq = static_cast<int>(row % num_q_heads), h = hq / group;
+    const uint2 raw = *reinterpret_cast<const uint2*>(q + row * kHeadDim + 4 * lane);
+    const float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
+                        __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u)};
+    const float4* rt = reinterpret_cast<const float4*>(kc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim);
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
+    for (int j0 = 0; j0 < kHeadDim; j0 += 4) {
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const float qj = __shfl_sync(kFull, x[jj], j0 >> 2);
+            const float4 r4 = __ldg(rt + (j0 + jj) * (kHeadDim / 4) + lane);
+            acc[0] = fmaf(r4.x, qj, acc[0]);
+            acc[1] = fmaf(r4.y, qj, acc[1]);
+            acc[2] = fmaf(r4.z, qj, acc[2]);
+            acc[3] = fmaf(r4.w, qj, acc[3]);
+        }
+    }
+    reinterpret_cast<float4*>(out + row * kHeadDim)[lane] =
+        make_float4(acc[0] * scale_log2, acc[1] * scale_log2, acc[2] * scale_log2, acc[3] * scale_log2);
 }
 
 constexpr int kMaxDynSmem = 227 * 1024;
@@ -1322,8 +1495,14 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int head_groups = group > 8 ? group / 8 : 1;
     const int64_t rows = static_cast<int64_t>(a.batch) * a.num_q_heads;
-    rotate_queries_kernel<<<static_cast<unsigned>((rows + 3) / 4), 128, 0, s>>>(
-        a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads, group, rows, a.scale_log2, a.qrot);
+    const unsigned qgrid = static_cast<unsigned>((rows + 3) / 4);
+    if constexpr (KF::MODE == kGroupwise)
+        rotate_queries_dense_kernel<<<qgrid, 128, 0, s>>>(a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads,
+                                                          group, rows, a.scale_log2, a.qrot);
+    else
+        rotate_queries_kernel<<<qgrid, 128, 0, s>>>(a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads,
+                                                    group, rows, a.scale_log2, a.qrot,
+                                                    KF::MODE == kQjl ? a.qjl_q : nullptr);
     const int64_t units = static_cast<int64_t>(a.items_per_unit) * a.batch * head_groups *
                           (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);
     const int grid = static_cast<int>(units < sms ? units : sms);
@@ -1345,6 +1524,8 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
 template <class F>
 bool same_format(const tq_codec* c) {
     const tq_format_desc& d = c->desc;
+    const int mode = d.qjl ? kQjl : (d.groupwise ? kGroupwise : kPlain);
+    if (mode != F::MODE) return false;
     if (F::N1 == 0) return d.n_groups == 1 && d.group_bits[0] == F::B0;
     return d.n_groups == 2 && d.group_bits[0] == F::B0 && d.group_size[0] == F::N0 && d.group_bits[1] == F::B1 &&
            d.group_size[1] == F::N1;
@@ -1355,11 +1536,19 @@ tq_status launch_heads(const DecodeArgs& a, const LutValues& tv, int group, cuda
     return group <= 4 ? launch_fmt<KF, VF, 4>(a, tv, group, s) : launch_fmt<KF, VF, 8>(a, tv, group, s);
 }
 
+// V formats the tensor-core kernel is instantiated for, per K format.
 template <class KF>
 tq_status dispatch_v(const DecodeArgs& a, const tq_codec* vc, const LutValues& tv, int group, cudaStream_t s) {
-    if (same_format<U4>(vc)) return launch_heads<KF, U4>(a, tv, group, s);
-    if (same_format<M43>(vc)) return launch_heads<KF, M43>(a, tv, group, s);
-    if (same_format<U3>(vc)) return launch_heads<KF, U3>(a, tv, group, s);
+    if constexpr (KF::MODE == kGroupwise) {
+        if (same_format<M43G>(vc)) return launch_heads<KF, M43G>(a, tv, group, s);
+    } else if constexpr (KF::MODE == kQjl) {
+        if (same_format<U4>(vc)) return launch_heads<KF, U4>(a, tv, group, s);
+        if (same_format<M43>(vc)) return launch_heads<KF, M43>(a, tv, group, s);
+    } else {
+        if (same_format<U4>(vc)) return launch_heads<KF, U4>(a, tv, group, s);
+        if (same_format<M43>(vc)) return launch_heads<KF, M43>(a, tv, group, s);
+        if (same_format<U3>(vc)) return launch_heads<KF, U3>(a, tv, group, s);
+    }
     return TQ_ERR_UNSUPPORTED;
 }
 
@@ -1369,17 +1558,28 @@ tq_status launch_decode_mma(const DecodeArgs& a, const tq_codec* kc, const tq_co
     if (a.block_size % 16 != 0) return TQ_ERR_UNSUPPORTED;
     if (a.split_tokens > 16 * kMaxItemTiles) return TQ_ERR_UNSUPPORTED;  // the producer's id buffer
     if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return TQ_ERR_UNSUPPORTED;
+    // One table per bit width serves K and V: every group of that width must
+    // share its centroids (group-wise codebooks are per group dimension).
     LutValues tv{};
+    bool set[5] = {false, false, false, false, false};
     for (const tq_codec* c : {kc, vc})
         for (int g = 0; g < c->desc.n_groups; ++g) {
             const int bits = c->desc.group_bits[g];
+            if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
             float* dst = bits == 4 ? tv.c4 : (bits == 3 ? tv.c3 : tv.c2);
-            for (int i = 0; i < (1 << bits); ++i) dst[i] = c->cent[g][i];
+            for (int i = 0; i < (1 << bits); ++i) {
+                if (set[bits] && dst[i] != c->cent[g][i]) return TQ_ERR_UNSUPPORTED;
+                dst[i] = c->cent[g][i];
+            }
+            set[bits] = true;
         }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (same_format<U4>(kc)) return dispatch_v<U4>(a, vc, tv, group, s);
     if (same_format<M43>(kc)) return dispatch_v<M43>(a, vc, tv, group, s);
     if (same_format<M42>(kc)) return dispatch_v<M42>(a, vc, tv, group, s);
+    if (same_format<M32Q>(kc)) return dispatch_v<M32Q>(a, vc, tv, group, s);
+    if (same_format<M43Q>(kc)) return dispatch_v<M43Q>(a, vc, tv, group, s);
+    if (same_format<M43G>(kc)) return dispatch_v<M43G>(a, vc, tv, group, s);
     return TQ_ERR_UNSUPPORTED;
 }
 

@@ -55,6 +55,8 @@ struct DecodeArgs {
     int32_t split_tokens, max_splits, items_per_unit;
     float* ws;                     // records [B][H_kv][items_per_unit][G][2 + 128]
     float* qrot;                   // rotated, scaled queries [B][H_q][128] in K packed order
+    float* qjl_q;                  // QJL keys: sqrt(pi/2)/128 * S q_r of the scaled rotated query,
+                                   // [B][H_q][128] in projection order
     int* d_err;
     // Test hook (TQ_TEST_WITHHOLD_COPIES=1): the tensor-core kernels' producer
     // issues no copies, so the compute warps' bounded waits expire and report

@@ -66,3 +66,43 @@ def test_groupwise_decode_matches_oracle(H, G, kgw, vgw):
             ref = prob.oracle(b, int(hq))
             assert np.abs(got[b, hq] - ref).max() <= 2e-3
             assert np.abs(ref).max() > 0.3
+
+
+@pytest.mark.parametrize("H,G,bs", [(8, 8, 16), (8, 4, 32), (2, 16, 16), (3, 2, 48)])
+def test_groupwise_decode_tensor_core_matches_oracle_and_general(monkeypatch, H, G, bs):
+    """Group-wise K and V (4-bit 64 + 3-bit 64) on the tensor-core kernel: per-group score chains and
+    per-group value weights, against the oracle and the general kernel."""
+    lens = [3, 16 * 2 + 9, 640, 2300]
+    prob = DecodeProblem(lens, H, G, ((4, 3), (64, 64), 63), ((4, 3), (64, 64), 64), window=10, block_size=bs,
+                         seed=90 + H * G, kgw=True, vgw=True)
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "tensor")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fast = prob.run(d_err=err).clone()
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "general")
+    slow = prob.run().clone()
+    torch.cuda.synchronize()
+    assert (fast - slow).abs().max().item() <= 1e-3
+    got = fast.cpu().numpy()
+    rng = np.random.default_rng(H + G)
+    for b in range(prob.B):
+        for hq in rng.choice(prob.Hq, 3, replace=False):
+            ref = prob.oracle(b, int(hq))
+            assert np.abs(got[b, hq] - ref).max() <= 2e-3
+            assert np.abs(ref).max() > 0.3
+
+
+def test_groupwise_format_without_tensor_core_instantiation_runs_general(monkeypatch):
+    """Group-wise K 4-bit 32 + 2-bit 96 with a plain 4-bit V: no tensor-core instantiation (and the two 4-bit
+    codebooks, for dimensions 32 and 128, could not share one table), so forcing the tensor-core path fails
+    and the default call runs the general kernel."""
+    prob = DecodeProblem([100, 900], 8, 4, ((4, 2), (32, 96), 65), ((4,), (128,), 66), window=4, block_size=16,
+                         seed=99, kgw=True)
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "tensor")
+    with pytest.raises(tq.UnsupportedFormatError):
+        prob.run()
+    monkeypatch.delenv("TQ_DECODE_KERNEL")
+    out = prob.run().cpu().numpy()
+    ref = prob.oracle(1, 5)
+    assert np.abs(out[1, 5] - ref).max() <= 2e-3

@@ -103,3 +103,33 @@ def test_qjl_value_codec_is_rejected_by_decode():
                          vqjl=True)
     with pytest.raises(tq.UnsupportedFormatError):
         prob.run()
+
+
+@pytest.mark.parametrize("H,G,kfmt,vfmt,bs", [
+    (8, 4, ((3, 2), (64, 64)), ((4, 3), (64, 64)), 16),   # block kernel, 4 query heads per item, 1 tile per block
+    (8, 8, ((4, 3), (64, 64)), ((4,), (128,)), 32),       # block kernel, 8 query heads, 2 tiles per block
+    (8, 16, ((3, 2), (64, 64)), ((4,), (128,)), 64),      # block kernel, any multiple of 16, 2 head groups
+    (2, 4, ((3, 2), (64, 64)), ((4,), (128,)), 16),       # per-head kernel, whole-sub-page copies
+    (3, 8, ((4, 3), (64, 64)), ((4, 3), (64, 64)), 48),   # per-head kernel, split copies
+])
+def test_qjl_decode_tensor_core_matches_oracle_and_general(monkeypatch, H, G, kfmt, vfmt, bs):
+    """QJL keys on the tensor-core kernel: the sign k-steps against the oracle and the general kernel."""
+    lens = [5, 16 * 3 + 7, 700, 2500]
+    prob = DecodeProblem(lens, H, G, (kfmt[0], kfmt[1], 43), (vfmt[0], vfmt[1], 44), window=12, block_size=bs,
+                         seed=5 * H + G, kqjl=True)
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "tensor")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fast = prob.run(d_err=err).clone()
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "general")
+    slow = prob.run().clone()
+    torch.cuda.synchronize()
+    assert (fast - slow).abs().max().item() <= 1e-3
+    got = fast.cpu().numpy()
+    rng = np.random.default_rng(H * G)
+    for b in range(prob.B):
+        for hq in rng.choice(prob.Hq, 3, replace=False):
+            ref = prob.oracle(b, int(hq))
+            assert np.abs(got[b, hq] - ref).max() <= 2e-3
+            assert np.abs(ref).max() > 0.3
