@@ -36,6 +36,7 @@ from quantized_paged_kv_pack_b200 import tq  # noqa: E402
 from quantized_paged_kv_pack_b200 import workloads as WL  # noqa: E402
 
 HEADLINE = "decode_llama70b_3p5bit"
+SMALL = "decode_gqa8_4k_4bit"
 EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl",
          "decode_llama8b_3p5bit_groupwise",
          "pack_llama8b_4bit"]
@@ -76,8 +77,7 @@ class DecodeSetup:
     """A decode workload resident on the GPU, with the pages written by tq_pack_kv."""
 
     def __init__(self, w: WL.Workload, seed_offset: int = 0):
-        if seed_offset:
-            w = WL.Workload(**{**w.__dict__, "seed": w.seed + 1000 * seed_offset})
+        w = rank_workload(w, seed_offset)
         self.w = w
         ks, vs = WL.codec_specs(w)
         self.kspec, self.vspec = ks, vs
@@ -200,14 +200,23 @@ class PackSetup:
 # --------------------------------------------------------------------------- measurement
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    """SM clocks and throttle reasons sampled while the timed region runs.
+
+    NVML (read-only queries) from a thread every 5 ms, so that a timed region of
+    tens of milliseconds still gets several samples; nvidia-smi (-lms 100) when
+    NVML is not importable. Nothing here changes a GPU setting.
+    """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
     def __init__(self, device_index=0):
         self.proc = None
+        self.thread = None
+        self.samples = []  # (sm MHz, max MHz, reasons)
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
@@ -215,7 +224,33 @@ class ClockSampler:
             sel = str(device_index)
         self.sel = sel
 
+    def _nvml_loop(self, nv, handle, stop):
+        mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+        while not stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+            except Exception:
+                break
+            self.samples.append((float(sm), float(mx), {n for n, b in self.REASON_BITS.items() if bits & b}))
+            stop.wait(0.005)
+
     def __enter__(self):
+        try:
+            import threading
+
+            import pynvml as nv
+
+            nv.nvmlInit()
+            handle = (nv.nvmlDeviceGetHandleByUUID(self.sel) if self.sel.startswith("GPU-")
+                      else nv.nvmlDeviceGetHandleByIndex(int(self.sel)))
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, handle, self.stop), daemon=True)
+            self.thread.start()
+            time.sleep(0.02)
+            return self
+        except Exception:
+            self.thread = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -226,8 +261,11 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            return
         time.sleep(0.15)
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -235,33 +273,31 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for ln in out.splitlines():
+                parts = [q.strip() for q in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, mx = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                self.samples.append((sm, mx, {n for n, v in zip(names, parts[5:9]) if v.lower() == "active"}))
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = set().union(*(r for _, _, r in self.samples))
+        return {"sm_mhz": statistics.median(sm for sm, _, _ in self.samples), "sm_max_mhz": self.samples[-1][1],
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 def time_steps(fns, steps, stream):
     """Run `steps` iterations of the callables in `fns` with events between them.
 
-    Returns (total ms, [per-callable mean ms]). Events are recorded on the
-    stream the library launches on (torch's current stream).
+    Returns (total ms, [per-callable mean ms], [per-step ms]). Events are
+    recorded on the stream the library launches on (torch's current stream).
     """
     n = len(fns)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
@@ -272,9 +308,14 @@ def time_steps(fns, steps, stream):
             f()
             ev[s][i + 1].record(stream)
     torch.cuda.synchronize()
-    total = sum(ev[s][0].elapsed_time(ev[s][n]) for s in range(steps))
+    per_step = [ev[s][0].elapsed_time(ev[s][n]) for s in range(steps)]
     parts = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps for i in range(n)]
-    return total, parts
+    return sum(per_step), parts, per_step
+
+
+def percentiles(xs):
+    q = np.percentile(np.asarray(xs, dtype=np.float64), [10, 50, 90])
+    return {"p10": float(q[0]), "p50": float(q[1]), "p90": float(q[2])}
 
 
 def measure_decode(setup: DecodeSetup, steps, warmup, dist_ctx=None, clocks=True):
@@ -290,12 +331,37 @@ def measure_decode(setup: DecodeSetup, steps, warmup, dist_ctx=None, clocks=True
     sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
     if sampler:
         sampler.__enter__()
-    total_ms, parts = time_steps(fns, steps, stream)
+    total_ms, parts, per_step = time_steps(fns, steps, stream)
     if sampler:
         sampler.__exit__(None, None, None)
     barrier(dist_ctx)
     total_ms = max_over_ranks(total_ms, dist_ctx)
-    return total_ms / steps, parts, (sampler.summary() if sampler else None)
+    return total_ms / steps, parts, (sampler.summary() if sampler else None), per_step
+
+
+def measure_latency(setup: DecodeSetup, reps, warmup, cold):
+    """Decode-call latency (partials + combine) in microseconds, p10 / p50 / p90.
+
+    cold: before every repetition, outside the event pair, a buffer of twice
+    the L2 size is written, so the call starts with none of its data in L2.
+    """
+    stream = torch.cuda.current_stream()
+    l2 = int(getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "L2_cache_size", 0)) or (126 << 20)
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device="cuda") if cold else None
+    for _ in range(warmup):
+        setup.decode()
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        setup.decode()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    del flush
+    return percentiles(times)
 
 
 def measure_decode_e2e(setup: DecodeSetup, steps, warmup):
@@ -319,17 +385,23 @@ def measure_decode_e2e(setup: DecodeSetup, steps, warmup):
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    total, _ = time_steps([step], steps, torch.cuda.current_stream())
+    total, _, _ = time_steps([step], steps, torch.cuda.current_stream())
     h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
     d2h = hout.numel() * 4
     return total / steps, h2d, d2h
 
 
-def measure_pack(setup: PackSetup, steps, warmup):
+def measure_pack(setup: PackSetup, steps, warmup, clocks=False):
     for _ in range(warmup):
         setup.step()
     torch.cuda.synchronize()
-    total, _ = time_steps([setup.step], steps, torch.cuda.current_stream())
+    sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if sampler:
+        sampler.__enter__()
+    total, _, _ = time_steps([setup.step], steps, torch.cuda.current_stream())
+    if sampler:
+        sampler.__exit__(None, None, None)
+        return total / steps, sampler.summary()
     return total / steps
 
 
@@ -353,15 +425,28 @@ def init_dist():
 def barrier(dist_ctx):
     if dist_ctx is not None:
         dist_ctx.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x, dist_ctx):
+    """The largest x over the ranks (step times: the job is as slow as its slowest replica)."""
     if dist_ctx is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist_ctx.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist_ctx.all_reduce(t, op=dist_ctx.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(w: WL.Workload, rank: int) -> WL.Workload:
+    """Rank r's replica of a workload: the same shapes, its own seeded data (weak scaling)."""
+    return WL.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
+
+
+def aggregate_gbs(world: int, bytes_per_rank_step: int, max_step_ms: float) -> float:
+    """Whole-job GB/s: the bytes every rank moved in a step over the slowest rank's step time."""
+    return world * bytes_per_rank_step / (max_step_ms * 1e-3) / 1e9
 
 
 # --------------------------------------------------------------------------- CPU oracle legs
@@ -493,7 +578,7 @@ def workload_of(args):
 def run_pack(args, w, dist_ctx, rank, world):
     """Headline on the pack workload: one step = tq_pack_kv over the whole batch."""
     setup = PackSetup(w)
-    ms = measure_pack(setup, args.steps, args.warmup)
+    ms, clocks = measure_pack(setup, args.steps, args.warmup, clocks=True)
     ms = max_over_ranks(ms, dist_ctx)
     peak, peak_kind = peaks()
     nbytes = setup.bytes()
@@ -509,7 +594,7 @@ def run_pack(args, w, dist_ctx, rank, world):
 
     for _ in range(args.warmup):
         e2e_step()
-    total, _ = time_steps([e2e_step], max(3, args.steps // 2), torch.cuda.current_stream())
+    total, _, _ = time_steps([e2e_step], max(3, args.steps // 2), torch.cuda.current_stream())
     e2e_ms = max_over_ranks(total / max(3, args.steps // 2), dist_ctx)
     gbs = world * nbytes / (ms * 1e-3) / 1e9
     line = {"metric": "TQ pack HBM GB/s (algorithmic bytes / step time)", "value": gbs, "unit": "GB/s",
@@ -524,7 +609,7 @@ def run_pack(args, w, dist_ctx, rank, world):
             "e2e": {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": hk.numel() * 2 + hv.numel() * 2 + hs.numel() * 8,
                     "d2h_bytes_per_step": 4},
-            "gpu_launches": args.steps}
+            "gpu_launches": args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -544,14 +629,14 @@ def run_ours(args):
             dist_ctx.destroy_process_group()
         return rc
     setup = DecodeSetup(w, seed_offset=rank)
-    step_ms, parts, clocks = measure_decode(setup, args.steps, args.warmup, dist_ctx)
+    step_ms, parts, clocks, per_step = measure_decode(setup, args.steps, args.warmup, dist_ctx)
     e2e_ms, h2d, d2h = measure_decode_e2e(setup, max(3, args.steps // 2), args.warmup)
     e2e_ms = max_over_ranks(e2e_ms, dist_ctx)
     peak, peak_kind = peaks()
     split_bytes = setup.decode_split_bytes()
     achieved = split_bytes / (parts[1] * 1e-3) / 1e9
     step_bytes = setup.step_bytes()
-    value = world * step_bytes / (step_ms * 1e-3) / 1e9
+    value = aggregate_gbs(world, step_bytes, step_ms)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -564,13 +649,14 @@ def run_ours(args):
                    "parallelism": f"{world} independent replicas (no collective)",
                    "l2": f"no flush: {split_bytes / 1e9:.2f} GB of pages read per step, L2 is 126 MB"},
         "kv_tokens_per_s": world * setup.kv_tokens() / (step_ms * 1e-3),
+        "step_ms_percentiles": percentiles(per_step),
         "step_breakdown_ms": {"window_append": parts[0], "decode_partials": parts[1], "decode_combine": parts[2]},
         "algorithmic_bytes_per_step": step_bytes,
         "roofline": {"bound": "hbm", "kernel": "decode_partials", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "frac_of_8TBs": achieved / 8000.0,
                      "traffic": stored_traffic(w.name, "tq_decode_mma.cu")},
-        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": aggregate_gbs(world, step_bytes, e2e_ms), "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 4 * args.steps,  # window append, query rotation, decode partials, combine
         "clocks": clocks,
@@ -589,7 +675,9 @@ def run_ours(args):
                 del setup
                 torch.cuda.empty_cache()
                 setup = DecodeSetup(ew)
-                ms, p, _ = measure_decode(setup, max(5, args.steps // 2), args.warmup, None, clocks=False)
+                n_steps = max(5, args.steps // 2)
+                ms, p, _, _ = measure_decode(setup, n_steps, args.warmup, None, clocks=False)
+                line["gpu_launches"] += 4 * n_steps
                 sb = setup.decode_split_bytes()
                 extra[name] = {"GB/s": setup.step_bytes() / (ms * 1e-3) / 1e9,
                                "kv_tokens_per_s": setup.kv_tokens() / (ms * 1e-3), "ms_per_step": ms,
@@ -605,6 +693,14 @@ def run_ours(args):
                 extra[name] = {"GB/s": gbs, "tokens_per_s": setup.k.shape[0] / (ms * 1e-3), "ms_per_step": ms,
                                "frac": gbs / peak, "traffic": stored_traffic(name, "tq_pack_mma.cu")}
                 line["gpu_launches"] += max(5, args.steps // 2)
+        # the small parity case: a latency, hot and with L2 flushed before each call
+        del setup
+        torch.cuda.empty_cache()
+        setup = DecodeSetup(WL.WORKLOADS[SMALL])
+        reps = max(20, args.steps)
+        extra[SMALL] = {"latency_us_hot": measure_latency(setup, reps, args.warmup, cold=False),
+                        "latency_us_cold": measure_latency(setup, reps, args.warmup, cold=True),
+                        "note": "decode call (query rotation, partials, combine); launch- and latency-bound"}
         line["per_workload"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)
