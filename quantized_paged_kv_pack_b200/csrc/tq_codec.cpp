@@ -360,13 +360,17 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
         return false;
     const int G = num_q_heads / num_kv_heads;
     if (G > 16) return false;
-    // Aim for about 4096 packed work items per call, splits of 512..4096 tokens
-    // (at most 32 tiles of 16 tokens for each of a CTA's 8 warps).
+    // Aim for about 4096 packed (sequence, KV head, split) items per call, splits
+    // of 512..4096 tokens (at most 32 tiles of 16 tokens for each of a CTA's 8 warps).
     double total = static_cast<double>(std::max(max_seq_len, 1)) * std::max(batch, 1) * num_kv_heads;
     int64_t s = static_cast<int64_t>(std::ceil(total / 4096.0));
     s = std::min<int64_t>(std::max<int64_t>(s, 512), 4096);
     s = (s + 63) / 64 * 64;
     s = (s + block_size - 1) / block_size * block_size;
+    if (block_size <= 4096) s = std::min<int64_t>(s, 4096 / block_size * block_size);  // e.g. 4080 for 48
+    // (Shorter splits that balance the grid's CTAs better measured slower on
+    // fixed-length batches: more items, and a CTA runs faster when others have
+    // finished. Variable lengths are balanced by the device work list instead.)
     plan->split_tokens = static_cast<int32_t>(s);
     plan->max_splits = static_cast<int32_t>(std::max<int64_t>(1, (max_seq_len + s - 1) / s));
     plan->items_per_unit = plan->max_splits + 1;
@@ -375,9 +379,12 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
     plan->record_bytes = static_cast<size_t>(batch) * num_kv_heads * plan->items_per_unit * plan->record_floats *
                          sizeof(float);
     plan->record_bytes = (plan->record_bytes + 255) / 256 * 256;
-    // then the rotated queries and their QJL projections: 2 x [batch][num_q_heads][128] fp32
-    plan->workspace_bytes =
+    // then the rotated queries and their QJL projections: 2 x [batch][num_q_heads][128] fp32,
+    // then the work list: [batch * items_per_unit][2] int32 and its count
+    plan->list_offset =
         plan->record_bytes + 2 * static_cast<size_t>(batch) * num_q_heads * kHeadDim * sizeof(float);
+    plan->workspace_bytes = plan->list_offset +
+                            (2 * static_cast<size_t>(batch) * plan->items_per_unit + 4) * sizeof(int32_t);
     return true;
 }
 

@@ -413,6 +413,8 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     a.ws = static_cast<float*>(workspace);
     a.qrot = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.record_bytes);
     a.qjl_q = a.qrot + static_cast<size_t>(batch) * num_q_heads * kHeadDim;
+    a.work_list = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + plan.list_offset);
+    a.work_count = a.work_list + 2 * static_cast<size_t>(batch) * plan.items_per_unit;
     a.d_err = d_err;
     const char* withhold = std::getenv("TQ_TEST_WITHHOLD_COPIES");
     a.withhold_copies = withhold && std::string(withhold) == "1";

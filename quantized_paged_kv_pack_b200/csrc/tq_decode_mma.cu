@@ -338,19 +338,35 @@ __device__ __forceinline__ bool item_range(const DecodeArgs& a, Item& it) {
     return true;
 }
 
-// Work slot -> item. Per-head items: (query-head group, KV head, sequence,
-// split). Block items (HB = 8): the KV heads are taken 8 at a time.
+// Work slot -> item. CTA c takes slots c, c + grid, c + 2 grid, ...; slot
+// r * grid + c stands for list position q = r * grid + c in even rounds r and
+// r * grid + (n_r - 1 - c) in odd ones (n_r: the slots of round r), so the
+// longest-first list is dealt in snake order. Position q = (k * hblocks + j) *
+// head_groups + hg is entry k of the work list (sequence, split), KV heads
+// from j * HB (HB = 8 for block items, else 1) and query-head group hg.
 template <int HB>
-__device__ __forceinline__ bool item_of(const DecodeArgs& a, int64_t slot, int head_groups, Item& it) {
+__device__ __forceinline__ bool item_of(const DecodeArgs& a, int64_t slot, int head_groups, int64_t total_slots,
+                                        Item& it) {
     const int hblocks = a.kc.num_heads / HB;
-    int64_t t = slot;
+    const int64_t grid = gridDim.x, r = slot / grid, c = slot - r * grid;
+    const int64_t n_r = total_slots - r * grid < grid ? total_slots - r * grid : grid;
+    int64_t t = r * grid + ((r & 1) ? n_r - 1 - c : c);
     it.hg = static_cast<int>(t % head_groups);
     t /= head_groups;
     it.h = static_cast<int>(t % hblocks) * HB;
     t /= hblocks;
-    it.b = static_cast<int>(t % a.batch);
-    it.split = static_cast<int>(t / a.batch);
+    const int2 e = __ldg(reinterpret_cast<const int2*>(a.work_list) + t);
+    it.b = e.x;
+    it.split = e.y;
     return item_range(a, it);
+}
+
+// Slots of this call: the listed items times the head blocks and groups,
+// at most the launch's bound.
+template <int HB>
+__device__ __forceinline__ int64_t listed_slots(const DecodeArgs& a, int head_groups, int64_t bound) {
+    const int64_t n = static_cast<int64_t>(__ldg(a.work_count)) * (a.kc.num_heads / HB) * head_groups;
+    return n < bound ? n : bound;
 }
 
 // Next packed item of this CTA at or after `slot`; false when none is left.
@@ -358,7 +374,7 @@ template <int HB>
 __device__ __forceinline__ bool next_packed(const DecodeArgs& a, int64_t& slot, int head_groups, int64_t total_slots,
                                             Item& it) {
     for (; slot < total_slots; slot += gridDim.x)
-        if (item_of<HB>(a, slot, head_groups, it) && !it.win) return true;
+        if (item_of<HB>(a, slot, head_groups, total_slots, it) && !it.win) return true;
     return false;
 }
 
@@ -1030,6 +1046,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
     static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
     extern __shared__ __align__(128) uint8_t dsm[];
     BlkSmem& sm = *reinterpret_cast<BlkSmem*>(dsm);
+    total_slots = listed_slots<kBlkWarps>(a, head_groups, total_slots);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, c = lane & 3;
     const int bs = a.block_size;
@@ -1075,7 +1092,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
 
     for (int64_t slot = blockIdx.x; slot < total_slots; slot += gridDim.x) {
         Item it;
-        if (!item_of<kBlkWarps>(a, slot, head_groups, it)) continue;
+        if (!item_of<kBlkWarps>(a, slot, head_groups, total_slots, it)) continue;
         const int h = it.h + warp;                    // this warp's KV head
         const int head0 = h * group + it.hg * 8;      // its first query head of the item
         float* rec = record_of(a, it.b, h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
@@ -1276,6 +1293,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
     static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
     extern __shared__ __align__(128) uint8_t dsm[];
     Smem<NW>& sm = *reinterpret_cast<Smem<NW>*>(dsm);
+    total_slots = listed_slots<1>(a, head_groups, total_slots);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, c = lane & 3;
     constexpr uint32_t kStageBytes = stage_bytes<KF, VF>();
@@ -1314,7 +1332,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
 
     for (int64_t slot = blockIdx.x; slot < total_slots; slot += gridDim.x) {
         Item it;
-        if (!item_of<1>(a, slot, head_groups, it)) continue;
+        if (!item_of<1>(a, slot, head_groups, total_slots, it)) continue;
         const int head0 = it.h * group + it.hg * 8;  // first query head of the item
         if (it.win) {
             window_state(a, it, it.h, head0, rows, it.t0 + warp, NW, lane, &sm.red_m[warp][0], &sm.red_l[warp][0],
@@ -1373,6 +1391,98 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
             }
         }
         named_sync<NW * 32>();
+    }
+}
+
+// Exclusive scan of x over the CTA (1024 threads); total gets the sum.
+__device__ __forceinline__ int block_exclusive_scan(int x, int* warp_tot, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int v = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, w, o);
+            if (lane >= o) w += y;
+        }
+        warp_tot[lane] = w;  // inclusive over the warps
+    }
+    __syncthreads();
+    const int excl = (warp ? warp_tot[warp - 1] : 0) + v - x;
+    total = warp_tot[nw - 1];
+    __syncthreads();  // warp_tot is reused by the next call
+    return excl;
+}
+
+// Work list of the tensor-core kernels: the (sequence, split) pairs of every
+// non-empty work item, longest first: every full split (sequence by
+// sequence), then the partial last splits by decreasing tile count (a
+// counting sort), then the windows; and their number. Dealt in snake order
+// (item_of), this balances the persistent CTAs about as well as greedy
+// longest-first assignment. One CTA of 1024 threads, two passes.
+constexpr int kListBuckets = kMaxItemTiles + 1;  // partial splits by tile count 1 .. 256
+
+__global__ void __launch_bounds__(1024) work_list_kernel(DecodeArgs a) {
+    __shared__ int cursor[kListBuckets];  // pass 1: partial splits per tile count; then write cursors
+    __shared__ int warp_tot[32];
+    __shared__ int tot_full, tot_win, base_full, base_win;
+    const int tid = threadIdx.x;
+    auto geometry = [&](int b, int& nf, int& part_tiles, int& win) {
+        int L = __ldg(a.seq_lens + b);
+        L = L < 0 ? 0 : (L > a.max_seq_len ? a.max_seq_len : L);
+        const int n_win = min(a.window, L), P = L - n_win;
+        nf = P / a.split_tokens;
+        const int rem = P - nf * a.split_tokens;
+        part_tiles = (rem + 15) >> 4;
+        win = n_win > 0;
+    };
+    for (int i = tid; i < kListBuckets; i += blockDim.x) cursor[i] = 0;
+    if (tid == 0) tot_full = tot_win = 0;
+    __syncthreads();
+    for (int b = tid; b < a.batch; b += blockDim.x) {
+        int nf, pt, win;
+        geometry(b, nf, pt, win);
+        if (nf) atomicAdd(&tot_full, nf);
+        if (pt) atomicAdd(&cursor[pt], 1);
+        if (win) atomicAdd(&tot_win, 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int pos = tot_full;
+        for (int k = kListBuckets - 1; k >= 1; --k) {
+            const int n = cursor[k];
+            cursor[k] = pos;
+            pos += n;
+        }
+        base_full = 0;
+        base_win = pos;
+        *a.work_count = pos + tot_win;
+    }
+    __syncthreads();
+    int2* list = reinterpret_cast<int2*>(a.work_list);
+    for (int b0 = 0; b0 < a.batch; b0 += blockDim.x) {
+        const int b = b0 + tid;
+        int nf = 0, pt = 0, win = 0;
+        if (b < a.batch) geometry(b, nf, pt, win);
+        int n_full, n_win;
+        const int of = block_exclusive_scan(nf, warp_tot, n_full);
+        const int ow = block_exclusive_scan(win, warp_tot, n_win);
+        for (int j = 0; j < nf; ++j) list[base_full + of + j] = make_int2(b, j);
+        if (pt) list[atomicAdd(&cursor[pt], 1)] = make_int2(b, nf);
+        if (win) list[base_win + ow] = make_int2(b, a.max_splits);
+        __syncthreads();
+        if (tid == 0) {
+            base_full += n_full;
+            base_win += n_win;
+        }
+        __syncthreads();
     }
 }
 
@@ -1495,6 +1605,7 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int head_groups = group > 8 ? group / 8 : 1;
     const int64_t rows = static_cast<int64_t>(a.batch) * a.num_q_heads;
+    work_list_kernel<<<1, 1024, 0, s>>>(a);
     const unsigned qgrid = static_cast<unsigned>((rows + 3) / 4);
     if constexpr (KF::MODE == kGroupwise)
         rotate_queries_dense_kernel<<<qgrid, 128, 0, s>>>(a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads,

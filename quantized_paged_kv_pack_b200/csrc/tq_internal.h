@@ -57,6 +57,9 @@ struct DecodeArgs {
     float* qrot;                   // rotated, scaled queries [B][H_q][128] in K packed order
     float* qjl_q;                  // QJL keys: sqrt(pi/2)/128 * S q_r of the scaled rotated query,
                                    // [B][H_q][128] in projection order
+    int32_t* work_list;            // tensor-core kernels: (sequence, split) pairs of the non-empty
+                                   // work items, [B * items_per_unit][2], built on the device
+    int32_t* work_count;           // number of pairs in work_list
     int* d_err;
     // Test hook (TQ_TEST_WITHHOLD_COPIES=1): the tensor-core kernels' producer
     // issues no copies, so the compute warps' bounded waits expire and report
@@ -107,6 +110,7 @@ struct SplitPlan {
     int32_t group;          // query heads per KV head
     size_t record_floats;   // floats per work item record
     size_t record_bytes;    // bytes of all records (256-byte multiple); rotated queries follow
+    size_t list_offset;     // byte offset of the work list (and then its count) in the workspace
     size_t workspace_bytes;
 };
 bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,

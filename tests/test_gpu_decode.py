@@ -243,3 +243,30 @@ def test_decode_boundary_tokens_dense(H, bs):
     rng = np.random.default_rng(H)
     pairs = [(b, int(hq)) for b in range(prob.B) for hq in rng.choice(prob.Hq, min(prob.Hq, 6), replace=False)]
     check(prob, pairs)
+
+
+@pytest.mark.parametrize("H", [8, 2])  # the block kernel and the per-head kernel
+def test_decode_many_sequences_work_list(monkeypatch, H):
+    """More sequences than the work-list scan takes in one pass (1024), many of them empty or window-only:
+    the tensor-core kernels deal only the listed items; every sequence is checked against the general
+    kernel and a sample against the oracle."""
+    rng = np.random.default_rng(11)
+    lens = rng.integers(0, 90, 1500)
+    lens[::7] = 0
+    lens[::11] = rng.integers(300, 700, len(lens[::11]))
+    prob = DecodeProblem(lens.tolist(), H, 4, M35, M35, window=16, block_size=16, seed=12)
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "tensor")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fast = prob.run(d_err=err).clone()
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "general")
+    slow = prob.run().clone()
+    torch.cuda.synchronize()
+    assert (fast - slow).abs().max().item() <= 1e-3
+    got = fast.cpu().numpy()
+    for b in [int(i) for i in rng.choice(np.flatnonzero(lens > 0), 6, replace=False)] + [1499]:
+        if lens[b] == 0:
+            continue
+        hq = int(rng.integers(prob.Hq))
+        assert np.abs(got[b, hq] - prob.oracle(b, hq)).max() <= ATOL
