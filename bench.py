@@ -37,6 +37,7 @@ from quantized_paged_kv_pack_b200 import workloads as WL  # noqa: E402
 
 HEADLINE = "decode_llama70b_3p5bit"
 SMALL = "decode_gqa8_4k_4bit"
+DECODE_LAUNCHES = 6  # per step with a window: append, work list, query rotation, window, partials, combine
 EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl",
          "decode_llama8b_3p5bit_groupwise",
          "pack_llama8b_4bit"]
@@ -658,7 +659,8 @@ def run_ours(args):
                      "traffic": stored_traffic(w.name, "tq_decode_mma.cu")},
         "e2e": {"value": aggregate_gbs(world, step_bytes, e2e_ms), "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,  # window append, query rotation, decode partials, combine
+        # window append, work list, query rotation, window, decode partials, combine
+        "gpu_launches": DECODE_LAUNCHES * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -677,7 +679,7 @@ def run_ours(args):
                 setup = DecodeSetup(ew)
                 n_steps = max(5, args.steps // 2)
                 ms, p, _, _ = measure_decode(setup, n_steps, args.warmup, None, clocks=False)
-                line["gpu_launches"] += 4 * n_steps
+                line["gpu_launches"] += DECODE_LAUNCHES * n_steps
                 sb = setup.decode_split_bytes()
                 extra[name] = {"GB/s": setup.step_bytes() / (ms * 1e-3) / 1e9,
                                "kv_tokens_per_s": setup.kv_tokens() / (ms * 1e-3), "ms_per_step": ms,

@@ -67,8 +67,7 @@ static_assert(kNW >= 1 && kNW <= 11, "11 compute warps fill the shared memory");
 constexpr int kStages = TQ_DECODE_STAGES;  // ring slots per compute warp
 constexpr int kLut = 65536;         // bytes of the dequantization table
 constexpr uint32_t kSpinLimit = 1u << 24;   // polls of a spinning wait
-constexpr uint32_t kWaitHintNs = 16384;     // sleep bound of one blocking wait attempt
-constexpr uint32_t kWaitRounds = 1u << 16;  // blocking wait attempts (about a second)
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bound of one mbarrier wait (global timer, 1 s)
 constexpr float kSlack = 8.0f;                 // log2 slack of the running max
 
 #pragma nv_diag_suppress 177  // not every format constant is used by every instantiation
@@ -196,23 +195,32 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// One wait attempt: the thread sleeps until phase `parity` of `bar` completes
-// or about kWaitHintNs pass; true when the phase completed.
+// One wait attempt: the thread may be suspended until phase `parity` of
+// `bar` completes or a system-dependent time passes; true when the phase
+// completed. (The form without a suspend-time hint measured about 1.5 %
+// faster; the hint's length made no difference.)
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity), "n"(kWaitHintNs)
+        : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
 }
-// Bounded wait for phase `parity` of `bar` (about a second at most); false
-// when the limit expired.
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait for phase `parity` of `bar`: false when kWaitLimitNs of the
+// global timer passed first.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitRounds; ++i)
-        if (mbar_try(bar, parity)) return true;
-    return false;
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    return true;
 }
 
 // NB bytes at shared address a (4-byte aligned when ALIGNED) into words.
@@ -879,27 +887,70 @@ __device__ __forceinline__ void window_state(const DecodeArgs& a, const Item& it
     }
     const __nv_bfloat16* kw = static_cast<const __nv_bfloat16*>(a.k_win);
     const __nv_bfloat16* vw = static_cast<const __nv_bfloat16*>(a.v_win);
-    for (int tk = t_first; tk < it.t1; tk += t_step) {
-        const int64_t base = ((static_cast<int64_t>(it.b) * H + h) * a.window + tk) * kHeadDim + 4 * lane;
-        const uint2 kr = *reinterpret_cast<const uint2*>(kw + base);
-        const uint2 vr = *reinterpret_cast<const uint2*>(vw + base);
-        const float kx[4] = {__uint_as_float(kr.x << 16), __uint_as_float(kr.x & 0xffff0000u),
-                             __uint_as_float(kr.y << 16), __uint_as_float(kr.y & 0xffff0000u)};
-        const float vx[4] = {__uint_as_float(vr.x << 16), __uint_as_float(vr.x & 0xffff0000u),
-                             __uint_as_float(vr.y << 16), __uint_as_float(vr.y & 0xffff0000u)};
+    const int64_t row0 = (static_cast<int64_t>(it.b) * H + h) * a.window;
+    const bool b4 = lane & 16, b3 = lane & 8;
+    // Four tokens at a time: their loads are issued together, and the four
+    // partial dot products of a head are summed over the warp by a transposed
+    // butterfly (the first two steps halve the values a lane carries; lane 8u
+    // ends with token u), then broadcast: 10 shuffles for 4 tokens instead of 20.
+    for (int t0 = t_first; t0 < it.t1; t0 += 4 * t_step) {
+        float kx[4][4], vx[4][4];
+        bool ok[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int tk = t0 + u * t_step;
+            ok[u] = tk < it.t1;
+            uint2 kr = make_uint2(0u, 0u), vr = make_uint2(0u, 0u);
+            if (ok[u]) {
+                const int64_t base = (row0 + tk) * kHeadDim + 4 * lane;
+                kr = *reinterpret_cast<const uint2*>(kw + base);
+                vr = *reinterpret_cast<const uint2*>(vw + base);
+            }
+            kx[u][0] = __uint_as_float(kr.x << 16);
+            kx[u][1] = __uint_as_float(kr.x & 0xffff0000u);
+            kx[u][2] = __uint_as_float(kr.y << 16);
+            kx[u][3] = __uint_as_float(kr.y & 0xffff0000u);
+            vx[u][0] = __uint_as_float(vr.x << 16);
+            vx[u][1] = __uint_as_float(vr.x & 0xffff0000u);
+            vx[u][2] = __uint_as_float(vr.y << 16);
+            vx[u][3] = __uint_as_float(vr.y & 0xffff0000u);
+        }
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
             if (g < rows) {
-                float sc = qv[g][0] * kx[0] + qv[g][1] * kx[1] + qv[g][2] * kx[2] + qv[g][3] * kx[3];
+                float p[4];
 #pragma unroll
-                for (int mm = 16; mm; mm >>= 1) sc += __shfl_xor_sync(kFull, sc, mm);
-                const float mn = fmaxf(m[g], sc);
-                const float alpha = ex2(m[g] - mn);
-                const float p = ex2(sc - mn);
-                l[g] = l[g] * alpha + p;
+                for (int u = 0; u < 4; ++u)
+                    p[u] = qv[g][0] * kx[u][0] + qv[g][1] * kx[u][1] + qv[g][2] * kx[u][2] + qv[g][3] * kx[u][3];
+                float q2[2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[g][i] = acc[g][i] * alpha + p * vx[i];
-                m[g] = mn;
+                for (int i = 0; i < 2; ++i) {  // lanes with bit 4 keep tokens 2, 3, the others 0, 1
+                    const float mine = b4 ? p[i + 2] : p[i], other = b4 ? p[i] : p[i + 2];
+                    q2[i] = mine + __shfl_xor_sync(kFull, other, 16);
+                }
+                float q1 = (b3 ? q2[1] : q2[0]) + __shfl_xor_sync(kFull, b3 ? q2[0] : q2[1], 8);
+                q1 += __shfl_xor_sync(kFull, q1, 4);
+                q1 += __shfl_xor_sync(kFull, q1, 2);
+                q1 += __shfl_xor_sync(kFull, q1, 1);
+                float sc[4], mx = m[g];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    sc[u] = ok[u] ? __shfl_sync(kFull, q1, 8 * u) : -INFINITY;
+                    mx = fmaxf(mx, sc[u]);
+                }
+                const float alpha = ex2(m[g] - mx);  // token t0 is valid, so mx is finite
+                float ls = l[g] * alpha;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[g][i] *= alpha;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float pu = ex2(sc[u] - mx);
+                    ls += pu;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[g][i] = fmaf(pu, vx[u][i], acc[g][i]);
+                }
+                l[g] = ls;
+                m[g] = mx;
             }
         }
     }
@@ -1096,10 +1147,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
         const int h = it.h + warp;                    // this warp's KV head
         const int head0 = h * group + it.hg * 8;      // its first query head of the item
         float* rec = record_of(a, it.b, h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
-        if (it.win) {
-            window_state(a, it, h, head0, rows, it.t0, 1, lane, rec, rec + 1, rec + 2, kHeadDim + 2, kHeadDim + 2);
-            continue;
-        }
+        if (it.win) continue;  // windows are not listed: window_kernel takes them
         const int64_t q_off = (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim;
         wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
         bool timed_out = false;
@@ -1334,10 +1382,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
         Item it;
         if (!item_of<1>(a, slot, head_groups, total_slots, it)) continue;
         const int head0 = it.h * group + it.hg * 8;  // first query head of the item
-        if (it.win) {
-            window_state(a, it, it.h, head0, rows, it.t0 + warp, NW, lane, &sm.red_m[warp][0], &sm.red_l[warp][0],
-                         &sm.red_o[warp][0][0], 1, kHeadDim);
-        } else {
+        if (it.win) continue;  // windows are not listed: window_kernel takes them
+        {
             const int64_t q_off = (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim;
             wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
             const int ntiles = (it.t1 - it.t0 + 15) >> 4;
@@ -1422,36 +1468,35 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_tot, int& t
 }
 
 // Work list of the tensor-core kernels: the (sequence, split) pairs of every
-// non-empty work item, longest first: every full split (sequence by
+// non-empty packed work item, longest first: every full split (sequence by
 // sequence), then the partial last splits by decreasing tile count (a
-// counting sort), then the windows; and their number. Dealt in snake order
-// (item_of), this balances the persistent CTAs about as well as greedy
-// longest-first assignment. One CTA of 1024 threads, two passes.
+// counting sort); and their number. Dealt in snake order (item_of), this
+// balances the persistent CTAs about as well as greedy longest-first
+// assignment. (The windows are window_kernel's.) One CTA of 1024 threads, two
+// passes.
 constexpr int kListBuckets = kMaxItemTiles + 1;  // partial splits by tile count 1 .. 256
 
 __global__ void __launch_bounds__(1024) work_list_kernel(DecodeArgs a) {
     __shared__ int cursor[kListBuckets];  // pass 1: partial splits per tile count; then write cursors
     __shared__ int warp_tot[32];
-    __shared__ int tot_full, tot_win, base_full, base_win;
+    __shared__ int tot_full, base_full;
     const int tid = threadIdx.x;
-    auto geometry = [&](int b, int& nf, int& part_tiles, int& win) {
+    auto geometry = [&](int b, int& nf, int& part_tiles) {
         int L = __ldg(a.seq_lens + b);
         L = L < 0 ? 0 : (L > a.max_seq_len ? a.max_seq_len : L);
-        const int n_win = min(a.window, L), P = L - n_win;
+        const int P = L - min(a.window, L);
         nf = P / a.split_tokens;
         const int rem = P - nf * a.split_tokens;
         part_tiles = (rem + 15) >> 4;
-        win = n_win > 0;
     };
     for (int i = tid; i < kListBuckets; i += blockDim.x) cursor[i] = 0;
-    if (tid == 0) tot_full = tot_win = 0;
+    if (tid == 0) tot_full = 0;
     __syncthreads();
     for (int b = tid; b < a.batch; b += blockDim.x) {
-        int nf, pt, win;
-        geometry(b, nf, pt, win);
+        int nf, pt;
+        geometry(b, nf, pt);
         if (nf) atomicAdd(&tot_full, nf);
         if (pt) atomicAdd(&cursor[pt], 1);
-        if (win) atomicAdd(&tot_win, 1);
     }
     __syncthreads();
     if (tid == 0) {
@@ -1462,27 +1507,70 @@ __global__ void __launch_bounds__(1024) work_list_kernel(DecodeArgs a) {
             pos += n;
         }
         base_full = 0;
-        base_win = pos;
-        *a.work_count = pos + tot_win;
+        *a.work_count = pos;
     }
     __syncthreads();
     int2* list = reinterpret_cast<int2*>(a.work_list);
     for (int b0 = 0; b0 < a.batch; b0 += blockDim.x) {
         const int b = b0 + tid;
-        int nf = 0, pt = 0, win = 0;
-        if (b < a.batch) geometry(b, nf, pt, win);
-        int n_full, n_win;
+        int nf = 0, pt = 0;
+        if (b < a.batch) geometry(b, nf, pt);
+        int n_full;
         const int of = block_exclusive_scan(nf, warp_tot, n_full);
-        const int ow = block_exclusive_scan(win, warp_tot, n_win);
         for (int j = 0; j < nf; ++j) list[base_full + of + j] = make_int2(b, j);
         if (pt) list[atomicAdd(&cursor[pt], 1)] = make_int2(b, nf);
-        if (win) list[base_win + ow] = make_int2(b, a.max_splits);
         __syncthreads();
-        if (tid == 0) {
-            base_full += n_full;
-            base_win += n_win;
+        if (tid == 0) base_full += n_full;
+        __syncthreads();
+    }
+}
+
+// The dense bf16 window of each (sequence, KV head, group of <= 8 query
+// heads), on CUDA cores: one CTA of kWinWarps warps, warp w takes window
+// tokens w, w + kWinWarps, ...; the warps merge their (max, sum, accumulator)
+// states in shared memory into the window's record (split max_splits).
+constexpr int kWinWarps = 4;
+
+__global__ void __launch_bounds__(kWinWarps * 32) window_kernel(DecodeArgs a, int group, int head_groups) {
+    __shared__ float red_m[kWinWarps][8], red_l[kWinWarps][8];
+    __shared__ float red_o[kWinWarps][8][kHeadDim];
+    const int H = a.kc.num_heads;
+    int64_t u = blockIdx.x;
+    Item it;
+    it.hg = static_cast<int>(u % head_groups);
+    u /= head_groups;
+    it.h = static_cast<int>(u % H);
+    it.b = static_cast<int>(u / H);
+    it.split = a.max_splits;
+    if (!item_range(a, it)) return;  // no window tokens
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = group < 8 ? group : 8;
+    const int head0 = it.h * group + it.hg * 8;
+    window_state(a, it, it.h, head0, rows, warp, kWinWarps, lane, &red_m[warp][0], &red_l[warp][0],
+                 &red_o[warp][0][0], 1, kHeadDim);
+    __syncthreads();
+    float* rec = record_of(a, it.b, it.h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
+    for (int e = threadIdx.x; e < rows * kHeadDim; e += kWinWarps * 32) {
+        const int g = e / kHeadDim, j = e - g * kHeadDim;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWinWarps; ++w) M = fmaxf(M, red_m[w][g]);
+        float Ls = 0.0f, A = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWinWarps; ++w) {
+            const float mw = red_m[w][g];
+            if (mw != -INFINITY) {
+                const float f = ex2(mw - M);
+                Ls += red_l[w][g] * f;
+                A += red_o[w][g][j] * f;
+            }
         }
-        __syncthreads();
+        float* rg = rec + g * (kHeadDim + 2);
+        rg[2 + j] = A;
+        if (j == 0) {
+            rg[0] = M;
+            rg[1] = Ls;
+        }
     }
 }
 
@@ -1606,6 +1694,9 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     const int head_groups = group > 8 ? group / 8 : 1;
     const int64_t rows = static_cast<int64_t>(a.batch) * a.num_q_heads;
     work_list_kernel<<<1, 1024, 0, s>>>(a);
+    if (a.window > 0 && a.batch > 0)
+        window_kernel<<<static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.kc.num_heads * head_groups),
+                        kWinWarps * 32, 0, s>>>(a, group, head_groups);
     const unsigned qgrid = static_cast<unsigned>((rows + 3) / 4);
     if constexpr (KF::MODE == kGroupwise)
         rotate_queries_dense_kernel<<<qgrid, 128, 0, s>>>(a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads,
