@@ -606,7 +606,7 @@ def run_pack(args, w, dist_ctx, rank, world):
             "tokens_per_s": world * setup.k.shape[0] / (ms * 1e-3),
             "roofline": {"bound": "hbm", "kernel": "pack", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / peak,
-                         "traffic": stored_traffic(w.name, "tq_pack_mma.cu")},
+                         "traffic": None if args.batch else stored_traffic(w.name, "tq_pack_mma.cu")},
             "e2e": {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": hk.numel() * 2 + hv.numel() * 2 + hs.numel() * 8,
                     "d2h_bytes_per_step": 4},
@@ -656,7 +656,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": "decode_partials", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "frac_of_8TBs": achieved / 8000.0,
-                     "traffic": stored_traffic(w.name, "tq_decode_mma.cu")},
+                     "traffic": None if args.batch else stored_traffic(w.name, "tq_decode_mma.cu")},
         "e2e": {"value": aggregate_gbs(world, step_bytes, e2e_ms), "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         # window append, work list, query rotation, window, decode partials, combine
