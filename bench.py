@@ -535,6 +535,15 @@ def oracle_decode_sample(w, kspec, vspec, lay, unit_source, budget_s: float, row
     return done_bytes / elapsed / 1e9, done_tok / elapsed, desc, threads
 
 
+def oracle_decode_sample_one_thread(w, kspec, vspec, lay, unit_source, budget_s: float, row_bytes):
+    """The same oracle sample with NumPy's BLAS and OpenMP pools held to one thread."""
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(limits=1):
+        gbs, tps, desc, _ = oracle_decode_sample(w, kspec, vspec, lay, unit_source, budget_s, row_bytes)
+    return gbs, tps, desc, 1
+
+
 # --------------------------------------------------------------------------- main
 
 def run_reference(args):
@@ -669,6 +678,11 @@ def run_ours(args):
             setup.kc.row_bytes + setup.vc.row_bytes)
         line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
                                 "kv_token_heads_per_s": tps}
+        gbs1, tps1, desc1, _ = oracle_decode_sample_one_thread(
+            w, setup.kspec, setup.vspec, setup.layout, lambda b, h: gpu_pages_unit(setup, b, h),
+            args.cpu_budget / 2, setup.kc.row_bytes + setup.vc.row_bytes)
+        line["cpu_baseline"]["one_thread"] = {"value": gbs1, "unit": "GB/s", "cores": 1, "sample": desc1,
+                                              "kv_token_heads_per_s": tps1}
     if world == 1 and not args.no_extra:
         extra = {}
         for name in EXTRA:

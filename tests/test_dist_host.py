@@ -98,3 +98,16 @@ def test_reference_arm_line_on_rank_zero():
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_oracle_baseline_sample_with_one_thread():
+    """The benchmark's CPU-oracle baseline, held to one thread, on the small parity workload."""
+    w = WL.WORKLOADS["decode_gqa8_4k_4bit"]
+    kspec, vspec = WL.codec_specs(w)
+    lay = WL.page_layout(w)
+    from oracle import tq_oracle as O
+
+    rb = sum(O.row_bytes(O.Format(128, 1, s.group_bits, s.group_size, None, s.seed)) for s in (kspec, vspec))
+    src = lambda b, h: bench.oracle_pages_unit(w, kspec, vspec, lay, b, h)  # noqa: E731
+    gbs, tps, desc, threads = bench.oracle_decode_sample_one_thread(w, kspec, vspec, lay, src, 0.0, rb)
+    assert threads == 1 and gbs > 0 and tps > 0 and "sequence 0" in desc
