@@ -683,6 +683,8 @@ def run_ours(args):
             args.cpu_budget / 2, setup.kc.row_bytes + setup.vc.row_bytes)
         line["cpu_baseline"]["one_thread"] = {"value": gbs1, "unit": "GB/s", "cores": 1, "sample": desc1,
                                               "kv_token_heads_per_s": tps1}
+        line["cpu_baseline"]["note"] = ("cores = the host threads NumPy's thread pools may use; the oracle is "
+                                        "mostly element-wise NumPy, and one_thread is its serial rate")
     if world == 1 and not args.no_extra:
         extra = {}
         for name in EXTRA:
