@@ -225,9 +225,20 @@ def test_row_bit_layout_golden(golden_dir):
     for case in _golden(golden_dir, "row_bit_layout.json")["cases"]:
         d = sum(case["group_size"])
         high = np.arange(case["group_size"][0])[None, :] if len(case["group_bits"]) == 2 else None
-        f = O.Format(d, 1, tuple(case["group_bits"]), tuple(case["group_size"]), high, 0)
-        row = O.encode_rows(np.array([case["indices"]]), np.array([case["norm"]]), f)[0]
+        qjl, gw = case.get("qjl", False), case.get("groupwise", False)
+        f = O.Format(d, 1, tuple(case["group_bits"]), tuple(case["group_size"]), high, 0, qjl=qjl, groupwise=gw)
+        idx = np.array([case["indices"]])
+        if gw:
+            row = O.encode_rows(idx, np.array([case["norms"]]), f)[0]
+        elif qjl:
+            row = O.encode_rows(idx, np.array([case["norm"]]), f, signs=np.array([case["signs"]]),
+                                g16=np.array([case["residual_norm"]]))[0]
+        else:
+            row = O.encode_rows(idx, np.array([case["norm"]]), f)[0]
+        assert len(row) == O.row_bytes(f)
         assert bytes(row).hex() == case["row_hex"]
+        back = O.decode_rows(row[None], f)
+        assert np.array_equal(back[0][0], case["indices"])
 
 
 def test_permutation_puts_high_coords_first():
