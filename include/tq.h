@@ -139,6 +139,20 @@ tq_status tq_codec_host_tables(const tq_format_desc* desc, uint16_t* centroids_f
 tq_status tq_codec_qjl_matrix(const tq_format_desc* desc, float* out);
 
 /*
+ * The group-wise rotations of a codec ([Design] "Recipe Strategy": the high
+ * channels come from calibration metadata; this library's group-wise reading,
+ * groupwise = 1): out, float [num_kv_heads][head_dim][head_dim], row-major,
+ * out[h][p][j] = R_h[p][j], the weight of original channel j in packed
+ * position p. Rows 0 .. group_size[0] - 1 are group 0 (channels
+ * high_coords[h], ascending), the rest group 1 (the other channels,
+ * ascending); each group's rows are the orthonormal natural-order Hadamard
+ * blocks of the powers of two that make up its size, largest first, applied
+ * after the sign flip s[j]. Host only; TQ_ERR_VALUE for an invalid
+ * descriptor or one without groupwise.
+ */
+tq_status tq_codec_group_rotation(const tq_format_desc* desc, float* out);
+
+/*
  * Validate `desc`, build the codec tables on the host and copy them to the
  * current device. *out receives the codec; free it with tq_free_codec (not
  * while kernels that use it are in flight).

@@ -414,6 +414,25 @@ tq_status tq_codec_host_tables(const tq_format_desc* desc, uint16_t* centroids_f
     return TQ_OK;
 }
 
+tq_status tq_codec_group_rotation(const tq_format_desc* desc, float* out) {
+    clear_error();
+    tq_status st = validate_desc(desc);
+    if (st != TQ_OK) return st;
+    if (!desc->groupwise) return fail(TQ_ERR_VALUE, "the format is not group-wise");
+    if (!out) return fail(TQ_ERR_VALUE, "null output pointer");
+    tq_codec c;
+    st = build_host_tables(desc, &c);
+    if (st != TQ_OK) return st;
+    const size_t d = static_cast<size_t>(desc->head_dim);
+    for (int h = 0; h < desc->num_kv_heads; ++h) {
+        const float* rt = c.rot_t.data() + static_cast<size_t>(h) * d * d;  // entry (j, p) = R_h[p][j]
+        float* r = out + static_cast<size_t>(h) * d * d;
+        for (size_t p = 0; p < d; ++p)
+            for (size_t j = 0; j < d; ++j) r[p * d + j] = rt[j * d + p];
+    }
+    return TQ_OK;
+}
+
 tq_status tq_codec_qjl_matrix(const tq_format_desc* desc, float* out) {
     clear_error();
     tq_status st = validate_desc(desc);

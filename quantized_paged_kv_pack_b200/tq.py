@@ -67,6 +67,7 @@ def lib():
         L.tq_last_error.restype = ctypes.c_char_p
         L.tq_codec_host_tables.argtypes = [P(_FormatDesc), _VP, _VP, _VP, _VP, _VP]
         L.tq_codec_qjl_matrix.argtypes = [P(_FormatDesc), _VP]
+        L.tq_codec_group_rotation.argtypes = [P(_FormatDesc), _VP]
         L.tq_make_codec.argtypes = [P(_FormatDesc), P(_VP)]
         L.tq_free_codec.argtypes = [_VP]
         L.tq_free_codec.restype = None
@@ -84,7 +85,7 @@ def lib():
                                        _I32, _I32, _VP, _VP]
         L.tq_byte_ledger.argtypes = [P(_FormatDesc), P(_FormatDesc), _I32, _VP, _I32, _I32, _I32, _I64, _I32,
                                      P(_Ledger)]
-        for name in ("tq_codec_host_tables", "tq_codec_qjl_matrix", "tq_make_codec", "tq_pack_kv", "tq_decode_paged",
+        for name in ("tq_codec_host_tables", "tq_codec_qjl_matrix", "tq_codec_group_rotation", "tq_make_codec", "tq_pack_kv", "tq_decode_paged",
                      "tq_decode_partials", "tq_decode_combine", "tq_byte_ledger", "tq_decode_paged_static",
                      "tq_window_append"):
             getattr(L, name).restype = ctypes.c_int
@@ -147,6 +148,15 @@ def qjl_matrix(head_dim, num_kv_heads, group_bits, group_size, high_coords=None,
     d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, True)
     out = np.zeros((head_dim, head_dim), np.float32)
     _check(lib().tq_codec_qjl_matrix(ctypes.byref(d), out.ctypes.data))
+    del keep
+    return out
+
+
+def group_rotation(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed=0) -> np.ndarray:
+    """R_h of a group-wise codec (tq_codec_group_rotation), float32 [H][head_dim][head_dim]; host only."""
+    d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, False, True)
+    out = np.zeros((num_kv_heads, head_dim, head_dim), np.float32)
+    _check(lib().tq_codec_group_rotation(ctypes.byref(d), out.ctypes.data))
     del keep
     return out
 

@@ -194,6 +194,22 @@ def test_groupwise_row_bytes_ledger_and_validation():
 
 
 
+@pytest.mark.parametrize("bits,sizes,seed", [((4, 3), (64, 64), 5), ((4, 2), (32, 96), 6), ((3, 2), (16, 112), 7),
+                                             ((2, 4), (80, 48), 8)])
+def test_group_rotation_equals_oracle(bits, sizes, seed):
+    """The library's R_h (built from its permutation, signs and Hadamard blocks) against the oracle's."""
+    H = 3
+    hc = _high(H, sizes[0], seed)
+    got = tq.group_rotation(D, H, bits, sizes, hc, seed)
+    f = O.Format(D, H, bits, sizes, hc, seed, groupwise=True)
+    for h in range(H):
+        ref = O.group_rotation(f, h)
+        assert np.array_equal(got[h], ref.astype(np.float32))
+        assert np.allclose(got[h].astype(np.float64) @ got[h].T.astype(np.float64), np.eye(D), atol=1e-6)
+    with pytest.raises(ValueError):
+        tq.group_rotation(D, H, (4, 3), (64, 64), None, seed)
+
+
 def test_recipe_slicing_by_tensor_parallel_partition(tmp_path):
     hc = _high(8, 32, 12)
     p = tmp_path / "recipe.json"
