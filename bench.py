@@ -440,6 +440,15 @@ def max_over_ranks(x, dist_ctx):
     return float(t.item())
 
 
+def guarded(sample):
+    """Run an oracle timing leg; a failure is reported in the line instead of ending the benchmark."""
+    try:
+        gbs, tps, desc, threads = sample()
+        return {"GB/s": gbs, "token_heads_per_s": tps, "cores": threads, "kind": "oracle", "sample": desc}
+    except Exception as e:  # noqa: BLE001 - a secondary, reported leg
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+
 def rank_workload(w: WL.Workload, rank: int) -> WL.Workload:
     """Rank r's replica of a workload: the same shapes, its own seeded data (weak scaling)."""
     return WL.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
@@ -533,6 +542,36 @@ def oracle_decode_sample(w, kspec, vspec, lay, unit_source, budget_s: float, row
     desc = (f"oracle decode of sequence {b} (L={L}, the median length), {units} of {w.num_kv_heads} KV heads, "
             f"all {G} query heads of each")
     return done_bytes / elapsed / 1e9, done_tok / elapsed, desc, threads
+
+
+def oracle_pack_sample(w, kspec, vspec, budget_s: float, chunk: int = 512):
+    """Time the oracle's pack (quantize, encode, page write) on 512-token chunks of sequence 0 until
+    ~budget_s of CPU work. Rows go to a pool of the chunk's own size: the per-row work is the same.
+
+    Returns (GB/s of algorithmic bytes, token-heads/s, description, threads).
+    """
+    from oracle import tq_oracle as O
+
+    H, bs = w.num_kv_heads, w.block_size
+    kf, vf = (O.Format(D, H, s.group_bits, s.group_size, s.high_coords, s.seed, qjl=s.qjl, groupwise=s.groupwise)
+              for s in (kspec, vspec))
+    per_token = H * D * 2 * 2 + H * (O.row_bytes(kf) + O.row_bytes(vf)) + 8
+    L = int(WL.seq_lens(w)[0])
+    done = 0
+    elapsed = 0.0
+    for t0 in range(0, L, chunk):
+        t1 = min(L, t0 + chunk)
+        k, v = WL.sequence_kv(w, 0, t0, t1, device="cpu")
+        k, v = k.float().numpy(), v.float().numpy()
+        slots = np.arange(t1 - t0, dtype=np.int64)
+        t_start = time.perf_counter()
+        O.pack_kv(k, v, slots, kf, vf, -(-(t1 - t0) // bs), bs)
+        elapsed += time.perf_counter() - t_start
+        done += t1 - t0
+        if elapsed >= budget_s:
+            break
+    desc = f"oracle pack of the first {done} tokens of sequence 0, all {H} KV heads, K and V"
+    return done * per_token / elapsed / 1e9, done * H / elapsed, desc, len(os.sched_getaffinity(0))
 
 
 def oracle_decode_sample_one_thread(w, kspec, vspec, lay, unit_source, budget_s: float, row_bytes):
@@ -702,6 +741,10 @@ def run_ours(args):
                                "decode_partials_GB/s": sb / (p[1] * 1e-3) / 1e9,
                                "decode_partials_frac": sb / (p[1] * 1e-3) / 1e9 / peak,
                                "traffic": stored_traffic(name, "tq_decode_mma.cu")}
+                if not args.no_cpu_baseline:
+                    extra[name]["cpu_oracle"] = guarded(lambda: oracle_decode_sample(
+                        ew, setup.kspec, setup.vspec, setup.layout, lambda b, h: gpu_pages_unit(setup, b, h),
+                        args.cpu_budget / 4, setup.kc.row_bytes + setup.vc.row_bytes))
             else:
                 del setup
                 torch.cuda.empty_cache()
@@ -710,6 +753,9 @@ def run_ours(args):
                 gbs = setup.bytes() / (ms * 1e-3) / 1e9
                 extra[name] = {"GB/s": gbs, "tokens_per_s": setup.k.shape[0] / (ms * 1e-3), "ms_per_step": ms,
                                "frac": gbs / peak, "traffic": stored_traffic(name, "tq_pack_mma.cu")}
+                if not args.no_cpu_baseline:
+                    ks, vs = WL.codec_specs(ew)
+                    extra[name]["cpu_oracle"] = guarded(lambda: oracle_pack_sample(ew, ks, vs, args.cpu_budget / 4))
                 line["gpu_launches"] += max(5, args.steps // 2)
         # the small parity case: a latency, hot and with L2 flushed before each call
         del setup

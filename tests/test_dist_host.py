@@ -111,3 +111,15 @@ def test_oracle_baseline_sample_with_one_thread():
     src = lambda b, h: bench.oracle_pages_unit(w, kspec, vspec, lay, b, h)  # noqa: E731
     gbs, tps, desc, threads = bench.oracle_decode_sample_one_thread(w, kspec, vspec, lay, src, 0.0, rb)
     assert threads == 1 and gbs > 0 and tps > 0 and "sequence 0" in desc
+
+
+def test_oracle_pack_sample_and_guard():
+    """The pack workload's CPU-oracle timing leg, and the guard that reports a failing leg in the line."""
+    w = WL.WORKLOADS["pack_llama8b_4bit"]
+    ks, vs = WL.codec_specs(w)
+    gbs, tps, desc, threads = bench.oracle_pack_sample(w, ks, vs, 0.0, chunk=64)
+    assert gbs > 0 and tps > 0 and "first 64 tokens" in desc and threads >= 1
+    ok = bench.guarded(lambda: (1.0, 2.0, "d", 3))
+    assert ok == {"GB/s": 1.0, "token_heads_per_s": 2.0, "cores": 3, "kind": "oracle", "sample": "d"}
+    bad = bench.guarded(lambda: 1 / 0)
+    assert bad["error"].startswith("ZeroDivisionError")
