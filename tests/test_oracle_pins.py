@@ -780,3 +780,45 @@ def test_groupwise_row_layout_and_reconstruction():
     # and close to x: each group within its codebook's error
     rel = np.linalg.norm(xr - x, axis=1) / np.linalg.norm(x, axis=1)
     assert np.all(rel < 0.5)
+
+
+def test_qjl_oracle_key_is_unbiased_over_codec_seeds():
+    """The oracle's own QJL key (quantize_qjl, then dequantize_rows) estimates q . x without bias.
+
+    One fixed x and q; the codec seed runs over 2000 values, so S comes from
+    the oracle's qjl_matrix (and the sign vector changes with it). Given the
+    rotation, the QJL identity E_S[sqrt(pi/2)/d S^T sign(S r)] = r / |r| makes
+    the key's expectation n R^T (c + r) = x, and its variance is bounded by
+    pi/(2d) |q|^2 |r|^2 n^2 (Zandieh et al., QJL). The fp16 norm and residual
+    norm add a bias of at most about 2^-11 |q . x|. The two mistakes that
+    leave a single-S check near zero are shown to fail the same mean test: the
+    constant sqrt(2/pi)/d in place of sqrt(pi/2)/d, and z = 1 - 2 bits.
+    """
+    d, n_seeds = 128, 2000
+    rng = np.random.default_rng(31)
+    x = O.bf16_round(rng.standard_normal(d) * 2.0)[None, :]
+    # q along x plus noise: the residual is correlated with the rotated vector
+    # (a Lloyd-Max error is orthogonal to the centroid, not to the input), so
+    # a wrong QJL scale or sign shifts q . key by a multiple of the distortion
+    q = x[0] / np.linalg.norm(x[0]) * 8.0 + rng.standard_normal(d)
+    exact = float(x[0] @ q)
+    est, mse_part, bound = np.empty(n_seeds), np.empty(n_seeds), np.empty(n_seeds)
+    for i in range(n_seeds):
+        f = O.Format(d, 1, (3,), (d,), None, 1000 + i, qjl=True)
+        idx, n16, u, signs, g16 = O.quantize_qjl(x, f, 0)
+        est[i] = float(O.dequantize_rows(idx, n16, f, 0, signs, g16)[0] @ q)
+        mse_part[i] = float(O.dequantize_rows(idx, n16, f, 0, signs, np.zeros_like(g16))[0] @ q)
+        bound[i] = math.pi / (2 * d) * float(q @ q) * float(g16[0]) ** 2 * float(n16[0]) ** 2
+    qjl_part = est - mse_part
+    sem = est.std(ddof=1) / math.sqrt(n_seeds)
+    fp16_bias = 2.0 ** -10 * abs(exact)
+    assert abs(est.mean() - exact) < 4 * sem + fp16_bias
+    # second moment of the error within the QJL variance bound (averaged over the draws)
+    assert np.mean((est - exact) ** 2) <= 1.1 * bound.mean()
+    # the QJL term carries signal: dropping it leaves the MSE part's shrinkage bias
+    assert abs(mse_part.mean() - exact) > 8 * sem + fp16_bias
+    wrong_const = mse_part + (2.0 / math.pi) * qjl_part  # sqrt(2/pi)/d instead of sqrt(pi/2)/d
+    wrong_sign = mse_part - qjl_part                       # z = 1 - 2 bits
+    for alt in (wrong_const, wrong_sign):
+        alt_sem = alt.std(ddof=1) / math.sqrt(n_seeds)
+        assert abs(alt.mean() - exact) > 8 * max(sem, alt_sem) + fp16_bias
