@@ -307,14 +307,22 @@ tq_status tq_decode_combine(const tq_codec* vc, const int32_t* seq_lens, int32_t
  *
  * Arguments mean what they mean for tq_decode_paged. The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current) and caches it, so make that first call before any
- * stream capture. A call whose tq_decode_workspace_bytes(...) exceeds
+ * that device current) and caches it. Under CUDA's lazy module loading (the
+ * default) that lookup is also what loads the library's device code on the
+ * device and so creates the array there: the first call reserves the
+ * 32 MiB and may synchronize. Make it at start-up, before the host runtime
+ * reserves the rest of device memory and before any stream capture; if the
+ * array cannot be created the call returns TQ_ERR_CUDA with "static
+ * workspace could not be loaded". A call whose tq_decode_workspace_bytes(...) exceeds
  * TQ_STATIC_WORKSPACE_BYTES returns TQ_ERR_VALUE before launching anything.
  * All calls share the array and it keeps the last call's contents (nothing
  * in it needs to start at zero); calls whose kernels overlap on the GPU, on
  * different streams or from different threads, race on it.
  */
 #define TQ_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+/* The size of the array this build of the library holds (its
+ * TQ_STATIC_WORKSPACE_BYTES), for bindings that do not read this header. */
+size_t tq_static_workspace_bytes(void);
 tq_status tq_decode_paged_static(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
                                  const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
                                  const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t max_seq_len,

@@ -47,8 +47,8 @@ tq_status static_workspace(void** out) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_workspace);
         if (e != cudaSuccess || !p)
-            return tq::fail(TQ_ERR_CUDA, std::string("cudaGetSymbolAddress of the static workspace: ") +
-                                             cudaGetErrorString(e));
+            return tq::fail(TQ_ERR_CUDA, std::string("static workspace could not be loaded on device ") +
+                                             std::to_string(dev) + " (" + cudaGetErrorString(e) + ")");
         g_device_addr[dev] = p;
     }
     *out = g_device_addr[dev];
@@ -56,6 +56,8 @@ tq_status static_workspace(void** out) {
 }
 
 }  // namespace
+
+extern "C" size_t tq_static_workspace_bytes(void) { return kStaticBytes; }
 
 extern "C" tq_status tq_decode_paged_static(const tq_codec* kc, const tq_codec* vc, const void* q,
                                             const void* k_pages, const void* v_pages, const int32_t* block_tables,

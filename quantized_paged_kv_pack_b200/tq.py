@@ -81,6 +81,8 @@ def lib():
         L.tq_decode_partials.argtypes = dec + [_VP, _SZ, _VP, _VP]
         L.tq_decode_combine.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _SZ, _VP]
         L.tq_decode_paged_static.argtypes = dec + [_VP, _VP, _VP]
+        L.tq_static_workspace_bytes.argtypes = []
+        L.tq_static_workspace_bytes.restype = _SZ
         L.tq_window_append.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP, _I64,
                                        _I32, _I32, _VP, _VP]
         L.tq_byte_ledger.argtypes = [P(_FormatDesc), P(_FormatDesc), _I32, _VP, _I32, _I32, _I32, _I64, _I32,
@@ -396,7 +398,9 @@ def decode_paged(kc: Codec, vc: Codec, q: torch.Tensor, k_pages: torch.Tensor, v
     return out
 
 
-STATIC_WORKSPACE_BYTES = 32 << 20
+def static_workspace_bytes() -> int:
+    """Size of the fixed scratch array behind decode_paged_static, as built into libtq.so."""
+    return int(lib().tq_static_workspace_bytes())
 
 
 def decode_paged_static(kc: Codec, vc: Codec, q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
@@ -408,8 +412,10 @@ def decode_paged_static(kc: Codec, vc: Codec, q: torch.Tensor, k_pages: torch.Te
 
     For callers that cannot call cudaMalloc (another runtime owns the device
     memory, or the path may not take cudaMalloc's implicit synchronization):
-    the split-K scratch is a fixed array of STATIC_WORKSPACE_BYTES inside the
-    library, shared by every call, so calls that overlap on the GPU race.
+    the split-K scratch is a fixed array of static_workspace_bytes() inside the
+    library, shared by every call, so calls that overlap on the GPU race. The
+    first call on a device loads that array there (it reserves the memory), so
+    make it at start-up, before another runtime takes the rest of the device.
     ``out`` should be preallocated by such callers; if it is None this
     wrapper creates it with torch for convenience.
     """

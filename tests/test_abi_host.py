@@ -228,3 +228,11 @@ def test_recipe_slicing_by_tensor_parallel_partition(tmp_path):
         tq.slice_recipe(spec, 0, 3)
     with pytest.raises(ValueError):
         tq.slice_recipe(spec, 4, 4)
+
+
+def test_static_workspace_size_matches_header():
+    """The binding reads the static array's size from the library; it must be the header's value."""
+    text = open(os.path.join(ROOT, "include", "tq.h")).read()
+    m = re.search(r"#define\s+TQ_STATIC_WORKSPACE_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", text)
+    assert m, "TQ_STATIC_WORKSPACE_BYTES not found in tq.h"
+    assert tq.static_workspace_bytes() == int(m.group(1)) << int(m.group(2))
