@@ -789,8 +789,10 @@ def byte_ledger(kfmt: Format, vfmt: Format, seq_lens: Sequence[int], window: int
     (4 with QJL: the residual norm too), K and V. codebooks: fp16 centroids
     and fp32 boundaries of every group of both codecs. transforms: d int8 signs
     and H_kv*d int16 permutation entries per codec, plus the fp32 d x d QJL
-    matrix of a QJL codec. window: the allocated bf16 window, K and V. block
-    tables: one int32 per used block.
+    matrix of a QJL codec, plus for a group-wise codec (R17) its per-head
+    rotation held as a dense fp32 d x d matrix R_h per KV head ("System
+    Invariants": the all-in ratio counts transforms). window: the allocated
+    bf16 window, K and V. block tables: one int32 per used block.
     """
     H, d = kfmt.num_kv_heads, kfmt.head_dim
     lens = [int(x) for x in seq_lens]
@@ -803,7 +805,8 @@ def byte_ledger(kfmt: Format, vfmt: Format, seq_lens: Sequence[int], window: int
     for fmt in (kfmt, vfmt):
         for b in fmt.group_bits:
             cb += (1 << b) * 2 + ((1 << b) - 1) * 4
-    transforms = 2 * (d + H * d * 2) + sum(4 * d * d for fmt in (kfmt, vfmt) if fmt.qjl)
+    transforms = (2 * (d + H * d * 2) + sum(4 * d * d for fmt in (kfmt, vfmt) if fmt.qjl)
+                  + sum(4 * H * d * d for fmt in (kfmt, vfmt) if fmt.groupwise))
     win = 2 * 2 * len(lens) * H * window * d
     bt = 4 * sum(-(-p // block_size) for p in packed)
     pool = num_blocks * H * block_size * (row_bytes(kfmt) + row_bytes(vfmt))

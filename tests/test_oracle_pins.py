@@ -822,3 +822,29 @@ def test_qjl_oracle_key_is_unbiased_over_codec_seeds():
     for alt in (wrong_const, wrong_sign):
         alt_sem = alt.std(ddof=1) / math.sqrt(n_seeds)
         assert abs(alt.mean() - exact) > 8 * max(sem, alt_sem) + fp16_bias
+
+
+def test_ledger_transform_bytes_are_the_transforms_a_decode_holds():
+    """transform_bytes = the nbytes of what the oracle builds for each codec: int8 signs, the int16
+    permutation of every head, the fp32 QJL matrix S of a QJL codec, and the dense fp32 rotation
+    R_h of every head of a group-wise codec ("System Invariants": the ratio counts transforms)."""
+    H = 3
+    rng = np.random.default_rng(4)
+    high = np.stack([np.sort(rng.choice(D, 64, replace=False)) for _ in range(H)])
+    cases = [O.Format(D, H, (4, 3), (64, 64), high, 5, groupwise=True),
+             O.Format(D, H, (3, 2), (64, 64), high, 6, qjl=True),
+             O.Format(D, H, (4,), (128,), None, 7)]
+    for kf in cases:
+        for vf in cases:
+            if vf.qjl:
+                continue
+            led = O.byte_ledger(kf, vf, [40, 7], 4, 16, 5)
+            expect = 0
+            for f in (kf, vf):
+                expect += O.hadamard_signs(f.seed, D).astype(np.int8).nbytes
+                expect += sum(O.permutation(f, h).astype(np.int16).nbytes for h in range(H))
+                if f.qjl:
+                    expect += O.qjl_matrix(f).astype(np.float32).nbytes
+                if f.groupwise:
+                    expect += sum(O.group_rotation(f, h).astype(np.float32).nbytes for h in range(H))
+            assert led.transform_bytes == expect, (kf, vf)
