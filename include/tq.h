@@ -121,7 +121,10 @@ typedef struct tq_codec tq_codec; /* opaque, immutable after tq_make_codec */
  * signs          out, int8   [head_dim], +1 or -1
  * perm           out, int16  [num_kv_heads][head_dim]: packed position ->
  *                rotated coordinate (group 0 coordinates ascending, then the rest)
- * row_bytes      out: index bytes of all groups + 2 (fp16 norm)
+ * row_bytes      out: index bytes of all groups, plus the QJL sign bytes
+ *                (head_dim / 8) of a QJL codec, plus the norm bytes: 2 (fp16
+ *                norm), or 4 for a QJL codec (norm, residual norm) and for a
+ *                group-wise codec (one norm per group)
  * Any output pointer may be NULL. Returns TQ_ERR_VALUE / TQ_ERR_UNSUPPORTED
  * for an invalid descriptor (the GPU format limits apply here too).
  */
@@ -160,7 +163,8 @@ tq_status tq_codec_group_rotation(const tq_format_desc* desc, float* out);
 tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out);
 void tq_free_codec(tq_codec* codec);
 
-/* Bytes of one packed row of this codec (index bytes of every group + 2). */
+/* Bytes of one packed row of this codec: index bytes of every group, the QJL
+ * sign bytes of a QJL codec, and 2 norm bytes (4 for QJL and group-wise). */
 int32_t tq_codec_row_bytes(const tq_codec* codec);
 
 /*
@@ -336,9 +340,12 @@ tq_status tq_decode_paged_static(const tq_codec* kc, const tq_codec* vc, const v
  *
  * dense_bytes        bf16 K and V of every token: 4 * num_kv_heads * head_dim * sum L_b
  * index_bytes        packed index bytes of the P_b packed tokens, K and V (storage)
- * norm_bytes         2 bytes per packed row, K and V
+ * norm_bytes         the norm bytes of every packed row, K and V: 2 per row, 4 for a
+ *                    QJL codec (norm, residual norm) or a group-wise codec (a norm per group)
  * codebook_bytes     fp16 centroids + fp32 boundaries of every group of both codecs
- * transform_bytes    per codec: head_dim int8 signs + num_kv_heads*head_dim int16 permutation
+ * transform_bytes    per codec: head_dim int8 signs + num_kv_heads*head_dim int16 permutation,
+ *                    + the fp32 head_dim^2 QJL matrix S of a QJL codec, + the dense fp32
+ *                    head_dim^2 rotation R_h per KV head that a group-wise codec keeps
  * window_bytes       the allocated bf16 windows, K and V
  * block_table_bytes  one int32 per used block
  * workspace_bytes    tq_decode_workspace_bytes for these sizes

@@ -392,6 +392,22 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
 
 using namespace tq;
 
+namespace tq {
+void build_pack_cells(const float* boundaries, int levels, PackCell* out) {
+    for (int e = 0; e < kPackCells; ++e) {
+        const double lo = e - 64 - 0.5, hi = e - 64 + 0.5;
+        int below = 0;
+        float thr = INFINITY;
+        for (int i = 0; i + 1 < levels; ++i) {
+            const double bv = static_cast<double>(boundaries[i]) * kPackCellScale;
+            if (bv < lo) ++below;
+            else if (bv <= hi) thr = static_cast<float>(bv);
+        }
+        out[e] = PackCell{thr, below};
+    }
+}
+}  // namespace tq
+
 extern "C" {
 
 const char* tq_last_error(void) { return g_last_error.c_str(); }
@@ -460,7 +476,10 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     const size_t off_s = (n_sign + 2 * n_cent + 2 * n_perm + 15) / 16 * 16;
     const size_t n_s = c->qjl_s.size() * sizeof(float);
     const size_t off_r = (off_s + n_s + 15) / 16 * 16, n_r = c->rot_t.size() * sizeof(float);
-    const size_t total = off_r + n_r;
+    // uniform 4-bit codecs also carry the tensor-core pack's quantizer cell table
+    const bool u4 = desc->n_groups == 1 && desc->group_bits[0] == 4 && !desc->qjl && !desc->groupwise;
+    const size_t off_c = (off_r + n_r + 15) / 16 * 16, n_c = u4 ? kPackCells * sizeof(PackCell) : 0;
+    const size_t total = off_c + n_c;
     std::vector<char> host(total);
     char* p = host.data();
     std::memcpy(p, c->sign, n_sign);
@@ -474,6 +493,7 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
             for (int j = 0; j < d; ++j) st[static_cast<size_t>(j) * d + i] = c->qjl_s[static_cast<size_t>(i) * d + j];
     }
     if (n_r) std::memcpy(p + off_r, c->rot_t.data(), n_r);
+    if (n_c) build_pack_cells(c->bound[0], 16, reinterpret_cast<PackCell*>(p + off_c));
     if (cudaGetDevice(&c->device) != cudaSuccess || cudaMalloc(&c->d_tables, total) != cudaSuccess) {
         cudaGetLastError();
         delete c;
@@ -493,6 +513,7 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     c->dev.pos = reinterpret_cast<const int16_t*>(base + n_sign + 2 * n_cent + n_perm);
     c->dev.qjl_st = n_s ? reinterpret_cast<const float*>(base + off_s) : nullptr;
     c->dev.rot_t = n_r ? reinterpret_cast<const float*>(base + off_r) : nullptr;
+    c->dev.cells = n_c ? reinterpret_cast<const PackCell*>(base + off_c) : nullptr;
     *out = c;
     return TQ_OK;
 }
@@ -545,7 +566,9 @@ tq_status tq_byte_ledger(const tq_format_desc* kdesc, const tq_format_desc* vdes
             int64_t L = int64_t(1) << desc->group_bits[g];
             r.codebook_bytes += L * 2 + (L - 1) * 4;
         }
-    r.transform_bytes = 2 * (d + H * d * 2) + 4 * d * d * ((kdesc->qjl ? 1 : 0) + (vdesc->qjl ? 1 : 0));
+    // signs and permutations of both codecs, S of a QJL codec, the per-head R_h of a group-wise codec
+    r.transform_bytes = 2 * (d + H * d * 2) + 4 * d * d * ((kdesc->qjl ? 1 : 0) + (vdesc->qjl ? 1 : 0)) +
+                        4 * H * d * d * ((kdesc->groupwise ? 1 : 0) + (vdesc->groupwise ? 1 : 0));
     r.window_bytes = 2 * 2 * static_cast<int64_t>(batch) * H * window * d;
     r.block_table_bytes = 4 * blocks;
     r.workspace_bytes = static_cast<int64_t>(

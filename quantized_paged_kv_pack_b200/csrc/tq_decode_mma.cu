@@ -47,6 +47,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 #include <type_traits>
 
@@ -326,6 +327,86 @@ __device__ __forceinline__ uint32_t lut_base(uint32_t lane_base) {
     return B == 4 ? lane_base : (B == 3 ? (lane_base | 128u) : (lane_base | 0x4080u));
 }
 
+// ---- tensor memory (TMEM) as per-warp storage -------------------------------------
+//
+// The block kernel keeps each warp's query fragments and value accumulators
+// in tensor memory between uses instead of in registers: a warp reaches only
+// its lane quarter (lanes 32 (warp % 4) .. + 31), thread i lane 32 (warp % 4)
+// + i, and the 32x32b shape moves one 32-bit column per register. Loads are
+// asynchronous: tm_wait_ld() waits for them, and tm_dep() then ties the
+// registers to that wait so that no use is scheduled before it.
+
+__device__ __forceinline__ void tm_ld4(uint32_t taddr, uint32_t* v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tm_st4(uint32_t taddr, const uint32_t* v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+                 :
+                 : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+                 : "memory");
+}
+__device__ __forceinline__ void tm_dep4(uint32_t* v) {
+    asm volatile("" : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]));
+}
+__device__ __forceinline__ void tm_ld16(uint32_t taddr, uint32_t* v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tm_st16(uint32_t taddr, const uint32_t* v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+                 :
+                 : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+                 : "memory");
+}
+__device__ __forceinline__ void tm_dep16(uint32_t* v) {
+    asm volatile("" : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]));
+}
+__device__ __forceinline__ void tm_ld32(uint32_t taddr, uint32_t* v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tm_st32(uint32_t taddr, const uint32_t* v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+                 :
+                 : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+                 : "memory");
+}
+__device__ __forceinline__ void tm_dep32(uint32_t* v) {
+    asm volatile("" : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31]));
+}
+__device__ __forceinline__ void tm_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tm_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tm_fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tm_fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void tm_ld(uint32_t taddr, uint32_t* v) {
+    static_assert(N == 4 || N == 16 || N == 32, "tm_ld width");
+    if constexpr (N == 4) tm_ld4(taddr, v);
+    else if constexpr (N == 16) tm_ld16(taddr, v);
+    else tm_ld32(taddr, v);
+}
+template <int N>
+__device__ __forceinline__ void tm_st(uint32_t taddr, const uint32_t* v) {
+    static_assert(N == 4 || N == 16 || N == 32, "tm_st width");
+    if constexpr (N == 4) tm_st4(taddr, v);
+    else if constexpr (N == 16) tm_st16(taddr, v);
+    else tm_st32(taddr, v);
+}
+template <int N>
+__device__ __forceinline__ void tm_dep(uint32_t* v) {
+    if constexpr (N == 4) tm_dep4(v);
+    else if constexpr (N == 16) tm_dep16(v);
+    else tm_dep32(v);
+}
+
 // ---- work items -----------------------------------------------------------------
 
 struct Item {
@@ -473,22 +554,74 @@ __device__ __forceinline__ void fill_table(uint32_t* table, const LutValues& tv,
 // against the projected query (the A operand is +-|r| per token, exact in
 // fp16); they land in the same accumulators as the index groups, so the
 // token's score is n (q'.c + sqrt(pi/2)/128 |r| (S q').z) before the norm.
-template <class KF, class VF, int NH>
+//
+// TM: the query fragments and the value accumulators live in this warp's
+// tensor-memory columns between uses (query fragments at kTmQ, QJL fragments
+// at kTmZ, accumulators at kTmO, the merge state at kTmS) and in registers
+// only inside scores() and values(), so the two sets are never live at once.
+template <class KF, class VF, int NH, bool TM = false>
 struct WarpTiles {
     static constexpr int HL = NH / 4;  // heads per lane
     static constexpr bool KQ = KF::MODE == kQjl, KG = KF::MODE == kGroupwise, VG = VF::MODE == kGroupwise;
-    uint32_t bq[8][2 * HL];            // query B fragments per k-step
-    uint32_t bz[KQ ? 8 : 1][2 * HL];   // QJL: projected-query B fragments per sign k-step
+    static constexpr int NQW = 16 * HL;  // words of the query fragments of one k-step set
+    static constexpr uint32_t kTmQ = 0, kTmZ = 32, kTmO = 64, kTmS = 96, kTmCols = 128;
+    uint32_t bq[TM ? 1 : 8][2 * HL];             // query B fragments per k-step (registers when !TM)
+    uint32_t bz[(KQ && !TM) ? 8 : 1][2 * HL];    // QJL: projected-query B fragments per sign k-step
     uint32_t bp[2 * HL];               // P' B fragments of the last scored tile (group 0 norms when VG)
     uint32_t bp1[VG ? 2 * HL : 1];     // VG: P' B fragments with the group-1 norms
-    float o[8][4];                     // value accumulators: row tile q, rows r / r + 8, columns 2c / 2c + 1
+    float o_[TM ? 1 : 8][4];           // value accumulators: row tile q, rows r / r + 8, columns 2c / 2c + 1
     float m_ref[HL], l_run[HL];
+    uint32_t tm = 0;                   // TM: this warp's tensor-memory address (lane quarter, first column)
+
+    __device__ __forceinline__ void load_query(uint32_t (&qf)[8][2 * HL], uint32_t (&zf)[KQ ? 8 : 1][2 * HL]) const {
+        if constexpr (TM) {
+            tm_ld<NQW>(tm + kTmQ, &qf[0][0]);
+            if constexpr (KQ) tm_ld<NQW>(tm + kTmZ, &zf[0][0]);
+            tm_wait_ld();
+            tm_dep<NQW>(&qf[0][0]);
+            if constexpr (KQ) tm_dep<NQW>(&zf[0][0]);
+        } else {
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+#pragma unroll
+                for (int i = 0; i < 2 * HL; ++i) {
+                    qf[s][i] = bq[s][i];
+                    if constexpr (KQ) zf[s][i] = bz[s][i];
+                }
+        }
+    }
+    __device__ __forceinline__ void load_acc(float (&o)[8][4]) const {
+        if constexpr (TM) {
+            uint32_t* w = reinterpret_cast<uint32_t*>(&o[0][0]);
+            tm_wait_st();  // the previous store of the accumulators has landed
+            tm_ld<32>(tm + kTmO, w);
+            tm_wait_ld();
+            tm_dep<32>(w);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[q][i] = o_[q][i];
+        }
+    }
+    __device__ __forceinline__ void store_acc(const float (&o)[8][4]) {
+        if constexpr (TM) {
+            tm_st<32>(tm + kTmO, reinterpret_cast<const uint32_t*>(&o[0][0]));
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o_[q][i] = o[q][i];
+        }
+    }
 
     // Rotated, scaled queries of the item's query heads (rows of them), fp32
     // [head][128] in the packed coordinate order; for QJL keys also their
     // projections qz, [head][128] in projection order.
     __device__ __forceinline__ void begin(const float* qr, const float* qz, int rows, int r, int c) {
         const int head = NH == 8 ? r : (r >> 1);
+        uint32_t qf[8][2 * HL];
+        uint32_t zf[KQ ? 8 : 1][2 * HL];
         if constexpr (KQ) {
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
@@ -506,13 +639,13 @@ struct WarpTiles {
                 split2(x0, x1, h01, l01);
                 split2(x2, x3, h23, l23);
                 if constexpr (NH == 8) {
-                    bz[s][0] = h01;
-                    bz[s][1] = h23;
-                    bz[s][2] = l01;
-                    bz[s][3] = l23;
+                    zf[s][0] = h01;
+                    zf[s][1] = h23;
+                    zf[s][2] = l01;
+                    zf[s][3] = l23;
                 } else {
-                    bz[s][0] = (r & 1) ? l01 : h01;
-                    bz[s][1] = (r & 1) ? l23 : h23;
+                    zf[s][0] = (r & 1) ? l01 : h01;
+                    zf[s][1] = (r & 1) ? l23 : h23;
                 }
             }
         }
@@ -526,17 +659,34 @@ struct WarpTiles {
             split2(x.x, x.y, h01, l01);
             split2(x.z, x.w, h23, l23);
             if constexpr (NH == 8) {
-                bq[s][0] = h01;
-                bq[s][1] = h23;
-                bq[s][2] = l01;
-                bq[s][3] = l23;
+                qf[s][0] = h01;
+                qf[s][1] = h23;
+                qf[s][2] = l01;
+                qf[s][3] = l23;
             } else {
-                bq[s][0] = (r & 1) ? l01 : h01;
-                bq[s][1] = (r & 1) ? l23 : h23;
+                qf[s][0] = (r & 1) ? l01 : h01;
+                qf[s][1] = (r & 1) ? l23 : h23;
             }
         }
+        float o[8][4];
 #pragma unroll
         for (int q = 0; q < 8; ++q) o[q][0] = o[q][1] = o[q][2] = o[q][3] = 0.0f;
+        if constexpr (TM) {
+            tm_wait_st();  // the last item's accumulators have landed before they are overwritten
+            tm_st<NQW>(tm + kTmQ, &qf[0][0]);
+            if constexpr (KQ) tm_st<NQW>(tm + kTmZ, &zf[0][0]);
+            tm_st<32>(tm + kTmO, reinterpret_cast<const uint32_t*>(&o[0][0]));
+            tm_wait_st();
+        } else {
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+#pragma unroll
+                for (int i = 0; i < 2 * HL; ++i) {
+                    bq[s][i] = qf[s][i];
+                    if constexpr (KQ) bz[s][i] = zf[s][i];
+                }
+            store_acc(o);
+        }
 #pragma unroll
         for (int e = 0; e < HL; ++e) {
             m_ref[e] = -INFINITY;
@@ -553,6 +703,9 @@ struct WarpTiles {
         // Independent accumulator chains (k-step parity, or the group when K is
         // group-wise; hi / lo for NH = 8) keep the MMA dependency depth at 4.
         constexpr int NC = NH == 8 ? 4 : 2;
+        uint32_t qf[8][2 * HL];
+        uint32_t zf[KQ ? 8 : 1][2 * HL];
+        load_query(qf, zf);
         float sacc[NC][4];
 #pragma unroll
         for (int u = 0; u < NC; ++u) sacc[u][0] = sacc[u][1] = sacc[u][2] = sacc[u][3] = 0.0f;
@@ -560,10 +713,10 @@ struct WarpTiles {
             constexpr int s_ = decltype(si)::value;
             constexpr int u = KG ? (s_ < KF::KS0 ? 0 : 1) : (s_ & 1);
             if constexpr (NH == 8) {
-                mma16816(sacc[u], a0, a1, a2, a3, bq[s_][0], bq[s_][1]);
-                mma16816(sacc[2 + u], a0, a1, a2, a3, bq[s_][2], bq[s_][3]);
+                mma16816(sacc[u], a0, a1, a2, a3, qf[s_][0], qf[s_][1]);
+                mma16816(sacc[2 + u], a0, a1, a2, a3, qf[s_][2], qf[s_][3]);
             } else {
-                mma16816(sacc[u], a0, a1, a2, a3, bq[s_][0], bq[s_][1]);
+                mma16816(sacc[u], a0, a1, a2, a3, qf[s_][0], qf[s_][1]);
             }
         };
         if constexpr (KQ) {
@@ -583,10 +736,10 @@ struct WarpTiles {
                 const uint32_t a2 = rn_a | (~prmt(ya, 0u, 0xB4A4u) & 0x80008000u);
                 const uint32_t a3 = rn_b | (~prmt(yb, 0u, 0xB4A4u) & 0x80008000u);
                 if constexpr (NH == 8) {
-                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, bz[s_][0], bz[s_][1]);
-                    mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, bz[s_][2], bz[s_][3]);
+                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, zf[s_][0], zf[s_][1]);
+                    mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, zf[s_][2], zf[s_][3]);
                 } else {
-                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, bz[s_][0], bz[s_][1]);
+                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, zf[s_][0], zf[s_][1]);
                 }
             });
         }
@@ -690,6 +843,8 @@ struct WarpTiles {
                 l_run[e] *= alpha[e];
                 if (grow) m_ref[e] = mx;
             }
+            float o[8][4];
+            load_acc(o);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 o[q][0] *= alpha[0];
@@ -697,6 +852,7 @@ struct WarpTiles {
                 o[q][2] *= alpha[0];
                 o[q][3] *= alpha[HL - 1];
             }
+            store_acc(o);
         }
         // P' = p 2^-kSlack n_V (weight x norm stays within fp16); the sums l_run
         // are kept in the same 2^-kSlack units. m_ref is finite here: the first
@@ -761,6 +917,8 @@ struct WarpTiles {
 
     // O^T += V^T P'^T for the tile last passed to scores(): V index rows at vbase.
     __device__ __forceinline__ void values(uint32_t vbase, uint32_t lane_base, int r, int c) {
+        float o[8][4];
+        load_acc(o);
         auto value_step = [&](auto qi, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
             constexpr int q = decltype(qi)::value;
             if constexpr (VG && q >= VF::MT0) {
@@ -816,6 +974,46 @@ struct WarpTiles {
                 value_step(std::integral_constant<int, VF::MT0 + q>{}, a0, a1, a2, a3);
             });
         }
+        store_acc(o);
+    }
+
+    // Pair merge (TM). The partner warp leaves its (max, sum) per head in its
+    // kTmS columns (its accumulators are already in its kTmO columns); the
+    // owner, in the same lane quarter, folds both into its own state.
+    __device__ __forceinline__ void export_state() {
+        const uint32_t v[4] = {__float_as_uint(m_ref[0]), __float_as_uint(m_ref[HL - 1]), __float_as_uint(l_run[0]),
+                               __float_as_uint(l_run[HL - 1])};
+        tm_st<4>(tm + kTmS, v);
+        tm_wait_st();  // this store and the accumulators' last one have landed
+    }
+    __device__ __forceinline__ void absorb(uint32_t partner) {
+        float o[8][4], po[8][4];
+        uint32_t ps[4];
+        load_acc(o);
+        uint32_t* pw = reinterpret_cast<uint32_t*>(&po[0][0]);
+        tm_ld<32>(partner + kTmO, pw);
+        tm_ld<4>(partner + kTmS, ps);
+        tm_wait_ld();
+        tm_dep<32>(pw);
+        tm_dep<4>(ps);
+        float f0[HL], f1[HL];
+#pragma unroll
+        for (int e = 0; e < HL; ++e) {
+            const float pm = __uint_as_float(ps[e]), pl = __uint_as_float(ps[2 + e]);
+            const float M = fmaxf(m_ref[e], pm);
+            f0[e] = m_ref[e] == -INFINITY ? 0.0f : ex2(m_ref[e] - M);
+            f1[e] = pm == -INFINITY ? 0.0f : ex2(pm - M);
+            l_run[e] = l_run[e] * f0[e] + pl * f1[e];
+            m_ref[e] = M;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            o[q][0] = o[q][0] * f0[0] + po[q][0] * f1[0];
+            o[q][1] = o[q][1] * f0[HL - 1] + po[q][1] * f1[HL - 1];
+            o[q][2] = o[q][2] * f0[0] + po[q][2] * f1[0];
+            o[q][3] = o[q][3] * f0[HL - 1] + po[q][3] * f1[HL - 1];
+        }
+        store_acc(o);
     }
 
     // Writes (max, sum, accumulator x 2^kSlack) of each of the lane's heads:
@@ -824,6 +1022,8 @@ struct WarpTiles {
     // r + 8 is p0 + 1.
     __device__ __forceinline__ void finish(float* m, float* l, float* acc, int ml_stride, int acc_stride, int rows,
                                            int r, int c) {
+        float o[8][4];
+        load_acc(o);
 #pragma unroll
         for (int e = 0; e < HL; ++e) {
             float lsum = l_run[e];
@@ -1198,6 +1398,178 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
             break;
         }
         wt.finish(rec, rec + 1, rec + 2, kHeadDim + 2, kHeadDim + 2, rows, r, c);
+    }
+}
+
+// ==== paired block kernel: two compute warps per KV head, state in tensor memory =========
+//
+// The same ring of 8-head page-block slots as the block kernel, read by 16
+// compute warps: warp w takes KV head w % 8 of the slots whose sequence number
+// has the parity w / 8 (the ring has an even number of slots, so each slot
+// serves one parity and its waits never skip a phase). Each warp keeps its
+// query fragments and value accumulators in its own tensor-memory columns
+// (WarpTiles<..., true>), which leaves room in the register file for twice the
+// warps. At the end of an item the odd warp of each head leaves its state in
+// tensor memory and the even warp, which reaches the same lane quarter, folds
+// it into its own and writes the record. An expired wait aborts the CTA: the
+// two warps of a head agree on it through a reduction barrier, so neither
+// waits for the other alone.
+
+constexpr int kPairWarps = 2 * kBlkWarps;  // compute warps
+constexpr uint32_t kTmemCols = 512;        // 4 warps per lane quarter x 128 columns
+
+struct PairSmem {
+    BlkSmem blk;    // ring barriers and the producer's block ids, as in the block kernel
+    uint32_t tmem;  // base address of the CTA's tensor memory
+    int abort;      // set when a compute warp's wait expired
+};
+
+// Barrier `id` over `count` threads that also returns whether any of them passed true.
+__device__ __forceinline__ bool bar_any(int id, int count, bool p) {
+    uint32_t res;
+    asm volatile(
+        "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.or.pred po, %2, %3, pi;\n selp.u32 %0, 1, 0, po;\n}"
+        : "=r"(res)
+        : "r"(static_cast<uint32_t>(p)), "r"(id), "r"(count)
+        : "memory");
+    return res != 0;
+}
+__device__ __forceinline__ void bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// The block kernel's producer, reused: its slot sequence does not depend on
+// which warps read a slot, only on the release count (8) of every slot.
+template <class KF, class VF, int NH, int TPB>
+__global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(DecodeArgs a, LutValues tv,
+                                                                               int group, int head_groups,
+                                                                               int64_t total_slots) {
+    static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
+    static_assert(TPB == 1 || TPB == 2, "16- or 32-token blocks");
+    extern __shared__ __align__(128) uint8_t dsm[];
+    PairSmem& sm = *reinterpret_cast<PairSmem*>(dsm);
+    total_slots = listed_slots<kBlkWarps>(a, head_groups, total_slots);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, c = lane & 3;
+    const int bs = a.block_size;
+
+    uint32_t dyn_bytes;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_bytes));
+    const uint32_t dsm_addr = smem_addr(dsm), dsm_end = dsm_addr + dyn_bytes;
+    BlkRing ring;
+    ring.stride = blk_slot_bytes<KF, VF>(bs);
+    ring.low = (dsm_addr + static_cast<uint32_t>(sizeof(PairSmem)) + 127) & ~127u;
+    const uint32_t lut_addr = (ring.low + (kLut - 1)) & ~uint32_t(kLut - 1);
+    ring.n_low = static_cast<int>((lut_addr - ring.low) / ring.stride);
+    ring.high = lut_addr + kLut;
+    const int n_high = ring.high < dsm_end ? static_cast<int>((dsm_end - ring.high) / ring.stride) : 0;
+    ring.n = min(ring.n_low + n_high, kBlkMaxSlots) & ~1;  // even
+    if (lut_addr + kLut > dsm_end || ring.n < 2) {
+        if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
+        return;
+    }
+    fill_table(reinterpret_cast<uint32_t*>(dsm + (lut_addr - dsm_addr)), tv, threadIdx.x, (kPairWarps + 1) * 32);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kBlkMaxSlots; ++s) {
+            mbar_init_count(smem_addr(&sm.blk.full[s]), 1);
+            mbar_init_count(smem_addr(&sm.blk.empty[s]), kBlkWarps);
+        }
+        sm.abort = 0;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sm.tmem)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tm_fence_before_sync();
+    __syncthreads();
+    tm_fence_after_sync();
+    if (warp == kPairWarps) {
+        produce_blk<KF, VF>(a, sm.blk, ring, head_groups, total_slots, lane);
+        return;
+    }
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&sm.tmem);
+    uint32_t lane_base;
+    asm volatile("or.b32 %0, %1, %2;" : "=r"(lane_base) : "r"(lut_addr), "r"(static_cast<uint32_t>(lane) << 2));
+    const uint32_t psel = (r & 1) ? 0x7632u : 0x5410u;
+    const int rows = group < NH ? group : NH;
+    const int hw = warp & (kBlkWarps - 1), par = warp / kBlkWarps;
+    const uint32_t k_sub = bs * (KF::RB + KF::NB), v_sub = bs * (VF::RB + VF::NB);
+    const uint32_t k_off = hw * k_sub, v_off = kBlkWarps * k_sub + hw * v_sub;
+    using Tiles = WarpTiles<KF, VF, NH, true>;
+    Tiles wt;
+    const uint32_t quarter = (32u * (warp & 3)) << 16;
+    wt.tm = tmem + quarter + Tiles::kTmCols * (warp >> 2);
+    const uint32_t partner_tm = tmem + quarter + Tiles::kTmCols * ((warp + kBlkWarps) >> 2);
+    constexpr int kBs = 16 * TPB;
+    uint32_t consumed = 0;
+    volatile int* abort_flag = &sm.abort;
+
+    for (int64_t slot = blockIdx.x; slot < total_slots; slot += gridDim.x) {
+        Item it;
+        if (!item_of<kBlkWarps>(a, slot, head_groups, total_slots, it)) continue;
+        if (it.win) continue;  // windows are not listed: window_kernel takes them
+        const int h = it.h + hw;                      // this warp's KV head
+        const int head0 = h * group + it.hg * 8;      // its first query head of the item
+        float* rec = record_of(a, it.b, h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
+        const int64_t q_off = (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim;
+        wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
+        const int ntiles = (it.t1 - it.t0 + 15) >> 4;
+        const int nslots = (ntiles + TPB - 1) / TPB;
+        bool bad = false;
+        for (int j = 0; j < nslots; ++j, ++consumed) {
+            if (static_cast<int>(consumed & 1u) != par) continue;
+            if (bad || *abort_flag) {
+                bad = true;
+                continue;
+            }
+            const int s = static_cast<int>(consumed % ring.n);
+            const bool ok = __all_sync(kFull, mbar_wait(smem_addr(&sm.blk.full[s]), (consumed / ring.n) & 1u));
+            if (!ok) {
+                bad = true;
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    if (a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
+                }
+                continue;
+            }
+            const uint32_t kb = ring.slot(s) + k_off, vb = ring.slot(s) + v_off;
+#pragma unroll
+            for (int t = 0; t < TPB; ++t) {
+                const int k = j * TPB + t;
+                if (TPB == 1 || k < ntiles)
+                    wt.step(kb + 16 * t * KF::RB, kb + kBs * KF::RB + 16 * KF::NB * t, vb + 16 * t * VF::RB,
+                            vb + kBs * VF::RB + 16 * VF::NB * t, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, psel,
+                            r, c);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&sm.blk.empty[s]));  // this warp is done with the slot
+        }
+        // Fold the odd warp's state into the even warp's; both agree on an abort.
+        if (par == 1) {
+            wt.export_state();
+            tm_fence_before_sync();
+        }
+        const bool abort = bar_any(1 + hw, 64, bad);
+        if (par == 0) {
+            tm_fence_after_sync();
+            if (!abort) wt.absorb(partner_tm);
+            tm_fence_before_sync();
+        }
+        bar_sync(1 + hw, 64);  // the odd warp's columns are free again
+        if (par == 1) tm_fence_after_sync();
+        if (abort) break;
+        if (par == 0) wt.finish(rec, rec + 1, rec + 2, kHeadDim + 2, kHeadDim + 2, rows, r, c);
+    }
+    // Every compute warp is done with tensor memory before warp 0 frees it.
+    tm_wait_st();
+    tm_fence_before_sync();
+    bar_sync(1 + kBlkWarps, kPairWarps * 32);
+    if (warp == 0) {
+        tm_fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
@@ -1672,9 +2044,10 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     const bool blk = a.kc.num_heads % kBlkWarps == 0 &&
                      static_cast<size_t>(blk_slot_bytes<KF, VF>(a.block_size)) * kBlkMinSlots <=
                          static_cast<size_t>(kMaxDynSmem) - kLut - 4096;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
+    const cudaError_t attr_err = once_per_device(dev, [] {
+        cudaError_t attr_err;
         attr_err = cudaFuncSetAttribute(decode_mma_kernel<KF, VF, NH, NW>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(head_bytes));
         if (attr_err == cudaSuccess)
@@ -1686,10 +2059,15 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
         if (attr_err == cudaSuccess)
             attr_err = cudaFuncSetAttribute(decode_blk_kernel<KF, VF, NH, 0>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(decode_pair_kernel<KF, VF, NH, 1>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(decode_pair_kernel<KF, VF, NH, 2>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+        return attr_err;
     });
     if (attr_err != cudaSuccess) return fail(TQ_ERR_CUDA, "cannot reserve shared memory for the decode kernel");
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int head_groups = group > 8 ? group / 8 : 1;
     const int64_t rows = static_cast<int64_t>(a.batch) * a.num_q_heads;
@@ -1709,8 +2087,16 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
                           (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);
     const int grid = static_cast<int>(units < sms ? units : sms);
     if (grid > 0) {
-        const dim3 threads((kBlkWarps + 1) * 32);
-        if (blk && a.block_size == 16)
+        const dim3 threads((kBlkWarps + 1) * 32), pair_threads((kPairWarps + 1) * 32);
+        static const bool pair = [] {
+            const char* e = std::getenv("TQ_DECODE_PAIR");
+            return !(e && e[0] == '0');
+        }();
+        if (blk && pair && a.block_size == 16)
+            decode_pair_kernel<KF, VF, NH, 1><<<grid, pair_threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
+        else if (blk && pair && a.block_size == 32)
+            decode_pair_kernel<KF, VF, NH, 2><<<grid, pair_threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
+        else if (blk && a.block_size == 16)
             decode_blk_kernel<KF, VF, NH, 1><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
         else if (blk && a.block_size == 32)
             decode_blk_kernel<KF, VF, NH, 2><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);

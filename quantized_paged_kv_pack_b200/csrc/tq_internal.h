@@ -1,7 +1,10 @@
 // Internal declarations shared by the host codec and the CUDA kernels of libtq.
 #pragma once
 
+#include <cuda_runtime_api.h>
+
 #include <cstdint>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -12,6 +15,20 @@ namespace tq {
 constexpr int kHeadDim = 128;   // the only head_dim the kernels implement
 constexpr int kMaxHeads = 1024;
 constexpr int kMaxLevels = 16;  // 4-bit codebooks at most on the GPU path
+
+// Quantizer cell table of a uniform 4-bit codec, used by the tensor-core
+// pack: a rotated unit coordinate u, scaled to v = 64 u, falls into cell
+// round(v) + 64 of 129 cells over [-64, 64]; a cell holds the number of
+// decision boundaries strictly below it and the one boundary inside it (in
+// units of v; +inf when none). The codec builds it on the host and copies it
+// to the device with its other tables.
+constexpr int kPackCells = 129;
+constexpr float kPackCellScale = 64.0f;
+struct PackCell {
+    float thr;       // boundary inside the cell, +inf if none
+    int32_t below;   // boundaries strictly below the cell
+};
+void build_pack_cells(const float* boundaries, int levels, PackCell* out);
 
 // Device-side view of one codec, passed to kernels by value.
 struct DevCodec {
@@ -34,6 +51,7 @@ struct DevCodec {
     const float* qjl_st;    // QJL: S transposed, [128][128] (entry j * 128 + i = S[i][j])
     int32_t groupwise;      // 1: group-wise rotation with per-group norms
     const float* rot_t;     // group-wise: R transposed per head, [H][128][128] (entry (h, j, p) = R_h[p][j])
+    const PackCell* cells;  // uniform 4-bit codecs: the pack's quantizer cell table [129]; else null
 };
 
 // Arguments of the decode kernels (device pointers; see tq_decode_paged).
@@ -88,6 +106,23 @@ struct tq_codec {
 };
 
 namespace tq {
+
+// Runs f() (which returns a cudaError_t) once per device ordinal for each
+// call site: settings such as a kernel's shared-memory attribute apply only to
+// the device that is current when they are made. A failure is returned and
+// retried on the next call.
+template <class F>
+cudaError_t once_per_device(int dev, F&& f) {
+    static std::mutex mu;
+    static std::vector<int8_t> done;
+    if (dev < 0) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (static_cast<size_t>(dev) >= done.size()) done.resize(static_cast<size_t>(dev) + 1, 0);
+    if (done[dev]) return cudaSuccess;
+    const cudaError_t e = f();
+    if (e == cudaSuccess) done[dev] = 1;
+    return e;
+}
 
 // Sets the thread-local error message and returns `st`.
 tq_status fail(tq_status st, const std::string& msg);

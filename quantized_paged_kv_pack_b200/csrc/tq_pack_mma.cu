@@ -44,13 +44,9 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kPW = 16;              // warps per CTA (one CTA per SM)
 constexpr int kRowPad = 272;         // bytes per staged input row (256 + 16: 8 rows hit 8 bank quads)
-constexpr int kCells = 129;          // v = 64 u in [-64, 64], cells round(v) + 64
-constexpr float kCellScale = 64.0f;
-
-struct QuantCell {                   // one table entry (8 bytes)
-    float thr;                       // boundary inside the cell (in units of v), +inf if none
-    int below;                       // boundaries strictly below the cell
-};
+constexpr int kCells = kPackCells;   // v = 64 u in [-64, 64], cells round(v) + 64
+constexpr float kCellScale = kPackCellScale;
+using QuantCell = PackCell;          // one table entry (8 bytes), built with the codec
 
 struct PackSmem {
     QuantCell cells[kCells][32];     // replicated per lane: conflict-free 8-byte lookups
@@ -138,7 +134,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
-__global__ void __launch_bounds__(kPW * 32, 1) pack_u4_kernel(DevCodec kc, DevCodec vc, QuantCell* __restrict__ g_cells,
+__global__ void __launch_bounds__(kPW * 32, 1) pack_u4_kernel(DevCodec kc, DevCodec vc, const QuantCell* __restrict__ g_cells,
                                                           const __nv_bfloat16* __restrict__ k,
                                                           const __nv_bfloat16* __restrict__ v,
                                                           const int64_t* __restrict__ slots, int num_tokens,
@@ -380,21 +376,6 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_u4_kernel(DevCodec kc, DevCo
     }
 }
 
-// Cell table of a codebook's boundaries (units of v = 64 u).
-void build_cells(const float* boundaries, int levels, QuantCell* out) {
-    for (int e = 0; e < kCells; ++e) {
-        const double lo = e - 64 - 0.5, hi = e - 64 + 0.5;
-        int below = 0;
-        float thr = INFINITY;
-        for (int i = 0; i + 1 < levels; ++i) {
-            const double bv = static_cast<double>(boundaries[i]) * kCellScale;
-            if (bv < lo) ++below;
-            else if (bv <= hi) thr = static_cast<float>(bv);
-        }
-        out[e] = QuantCell{thr, below};
-    }
-}
-
 }  // namespace
 
 // Launches the uniform 4-bit fast path; TQ_ERR_UNSUPPORTED when it does not apply.
@@ -410,27 +391,23 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
     const int64_t n_units = (num_tokens + 15) / 16 * kc->desc.num_kv_heads * 2;
     if (capacity > INT32_MAX || n_units > INT32_MAX || num_tokens > INT32_MAX - 16) return TQ_ERR_UNSUPPORTED;
     const int bs_log2 = (block_size & (block_size - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(block_size)) : -1;
-    // The cell table depends only on the 4-bit codebook, the same for every codec.
-    static std::once_flag once;
-    static QuantCell* d_cells = nullptr;
-    static cudaError_t err = cudaSuccess;
-    std::call_once(once, [&] {
-        QuantCell host[kCells];
-        build_cells(kc->bound[0], 16, host);
-        err = cudaMalloc(&d_cells, sizeof(host));
-        if (err == cudaSuccess) err = cudaMemcpy(d_cells, host, sizeof(host), cudaMemcpyHostToDevice);
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(pack_u4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sizeof(PackSmem)));
+    // The quantizer cell table comes with the K codec (every uniform 4-bit
+    // codebook is the same). The kernel's shared-memory size is set once per
+    // device.
+    if (!kc->dev.cells) return TQ_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
+    const cudaError_t err = once_per_device(dev, [] {
+        return cudaFuncSetAttribute(pack_u4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(sizeof(PackSmem)));
     });
     if (err != cudaSuccess) return fail(TQ_ERR_CUDA, "pack fast path setup failed");
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
+    int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t want = (n_units + kPW - 1) / kPW;
     const int grid = static_cast<int>(want < sms ? want : sms);
     pack_u4_kernel<<<grid, kPW * 32, sizeof(PackSmem), static_cast<cudaStream_t>(stream)>>>(
-        kc->dev, vc->dev, d_cells, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        kc->dev, vc->dev, kc->dev.cells, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
         slot_mapping, static_cast<int>(num_tokens), static_cast<uint8_t*>(k_pages), static_cast<uint8_t*>(v_pages),
         static_cast<int>(capacity), block_size, bs_log2, d_err);
     return TQ_OK;

@@ -105,15 +105,16 @@ WORKLOADS = {
         (3, 2), (64, 64), (4, 3), (64, 64), 61, 62, 8, True, "fixed:16384", k_qjl=True,
         description="decode batch 16, 32 query / 8 KV heads (Llama-3.1-8B), context 16384, block 16, "
                     "K 2.5-bit MSE (64 channels at 3 bits + 64 at 2) plus the 1-bit QJL residual stage "
-                    "(3.5 bits per channel), V 3.5-bit, 128-token bf16 window; QJL keys run on the general "
-                    "CUDA-core kernel"),
+                    "(3.5 bits per channel), V 3.5-bit, 128-token bf16 window; QJL keys are scored on the tensor cores "
+                    "(sign k-steps)"),
     "decode_llama8b_3p5bit_groupwise": Workload(
         "decode_llama8b_3p5bit_groupwise", "decode", 1007, 16, 32, 8, 128, 16, 128,
         (4, 3), (64, 64), (4, 3), (64, 64), 71, 72, 8, True, "fixed:16384", groupwise=True,
         description="decode batch 16, 32 query / 8 KV heads (Llama-3.1-8B), context 16384, block 16, "
                     "K and V 3.5-bit group-wise: 64 original channels (the outlier channels among them) "
                     "at 4 bits and the other 64 at 3 bits, each group rotated on its own with its own norm, "
-                    "128-token bf16 window; group-wise formats run on the general CUDA-core kernel"),
+                    "128-token bf16 window; group-wise K and V run on the tensor-core kernel "
+                    "(query rotated by the dense per-head R_h)"),
 }
 
 

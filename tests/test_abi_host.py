@@ -236,3 +236,22 @@ def test_static_workspace_size_matches_header():
     m = re.search(r"#define\s+TQ_STATIC_WORKSPACE_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", text)
     assert m, "TQ_STATIC_WORKSPACE_BYTES not found in tq.h"
     assert tq.static_workspace_bytes() == int(m.group(1)) << int(m.group(2))
+
+
+def test_device_allocation_and_setup_are_per_codec_and_per_device():
+    """The library allocates device memory only in tq_make_codec (the header's contract), and
+    device settings are made once per device, not once per process: no source under csrc/ keeps
+    a process-wide device pointer or a call_once around CUDA state."""
+    csrc = os.path.join(ROOT, "quantized_paged_kv_pack_b200", "csrc")
+    allocs = []
+    for name in sorted(os.listdir(csrc)):
+        text = open(os.path.join(csrc, name)).read()
+        code = re.sub(r"//[^\n]*|/\*.*?\*/", "", text, flags=re.S)
+        assert "call_once" not in code and "once_flag" not in code, name
+        for m in re.finditer(r"\bcudaMalloc\w*\s*\(", code):
+            start, end = code.find("tq_status tq_make_codec("), code.find("void tq_free_codec(")
+            allocs.append((name, 0 <= start < m.start() < end))
+    assert allocs == [("tq_codec.cpp", True)], allocs
+    codec = open(os.path.join(csrc, "tq_codec.cpp")).read()
+    make = codec[codec.index("tq_status tq_make_codec("):codec.index("void tq_free_codec(")]
+    assert "build_pack_cells" in make and "dev.cells" in make  # the pack's cell table rides in that allocation
