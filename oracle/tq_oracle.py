@@ -76,6 +76,18 @@ R17 Group-wise rotation (the original-channel reading of the high/low
     n_g = |x[ch_g]| (fp16) and codebook (Lloyd-Max for dimension |g|);
     u_g = y_g / n_g. Row = [group-0 indices][group-1 indices][n_0][n_1];
     the norm area of a sub-page holds (n_0, n_1) per row.
+R18 The recipe row as printed (TurboQuant "Design" page, "Recipe Strategy":
+    two groups, each [MSE indices][QJL signs][vector norm][residual norm]):
+    groupwise and qjl together. Each group is quantized as in R17 (its own
+    block-Hadamard rotation, norm n_g and dimension-n_g codebook); its
+    residual r_g = u_g - c_g[idx_g] (the group's rotated order) gets fp16 norm
+    gamma_g and n_g sign bits [(S_g r_g)_i >= 0], S_g an n_g x n_g matrix of
+    iid N(0, 1) (recipe_qjl_matrix). The key is, per group, n_g B_g^T (c_g +
+    sqrt(pi/2)/n_g gamma_g S_g^T z_g) on the group's channels. The logical
+    row keeps the printed order; in a sub-page the index area holds each
+    group's [indices][signs] (group 0, then group 1) and the norm area its
+    (n_g, gamma_g) pairs, so index rows stay whole bytes apart from the norms
+    as in R6.
 R14 Boundary-token preservation: the first S and the last W tokens of a
     sequence stay dense, the ones between are packed (boundary_dense_tokens).
     Attention is a sum over keys, so the dense ones may sit in one buffer in
@@ -129,8 +141,10 @@ class Format:
 
     def __post_init__(self):
         d = self.head_dim
-        if self.groupwise and (len(self.group_bits) != 2 or self.qjl):
-            raise ValueError("group-wise rotation needs two groups and no QJL stage")
+        if self.groupwise and len(self.group_bits) != 2:
+            raise ValueError("group-wise rotation needs two groups")
+        if self.groupwise and self.qjl and any(n % 8 for n in self.group_size):
+            raise ValueError("the recipe row needs whole sign bytes per group")
         if len(self.group_bits) != len(self.group_size) or len(self.group_bits) not in (1, 2):
             raise ValueError("one or two channel groups")
         if sum(self.group_size) != d:
@@ -368,8 +382,16 @@ def index_bytes(fmt: Format) -> int:
 
 
 def norm_bytes(fmt: Format) -> int:
-    """fp16 norm, then the fp16 residual norm with QJL (R16) or the group-1 norm (R17)."""
+    """fp16 norm, then the fp16 residual norm with QJL (R16) or the group-1 norm (R17);
+    the recipe row (R18) holds (norm, residual norm) of each group."""
+    if fmt.qjl and fmt.groupwise:
+        return 8
     return 4 if (fmt.qjl or fmt.groupwise) else 2
+
+
+def recipe(fmt: Format) -> bool:
+    """The recipe row of R18: group-wise rotation with a QJL stage per group."""
+    return bool(fmt.qjl and fmt.groupwise)
 
 
 def pow2_blocks(n: int):
@@ -476,12 +498,47 @@ def qjl_matrix(fmt: Format) -> np.ndarray:
     return _qjl_matrix_cached(int(fmt.seed), int(fmt.head_dim)).copy()
 
 
+@functools.lru_cache(maxsize=None)
+def _recipe_matrix_cached(seed: int, group: int, n: int) -> np.ndarray:
+    x = splitmix64(seed ^ QJL_SEED_XOR ^ ((group + 1) << 56), 2 * n * n)
+    a = np.array(x[0::2], dtype=np.uint64)
+    b = np.array(x[1::2], dtype=np.uint64)
+    u1 = ((a >> np.uint64(11)).astype(np.float64) + 1.0) * 2.0 ** -53  # (0, 1]
+    u2 = (b >> np.uint64(11)).astype(np.float64) * 2.0 ** -53          # [0, 1)
+    z = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)         # Box-Muller, cosine branch
+    return z.astype(np.float32).astype(np.float64).reshape(n, n)
+
+
+def recipe_qjl_matrix(fmt: Format, group: int) -> np.ndarray:
+    """S_g of R18 (n_g x n_g): the R16 construction on the SplitMix64 stream seeded with
+    seed ^ QJL_SEED_XOR ^ ((g + 1) << 56), one stream per group."""
+    return _recipe_matrix_cached(int(fmt.seed), int(group), int(fmt.group_size[group])).copy()
+
+
+def _quantize_recipe(x, fmt: Format, head: int):
+    """quantize_qjl() under R18: signs [..., d] (group 0's n_0 bits, then group 1's) and
+    g16 [..., 2] (the groups' fp16 residual norms)."""
+    idx, n16, u = _quantize_groupwise(x, fmt, head)
+    signs = np.empty(idx.shape, dtype=np.int64)
+    g16 = []
+    start = 0
+    for g, (b, size) in enumerate(zip(fmt.group_bits, fmt.group_size)):
+        c, _ = codebook(b, size)
+        r = u[..., start:start + size] - c[idx[..., start:start + size]]
+        g16.append(fp16_round(np.sqrt(np.sum(r * r, axis=-1))))
+        signs[..., start:start + size] = (r @ recipe_qjl_matrix(fmt, g).T >= 0).astype(np.int64)
+        start += size
+    return idx, n16, u, signs, np.stack(g16, axis=-1)
+
+
 def quantize_qjl(x, fmt: Format, head: int):
     """quantize() plus the QJL stage (R16): returns (idx, n16, u, signs, g16).
 
     signs[..., i] in {0, 1} (1: (S r)_i >= 0), g16 = fp16(||r||), r the
     residual of u in rotated coordinate order.
     """
+    if recipe(fmt):
+        return _quantize_recipe(x, fmt, head)
     idx, n16, u = quantize(x, fmt, head)
     d = fmt.head_dim
     c_hat = np.empty(idx.shape, dtype=np.float64)
@@ -522,9 +579,37 @@ def _fp16_bytes(n16):
     return np.asarray(n16, dtype=np.float64).astype(np.float16).view(np.uint8).reshape(np.shape(n16) + (2,))
 
 
+def _bits(seg, b):
+    """LSB-first bitstream bytes of the indices seg[..., n] at b bits each."""
+    seg = np.asarray(seg, dtype=np.int64)
+    if np.any(seg < 0) or np.any(seg >= (1 << b)):
+        raise ValueError("index out of range for its group")
+    bits = (seg[..., :, None] >> np.arange(b)) & 1
+    return np.packbits(bits.reshape(seg.shape[:-1] + (seg.shape[-1] * b,)).astype(np.uint8), axis=-1,
+                       bitorder="little")
+
+
+def _unbits(data, n, b):
+    bits = np.unpackbits(np.asarray(data, dtype=np.uint8), axis=-1, bitorder="little")
+    bits = bits.reshape(data.shape[:-1] + (n, b))
+    return (bits.astype(np.int64) << np.arange(b)).sum(axis=-1)
+
+
 def encode_rows(idx, n16, fmt: Format, signs=None, g16=None) -> np.ndarray:
-    """Pack indices (packed order) and fp16 norms into rows of ``row_bytes`` (R6; R16 with QJL)."""
+    """Pack indices (packed order) and fp16 norms into rows of ``row_bytes`` (R6; R16 with QJL;
+    R18 for the recipe row, in its printed field order)."""
     idx = np.asarray(idx, dtype=np.int64)
+    if recipe(fmt):
+        if signs is None or g16 is None:
+            raise ValueError("the recipe row needs the signs and the residual norms")
+        n16, g16 = np.asarray(n16, dtype=np.float64), np.asarray(g16, dtype=np.float64)
+        parts, start = [], 0
+        for g, (b, size) in enumerate(zip(fmt.group_bits, fmt.group_size)):
+            parts.append(_bits(idx[..., start:start + size], b))
+            parts.append(_bits(np.asarray(signs)[..., start:start + size], 1))
+            parts += [_fp16_bytes(n16[..., g]), _fp16_bytes(g16[..., g])]
+            start += size
+        return np.concatenate(parts, axis=-1)
     lead = idx.shape[:-1]
     parts = []
     start = 0
@@ -558,6 +643,18 @@ def decode_rows(rows, fmt: Format):
     lead = rows.shape[:-1]
     if rows.shape[-1] != row_bytes(fmt):
         raise ValueError("row length does not match the format")
+    if recipe(fmt):
+        idx, signs, n16, g16, off = [], [], [], [], 0
+        for b, size in zip(fmt.group_bits, fmt.group_size):
+            idx.append(_unbits(rows[..., off:off + size * b // 8], size, b))
+            off += size * b // 8
+            signs.append(_unbits(rows[..., off:off + size // 8], size, 1))
+            off += size // 8
+            n16.append(rows[..., off:off + 2].copy().view(np.float16).reshape(lead).astype(np.float64))
+            g16.append(rows[..., off + 2:off + 4].copy().view(np.float16).reshape(lead).astype(np.float64))
+            off += 4
+        return (np.concatenate(idx, axis=-1), np.stack(n16, axis=-1), np.concatenate(signs, axis=-1),
+                np.stack(g16, axis=-1))
     idx = []
     off = 0
     for b, size in zip(fmt.group_bits, fmt.group_size):
@@ -587,6 +684,20 @@ def dequantize_rows(idx, n16, fmt: Format, head: int, signs=None, g16=None):
     """
     idx = np.asarray(idx, dtype=np.int64)
     d = fmt.head_dim
+    if recipe(fmt):  # R18: per group c_g + sqrt(pi/2)/n_g gamma_g S_g^T z_g, scaled by n_g, then R^T
+        if signs is None or g16 is None:
+            raise ValueError("the recipe row needs the signs and the residual norms")
+        vals = np.empty(idx.shape, dtype=np.float64)
+        start = 0
+        for g, (b, size) in enumerate(zip(fmt.group_bits, fmt.group_size)):
+            c, _ = codebook(b, size)
+            z = 2.0 * np.asarray(signs, dtype=np.float64)[..., start:start + size] - 1.0
+            gam = np.asarray(g16, dtype=np.float64)[..., g:g + 1]
+            seg = c[idx[..., start:start + size]] + (math.sqrt(math.pi / 2.0) / size) * gam * (
+                z @ recipe_qjl_matrix(fmt, g))
+            vals[..., start:start + size] = seg * np.asarray(n16, dtype=np.float64)[..., g:g + 1]
+            start += size
+        return vals @ group_rotation(fmt, head)
     vals = np.empty(idx.shape, dtype=np.float64)
     start = 0
     for b, size in zip(fmt.group_bits, fmt.group_size):
@@ -617,12 +728,27 @@ def subpage_bytes(fmt: Format, block_size: int) -> int:
     return block_size * row_bytes(fmt)
 
 
+def subpage_byte_order(fmt: Format) -> np.ndarray:
+    """Logical row bytes in the order a sub-page stores them: the first index_bytes(fmt) go to
+    the row's place in the index area, the rest to its place in the norm area (R6). For the recipe
+    row (R18) that is each group's [indices][signs], then each group's (norm, residual norm)."""
+    if not recipe(fmt):
+        return np.arange(row_bytes(fmt))
+    heads, tails, off = [], [], 0
+    for b, size in zip(fmt.group_bits, fmt.group_size):
+        a = size * b // 8 + size // 8
+        heads.append(np.arange(off, off + a))
+        tails.append(np.arange(off + a, off + a + 4))
+        off += a + 4
+    return np.concatenate(heads + tails)
+
+
 def write_rows(pages, blocks, head: int, offsets, rows, fmt: Format, block_size: int):
     """Store logical rows at (block, offset) of one head's sub-pages (R6 layout)."""
     ib, nb = index_bytes(fmt), norm_bytes(fmt)
     blocks = np.asarray(blocks, dtype=np.int64)
     offsets = np.asarray(offsets, dtype=np.int64)
-    rows = np.asarray(rows, dtype=np.uint8)
+    rows = np.asarray(rows, dtype=np.uint8)[..., subpage_byte_order(fmt)]
     cols = offsets[:, None] * ib + np.arange(ib)[None, :]
     pages[blocks[:, None], head, cols] = rows[:, :ib]
     ncols = block_size * ib + nb * offsets[:, None] + np.arange(nb)[None, :]
@@ -636,7 +762,10 @@ def read_rows(pages, blocks, head: int, offsets, fmt: Format, block_size: int):
     offsets = np.asarray(offsets, dtype=np.int64)
     cols = offsets[:, None] * ib + np.arange(ib)[None, :]
     ncols = block_size * ib + nb * offsets[:, None] + np.arange(nb)[None, :]
-    return np.concatenate((pages[blocks[:, None], head, cols], pages[blocks[:, None], head, ncols]), axis=-1)
+    stored = np.concatenate((pages[blocks[:, None], head, cols], pages[blocks[:, None], head, ncols]), axis=-1)
+    rows = np.empty_like(stored)
+    rows[..., subpage_byte_order(fmt)] = stored
+    return rows
 
 
 def pack_kv(k, v, slot_mapping, kfmt: Format, vfmt: Format, num_blocks: int, block_size: int,
@@ -789,7 +918,8 @@ def byte_ledger(kfmt: Format, vfmt: Format, seq_lens: Sequence[int], window: int
     (4 with QJL: the residual norm too), K and V. codebooks: fp16 centroids
     and fp32 boundaries of every group of both codecs. transforms: d int8 signs
     and H_kv*d int16 permutation entries per codec, plus the fp32 d x d QJL
-    matrix of a QJL codec, plus for a group-wise codec (R17) its per-head
+    matrix of a QJL codec (one n_g x n_g S_g per group for the recipe row,
+    R18), plus for a group-wise codec (R17) its per-head
     rotation held as a dense fp32 d x d matrix R_h per KV head ("System
     Invariants": the all-in ratio counts transforms). window: the allocated
     bf16 window, K and V. block tables: one int32 per used block.
@@ -805,8 +935,12 @@ def byte_ledger(kfmt: Format, vfmt: Format, seq_lens: Sequence[int], window: int
     for fmt in (kfmt, vfmt):
         for b in fmt.group_bits:
             cb += (1 << b) * 2 + ((1 << b) - 1) * 4
-    transforms = (2 * (d + H * d * 2) + sum(4 * d * d for fmt in (kfmt, vfmt) if fmt.qjl)
-                  + sum(4 * H * d * d for fmt in (kfmt, vfmt) if fmt.groupwise))
+    transforms = 2 * (d + H * d * 2)
+    for fmt in (kfmt, vfmt):
+        if fmt.qjl:  # S (R16), or one S_g per group for the recipe row (R18)
+            transforms += sum(4 * n * n for n in fmt.group_size) if fmt.groupwise else 4 * d * d
+        if fmt.groupwise:
+            transforms += 4 * H * d * d
     win = 2 * 2 * len(lens) * H * window * d
     bt = 4 * sum(-(-p // block_size) for p in packed)
     pool = num_blocks * H * block_size * (row_bytes(kfmt) + row_bytes(vfmt))

@@ -848,3 +848,149 @@ def test_ledger_transform_bytes_are_the_transforms_a_decode_holds():
                 if f.groupwise:
                     expect += sum(O.group_rotation(f, h).astype(np.float32).nbytes for h in range(H))
             assert led.transform_bytes == expect, (kf, vf)
+
+
+# ---- the recipe row as printed (R18): group-wise rotation with a QJL stage per group ---------
+
+def _recipe_format(bits=(4, 3), sizes=(64, 64), H=2, seed=11, d=D):
+    rng = np.random.default_rng(seed)
+    high = np.stack([np.sort(rng.choice(d, sizes[0], replace=False)) for _ in range(H)])
+    return O.Format(d, H, bits, sizes, high, seed, qjl=True, groupwise=True)
+
+
+def test_recipe_row_layout_by_hand():
+    """Two groups, each [MSE indices][QJL signs][vector norm][residual norm], decoded bit by bit."""
+    rng = np.random.default_rng(21)
+    d = 32
+    f = _recipe_format((3, 2), (16, 16), H=1, seed=4, d=d)
+    assert O.row_bytes(f) == (6 + 2 + 4) + (4 + 2 + 4)
+    x = O.bf16_round(rng.standard_normal((5, d)) * 3)
+    idx, n16, u, signs, g16 = O.quantize_qjl(x, f, 0)
+    rows = O.encode_rows(idx, n16, f, signs, g16)
+    for t in range(5):
+        row = rows[t]
+        bit = lambda k: (int(row[k // 8]) >> (k % 8)) & 1
+        pos = 0
+        for g, (b, n) in enumerate(((3, 16), (2, 16))):
+            for p in range(n):
+                assert sum(bit(pos + j) << j for j in range(b)) == idx[t, 16 * g + p]
+                pos += b
+            for p in range(n):
+                assert bit(pos) == signs[t, 16 * g + p]
+                pos += 1
+            nb = pos // 8
+            assert struct.unpack("<e", bytes(row[nb:nb + 2]))[0] == n16[t, g]
+            assert struct.unpack("<e", bytes(row[nb + 2:nb + 4]))[0] == g16[t, g]
+            pos += 32
+        assert pos == 8 * O.row_bytes(f)
+    back = O.decode_rows(rows, f)
+    for a, b in zip(back, (idx, n16, signs, g16)):
+        assert np.array_equal(a, b)
+
+
+def test_recipe_subpage_order_and_round_trip():
+    """In a sub-page: each group's [indices][signs] in the index area, each group's (norm, residual
+    norm) in the norm area; rows written and read back are unchanged."""
+    f = _recipe_format((4, 2), (32, 96), H=1, seed=5)
+    a0, a1 = 32 * 4 // 8 + 4, 96 * 2 // 8 + 12
+    order = O.subpage_byte_order(f)
+    assert O.index_bytes(f) == a0 + a1 and O.norm_bytes(f) == 8
+    assert np.array_equal(order[:a0], np.arange(a0))
+    assert np.array_equal(order[a0:a0 + a1], np.arange(a0 + 4, a0 + 4 + a1))
+    assert np.array_equal(order[a0 + a1:], np.r_[a0:a0 + 4, a0 + a1 + 4:a0 + a1 + 8])
+    rng = np.random.default_rng(3)
+    bs, nb = 4, 3
+    pages = np.zeros((nb, 1, O.subpage_bytes(f, bs)), np.uint8)
+    rows = rng.integers(0, 256, (6, O.row_bytes(f)), dtype=np.uint8)
+    blocks, offs = np.array([0, 0, 1, 2, 2, 1]), np.array([0, 3, 1, 2, 0, 3])
+    O.write_rows(pages, blocks, 0, offs, rows, f, bs)
+    assert np.array_equal(O.read_rows(pages, blocks, 0, offs, f, bs), rows)
+    # the index bytes of the row at offset 3 of block 0 sit at 3 * index_bytes, its norms after the index area
+    ib = O.index_bytes(f)
+    assert np.array_equal(pages[0, 0, 3 * ib:4 * ib], rows[1, order[:ib]])
+    assert np.array_equal(pages[0, 0, bs * ib + 3 * 8:bs * ib + 4 * 8], rows[1, order[ib:]])
+
+
+def test_recipe_matrices_are_standard_normal_and_distinct():
+    import scipy.stats
+    f = _recipe_format((4, 3), (64, 64), seed=8)
+    S0, S1 = O.recipe_qjl_matrix(f, 0), O.recipe_qjl_matrix(f, 1)
+    assert S0.shape == (64, 64) and S1.shape == (64, 64)
+    assert np.all(S0 == S0.astype(np.float32)) and np.all(S1 == S1.astype(np.float32))
+    for S in (S0, S1):
+        assert scipy.stats.kstest(S.ravel(), "norm").pvalue > 1e-3
+    assert abs(np.corrcoef(S0.ravel(), S1.ravel())[0, 1]) < 0.05
+    assert abs(np.corrcoef(S0.ravel(), O.qjl_matrix(O.Format(64, 1, (4,), (64,), None, 8, qjl=True)).ravel())[0, 1]) < 0.05
+
+
+def test_recipe_key_without_residual_is_the_groupwise_key():
+    """With every residual norm set to 0 the recipe key is the R17 group-wise key of the same
+    indices and norms (the QJL term is the only addition)."""
+    rng = np.random.default_rng(9)
+    f = _recipe_format((4, 3), (64, 64), H=2, seed=13)
+    fg = O.Format(D, 2, (4, 3), (64, 64), f.high_coords, 13, groupwise=True)
+    x = O.bf16_round(rng.standard_normal((7, D)) * 2)
+    idx, n16, _, signs, g16 = O.quantize_qjl(x, f, 1)
+    gi, gn, _ = O.quantize(x, fg, 1)
+    assert np.array_equal(idx, gi) and np.array_equal(n16, gn)
+    key0 = O.dequantize_rows(idx, n16, f, 1, signs, np.zeros_like(g16))
+    assert np.allclose(key0, O.dequantize_rows(gi, gn, fg, 1), atol=1e-12)
+
+
+def test_recipe_key_is_unbiased_over_codec_seeds():
+    """For one fixed x and q over 1500 codec seeds (so every S_g comes from recipe_qjl_matrix):
+    the mean of q.key equals q.x within 4 sigma, the mean squared error stays inside the sum of
+    the groups' QJL bounds pi/(2 n_g) |q_g|^2 gamma_g^2 n_g^2, and the wrong constant
+    sqrt(2/pi)/n_g or the inverted sign convention fail the same mean check."""
+    d, n_seeds = D, 1500
+    rng = np.random.default_rng(41)
+    x = O.bf16_round(rng.standard_normal(d) * 2.0)[None, :]
+    q = x[0] / np.linalg.norm(x[0]) * 8.0 + rng.standard_normal(d)
+    high = np.sort(rng.choice(d, 64, replace=False))[None, :]
+    exact = float(x[0] @ q)
+    est, mse_part, bound = np.empty(n_seeds), np.empty(n_seeds), np.empty(n_seeds)
+    for i in range(n_seeds):
+        f = O.Format(d, 1, (3, 2), (64, 64), high, 500 + i, qjl=True, groupwise=True)
+        idx, n16, u, signs, g16 = O.quantize_qjl(x, f, 0)
+        est[i] = float(O.dequantize_rows(idx, n16, f, 0, signs, g16)[0] @ q)
+        mse_part[i] = float(O.dequantize_rows(idx, n16, f, 0, signs, np.zeros_like(g16))[0] @ q)
+        qg = O.group_rotation(f, 0) @ q  # the query in the groups' rotated coordinates
+        bound[i] = sum(math.pi / (2 * 64) * float(qg[64 * g:64 * (g + 1)] @ qg[64 * g:64 * (g + 1)])
+                       * float(g16[0, g]) ** 2 * float(n16[0, g]) ** 2 for g in range(2))
+    qjl_part = est - mse_part
+    sem = est.std(ddof=1) / math.sqrt(n_seeds)
+    fp16_bias = 2.0 ** -10 * abs(exact)
+    assert abs(est.mean() - exact) < 4 * sem + fp16_bias
+    assert np.mean((est - exact) ** 2) <= 1.15 * bound.mean()
+    assert abs(mse_part.mean() - exact) > 8 * sem + fp16_bias
+    for alt in (mse_part + (2.0 / math.pi) * qjl_part, mse_part - qjl_part):
+        alt_sem = alt.std(ddof=1) / math.sqrt(n_seeds)
+        assert abs(alt.mean() - exact) > 8 * max(sem, alt_sem) + fp16_bias
+
+
+def test_recipe_attention_and_ledger():
+    """decode_attention over recipe pages equals dense attention over the recipe keys; the ledger
+    counts 8 norm bytes per row and the two S_g and R_h as transforms."""
+    rng = np.random.default_rng(17)
+    H, bs = 2, 4
+    kf = _recipe_format((4, 3), (64, 64), H=H, seed=2)
+    vf = O.Format(D, H, (4, 3), (64, 64), kf.high_coords, 3, groupwise=True)
+    T = 10
+    k = O.bf16_round(rng.standard_normal((T, H, D)))
+    v = O.bf16_round(rng.standard_normal((T, H, D)))
+    kp, vp = O.pack_kv(k, v, np.arange(T), kf, vf, 3, bs)
+    q = O.bf16_round(rng.standard_normal((1, 2 * H, D)))
+    out = O.decode_attention(q, kp, vp, np.array([[0, 1, 2]]), [T], np.zeros((1, H, 1, D)),
+                             np.zeros((1, H, 1, D)), 0, 0.2, kf, vf, bs)
+    for h in range(H):
+        idx, n16, _, signs, g16 = O.quantize_qjl(k[:, h], kf, h)
+        keys = O.dequantize_rows(idx, n16, kf, h, signs, g16)
+        vi, vn, _ = O.quantize(v[:, h], vf, h)
+        vals = O.dequantize_rows(vi, vn, vf, h)
+        for g in range(2):
+            ref = O.dense_attention(q[0, 2 * h + g], keys, vals, 0.2)
+            assert np.abs(out[0, 2 * h + g] - ref).max() < 1e-12
+    led = O.byte_ledger(kf, vf, [T], 0, bs, 3)
+    assert led.norm_bytes == T * H * (8 + 4)
+    expect = 2 * (D + H * D * 2) + 4 * (64 * 64 + 64 * 64) + 2 * 4 * H * D * D
+    assert led.transform_bytes == expect
