@@ -345,6 +345,9 @@ def measure_latency(setup: DecodeSetup, reps, warmup, cold):
 
     cold: before every repetition, outside the event pair, a buffer of twice
     the L2 size is written, so the call starts with none of its data in L2.
+    Before the first event a spin kernel of about 100 us keeps the GPU busy
+    while the host enqueues the call's launches, so the pair times the GPU's
+    work, not the host's launch latency.
     """
     stream = torch.cuda.current_stream()
     l2 = int(getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "L2_cache_size", 0)) or (126 << 20)
@@ -356,6 +359,7 @@ def measure_latency(setup: DecodeSetup, reps, warmup, cold):
         if flush is not None:
             flush.fill_(1.0)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(200_000)  # the spacer (about 100 us at ~2 GHz)
         e0.record(stream)
         setup.decode()
         e1.record(stream)

@@ -92,7 +92,20 @@ typedef enum {
  *                largest first (96 = 64 + 32); each group has its own fp16 norm
  *                and a Lloyd-Max codebook for its own dimension. Row: the two
  *                index bitstreams, then the two norms (norm area: 4 bytes per
- *                row). Pack and decode run it on the general kernels.
+ *                row).
+ *                qjl = 1 together with groupwise = 1 is the recipe row as the
+ *                Design page prints it ("Recipe Strategy": two groups, each
+ *                [MSE indices][QJL signs][vector norm][residual norm]): each
+ *                group is quantized as above and adds the fp16 norm |r_g| of
+ *                its residual r_g = u_g - c_g[idx] (the group's rotated order)
+ *                and group_size[g] sign bits [(S_g r_g)_i >= 0], S_g a
+ *                group_size[g]^2 Gaussian matrix (tq_codec_qjl_matrix). In a
+ *                sub-page the index part of a row is [group-0 indices][group-0
+ *                signs][group-1 indices][group-1 signs] and its norm area holds
+ *                (n_0, |r_0|, n_1, |r_1|), 8 bytes. The key is, per group,
+ *                n_g B_g^T (c_g + sqrt(pi/2)/group_size[g] |r_g| S_g^T z_g) on
+ *                the group's channels. Decode accepts it for K only, on the
+ *                general kernel.
  */
 typedef struct {
     int32_t head_dim;
@@ -124,7 +137,8 @@ typedef struct tq_codec tq_codec; /* opaque, immutable after tq_make_codec */
  * row_bytes      out: index bytes of all groups, plus the QJL sign bytes
  *                (head_dim / 8) of a QJL codec, plus the norm bytes: 2 (fp16
  *                norm), or 4 for a QJL codec (norm, residual norm) and for a
- *                group-wise codec (one norm per group)
+ *                group-wise codec (one norm per group), or 8 for the recipe row
+ *                (qjl and groupwise: norm and residual norm per group)
  * Any output pointer may be NULL. Returns TQ_ERR_VALUE / TQ_ERR_UNSUPPORTED
  * for an invalid descriptor (the GPU format limits apply here too).
  */
@@ -137,7 +151,11 @@ tq_status tq_codec_host_tables(const tq_format_desc* desc, uint16_t* centroids_f
  * from SplitMix64 seeded with hadamard_seed ^ 0x51534A4C00000001: outputs
  * 2k and 2k + 1 (k = i * head_dim + j) give u1 = ((x >> 11) + 1) 2^-53 and
  * u2 = (x >> 11) 2^-53, S = sqrt(-2 ln u1) cos(2 pi u2) in double, rounded to
- * float. Host only; TQ_ERR_VALUE for an invalid descriptor.
+ * float. For the recipe row (qjl and groupwise) out receives S_0 then S_1,
+ * each group_size[g] x group_size[g] row-major (at most head_dim^2 floats in
+ * all), made the same way from the stream seeded with hadamard_seed ^
+ * 0x51534A4C00000001 ^ ((g + 1) << 56). Host only; TQ_ERR_VALUE for an
+ * invalid descriptor.
  */
 tq_status tq_codec_qjl_matrix(const tq_format_desc* desc, float* out);
 

@@ -185,6 +185,20 @@ uint64_t splitmix64_next(uint64_t& state) {
 }
 
 // S of the QJL stage, row-major [d][d] (see tq_codec_qjl_matrix in tq.h).
+// n x n iid N(0, 1) entries (fp32): the Box-Muller cosine branch over pairs of
+// SplitMix64 outputs from `stream_seed`, row-major, appended to out.
+void gaussian_matrix(uint64_t stream_seed, int n, std::vector<float>& out) {
+    const size_t base = out.size();
+    out.resize(base + static_cast<size_t>(n) * n);
+    uint64_t state = stream_seed;
+    for (size_t k = base; k < out.size(); ++k) {
+        const uint64_t a = splitmix64_next(state), b = splitmix64_next(state);
+        const double u1 = (static_cast<double>(a >> 11) + 1.0) * 0x1p-53;  // (0, 1]
+        const double u2 = static_cast<double>(b >> 11) * 0x1p-53;          // [0, 1)
+        out[k] = static_cast<float>(std::sqrt(-2.0 * std::log(u1)) * std::cos(2.0 * M_PI * u2));
+    }
+}
+
 void qjl_matrix(uint64_t seed, int d, std::vector<float>& out) {
     out.resize(static_cast<size_t>(d) * d);
     uint64_t state = seed ^ 0x51534A4C00000001ull;
@@ -230,8 +244,7 @@ tq_status validate_desc(const tq_format_desc* d) {
     if (total != d->head_dim) return fail(TQ_ERR_VALUE, "group sizes must sum to head_dim");
     if (d->qjl != 0 && d->qjl != 1) return fail(TQ_ERR_VALUE, "qjl must be 0 or 1");
     if (d->groupwise != 0 && d->groupwise != 1) return fail(TQ_ERR_VALUE, "groupwise must be 0 or 1");
-    if (d->groupwise && (d->n_groups != 2 || d->qjl))
-        return fail(TQ_ERR_VALUE, "group-wise rotation needs two groups and no QJL stage");
+    if (d->groupwise && d->n_groups != 2) return fail(TQ_ERR_VALUE, "group-wise rotation needs two groups");
     if (d->n_groups == 1) {
         if (d->high_coords) return fail(TQ_ERR_VALUE, "high_coords given for a one-group format");
     } else {
@@ -295,11 +308,20 @@ tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c) {
     }
     int bytes = 0;
     for (int g = 0; g < desc->n_groups; ++g) bytes += desc->group_bits[g] * desc->group_size[g] / 8;
-    const int sign_bytes = desc->qjl ? d / 8 : 0, norm_bytes = (desc->qjl || desc->groupwise) ? 4 : 2;
+    const bool recipe = desc->qjl && desc->groupwise;
+    const int sign_bytes = desc->qjl ? d / 8 : 0;
+    const int norm_bytes = recipe ? 8 : ((desc->qjl || desc->groupwise) ? 4 : 2);
     c->index_bytes = bytes + sign_bytes;
     c->row_bytes = c->index_bytes + norm_bytes;
     c->qjl_s.clear();
-    if (desc->qjl) qjl_matrix(desc->hadamard_seed, d, c->qjl_s);
+    if (recipe) {
+        // the recipe row: one n_g x n_g S_g per group, each from its own stream
+        for (int g = 0; g < 2; ++g)
+            gaussian_matrix(desc->hadamard_seed ^ 0x51534A4C00000001ull ^ (static_cast<uint64_t>(g + 1) << 56),
+                            desc->group_size[g], c->qjl_s);
+    } else if (desc->qjl) {
+        qjl_matrix(desc->hadamard_seed, d, c->qjl_s);
+    }
     c->rot_t.clear();
     if (desc->groupwise) {
         // R_h: rows = packed positions, columns = channels; perm[h] lists group 0's
@@ -341,7 +363,11 @@ tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c) {
         v.byte_off[g] = b0;
         p0 += v.size[g];
         b0 += v.size[g] * v.bits[g] / 8;
+        // the recipe row: each group's sign bits follow its own index bitstream
+        v.sign_off[g] = recipe ? b0 : bytes;
+        if (recipe) b0 += v.size[g] / 8;
     }
+    v.recipe = recipe ? 1 : 0;
     v.index_bytes = c->index_bytes;
     v.row_bytes = c->row_bytes;
     v.qjl = desc->qjl;
@@ -454,6 +480,13 @@ tq_status tq_codec_qjl_matrix(const tq_format_desc* desc, float* out) {
     tq_status st = validate_desc(desc);
     if (st != TQ_OK) return st;
     if (!out) return fail(TQ_ERR_VALUE, "null output pointer");
+    if (desc->qjl && desc->groupwise) {  // the recipe row: S_0 then S_1
+        tq_codec c;
+        st = build_host_tables(desc, &c);
+        if (st != TQ_OK) return st;
+        std::memcpy(out, c.qjl_s.data(), c.qjl_s.size() * sizeof(float));
+        return TQ_OK;
+    }
     std::vector<float> s;
     qjl_matrix(desc->hadamard_seed, desc->head_dim, s);
     std::memcpy(out, s.data(), s.size() * sizeof(float));
@@ -487,7 +520,17 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     std::memcpy(p + n_sign + n_cent, c->bound, n_cent);
     std::memcpy(p + n_sign + 2 * n_cent, c->perm.data(), n_perm);
     std::memcpy(p + n_sign + 2 * n_cent + n_perm, c->pos.data(), n_perm);
-    if (n_s) {  // QJL: S transposed, so that a warp reads one row of S^T per coordinate j
+    if (n_s && c->dev.recipe) {  // recipe row: S_0^T then S_1^T, each n_g x n_g
+        float* st = reinterpret_cast<float*>(p + off_s);
+        size_t off = 0;
+        for (int g = 0; g < 2; ++g) {
+            const int n = desc->group_size[g];
+            for (int i = 0; i < n; ++i)
+                for (int j = 0; j < n; ++j)
+                    st[off + static_cast<size_t>(j) * n + i] = c->qjl_s[off + static_cast<size_t>(i) * n + j];
+            off += static_cast<size_t>(n) * n;
+        }
+    } else if (n_s) {  // QJL: S transposed, so that a warp reads one row of S^T per coordinate j
         float* st = reinterpret_cast<float*>(p + off_s);
         for (int i = 0; i < d; ++i)
             for (int j = 0; j < d; ++j) st[static_cast<size_t>(j) * d + i] = c->qjl_s[static_cast<size_t>(i) * d + j];
@@ -560,14 +603,15 @@ tq_status tq_byte_ledger(const tq_format_desc* kdesc, const tq_format_desc* vdes
     tq_ledger r{};
     r.dense_bytes = 2 * 2 * H * d * total;
     r.index_bytes = packed * H * (kc.index_bytes + vc.index_bytes);
-    r.norm_bytes = packed * H * ((kdesc->qjl || kdesc->groupwise ? 4 : 2) + (vdesc->qjl || vdesc->groupwise ? 4 : 2));
+    r.norm_bytes = packed * H * ((kc.row_bytes - kc.index_bytes) + (vc.row_bytes - vc.index_bytes));
     for (const tq_format_desc* desc : {kdesc, vdesc})
         for (int g = 0; g < desc->n_groups; ++g) {
             int64_t L = int64_t(1) << desc->group_bits[g];
             r.codebook_bytes += L * 2 + (L - 1) * 4;
         }
-    // signs and permutations of both codecs, S of a QJL codec, the per-head R_h of a group-wise codec
-    r.transform_bytes = 2 * (d + H * d * 2) + 4 * d * d * ((kdesc->qjl ? 1 : 0) + (vdesc->qjl ? 1 : 0)) +
+    // signs and permutations of both codecs, S of a QJL codec (S_0 and S_1 of a recipe row), the
+    // per-head R_h of a group-wise codec
+    r.transform_bytes = 2 * (d + H * d * 2) + 4 * static_cast<int64_t>(kc.qjl_s.size() + vc.qjl_s.size()) +
                         4 * H * d * d * ((kdesc->groupwise ? 1 : 0) + (vdesc->groupwise ? 1 : 0));
     r.window_bytes = 2 * 2 * static_cast<int64_t>(batch) * H * window * d;
     r.block_table_bytes = 4 * blocks;

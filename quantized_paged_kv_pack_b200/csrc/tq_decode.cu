@@ -142,7 +142,21 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
     }
     __syncthreads();
     const bool qjl = a.kc.qjl && !is_win;
-    if (qjl) {
+    const bool recipe = a.kc.recipe && !is_win;
+    if (recipe) {
+        // recipe row: per group, (S_g q_g)_i = sum_j S_g^T[j][i] q_r[pos0_g + j] at packed position
+        // pos0_g + i, times sqrt(pi/2)/n_g, the group's estimator constant.
+        const int n0 = a.kc.pos0[1];
+        for (int e = threadIdx.x; e < G * kHeadDim; e += kWarps * 32) {
+            const int g = e / kHeadDim, p = e - g * kHeadDim;
+            const int grp = p >= n0 ? 1 : 0, n = a.kc.size[grp], p0 = a.kc.pos0[grp], i = p - p0;
+            const float* st = a.kc.qjl_st + (grp ? static_cast<int64_t>(n0) * n0 : 0);
+            float acc = 0.0f;
+            for (int j = 0; j < n; ++j) acc = fmaf(__ldg(st + j * n + i), qs[g][p0 + j], acc);
+            sq[g][p] = acc * (1.2533141373155003f / n);  // sqrt(pi/2) / n_g
+        }
+        __syncthreads();
+    } else if (qjl) {
         // (S q_r)_i = sum_j S^T[j][i] q_r[j], q_r[j] = qs[pos(j)]; times sqrt(pi/2)/d, the estimator's constant.
         for (int e = threadIdx.x; e < G * kHeadDim; e += kWarps * 32) {
             const int g = e / kHeadDim, i = e - g * kHeadDim;
@@ -165,6 +179,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
     const int bs = a.block_size;
     for (int t = t0 + warp; t < t1; t += kWarps) {
         float kv[4], vv[4], nk = 1.0f, nv = 1.0f, gk = 0.0f, zk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float wk[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // recipe row: n_g |r_g| of each position's group
         if (is_win) {
             const int64_t base = ((static_cast<int64_t>(b) * H + h) * a.window + t) * kHeadDim + 4 * lane;
 #pragma unroll
@@ -194,7 +209,18 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
             }
             nk = row_norm(ksub, a.kc, bs, off);
             nv = row_norm(vsub, a.vc, bs, off);
-            if (a.kc.groupwise) {  // per-group norms: fold each position's norm into its centroid
+            if (recipe) {  // norm area (n_0, |r_0|, n_1, |r_1|); signs after each group's indices
+                const float n0k = nk, r0k = row_norm(ksub, a.kc, bs, off, 1);
+                const float n1k = row_norm(ksub, a.kc, bs, off, 2), r1k = row_norm(ksub, a.kc, bs, off, 3);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int p = 4 * lane + i, grp = p >= a.kc.pos0[1] ? 1 : 0, sp = p - a.kc.pos0[grp];
+                    kv[i] *= grp ? n1k : n0k;
+                    wk[i] = grp ? n1k * r1k : n0k * r0k;
+                    zk[i] = ((krow[a.kc.sign_off[grp] + (sp >> 3)] >> (sp & 7)) & 1u) ? 1.0f : -1.0f;
+                }
+                nk = 1.0f;
+            } else if (a.kc.groupwise) {  // per-group norms: fold each position's norm into its centroid
                 const float nk1 = row_norm(ksub, a.kc, bs, off, 1);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) kv[i] *= (4 * lane + i >= a.kc.pos0[1]) ? nk1 : nk;
@@ -206,7 +232,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
                 for (int i = 0; i < 4; ++i) vv[i] *= (4 * lane + i >= a.vc.pos0[1]) ? nv1 : nv;
                 nv = 1.0f;
             }
-            if (qjl) {
+            if (qjl && !recipe) {
                 // sign bits 4l .. 4l+3 of the QJL stream (after the index bitstreams)
                 const unsigned bits = (krow[a.kc.mse_bytes + (lane >> 1)] >> (4 * (lane & 1))) & 0xFu;
 #pragma unroll
@@ -219,7 +245,10 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
             float s = 0.0f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) s += qs[g][4 * lane + i] * kv[i];
-            if (qjl) {
+            if (recipe) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s += wk[i] * sq[g][4 * lane + i] * zk[i];  // n_g |r_g| (S_g q_g)_i z_i
+            } else if (qjl) {
                 float t = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) t += sq[g][4 * lane + i] * zk[i];
@@ -318,6 +347,67 @@ __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, c
         x = vc.sign[j] * y[j] * 0.08838834764831845f;
     }
     out[(static_cast<int64_t>(b) * num_q_heads + hq) * kHeadDim + j] = Ls > 0.0f ? (x + win) / Ls : 0.0f;
+}
+
+// Group-wise V: the same merge, then x = R_h^T y. One CTA per (b, KV head)
+// with 128 threads per query head (up to 8 heads at a time): R_h^T is staged
+// once in shared memory with a row pitch of 129 floats (thread j reads row j
+// without bank conflicts), instead of every query head reading the 64 KB
+// matrix from L2 with row-strided loads.
+constexpr int kGwPitch = kHeadDim + 1;
+constexpr int kGwHeads = 8;
+constexpr size_t kGwCombineSmem = (static_cast<size_t>(kHeadDim) * kGwPitch + kGwHeads * kHeadDim) * sizeof(float);
+
+__global__ void __launch_bounds__(kHeadDim * kGwHeads) decode_combine_gw_kernel(
+    DevCodec vc, const int32_t* seq_lens, int32_t num_q_heads, int32_t max_seq_len, int32_t window,
+    int32_t split_tokens, int32_t max_splits, int32_t items_per_unit, int32_t G, const float* ws, float* out) {
+    extern __shared__ float gsm[];
+    float* rts = gsm;                               // [128][129]: R_h^T, row j at j * 129
+    float* ys = gsm + kHeadDim * kGwPitch;          // [kGwHeads][128]
+    const int H = vc.num_heads, h = blockIdx.x % H, b = blockIdx.x / H;
+    const int j = threadIdx.x & (kHeadDim - 1), gl = threadIdx.x >> 7, nthreads = blockDim.x;
+    const float* rt = vc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim;
+    for (int e = threadIdx.x; e < kHeadDim * kHeadDim; e += nthreads)
+        rts[(e >> 7) * kGwPitch + (e & (kHeadDim - 1))] = rt[e];
+    int L = seq_lens[b];
+    L = L < 0 ? 0 : (L > max_seq_len ? max_seq_len : L);
+    const int n_win = min(window, L), P = L - n_win;
+    const int ns = (P + split_tokens - 1) / split_tokens;
+    const float* unit = ws + (static_cast<int64_t>(b) * H + h) * items_per_unit * static_cast<int64_t>(G) * (kHeadDim + 2);
+    const int per = nthreads / kHeadDim;  // query heads per pass
+    for (int g0 = 0; g0 < G; g0 += per) {
+        const int g = g0 + gl;
+        float Ls = 0.0f, rot = 0.0f, win = 0.0f;
+        if (g < G) {
+            auto rec = [&](int i) { return unit + (static_cast<int64_t>(i) * G + g) * (kHeadDim + 2); };
+            float M = -INFINITY;
+            for (int i = 0; i < ns; ++i) M = fmaxf(M, rec(i)[0]);
+            if (n_win) M = fmaxf(M, rec(max_splits)[0]);
+            if (M != -INFINITY) {
+                for (int i = 0; i < ns; ++i) {
+                    const float f = exp2f(rec(i)[0] - M);
+                    Ls += rec(i)[1] * f;
+                    rot += rec(i)[2 + j] * f;
+                }
+                if (n_win) {
+                    const float f = exp2f(rec(max_splits)[0] - M);
+                    Ls += rec(max_splits)[1] * f;
+                    win = rec(max_splits)[2 + j] * f;
+                }
+            }
+            ys[gl * kHeadDim + j] = rot;  // packed positions
+        }
+        __syncthreads();  // (the first pass also waits for the staged R_h^T)
+        if (g < G) {
+            const float* rj = rts + j * kGwPitch;
+            const float* y = ys + gl * kHeadDim;
+            float x = 0.0f;
+#pragma unroll 8
+            for (int p = 0; p < kHeadDim; ++p) x = fmaf(rj[p], y[p], x);
+            out[(static_cast<int64_t>(b) * num_q_heads + h * G + g) * kHeadDim + j] = Ls > 0.0f ? (x + win) / Ls : 0.0f;
+        }
+        __syncthreads();
+    }
 }
 
 tq_status check_decode_args(const tq_codec* kc, const tq_codec* vc, int32_t batch, int32_t num_q_heads,
@@ -454,9 +544,24 @@ extern "C" tq_status tq_decode_combine(const tq_codec* vc, const int32_t* seq_le
     if (batch == 0) return TQ_OK;
     if (!out || !seq_lens) return fail(TQ_ERR_VALUE, "null buffer");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    decode_combine_kernel<<<dim3(num_q_heads, batch), kHeadDim, 0, s>>>(
-        vc->dev, seq_lens, num_q_heads, max_seq_len, window, plan.split_tokens, plan.max_splits,
-        plan.items_per_unit, plan.group, static_cast<const float*>(workspace), out);
+    if (vc->desc.groupwise) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
+        const cudaError_t e = once_per_device(dev, [] {
+            return cudaFuncSetAttribute(decode_combine_gw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kGwCombineSmem));
+        });
+        if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "cannot reserve shared memory for the combine kernel");
+        const int threads = kHeadDim * std::min(plan.group, kGwHeads);
+        decode_combine_gw_kernel<<<static_cast<unsigned>(batch) * vc->desc.num_kv_heads, threads, kGwCombineSmem,
+                                   s>>>(vc->dev, seq_lens, num_q_heads, max_seq_len, window, plan.split_tokens,
+                                        plan.max_splits, plan.items_per_unit, plan.group,
+                                        static_cast<const float*>(workspace), out);
+    } else {
+        decode_combine_kernel<<<dim3(num_q_heads, batch), kHeadDim, 0, s>>>(
+            vc->dev, seq_lens, num_q_heads, max_seq_len, window, plan.split_tokens, plan.max_splits,
+            plan.items_per_unit, plan.group, static_cast<const float*>(workspace), out);
+    }
     return finish(s, nullptr, "decode combine");
 }
 

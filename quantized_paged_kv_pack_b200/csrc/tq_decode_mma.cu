@@ -249,6 +249,26 @@ __device__ __forceinline__ Words<(NB + 3) / 4> lds_span(uint32_t a) {
     return r;
 }
 
+// NB bytes at shared address a + off, where a is 4-byte aligned and off is a
+// per-lane constant: the alignment split of off (word offset and shift) does
+// not depend on a, so the compiler computes it once per lane.
+template <int NB, bool ALIGNED>
+__device__ __forceinline__ Words<(NB + 3) / 4> lds_span_off(uint32_t a, uint32_t off) {
+    if constexpr (ALIGNED) {
+        return lds_span<NB, true>(a + off);
+    } else {
+        constexpr int NW = (NB + 3) / 4;
+        const uint32_t base = a + (off & ~3u), sh = (off & 3u) * 8;
+        Words<NW> r;
+        uint32_t raw[NW + 1];
+#pragma unroll
+        for (int i = 0; i <= NW; ++i) raw[i] = lds32(base + 4 * i);
+#pragma unroll
+        for (int i = 0; i < NW; ++i) r.w[i] = __funnelshift_r(raw[i], raw[i + 1], sh);
+        return r;
+    }
+}
+
 // Lookup address of the index pair at bits [OFF, OFF + 2B) of a lane's chunk.
 template <int B, int OFF, int NW>
 __device__ __forceinline__ uint32_t pair_addr(const uint32_t (&w)[NW], uint32_t base) {
@@ -694,32 +714,49 @@ struct WarpTiles {
         }
     }
 
-    // Scores of one 16-token tile (K index rows at kbase, norms at knorm) and
-    // the online-softmax update; leaves the tile's P' (V norms at vnorm) in bp
-    // for values(). Tokens at or past nvalid are padding.
-    __device__ __forceinline__ void scores(uint32_t kbase, uint32_t knorm, uint32_t vnorm, int nvalid,
-                                           uint32_t lane_base, uint32_t psel, int r, int c) {
+    // Scores of one 16-token block (K index rows at kbase, norms at knorm), in
+    // log2 units and before any max: sc[e][0] for token r, sc[e][1] for token
+    // r + 8 of the lane's head e; -inf for tokens at or past nvalid (padding).
+    __device__ __forceinline__ void block_scores(const uint32_t (&qf)[8][2 * HL],
+                                                 const uint32_t (&zf)[KQ ? 8 : 1][2 * HL], uint32_t kbase,
+                                                 uint32_t knorm, int nvalid, uint32_t lane_base, int r, int c,
+                                                 float (&sc)[HL][2]) const {
         // ---- S^T = K^ Q'^T: rows tokens r, r + 8 ----
         // Independent accumulator chains (k-step parity, or the group when K is
         // group-wise; hi / lo for NH = 8) keep the MMA dependency depth at 4.
         constexpr int NC = NH == 8 ? 4 : 2;
-        uint32_t qf[8][2 * HL];
-        uint32_t zf[KQ ? 8 : 1][2 * HL];
-        load_query(qf, zf);
+        // QJL keys in tensor memory: the sign fragments are loaded for the
+        // sign k-steps and the index fragments after them, never both at once.
+        constexpr bool kOwnLoads = KQ && TM;
         float sacc[NC][4];
 #pragma unroll
         for (int u = 0; u < NC; ++u) sacc[u][0] = sacc[u][1] = sacc[u][2] = sacc[u][3] = 0.0f;
+        uint32_t ql[kOwnLoads ? 8 : 1][2 * HL];
         auto score_step = [&](auto si, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
             constexpr int s_ = decltype(si)::value;
             constexpr int u = KG ? (s_ < KF::KS0 ? 0 : 1) : (s_ & 1);
+            const auto& Q = [&]() -> const auto& {
+                if constexpr (kOwnLoads) return ql;
+                else return qf;
+            }();
             if constexpr (NH == 8) {
-                mma16816(sacc[u], a0, a1, a2, a3, qf[s_][0], qf[s_][1]);
-                mma16816(sacc[2 + u], a0, a1, a2, a3, qf[s_][2], qf[s_][3]);
+                mma16816(sacc[u], a0, a1, a2, a3, Q[s_][0], Q[s_][1]);
+                mma16816(sacc[2 + u], a0, a1, a2, a3, Q[s_][2], Q[s_][3]);
             } else {
-                mma16816(sacc[u], a0, a1, a2, a3, qf[s_][0], qf[s_][1]);
+                mma16816(sacc[u], a0, a1, a2, a3, Q[s_][0], Q[s_][1]);
             }
         };
         if constexpr (KQ) {
+            uint32_t zl[kOwnLoads ? 8 : 1][2 * HL];
+            if constexpr (kOwnLoads) {
+                tm_ld<NQW>(tm + kTmZ, &zl[0][0]);
+                tm_wait_ld();
+                tm_dep<NQW>(&zl[0][0]);
+            }
+            const auto& Z = [&]() -> const auto& {
+                if constexpr (kOwnLoads) return zl;
+                else return zf;
+            }();
             // Sign k-step s takes bits s, s + 8, s + 16, s + 24 of the lane's word
             // (projections 32c + ...): shifted to the top of bytes 0..3, prmt
             // turns each into an all-ones or all-zero byte in the high byte of
@@ -736,18 +773,23 @@ struct WarpTiles {
                 const uint32_t a2 = rn_a | (~prmt(ya, 0u, 0xB4A4u) & 0x80008000u);
                 const uint32_t a3 = rn_b | (~prmt(yb, 0u, 0xB4A4u) & 0x80008000u);
                 if constexpr (NH == 8) {
-                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, zf[s_][0], zf[s_][1]);
-                    mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, zf[s_][2], zf[s_][3]);
+                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, Z[s_][0], Z[s_][1]);
+                    mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, Z[s_][2], Z[s_][3]);
                 } else {
-                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, zf[s_][0], zf[s_][1]);
+                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, Z[s_][0], Z[s_][1]);
                 }
             });
+        }
+        if constexpr (kOwnLoads) {
+            tm_ld<NQW>(tm + kTmQ, &ql[0][0]);
+            tm_wait_ld();
+            tm_dep<NQW>(&ql[0][0]);
         }
         {
             constexpr int KW0 = (KF::KC0 + 3) / 4;
             constexpr bool A0 = KF::KC0 % 4 == 0;
-            const Words<KW0> k0a = lds_span<KF::KC0, A0>(kbase + r * KF::RB + c * KF::KC0);
-            const Words<KW0> k0b = lds_span<KF::KC0, A0>(kbase + (r + 8) * KF::RB + c * KF::KC0);
+            const Words<KW0> k0a = lds_span_off<KF::KC0, A0>(kbase + r * KF::RB, c * KF::KC0);
+            const Words<KW0> k0b = lds_span_off<KF::KC0, A0>(kbase + (r + 8) * KF::RB, c * KF::KC0);
             const uint32_t base0 = lut_base<KF::B0>(lane_base);
             static_for<0, KF::KS0>([&](auto si) {
                 constexpr int s_ = decltype(si)::value;
@@ -761,8 +803,8 @@ struct WarpTiles {
                 constexpr int KW1 = (KF::KC1 + 3) / 4;
                 constexpr bool A1 = (KF::KC1 % 4 == 0) && (KF::BOFF1 % 4 == 0);
                 const uint32_t g1 = KF::BOFF1 + c * KF::KC1;
-                const Words<KW1> k1a = lds_span<KF::KC1, A1>(kbase + r * KF::RB + g1);
-                const Words<KW1> k1b = lds_span<KF::KC1, A1>(kbase + (r + 8) * KF::RB + g1);
+                const Words<KW1> k1a = lds_span_off<KF::KC1, A1>(kbase + r * KF::RB, g1);
+                const Words<KW1> k1b = lds_span_off<KF::KC1, A1>(kbase + (r + 8) * KF::RB, g1);
                 const uint32_t base1 = lut_base<KF::B1>(lane_base);
                 static_for<0, KF::KS1>([&](auto si) {
                     constexpr int s_ = decltype(si)::value;
@@ -775,11 +817,9 @@ struct WarpTiles {
             }
         }
 
-        // ---- online softmax over the lane's heads, tokens r and r + 8 ----
+        // ---- scores of the lane's heads, tokens r and r + 8 ----
         const float nk0 = f16_at(knorm + KF::NB * r), nk1 = f16_at(knorm + KF::NB * (r + 8));
-        const float nv0 = f16_at(vnorm + VF::NB * r), nv1 = f16_at(vnorm + VF::NB * (r + 8));
         const bool ok0 = r < nvalid, ok1 = r + 8 < nvalid;
-        float sc[HL][2];  // head e of the lane, token r (0) or r + 8 (1)
         if constexpr (NH == 8 && KG) {
             // chains 0 / 2: group 0 hi / lo; chains 1 / 3: group 1
             const float mk0 = f16_at(knorm + KF::NB * r + 2), mk1 = f16_at(knorm + KF::NB * (r + 8) + 2);
@@ -820,11 +860,18 @@ struct WarpTiles {
             sc[0][0] = ok0 ? (h0 + l0) * nk0 : -INFINITY;
             sc[0][1] = ok1 ? (h1 + l1) * nk1 : -INFINITY;
         }
-        // The reference max only moves when a score exceeds it by more than
-        // 2^kSlack; the shuffles and rescale run only then.
+    }
+
+    // Online-softmax update for the scores of NB blocks. The reference max
+    // only moves when a score exceeds it by more than 2^kSlack; the shuffles
+    // and the rescale of the accumulators run only then.
+    template <int NB>
+    __device__ __forceinline__ void update(const float (&sc)[NB][HL][2]) {
         bool over = false;
 #pragma unroll
-        for (int e = 0; e < HL; ++e) over |= fmaxf(sc[e][0], sc[e][1]) > m_ref[e] + kSlack;
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int e = 0; e < HL; ++e) over |= fmaxf(sc[b][e][0], sc[b][e][1]) > m_ref[e] + kSlack;
         // The trip count is opaque to the compiler (0 or 1 at run time), so the
         // rescale stays a branch instead of predicated straight-line code.
         int rare = __any_sync(kFull, over) ? 1 : 0;
@@ -834,7 +881,9 @@ struct WarpTiles {
             float alpha[HL];
 #pragma unroll
             for (int e = 0; e < HL; ++e) {
-                float mx = fmaxf(sc[e][0], sc[e][1]);
+                float mx = fmaxf(sc[0][e][0], sc[0][e][1]);
+#pragma unroll
+                for (int b = 1; b < NB; ++b) mx = fmaxf(mx, fmaxf(sc[b][e][0], sc[b][e][1]));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
@@ -854,10 +903,18 @@ struct WarpTiles {
             }
             store_acc(o);
         }
-        // P' = p 2^-kSlack n_V (weight x norm stays within fp16); the sums l_run
-        // are kept in the same 2^-kSlack units. m_ref is finite here: the first
-        // tile of an item always takes the branch above (a valid score exceeds
-        // -inf + kSlack), which sets it.
+    }
+
+    // The block's weights after update(): P' = p 2^-kSlack n_V (weight x norm
+    // stays within fp16) as B fragments in bpo (bpo1: with the group-1 norms
+    // when V is group-wise); the sums l_run are kept in the same 2^-kSlack
+    // units. m_ref is finite here: the first block of an item always moves it
+    // (a valid score exceeds -inf + kSlack).
+    __device__ __forceinline__ void block_weights(const float (&sc)[HL][2], uint32_t vnorm, int nvalid, uint32_t psel,
+                                                  int r, int c, uint32_t (&bpo)[2 * HL],
+                                                  uint32_t (&bpo1)[VG ? 2 * HL : 1]) {
+        const bool ok0 = r < nvalid, ok1 = r + 8 < nvalid;
+        const float nv0 = f16_at(vnorm + VF::NB * r), nv1 = f16_at(vnorm + VF::NB * (r + 8));
         const float nv0m = ok0 ? nv0 : 0.0f, nv1m = ok1 ? nv1 : 0.0f;  // padding rows may hold anything
         float p[HL][2];
 #pragma unroll
@@ -867,12 +924,26 @@ struct WarpTiles {
             p[e][1] = ex2(sc[e][1] - mb);
             l_run[e] += p[e][0] + p[e][1];
         }
-        weights(p, nv0m, nv1m, psel, r, c, bp);
+        weights(p, nv0m, nv1m, psel, r, c, bpo);
         if constexpr (VG) {
             const float mv0 = ok0 ? f16_at(vnorm + VF::NB * r + 2) : 0.0f;
             const float mv1 = ok1 ? f16_at(vnorm + VF::NB * (r + 8) + 2) : 0.0f;
-            weights(p, mv0, mv1, psel, r, c, bp1);
+            weights(p, mv0, mv1, psel, r, c, bpo1);
         }
+    }
+
+    // Scores of one 16-token tile (K index rows at kbase, norms at knorm) and
+    // the online-softmax update; leaves the tile's P' (V norms at vnorm) in bp
+    // for values(). Tokens at or past nvalid are padding.
+    __device__ __forceinline__ void scores(uint32_t kbase, uint32_t knorm, uint32_t vnorm, int nvalid,
+                                           uint32_t lane_base, uint32_t psel, int r, int c) {
+        uint32_t qf[8][2 * HL];
+        uint32_t zf[KQ ? 8 : 1][2 * HL];
+        if constexpr (!(KQ && TM)) load_query(qf, zf);
+        float sc[1][HL][2];
+        block_scores(qf, zf, kbase, knorm, nvalid, lane_base, r, c, sc[0]);
+        update<1>(sc);
+        block_weights(sc[0], vnorm, nvalid, psel, r, c, bp, bp1);
     }
 
     // B fragments of P'^T (P' = p n_V for the V norms n0 of token r and n1 of
@@ -919,14 +990,22 @@ struct WarpTiles {
     __device__ __forceinline__ void values(uint32_t vbase, uint32_t lane_base, int r, int c) {
         float o[8][4];
         load_acc(o);
+        values_block(o, vbase, bp, bp1, lane_base, r, c);
+        store_acc(o);
+    }
+
+    // o += V^T P'^T for one 16-token block: V index rows at vbase, P' fragments bpo (bpo1).
+    __device__ __forceinline__ void values_block(float (&o)[8][4], uint32_t vbase, const uint32_t (&bpo)[2 * HL],
+                                                 const uint32_t (&bpo1)[VG ? 2 * HL : 1], uint32_t lane_base, int r,
+                                                 int c) const {
         auto value_step = [&](auto qi, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
             constexpr int q = decltype(qi)::value;
             if constexpr (VG && q >= VF::MT0) {
-                mma16816(o[q], a0, a1, a2, a3, bp1[0], bp1[1]);
-                if constexpr (NH == 8) mma16816(o[q], a0, a1, a2, a3, bp1[2], bp1[3]);
+                mma16816(o[q], a0, a1, a2, a3, bpo1[0], bpo1[1]);
+                if constexpr (NH == 8) mma16816(o[q], a0, a1, a2, a3, bpo1[2], bpo1[3]);
             } else {
-                mma16816(o[q], a0, a1, a2, a3, bp[0], bp[1]);
-                if constexpr (NH == 8) mma16816(o[q], a0, a1, a2, a3, bp[2], bp[3]);
+                mma16816(o[q], a0, a1, a2, a3, bpo[0], bpo[1]);
+                if constexpr (NH == 8) mma16816(o[q], a0, a1, a2, a3, bpo[2], bpo[3]);
             }
         };
 
@@ -936,10 +1015,10 @@ struct WarpTiles {
         {
             constexpr int NW0 = (VF::VC0 + 3) / 4;
             constexpr bool A0 = VF::VC0 % 4 == 0;
-            const Words<NW0> t0 = lds_span<VF::VC0, A0>(r0 + r * VF::VC0);
-            const Words<NW0> t1 = lds_span<VF::VC0, A0>(r1 + r * VF::VC0);
-            const Words<NW0> t8 = lds_span<VF::VC0, A0>(r8 + r * VF::VC0);
-            const Words<NW0> t9 = lds_span<VF::VC0, A0>(r9 + r * VF::VC0);
+            const Words<NW0> t0 = lds_span_off<VF::VC0, A0>(r0, r * VF::VC0);
+            const Words<NW0> t1 = lds_span_off<VF::VC0, A0>(r1, r * VF::VC0);
+            const Words<NW0> t8 = lds_span_off<VF::VC0, A0>(r8, r * VF::VC0);
+            const Words<NW0> t9 = lds_span_off<VF::VC0, A0>(r9, r * VF::VC0);
             uint32_t e01[NW0], o01[NW0], e89[NW0], o89[NW0];
             interleave<VF::B0, NW0>(t0.w, t1.w, e01, o01);
             interleave<VF::B0, NW0>(t8.w, t9.w, e89, o89);
@@ -957,10 +1036,10 @@ struct WarpTiles {
             constexpr int NW1 = (VF::VC1 + 3) / 4;
             constexpr bool A1 = (VF::VC1 % 4 == 0) && (VF::BOFF1 % 4 == 0);
             const uint32_t g1 = VF::BOFF1 + r * VF::VC1;
-            const Words<NW1> t0 = lds_span<VF::VC1, A1>(r0 + g1);
-            const Words<NW1> t1 = lds_span<VF::VC1, A1>(r1 + g1);
-            const Words<NW1> t8 = lds_span<VF::VC1, A1>(r8 + g1);
-            const Words<NW1> t9 = lds_span<VF::VC1, A1>(r9 + g1);
+            const Words<NW1> t0 = lds_span_off<VF::VC1, A1>(r0, g1);
+            const Words<NW1> t1 = lds_span_off<VF::VC1, A1>(r1, g1);
+            const Words<NW1> t8 = lds_span_off<VF::VC1, A1>(r8, g1);
+            const Words<NW1> t9 = lds_span_off<VF::VC1, A1>(r9, g1);
             uint32_t e01[NW1], o01[NW1], e89[NW1], o89[NW1];
             interleave<VF::B1, NW1>(t0.w, t1.w, e01, o01);
             interleave<VF::B1, NW1>(t8.w, t9.w, e89, o89);
@@ -974,6 +1053,39 @@ struct WarpTiles {
                 value_step(std::integral_constant<int, VF::MT0 + q>{}, a0, a1, a2, a3);
             });
         }
+    }
+
+    // Two 16-token blocks as one step (a 32-token block, or two 16-token
+    // blocks of consecutive slots): one load of the query fragments, one
+    // softmax update and one pass over the accumulators.
+    __device__ __forceinline__ void step2(uint32_t kb0, uint32_t kn0, uint32_t vb0, uint32_t vn0, int nv0,
+                                          uint32_t kb1, uint32_t kn1, uint32_t vb1, uint32_t vn1, int nv1,
+                                          uint32_t lane_base, uint32_t psel, int r, int c) {
+        float sc[2][HL][2];
+        if constexpr (KQ || KG || VG) {
+            // these keep more per block: the fragments are reloaded so the two blocks never hold them at once
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                uint32_t qf[8][2 * HL];
+                uint32_t zf[KQ ? 8 : 1][2 * HL];
+                if constexpr (!(KQ && TM)) load_query(qf, zf);
+                block_scores(qf, zf, b ? kb1 : kb0, b ? kn1 : kn0, b ? nv1 : nv0, lane_base, r, c, sc[b]);
+            }
+        } else {
+            uint32_t qf[8][2 * HL];
+            uint32_t zf[KQ ? 8 : 1][2 * HL];
+            load_query(qf, zf);
+            block_scores(qf, zf, kb0, kn0, nv0, lane_base, r, c, sc[0]);
+            block_scores(qf, zf, kb1, kn1, nv1, lane_base, r, c, sc[1]);
+        }
+        update<2>(sc);
+        uint32_t p0[2 * HL], p1[2 * HL], g0[VG ? 2 * HL : 1], g1[VG ? 2 * HL : 1];
+        block_weights(sc[0], vn0, nv0, psel, r, c, p0, g0);
+        block_weights(sc[1], vn1, nv1, psel, r, c, p1, g1);
+        float o[8][4];
+        load_acc(o);
+        values_block(o, vb0, p0, g0, lane_base, r, c);
+        values_block(o, vb1, p1, g1, lane_base, r, c);
         store_acc(o);
     }
 
@@ -1404,9 +1516,12 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
 // ==== paired block kernel: two compute warps per KV head, state in tensor memory =========
 //
 // The same ring of 8-head page-block slots as the block kernel, read by 16
-// compute warps: warp w takes KV head w % 8 of the slots whose sequence number
-// has the parity w / 8 (the ring has an even number of slots, so each slot
-// serves one parity and its waits never skip a phase). Each warp keeps its
+// compute warps: warp w takes KV head w % 8 of the slots in every other run of
+// 32 tokens (two 16-token slots, or one 32-token slot), the runs of parity
+// w / 8. The ring holds a multiple of 4 slots, so each ring position always
+// serves the same eight warps and their waits never skip a phase. A warp
+// handles its 32 tokens as one step: one load of its query fragments, one
+// softmax update and one pass over its accumulators. Each warp keeps its
 // query fragments and value accumulators in its own tensor-memory columns
 // (WarpTiles<..., true>), which leaves room in the register file for twice the
 // warps. At the end of an item the odd warp of each head leaves its state in
@@ -1463,8 +1578,11 @@ __global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(D
     ring.n_low = static_cast<int>((lut_addr - ring.low) / ring.stride);
     ring.high = lut_addr + kLut;
     const int n_high = ring.high < dsm_end ? static_cast<int>((dsm_end - ring.high) / ring.stride) : 0;
-    ring.n = min(ring.n_low + n_high, kBlkMaxSlots) & ~1;  // even
-    if (lut_addr + kLut > dsm_end || ring.n < 2) {
+    // runs of two 16-token slots (or single 32-token slots) alternate between two warps: the ring
+    // holds a whole number of run pairs
+    constexpr int kRunPair = 2 * (2 / TPB);
+    ring.n = min(ring.n_low + n_high, kBlkMaxSlots) / kRunPair * kRunPair;
+    if (lut_addr + kLut > dsm_end || ring.n < kRunPair) {
         if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
         return;
     }
@@ -1504,8 +1622,20 @@ __global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(D
     wt.tm = tmem + quarter + Tiles::kTmCols * (warp >> 2);
     const uint32_t partner_tm = tmem + quarter + Tiles::kTmCols * ((warp + kBlkWarps) >> 2);
     constexpr int kBs = 16 * TPB;
-    uint32_t consumed = 0;
     volatile int* abort_flag = &sm.abort;
+    // Absolute slot a (the a-th slot the producer fills) sits at ring
+    // position a % ring.n with phase (a / ring.n) & 1, tracked incrementally.
+    // Slots are owned in runs of SPG (32 tokens): run a / SPG goes to the warp
+    // of that parity, so each ring position always serves the same warps.
+    constexpr int SPG = 2 / TPB;
+    uint32_t consumed = 0, pos = 0, phase = 0;
+    auto advance = [&](int n) {
+        for (int t = 0; t < n; ++t)
+            if (++pos == static_cast<uint32_t>(ring.n)) {
+                pos = 0;
+                phase ^= 1u;
+            }
+    };
 
     for (int64_t slot = blockIdx.x; slot < total_slots; slot += gridDim.x) {
         Item it;
@@ -1518,35 +1648,64 @@ __global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(D
         wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
         const int ntiles = (it.t1 - it.t0 + 15) >> 4;
         const int nslots = (ntiles + TPB - 1) / TPB;
-        bool bad = false;
-        for (int j = 0; j < nslots; ++j, ++consumed) {
-            if (static_cast<int>(consumed & 1u) != par) continue;
-            if (bad || *abort_flag) {
-                bad = true;
-                continue;
-            }
-            const int s = static_cast<int>(consumed % ring.n);
-            const bool ok = __all_sync(kFull, mbar_wait(smem_addr(&sm.blk.full[s]), (consumed / ring.n) & 1u));
-            if (!ok) {
-                bad = true;
-                if (lane == 0) {
-                    *abort_flag = 1;
-                    if (a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
+        auto nvalid = [&](int k) { return min(16, it.t1 - (it.t0 + 16 * k)); };
+        bool bad = __any_sync(kFull, *abort_flag != 0);  // one value for the whole warp
+        for (int j = 0; j < nslots;) {
+            const uint32_t abs_slot = consumed + j;
+            const bool mine = static_cast<int>((abs_slot / SPG) & 1u) == par;
+            // with 16-token blocks, the two slots of a run are taken together
+            const bool two = TPB == 1 && (abs_slot & 1u) == 0 && j + 1 < nslots;
+            const int span = two ? 2 : 1;
+            if (mine && !bad) {
+                const uint32_t s0 = pos;
+                uint32_t s1 = pos + 1, ph1 = phase;
+                if (s1 == static_cast<uint32_t>(ring.n)) {
+                    s1 = 0;
+                    ph1 ^= 1u;
                 }
-                continue;
+                bool ok = mbar_wait(smem_addr(&sm.blk.full[s0]), phase);
+                if (two && ok) ok = mbar_wait(smem_addr(&sm.blk.full[s1]), ph1);
+                if (!__all_sync(kFull, ok)) {
+                    bad = true;
+                    if (lane == 0) {
+                        *abort_flag = 1;
+                        if (a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
+                    }
+                } else {
+                    const uint32_t kb0 = ring.slot(static_cast<int>(s0)) + k_off;
+                    const uint32_t vb0 = ring.slot(static_cast<int>(s0)) + v_off;
+                    if constexpr (TPB == 1) {
+                        if (two) {
+                            const uint32_t kb1 = ring.slot(static_cast<int>(s1)) + k_off;
+                            const uint32_t vb1 = ring.slot(static_cast<int>(s1)) + v_off;
+                            wt.step2(kb0, kb0 + 16 * KF::RB, vb0, vb0 + 16 * VF::RB, nvalid(j), kb1,
+                                     kb1 + 16 * KF::RB, vb1, vb1 + 16 * VF::RB, nvalid(j + 1), lane_base, psel, r,
+                                     c);
+                        } else {
+                            wt.step(kb0, kb0 + 16 * KF::RB, vb0, vb0 + 16 * VF::RB, nvalid(j), lane_base, psel, r,
+                                    c);
+                        }
+                    } else {
+                        const int k = 2 * j;
+                        if (k + 1 < ntiles)
+                            wt.step2(kb0, kb0 + kBs * KF::RB, vb0, vb0 + kBs * VF::RB, nvalid(k), kb0 + 16 * KF::RB,
+                                     kb0 + kBs * KF::RB + 16 * KF::NB, vb0 + 16 * VF::RB,
+                                     vb0 + kBs * VF::RB + 16 * VF::NB, nvalid(k + 1), lane_base, psel, r, c);
+                        else
+                            wt.step(kb0, kb0 + kBs * KF::RB, vb0, vb0 + kBs * VF::RB, nvalid(k), lane_base, psel, r,
+                                    c);
+                    }
+                    __syncwarp();
+                    if (lane == 0) {  // this warp is done with the slot(s)
+                        mbar_arrive(smem_addr(&sm.blk.empty[s0]));
+                        if (two) mbar_arrive(smem_addr(&sm.blk.empty[s1]));
+                    }
+                }
             }
-            const uint32_t kb = ring.slot(s) + k_off, vb = ring.slot(s) + v_off;
-#pragma unroll
-            for (int t = 0; t < TPB; ++t) {
-                const int k = j * TPB + t;
-                if (TPB == 1 || k < ntiles)
-                    wt.step(kb + 16 * t * KF::RB, kb + kBs * KF::RB + 16 * KF::NB * t, vb + 16 * t * VF::RB,
-                            vb + kBs * VF::RB + 16 * VF::NB * t, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, psel,
-                            r, c);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&sm.blk.empty[s]));  // this warp is done with the slot
+            advance(span);
+            j += span;
         }
+        consumed += static_cast<uint32_t>(nslots);
         // Fold the odd warp's state into the even warp's; both agree on an abort.
         if (par == 1) {
             wt.export_state();
@@ -1946,91 +2105,97 @@ __global__ void __launch_bounds__(kWinWarps * 32) window_kernel(DecodeArgs a, in
     }
 }
 
-// Rotated queries: q_r = pi_K(H(s_K * q) / sqrt(128)) * scale * log2(e), one warp per (b, query head).
-// With QJL keys also qjl_out = sqrt(pi/2)/128 * S q_r, S applied in rotated
-// (not packed) coordinate order, as the residual it projected.
-__global__ void __launch_bounds__(128) rotate_queries_kernel(DevCodec kc, const __nv_bfloat16* q, int num_q_heads,
-                                                              int group, int64_t total, float scale_log2, float* out,
-                                                              float* qjl_out) {
-    const int lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
-    if (row >= total) return;
-    const int hq = static_cast<int>(row % num_q_heads), h = hq / group;
-    const uint2 raw = *reinterpret_cast<const uint2*>(q + row * kHeadDim + 4 * lane);
-    float z[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u), __uint_as_float(raw.y << 16),
-                  __uint_as_float(raw.y & 0xffff0000u)};
+// Rotated queries: q_r = pi_K(H(s_K * q) / sqrt(128)) * scale * log2(e). A CTA
+// of 8 warps takes 8 consecutive (b, query head) rows, one warp per row. With
+// QJL keys it also writes qjl_out = sqrt(pi/2)/128 * S q_r, S applied in
+// rotated (not packed) coordinate order, as the residual it projected: the
+// rows' q_r go to shared memory and thread i computes output i of 4 rows, so
+// the CTA reads S (64 KB, from L2) once for its 8 rows.
+constexpr int kRotRows = 8;
+
+__global__ void __launch_bounds__(kRotRows * 32) rotate_queries_kernel(DevCodec kc, const __nv_bfloat16* q,
+                                                                        int num_q_heads, int group, int64_t total,
+                                                                        float scale_log2, float* out,
+                                                                        float* qjl_out) {
+    __shared__ float zs[kRotRows][kHeadDim];  // q_r of the CTA's rows, rotated order
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRotRows;
+    const int64_t row = row0 + w;
+    if (row < total) {
+        const int hq = static_cast<int>(row % num_q_heads), h = hq / group;
+        const uint2 raw = *reinterpret_cast<const uint2*>(q + row * kHeadDim + 4 * lane);
+        float z[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
+                      __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u)};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) z[i] *= kc.sign[4 * lane + i];
-    {
-        const float p0 = z[0] + z[1], p1 = z[0] - z[1], p2 = z[2] + z[3], p3 = z[2] - z[3];
-        z[0] = p0 + p2;
-        z[2] = p0 - p2;
-        z[1] = p1 + p3;
-        z[3] = p1 - p3;
-    }
+        for (int i = 0; i < 4; ++i) z[i] *= kc.sign[4 * lane + i];
+        {
+            const float p0 = z[0] + z[1], p1 = z[0] - z[1], p2 = z[2] + z[3], p3 = z[2] - z[3];
+            z[0] = p0 + p2;
+            z[2] = p0 - p2;
+            z[1] = p1 + p3;
+            z[3] = p1 - p3;
+        }
 #pragma unroll
-    for (int m = 1; m < 32; m <<= 1)
+        for (int m = 1; m < 32; m <<= 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float p = __shfl_xor_sync(kFull, z[i], m);
+                z[i] = (lane & m) ? (p - z[i]) : (z[i] + p);
+            }
+        const float sc = scale_log2 * 0.08838834764831845f;  // 1/sqrt(128)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float p = __shfl_xor_sync(kFull, z[i], m);
-            z[i] = (lane & m) ? (p - z[i]) : (z[i] + p);
+            z[i] *= sc;
+            out[row * kHeadDim + kc.pos[h * kHeadDim + 4 * lane + i]] = z[i];
+            zs[w][4 * lane + i] = z[i];
         }
-    const float sc = scale_log2 * 0.08838834764831845f;  // 1/sqrt(128)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        z[i] *= sc;
-        out[row * kHeadDim + kc.pos[h * kHeadDim + 4 * lane + i]] = z[i];
     }
-    if (qjl_out != nullptr) {
-        // (S q_r)_i = sum_j S[i][j] q_r[j]; lane: outputs 4 lane .. 4 lane + 3
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (qjl_out == nullptr) return;  // uniform over the CTA
+    __syncthreads();
+    // (S q_r)_i = sum_j S[i][j] q_r[j]: thread (i, half) for rows 4 half .. 4 half + 3
+    const int i = threadIdx.x & (kHeadDim - 1), r0 = (threadIdx.x >> 7) * 4;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 4
-        for (int j0 = 0; j0 < kHeadDim; j0 += 4) {
+    for (int j = 0; j < kHeadDim; ++j) {
+        const float sij = __ldg(kc.qjl_st + j * kHeadDim + i);  // S^T row j, coalesced over i
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const float qj = __shfl_sync(kFull, z[jj], j0 >> 2);
-                const float4 s4 = __ldg(reinterpret_cast<const float4*>(kc.qjl_st + (j0 + jj) * kHeadDim) + lane);
-                acc[0] = fmaf(s4.x, qj, acc[0]);
-                acc[1] = fmaf(s4.y, qj, acc[1]);
-                acc[2] = fmaf(s4.z, qj, acc[2]);
-                acc[3] = fmaf(s4.w, qj, acc[3]);
-            }
-        }
-        constexpr float kappa = 1.2533141373155003f / kHeadDim;  // sqrt(pi/2) / d, the estimator's constant
-        reinterpret_cast<float4*>(qjl_out + row * kHeadDim)[lane] =
-            make_float4(acc[0] * kappa, acc[1] * kappa, acc[2] * kappa, acc[3] * kappa);
+        for (int k = 0; k < 4; ++k) acc[k] = fmaf(sij, zs[r0 + k][j], acc[k]);
     }
+    constexpr float kappa = 1.2533141373155003f / kHeadDim;  // sqrt(pi/2) / d, the estimator's constant
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        if (row0 + r0 + k < total) qjl_out[(row0 + r0 + k) * kHeadDim + i] = acc[k] * kappa;
 }
 
 // Group-wise K: q_r = R_h q * scale * log2(e) in packed order (R_h from the
-// codec: rot_t entry (h, j, p) = R_h[p][j]); one warp per (b, query head),
-// lane: packed positions 4 lane .. 4 lane + 3.
-__global__ void __launch_bounds__(128) rotate_queries_dense_kernel(DevCodec kc, const __nv_bfloat16* q,
-                                                                    int num_q_heads, int group, int64_t total,
-                                                                    float scale_log2, float* out) {
-    const int lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
-    if (row >= total) return;
-    const int hq = static_cast<int>(row % num_q_heads), h = hq / group;
-    const uint2 raw = *reinterpret_cast<const uint2*>(q + row * kHeadDim + 4 * lane);
-    const float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
-                        __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u)};
-    const float4* rt = reinterpret_cast<const float4*>(kc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim);
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 4
-    for (int j0 = 0; j0 < kHeadDim; j0 += 4) {
+// codec: rot_t entry (h, j, p) = R_h[p][j]). One CTA per (b, KV head) takes
+// the head's query rows (group <= 16) together: their q goes to shared
+// memory, thread p computes packed position p of every row, and the CTA reads
+// R_h (64 KB, rows contiguous over p) once.
+__global__ void __launch_bounds__(kHeadDim) rotate_queries_dense_kernel(DevCodec kc, const __nv_bfloat16* q,
+                                                                         int num_q_heads, int group,
+                                                                         float scale_log2, float* out) {
+    __shared__ float qs[16][kHeadDim];
+    const int H = kc.num_heads, p = threadIdx.x;
+    const int h = blockIdx.x % H, b = blockIdx.x / H;
+    const int64_t row0 = static_cast<int64_t>(b) * num_q_heads + static_cast<int64_t>(h) * group;
+    for (int g = 0; g < group; ++g)
+        qs[g][p] = __bfloat162float(q[(row0 + g) * kHeadDim + p]);
+    __syncthreads();
+    const float* rt = kc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim;
+    float acc[16];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const float qj = __shfl_sync(kFull, x[jj], j0 >> 2);
-            const float4 r4 = __ldg(rt + (j0 + jj) * (kHeadDim / 4) + lane);
-            acc[0] = fmaf(r4.x, qj, acc[0]);
-            acc[1] = fmaf(r4.y, qj, acc[1]);
-            acc[2] = fmaf(r4.z, qj, acc[2]);
-            acc[3] = fmaf(r4.w, qj, acc[3]);
-        }
+    for (int g = 0; g < 16; ++g) acc[g] = 0.0f;
+#pragma unroll 2
+    for (int j = 0; j < kHeadDim; ++j) {
+        const float rjp = __ldg(rt + j * kHeadDim + p);
+#pragma unroll
+        for (int g = 0; g < 16; ++g)
+            if (g < group) acc[g] = fmaf(rjp, qs[g][j], acc[g]);
     }
-    reinterpret_cast<float4*>(out + row * kHeadDim)[lane] =
-        make_float4(acc[0] * scale_log2, acc[1] * scale_log2, acc[2] * scale_log2, acc[3] * scale_log2);
+#pragma unroll
+    for (int g = 0; g < 16; ++g)
+        if (g < group) out[(row0 + g) * kHeadDim + p] = acc[g] * scale_log2;
 }
 
 constexpr int kMaxDynSmem = 227 * 1024;
@@ -2075,14 +2240,13 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     if (a.window > 0 && a.batch > 0)
         window_kernel<<<static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.kc.num_heads * head_groups),
                         kWinWarps * 32, 0, s>>>(a, group, head_groups);
-    const unsigned qgrid = static_cast<unsigned>((rows + 3) / 4);
     if constexpr (KF::MODE == kGroupwise)
-        rotate_queries_dense_kernel<<<qgrid, 128, 0, s>>>(a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads,
-                                                          group, rows, a.scale_log2, a.qrot);
+        rotate_queries_dense_kernel<<<static_cast<unsigned>(a.batch) * a.kc.num_heads, kHeadDim, 0, s>>>(
+            a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads, group, a.scale_log2, a.qrot);
     else
-        rotate_queries_kernel<<<qgrid, 128, 0, s>>>(a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads,
-                                                    group, rows, a.scale_log2, a.qrot,
-                                                    KF::MODE == kQjl ? a.qjl_q : nullptr);
+        rotate_queries_kernel<<<static_cast<unsigned>((rows + kRotRows - 1) / kRotRows), kRotRows * 32, 0, s>>>(
+            a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads, group, rows, a.scale_log2, a.qrot,
+            KF::MODE == kQjl ? a.qjl_q : nullptr);
     const int64_t units = static_cast<int64_t>(a.items_per_unit) * a.batch * head_groups *
                           (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);
     const int grid = static_cast<int>(units < sms ? units : sms);
@@ -2092,9 +2256,13 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
             const char* e = std::getenv("TQ_DECODE_PAIR");
             return !(e && e[0] == '0');
         }();
-        if (blk && pair && a.block_size == 16)
+        // The paired kernel wants two run pairs of slots beside the table (one more slot than that
+        // covers the ring's split around the 64 KB-aligned table).
+        const bool pair_fits = static_cast<size_t>(blk_slot_bytes<KF, VF>(a.block_size)) * 5 <=
+                               static_cast<size_t>(kMaxDynSmem) - kLut - 4096;
+        if (blk && pair && pair_fits && a.block_size == 16)
             decode_pair_kernel<KF, VF, NH, 1><<<grid, pair_threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
-        else if (blk && pair && a.block_size == 32)
+        else if (blk && pair && pair_fits && a.block_size == 32)
             decode_pair_kernel<KF, VF, NH, 2><<<grid, pair_threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
         else if (blk && a.block_size == 16)
             decode_blk_kernel<KF, VF, NH, 1><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
@@ -2112,6 +2280,7 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
 template <class F>
 bool same_format(const tq_codec* c) {
     const tq_format_desc& d = c->desc;
+    if (d.qjl && d.groupwise) return false;  // the recipe row runs on the general kernel
     const int mode = d.qjl ? kQjl : (d.groupwise ? kGroupwise : kPlain);
     if (mode != F::MODE) return false;
     if (F::N1 == 0) return d.n_groups == 1 && d.group_bits[0] == F::B0;

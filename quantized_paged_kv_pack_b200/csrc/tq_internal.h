@@ -51,6 +51,10 @@ struct DevCodec {
     const float* qjl_st;    // QJL: S transposed, [128][128] (entry j * 128 + i = S[i][j])
     int32_t groupwise;      // 1: group-wise rotation with per-group norms
     const float* rot_t;     // group-wise: R transposed per head, [H][128][128] (entry (h, j, p) = R_h[p][j])
+    int32_t recipe;         // 1: the recipe row (group-wise and QJL): per group [indices][signs], norms
+                            // (n_g, residual norm_g) per group; qjl_st is then S_0^T then S_1^T (n_g x n_g)
+    int32_t sign_off[2];    // byte offset of each group's QJL sign bits in the index part (QJL: the one
+                            // stream after the index bitstreams)
     const PackCell* cells;  // uniform 4-bit codecs: the pack's quantizer cell table [129]; else null
 };
 

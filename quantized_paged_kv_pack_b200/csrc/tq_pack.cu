@@ -161,6 +161,82 @@ __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8
     __syncwarp();
 }
 
+// The recipe row (group-wise rotation with a QJL stage per group), after the
+// indices: per group the fp16 residual norm |r_g|, the n_g sign bits
+// [(S_g r_g)_i >= 0] (S_g^T rows from the codec, coalesced), then the index
+// part [g0 indices][g0 signs][g1 indices][g1 signs] and the norm part
+// (n_0, |r_0|, n_1, |r_1|). Lane l holds packed positions l + 32k.
+__device__ void pack_recipe_tail(const DevCodec& c, const float (&res)[4], const unsigned short (&n16)[2],
+                                 uint8_t* sub, int64_t offset, int block_size, const uint8_t* idx_buf,
+                                 float* r_buf, int lane) {
+    const int n0 = c.pos0[1];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) r_buf[lane + 32 * k] = res[k];  // packed order (x_buf is no longer read)
+    unsigned short g16[2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        float rr = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int p = lane + 32 * k;
+            if ((p >= n0) == (g == 1)) rr += res[k] * res[k];
+        }
+        g16[g] = __half_as_ushort(__float2half_rn(sqrtf(warp_sum(rr))));
+    }
+    __syncwarp();
+    // (S_g r_g)_i for position p = pos0[g] + i
+    float proj[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int g = 0; g < 2; ++g) {
+        const int n = c.size[g], p0 = c.pos0[g];
+        const float* st = c.qjl_st + (g ? static_cast<int64_t>(n0) * n0 : 0);
+        for (int j = 0; j < n; ++j) {
+            const float r = r_buf[p0 + j];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = lane + 32 * k - p0;
+                if (i >= 0 && i < n) proj[k] = fmaf(__ldg(st + j * n + i), r, proj[k]);
+            }
+        }
+    }
+    uint32_t sw[4];  // sign bit of packed position p at bit p % 32 of sw[p / 32]
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sw[k] = __ballot_sync(kFull, proj[k] >= 0.0f);
+    // index part, 16 bits per lane and round
+    const int half_words = c.index_bytes / 2;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(sub + offset * c.index_bytes);
+    for (int hw = lane; hw < half_words; hw += 32) {
+        unsigned word = 0;
+        for (int i = 0; i < 16; ++i) {
+            const int B = 16 * hw + i;
+            unsigned bit;
+            if (B < 8 * c.sign_off[0]) {  // group 0 indices
+                const int q = B / c.bits[0], r = B - q * c.bits[0];
+                bit = (idx_buf[q] >> r) & 1u;
+            } else if (B < 8 * c.byte_off[1]) {  // group 0 signs
+                const int p = B - 8 * c.sign_off[0];
+                bit = (sw[p >> 5] >> (p & 31)) & 1u;
+            } else if (B < 8 * c.sign_off[1]) {  // group 1 indices
+                const int lb = B - 8 * c.byte_off[1];
+                const int q = lb / c.bits[1], r = lb - q * c.bits[1];
+                bit = (idx_buf[n0 + q] >> r) & 1u;
+            } else {  // group 1 signs
+                const int p = n0 + B - 8 * c.sign_off[1];
+                bit = (sw[p >> 5] >> (p & 31)) & 1u;
+            }
+            word |= bit << i;
+        }
+        dst[hw] = static_cast<uint16_t>(word);
+    }
+    uint16_t* nrm = reinterpret_cast<uint16_t*>(sub + block_size * c.index_bytes + c.norm_bytes * offset);
+    if (lane == 0) {
+        nrm[0] = n16[0];
+        nrm[1] = g16[0];
+        nrm[2] = n16[1];
+        nrm[3] = g16[1];
+    }
+    __syncwarp();
+}
+
 // Group-wise rotation (two groups of original channels, each rotated on its
 // own by the per-head matrix R_h, rows = packed positions): y = R_h x, one fp16
 // norm per group from the exact squares of its channels, u_p = y_p / n_g(p).
@@ -193,6 +269,7 @@ __device__ void pack_vector_groupwise(const DevCodec& c, const float (&x)[4], in
 #pragma unroll
         for (int k = 0; k < 4; ++k) y[k] = fmaf(__ldg(rt + j * kHeadDim + 32 * k), xj, y[k]);
     }
+    float res[4];  // recipe row: residuals u - c[idx] of the lane's positions
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int p = lane + 32 * k;
@@ -202,8 +279,13 @@ __device__ void pack_vector_groupwise(const DevCodec& c, const float (&x)[4], in
         int idx = 0;
         for (int q = 0; q < levels - 1; ++q) idx += (c.bound[g * 16 + q] < u) ? 1 : 0;
         idx_buf[p] = static_cast<uint8_t>(idx);
+        res[k] = u - c.cent[g * 16 + idx];
     }
     __syncwarp();
+    if (c.recipe) {
+        pack_recipe_tail(c, res, n16, sub, offset, block_size, idx_buf, x_buf, lane);
+        return;
+    }
     const int half_words = c.mse_bytes / 2;
     unsigned word = 0;
     if (lane < half_words) {

@@ -154,6 +154,17 @@ def qjl_matrix(head_dim, num_kv_heads, group_bits, group_size, high_coords=None,
     return out
 
 
+def recipe_qjl_matrices(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed=0):
+    """S_0 and S_1 of a recipe-row codec (qjl and groupwise; tq_codec_qjl_matrix), float32
+    [group_size[g]][group_size[g]] each; host only."""
+    d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, True, True)
+    out = np.zeros(head_dim * head_dim, np.float32)
+    _check(lib().tq_codec_qjl_matrix(ctypes.byref(d), out.ctypes.data))
+    del keep
+    n0, n1 = group_size
+    return out[:n0 * n0].reshape(n0, n0), out[n0 * n0:n0 * n0 + n1 * n1].reshape(n1, n1)
+
+
 def group_rotation(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed=0) -> np.ndarray:
     """R_h of a group-wise codec (tq_codec_group_rotation), float32 [H][head_dim][head_dim]; host only."""
     d, keep = _desc(head_dim, num_kv_heads, group_bits, group_size, high_coords, seed, False, True)

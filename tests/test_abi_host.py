@@ -189,8 +189,6 @@ def test_groupwise_row_bytes_ledger_and_validation():
         assert got[key] == getattr(ref, key), key
     with pytest.raises(ValueError):  # group-wise needs two groups
         tq.codec_host_tables(D, H, (3,), (128,), None, 3, groupwise=True)
-    with pytest.raises(ValueError):  # and no QJL stage
-        tq.codec_host_tables(D, H, (4, 2), (32, 96), hc, 3, qjl=True, groupwise=True)
 
 
 
@@ -255,3 +253,31 @@ def test_device_allocation_and_setup_are_per_codec_and_per_device():
     codec = open(os.path.join(csrc, "tq_codec.cpp")).read()
     make = codec[codec.index("tq_status tq_make_codec("):codec.index("void tq_free_codec(")]
     assert "build_pack_cells" in make and "dev.cells" in make  # the pack's cell table rides in that allocation
+
+
+def test_recipe_row_host_tables_matrices_and_ledger():
+    """The recipe row (qjl and groupwise): row bytes, the two S_g bit for bit, and the ledger
+    field by field against the oracle."""
+    H, Hq, W, bs = 4, 16, 32, 16
+    hc = _high(H, 64, 6)
+    for bits, sizes in (((4, 3), (64, 64)), ((4, 2), (32, 96))):
+        hcs = _high(H, sizes[0], 6)
+        t = tq.codec_host_tables(D, H, bits, sizes, hcs, 9, qjl=True, groupwise=True)
+        f = O.Format(D, H, bits, sizes, hcs, 9, qjl=True, groupwise=True)
+        assert t["row_bytes"] == O.row_bytes(f)
+        S0, S1 = tq.recipe_qjl_matrices(D, H, bits, sizes, hcs, 9)
+        assert np.array_equal(S0.astype(np.float64), O.recipe_qjl_matrix(f, 0))
+        assert np.array_equal(S1.astype(np.float64), O.recipe_qjl_matrix(f, 1))
+    assert O.row_bytes(O.Format(D, H, (4, 3), (64, 64), hc, 9, qjl=True, groupwise=True)) == 32 + 8 + 24 + 8 + 8
+    lens = [0, 9, 32, 33, 700]
+    ksp = {"group_bits": (4, 3), "group_size": (64, 64), "seed": 9, "high_coords": hc, "qjl": True,
+           "groupwise": True}
+    vsp = {"group_bits": (4, 3), "group_size": (64, 64), "seed": 2, "high_coords": hc, "groupwise": True}
+    nb = sum(-(-(L - min(W, L)) // bs) for L in lens) + 2
+    got = tq.host_ledger(H, ksp, vsp, lens, W, Hq, bs, nb)
+    ws = tq.decode_workspace_bytes(len(lens), Hq, H, max(lens), bs)
+    kf = O.Format(D, H, (4, 3), (64, 64), hc, 9, qjl=True, groupwise=True)
+    vf = O.Format(D, H, (4, 3), (64, 64), hc, 2, groupwise=True)
+    ref = O.byte_ledger(kf, vf, lens, W, bs, nb, workspace_bytes=ws)
+    for key in ("index_bytes", "norm_bytes", "transform_bytes", "page_pool_bytes", "metadata_bytes"):
+        assert got[key] == getattr(ref, key), key

@@ -144,10 +144,31 @@ def _workload_problem(name, n_seq):
     return w, kc, vc, kf, vf, layout, kp, vp, kw, vw
 
 
+def _checked_sequences(layout, bs, split=4096, n=8):
+    """At least n sequences: the shortest, the median, the longest, and ones whose packed length ends
+    inside a block and inside a split (every split of the benchmark workloads holds 4096 tokens)."""
+    L, P = layout.seq_lens, layout.packed_lens
+    order = np.argsort(L, kind="stable")
+    picks = [int(order[0]), int(order[len(order) // 2]), int(order[-1])]
+    for b in order:
+        if len(picks) >= n:
+            break
+        if P[b] % bs and P[b] % split and int(b) not in picks:
+            picks.append(int(b))
+    for b in order[::-1]:
+        if len(picks) >= n:
+            break
+        if int(b) not in picks:
+            picks.append(int(b))
+    return picks
+
+
 @pytest.mark.parametrize("name", ["decode_llama8b_4bit", "decode_llama70b_3p5bit", "decode_llama8b_2p5bit",
                                   "decode_llama8b_3p5bit_qjl", "decode_llama8b_3p5bit_groupwise"])
-def test_decode_full_size_workloads_sampled(name):
-    """Full-size workloads in the benchmark's launch; the oracle checks sampled outputs."""
+def test_decode_full_size_workloads(name, monkeypatch):
+    """Full-size workloads in the benchmark's launch: every query head of 8 sequences against the
+    oracle (element by element), and, on the three headline-format workloads, every output against
+    the general CUDA-core kernel on the same cache."""
     w, kc, vc, kf, vf, layout, kp, vp, kw, vw = _workload_problem(name, None)
     q = W.queries(w, device="cuda")
     bt = torch.as_tensor(layout.block_tables, device="cuda")
@@ -160,22 +181,29 @@ def test_decode_full_size_workloads_sampled(name):
     assert err.item() == 0
     got = out.cpu().numpy()
     G = w.num_q_heads // w.num_kv_heads
-    order = np.argsort(layout.seq_lens)
-    picks = [int(order[0]), int(order[len(order) // 2]), int(order[-1])]
-    rng = np.random.default_rng(1)
+    picks = _checked_sequences(layout, w.block_size)
+    assert len(picks) >= 8
+    P = layout.packed_lens
+    assert any(P[b] % w.block_size and P[b] % 4096 for b in picks) or not np.any(P % w.block_size)
     for b in picks:
-        for hq in rng.choice(w.num_q_heads, 2, replace=False):
-            h = hq // G
-            L, P = int(layout.seq_lens[b]), int(layout.packed_lens[b])
-            nblk = -(-P // w.block_size)
-            blocks = torch.as_tensor(layout.block_tables[b, :nblk].astype(np.int64), device="cuda")
-            ref = O.decode_attention(q[b:b + 1, hq:hq + 1].float().cpu().numpy().astype(np.float64),
+        L, Pb = int(layout.seq_lens[b]), int(P[b])
+        nblk = -(-Pb // w.block_size)
+        blocks = torch.as_tensor(layout.block_tables[b, :nblk].astype(np.int64), device="cuda")
+        for h in range(w.num_kv_heads):
+            ref = O.decode_attention(q[b:b + 1, h * G:(h + 1) * G].float().cpu().numpy().astype(np.float64),
                                      kp[blocks][:, h:h + 1].cpu().numpy(), vp[blocks][:, h:h + 1].cpu().numpy(),
                                      np.arange(nblk)[None], [L], kw[b:b + 1, h:h + 1].float().cpu().numpy(),
                                      vw[b:b + 1, h:h + 1].float().cpu().numpy(), w.window, 1 / math.sqrt(D),
-                                     slice_format(kf, h), slice_format(vf, h), w.block_size)[0, 0]
-            assert np.abs(got[b, hq] - ref).max() <= ATOL
+                                     slice_format(kf, h), slice_format(vf, h), w.block_size)[0]
+            assert np.abs(got[b, h * G:(h + 1) * G] - ref).max() <= ATOL, (b, h)
             assert np.abs(ref).max() > 0.5
+    if name in ("decode_llama8b_4bit", "decode_llama70b_3p5bit", "decode_llama8b_2p5bit"):
+        monkeypatch.setenv("TQ_DECODE_KERNEL", "general")
+        general = tq.decode_paged(kc, vc, q, kp, vp, w.block_size, bt, sl, maxL, kw, vw, w.window,
+                                  1 / math.sqrt(D), d_err=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        assert (general - out).abs().max().item() <= ATOL
 
 
 def test_tensor_core_and_general_kernels_agree(monkeypatch):

@@ -248,3 +248,38 @@ def test_fast_and_general_pack_kernels_agree(monkeypatch):
             compare_rows(rows_of(pages, s, bs, f, H), x, f, range(H))
         same = (out[0][i] == out[1][i]).mean()
         assert same > 0.999
+
+
+def test_pack_workload_whole_sequence_and_mse_full_size():
+    """The full pack workload in the benchmark's launch (262144 tokens, one call): every row of one
+    whole 8192-token sequence (all 8 KV heads, K and V) against the oracle, and the reconstruction
+    MSE of those GPU rows within 2 % of the oracle's own rows (the uniform 4-bit tensor-core pack)."""
+    w = W.WORKLOADS["pack_llama8b_4bit"]
+    kc, vc, kf, vf = workload_codecs(w)
+    k, v, slots, layout = W.pack_batch(w, device="cuda")
+    kp, vp = tq.page_pool(kc, layout.num_blocks, w.block_size), tq.page_pool(vc, layout.num_blocks, w.block_size)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, w.block_size, d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    seq_len = int(layout.seq_lens[0])
+    b = 5  # a sequence in the middle of the batch
+    pick = np.arange(b * seq_len, (b + 1) * seq_len)
+    s = slots[pick]
+    flips = total = 0
+    for pages, src, f in ((kp, k, kf), (vp, v, vf)):
+        sub = pages[torch.as_tensor(s // w.block_size, device="cuda")].cpu().numpy()
+        rows = np.stack([O.read_rows(sub, np.arange(len(s)), h, s % w.block_size, f, w.block_size)
+                         for h in range(w.num_kv_heads)], axis=1)
+        x = src[torch.as_tensor(pick, device="cuda")].float().cpu().numpy().astype(np.float64)
+        a, c = compare_rows(rows, x, f, range(w.num_kv_heads))
+        flips, total = flips + a, total + c
+        mse_gpu = mse_ref = 0.0
+        for h in range(w.num_kv_heads):
+            f1 = slice_format(f, h)
+            gi, gn = O.decode_rows(rows[:, h], f1)
+            ri, rn, _ = O.quantize(x[:, h], f1, 0)
+            mse_gpu += ((O.dequantize_rows(gi, gn, f1, 0) - x[:, h]) ** 2).sum()
+            mse_ref += ((O.dequantize_rows(ri, rn, f1, 0) - x[:, h]) ** 2).sum()
+        assert abs(mse_gpu / mse_ref - 1) <= 0.02
+    assert flips <= MAX_FLIP_FRACTION * total

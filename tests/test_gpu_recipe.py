@@ -1,0 +1,118 @@
+"""GPU parity of the recipe row as printed (group-wise rotation with a QJL stage per group):
+pack rows and decode against the oracle (through the C ABI)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import tq_oracle as O
+from quantized_paged_kv_pack_b200 import tq
+
+from helpers import D, DecodeProblem, codec_pair, random_kv, slice_format
+
+pytestmark = pytest.mark.gpu
+
+BOUNDARY_REL = 1e-5
+SIGN_REL = 1e-4  # a sign may differ only where |(S_g r_g)_i| is this small against |r_g| sqrt(n_g)
+
+
+def check_recipe_rows(rows, x, fmt, heads):
+    """GPU rows [N][H][row] against the oracle's recipe quantization of x [N][H][d]."""
+    compared = 0
+    for h in heads:
+        f1 = slice_format(fmt, h)
+        idx, n16, u, signs, g16 = O.quantize_qjl(x[:, h], f1, 0)
+        gidx, gn16, gsigns, gg16 = O.decode_rows(rows[:, h], f1)
+        assert np.array_equal(gn16.astype(np.float16).view(np.uint16), n16.astype(np.float16).view(np.uint16))
+        flips = gidx != idx
+        if flips.any():
+            margin = O.boundary_margin(u, f1)
+            assert np.all(margin[flips] <= BOUNDARY_REL), "index mismatch away from a codebook boundary"
+        ok = ~np.any(flips, axis=-1)
+        gd = gg16[ok] != g16[ok]
+        if gd.any():
+            rel = np.abs(gg16[ok][gd] - g16[ok][gd]) / np.maximum(g16[ok][gd], 1e-30)
+            assert np.all(rel < 2e-3), "residual norm differs by more than one fp16 step"
+            assert gd.sum() <= max(2, 0.002 * gd.size)
+        start = 0
+        for g, (b, n) in enumerate(zip(f1.group_bits, f1.group_size)):
+            c, _ = O.codebook(b, n)
+            r = u[:, start:start + n] - c[idx[:, start:start + n]]
+            proj = r @ O.recipe_qjl_matrix(f1, g).T
+            scale = np.linalg.norm(r, axis=-1, keepdims=True) * math.sqrt(n)
+            diff = (gsigns[:, start:start + n] != signs[:, start:start + n]) & ok[:, None]
+            assert np.all(np.abs(proj[diff]) <= SIGN_REL * np.broadcast_to(scale, proj.shape)[diff]), \
+                "QJL sign mismatch away from zero"
+            start += n
+        compared += int(ok.sum())
+    return compared
+
+
+@pytest.mark.parametrize("kfmt", [((4, 3), (64, 64)), ((4, 2), (32, 96)), ((3, 2), (16, 112))])
+@pytest.mark.parametrize("T,H,bs", [(37, 2, 16), (300, 8, 32)])
+def test_recipe_pack_matches_oracle(kfmt, T, H, bs):
+    kc, kf = codec_pair(H, *kfmt, 51, qjl=True, groupwise=True)
+    vc, vf = codec_pair(H, (4, 3), (64, 64), 52, groupwise=True)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(T + 3 * H)
+    k, v = random_kv(T, H, gen)
+    nb = -(-T // bs) + 2
+    slots = np.random.default_rng(T).permutation(nb * bs)[:T].astype(np.int64)
+    kp, vp = tq.page_pool(kc, nb, bs), tq.page_pool(vc, nb, bs)
+    assert kc.row_bytes == O.row_bytes(kf)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, bs, d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    x = k.float().cpu().numpy().astype(np.float64)
+    rows = np.stack([O.read_rows(kp.cpu().numpy(), slots // bs, h, slots % bs, kf, bs) for h in range(H)], 1)
+    assert check_recipe_rows(rows, x, kf, range(H)) > 0.9 * T * H
+
+
+@pytest.mark.parametrize("H,G,bs", [(2, 4, 16), (8, 8, 32)])
+def test_recipe_decode_matches_oracle(H, G, bs):
+    """Recipe-row keys (general kernel) with group-wise values, against the oracle on the same
+    GPU-written pages."""
+    lens = [1, 17, 300, 2100]
+    prob = DecodeProblem(lens, H, G, ((4, 3), (64, 64), 61), ((4, 3), (64, 64), 62), window=8, block_size=bs,
+                         seed=H + G, kqjl=True, kgw=True, vgw=True)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = prob.run(d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = out.cpu().numpy()
+    worst = 0.0
+    for b in range(prob.B):
+        for hq in range(prob.Hq):
+            ref = prob.oracle(b, hq)
+            worst = max(worst, float(np.abs(got[b, hq] - ref).max()))
+            assert np.abs(ref).max() > 0.3
+    assert worst <= 2e-3, worst
+
+
+def test_recipe_window_append_rows_equal_pack():
+    """tq_window_append packs an evicted token through the same routine: the row it writes for the
+    recipe format equals the row tq_pack_kv writes for that token."""
+    H, bs, W = 2, 16, 4
+    kc, kf = codec_pair(H, (4, 3), (64, 64), 71, qjl=True, groupwise=True)
+    vc, vf = codec_pair(H, (4, 3), (64, 64), 72, groupwise=True)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    k, v = random_kv(W + 1, H, gen)
+    # the window holds tokens 0..W-1 (ring slots t % W); appending token W evicts token 0 to packed slot 0
+    kw = k[:W].transpose(0, 1).unsqueeze(0).contiguous()
+    vw = v[:W].transpose(0, 1).unsqueeze(0).contiguous()
+    bt = torch.zeros(1, 2, dtype=torch.int32, device="cuda")
+    bt[0, 0] = 1
+    sl = torch.tensor([W], dtype=torch.int32, device="cuda")
+    kp, vp = tq.page_pool(kc, 3, bs), tq.page_pool(vc, 3, bs)
+    tq.window_append(kc, vc, k[W:W + 1].view(1, H, D), v[W:W + 1].view(1, H, D), kw, vw, W, 0, sl, bt, kp, vp, bs)
+    kq, vq = tq.page_pool(kc, 3, bs), tq.page_pool(vc, 3, bs)
+    tq.pack_kv(kc, vc, k[:1].contiguous(), v[:1].contiguous(), torch.tensor([bs], device="cuda"), kq, vq, bs)
+    torch.cuda.synchronize()
+    for a, b, f in ((kp, kq, kf), (vp, vq, vf)):
+        ra = np.stack([O.read_rows(a.cpu().numpy(), [1], h, [0], f, bs) for h in range(H)])
+        rb = np.stack([O.read_rows(b.cpu().numpy(), [1], h, [0], f, bs) for h in range(H)])
+        assert np.array_equal(ra, rb)
