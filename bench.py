@@ -40,7 +40,7 @@ SMALL = "decode_gqa8_4k_4bit"
 DECODE_LAUNCHES = 6  # per step with a window: append, work list, query rotation, window, partials, combine
 EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl",
          "decode_llama8b_3p5bit_groupwise",
-         "pack_llama8b_4bit"]
+         "pack_llama8b_4bit", "pack_llama70b_3p5bit", "pack_llama8b_2p5bit"]
 D = 128
 METRIC = "paged TQ decode HBM GB/s (algorithmic bytes / step time)"
 

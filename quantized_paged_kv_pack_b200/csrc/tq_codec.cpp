@@ -380,25 +380,50 @@ tq_status build_host_tables(const tq_format_desc* desc, tq_codec* c) {
 }
 
 bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,
-                     int32_t block_size, SplitPlan* plan) {
+                     int32_t block_size, int32_t sms, SplitPlan* plan) {
     if (batch < 0 || num_kv_heads < 1 || num_q_heads < num_kv_heads || num_q_heads % num_kv_heads ||
         max_seq_len < 0 || block_size < 1)
         return false;
     const int G = num_q_heads / num_kv_heads;
     if (G > 16) return false;
-    // Aim for about 4096 packed (sequence, KV head, split) items per call, splits
-    // of 512..4096 tokens (at most 32 tiles of 16 tokens for each of a CTA's 8 warps).
+    // The longest split: about 4096 packed (sequence, KV head, split) items per call, splits of
+    // 512..4096 tokens (at most 32 tiles of 16 tokens for each of a CTA's 8 warps).
     double total = static_cast<double>(std::max(max_seq_len, 1)) * std::max(batch, 1) * num_kv_heads;
     int64_t s = static_cast<int64_t>(std::ceil(total / 4096.0));
     s = std::min<int64_t>(std::max<int64_t>(s, 512), 4096);
     s = (s + 63) / 64 * 64;
     s = (s + block_size - 1) / block_size * block_size;
     if (block_size <= 4096) s = std::min<int64_t>(s, 4096 / block_size * block_size);  // e.g. 4080 for 48
-    // (Shorter splits that balance the grid's CTAs better measured slower on
-    // fixed-length batches: more items, and a CTA runs faster when others have
-    // finished. Variable lengths are balanced by the device work list instead.)
+    // The shortest split the choice below may take (down to 3/4 of the longest); the workspace is
+    // sized for it, so its size does not depend on the device.
+    const int64_t s_lo = std::max<int64_t>(block_size, (s * 3 / 4 + block_size - 1) / block_size * block_size);
+    // Choice: the persistent CTAs (one per SM) deal the items in rounds, so with every sequence
+    // at the longest length the step takes rounds x (split tiles + a per-item overhead of about 3
+    // tiles); take the split count per sequence that minimises that. A batch of equal lengths
+    // whose item count just exceeds a multiple of the SM count gets shorter splits that fill the
+    // last round instead of leaving most CTAs idle in it.
+    const int64_t P = std::max<int64_t>(max_seq_len, 1);
+    const int64_t units = static_cast<int64_t>(std::max(batch, 1)) *
+                          (num_kv_heads % 8 == 0 ? num_kv_heads / 8 : num_kv_heads) * (G > 8 ? G / 8 : 1);
+    if (sms > 0) {
+        double best = -1.0;
+        int64_t best_s = s;
+        for (int64_t n = (P + s - 1) / s; n <= (P + s_lo - 1) / s_lo; ++n) {
+            int64_t cand = (P + n - 1) / n;
+            cand = (cand + block_size - 1) / block_size * block_size;
+            if (cand < s_lo || cand > s) continue;
+            const int64_t items = units * ((P + cand - 1) / cand);
+            const int64_t rounds = (items + sms - 1) / sms;
+            const double cost = static_cast<double>(rounds) * (static_cast<double>((cand + 15) / 16) + 3.0);
+            if (best < 0 || cost < best) {
+                best = cost;
+                best_s = cand;
+            }
+        }
+        s = best_s;
+    }
     plan->split_tokens = static_cast<int32_t>(s);
-    plan->max_splits = static_cast<int32_t>(std::max<int64_t>(1, (max_seq_len + s - 1) / s));
+    plan->max_splits = static_cast<int32_t>(std::max<int64_t>(1, (max_seq_len + s_lo - 1) / s_lo));
     plan->items_per_unit = plan->max_splits + 1;
     plan->group = G;
     plan->record_floats = static_cast<size_t>(G) * (kHeadDim + 2);
@@ -509,9 +534,11 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     const size_t off_s = (n_sign + 2 * n_cent + 2 * n_perm + 15) / 16 * 16;
     const size_t n_s = c->qjl_s.size() * sizeof(float);
     const size_t off_r = (off_s + n_s + 15) / 16 * 16, n_r = c->rot_t.size() * sizeof(float);
-    // uniform 4-bit codecs also carry the tensor-core pack's quantizer cell table
-    const bool u4 = desc->n_groups == 1 && desc->group_bits[0] == 4 && !desc->qjl && !desc->groupwise;
-    const size_t off_c = (off_r + n_r + 15) / 16 * 16, n_c = u4 ? kPackCells * sizeof(PackCell) : 0;
+    // plain codecs (no QJL stage, no group-wise rotation) also carry the tensor-core pack's
+    // quantizer cell table of each group
+    const bool plain = !desc->qjl && !desc->groupwise;
+    const size_t off_c = (off_r + n_r + 15) / 16 * 16;
+    const size_t n_c = plain ? static_cast<size_t>(desc->n_groups) * kPackCells * sizeof(PackCell) : 0;
     const size_t total = off_c + n_c;
     std::vector<char> host(total);
     char* p = host.data();
@@ -536,7 +563,8 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
             for (int j = 0; j < d; ++j) st[static_cast<size_t>(j) * d + i] = c->qjl_s[static_cast<size_t>(i) * d + j];
     }
     if (n_r) std::memcpy(p + off_r, c->rot_t.data(), n_r);
-    if (n_c) build_pack_cells(c->bound[0], 16, reinterpret_cast<PackCell*>(p + off_c));
+    for (int g = 0; n_c && g < desc->n_groups; ++g)
+        build_pack_cells(c->bound[g], 1 << desc->group_bits[g], reinterpret_cast<PackCell*>(p + off_c) + g * kPackCells);
     if (cudaGetDevice(&c->device) != cudaSuccess || cudaMalloc(&c->d_tables, total) != cudaSuccess) {
         cudaGetLastError();
         delete c;
@@ -572,7 +600,7 @@ int32_t tq_codec_row_bytes(const tq_codec* codec) { return codec ? codec->row_by
 size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,
                                  int32_t block_size) {
     SplitPlan plan;
-    if (!make_split_plan(batch, num_q_heads, num_kv_heads, max_seq_len, block_size, &plan)) return 0;
+    if (!make_split_plan(batch, num_q_heads, num_kv_heads, max_seq_len, block_size, 0, &plan)) return 0;
     return plan.workspace_bytes;
 }
 

@@ -424,7 +424,12 @@ tq_status check_decode_args(const tq_codec* kc, const tq_codec* vc, int32_t batc
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
         return fail(TQ_ERR_UNSUPPORTED, "query heads per KV head must be 1, 2, 4, 8 or 16");
     if (vc->desc.qjl) return fail(TQ_ERR_UNSUPPORTED, "decode implements the QJL stage for keys only");
-    if (!make_split_plan(batch, num_q_heads, H, max_seq_len, block_size, plan))
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        sms = 0;
+    }
+    if (!make_split_plan(batch, num_q_heads, H, max_seq_len, block_size, sms, plan))
         return fail(TQ_ERR_VALUE, "invalid decode sizes");
     if (workspace_bytes < plan->workspace_bytes) return fail(TQ_ERR_VALUE, "workspace smaller than tq_decode_workspace_bytes");
     if (batch > 0 && !workspace) return fail(TQ_ERR_VALUE, "null workspace");

@@ -46,6 +46,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
@@ -252,17 +253,26 @@ __device__ __forceinline__ Words<(NB + 3) / 4> lds_span(uint32_t a) {
 // NB bytes at shared address a + off, where a is 4-byte aligned and off is a
 // per-lane constant: the alignment split of off (word offset and shift) does
 // not depend on a, so the compiler computes it once per lane.
-template <int NB, bool ALIGNED>
+// BASE0 + lane * STEP is the per-lane offset for lanes 0..LANES-1 (a
+// compile-time pattern): only as many words are read as the worst of those
+// offsets needs.
+template <int NB, bool ALIGNED, int BASE0 = 0, int STEP = 0, int LANES = 1>
 __device__ __forceinline__ Words<(NB + 3) / 4> lds_span_off(uint32_t a, uint32_t off) {
     if constexpr (ALIGNED) {
         return lds_span<NB, true>(a + off);
     } else {
         constexpr int NW = (NB + 3) / 4;
+        constexpr int MIS = [] {
+            int m = 0;
+            for (int l = 0; l < LANES; ++l) m = ((BASE0 + l * STEP) & 3) > m ? ((BASE0 + l * STEP) & 3) : m;
+            return LANES > 1 ? m : 3;
+        }();
+        constexpr int NR = (MIS + NB + 3) / 4;  // words that hold the span at the worst misalignment
         const uint32_t base = a + (off & ~3u), sh = (off & 3u) * 8;
         Words<NW> r;
         uint32_t raw[NW + 1];
 #pragma unroll
-        for (int i = 0; i <= NW; ++i) raw[i] = lds32(base + 4 * i);
+        for (int i = 0; i <= NW; ++i) raw[i] = i < NR ? lds32(base + 4 * i) : 0u;
 #pragma unroll
         for (int i = 0; i < NW; ++i) r.w[i] = __funnelshift_r(raw[i], raw[i + 1], sh);
         return r;
@@ -788,8 +798,8 @@ struct WarpTiles {
         {
             constexpr int KW0 = (KF::KC0 + 3) / 4;
             constexpr bool A0 = KF::KC0 % 4 == 0;
-            const Words<KW0> k0a = lds_span_off<KF::KC0, A0>(kbase + r * KF::RB, c * KF::KC0);
-            const Words<KW0> k0b = lds_span_off<KF::KC0, A0>(kbase + (r + 8) * KF::RB, c * KF::KC0);
+            const Words<KW0> k0a = lds_span_off<KF::KC0, A0, 0, KF::KC0, 4>(kbase + r * KF::RB, c * KF::KC0);
+            const Words<KW0> k0b = lds_span_off<KF::KC0, A0, 0, KF::KC0, 4>(kbase + (r + 8) * KF::RB, c * KF::KC0);
             const uint32_t base0 = lut_base<KF::B0>(lane_base);
             static_for<0, KF::KS0>([&](auto si) {
                 constexpr int s_ = decltype(si)::value;
@@ -803,8 +813,8 @@ struct WarpTiles {
                 constexpr int KW1 = (KF::KC1 + 3) / 4;
                 constexpr bool A1 = (KF::KC1 % 4 == 0) && (KF::BOFF1 % 4 == 0);
                 const uint32_t g1 = KF::BOFF1 + c * KF::KC1;
-                const Words<KW1> k1a = lds_span_off<KF::KC1, A1>(kbase + r * KF::RB, g1);
-                const Words<KW1> k1b = lds_span_off<KF::KC1, A1>(kbase + (r + 8) * KF::RB, g1);
+                const Words<KW1> k1a = lds_span_off<KF::KC1, A1, KF::BOFF1, KF::KC1, 4>(kbase + r * KF::RB, g1);
+                const Words<KW1> k1b = lds_span_off<KF::KC1, A1, KF::BOFF1, KF::KC1, 4>(kbase + (r + 8) * KF::RB, g1);
                 const uint32_t base1 = lut_base<KF::B1>(lane_base);
                 static_for<0, KF::KS1>([&](auto si) {
                     constexpr int s_ = decltype(si)::value;
@@ -1015,10 +1025,10 @@ struct WarpTiles {
         {
             constexpr int NW0 = (VF::VC0 + 3) / 4;
             constexpr bool A0 = VF::VC0 % 4 == 0;
-            const Words<NW0> t0 = lds_span_off<VF::VC0, A0>(r0, r * VF::VC0);
-            const Words<NW0> t1 = lds_span_off<VF::VC0, A0>(r1, r * VF::VC0);
-            const Words<NW0> t8 = lds_span_off<VF::VC0, A0>(r8, r * VF::VC0);
-            const Words<NW0> t9 = lds_span_off<VF::VC0, A0>(r9, r * VF::VC0);
+            const Words<NW0> t0 = lds_span_off<VF::VC0, A0, 0, VF::VC0, 8>(r0, r * VF::VC0);
+            const Words<NW0> t1 = lds_span_off<VF::VC0, A0, 0, VF::VC0, 8>(r1, r * VF::VC0);
+            const Words<NW0> t8 = lds_span_off<VF::VC0, A0, 0, VF::VC0, 8>(r8, r * VF::VC0);
+            const Words<NW0> t9 = lds_span_off<VF::VC0, A0, 0, VF::VC0, 8>(r9, r * VF::VC0);
             uint32_t e01[NW0], o01[NW0], e89[NW0], o89[NW0];
             interleave<VF::B0, NW0>(t0.w, t1.w, e01, o01);
             interleave<VF::B0, NW0>(t8.w, t9.w, e89, o89);
@@ -1036,10 +1046,10 @@ struct WarpTiles {
             constexpr int NW1 = (VF::VC1 + 3) / 4;
             constexpr bool A1 = (VF::VC1 % 4 == 0) && (VF::BOFF1 % 4 == 0);
             const uint32_t g1 = VF::BOFF1 + r * VF::VC1;
-            const Words<NW1> t0 = lds_span_off<VF::VC1, A1>(r0, g1);
-            const Words<NW1> t1 = lds_span_off<VF::VC1, A1>(r1, g1);
-            const Words<NW1> t8 = lds_span_off<VF::VC1, A1>(r8, g1);
-            const Words<NW1> t9 = lds_span_off<VF::VC1, A1>(r9, g1);
+            const Words<NW1> t0 = lds_span_off<VF::VC1, A1, VF::BOFF1, VF::VC1, 8>(r0, g1);
+            const Words<NW1> t1 = lds_span_off<VF::VC1, A1, VF::BOFF1, VF::VC1, 8>(r1, g1);
+            const Words<NW1> t8 = lds_span_off<VF::VC1, A1, VF::BOFF1, VF::VC1, 8>(r8, g1);
+            const Words<NW1> t9 = lds_span_off<VF::VC1, A1, VF::BOFF1, VF::VC1, 8>(r9, g1);
             uint32_t e01[NW1], o01[NW1], e89[NW1], o89[NW1];
             interleave<VF::B1, NW1>(t0.w, t1.w, e01, o01);
             interleave<VF::B1, NW1>(t8.w, t9.w, e89, o89);
@@ -1530,8 +1540,19 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
 // two warps of a head agree on it through a reduction barrier, so neither
 // waits for the other alone.
 
-constexpr int kPairWarps = 2 * kBlkWarps;  // compute warps
+constexpr int kPairWarps = 2 * kBlkWarps;  // compute warps (warpgroups 0-3)
+constexpr int kPairThreads = (kPairWarps + 4) * 32;  // + warpgroup 4: the producer warp and three idle
 constexpr uint32_t kTmemCols = 512;        // 4 warps per lane quarter x 128 columns
+// Registers per thread: the launch gives every thread kPairLaunchRegs (the
+// compiler's figure for 640 threads, 5 warps per SM sub-partition); then the
+// producer warpgroup gives back down to kPairProducerRegs and the compute
+// warpgroups take kPairComputeRegs. The block holds 640 x 96 = 61440
+// registers; 512 x 112 + 128 x 32 = 61440 fit in them, and each SM
+// sub-partition (4 compute warps and one of warpgroup 4) needs 15360 of its
+// 16384.
+constexpr int kPairLaunchRegs = 96, kPairProducerRegs = 32, kPairComputeRegs = 112;
+static_assert(kPairWarps * 32 * kPairComputeRegs + 128 * kPairProducerRegs <= kPairThreads * kPairLaunchRegs,
+              "register split above the launch allocation");
 
 struct PairSmem {
     BlkSmem blk;    // ring barriers and the producer's block ids, as in the block kernel
@@ -1556,7 +1577,7 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
 // The block kernel's producer, reused: its slot sequence does not depend on
 // which warps read a slot, only on the release count (8) of every slot.
 template <class KF, class VF, int NH, int TPB>
-__global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(DecodeArgs a, LutValues tv,
+__global__ void __launch_bounds__(kPairThreads, 1) decode_pair_kernel(DecodeArgs a, LutValues tv,
                                                                                int group, int head_groups,
                                                                                int64_t total_slots) {
     static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
@@ -1586,7 +1607,7 @@ __global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(D
         if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
         return;
     }
-    fill_table(reinterpret_cast<uint32_t*>(dsm + (lut_addr - dsm_addr)), tv, threadIdx.x, (kPairWarps + 1) * 32);
+    fill_table(reinterpret_cast<uint32_t*>(dsm + (lut_addr - dsm_addr)), tv, threadIdx.x, kPairThreads);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kBlkMaxSlots; ++s) {
             mbar_init_count(smem_addr(&sm.blk.full[s]), 1);
@@ -1604,10 +1625,12 @@ __global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(D
     tm_fence_before_sync();
     __syncthreads();
     tm_fence_after_sync();
-    if (warp == kPairWarps) {
-        produce_blk<KF, VF>(a, sm.blk, ring, head_groups, total_slots, lane);
+    if (warp >= kPairWarps) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairProducerRegs));
+        if (warp == kPairWarps) produce_blk<KF, VF>(a, sm.blk, ring, head_groups, total_slots, lane);
         return;
     }
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPairComputeRegs));
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&sm.tmem);
     uint32_t lane_base;
     asm volatile("or.b32 %0, %1, %2;" : "=r"(lane_base) : "r"(lut_addr), "r"(static_cast<uint32_t>(lane) << 2));
@@ -1628,14 +1651,8 @@ __global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(D
     // Slots are owned in runs of SPG (32 tokens): run a / SPG goes to the warp
     // of that parity, so each ring position always serves the same warps.
     constexpr int SPG = 2 / TPB;
-    uint32_t consumed = 0, pos = 0, phase = 0;
-    auto advance = [&](int n) {
-        for (int t = 0; t < n; ++t)
-            if (++pos == static_cast<uint32_t>(ring.n)) {
-                pos = 0;
-                phase ^= 1u;
-            }
-    };
+    const uint32_t ring_n = static_cast<uint32_t>(ring.n);
+    uint32_t consumed = 0, pos_c = 0, phase_c = 0;  // absolute slot, ring position and phase of the item start
 
     for (int64_t slot = blockIdx.x; slot < total_slots; slot += gridDim.x) {
         Item it;
@@ -1648,22 +1665,32 @@ __global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(D
         wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
         const int ntiles = (it.t1 - it.t0 + 15) >> 4;
         const int nslots = (ntiles + TPB - 1) / TPB;
-        auto nvalid = [&](int k) { return min(16, it.t1 - (it.t0 + 16 * k)); };
+        const int tok_end = it.t1 - it.t0;
         bool bad = __any_sync(kFull, *abort_flag != 0);  // one value for the whole warp
-        for (int j = 0; j < nslots;) {
-            const uint32_t abs_slot = consumed + j;
-            const bool mine = static_cast<int>((abs_slot / SPG) & 1u) == par;
-            // with 16-token blocks, the two slots of a run are taken together
-            const bool two = TPB == 1 && (abs_slot & 1u) == 0 && j + 1 < nslots;
+        // This warp's first slot of the item: the item's first slot when its run is ours, else the
+        // first slot of the next run. Runs of this warp then follow every 2 SPG slots.
+        int j = 0;
+        {
+            const uint32_t run0 = consumed / SPG, off0 = consumed % SPG;
+            if (static_cast<int>(run0 & 1u) != par) j = SPG - static_cast<int>(off0);
+        }
+        uint32_t pos = pos_c + static_cast<uint32_t>(j), phase = phase_c;
+        if (pos >= ring_n) {
+            pos -= ring_n;
+            phase ^= 1u;
+        }
+        while (j < nslots) {
+            // with 16-token blocks the two slots of a run are taken together (the first run of an item
+            // may start on its second slot, and the last may be cut short by the item's end)
+            const bool two = TPB == 1 && ((consumed + static_cast<uint32_t>(j)) & 1u) == 0 && j + 1 < nslots;
             const int span = two ? 2 : 1;
-            if (mine && !bad) {
-                const uint32_t s0 = pos;
+            if (!bad) {
                 uint32_t s1 = pos + 1, ph1 = phase;
-                if (s1 == static_cast<uint32_t>(ring.n)) {
+                if (s1 == ring_n) {
                     s1 = 0;
                     ph1 ^= 1u;
                 }
-                bool ok = mbar_wait(smem_addr(&sm.blk.full[s0]), phase);
+                bool ok = mbar_wait(smem_addr(&sm.blk.full[pos]), phase);
                 if (two && ok) ok = mbar_wait(smem_addr(&sm.blk.full[s1]), ph1);
                 if (!__all_sync(kFull, ok)) {
                     bad = true;
@@ -1672,38 +1699,49 @@ __global__ void __launch_bounds__((kPairWarps + 1) * 32, 1) decode_pair_kernel(D
                         if (a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
                     }
                 } else {
-                    const uint32_t kb0 = ring.slot(static_cast<int>(s0)) + k_off;
-                    const uint32_t vb0 = ring.slot(static_cast<int>(s0)) + v_off;
+                    const uint32_t sb0 = ring.slot(static_cast<int>(pos));
+                    const uint32_t kb0 = sb0 + k_off, vb0 = sb0 + v_off;
+                    const int tok0 = (TPB * j) * 16;  // first token of the step within the item
                     if constexpr (TPB == 1) {
                         if (two) {
-                            const uint32_t kb1 = ring.slot(static_cast<int>(s1)) + k_off;
-                            const uint32_t vb1 = ring.slot(static_cast<int>(s1)) + v_off;
-                            wt.step2(kb0, kb0 + 16 * KF::RB, vb0, vb0 + 16 * VF::RB, nvalid(j), kb1,
-                                     kb1 + 16 * KF::RB, vb1, vb1 + 16 * VF::RB, nvalid(j + 1), lane_base, psel, r,
-                                     c);
+                            const uint32_t sb1 = ring.slot(static_cast<int>(s1));
+                            const uint32_t kb1 = sb1 + k_off, vb1 = sb1 + v_off;
+                            wt.step2(kb0, kb0 + 16 * KF::RB, vb0, vb0 + 16 * VF::RB, min(16, tok_end - tok0), kb1,
+                                     kb1 + 16 * KF::RB, vb1, vb1 + 16 * VF::RB, min(16, tok_end - tok0 - 16),
+                                     lane_base, psel, r, c);
                         } else {
-                            wt.step(kb0, kb0 + 16 * KF::RB, vb0, vb0 + 16 * VF::RB, nvalid(j), lane_base, psel, r,
-                                    c);
+                            wt.step(kb0, kb0 + 16 * KF::RB, vb0, vb0 + 16 * VF::RB, min(16, tok_end - tok0),
+                                    lane_base, psel, r, c);
                         }
                     } else {
-                        const int k = 2 * j;
-                        if (k + 1 < ntiles)
-                            wt.step2(kb0, kb0 + kBs * KF::RB, vb0, vb0 + kBs * VF::RB, nvalid(k), kb0 + 16 * KF::RB,
+                        if (tok0 + 16 < tok_end)
+                            wt.step2(kb0, kb0 + kBs * KF::RB, vb0, vb0 + kBs * VF::RB, 16, kb0 + 16 * KF::RB,
                                      kb0 + kBs * KF::RB + 16 * KF::NB, vb0 + 16 * VF::RB,
-                                     vb0 + kBs * VF::RB + 16 * VF::NB, nvalid(k + 1), lane_base, psel, r, c);
+                                     vb0 + kBs * VF::RB + 16 * VF::NB, min(16, tok_end - tok0 - 16), lane_base, psel,
+                                     r, c);
                         else
-                            wt.step(kb0, kb0 + kBs * KF::RB, vb0, vb0 + kBs * VF::RB, nvalid(k), lane_base, psel, r,
-                                    c);
+                            wt.step(kb0, kb0 + kBs * KF::RB, vb0, vb0 + kBs * VF::RB, min(16, tok_end - tok0),
+                                    lane_base, psel, r, c);
                     }
                     __syncwarp();
                     if (lane == 0) {  // this warp is done with the slot(s)
-                        mbar_arrive(smem_addr(&sm.blk.empty[s0]));
+                        mbar_arrive(smem_addr(&sm.blk.empty[pos]));
                         if (two) mbar_arrive(smem_addr(&sm.blk.empty[s1]));
                     }
                 }
             }
-            advance(span);
-            j += span;
+            // to this warp's next run: past this run and the partner's run of SPG slots
+            j += span + SPG;
+            pos += static_cast<uint32_t>(span + SPG);
+            if (pos >= ring_n) {
+                pos -= ring_n;
+                phase ^= 1u;
+            }
+        }
+        {
+            const uint32_t np = pos_c + static_cast<uint32_t>(nslots);
+            phase_c ^= (np / ring_n) & 1u;
+            pos_c = np % ring_n;
         }
         consumed += static_cast<uint32_t>(nslots);
         // Fold the odd warp's state into the even warp's; both agree on an abort.
@@ -2211,7 +2249,16 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
                          static_cast<size_t>(kMaxDynSmem) - kLut - 4096;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
+    // The paired kernel's register split assumes the compiler gave it kPairLaunchRegs per thread;
+    // with any other figure the compute warps' request could not be met, so that kernel is not used.
+    static std::atomic<int> pair_regs_ok{0};
     const cudaError_t attr_err = once_per_device(dev, [] {
+        cudaFuncAttributes fa1{}, fa2{};
+        const bool ok = cudaFuncGetAttributes(&fa1, decode_pair_kernel<KF, VF, NH, 1>) == cudaSuccess &&
+                        cudaFuncGetAttributes(&fa2, decode_pair_kernel<KF, VF, NH, 2>) == cudaSuccess &&
+                        fa1.numRegs == kPairLaunchRegs && fa2.numRegs == kPairLaunchRegs;
+        pair_regs_ok.store(ok ? 1 : 0);
+        cudaGetLastError();
         cudaError_t attr_err;
         attr_err = cudaFuncSetAttribute(decode_mma_kernel<KF, VF, NH, NW>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(head_bytes));
@@ -2251,11 +2298,12 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
                           (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);
     const int grid = static_cast<int>(units < sms ? units : sms);
     if (grid > 0) {
-        const dim3 threads((kBlkWarps + 1) * 32), pair_threads((kPairWarps + 1) * 32);
-        static const bool pair = [] {
+        const dim3 threads((kBlkWarps + 1) * 32), pair_threads(kPairThreads);
+        static const bool pair_env = [] {
             const char* e = std::getenv("TQ_DECODE_PAIR");
             return !(e && e[0] == '0');
         }();
+        const bool pair = pair_env && pair_regs_ok.load() == 1;
         // The paired kernel wants two run pairs of slots beside the table (one more slot than that
         // covers the ring's split around the 64 KB-aligned table).
         const bool pair_fits = static_cast<size_t>(blk_slot_bytes<KF, VF>(a.block_size)) * 5 <=

@@ -16,12 +16,14 @@ constexpr int kHeadDim = 128;   // the only head_dim the kernels implement
 constexpr int kMaxHeads = 1024;
 constexpr int kMaxLevels = 16;  // 4-bit codebooks at most on the GPU path
 
-// Quantizer cell table of a uniform 4-bit codec, used by the tensor-core
-// pack: a rotated unit coordinate u, scaled to v = 64 u, falls into cell
-// round(v) + 64 of 129 cells over [-64, 64]; a cell holds the number of
-// decision boundaries strictly below it and the one boundary inside it (in
-// units of v; +inf when none). The codec builds it on the host and copies it
-// to the device with its other tables.
+// Quantizer cell table of one codebook, used by the tensor-core packs: a
+// rotated unit coordinate u, scaled to v = 64 u, falls into cell round(v) + 64
+// of 129 cells over [-64, 64]; a cell holds the number of decision boundaries
+// strictly below it and the one boundary inside it (in units of v; +inf when
+// none). At head_dim 128 adjacent boundaries of the 2-, 3- and 4-bit
+// codebooks are more than one unit of v apart, so no cell holds two. A plain
+// codec builds one per group on the host and copies them to the device with
+// its other tables.
 constexpr int kPackCells = 129;
 constexpr float kPackCellScale = 64.0f;
 struct PackCell {
@@ -55,7 +57,8 @@ struct DevCodec {
                             // (n_g, residual norm_g) per group; qjl_st is then S_0^T then S_1^T (n_g x n_g)
     int32_t sign_off[2];    // byte offset of each group's QJL sign bits in the index part (QJL: the one
                             // stream after the index bitstreams)
-    const PackCell* cells;  // uniform 4-bit codecs: the pack's quantizer cell table [129]; else null
+    const PackCell* cells;  // plain codecs: the pack's quantizer cell table of each group [n_groups][129];
+                            // else null
 };
 
 // Arguments of the decode kernels (device pointers; see tq_decode_paged).
@@ -152,8 +155,11 @@ struct SplitPlan {
     size_t list_offset;     // byte offset of the work list (and then its count) in the workspace
     size_t workspace_bytes;
 };
+// sms: the device's SM count (the grid of the persistent decode kernels), used to choose the
+// split length; 0 keeps the longest split. The workspace layout (max_splits, items_per_unit and
+// the sizes) is the same for every sms.
 bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,
-                     int32_t block_size, SplitPlan* plan);
+                     int32_t block_size, int32_t sms, SplitPlan* plan);
 
 // Uniform 4-bit pack on the tensor cores; TQ_ERR_UNSUPPORTED (nothing
 // launched) for other formats or unaligned pools.

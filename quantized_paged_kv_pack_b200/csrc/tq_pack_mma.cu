@@ -98,10 +98,23 @@ __device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
     return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     uint2 v;
     asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
     return v;
+}
+
+template <int B, int E, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (B < E) {
+        f(std::integral_constant<int, B>{});
+        static_for<B + 1, E>(f);
+    }
 }
 
 template <int I = 0, class F>
@@ -376,14 +389,368 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_u4_kernel(DevCodec kc, DevCo
     }
 }
 
+// ==== tensor-core pack for plain formats of 2-, 3- and 4-bit groups ==============
+//
+// The rotation and the norm are the uniform 4-bit kernel's. The quantizer
+// uses the cell table of the coordinate's group (the tables of the 2-, 3- and
+// 4-bit codebooks, 16 copies each: lanes l and l + 16 share a copy, and an
+// 8-byte load serves the half-warps apart, so the lookups are free of bank
+// conflicts). A group is a set of packed positions: rotated coordinate j sits
+// at packed position pos_h[j] (group 0 first). Each lane keeps its indices in
+// registers until the unit's input buffer is no longer read, writes them as
+// bytes at their packed positions into that buffer (rows padded to 132 bytes
+// so the lanes of one coordinate in 8 rows hit 8 banks), then each lane packs
+// eight positions at a time into b bytes of the row, LSB-first. The format
+// is a template parameter (bit widths, group sizes and byte offsets are
+// constants) and a launch packs the tokens of one codec, K or V.
+
+constexpr int kStagePitch = 132;
+
+struct PackTcSmem {
+    QuantCell cells[3][kCells][16];  // codebooks of 2, 3, 4 bits (index bits - 2), 16 copies
+    uint32_t bfrag[1][8][2][32][2];  // [codec][a][n-tile][lane][reg]: B operands (+-1 bf16 pairs)
+    uint8_t rows[kPW][16][72];       // staged index rows of a warp's 16 tokens (pitch 72: 16 rows, 16 bank pairs)
+    unsigned short norms[kPW][16];
+    int slot32[kPW][16];             // the unit's slots: -1 padding, capacity when past the pool
+    uint8_t xbuf[kPW][2][16][kRowPad];  // double-buffered input rows (bf16); the current one then stages indices
+};
+static_assert(16 * kStagePitch <= 16 * kRowPad, "index staging fits in an input buffer");
+
+// The 8 indices (bytes) x0..x7 of lo = [x0 x1 x2 x3], hi = [x4 x5 x6 x7], b bits each, LSB-first.
+template <int B>
+__device__ __forceinline__ uint32_t pack8(uint32_t lo, uint32_t hi) {
+    if constexpr (B == 4) {
+        const uint32_t x = lo | (lo >> 4), y = hi | (hi >> 4);  // bytes 0, 2: two nibbles each
+        return __byte_perm(x, y, 0x6420);
+    } else if constexpr (B == 2) {
+        const uint32_t x = lo | (lo >> 6), y = hi | (hi >> 6);  // bytes 0, 2: two 2-bit fields each
+        const uint32_t x2 = (x & 0xFu) | ((x >> 12) & 0xF0u), y2 = (y & 0xFu) | ((y >> 12) & 0xF0u);
+        return x2 | (y2 << 8);
+    } else {
+        const uint32_t x = lo | (lo >> 5), y = hi | (hi >> 5);  // bytes 0, 2: two 3-bit fields each
+        const uint32_t x2 = (x & 0x3Fu) | ((x >> 10) & 0xFC0u), y2 = (y & 0x3Fu) | ((y >> 10) & 0xFC0u);
+        return x2 | (y2 << 12);
+    }
+}
+
+template <int B0_, int N0_, int B1_, int N1_>
+struct PackFmt {
+    static constexpr int B0 = B0_, N0 = N0_, B1 = B1_, N1 = N1_;
+    static constexpr int NG = N1 > 0 ? 2 : 1;
+    static constexpr int IB = (B0 * N0 + B1 * N1) / 8;  // index bytes of a row
+    static constexpr int BOFF1 = B0 * N0 / 8;           // byte offset of group 1
+    static_assert(N0 + N1 == kHeadDim && IB % 8 == 0 && IB <= 64, "whole 8-byte index rows of head_dim 128");
+};
+using PU4 = PackFmt<4, 128, 0, 0>;
+using PU3 = PackFmt<3, 128, 0, 0>;
+using PM43 = PackFmt<4, 64, 3, 64>;
+using PM42 = PackFmt<4, 32, 2, 96>;
+
+template <class F>
+__global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const __nv_bfloat16* __restrict__ src,
+                                                          const int64_t* __restrict__ slots, int num_tokens,
+                                                          uint8_t* __restrict__ pages, int capacity, int block_size,
+                                                          int bs_log2, int* __restrict__ d_err) {
+    extern __shared__ __align__(16) uint8_t psm_raw[];
+    PackTcSmem& sm = *reinterpret_cast<PackTcSmem*>(psm_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, c = lane & 3;
+
+    // Cell tables of the format's groups.
+    for (int g = 0; g < F::NG; ++g) {
+        const int bi = (g ? F::B1 : F::B0) - 2;
+        for (int i = threadIdx.x; i < kCells * 16; i += kPW * 32)
+            sm.cells[bi][i >> 4][i & 15] = cd.cells[g * kCells + (i >> 4)];
+    }
+    for (int i = threadIdx.x; i < 8 * 2 * 32; i += kPW * 32) {
+        const int ln = i & 31, t = (i >> 5) & 1, a = (i >> 6) & 7;
+        const int rr = ln >> 2, cc = ln & 3;
+        const int bp = 8 * t + rr;
+        uint32_t regs[2];
+        for (int q = 0; q < 2; ++q) {
+            unsigned short hh[2];
+            for (int e = 0; e < 2; ++e) {
+                const int b = 2 * cc + 8 * q + e;
+                const float val = cd.sign[16 * a + b] * ((__popc(bp & b) & 1) ? -1.0f : 1.0f);
+                hh[e] = val > 0 ? 0x3F80 : 0xBF80;
+            }
+            regs[q] = static_cast<uint32_t>(hh[0]) | (static_cast<uint32_t>(hh[1]) << 16);
+        }
+        sm.bfrag[0][a][t][ln][0] = regs[0];
+        sm.bfrag[0][a][t][ln][1] = regs[1];
+    }
+    __syncthreads();
+
+    const int H = cd.num_heads;
+    const int units = (num_tokens + 15) / 16 * H;  // (16-token group, KV head)
+    // cell e of table bi for this lane: cells_lane + (bi * kCells + e) * 128
+    const uint32_t cells_lane = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.cells[0][0][lane & 15]));
+    const uint32_t xbuf0 = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.xbuf[warp][0][0][0]));
+    auto issue = [&](int uu, int buf) {
+        const int tg_ = uu / H, h_ = uu - tg_ * H;
+        const __nv_bfloat16* src_ = src;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int piece = lane + 32 * i, tok = piece >> 4, part = piece & 15;
+            const int t = tg_ * 16 + tok;
+            const bool live = t < num_tokens;
+            const __nv_bfloat16* g = src_ + (static_cast<int64_t>(live ? t : 0) * H + h_) * kHeadDim + 8 * part;
+            cp_async16(xbuf0 + (buf * 16 + tok) * kRowPad + 16 * part, g, live ? 16u : 0u);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    const int stride = gridDim.x * kPW;
+    int u = blockIdx.x * kPW + warp;
+    if (u < units) issue(u, 0);
+    for (int it = 0; u < units; u += stride, ++it) {
+        const int cur = it & 1;
+        const int tg = u / H, h = u - tg * H;
+        const int t0 = tg * 16;
+        constexpr int n0 = F::N0, ng = F::NG;
+
+        if (lane < 16) {
+            int64_t sl = -1;
+            if (t0 + lane < num_tokens) sl = __ldg(slots + t0 + lane);
+            sm.slot32[warp][lane] = sl < 0 ? -1 : (sl >= capacity ? capacity : static_cast<int>(sl));
+        }
+
+        if (u + stride < units) {
+            issue(u + stride, cur ^ 1);
+        } else {
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncwarp();
+
+        const uint32_t frag_row = xbuf0 + (cur * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)) * kRowPad +
+                                  ((lane >> 4) & 1) * 16;
+        const uint32_t stage = xbuf0 + cur * 16 * kRowPad;  // [16][kStagePitch] index bytes, packed order
+        float n_tok[2];
+        unsigned short n16[2];
+        // the lane's indices: idxr[t][a] bytes (j, token r), (j + 1, token r), (j, token r + 8), (j + 1, token r + 8)
+        uint32_t idxr[2][8];
+        const int16_t* posh = cd.pos + h * kHeadDim;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            uint2 xa[8], xb[8];
+#pragma unroll
+            for (int a = 0; a < 8; ++a) ldsm_x4(frag_row + 32 * a, xa[a].x, xb[a].x, xa[a].y, xb[a].y);
+            if (t == 0) {
+                float ss_lo, ss_hi;
+                {
+                    uint64_t acc_lo = 0, acc_hi = 0;
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) {
+                        const uint64_t l01 = bf16x2_to_f32x2(xa[a].x), l23 = bf16x2_to_f32x2(xa[a].y);
+                        const uint64_t h01 = bf16x2_to_f32x2(xb[a].x), h23 = bf16x2_to_f32x2(xb[a].y);
+                        acc_lo = fma2(l01, l01, fma2(l23, l23, acc_lo));
+                        acc_hi = fma2(h01, h01, fma2(h23, h23, acc_hi));
+                    }
+                    float p, q;
+                    upk(acc_lo, p, q);
+                    ss_lo = p + q;
+                    upk(acc_hi, p, q);
+                    ss_hi = p + q;
+                }
+                ss_lo += __shfl_xor_sync(kFull, ss_lo, 1);
+                ss_lo += __shfl_xor_sync(kFull, ss_lo, 2);
+                ss_hi += __shfl_xor_sync(kFull, ss_hi, 1);
+                ss_hi += __shfl_xor_sync(kFull, ss_hi, 2);
+                bool risky[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float ss = i ? ss_hi : ss_lo;
+                    const float n32 = sqrtf(ss);
+                    bool rk = !(ss > 1e-30f && ss < 1e30f) || n32 > 60000.0f;
+                    const __half hh = __float2half_rn(n32);
+                    const unsigned short hb = __half_as_ushort(hh);
+                    if (!rk) {
+                        const float hf = __half2float(hh);
+                        const float up = __half2float(__ushort_as_half(static_cast<unsigned short>(hb + 1)));
+                        const float dn = __half2float(__ushort_as_half(static_cast<unsigned short>(hb - 1)));
+                        const float tol = 1e-6f * n32;
+                        rk = fabsf(n32 - 0.5f * (hf + up)) <= tol || fabsf(n32 - 0.5f * (hf + dn)) <= tol;
+                    }
+                    risky[i] = rk;
+                    n_tok[i] = n32;
+                    n16[i] = hb;
+                }
+                if (__any_sync(kFull, risky[0] || risky[1])) {
+                    double d_lo = 0.0, d_hi = 0.0;
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) {
+                        const double l0 = __uint_as_float(xa[a].x << 16), l1 = __uint_as_float(xa[a].x & 0xffff0000u);
+                        const double l2 = __uint_as_float(xa[a].y << 16), l3 = __uint_as_float(xa[a].y & 0xffff0000u);
+                        const double h0 = __uint_as_float(xb[a].x << 16), h1 = __uint_as_float(xb[a].x & 0xffff0000u);
+                        const double h2 = __uint_as_float(xb[a].y << 16), h3 = __uint_as_float(xb[a].y & 0xffff0000u);
+                        d_lo += l0 * l0 + l1 * l1 + l2 * l2 + l3 * l3;
+                        d_hi += h0 * h0 + h1 * h1 + h2 * h2 + h3 * h3;
+                    }
+                    d_lo = warp4_sum_d(d_lo);
+                    d_hi = warp4_sum_d(d_hi);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        if (risky[i]) {
+                            const double nd = sqrt(i ? d_hi : d_lo);
+                            n16[i] = __half_as_ushort(__double2half(nd));
+                            n_tok[i] = static_cast<float>(nd);
+                        }
+                    }
+                }
+            }
+            uint64_t kq2[2];  // v = z * 64 / (sqrt(128) n) per token
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float kq = n_tok[i] > 0.0f ? kCellScale / (n_tok[i] * 11.313708498984761f) : 0.0f;
+                if (!(kq < 3.0e38f)) kq = 0.0f;  // norms too small to scale: the zero vector
+                kq2[i] = pk(kq, kq);
+            }
+            uint64_t zq[8][2];  // [a][token]: rotated coordinates 16 a + 8 t + 2 c + {0, 1}
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const uint2 bf = *reinterpret_cast<const uint2*>(&sm.bfrag[0][a][t][lane][0]);
+                float zc[4];
+                mma_bf16(zc, xa[a].x, xb[a].x, xa[a].y, xb[a].y, bf.x, bf.y);
+                zq[a][0] = pk(zc[0], zc[1]);
+                zq[a][1] = pk(zc[2], zc[3]);
+            }
+#pragma unroll
+            for (int m = 1; m < 8; m <<= 1)
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+                    if (!(a & m))
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const uint64_t x0 = zq[a][i], x1 = zq[a | m][i];
+                            zq[a][i] = add2(x0, x1);
+                            zq[a | m][i] = sub2(x0, x1);
+                        }
+            // Quantize with the cell table of each coordinate's group.
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const int j = 16 * a + 8 * t + 2 * c;
+                uint32_t pp = static_cast<uint32_t>(j) | (static_cast<uint32_t>(j + 1) << 16);
+                if (ng == 2) pp = __ldg(reinterpret_cast<const unsigned int*>(posh + j));  // positions of j, j + 1
+                // address of cell round(v) + 64 = bits(v + 1.5 * 2^23) - 0x4B400000 + 64
+                constexpr uint32_t kTab0 = static_cast<uint32_t>((F::B0 - 2) * kCells) * 128u + 64u * 128u -
+                                           0x4B400000u * 128u;
+                constexpr uint32_t kTab1 = static_cast<uint32_t>(((F::NG == 2 ? F::B1 : F::B0) - 2) * kCells) * 128u +
+                                           64u * 128u - 0x4B400000u * 128u;
+                uint32_t tab[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int pe = static_cast<int>((pp >> (16 * e)) & 0xffffu);
+                    tab[e] = cells_lane + ((ng == 2 && pe >= n0) ? kTab1 : kTab0);
+                }
+                uint32_t w = 0;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint64_t vv = mul2(zq[a][i], kq2[i]);
+                    const uint64_t mm = add2(vv, pk(12582912.0f, 12582912.0f));
+                    float v0, v1, m0, m1;
+                    upk(vv, v0, v1);
+                    upk(mm, m0, m1);
+                    const uint2 e0 = lds64(__float_as_uint(m0) * 128u + tab[0]);
+                    const uint2 e1 = lds64(__float_as_uint(m1) * 128u + tab[1]);
+                    const uint32_t i0 = e0.y + (v0 > __uint_as_float(e0.x) ? 1u : 0u);
+                    const uint32_t i1 = e1.y + (v1 > __uint_as_float(e1.x) ? 1u : 0u);
+                    w |= (i0 | (i1 << 8)) << (16 * i);
+                }
+                idxr[t][a] = w;
+            }
+        }
+        __syncwarp();  // every lane has read its fragments: the input buffer now stages the indices
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const int j = 16 * a + 8 * t + 2 * c;
+                uint32_t pp = static_cast<uint32_t>(j) | (static_cast<uint32_t>(j + 1) << 16);
+                if (ng == 2) pp = __ldg(reinterpret_cast<const unsigned int*>(posh + j));
+                const uint32_t w = idxr[t][a];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint32_t row = stage + static_cast<uint32_t>((r + 8 * i) * kStagePitch);
+                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(row + (pp & 0xffffu)), "r"((w >> (16 * i)) & 0xffu)
+                                 : "memory");
+                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(row + (pp >> 16)), "r"((w >> (16 * i + 8)) & 0xffu)
+                                 : "memory");
+                }
+            }
+        if (c == 0) {
+            sm.norms[warp][r] = n16[0];
+            sm.norms[warp][r + 8] = n16[1];
+        }
+        __syncwarp();
+
+        // Pack: in round k lanes 0-15 take packed positions 16 k .. 16 k + 7 of token lane and lanes
+        // 16-31 positions 16 k + 8 .. 16 k + 15 of token lane - 16 (one group for the whole warp,
+        // since groups start on multiples of 16), into b bytes of the row, LSB-first.
+        {
+            const int tok = lane & 15, hi8 = (lane >> 4) * 8;
+            const uint32_t srow = stage + static_cast<uint32_t>(tok * kStagePitch);
+            uint8_t* drow = &sm.rows[warp][tok][0];
+            static_for<0, 8>([&](auto kc) {
+                constexpr int K = decltype(kc)::value;
+                constexpr bool G1 = F::NG == 2 && 16 * K >= F::N0;
+                constexpr int B = G1 ? F::B1 : F::B0;
+                const int p = 16 * K + hi8;
+                const uint32_t lo = lds32(srow + p), hi = lds32(srow + p + 4);
+                uint8_t* dst = drow + (G1 ? F::BOFF1 + (p - F::N0) * B / 8 : p * B / 8);
+                if constexpr (B == 4) {
+                    *reinterpret_cast<uint32_t*>(dst) = pack8<4>(lo, hi);
+                } else if constexpr (B == 2) {
+                    *reinterpret_cast<unsigned short*>(dst) = static_cast<unsigned short>(pack8<2>(lo, hi));
+                } else {
+                    const uint32_t w = pack8<3>(lo, hi);
+                    dst[0] = static_cast<uint8_t>(w);
+                    dst[1] = static_cast<uint8_t>(w >> 8);
+                    dst[2] = static_cast<uint8_t>(w >> 16);
+                }
+            });
+        }
+        __syncwarp();
+
+        // Write the rows in 8-byte pieces (index rows are whole multiples of 8 bytes), and the norms.
+        constexpr int ib = F::IB, rb = F::IB + 2;
+        const int pieces = ib / 8;
+        for (int q = lane; q < 16 * pieces; q += 32) {
+            const int row = q / pieces, part = q - row * pieces;
+            const int slot = sm.slot32[warp][row];
+            if (slot >= 0 && slot < capacity) {
+                const int blk = bs_log2 >= 0 ? slot >> bs_log2 : slot / block_size;
+                const int off = slot - blk * block_size;
+                uint8_t* sub = pages + (static_cast<int64_t>(blk) * H + h) * block_size * rb;
+                *reinterpret_cast<uint2*>(sub + off * ib + 8 * part) =
+                    *reinterpret_cast<const uint2*>(&sm.rows[warp][row][8 * part]);
+                if (part == 0)
+                    *reinterpret_cast<unsigned short*>(sub + block_size * ib + 2 * off) = sm.norms[warp][row];
+            } else if (slot >= capacity && part == 0 && d_err) {
+                atomicOr(d_err, TQ_DERR_SLOT);
+            }
+        }
+        __syncwarp();
+    }
+}
+
 }  // namespace
 
-// Launches the uniform 4-bit fast path; TQ_ERR_UNSUPPORTED when it does not apply.
+// Launches a tensor-core pack (uniform 4-bit, or another plain format); TQ_ERR_UNSUPPORTED when none applies.
 tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
                          const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
                          int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream) {
-    for (const tq_codec* c : {kc, vc})
-        if (c->desc.n_groups != 1 || c->desc.group_bits[0] != 4 || c->desc.qjl) return TQ_ERR_UNSUPPORTED;
+    // Uniform 4-bit K and V: the 4-bit kernel. Other plain formats (no QJL stage, no group-wise
+    // rotation) with 2-, 3- and 4-bit groups and whole 8-byte index rows: the general tensor-core kernel.
+    bool u4 = true, plain = true;
+    for (const tq_codec* c : {kc, vc}) {
+        const tq_format_desc& d = c->desc;
+        if (d.n_groups != 1 || d.group_bits[0] != 4 || d.qjl || d.groupwise) u4 = false;
+        const bool inst = (d.n_groups == 1 && (d.group_bits[0] == 4 || d.group_bits[0] == 3)) ||
+                          (d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 64 && d.group_bits[1] == 3) ||
+                          (d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 32 && d.group_bits[1] == 2);
+        if (d.qjl || d.groupwise || !inst || !c->dev.cells) plain = false;
+    }
+    if (!u4 && !plain) return TQ_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 15) return TQ_ERR_UNSUPPORTED;
     if (block_size % 8 != 0) return TQ_ERR_UNSUPPORTED;  // 16-byte aligned rows and norm arrays
     // 32-bit index arithmetic in the kernel: slots, tokens and work units must fit.
@@ -394,22 +761,49 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
     // The quantizer cell table comes with the K codec (every uniform 4-bit
     // codebook is the same). The kernel's shared-memory size is set once per
     // device.
-    if (!kc->dev.cells) return TQ_ERR_UNSUPPORTED;
+    if (!kc->dev.cells || !vc->dev.cells) return TQ_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
     const cudaError_t err = once_per_device(dev, [] {
-        return cudaFuncSetAttribute(pack_u4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(sizeof(PackSmem)));
+        cudaError_t e = cudaFuncSetAttribute(pack_u4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(sizeof(PackSmem)));
+        for (auto kern : {pack_tc_kernel<PU4>, pack_tc_kernel<PU3>, pack_tc_kernel<PM43>, pack_tc_kernel<PM42>})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(PackTcSmem)));
+        return e;
     });
     if (err != cudaSuccess) return fail(TQ_ERR_CUDA, "pack fast path setup failed");
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t want = (n_units + kPW - 1) / kPW;
     const int grid = static_cast<int>(want < sms ? want : sms);
-    pack_u4_kernel<<<grid, kPW * 32, sizeof(PackSmem), static_cast<cudaStream_t>(stream)>>>(
-        kc->dev, vc->dev, kc->dev.cells, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-        slot_mapping, static_cast<int>(num_tokens), static_cast<uint8_t*>(k_pages), static_cast<uint8_t*>(v_pages),
-        static_cast<int>(capacity), block_size, bs_log2, d_err);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (u4) {
+        pack_u4_kernel<<<grid, kPW * 32, sizeof(PackSmem), st>>>(
+            kc->dev, vc->dev, kc->dev.cells, static_cast<const __nv_bfloat16*>(k),
+            static_cast<const __nv_bfloat16*>(v), slot_mapping, static_cast<int>(num_tokens),
+            static_cast<uint8_t*>(k_pages), static_cast<uint8_t*>(v_pages), static_cast<int>(capacity), block_size,
+            bs_log2, d_err);
+        return TQ_OK;
+    }
+    // One launch per codec; the grid covers that codec's units (half of the pair's).
+    const int64_t want1 = ((num_tokens + 15) / 16 * kc->desc.num_kv_heads + kPW - 1) / kPW;
+    const int grid1 = static_cast<int>(want1 < sms ? want1 : sms);
+    const struct { const tq_codec* c; const void* x; void* pages; } sides[2] = {{kc, k, k_pages}, {vc, v, v_pages}};
+    for (const auto& sd : sides) {
+        const tq_format_desc& d = sd.c->desc;
+        auto go = [&](auto kernel) {
+            kernel<<<grid1, kPW * 32, sizeof(PackTcSmem), st>>>(sd.c->dev, static_cast<const __nv_bfloat16*>(sd.x),
+                                                              slot_mapping, static_cast<int>(num_tokens),
+                                                              static_cast<uint8_t*>(sd.pages),
+                                                              static_cast<int>(capacity), block_size, bs_log2, d_err);
+        };
+        if (d.n_groups == 1 && d.group_bits[0] == 4) go(pack_tc_kernel<PU4>);
+        else if (d.n_groups == 1 && d.group_bits[0] == 3) go(pack_tc_kernel<PU3>);
+        else if (d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 64 && d.group_bits[1] == 3) go(pack_tc_kernel<PM43>);
+        else go(pack_tc_kernel<PM42>);
+    }
     return TQ_OK;
 }
 

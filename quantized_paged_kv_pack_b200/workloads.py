@@ -83,6 +83,18 @@ WORKLOADS = {
         (4,), (128,), (4,), (128,), 0, 1, 8, True, "fixed:8192",
         description="pack 32 sequences x 8192 tokens, 8 KV heads (Llama-3.1-8B KV shapes), "
                     "block 16, shuffled slot mapping, uniform 4-bit K and V"),
+    "pack_llama70b_3p5bit": Workload(
+        "pack_llama70b_3p5bit", "pack", 1008, 32, 64, 8, 128, 16, 0,
+        (4, 3), (64, 64), (4, 3), (64, 64), 0, 1, 8, True, "fixed:8192",
+        description="pack 32 sequences x 8192 tokens, 8 KV heads (the Llama-3.1-70B decode shapes), "
+                    "block 16, shuffled slot mapping, K and V 3.5-bit (64 channels at 4 bits + 64 at 3 "
+                    "bits, independent tables)"),
+    "pack_llama8b_2p5bit": Workload(
+        "pack_llama8b_2p5bit", "pack", 1009, 32, 32, 8, 128, 32, 0,
+        (4, 2), (32, 96), (3,), (128,), 0, 1, 8, True, "fixed:8192",
+        description="pack 32 sequences x 8192 tokens, 8 KV heads, block 32, shuffled slot mapping, "
+                    "K 2.5-bit (32 channels at 4 bits + 96 at 2 bits), V uniform 3-bit (the formats of "
+                    "the batch-256 decode workload)"),
     "decode_llama8b_4bit": Workload(
         "decode_llama8b_4bit", "decode", 1003, 64, 32, 8, 128, 16, 64,
         (4,), (128,), (4,), (128,), 0, 1, 8, True, "uniform:1024:32768",

@@ -224,10 +224,16 @@ def test_pack_edge_values_uniform_4bit_fast_path():
     assert np.array_equal(vp.cpu().numpy(), rv)
 
 
-def test_fast_and_general_pack_kernels_agree(monkeypatch):
-    H, T, bs = 4, 700, 16
-    kc, kf = codec_pair(H, (4,), (128,), 8)
-    vc, vf = codec_pair(H, (4,), (128,), 9)
+@pytest.mark.parametrize("kspec,vspec,bs", [(((4,), (128,)), ((4,), (128,)), 16),
+                                             (((4, 3), (64, 64)), ((4, 3), (64, 64)), 16),
+                                             (((4, 2), (32, 96)), ((3,), (128,)), 32),
+                                             (((2,), (128,)), ((4, 3), (64, 64)), 48)])
+def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs):
+    """The tensor-core packs (uniform 4-bit, and the plain 2/3/4-bit mixes) against the general
+    kernel and the oracle on the same tokens."""
+    H, T = 4, 700
+    kc, kf = codec_pair(H, *kspec, 8)
+    vc, vf = codec_pair(H, *vspec, 9)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(5)
     k, v = random_kv(T, H, gen)
