@@ -304,6 +304,8 @@ __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, c
                                                                    int32_t max_splits, int32_t items_per_unit,
                                                                    int32_t G, const float* ws, float* out) {
     __shared__ float y[kHeadDim];
+    // Launched as a dependent of the partials: the split records are read only after they are complete.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int hq = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
     const int H = vc.num_heads, h = hq / G, g = hq - h * G;
     int L = seq_lens[b];
@@ -369,6 +371,9 @@ __global__ void __launch_bounds__(kHeadDim * kGwHeads) decode_combine_gw_kernel(
     const float* rt = vc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim;
     for (int e = threadIdx.x; e < kHeadDim * kHeadDim; e += nthreads)
         rts[(e >> 7) * kGwPitch + (e & (kHeadDim - 1))] = rt[e];
+    // Launched as a dependent of the partials: R_h^T is staged while they end; the split records are
+    // read only after they are complete.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     int L = seq_lens[b];
     L = L < 0 ? 0 : (L > max_seq_len ? max_seq_len : L);
     const int n_win = min(window, L), P = L - n_win;
@@ -552,20 +557,23 @@ extern "C" tq_status tq_decode_combine(const tq_codec* vc, const int32_t* seq_le
     if (vc->desc.groupwise) {
         int dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
-        const cudaError_t e = once_per_device(dev, [] {
+        cudaError_t e = once_per_device(dev, [] {
             return cudaFuncSetAttribute(decode_combine_gw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         static_cast<int>(kGwCombineSmem));
         });
         if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "cannot reserve shared memory for the combine kernel");
         const int threads = kHeadDim * std::min(plan.group, kGwHeads);
-        decode_combine_gw_kernel<<<static_cast<unsigned>(batch) * vc->desc.num_kv_heads, threads, kGwCombineSmem,
-                                   s>>>(vc->dev, seq_lens, num_q_heads, max_seq_len, window, plan.split_tokens,
-                                        plan.max_splits, plan.items_per_unit, plan.group,
-                                        static_cast<const float*>(workspace), out);
+        e = launch_dependent(decode_combine_gw_kernel, dim3(static_cast<unsigned>(batch) * vc->desc.num_kv_heads),
+                             dim3(threads), kGwCombineSmem, s, vc->dev, seq_lens, num_q_heads, max_seq_len, window,
+                             plan.split_tokens, plan.max_splits, plan.items_per_unit, plan.group,
+                             static_cast<const float*>(workspace), out);
+        if (e != cudaSuccess) return fail(TQ_ERR_CUDA, std::string("combine launch: ") + cudaGetErrorString(e));
     } else {
-        decode_combine_kernel<<<dim3(num_q_heads, batch), kHeadDim, 0, s>>>(
-            vc->dev, seq_lens, num_q_heads, max_seq_len, window, plan.split_tokens, plan.max_splits,
-            plan.items_per_unit, plan.group, static_cast<const float*>(workspace), out);
+        const cudaError_t e = launch_dependent(
+            decode_combine_kernel, dim3(num_q_heads, batch), dim3(kHeadDim), 0, s, vc->dev, seq_lens, num_q_heads,
+            max_seq_len, window, plan.split_tokens, plan.max_splits, plan.items_per_unit, plan.group,
+            static_cast<const float*>(workspace), out);
+        if (e != cudaSuccess) return fail(TQ_ERR_CUDA, std::string("combine launch: ") + cudaGetErrorString(e));
     }
     return finish(s, nullptr, "decode combine");
 }

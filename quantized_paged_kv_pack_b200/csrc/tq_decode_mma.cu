@@ -439,6 +439,16 @@ __device__ __forceinline__ void tm_dep(uint32_t* v) {
 
 // ---- work items -----------------------------------------------------------------
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream still runs;
+// griddep_wait() returns once that kernel has completed and its writes are
+// visible, so nothing it writes is read before. griddep_launch_dependents()
+// lets the next such kernel start.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 struct Item {
     int b, h, hg, split, t0, t1;  // h: the KV head (per-head items) or the first of 8 (block items)
     bool win;
@@ -1183,14 +1193,15 @@ struct WarpTiles {
 // t_first, t_first + t_step, ... < it.t1, on CUDA cores (lane: 4 coordinates).
 // Writes (max, sum, accumulator) per query head g < rows: m[g * ml_stride],
 // l[g * ml_stride], acc[g * acc_stride + coordinate] (acc 8-byte aligned).
+template <int NH>
 __device__ __forceinline__ void window_state(const DecodeArgs& a, const Item& it, int h, int head0, int rows,
                                              int t_first, int t_step, int lane, float* m_out, float* l_out,
                                              float* acc_out, int ml_stride, int acc_stride) {
     const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
     const int H = a.kc.num_heads;
-    float qv[8][4], m[8], l[8], acc[8][4];
+    float qv[NH][4], m[NH], l[NH], acc[NH][4];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
+    for (int g = 0; g < NH; ++g) {
         m[g] = -INFINITY;
         l[g] = 0.0f;
 #pragma unroll
@@ -1238,7 +1249,7 @@ __device__ __forceinline__ void window_state(const DecodeArgs& a, const Item& it
             vx[u][3] = __uint_as_float(vr.y & 0xffff0000u);
         }
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
+        for (int g = 0; g < NH; ++g) {
             if (g < rows) {
                 float p[4];
 #pragma unroll
@@ -1277,7 +1288,7 @@ __device__ __forceinline__ void window_state(const DecodeArgs& a, const Item& it
         }
     }
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
+    for (int g = 0; g < NH; ++g) {
         if (g < rows) {
             if (lane == 0) {
                 m_out[g * ml_stride] = m[g];
@@ -1419,7 +1430,6 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
     static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
     extern __shared__ __align__(128) uint8_t dsm[];
     BlkSmem& sm = *reinterpret_cast<BlkSmem*>(dsm);
-    total_slots = listed_slots<kBlkWarps>(a, head_groups, total_slots);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, c = lane & 3;
     const int bs = a.block_size;
@@ -1437,6 +1447,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
     const int n_high = ring.high < dsm_end ? static_cast<int>((dsm_end - ring.high) / ring.stride) : 0;
     ring.n = min(ring.n_low + n_high, kBlkMaxSlots);
     if (lut_addr + kLut > dsm_end || ring.n < 2) {
+        griddep_wait();
         if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
         return;
     }
@@ -1449,6 +1460,11 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
+    // The table and barriers above overlap the prologue's end; its work list and queries are read
+    // from here on.
+    griddep_wait();
+    griddep_launch_dependents();
+    total_slots = listed_slots<kBlkWarps>(a, head_groups, total_slots);
     if (warp == kBlkWarps) {
         produce_blk<KF, VF>(a, sm, ring, head_groups, total_slots, lane);
         return;
@@ -1469,7 +1485,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
         const int h = it.h + warp;                    // this warp's KV head
         const int head0 = h * group + it.hg * 8;      // its first query head of the item
         float* rec = record_of(a, it.b, h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
-        if (it.win) continue;  // windows are not listed: window_kernel takes them
+        if (it.win) continue;  // windows are not listed: the prologue's window CTAs take them
         const int64_t q_off = (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim;
         wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
         bool timed_out = false;
@@ -1584,7 +1600,6 @@ __global__ void __launch_bounds__(kPairThreads, 1) decode_pair_kernel(DecodeArgs
     static_assert(TPB == 1 || TPB == 2, "16- or 32-token blocks");
     extern __shared__ __align__(128) uint8_t dsm[];
     PairSmem& sm = *reinterpret_cast<PairSmem*>(dsm);
-    total_slots = listed_slots<kBlkWarps>(a, head_groups, total_slots);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, c = lane & 3;
     const int bs = a.block_size;
@@ -1604,6 +1619,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) decode_pair_kernel(DecodeArgs
     constexpr int kRunPair = 2 * (2 / TPB);
     ring.n = min(ring.n_low + n_high, kBlkMaxSlots) / kRunPair * kRunPair;
     if (lut_addr + kLut > dsm_end || ring.n < kRunPair) {
+        griddep_wait();
         if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
         return;
     }
@@ -1625,6 +1641,11 @@ __global__ void __launch_bounds__(kPairThreads, 1) decode_pair_kernel(DecodeArgs
     tm_fence_before_sync();
     __syncthreads();
     tm_fence_after_sync();
+    // The table, barriers and tensor memory above overlap the prologue's end; its work list and
+    // queries are read from here on.
+    griddep_wait();
+    griddep_launch_dependents();
+    total_slots = listed_slots<kBlkWarps>(a, head_groups, total_slots);
     if (warp >= kPairWarps) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairProducerRegs));
         if (warp == kPairWarps) produce_blk<KF, VF>(a, sm.blk, ring, head_groups, total_slots, lane);
@@ -1657,7 +1678,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) decode_pair_kernel(DecodeArgs
     for (int64_t slot = blockIdx.x; slot < total_slots; slot += gridDim.x) {
         Item it;
         if (!item_of<kBlkWarps>(a, slot, head_groups, total_slots, it)) continue;
-        if (it.win) continue;  // windows are not listed: window_kernel takes them
+        if (it.win) continue;  // windows are not listed: the prologue's window CTAs take them
         const int h = it.h + hw;                      // this warp's KV head
         const int head0 = h * group + it.hg * 8;      // its first query head of the item
         float* rec = record_of(a, it.b, h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
@@ -1910,7 +1931,6 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
     static_assert(NH == 4 || NH == 8, "4 or 8 query heads per item");
     extern __shared__ __align__(128) uint8_t dsm[];
     Smem<NW>& sm = *reinterpret_cast<Smem<NW>*>(dsm);
-    total_slots = listed_slots<1>(a, head_groups, total_slots);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, c = lane & 3;
     constexpr uint32_t kStageBytes = stage_bytes<KF, VF>();
@@ -1920,6 +1940,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
         (dsm_addr + static_cast<uint32_t>(smem_head_bytes<NW>()) + (kLut - 1)) & ~uint32_t(kLut - 1);
     const uint32_t ring_addr = lut_addr + kLut;
     if (ring_addr + NW * kStages * kStageBytes > dsm_addr + smem_bytes<NW, kStageBytes>()) {
+        griddep_wait();
         if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_LAUNCH);
         return;
     }
@@ -1934,6 +1955,11 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
+    // The table and barriers above overlap the prologue's end; its work list and queries are read
+    // from here on.
+    griddep_wait();
+    griddep_launch_dependents();
+    total_slots = listed_slots<1>(a, head_groups, total_slots);
     if (warp == NW) {
         produce_head<KF, VF, NW>(a, sm, ring_addr, head_groups, total_slots, lane);
         return;
@@ -1951,7 +1977,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
         Item it;
         if (!item_of<1>(a, slot, head_groups, total_slots, it)) continue;
         const int head0 = it.h * group + it.hg * 8;  // first query head of the item
-        if (it.win) continue;  // windows are not listed: window_kernel takes them
+        if (it.win) continue;  // windows are not listed: the prologue's window CTAs take them
         {
             const int64_t q_off = (static_cast<int64_t>(it.b) * a.num_q_heads + head0) * kHeadDim;
             wt.begin(a.qrot + q_off, a.qjl_q + q_off, rows, r, c);
@@ -2009,7 +2035,33 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
     }
 }
 
-// Exclusive scan of x over the CTA (1024 threads); total gets the sum.
+// ---- The decode prologue: one launch of kProThreads-thread CTAs that builds
+// the work list (CTA 0), rotates the queries (the next n_rot CTAs) and
+// attends over the dense windows (the rest), so the decode kernel follows one
+// launch instead of three.
+constexpr int kProThreads = 256, kProWarps = kProThreads / 32;
+constexpr int kListBuckets = kMaxItemTiles + 1;  // partial splits by tile count 1 .. 256
+static_assert(kProThreads == kMaxItemTiles, "one thread per partial-split bucket");
+constexpr int kRotRows = kProWarps;  // query rows per rotation CTA, one per warp
+
+union ProSmem {
+    struct {
+        int cursor[kListBuckets];  // partial splits per tile count, then write cursors
+        int warp_tot[32];
+        int tot_full, base_full;
+    } wl;
+    float zs[kRotRows][kHeadDim];  // rotated rows of a rotation CTA
+    struct {
+        float qs[16][kHeadDim];    // group-wise: the head's query rows
+        float part[16][kHeadDim];  // second half's partial products
+    } dense;
+    struct {
+        float m[kProWarps][8], l[kProWarps][8];
+        float o[kProWarps][8][kHeadDim];
+    } win;
+};
+
+// Exclusive scan of x over the CTA; total gets the sum.
 __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_tot, int& total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     int v = x;
@@ -2039,16 +2091,11 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_tot, int& t
 // Work list of the tensor-core kernels: the (sequence, split) pairs of every
 // non-empty packed work item, longest first: every full split (sequence by
 // sequence), then the partial last splits by decreasing tile count (a
-// counting sort); and their number. Dealt in snake order (item_of), this
-// balances the persistent CTAs about as well as greedy longest-first
-// assignment. (The windows are window_kernel's.) One CTA of 1024 threads, two
-// passes.
-constexpr int kListBuckets = kMaxItemTiles + 1;  // partial splits by tile count 1 .. 256
-
-__global__ void __launch_bounds__(1024) work_list_kernel(DecodeArgs a) {
-    __shared__ int cursor[kListBuckets];  // pass 1: partial splits per tile count; then write cursors
-    __shared__ int warp_tot[32];
-    __shared__ int tot_full, base_full;
+// counting sort whose bucket offsets come from one scan over the CTA); and
+// their number. Dealt in snake order (item_of), this balances the persistent
+// CTAs about as well as greedy longest-first assignment.
+__device__ __forceinline__ void build_work_list(const DecodeArgs& a, ProSmem& sm) {
+    auto& s = sm.wl;
     const int tid = threadIdx.x;
     auto geometry = [&](int b, int& nf, int& part_tiles) {
         int L = __ldg(a.seq_lens + b);
@@ -2058,80 +2105,80 @@ __global__ void __launch_bounds__(1024) work_list_kernel(DecodeArgs a) {
         const int rem = P - nf * a.split_tokens;
         part_tiles = (rem + 15) >> 4;
     };
-    for (int i = tid; i < kListBuckets; i += blockDim.x) cursor[i] = 0;
-    if (tid == 0) tot_full = 0;
+    for (int i = tid; i < kListBuckets; i += kProThreads) s.cursor[i] = 0;
+    if (tid == 0) s.tot_full = 0;
     __syncthreads();
-    for (int b = tid; b < a.batch; b += blockDim.x) {
+    for (int b = tid; b < a.batch; b += kProThreads) {
         int nf, pt;
         geometry(b, nf, pt);
-        if (nf) atomicAdd(&tot_full, nf);
-        if (pt) atomicAdd(&cursor[pt], 1);
+        if (nf) atomicAdd(&s.tot_full, nf);
+        if (pt) atomicAdd(&s.cursor[pt], 1);
     }
     __syncthreads();
-    if (tid == 0) {
-        int pos = tot_full;
-        for (int k = kListBuckets - 1; k >= 1; --k) {
-            const int n = cursor[k];
-            cursor[k] = pos;
-            pos += n;
+    {
+        // thread t owns bucket kMaxItemTiles - t: the longest partial splits come first, after
+        // the full ones (every thread reads its count before the scan's first barrier)
+        const int k = kMaxItemTiles - tid;
+        int n_part;
+        const int of = block_exclusive_scan(s.cursor[k], s.warp_tot, n_part);
+        s.cursor[k] = s.tot_full + of;
+        if (tid == 0) {
+            s.base_full = 0;
+            *a.work_count = s.tot_full + n_part;
         }
-        base_full = 0;
-        *a.work_count = pos;
     }
     __syncthreads();
     int2* list = reinterpret_cast<int2*>(a.work_list);
-    for (int b0 = 0; b0 < a.batch; b0 += blockDim.x) {
+    for (int b0 = 0; b0 < a.batch; b0 += kProThreads) {
         const int b = b0 + tid;
         int nf = 0, pt = 0;
         if (b < a.batch) geometry(b, nf, pt);
         int n_full;
-        const int of = block_exclusive_scan(nf, warp_tot, n_full);
-        for (int j = 0; j < nf; ++j) list[base_full + of + j] = make_int2(b, j);
-        if (pt) list[atomicAdd(&cursor[pt], 1)] = make_int2(b, nf);
+        const int of = block_exclusive_scan(nf, s.warp_tot, n_full);
+        for (int j = 0; j < nf; ++j) list[s.base_full + of + j] = make_int2(b, j);
+        if (pt) list[atomicAdd(&s.cursor[pt], 1)] = make_int2(b, nf);
         __syncthreads();
-        if (tid == 0) base_full += n_full;
+        if (tid == 0) s.base_full += n_full;
         __syncthreads();
     }
 }
 
-// The dense bf16 window of each (sequence, KV head, group of <= 8 query
-// heads), on CUDA cores: one CTA of kWinWarps warps, warp w takes window
-// tokens w, w + kWinWarps, ...; the warps merge their (max, sum, accumulator)
-// states in shared memory into the window's record (split max_splits).
-constexpr int kWinWarps = 4;
-
-__global__ void __launch_bounds__(kWinWarps * 32) window_kernel(DecodeArgs a, int group, int head_groups) {
-    __shared__ float red_m[kWinWarps][8], red_l[kWinWarps][8];
-    __shared__ float red_o[kWinWarps][8][kHeadDim];
+// The dense bf16 window of one (sequence, KV head, group of <= 8 query heads),
+// on CUDA cores: warp w takes window tokens w, w + kProWarps, ...; the warps
+// merge their (max, sum, accumulator) states in shared memory into the
+// window's record (split max_splits).
+template <int NH>
+__device__ __forceinline__ void window_unit(const DecodeArgs& a, int group, int head_groups, int64_t u,
+                                            ProSmem& sm) {
+    auto& s = sm.win;
     const int H = a.kc.num_heads;
-    int64_t u = blockIdx.x;
     Item it;
     it.hg = static_cast<int>(u % head_groups);
     u /= head_groups;
     it.h = static_cast<int>(u % H);
     it.b = static_cast<int>(u / H);
     it.split = a.max_splits;
-    if (!item_range(a, it)) return;  // no window tokens
+    if (!item_range(a, it)) return;  // no window tokens (the same for the whole CTA)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rows = group < 8 ? group : 8;
+    const int rows = group < NH ? group : NH;
     const int head0 = it.h * group + it.hg * 8;
-    window_state(a, it, it.h, head0, rows, warp, kWinWarps, lane, &red_m[warp][0], &red_l[warp][0],
-                 &red_o[warp][0][0], 1, kHeadDim);
+    window_state<NH>(a, it, it.h, head0, rows, warp, kProWarps, lane, &s.m[warp][0], &s.l[warp][0], &s.o[warp][0][0],
+                 1, kHeadDim);
     __syncthreads();
     float* rec = record_of(a, it.b, it.h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
-    for (int e = threadIdx.x; e < rows * kHeadDim; e += kWinWarps * 32) {
+    for (int e = threadIdx.x; e < rows * kHeadDim; e += kProThreads) {
         const int g = e / kHeadDim, j = e - g * kHeadDim;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWinWarps; ++w) M = fmaxf(M, red_m[w][g]);
+        for (int w = 0; w < kProWarps; ++w) M = fmaxf(M, s.m[w][g]);
         float Ls = 0.0f, A = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kWinWarps; ++w) {
-            const float mw = red_m[w][g];
+        for (int w = 0; w < kProWarps; ++w) {
+            const float mw = s.m[w][g];
             if (mw != -INFINITY) {
                 const float f = ex2(mw - M);
-                Ls += red_l[w][g] * f;
-                A += red_o[w][g][j] * f;
+                Ls += s.l[w][g] * f;
+                A += s.o[w][g][j] * f;
             }
         }
         float* rg = rec + g * (kHeadDim + 2);
@@ -2143,24 +2190,22 @@ __global__ void __launch_bounds__(kWinWarps * 32) window_kernel(DecodeArgs a, in
     }
 }
 
-// Rotated queries: q_r = pi_K(H(s_K * q) / sqrt(128)) * scale * log2(e). A CTA
-// of 8 warps takes 8 consecutive (b, query head) rows, one warp per row. With
-// QJL keys it also writes qjl_out = sqrt(pi/2)/128 * S q_r, S applied in
-// rotated (not packed) coordinate order, as the residual it projected: the
-// rows' q_r go to shared memory and thread i computes output i of 4 rows, so
-// the CTA reads S (64 KB, from L2) once for its 8 rows.
-constexpr int kRotRows = 8;
-
-__global__ void __launch_bounds__(kRotRows * 32) rotate_queries_kernel(DevCodec kc, const __nv_bfloat16* q,
-                                                                        int num_q_heads, int group, int64_t total,
-                                                                        float scale_log2, float* out,
-                                                                        float* qjl_out) {
-    __shared__ float zs[kRotRows][kHeadDim];  // q_r of the CTA's rows, rotated order
+// Rotated queries: q_r = pi_K(H(s_K * q) / sqrt(128)) * scale * log2(e). Rotation
+// CTA `blk` takes the kRotRows consecutive (b, query head) rows from
+// blk * kRotRows, one warp per row. With QJL keys it also writes
+// qjl_out = sqrt(pi/2)/128 * S q_r, S applied in rotated (not packed)
+// coordinate order, as the residual it projected: the rows' q_r go to shared
+// memory and thread i computes output i of 4 rows, so the CTA reads S (64 KB,
+// from L2) once for its rows.
+__device__ __forceinline__ void rotate_rows(const DecodeArgs& a, int group, int64_t total, int64_t blk,
+                                            float* qjl_out, ProSmem& sm) {
+    const DevCodec& kc = a.kc;
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRotRows;
+    const int64_t row0 = blk * kRotRows;
     const int64_t row = row0 + w;
     if (row < total) {
-        const int hq = static_cast<int>(row % num_q_heads), h = hq / group;
+        const int hq = static_cast<int>(row % a.num_q_heads), h = hq / group;
         const uint2 raw = *reinterpret_cast<const uint2*>(q + row * kHeadDim + 4 * lane);
         float z[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
                       __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u)};
@@ -2180,24 +2225,25 @@ __global__ void __launch_bounds__(kRotRows * 32) rotate_queries_kernel(DevCodec 
                 const float p = __shfl_xor_sync(kFull, z[i], m);
                 z[i] = (lane & m) ? (p - z[i]) : (z[i] + p);
             }
-        const float sc = scale_log2 * 0.08838834764831845f;  // 1/sqrt(128)
+        const float sc = a.scale_log2 * 0.08838834764831845f;  // 1/sqrt(128)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             z[i] *= sc;
-            out[row * kHeadDim + kc.pos[h * kHeadDim + 4 * lane + i]] = z[i];
-            zs[w][4 * lane + i] = z[i];
+            a.qrot[row * kHeadDim + kc.pos[h * kHeadDim + 4 * lane + i]] = z[i];
+            sm.zs[w][4 * lane + i] = z[i];
         }
     }
     if (qjl_out == nullptr) return;  // uniform over the CTA
     __syncthreads();
     // (S q_r)_i = sum_j S[i][j] q_r[j]: thread (i, half) for rows 4 half .. 4 half + 3
+    static_assert(kRotRows == 8 && kProThreads == 2 * kHeadDim, "two halves of four rows");
     const int i = threadIdx.x & (kHeadDim - 1), r0 = (threadIdx.x >> 7) * 4;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 4
     for (int j = 0; j < kHeadDim; ++j) {
         const float sij = __ldg(kc.qjl_st + j * kHeadDim + i);  // S^T row j, coalesced over i
 #pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] = fmaf(sij, zs[r0 + k][j], acc[k]);
+        for (int k = 0; k < 4; ++k) acc[k] = fmaf(sij, sm.zs[r0 + k][j], acc[k]);
     }
     constexpr float kappa = 1.2533141373155003f / kHeadDim;  // sqrt(pi/2) / d, the estimator's constant
 #pragma unroll
@@ -2206,34 +2252,66 @@ __global__ void __launch_bounds__(kRotRows * 32) rotate_queries_kernel(DevCodec 
 }
 
 // Group-wise K: q_r = R_h q * scale * log2(e) in packed order (R_h from the
-// codec: rot_t entry (h, j, p) = R_h[p][j]). One CTA per (b, KV head) takes
-// the head's query rows (group <= 16) together: their q goes to shared
-// memory, thread p computes packed position p of every row, and the CTA reads
-// R_h (64 KB, rows contiguous over p) once.
-__global__ void __launch_bounds__(kHeadDim) rotate_queries_dense_kernel(DevCodec kc, const __nv_bfloat16* q,
-                                                                         int num_q_heads, int group,
-                                                                         float scale_log2, float* out) {
-    __shared__ float qs[16][kHeadDim];
-    const int H = kc.num_heads, p = threadIdx.x;
-    const int h = blockIdx.x % H, b = blockIdx.x / H;
-    const int64_t row0 = static_cast<int64_t>(b) * num_q_heads + static_cast<int64_t>(h) * group;
-    for (int g = 0; g < group; ++g)
-        qs[g][p] = __bfloat162float(q[(row0 + g) * kHeadDim + p]);
+// codec: rot_t entry (h, j, p) = R_h[p][j]). Rotation CTA `unit` = (b, KV
+// head) takes the head's query rows (group <= 16) together: their q goes to
+// shared memory, thread (p, half) sums packed position p of every row over
+// half of the j range, and the CTA reads R_h (64 KB, rows contiguous over p)
+// once.
+__device__ __forceinline__ void rotate_rows_dense(const DecodeArgs& a, int group, int64_t unit, ProSmem& sm) {
+    const DevCodec& kc = a.kc;
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+    const int H = kc.num_heads, p = threadIdx.x & (kHeadDim - 1), half = threadIdx.x >> 7;
+    const int h = static_cast<int>(unit % H);
+    const int64_t b = unit / H;
+    const int64_t row0 = b * a.num_q_heads + static_cast<int64_t>(h) * group;
+    for (int g = half; g < group; g += 2) sm.dense.qs[g][p] = __bfloat162float(q[(row0 + g) * kHeadDim + p]);
     __syncthreads();
     const float* rt = kc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim;
     float acc[16];
 #pragma unroll
     for (int g = 0; g < 16; ++g) acc[g] = 0.0f;
+    const int j0 = half * (kHeadDim / 2);
 #pragma unroll 2
-    for (int j = 0; j < kHeadDim; ++j) {
+    for (int j = j0; j < j0 + kHeadDim / 2; ++j) {
         const float rjp = __ldg(rt + j * kHeadDim + p);
 #pragma unroll
         for (int g = 0; g < 16; ++g)
-            if (g < group) acc[g] = fmaf(rjp, qs[g][j], acc[g]);
+            if (g < group) acc[g] = fmaf(rjp, sm.dense.qs[g][j], acc[g]);
     }
+    if (half) {
 #pragma unroll
-    for (int g = 0; g < 16; ++g)
-        if (g < group) out[(row0 + g) * kHeadDim + p] = acc[g] * scale_log2;
+        for (int g = 0; g < 16; ++g)
+            if (g < group) sm.dense.part[g][p] = acc[g];
+    }
+    __syncthreads();
+    if (!half) {
+#pragma unroll
+        for (int g = 0; g < 16; ++g)
+            if (g < group) a.qrot[(row0 + g) * kHeadDim + p] = (acc[g] + sm.dense.part[g][p]) * a.scale_log2;
+    }
+}
+
+// CTA 0: the work list; CTAs 1 .. n_rot: query rotation; the rest: windows
+// (b, KV head, query-head group). The decode kernel that follows may start as
+// soon as every CTA here has begun (it waits for this grid's results itself).
+template <int KMODE, int NH>
+__global__ void __launch_bounds__(kProThreads, NH == 4 ? 2 : 1) decode_prologue_kernel(DecodeArgs a, int group,
+                                                                                      int head_groups,
+                                                                      int64_t n_rot) {
+    __shared__ ProSmem sm;
+    griddep_launch_dependents();
+    const int64_t blk = blockIdx.x;
+    if (blk == 0) {
+        build_work_list(a, sm);
+    } else if (blk <= n_rot) {
+        if constexpr (KMODE == kGroupwise)
+            rotate_rows_dense(a, group, blk - 1, sm);
+        else
+            rotate_rows(a, group, static_cast<int64_t>(a.batch) * a.num_q_heads, blk - 1,
+                        KMODE == kQjl ? a.qjl_q : nullptr, sm);
+    } else {
+        window_unit<NH>(a, group, head_groups, blk - 1 - n_rot, sm);
+    }
 }
 
 constexpr int kMaxDynSmem = 227 * 1024;
@@ -2283,44 +2361,46 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int head_groups = group > 8 ? group / 8 : 1;
     const int64_t rows = static_cast<int64_t>(a.batch) * a.num_q_heads;
-    work_list_kernel<<<1, 1024, 0, s>>>(a);
-    if (a.window > 0 && a.batch > 0)
-        window_kernel<<<static_cast<unsigned>(static_cast<int64_t>(a.batch) * a.kc.num_heads * head_groups),
-                        kWinWarps * 32, 0, s>>>(a, group, head_groups);
-    if constexpr (KF::MODE == kGroupwise)
-        rotate_queries_dense_kernel<<<static_cast<unsigned>(a.batch) * a.kc.num_heads, kHeadDim, 0, s>>>(
-            a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads, group, a.scale_log2, a.qrot);
-    else
-        rotate_queries_kernel<<<static_cast<unsigned>((rows + kRotRows - 1) / kRotRows), kRotRows * 32, 0, s>>>(
-            a.kc, static_cast<const __nv_bfloat16*>(a.q), a.num_q_heads, group, rows, a.scale_log2, a.qrot,
-            KF::MODE == kQjl ? a.qjl_q : nullptr);
+    // One prologue launch builds the work list, rotates the queries and attends over the windows.
+    const int64_t n_rot = KF::MODE == kGroupwise ? static_cast<int64_t>(a.batch) * a.kc.num_heads
+                                                 : (rows + kRotRows - 1) / kRotRows;
+    const int64_t n_win = a.window > 0 ? static_cast<int64_t>(a.batch) * a.kc.num_heads * head_groups : 0;
+    if (1 + n_rot + n_win > INT32_MAX) return TQ_ERR_UNSUPPORTED;
+    decode_prologue_kernel<KF::MODE, NH><<<static_cast<unsigned>(1 + n_rot + n_win), kProThreads, 0, s>>>(
+        a, group, head_groups, n_rot);
     const int64_t units = static_cast<int64_t>(a.items_per_unit) * a.batch * head_groups *
                           (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);
     const int grid = static_cast<int>(units < sms ? units : sms);
     if (grid > 0) {
         const dim3 threads((kBlkWarps + 1) * 32), pair_threads(kPairThreads);
-        static const bool pair_env = [] {
-            const char* e = std::getenv("TQ_DECODE_PAIR");
-            return !(e && e[0] == '0');
-        }();
-        const bool pair = pair_env && pair_regs_ok.load() == 1;
+        // TQ_DECODE_PAIR=0 takes the block kernel instead of the paired one, for cross-checks.
+        const char* pair_env = std::getenv("TQ_DECODE_PAIR");
+        const bool pair = !(pair_env && pair_env[0] == '0') && pair_regs_ok.load() == 1;
         // The paired kernel wants two run pairs of slots beside the table (one more slot than that
         // covers the ring's split around the 64 KB-aligned table).
         const bool pair_fits = static_cast<size_t>(blk_slot_bytes<KF, VF>(a.block_size)) * 5 <=
                                static_cast<size_t>(kMaxDynSmem) - kLut - 4096;
+        // The decode kernel may start while the prologue ends (it waits for the prologue's results).
+        cudaError_t le;
         if (blk && pair && pair_fits && a.block_size == 16)
-            decode_pair_kernel<KF, VF, NH, 1><<<grid, pair_threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
+            le = launch_dependent(decode_pair_kernel<KF, VF, NH, 1>, grid, pair_threads, kMaxDynSmem, s, a, tv, group,
+                                  head_groups, units);
         else if (blk && pair && pair_fits && a.block_size == 32)
-            decode_pair_kernel<KF, VF, NH, 2><<<grid, pair_threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
+            le = launch_dependent(decode_pair_kernel<KF, VF, NH, 2>, grid, pair_threads, kMaxDynSmem, s, a, tv, group,
+                                  head_groups, units);
         else if (blk && a.block_size == 16)
-            decode_blk_kernel<KF, VF, NH, 1><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
+            le = launch_dependent(decode_blk_kernel<KF, VF, NH, 1>, grid, threads, kMaxDynSmem, s, a, tv, group,
+                                  head_groups, units);
         else if (blk && a.block_size == 32)
-            decode_blk_kernel<KF, VF, NH, 2><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
+            le = launch_dependent(decode_blk_kernel<KF, VF, NH, 2>, grid, threads, kMaxDynSmem, s, a, tv, group,
+                                  head_groups, units);
         else if (blk)
-            decode_blk_kernel<KF, VF, NH, 0><<<grid, threads, kMaxDynSmem, s>>>(a, tv, group, head_groups, units);
+            le = launch_dependent(decode_blk_kernel<KF, VF, NH, 0>, grid, threads, kMaxDynSmem, s, a, tv, group,
+                                  head_groups, units);
         else
-            decode_mma_kernel<KF, VF, NH, NW><<<grid, (NW + 1) * 32, head_bytes, s>>>(a, tv, group, head_groups,
-                                                                                      units);
+            le = launch_dependent(decode_mma_kernel<KF, VF, NH, NW>, grid, dim3((NW + 1) * 32), head_bytes, s, a, tv,
+                                  group, head_groups, units);
+        if (le != cudaSuccess) return fail(TQ_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(le));
     }
     return TQ_OK;
 }

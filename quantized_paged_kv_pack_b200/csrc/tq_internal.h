@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "tq.h"
@@ -130,6 +131,27 @@ cudaError_t once_per_device(int dev, F&& f) {
     if (e == cudaSuccess) done[dev] = 1;
     return e;
 }
+
+#ifdef __CUDACC__
+// Launches `kernel` with programmatic stream serialization: it may start while
+// the previous kernel in `stream` is still running, and must call
+// griddepcontrol.wait before it reads anything that kernel writes.
+template <class... KArgs, class... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+#endif
 
 // Sets the thread-local error message and returns `st`.
 tq_status fail(tq_status st, const std::string& msg);

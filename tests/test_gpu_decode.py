@@ -240,6 +240,27 @@ def test_decode_eight_kv_heads_windows_and_block_sizes(window, bs):
     check(prob, pairs)
 
 
+
+@pytest.mark.parametrize("kspec,vspec,G,bs", [(U4, U4, 8, 16), (M35, M35, 4, 32), (M25, U3, 8, 32),
+                                               (M35, U4, 2, 16)])
+def test_block_kernel_and_paired_kernel_agree(kspec, vspec, G, bs, monkeypatch):
+    """TQ_DECODE_PAIR=0 runs the one-warp-per-head block kernel that the paired kernel replaces (it
+    remains the path when the paired kernel's ring does not fit): both against the oracle and each
+    other, with ragged lengths, a window and splits cut mid-block."""
+    lens = [1, bs - 1, 5 * bs + 3, 4700, 9000]
+    prob = DecodeProblem(lens, 8, G, kspec, (vspec[0], vspec[1], vspec[2] + 10), window=24, block_size=bs,
+                         seed=200 + G + bs)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    paired = prob.run(d_err=err).clone()
+    monkeypatch.setenv("TQ_DECODE_PAIR", "0")
+    block = prob.run(d_err=err).clone()
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert (paired - block).abs().max().item() <= ATOL
+    rng = np.random.default_rng(G + bs)
+    pairs = [(b, int(hq)) for b in range(prob.B) for hq in rng.choice(prob.Hq, 6, replace=False)]
+    check(prob, pairs)
+
 def test_decode_sixteen_kv_heads_gqa16():
     """Two groups of 8 KV heads, two query-head groups per KV head."""
     prob = DecodeProblem([5000, 700], 16, 16, U4, M35, window=16, block_size=16, seed=31)
