@@ -39,7 +39,7 @@ HEADLINE = "decode_llama70b_3p5bit"
 SMALL = "decode_gqa8_4k_4bit"
 DECODE_LAUNCHES = 4  # per step: window append, prologue (work list, query rotation, windows), partials, combine
 EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl",
-         "decode_llama8b_3p5bit_groupwise",
+         "decode_llama8b_3p5bit_groupwise", "decode_llama8b_3p5bit_recipe",
          "pack_llama8b_4bit", "pack_llama70b_3p5bit", "pack_llama8b_2p5bit"]
 D = 128
 METRIC = "paged TQ decode HBM GB/s (algorithmic bytes / step time)"

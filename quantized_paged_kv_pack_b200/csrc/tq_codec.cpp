@@ -387,12 +387,13 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
     const int G = num_q_heads / num_kv_heads;
     if (G > 16) return false;
     // The longest split: about 4096 packed (sequence, KV head, split) items per call, splits of
-    // 512..4096 tokens (at most 32 tiles of 16 tokens for each of a CTA's 8 warps). A call of at most
-    // 65536 tokens over all sequences and heads takes splits down to 128 tokens instead, so that its
-    // few items spread over more CTAs: it is latency-bound, not bound by the per-item overhead.
+    // 512..4096 tokens (at most 32 tiles of 16 tokens for each of a CTA's 8 warps). Shorter splits
+    // for small calls measured slower: one 4096-token sequence took 26 us per call with 96-token
+    // splits against 21.5 us with 512 (the per-item cost and the combine's longer merge outweigh
+    // the wider spread).
     double total = static_cast<double>(std::max(max_seq_len, 1)) * std::max(batch, 1) * num_kv_heads;
     int64_t s = static_cast<int64_t>(std::ceil(total / 4096.0));
-    s = std::min<int64_t>(std::max<int64_t>(s, total <= 65536.0 ? 128 : 512), 4096);
+    s = std::min<int64_t>(std::max<int64_t>(s, 512), 4096);
     s = (s + 63) / 64 * 64;
     s = (s + block_size - 1) / block_size * block_size;
     if (block_size <= 4096) s = std::min<int64_t>(s, 4096 / block_size * block_size);  // e.g. 4080 for 48

@@ -298,12 +298,66 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
     }
 }
 
+// Log-sum-exp merge of the split records of one (sequence, query head), over
+// the 128 threads j of a group (4 warps; a CTA may hold several groups, all
+// with the same ns and n_win: the barriers inside are CTA-wide). Returns the
+// merged sum ls, accumulator position j (rot) and the window record's share
+// (win), all relative to the largest record max. The records are read in
+// parallel: first every max (thread j takes splits j, j + 128, ...), then per
+// chunk of 128 splits each thread's weight goes to shared memory and the
+// accumulator sums its column with eight loads in flight. fw: the group's 128
+// floats of shared scratch, red: its 4.
+__device__ __forceinline__ void merge_splits(const float* unit, int G, int g, int ns, int n_win, int max_splits,
+                                             int j, float* fw, float* red, float& ls, float& rot, float& win) {
+    auto rec = [&](int i) { return unit + (static_cast<int64_t>(i) * G + g) * (kHeadDim + 2); };
+    const int lane = j & 31, wg = j >> 5;
+    float m = -INFINITY;
+    for (int i = j; i < ns; i += kHeadDim) m = fmaxf(m, rec(i)[0]);
+    if (n_win && j == 0) m = fmaxf(m, rec(max_splits)[0]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+    if (lane == 0) red[wg] = m;
+    __syncthreads();
+    const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();  // red is written again below
+    ls = 0.0f;
+    rot = 0.0f;
+    win = 0.0f;
+    if (M == -INFINITY) return;  // no record: the same for every group of the CTA (one sequence)
+    float lpart = 0.0f;
+    for (int c0 = 0; c0 < ns; c0 += kHeadDim) {
+        float f = 0.0f;
+        if (c0 + j < ns) {
+            const float* r = rec(c0 + j);
+            f = exp2f(r[0] - M);
+            lpart += r[1] * f;
+        }
+        fw[j] = f;
+        __syncthreads();
+        const int n = min(kHeadDim, ns - c0);
+#pragma unroll 8
+        for (int k = 0; k < n; ++k) rot = fmaf(rec(c0 + k)[2 + j], fw[k], rot);
+        __syncthreads();  // fw is written again by the next chunk
+    }
+    lpart = warp_sum(lpart);
+    if (lane == 0) red[wg] = lpart;
+    __syncthreads();
+    ls = (red[0] + red[1]) + (red[2] + red[3]);
+    if (n_win) {
+        const float* r = rec(max_splits);
+        const float f = exp2f(r[0] - M);
+        ls += r[1] * f;
+        win = r[2 + j] * f;
+    }
+}
+
 __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, const int32_t* seq_lens,
                                                                    int32_t num_q_heads, int32_t max_seq_len,
                                                                    int32_t window, int32_t split_tokens,
                                                                    int32_t max_splits, int32_t items_per_unit,
                                                                    int32_t G, const float* ws, float* out) {
     __shared__ float y[kHeadDim];
+    __shared__ float red[4];
     // Launched as a dependent of the partials: the split records are read only after they are complete.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int hq = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
@@ -313,23 +367,9 @@ __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, c
     const int n_win = min(window, L), P = L - n_win;
     const int ns = (P + split_tokens - 1) / split_tokens;
     const float* unit = ws + (static_cast<int64_t>(b) * H + h) * items_per_unit * static_cast<int64_t>(G) * (kHeadDim + 2);
-    auto rec = [&](int i) { return unit + (static_cast<int64_t>(i) * G + g) * (kHeadDim + 2); };
-    float M = -INFINITY;
-    for (int i = 0; i < ns; ++i) M = fmaxf(M, rec(i)[0]);
-    if (n_win) M = fmaxf(M, rec(max_splits)[0]);
-    float Ls = 0.0f, rot = 0.0f, win = 0.0f;
-    if (M != -INFINITY) {
-        for (int i = 0; i < ns; ++i) {
-            const float f = exp2f(rec(i)[0] - M);
-            Ls += rec(i)[1] * f;
-            rot += rec(i)[2 + j] * f;
-        }
-        if (n_win) {
-            const float f = exp2f(rec(max_splits)[0] - M);
-            Ls += rec(max_splits)[1] * f;
-            win = rec(max_splits)[2 + j] * f;
-        }
-    }
+    float Ls, rot, win;
+    merge_splits(unit, G, g, ns, n_win, max_splits, j, y, red, Ls, rot, win);
+    __syncthreads();  // y served as the merge's scratch
     float x;
     if (vc.groupwise) {
         y[j] = rot;  // packed positions
@@ -358,7 +398,8 @@ __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, c
 // matrix from L2 with row-strided loads.
 constexpr int kGwPitch = kHeadDim + 1;
 constexpr int kGwHeads = 8;
-constexpr size_t kGwCombineSmem = (static_cast<size_t>(kHeadDim) * kGwPitch + kGwHeads * kHeadDim) * sizeof(float);
+constexpr size_t kGwCombineSmem =
+    (static_cast<size_t>(kHeadDim) * kGwPitch + kGwHeads * kHeadDim + kGwHeads * 4) * sizeof(float);
 
 __global__ void __launch_bounds__(kHeadDim * kGwHeads) decode_combine_gw_kernel(
     DevCodec vc, const int32_t* seq_lens, int32_t num_q_heads, int32_t max_seq_len, int32_t window,
@@ -366,6 +407,7 @@ __global__ void __launch_bounds__(kHeadDim * kGwHeads) decode_combine_gw_kernel(
     extern __shared__ float gsm[];
     float* rts = gsm;                               // [128][129]: R_h^T, row j at j * 129
     float* ys = gsm + kHeadDim * kGwPitch;          // [kGwHeads][128]
+    float* reds = ys + kGwHeads * kHeadDim;         // [kGwHeads][4]
     const int H = vc.num_heads, h = blockIdx.x % H, b = blockIdx.x / H;
     const int j = threadIdx.x & (kHeadDim - 1), gl = threadIdx.x >> 7, nthreads = blockDim.x;
     const float* rt = vc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim;
@@ -381,27 +423,14 @@ __global__ void __launch_bounds__(kHeadDim * kGwHeads) decode_combine_gw_kernel(
     const float* unit = ws + (static_cast<int64_t>(b) * H + h) * items_per_unit * static_cast<int64_t>(G) * (kHeadDim + 2);
     const int per = nthreads / kHeadDim;  // query heads per pass
     for (int g0 = 0; g0 < G; g0 += per) {
+        // Every group takes part in each pass (the merge's barriers are CTA-wide). G is 1, 2, 4, 8 or
+        // 16, so no group runs past G; were one to, it would repeat head G - 1 and write nothing.
         const int g = g0 + gl;
-        float Ls = 0.0f, rot = 0.0f, win = 0.0f;
-        if (g < G) {
-            auto rec = [&](int i) { return unit + (static_cast<int64_t>(i) * G + g) * (kHeadDim + 2); };
-            float M = -INFINITY;
-            for (int i = 0; i < ns; ++i) M = fmaxf(M, rec(i)[0]);
-            if (n_win) M = fmaxf(M, rec(max_splits)[0]);
-            if (M != -INFINITY) {
-                for (int i = 0; i < ns; ++i) {
-                    const float f = exp2f(rec(i)[0] - M);
-                    Ls += rec(i)[1] * f;
-                    rot += rec(i)[2 + j] * f;
-                }
-                if (n_win) {
-                    const float f = exp2f(rec(max_splits)[0] - M);
-                    Ls += rec(max_splits)[1] * f;
-                    win = rec(max_splits)[2 + j] * f;
-                }
-            }
-            ys[gl * kHeadDim + j] = rot;  // packed positions
-        }
+        float Ls, rot, win;
+        merge_splits(unit, G, g < G ? g : G - 1, ns, n_win, max_splits, j, ys + gl * kHeadDim, reds + gl * 4, Ls,
+                     rot, win);
+        __syncthreads();  // ys served as the merge's scratch
+        ys[gl * kHeadDim + j] = rot;  // packed positions
         __syncthreads();  // (the first pass also waits for the staged R_h^T)
         if (g < G) {
             const float* rj = rts + j * kGwPitch;

@@ -300,6 +300,14 @@ __device__ __forceinline__ uint32_t pair_addr(const uint32_t (&w)[NW], uint32_t 
     }
 }
 
+// Transpose of an 8x8 fp16 matrix held one row-pair per lane (lane l: row l / 4,
+// columns 2 (l % 4), +1), returned in the same layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 // Interleave two tokens' chunks: field k of e holds (index of a, index of b)
 // at chunk position 2k, field k of o at position 2k + 1.
 template <int B, int NW>
@@ -666,13 +674,13 @@ struct WarpTiles {
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 // sign k-step s: B rows (2c, 2c+1) and (2c+8, 2c+9) are projections
-                // 32c + s + (0, 8) and 32c + s + (16, 24)
+                // 32c + s + (0, 16) and 32c + s + (8, 24)
                 float x0 = 0.0f, x1 = 0.0f, x2 = 0.0f, x3 = 0.0f;
                 if (head < rows) {
                     const float* z = qz + head * kHeadDim + 32 * c + s;
                     x0 = __ldcg(z);
-                    x1 = __ldcg(z + 8);
-                    x2 = __ldcg(z + 16);
+                    x1 = __ldcg(z + 16);
+                    x2 = __ldcg(z + 8);
                     x3 = __ldcg(z + 24);
                 }
                 uint32_t h01, l01, h23, l23;
@@ -777,21 +785,20 @@ struct WarpTiles {
                 if constexpr (kOwnLoads) return zl;
                 else return zf;
             }();
-            // Sign k-step s takes bits s, s + 8, s + 16, s + 24 of the lane's word
-            // (projections 32c + ...): shifted to the top of bytes 0..3, prmt
-            // turns each into an all-ones or all-zero byte in the high byte of
-            // a half, which becomes the sign of +-|r|.
+            // Sign k-step s takes bits (s, s + 16) of the lane's word (projections
+            // 32c + ...) for its k columns (2c, 2c + 1) and bits (s + 8, s + 24)
+            // for (2c + 8, 2c + 9): one shift puts such a pair at bits 15 and 31,
+            // the sign bits of the two halves of +-|r| (a clear bit is -).
             const uint32_t wa = lds32(kbase + r * KF::RB + KF::IB + 4 * c);
             const uint32_t wb = lds32(kbase + (r + 8) * KF::RB + KF::IB + 4 * c);
             const uint32_t ga = lds16(knorm + KF::NB * r + 2), gb = lds16(knorm + KF::NB * (r + 8) + 2);
             const uint32_t rn_a = ga | (ga << 16), rn_b = gb | (gb << 16);
             static_for<0, 8>([&](auto si) {
                 constexpr int s_ = decltype(si)::value;
-                const uint32_t ya = wa << (7 - s_), yb = wb << (7 - s_);
-                const uint32_t a0 = rn_a | (~prmt(ya, 0u, 0x9484u) & 0x80008000u);
-                const uint32_t a1 = rn_b | (~prmt(yb, 0u, 0x9484u) & 0x80008000u);
-                const uint32_t a2 = rn_a | (~prmt(ya, 0u, 0xB4A4u) & 0x80008000u);
-                const uint32_t a3 = rn_b | (~prmt(yb, 0u, 0xB4A4u) & 0x80008000u);
+                const uint32_t a0 = rn_a | (~(wa << (15 - s_)) & 0x80008000u);
+                const uint32_t a1 = rn_b | (~(wb << (15 - s_)) & 0x80008000u);
+                const uint32_t a2 = rn_a | (~(wa << (7 - s_)) & 0x80008000u);
+                const uint32_t a3 = rn_b | (~(wb << (7 - s_)) & 0x80008000u);
                 if constexpr (NH == 8) {
                     mma16816(sacc[s_ & 1], a0, a1, a2, a3, Z[s_][0], Z[s_][1]);
                     mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, Z[s_][2], Z[s_][3]);
@@ -930,8 +937,8 @@ struct WarpTiles {
     // when V is group-wise); the sums l_run are kept in the same 2^-kSlack
     // units. m_ref is finite here: the first block of an item always moves it
     // (a valid score exceeds -inf + kSlack).
-    __device__ __forceinline__ void block_weights(const float (&sc)[HL][2], uint32_t vnorm, int nvalid, uint32_t psel,
-                                                  int r, int c, uint32_t (&bpo)[2 * HL],
+    __device__ __forceinline__ void block_weights(const float (&sc)[HL][2], uint32_t vnorm, int nvalid, int r,
+                                                  uint32_t (&bpo)[2 * HL],
                                                   uint32_t (&bpo1)[VG ? 2 * HL : 1]) {
         const bool ok0 = r < nvalid, ok1 = r + 8 < nvalid;
         const float nv0 = f16_at(vnorm + VF::NB * r), nv1 = f16_at(vnorm + VF::NB * (r + 8));
@@ -944,11 +951,11 @@ struct WarpTiles {
             p[e][1] = ex2(sc[e][1] - mb);
             l_run[e] += p[e][0] + p[e][1];
         }
-        weights(p, nv0m, nv1m, psel, r, c, bpo);
+        weights(p, nv0m, nv1m, bpo);
         if constexpr (VG) {
             const float mv0 = ok0 ? f16_at(vnorm + VF::NB * r + 2) : 0.0f;
             const float mv1 = ok1 ? f16_at(vnorm + VF::NB * (r + 8) + 2) : 0.0f;
-            weights(p, mv0, mv1, psel, r, c, bpo1);
+            weights(p, mv0, mv1, bpo1);
         }
     }
 
@@ -956,53 +963,48 @@ struct WarpTiles {
     // the online-softmax update; leaves the tile's P' (V norms at vnorm) in bp
     // for values(). Tokens at or past nvalid are padding.
     __device__ __forceinline__ void scores(uint32_t kbase, uint32_t knorm, uint32_t vnorm, int nvalid,
-                                           uint32_t lane_base, uint32_t psel, int r, int c) {
+                                           uint32_t lane_base, int r, int c) {
         uint32_t qf[8][2 * HL];
         uint32_t zf[KQ ? 8 : 1][2 * HL];
         if constexpr (!(KQ && TM)) load_query(qf, zf);
         float sc[1][HL][2];
         block_scores(qf, zf, kbase, knorm, nvalid, lane_base, r, c, sc[0]);
         update<1>(sc);
-        block_weights(sc[0], vnorm, nvalid, psel, r, c, bp, bp1);
+        block_weights(sc[0], vnorm, nvalid, r, bp, bp1);
     }
 
     // B fragments of P'^T (P' = p n_V for the V norms n0 of token r and n1 of
-    // token r + 8): rows tokens (2c, 2c+1) and (2c+8, 2c+9), column r. Tokens
-    // 2c and 2c + 8 sit in lane 8c + (r >> 1), tokens 2c + 1 and 2c + 9 four
-    // lanes on.
-    __device__ __forceinline__ static void weights(const float (&p)[HL][2], float n0, float n1, uint32_t psel, int r,
-                                                   int c, uint32_t (&out)[2 * HL]) {
-        const int srcA = 8 * c + (r >> 1), srcB = srcA + 4;
+    // token r + 8): rows tokens (2c, 2c+1) and (2c+8, 2c+9), column r, made
+    // from the lane's own values by an in-register 8x8 transpose (movmatrix).
+    __device__ __forceinline__ static void weights(const float (&p)[HL][2], float n0, float n1,
+                                                   uint32_t (&out)[2 * HL]) {
         if constexpr (NH == 8) {
-            // Per token: (head 2c, head 2c + 1) as hi and lo half2.
+            // Per token: (head 2c, head 2c + 1) as hi and lo half2, i.e. rows r (tokens 0..7) and
+            // r + 8 (tokens 8..15) of two 8x8 row-major fp16 matrices [token][head]; their
+            // transposes in the same fragment layout are the B fragments [token 2c, 2c+1][head r].
             uint32_t th0, tl0, th1, tl1;
             split2(p[0][0] * n0, p[1][0] * n0, th0, tl0);
             split2(p[0][1] * n1, p[1][1] * n1, th1, tl1);
-            const uint32_t xa = __shfl_sync(kFull, th0, srcA), xb = __shfl_sync(kFull, th0, srcB);
-            const uint32_t ya = __shfl_sync(kFull, th1, srcA), yb = __shfl_sync(kFull, th1, srcB);
-            const uint32_t xla = __shfl_sync(kFull, tl0, srcA), xlb = __shfl_sync(kFull, tl0, srcB);
-            const uint32_t yla = __shfl_sync(kFull, tl1, srcA), ylb = __shfl_sync(kFull, tl1, srcB);
-            out[0] = prmt(xa, xb, psel);
-            out[1] = prmt(ya, yb, psel);
-            out[2] = prmt(xla, xlb, psel);
-            out[3] = prmt(yla, ylb, psel);
+            out[0] = movmatrix_t(th0);
+            out[1] = movmatrix_t(th1);
+            out[2] = movmatrix_t(tl0);
+            out[3] = movmatrix_t(tl1);
         } else {
-            // Per lane: (token r, token r + 8) as hi and lo half2.
+            // Columns are (head, hi / lo): per token, (hi, lo) of head c at columns 2c and 2c + 1 is
+            // row r (tokens 0..7) or r + 8 (tokens 8..15) of an 8x8 row-major fp16 matrix
+            // [token][column]; the transposes are the B fragments [token 2c, 2c+1][column r].
             uint32_t xh, xl;
             split2(p[0][0] * n0, p[0][1] * n1, xh, xl);
-            const uint32_t xa = __shfl_sync(kFull, xh, srcA), ya = __shfl_sync(kFull, xl, srcA);
-            const uint32_t xb = __shfl_sync(kFull, xh, srcB), yb = __shfl_sync(kFull, xl, srcB);
-            const uint32_t pa = (r & 1) ? ya : xa, pb = (r & 1) ? yb : xb;
-            out[0] = prmt(pa, pb, 0x5410u);
-            out[1] = prmt(pa, pb, 0x7632u);
+            out[0] = movmatrix_t(prmt(xh, xl, 0x5410u));
+            out[1] = movmatrix_t(prmt(xh, xl, 0x7632u));
         }
     }
 
     // One 16-token tile: K index rows at kbase (norms at knorm), V index rows at
     // vbase (norms at vnorm); tokens at or past nvalid are padding.
     __device__ __forceinline__ void step(uint32_t kbase, uint32_t knorm, uint32_t vbase, uint32_t vnorm, int nvalid,
-                                         uint32_t lane_base, uint32_t psel, int r, int c) {
-        scores(kbase, knorm, vnorm, nvalid, lane_base, psel, r, c);
+                                         uint32_t lane_base, int r, int c) {
+        scores(kbase, knorm, vnorm, nvalid, lane_base, r, c);
         values(vbase, lane_base, r, c);
     }
 
@@ -1080,7 +1082,7 @@ struct WarpTiles {
     // softmax update and one pass over the accumulators.
     __device__ __forceinline__ void step2(uint32_t kb0, uint32_t kn0, uint32_t vb0, uint32_t vn0, int nv0,
                                           uint32_t kb1, uint32_t kn1, uint32_t vb1, uint32_t vn1, int nv1,
-                                          uint32_t lane_base, uint32_t psel, int r, int c) {
+                                          uint32_t lane_base, int r, int c) {
         float sc[2][HL][2];
         if constexpr (KQ || KG || VG) {
             // these keep more per block: the fragments are reloaded so the two blocks never hold them at once
@@ -1100,8 +1102,8 @@ struct WarpTiles {
         }
         update<2>(sc);
         uint32_t p0[2 * HL], p1[2 * HL], g0[VG ? 2 * HL : 1], g1[VG ? 2 * HL : 1];
-        block_weights(sc[0], vn0, nv0, psel, r, c, p0, g0);
-        block_weights(sc[1], vn1, nv1, psel, r, c, p1, g1);
+        block_weights(sc[0], vn0, nv0, r, p0, g0);
+        block_weights(sc[1], vn1, nv1, r, p1, g1);
         float o[8][4];
         load_acc(o);
         values_block(o, vb0, p0, g0, lane_base, r, c);
@@ -1471,7 +1473,6 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
     }
     uint32_t lane_base;
     asm volatile("or.b32 %0, %1, %2;" : "=r"(lane_base) : "r"(lut_addr), "r"(static_cast<uint32_t>(lane) << 2));
-    const uint32_t psel = (r & 1) ? 0x7632u : 0x5410u;
     const int rows = group < NH ? group : NH;
     // This warp's head within a slot: K sub-page at k_off, V sub-page at v_off.
     const uint32_t k_sub = bs * (KF::RB + KF::NB), v_sub = bs * (VF::RB + VF::NB);
@@ -1503,7 +1504,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
                 for (int j = 0; j < TPB && k + j < ntiles; ++j)
                     wt.step(kb + 16 * j * KF::RB, kb + kBs * KF::RB + 16 * KF::NB * j, vb + 16 * j * VF::RB,
                             vb + kBs * VF::RB + 16 * VF::NB * j, min(16, it.t1 - (it.t0 + 16 * (k + j))), lane_base,
-                            psel, r, c);
+                            r, c);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with the slot
             }
@@ -1522,7 +1523,7 @@ __global__ void __launch_bounds__((kBlkWarps + 1) * 32, 1) decode_blk_kernel(Dec
                     vb = ring.slot(s) + v_off;
                 }
                 wt.step(kb + 16 * j * KF::RB, kb + bs * KF::RB + 16 * KF::NB * j, vb + 16 * j * VF::RB,
-                        vb + bs * VF::RB + 16 * VF::NB * j, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, psel, r, c);
+                        vb + bs * VF::RB + 16 * VF::NB * j, min(16, it.t1 - (it.t0 + 16 * k)), lane_base, r, c);
                 if (++j == tpb || k + 1 == ntiles) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with the slot
@@ -1655,7 +1656,6 @@ __global__ void __launch_bounds__(kPairThreads, 1) decode_pair_kernel(DecodeArgs
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&sm.tmem);
     uint32_t lane_base;
     asm volatile("or.b32 %0, %1, %2;" : "=r"(lane_base) : "r"(lut_addr), "r"(static_cast<uint32_t>(lane) << 2));
-    const uint32_t psel = (r & 1) ? 0x7632u : 0x5410u;
     const int rows = group < NH ? group : NH;
     const int hw = warp & (kBlkWarps - 1), par = warp / kBlkWarps;
     const uint32_t k_sub = bs * (KF::RB + KF::NB), v_sub = bs * (VF::RB + VF::NB);
@@ -1729,20 +1729,20 @@ __global__ void __launch_bounds__(kPairThreads, 1) decode_pair_kernel(DecodeArgs
                             const uint32_t kb1 = sb1 + k_off, vb1 = sb1 + v_off;
                             wt.step2(kb0, kb0 + 16 * KF::RB, vb0, vb0 + 16 * VF::RB, min(16, tok_end - tok0), kb1,
                                      kb1 + 16 * KF::RB, vb1, vb1 + 16 * VF::RB, min(16, tok_end - tok0 - 16),
-                                     lane_base, psel, r, c);
+                                     lane_base, r, c);
                         } else {
                             wt.step(kb0, kb0 + 16 * KF::RB, vb0, vb0 + 16 * VF::RB, min(16, tok_end - tok0),
-                                    lane_base, psel, r, c);
+                                    lane_base, r, c);
                         }
                     } else {
                         if (tok0 + 16 < tok_end)
                             wt.step2(kb0, kb0 + kBs * KF::RB, vb0, vb0 + kBs * VF::RB, 16, kb0 + 16 * KF::RB,
                                      kb0 + kBs * KF::RB + 16 * KF::NB, vb0 + 16 * VF::RB,
-                                     vb0 + kBs * VF::RB + 16 * VF::NB, min(16, tok_end - tok0 - 16), lane_base, psel,
+                                     vb0 + kBs * VF::RB + 16 * VF::NB, min(16, tok_end - tok0 - 16), lane_base,
                                      r, c);
                         else
                             wt.step(kb0, kb0 + kBs * KF::RB, vb0, vb0 + kBs * VF::RB, min(16, tok_end - tok0),
-                                    lane_base, psel, r, c);
+                                    lane_base, r, c);
                     }
                     __syncwarp();
                     if (lane == 0) {  // this warp is done with the slot(s)
@@ -1966,7 +1966,6 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
     }
     uint32_t lane_base;
     asm volatile("or.b32 %0, %1, %2;" : "=r"(lane_base) : "r"(lut_addr), "r"(static_cast<uint32_t>(lane) << 2));
-    const uint32_t psel = (r & 1) ? 0x7632u : 0x5410u;
     const int rows = group < NH ? group : NH;
     const uint32_t my_ring = ring_addr + static_cast<uint32_t>(warp * kStages * kStageBytes);
     uint32_t consumed = 0;
@@ -1992,7 +1991,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_mma_kernel(DecodeArgs
                 // Slot layout: [K rows][K norms][V rows][V norms].
                 const uint32_t kbase = my_ring + st * kStageBytes, vbase = kbase + 16 * (KF::RB + KF::NB);
                 wt.step(kbase, kbase + 16 * KF::RB, vbase, vbase + 16 * VF::RB,
-                        min(16, it.t1 - (it.t0 + 16 * (warp + k * NW))), lane_base, psel, r, c);
+                        min(16, it.t1 - (it.t0 + 16 * (warp + k * NW))), lane_base, r, c);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&sm.empty[warp][st]));  // slot free for the producer
                 ++consumed;
@@ -2239,7 +2238,8 @@ __device__ __forceinline__ void rotate_rows(const DecodeArgs& a, int group, int6
     static_assert(kRotRows == 8 && kProThreads == 2 * kHeadDim, "two halves of four rows");
     const int i = threadIdx.x & (kHeadDim - 1), r0 = (threadIdx.x >> 7) * 4;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 4
+    // 16 loads of S (from L2) in flight per thread: this loop is the prologue's longest chain
+#pragma unroll 16
     for (int j = 0; j < kHeadDim; ++j) {
         const float sij = __ldg(kc.qjl_st + j * kHeadDim + i);  // S^T row j, coalesced over i
 #pragma unroll
@@ -2271,7 +2271,8 @@ __device__ __forceinline__ void rotate_rows_dense(const DecodeArgs& a, int group
 #pragma unroll
     for (int g = 0; g < 16; ++g) acc[g] = 0.0f;
     const int j0 = half * (kHeadDim / 2);
-#pragma unroll 2
+    // 16 loads of R_h (from L2) in flight per thread: this loop is the prologue's longest chain
+#pragma unroll 16
     for (int j = j0; j < j0 + kHeadDim / 2; ++j) {
         const float rjp = __ldg(rt + j * kHeadDim + p);
 #pragma unroll

@@ -127,6 +127,14 @@ WORKLOADS = {
                     "at 4 bits and the other 64 at 3 bits, each group rotated on its own with its own norm, "
                     "128-token bf16 window; group-wise K and V run on the tensor-core kernel "
                     "(query rotated by the dense per-head R_h)"),
+    "decode_llama8b_3p5bit_recipe": Workload(
+        "decode_llama8b_3p5bit_recipe", "decode", 1010, 16, 32, 8, 128, 16, 128,
+        (3, 2), (64, 64), (4, 3), (64, 64), 81, 82, 8, True, "fixed:16384", k_qjl=True, groupwise=True,
+        description="decode batch 16, 32 query / 8 KV heads (Llama-3.1-8B), context 16384, block 16, "
+                    "K in the recipe row as printed: two group-wise groups (64 original channels, the "
+                    "outliers among them, at 3 bits + 64 at 2), each with its QJL signs, norm and residual "
+                    "norm (3.5 bits per channel); V 3.5-bit group-wise; 128-token bf16 window; runs on the "
+                    "general CUDA-core decode kernel"),
 }
 
 

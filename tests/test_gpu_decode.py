@@ -59,6 +59,13 @@ def test_decode_gqa16_and_long_sequence_spans_many_splits():
     check(prob)
 
 
+def test_decode_more_splits_than_combine_threads():
+    """80,000 packed tokens in 512-token splits: 157 split records, more than the combine's 128 threads
+    take in one chunk."""
+    prob = DecodeProblem([80000, 700], 1, 4, U4, U4, window=8, block_size=16, seed=6)
+    check(prob)
+
+
 def test_decode_full_small_workload():
     """The oracle-sized workload in full: 1 sequence, GQA 8, context 4096, 4-bit."""
     w = W.WORKLOADS["decode_gqa8_4k_4bit"]
@@ -164,7 +171,8 @@ def _checked_sequences(layout, bs, n=8):
 
 
 @pytest.mark.parametrize("name", ["decode_llama8b_4bit", "decode_llama70b_3p5bit", "decode_llama8b_2p5bit",
-                                  "decode_llama8b_3p5bit_qjl", "decode_llama8b_3p5bit_groupwise"])
+                                  "decode_llama8b_3p5bit_qjl", "decode_llama8b_3p5bit_groupwise",
+                                  "decode_llama8b_3p5bit_recipe"])
 def test_decode_full_size_workloads(name, monkeypatch):
     """Full-size workloads in the benchmark's launch: every query head of 8 sequences against the
     oracle (element by element), and, on the three headline-format workloads, every output against

@@ -51,9 +51,11 @@ def test_groupwise_pack_matches_oracle(kfmt, vfmt, T, H, bs):
     assert flips <= max(1, MAX_FLIP_FRACTION * total)
 
 
-@pytest.mark.parametrize("H,G,kgw,vgw", [(2, 4, True, True), (8, 8, True, False), (8, 2, False, True)])
+@pytest.mark.parametrize("H,G,kgw,vgw", [(2, 4, True, True), (8, 8, True, False), (8, 2, False, True),
+                                         (2, 16, False, True)])
 def test_groupwise_decode_matches_oracle(H, G, kgw, vgw):
-    """Decode (general kernel) and its combine (the per-group inverse rotation) against the oracle."""
+    """Decode (general kernel) and its combine (the per-group inverse rotation) against the oracle; 16
+    query heads per KV head take the combine's 8 head groups twice."""
     lens = [1, 33, 400, 1900]
     prob = DecodeProblem(lens, H, G, ((4, 2), (32, 96), 61), ((4, 3), (64, 64), 62), window=16, block_size=16,
                          seed=70 + H, kgw=kgw, vgw=vgw)
