@@ -91,13 +91,21 @@ struct Fmt {
 // What a row holds besides its index groups. Plain: one fp16 norm. Group-wise
 // (the high channels are original channels, each group rotated on its own):
 // one fp16 norm per group. QJL keys: the 128 residual sign bits after the
-// index groups, and the norm followed by the residual norm.
-constexpr int kPlain = 0, kGroupwise = 1, kQjl = 2;
+// index groups, and the norm followed by the residual norm. The recipe row
+// (group-wise with a QJL stage per group): each group's indices followed by
+// its sign bits (one per coordinate of the group), and the norms
+// (n_0, |r_0|, n_1, |r_1|).
+constexpr int kPlain = 0, kGroupwise = 1, kQjl = 2, kRecipe = 3;
 template <class F, int MODE_>
 struct Row : F {
     static constexpr int MODE = MODE_;
-    static constexpr int RB = F::IB + (MODE_ == kQjl ? kHeadDim / 8 : 0);  // bytes of an index row
-    static constexpr int NB = MODE_ == kPlain ? 2 : 4;                     // bytes of a row's norms
+    static constexpr bool SIGNS = MODE_ == kQjl || MODE_ == kRecipe;
+    static constexpr int RB = F::IB + (SIGNS ? kHeadDim / 8 : 0);  // bytes of an index row
+    static constexpr int NB = MODE_ == kPlain ? 2 : (MODE_ == kRecipe ? 8 : 4);  // bytes of a row's norms
+    // group 1's indices follow group 0's signs in the recipe row
+    static constexpr int BOFF1 = F::BOFF1 + (MODE_ == kRecipe ? F::N0 / 8 : 0);
+    static constexpr int SO0 = F::BOFF1, SO1 = BOFF1 + F::B1 * F::N1 / 8;  // recipe: each group's sign bits
+    static constexpr int N1OFF = MODE_ == kRecipe ? 4 : 2;  // byte offset of group 1's norm
 };
 using U4 = Row<Fmt<4, 128, 0, 0>, kPlain>;
 using U3 = Row<Fmt<3, 128, 0, 0>, kPlain>;
@@ -106,6 +114,8 @@ using M42 = Row<Fmt<4, 32, 2, 96>, kPlain>;
 using M32Q = Row<Fmt<3, 64, 2, 64>, kQjl>;
 using M43Q = Row<Fmt<4, 64, 3, 64>, kQjl>;
 using M43G = Row<Fmt<4, 64, 3, 64>, kGroupwise>;
+using M32R = Row<Fmt<3, 64, 2, 64>, kRecipe>;
+static_assert(M32R::RB == 56 && M32R::BOFF1 == 32 && M32R::SO0 == 24 && M32R::SO1 == 48, "recipe row layout");
 
 // Bytes of one ring slot: 16 index rows of K followed by their 16 norms, then
 // the same for V; a multiple of 16, the copy granule.
@@ -610,7 +620,10 @@ __device__ __forceinline__ void fill_table(uint32_t* table, const LutValues& tv,
 template <class KF, class VF, int NH, bool TM = false>
 struct WarpTiles {
     static constexpr int HL = NH / 4;  // heads per lane
-    static constexpr bool KQ = KF::MODE == kQjl, KG = KF::MODE == kGroupwise, VG = VF::MODE == kGroupwise;
+    static constexpr bool KR = KF::MODE == kRecipe;
+    static constexpr bool KQ = KF::MODE == kQjl || KR, KG = KF::MODE == kGroupwise || KR,
+                          VG = VF::MODE == kGroupwise;
+    static_assert(!KR || (KF::N0 == 64 && KF::N1 == 64), "recipe keys: two groups of 64");
     static constexpr int NQW = 16 * HL;  // words of the query fragments of one k-step set
     static constexpr uint32_t kTmQ = 0, kTmZ = 32, kTmO = 64, kTmS = 96, kTmCols = 128;
     uint32_t bq[TM ? 1 : 8][2 * HL];             // query B fragments per k-step (registers when !TM)
@@ -674,14 +687,24 @@ struct WarpTiles {
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 // sign k-step s: B rows (2c, 2c+1) and (2c+8, 2c+9) are projections
-                // 32c + s + (0, 16) and 32c + s + (8, 24)
+                // 32c + s + (0, 16) and 32c + s + (8, 24); for the recipe row,
+                // k-step 4g + s' of group g: projections 64g + 16c + s' + (0, 8) and
+                // 64g + 16c + s' + (4, 12)
                 float x0 = 0.0f, x1 = 0.0f, x2 = 0.0f, x3 = 0.0f;
                 if (head < rows) {
-                    const float* z = qz + head * kHeadDim + 32 * c + s;
-                    x0 = __ldcg(z);
-                    x1 = __ldcg(z + 16);
-                    x2 = __ldcg(z + 8);
-                    x3 = __ldcg(z + 24);
+                    if constexpr (KR) {
+                        const float* z = qz + head * kHeadDim + 64 * (s >> 2) + 16 * c + (s & 3);
+                        x0 = __ldcg(z);
+                        x1 = __ldcg(z + 8);
+                        x2 = __ldcg(z + 4);
+                        x3 = __ldcg(z + 12);
+                    } else {
+                        const float* z = qz + head * kHeadDim + 32 * c + s;
+                        x0 = __ldcg(z);
+                        x1 = __ldcg(z + 16);
+                        x2 = __ldcg(z + 8);
+                        x3 = __ldcg(z + 24);
+                    }
                 }
                 uint32_t h01, l01, h23, l23;
                 split2(x0, x1, h01, l01);
@@ -789,23 +812,54 @@ struct WarpTiles {
             // 32c + ...) for its k columns (2c, 2c + 1) and bits (s + 8, s + 24)
             // for (2c + 8, 2c + 9): one shift puts such a pair at bits 15 and 31,
             // the sign bits of the two halves of +-|r| (a clear bit is -).
-            const uint32_t wa = lds32(kbase + r * KF::RB + KF::IB + 4 * c);
-            const uint32_t wb = lds32(kbase + (r + 8) * KF::RB + KF::IB + 4 * c);
-            const uint32_t ga = lds16(knorm + KF::NB * r + 2), gb = lds16(knorm + KF::NB * (r + 8) + 2);
-            const uint32_t rn_a = ga | (ga << 16), rn_b = gb | (gb << 16);
-            static_for<0, 8>([&](auto si) {
-                constexpr int s_ = decltype(si)::value;
-                const uint32_t a0 = rn_a | (~(wa << (15 - s_)) & 0x80008000u);
-                const uint32_t a1 = rn_b | (~(wb << (15 - s_)) & 0x80008000u);
-                const uint32_t a2 = rn_a | (~(wa << (7 - s_)) & 0x80008000u);
-                const uint32_t a3 = rn_b | (~(wb << (7 - s_)) & 0x80008000u);
-                if constexpr (NH == 8) {
-                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, Z[s_][0], Z[s_][1]);
-                    mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, Z[s_][2], Z[s_][3]);
-                } else {
-                    mma16816(sacc[s_ & 1], a0, a1, a2, a3, Z[s_][0], Z[s_][1]);
-                }
-            });
+            if constexpr (KR) {
+                // Recipe row: group g's 64 sign bits follow its indices, lane c takes
+                // projections 16c .. 16c + 15 of the group (bits 16c.. of its stream):
+                // with byte 1 of that half-word moved to byte 2, bits (s', s' + 8) sit 16
+                // apart for k columns (2c, 2c + 1) of k-step s' and bits (s' + 4, s' + 12)
+                // for (2c + 8, 2c + 9). The k-steps of group g accumulate in its chain,
+                // which takes n_g: n_g (q'.c + |r_g| (kappa_g S_g q'_g).z_g).
+                static_for<0, 2>([&](auto gi) {
+                    constexpr int g = decltype(gi)::value;
+                    constexpr int SO = g ? KF::SO1 : KF::SO0;
+                    const uint32_t wa = prmt(lds16(kbase + r * KF::RB + SO + 2 * c), 0u, 0x4140u);
+                    const uint32_t wb = prmt(lds16(kbase + (r + 8) * KF::RB + SO + 2 * c), 0u, 0x4140u);
+                    const uint32_t ga = lds16(knorm + KF::NB * r + 2 + 4 * g);
+                    const uint32_t gb = lds16(knorm + KF::NB * (r + 8) + 2 + 4 * g);
+                    const uint32_t rn_a = ga | (ga << 16), rn_b = gb | (gb << 16);
+                    static_for<0, 4>([&](auto si) {
+                        constexpr int s_ = decltype(si)::value;
+                        const uint32_t a0 = rn_a | (~(wa << (15 - s_)) & 0x80008000u);
+                        const uint32_t a1 = rn_b | (~(wb << (15 - s_)) & 0x80008000u);
+                        const uint32_t a2 = rn_a | (~(wa << (11 - s_)) & 0x80008000u);
+                        const uint32_t a3 = rn_b | (~(wb << (11 - s_)) & 0x80008000u);
+                        if constexpr (NH == 8) {
+                            mma16816(sacc[g], a0, a1, a2, a3, Z[4 * g + s_][0], Z[4 * g + s_][1]);
+                            mma16816(sacc[2 + g], a0, a1, a2, a3, Z[4 * g + s_][2], Z[4 * g + s_][3]);
+                        } else {
+                            mma16816(sacc[g], a0, a1, a2, a3, Z[4 * g + s_][0], Z[4 * g + s_][1]);
+                        }
+                    });
+                });
+            } else {
+                const uint32_t wa = lds32(kbase + r * KF::RB + KF::IB + 4 * c);
+                const uint32_t wb = lds32(kbase + (r + 8) * KF::RB + KF::IB + 4 * c);
+                const uint32_t ga = lds16(knorm + KF::NB * r + 2), gb = lds16(knorm + KF::NB * (r + 8) + 2);
+                const uint32_t rn_a = ga | (ga << 16), rn_b = gb | (gb << 16);
+                static_for<0, 8>([&](auto si) {
+                    constexpr int s_ = decltype(si)::value;
+                    const uint32_t a0 = rn_a | (~(wa << (15 - s_)) & 0x80008000u);
+                    const uint32_t a1 = rn_b | (~(wb << (15 - s_)) & 0x80008000u);
+                    const uint32_t a2 = rn_a | (~(wa << (7 - s_)) & 0x80008000u);
+                    const uint32_t a3 = rn_b | (~(wb << (7 - s_)) & 0x80008000u);
+                    if constexpr (NH == 8) {
+                        mma16816(sacc[s_ & 1], a0, a1, a2, a3, Z[s_][0], Z[s_][1]);
+                        mma16816(sacc[2 + (s_ & 1)], a0, a1, a2, a3, Z[s_][2], Z[s_][3]);
+                    } else {
+                        mma16816(sacc[s_ & 1], a0, a1, a2, a3, Z[s_][0], Z[s_][1]);
+                    }
+                });
+            }
         }
         if constexpr (kOwnLoads) {
             tm_ld<NQW>(tm + kTmQ, &ql[0][0]);
@@ -849,7 +903,7 @@ struct WarpTiles {
         const bool ok0 = r < nvalid, ok1 = r + 8 < nvalid;
         if constexpr (NH == 8 && KG) {
             // chains 0 / 2: group 0 hi / lo; chains 1 / 3: group 1
-            const float mk0 = f16_at(knorm + KF::NB * r + 2), mk1 = f16_at(knorm + KF::NB * (r + 8) + 2);
+            const float mk0 = f16_at(knorm + KF::NB * r + KF::N1OFF), mk1 = f16_at(knorm + KF::NB * (r + 8) + KF::N1OFF);
             float x0, x1, y0, y1;
             upk(add2(mul2(add2(pk(sacc[0][0], sacc[0][1]), pk(sacc[2][0], sacc[2][1])), pk(nk0, nk0)),
                      mul2(add2(pk(sacc[1][0], sacc[1][1]), pk(sacc[3][0], sacc[3][1])), pk(mk0, mk0))),
@@ -877,7 +931,7 @@ struct WarpTiles {
             sc[HL - 1][1] = ok1 ? y1 : -INFINITY;
         } else if constexpr (KG) {
             // chain 0: group 0 (hi, lo columns); chain 1: group 1
-            const float mk0 = f16_at(knorm + KF::NB * r + 2), mk1 = f16_at(knorm + KF::NB * (r + 8) + 2);
+            const float mk0 = f16_at(knorm + KF::NB * r + KF::N1OFF), mk1 = f16_at(knorm + KF::NB * (r + 8) + KF::N1OFF);
             sc[0][0] = ok0 ? (sacc[0][0] + sacc[0][1]) * nk0 + (sacc[1][0] + sacc[1][1]) * mk0 : -INFINITY;
             sc[0][1] = ok1 ? (sacc[0][2] + sacc[0][3]) * nk1 + (sacc[1][2] + sacc[1][3]) * mk1 : -INFINITY;
         } else {
@@ -2053,6 +2107,7 @@ union ProSmem {
     struct {
         float qs[16][kHeadDim];    // group-wise: the head's query rows
         float part[16][kHeadDim];  // second half's partial products
+        float qr[16][kHeadDim];    // recipe keys: the rotated rows
     } dense;
     struct {
         float m[kProWarps][8], l[kProWarps][8];
@@ -2257,6 +2312,7 @@ __device__ __forceinline__ void rotate_rows(const DecodeArgs& a, int group, int6
 // shared memory, thread (p, half) sums packed position p of every row over
 // half of the j range, and the CTA reads R_h (64 KB, rows contiguous over p)
 // once.
+template <bool RECIPE>
 __device__ __forceinline__ void rotate_rows_dense(const DecodeArgs& a, int group, int64_t unit, ProSmem& sm) {
     const DevCodec& kc = a.kc;
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
@@ -2288,7 +2344,25 @@ __device__ __forceinline__ void rotate_rows_dense(const DecodeArgs& a, int group
     if (!half) {
 #pragma unroll
         for (int g = 0; g < 16; ++g)
-            if (g < group) a.qrot[(row0 + g) * kHeadDim + p] = (acc[g] + sm.dense.part[g][p]) * a.scale_log2;
+            if (g < group) {
+                const float y = (acc[g] + sm.dense.part[g][p]) * a.scale_log2;
+                a.qrot[(row0 + g) * kHeadDim + p] = y;
+                if constexpr (RECIPE) sm.dense.qr[g][p] = y;
+            }
+    }
+    if constexpr (RECIPE) {
+        // Per group g of 64 packed positions: (kappa S_g q'_g)_i = kappa sum_j S_g^T[j][i] q'[64g + j],
+        // kappa = sqrt(pi/2)/64, written at packed position 64g + i (S_0^T then S_1^T in the codec).
+        __syncthreads();
+        constexpr float kappa = 1.2533141373155003f / 64.0f;
+        const int grp = p >> 6, i = p & 63;
+        const float* st = kc.qjl_st + grp * 64 * 64;
+        for (int g = half; g < group; g += 2) {
+            float z = 0.0f;
+#pragma unroll 16
+            for (int j = 0; j < 64; ++j) z = fmaf(__ldg(st + j * 64 + i), sm.dense.qr[g][64 * grp + j], z);
+            a.qjl_q[(row0 + g) * kHeadDim + p] = z * kappa;
+        }
     }
 }
 
@@ -2305,8 +2379,8 @@ __global__ void __launch_bounds__(kProThreads, NH == 4 ? 2 : 1) decode_prologue_
     if (blk == 0) {
         build_work_list(a, sm);
     } else if (blk <= n_rot) {
-        if constexpr (KMODE == kGroupwise)
-            rotate_rows_dense(a, group, blk - 1, sm);
+        if constexpr (KMODE == kGroupwise || KMODE == kRecipe)
+            rotate_rows_dense<KMODE == kRecipe>(a, group, blk - 1, sm);
         else
             rotate_rows(a, group, static_cast<int64_t>(a.batch) * a.num_q_heads, blk - 1,
                         KMODE == kQjl ? a.qjl_q : nullptr, sm);
@@ -2363,7 +2437,7 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     const int head_groups = group > 8 ? group / 8 : 1;
     const int64_t rows = static_cast<int64_t>(a.batch) * a.num_q_heads;
     // One prologue launch builds the work list, rotates the queries and attends over the windows.
-    const int64_t n_rot = KF::MODE == kGroupwise ? static_cast<int64_t>(a.batch) * a.kc.num_heads
+    const int64_t n_rot = (KF::MODE == kGroupwise || KF::MODE == kRecipe) ? static_cast<int64_t>(a.batch) * a.kc.num_heads
                                                  : (rows + kRotRows - 1) / kRotRows;
     const int64_t n_win = a.window > 0 ? static_cast<int64_t>(a.batch) * a.kc.num_heads * head_groups : 0;
     if (1 + n_rot + n_win > INT32_MAX) return TQ_ERR_UNSUPPORTED;
@@ -2409,9 +2483,14 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
 template <class F>
 bool same_format(const tq_codec* c) {
     const tq_format_desc& d = c->desc;
-    if (d.qjl && d.groupwise) return false;  // the recipe row runs on the general kernel
-    const int mode = d.qjl ? kQjl : (d.groupwise ? kGroupwise : kPlain);
+    const int mode = d.qjl ? (d.groupwise ? kRecipe : kQjl) : (d.groupwise ? kGroupwise : kPlain);
     if (mode != F::MODE) return false;
+    if constexpr (F::MODE == kRecipe) {
+        // the kernel's compile-time row layout must be the codec's
+        if (!c->dev.recipe || c->dev.sign_off[0] != F::SO0 || c->dev.sign_off[1] != F::SO1 ||
+            c->dev.byte_off[1] != F::BOFF1 || c->dev.row_bytes != F::RB + F::NB)
+            return false;
+    }
     if (F::N1 == 0) return d.n_groups == 1 && d.group_bits[0] == F::B0;
     return d.n_groups == 2 && d.group_bits[0] == F::B0 && d.group_size[0] == F::N0 && d.group_bits[1] == F::B1 &&
            d.group_size[1] == F::N1;
@@ -2425,7 +2504,7 @@ tq_status launch_heads(const DecodeArgs& a, const LutValues& tv, int group, cuda
 // V formats the tensor-core kernel is instantiated for, per K format.
 template <class KF>
 tq_status dispatch_v(const DecodeArgs& a, const tq_codec* vc, const LutValues& tv, int group, cudaStream_t s) {
-    if constexpr (KF::MODE == kGroupwise) {
+    if constexpr (KF::MODE == kGroupwise || KF::MODE == kRecipe) {
         if (same_format<M43G>(vc)) return launch_heads<KF, M43G>(a, tv, group, s);
     } else if constexpr (KF::MODE == kQjl) {
         if (same_format<U4>(vc)) return launch_heads<KF, U4>(a, tv, group, s);
@@ -2466,6 +2545,7 @@ tq_status launch_decode_mma(const DecodeArgs& a, const tq_codec* kc, const tq_co
     if (same_format<M32Q>(kc)) return dispatch_v<M32Q>(a, vc, tv, group, s);
     if (same_format<M43Q>(kc)) return dispatch_v<M43Q>(a, vc, tv, group, s);
     if (same_format<M43G>(kc)) return dispatch_v<M43G>(a, vc, tv, group, s);
+    if (same_format<M32R>(kc)) return dispatch_v<M32R>(a, vc, tv, group, s);
     return TQ_ERR_UNSUPPORTED;
 }
 

@@ -92,6 +92,37 @@ def test_recipe_decode_matches_oracle(H, G, bs):
     assert worst <= 2e-3, worst
 
 
+@pytest.mark.parametrize("H,G,bs", [(8, 4, 16), (8, 8, 32), (2, 16, 16), (3, 2, 48)])
+def test_recipe_decode_tensor_core_matches_oracle_and_general(monkeypatch, H, G, bs):
+    """Recipe-row keys in the tensor-core formats (3/2-bit 64/64 groups, each with its QJL signs and
+    residual norm; group-wise 4/3-bit values): TQ_DECODE_KERNEL=tensor fails unless the tensor-core
+    kernel runs it. Paired, block and per-head layouts against the general kernel and the oracle."""
+    lens = [1, 17, 300, 2100, 5000]
+    prob = DecodeProblem(lens, H, G, ((3, 2), (64, 64), 63), ((4, 3), (64, 64), 64), window=8, block_size=bs,
+                         seed=40 + H + G, kqjl=True, kgw=True, vgw=True)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "tensor")
+    fast = prob.run(d_err=err).clone()
+    monkeypatch.setenv("TQ_DECODE_PAIR", "0")
+    block = prob.run(d_err=err).clone()
+    monkeypatch.delenv("TQ_DECODE_PAIR")
+    monkeypatch.setenv("TQ_DECODE_KERNEL", "general")
+    general = prob.run(d_err=err).clone()
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert (fast - general).abs().max().item() <= 2e-3
+    assert (block - general).abs().max().item() <= 2e-3
+    got = fast.cpu().numpy()
+    rng = np.random.default_rng(H * G)
+    worst = 0.0
+    for b in range(prob.B):
+        for hq in rng.choice(prob.Hq, min(prob.Hq, 6), replace=False):
+            ref = prob.oracle(b, int(hq))
+            worst = max(worst, float(np.abs(got[b, hq] - ref).max()))
+            assert np.abs(ref).max() > 0.3
+    assert worst <= 2e-3, worst
+
+
 def test_recipe_window_append_rows_equal_pack():
     """tq_window_append packs an evicted token through the same routine: the row it writes for the
     recipe format equals the row tq_pack_kv writes for that token."""
