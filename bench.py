@@ -751,6 +751,8 @@ def run_ours(args):
                 sb = setup.decode_split_bytes()
                 extra[name] = {"GB/s": setup.step_bytes() / (ms * 1e-3) / 1e9,
                                "kv_tokens_per_s": setup.kv_tokens() / (ms * 1e-3), "ms_per_step": ms,
+                               "step_breakdown_ms": {"window_append": p[0], "decode_partials": p[1],
+                                                     "decode_combine": p[2]},
                                "decode_partials_GB/s": sb / (p[1] * 1e-3) / 1e9,
                                "decode_partials_frac": sb / (p[1] * 1e-3) / 1e9 / peak,
                                "traffic": stored_traffic(name, "tq_decode_mma.cu")}

@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, c
                                                                    int32_t window, int32_t split_tokens,
                                                                    int32_t max_splits, int32_t items_per_unit,
                                                                    int32_t G, const float* ws, float* out) {
-    __shared__ float y[kHeadDim];
+    __shared__ float y[kHeadDim], y2[kHeadDim];
     __shared__ float red[4];
     // Launched as a dependent of the partials: the split records are read only after they are complete.
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -380,13 +380,27 @@ __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, c
     } else {
         y[vc.perm[h * kHeadDim + j]] = rot;  // back to rotated coordinate order
         __syncthreads();
-        for (int len = 1; len < kHeadDim; len <<= 1) {  // Walsh-Hadamard, natural order
-            float mine = y[j], other = y[j ^ len];
-            __syncthreads();
-            y[j] = (j & len) ? (other - mine) : (mine + other);
-            __syncthreads();
+        // Walsh-Hadamard, natural order: strides 1 .. 16 inside a warp by shuffles, 32 and 64
+        // through shared memory (y2, then y again: y was last read before the first barrier)
+        float v = y[j];
+#pragma unroll
+        for (int len = 1; len < 32; len <<= 1) {
+            const float o = __shfl_xor_sync(kFull, v, len);
+            v = (j & len) ? (o - v) : (v + o);
         }
-        x = vc.sign[j] * y[j] * 0.08838834764831845f;
+        y2[j] = v;
+        __syncthreads();
+        {
+            const float o = y2[j ^ 32];
+            v = (j & 32) ? (o - v) : (v + o);
+        }
+        y[j] = v;
+        __syncthreads();
+        {
+            const float o = y[j ^ 64];
+            v = (j & 64) ? (o - v) : (v + o);
+        }
+        x = vc.sign[j] * v * 0.08838834764831845f;
     }
     out[(static_cast<int64_t>(b) * num_q_heads + hq) * kHeadDim + j] = Ls > 0.0f ? (x + win) / Ls : 0.0f;
 }
@@ -411,8 +425,16 @@ __global__ void __launch_bounds__(kHeadDim * kGwHeads) decode_combine_gw_kernel(
     const int H = vc.num_heads, h = blockIdx.x % H, b = blockIdx.x / H;
     const int j = threadIdx.x & (kHeadDim - 1), gl = threadIdx.x >> 7, nthreads = blockDim.x;
     const float* rt = vc.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim;
-    for (int e = threadIdx.x; e < kHeadDim * kHeadDim; e += nthreads)
-        rts[(e >> 7) * kGwPitch + (e & (kHeadDim - 1))] = rt[e];
+    // 16-byte loads, eight in flight per thread (R_h^T comes from L2)
+#pragma unroll 8
+    for (int e4 = threadIdx.x; e4 < kHeadDim * kHeadDim / 4; e4 += nthreads) {
+        const float4 v4 = __ldg(reinterpret_cast<const float4*>(rt) + e4);
+        float* d = rts + (e4 >> 5) * kGwPitch + 4 * (e4 & 31);
+        d[0] = v4.x;
+        d[1] = v4.y;
+        d[2] = v4.z;
+        d[3] = v4.w;
+    }
     // Launched as a dependent of the partials: R_h^T is staged while they end; the split records are
     // read only after they are complete.
     asm volatile("griddepcontrol.wait;" ::: "memory");

@@ -617,6 +617,20 @@ __device__ __forceinline__ void fill_table(uint32_t* table, const LutValues& tv,
 // tensor-memory columns between uses (query fragments at kTmQ, QJL fragments
 // at kTmZ, accumulators at kTmO, the merge state at kTmS) and in registers
 // only inside scores() and values(), so the two sets are never live at once.
+// Where the prologue stores projection i of the projected query, so that a
+// lane's four B-fragment values of a sign k-step are one 16-byte load. QJL
+// keys: lane c's k-step s takes projections 32c + s + (0, 16, 8, 24), stored
+// at 32c + 4s + (0, 1, 2, 3). Recipe keys: group g's k-step s' in lane c takes
+// 64g + 16c + s' + (0, 8, 4, 12), stored at 64g + 16c + 4s' + (0, 1, 2, 3).
+__device__ __forceinline__ int qjl_slot(int i) {
+    const int rem = i & 31, t = ((rem >> 3) & 1) * 2 + (rem >> 4);
+    return (i & ~31) + 4 * (rem & 7) + t;
+}
+__device__ __forceinline__ int recipe_slot(int p) {
+    const int rem = p & 15, t = ((rem >> 2) & 1) * 2 + (rem >> 3);
+    return (p & ~15) + 4 * (rem & 3) + t;
+}
+
 template <class KF, class VF, int NH, bool TM = false>
 struct WarpTiles {
     static constexpr int HL = NH / 4;  // heads per lane
@@ -683,6 +697,9 @@ struct WarpTiles {
         const int head = NH == 8 ? r : (r >> 1);
         uint32_t qf[8][2 * HL];
         uint32_t zf[KQ ? 8 : 1][2 * HL];
+        // With tensor memory each fragment set is stored as soon as it is built, so the two sets
+        // are never live in registers together.
+        if constexpr (TM) tm_wait_st();  // the last item's stores have landed before these columns are rewritten
         if constexpr (KQ) {
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
@@ -692,19 +709,13 @@ struct WarpTiles {
                 // 64g + 16c + s' + (4, 12)
                 float x0 = 0.0f, x1 = 0.0f, x2 = 0.0f, x3 = 0.0f;
                 if (head < rows) {
-                    if constexpr (KR) {
-                        const float* z = qz + head * kHeadDim + 64 * (s >> 2) + 16 * c + (s & 3);
-                        x0 = __ldcg(z);
-                        x1 = __ldcg(z + 8);
-                        x2 = __ldcg(z + 4);
-                        x3 = __ldcg(z + 12);
-                    } else {
-                        const float* z = qz + head * kHeadDim + 32 * c + s;
-                        x0 = __ldcg(z);
-                        x1 = __ldcg(z + 16);
-                        x2 = __ldcg(z + 8);
-                        x3 = __ldcg(z + 24);
-                    }
+                    // the four projections are adjacent in the stored order (qjl_slot, recipe_slot)
+                    const int at = KR ? 64 * (s >> 2) + 16 * c + 4 * (s & 3) : 32 * c + 4 * s;
+                    const float4 z4 = __ldcg(reinterpret_cast<const float4*>(qz + head * kHeadDim + at));
+                    x0 = z4.x;
+                    x1 = z4.y;
+                    x2 = z4.z;
+                    x3 = z4.w;
                 }
                 uint32_t h01, l01, h23, l23;
                 split2(x0, x1, h01, l01);
@@ -719,6 +730,7 @@ struct WarpTiles {
                     zf[s][1] = (r & 1) ? l23 : h23;
                 }
             }
+            if constexpr (TM) tm_st<NQW>(tm + kTmZ, &zf[0][0]);
         }
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
@@ -743,9 +755,7 @@ struct WarpTiles {
 #pragma unroll
         for (int q = 0; q < 8; ++q) o[q][0] = o[q][1] = o[q][2] = o[q][3] = 0.0f;
         if constexpr (TM) {
-            tm_wait_st();  // the last item's accumulators have landed before they are overwritten
             tm_st<NQW>(tm + kTmQ, &qf[0][0]);
-            if constexpr (KQ) tm_st<NQW>(tm + kTmZ, &zf[0][0]);
             tm_st<32>(tm + kTmO, reinterpret_cast<const uint32_t*>(&o[0][0]));
             tm_wait_st();
         } else {
@@ -2303,7 +2313,7 @@ __device__ __forceinline__ void rotate_rows(const DecodeArgs& a, int group, int6
     constexpr float kappa = 1.2533141373155003f / kHeadDim;  // sqrt(pi/2) / d, the estimator's constant
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-        if (row0 + r0 + k < total) qjl_out[(row0 + r0 + k) * kHeadDim + i] = acc[k] * kappa;
+        if (row0 + r0 + k < total) qjl_out[(row0 + r0 + k) * kHeadDim + qjl_slot(i)] = acc[k] * kappa;
 }
 
 // Group-wise K: q_r = R_h q * scale * log2(e) in packed order (R_h from the
@@ -2361,7 +2371,7 @@ __device__ __forceinline__ void rotate_rows_dense(const DecodeArgs& a, int group
             float z = 0.0f;
 #pragma unroll 16
             for (int j = 0; j < 64; ++j) z = fmaf(__ldg(st + j * 64 + i), sm.dense.qr[g][64 * grp + j], z);
-            a.qjl_q[(row0 + g) * kHeadDim + p] = z * kappa;
+            a.qjl_q[(row0 + g) * kHeadDim + recipe_slot(p)] = z * kappa;
         }
     }
 }
