@@ -328,10 +328,20 @@ def percentiles(xs):
 
 
 def measure_decode(setup: DecodeSetup, steps, warmup, dist_ctx=None, clocks=True):
+    """The step (window append, then the whole decode call) timed with events only between steps, as
+    a caller runs it: an event between two kernels would stop the later one from launching while the
+    earlier one ends. The phase breakdown (append, partials, combine) comes from a second pass with
+    events between the phases."""
     stream = torch.cuda.current_stream()
-    fns = [setup.pack, lambda: setup.decode("partials"), lambda: setup.decode("combine")]
+    phases = [setup.pack, lambda: setup.decode("partials"), lambda: setup.decode("combine")]
+
+    def step():
+        setup.pack()
+        setup.decode("all")
+
     for _ in range(warmup):
-        for f in fns:
+        step()
+        for f in phases:
             f()
     torch.cuda.synchronize()
     if setup.err.item():
@@ -340,9 +350,10 @@ def measure_decode(setup: DecodeSetup, steps, warmup, dist_ctx=None, clocks=True
     sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
     if sampler:
         sampler.__enter__()
-    total_ms, parts, per_step = time_steps(fns, steps, stream)
+    total_ms, _, per_step = time_steps([step], steps, stream)
     if sampler:
         sampler.__exit__(None, None, None)
+    _, parts, _ = time_steps(phases, steps, stream)
     barrier(dist_ctx)
     total_ms = max_over_ranks(total_ms, dist_ctx)
     return total_ms / steps, parts, (sampler.summary() if sampler else None), per_step

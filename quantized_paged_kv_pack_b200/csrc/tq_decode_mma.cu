@@ -2385,6 +2385,9 @@ __global__ void __launch_bounds__(kProThreads, NH == 4 ? 2 : 1) decode_prologue_
                                                                       int64_t n_rot) {
     __shared__ ProSmem sm;
     griddep_launch_dependents();
+    // Launched as a dependent of whatever ran before in the stream (the step's window append, say):
+    // nothing is read before that kernel is complete; only the launch overlaps its end.
+    griddep_wait();
     const int64_t blk = blockIdx.x;
     if (blk == 0) {
         build_work_list(a, sm);
@@ -2451,8 +2454,10 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
                                                  : (rows + kRotRows - 1) / kRotRows;
     const int64_t n_win = a.window > 0 ? static_cast<int64_t>(a.batch) * a.kc.num_heads * head_groups : 0;
     if (1 + n_rot + n_win > INT32_MAX) return TQ_ERR_UNSUPPORTED;
-    decode_prologue_kernel<KF::MODE, NH><<<static_cast<unsigned>(1 + n_rot + n_win), kProThreads, 0, s>>>(
-        a, group, head_groups, n_rot);
+    const cudaError_t pe = launch_dependent(decode_prologue_kernel<KF::MODE, NH>,
+                                            dim3(static_cast<unsigned>(1 + n_rot + n_win)), dim3(kProThreads), 0, s,
+                                            a, group, head_groups, n_rot);
+    if (pe != cudaSuccess) return fail(TQ_ERR_CUDA, std::string("decode prologue launch: ") + cudaGetErrorString(pe));
     const int64_t units = static_cast<int64_t>(a.items_per_unit) * a.batch * head_groups *
                           (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);
     const int grid = static_cast<int>(units < sms ? units : sms);

@@ -364,6 +364,8 @@ window_append_kernel(DevCodec kc, DevCodec vc, const __nv_bfloat16* __restrict__
                      int* __restrict__ d_err) {
     __shared__ uint8_t idx_buf[kPackWarps][kHeadDim];
     __shared__ float r_buf[kPackWarps][kHeadDim];
+    // A decode call that follows may launch its first kernel now; that kernel waits for this one.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = kc.num_heads;
     const int64_t n_vec = static_cast<int64_t>(batch) * H * 2;
