@@ -37,7 +37,7 @@ from quantized_paged_kv_pack_b200 import workloads as WL  # noqa: E402
 
 HEADLINE = "decode_llama70b_3p5bit"
 SMALL = "decode_gqa8_4k_4bit"
-DECODE_LAUNCHES = 4  # per step: window append, prologue (work list, query rotation, windows), partials, combine
+DECODE_LAUNCHES = 3  # per step: prologue (work list, query rotation, windows, the append), decode, combine
 EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl",
          "decode_llama8b_3p5bit_groupwise", "decode_llama8b_3p5bit_recipe",
          "pack_llama8b_4bit", "pack_llama70b_3p5bit", "pack_llama8b_2p5bit"]
@@ -165,6 +165,16 @@ class DecodeSetup:
         tq.window_append(self.kc, self.vc, self.new_k if k is None else k, self.new_v if v is None else v,
                          self.kw if w.window else None, self.vw if w.window else None, w.window, 0, self.sl,
                          self.bt, self.kp, self.vp, w.block_size, d_err=self.err)
+
+    def step(self, k=None, v=None, q=None, out=None):
+        """The whole step in one call: tq_window_append_decode (the append runs in the decode's first
+        kernel; the results are those of pack() then decode())."""
+        w = self.w
+        return tq.window_append_decode(self.kc, self.vc, self.new_k if k is None else k,
+                                       self.new_v if v is None else v, self.kw if w.window else None,
+                                       self.vw if w.window else None, w.window, 0, self.q if q is None else q,
+                                       self.kp, self.vp, w.block_size, self.bt, self.sl, self.max_len, self.scale,
+                                       out=self.out if out is None else out, workspace=self.ws, d_err=self.err)
 
     def decode(self, phase="all", q=None, out=None):
         w = self.w
@@ -328,16 +338,13 @@ def percentiles(xs):
 
 
 def measure_decode(setup: DecodeSetup, steps, warmup, dist_ctx=None, clocks=True):
-    """The step (window append, then the whole decode call) timed with events only between steps, as
-    a caller runs it: an event between two kernels would stop the later one from launching while the
-    earlier one ends. The phase breakdown (append, partials, combine) comes from a second pass with
-    events between the phases."""
+    """The step (tq_window_append_decode: the window append and the decode call in three launches)
+    timed with events only between steps, as a caller runs it: an event between two kernels would stop
+    the later one from launching while the earlier one ends. The phase breakdown (append, partials,
+    combine, as three separate calls) comes from a second pass with events between the phases."""
     stream = torch.cuda.current_stream()
     phases = [setup.pack, lambda: setup.decode("partials"), lambda: setup.decode("combine")]
-
-    def step():
-        setup.pack()
-        setup.decode("all")
+    step = setup.step
 
     for _ in range(warmup):
         step()
@@ -402,8 +409,7 @@ def measure_decode_e2e(setup: DecodeSetup, steps, warmup):
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
-        setup.pack(dk, dv)
-        setup.decode("all", q=dq, out=dout)
+        setup.step(dk, dv, q=dq, out=dout)
         hout.copy_(dout, non_blocking=True)
 
     for _ in range(warmup):

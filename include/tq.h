@@ -249,6 +249,27 @@ tq_status tq_window_append(const tq_codec* kc, const tq_codec* vc, const void* k
                            int64_t num_blocks, int32_t block_size, int32_t batch, int32_t* d_err, void* stream);
 
 /*
+ * tq_window_append_decode - one decode step: tq_window_append followed by
+ * tq_decode_paged on the same stream, with window' = sinks + window and the
+ * same seq_lens (the lengths before the append), in fewer launches. The
+ * append runs inside the decode's first kernel; that kernel's window
+ * attention reads the new token from k_new / v_new for the dense slot it
+ * takes, and the decode reads the pages only after the append is complete.
+ * The results (out, the dense buffers, the pages, d_err) are those of the two
+ * calls. Formats without a tensor-core decode run the two calls as they are.
+ * Arguments mean what they mean for tq_window_append and tq_decode_paged;
+ * the workspace is sized for window' = sinks + window.
+ * This library's own extension: the pages describe the step, not the call.
+ */
+tq_status tq_window_append_decode(const tq_codec* kc, const tq_codec* vc, const void* k_new, const void* v_new,
+                                  void* k_win, void* v_win, int32_t window, int32_t sinks, const void* q,
+                                  void* k_pages, void* v_pages, const int32_t* block_tables,
+                                  int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch,
+                                  int32_t num_q_heads, int32_t max_seq_len, float softmax_scale, int64_t num_blocks,
+                                  int32_t block_size, float* out, void* workspace, size_t workspace_bytes,
+                                  int32_t* d_err, void* stream);
+
+/*
  * Workspace bytes that tq_decode_paged needs for these sizes; bounded by the
  * runtime shape ([Design] "Serving Route Design": keep workspace bounded).
  * Returns 0 for invalid sizes.

@@ -516,13 +516,25 @@ tq_status finish(cudaStream_t s, int32_t* d_err, const char* what) {
 
 using namespace tq;
 
-extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
-                                        const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
-                                        const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
-                                        int32_t max_seq_len, const void* k_win, const void* v_win, int32_t window,
-                                        float softmax_scale, int64_t num_blocks, int32_t block_size,
-                                        void* workspace, size_t workspace_bytes, int32_t* d_err, void* stream) {
-    clear_error();
+namespace tq {
+namespace {
+// The step's window append, fused into the decode prologue (tq_window_append_decode).
+struct FusedAppend {
+    const void* k_new;
+    const void* v_new;
+    void* k_win;
+    void* v_win;
+    void* k_pages;
+    void* v_pages;
+    int32_t window, sinks;  // the append's W and S; the decode's window is S + W
+};
+
+tq_status decode_partials_impl(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
+                               const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t max_seq_len,
+                               const void* k_win, const void* v_win, int32_t window, float softmax_scale,
+                               int64_t num_blocks, int32_t block_size, void* workspace, size_t workspace_bytes,
+                               int32_t* d_err, void* stream, const FusedAppend* app) {
     SplitPlan plan;
     tq_status st = check_decode_args(kc, vc, batch, num_q_heads, max_seq_len, window, block_size, workspace_bytes,
                                      workspace, &plan);
@@ -540,7 +552,7 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
         return fail(TQ_ERR_VALUE, "q and the windows must be 8-byte aligned");
     if (static_cast<int64_t>(max_blocks_per_seq) * block_size < static_cast<int64_t>(max_seq_len) - window)
         return fail(TQ_ERR_VALUE, "max_blocks_per_seq * block_size cannot hold max_seq_len - window tokens");
-    DecodeArgs a;
+    DecodeArgs a{};
     a.kc = kc->dev;
     a.vc = vc->dev;
     a.q = q;
@@ -569,6 +581,17 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
     a.d_err = d_err;
     const char* withhold = std::getenv("TQ_TEST_WITHHOLD_COPIES");
     a.withhold_copies = withhold && std::string(withhold) == "1";
+    if (app) {
+        a.app_on = 1;
+        a.k_new = app->k_new;
+        a.v_new = app->v_new;
+        a.k_win_w = app->k_win;
+        a.v_win_w = app->v_win;
+        a.k_pages_w = static_cast<uint8_t*>(app->k_pages);
+        a.v_pages_w = static_cast<uint8_t*>(app->v_pages);
+        a.app_window = app->window;
+        a.app_sinks = app->sinks;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // Tensor-core kernel for the formats it is instantiated for (block sizes a
     // multiple of 16); the general kernel covers every other valid format.
@@ -583,6 +606,14 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
         if (forced == "tensor") return fail(TQ_ERR_UNSUPPORTED, "no tensor-core decode for these formats");
         clear_error();
     }
+    if (app) {
+        // the general kernel takes no fused append: append first, as a separate launch
+        st = tq_window_append(kc, vc, app->k_new, app->v_new, app->k_win, app->v_win, app->window, app->sinks,
+                              seq_lens, block_tables, max_blocks_per_seq, app->k_pages, app->v_pages, num_blocks,
+                              block_size, batch, d_err, stream);
+        if (st != TQ_OK) return st;
+        a.app_on = 0;
+    }
     dim3 grid(plan.items_per_unit, kc->desc.num_kv_heads, batch);
     switch (plan.group) {
         case 1: decode_partials_kernel<1><<<grid, kWarps * 32, 0, s>>>(a); break;
@@ -592,6 +623,20 @@ extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, 
         default: decode_partials_kernel<16><<<grid, kWarps * 32, 0, s>>>(a); break;
     }
     return finish(s, d_err, "decode partials");
+}
+}  // namespace
+}  // namespace tq
+
+extern "C" tq_status tq_decode_partials(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,
+                                        const void* v_pages, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                        const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                        int32_t max_seq_len, const void* k_win, const void* v_win, int32_t window,
+                                        float softmax_scale, int64_t num_blocks, int32_t block_size,
+                                        void* workspace, size_t workspace_bytes, int32_t* d_err, void* stream) {
+    clear_error();
+    return decode_partials_impl(kc, vc, q, k_pages, v_pages, block_tables, max_blocks_per_seq, seq_lens, batch,
+                                num_q_heads, max_seq_len, k_win, v_win, window, softmax_scale, num_blocks, block_size,
+                                workspace, workspace_bytes, d_err, stream, nullptr);
 }
 
 extern "C" tq_status tq_decode_combine(const tq_codec* vc, const int32_t* seq_lens, int32_t batch,
@@ -627,6 +672,31 @@ extern "C" tq_status tq_decode_combine(const tq_codec* vc, const int32_t* seq_le
         if (e != cudaSuccess) return fail(TQ_ERR_CUDA, std::string("combine launch: ") + cudaGetErrorString(e));
     }
     return finish(s, nullptr, "decode combine");
+}
+
+extern "C" tq_status tq_window_append_decode(const tq_codec* kc, const tq_codec* vc, const void* k_new,
+                                             const void* v_new, void* k_win, void* v_win, int32_t window,
+                                             int32_t sinks, const void* q, void* k_pages, void* v_pages,
+                                             const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                             const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                             int32_t max_seq_len, float softmax_scale, int64_t num_blocks,
+                                             int32_t block_size, float* out, void* workspace, size_t workspace_bytes,
+                                             int32_t* d_err, void* stream) {
+    clear_error();
+    tq_status st = validate_window_append(kc, vc, k_new, v_new, k_win, v_win, window, sinks, seq_lens, block_tables,
+                                          max_blocks_per_seq, k_pages, v_pages, num_blocks, block_size, batch);
+    if (st != TQ_OK) return st;
+    if (window > INT32_MAX - sinks) return fail(TQ_ERR_VALUE, "window + sinks overflows");
+    const int32_t dense = window + sinks;
+    if (batch > 0) {
+        const FusedAppend app{k_new, v_new, k_win, v_win, k_pages, v_pages, window, sinks};
+        st = decode_partials_impl(kc, vc, q, k_pages, v_pages, block_tables, max_blocks_per_seq, seq_lens, batch,
+                                  num_q_heads, max_seq_len, k_win, v_win, dense, softmax_scale, num_blocks,
+                                  block_size, workspace, workspace_bytes, d_err, stream, &app);
+        if (st != TQ_OK) return st;
+    }
+    return tq_decode_combine(vc, seq_lens, batch, num_q_heads, max_seq_len, dense, block_size, out, workspace,
+                             workspace_bytes, stream);
 }
 
 extern "C" tq_status tq_decode_paged(const tq_codec* kc, const tq_codec* vc, const void* q, const void* k_pages,

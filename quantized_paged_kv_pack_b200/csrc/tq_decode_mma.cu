@@ -53,6 +53,7 @@
 #include <type_traits>
 
 #include "tq_internal.h"
+#include "tq_pack_vector.cuh"
 
 namespace tq {
 namespace {
@@ -1260,9 +1261,13 @@ struct WarpTiles {
 // Writes (max, sum, accumulator) per query head g < rows: m[g * ml_stride],
 // l[g * ml_stride], acc[g * acc_stride + coordinate] (acc 8-byte aligned).
 template <int NH>
+// t_new >= 0: dense slot t_new holds the step's new token, read from kn / vn (rows of 128) instead of
+// the buffer (a fused window append may be writing that slot).
 __device__ __forceinline__ void window_state(const DecodeArgs& a, const Item& it, int h, int head0, int rows,
                                              int t_first, int t_step, int lane, float* m_out, float* l_out,
-                                             float* acc_out, int ml_stride, int acc_stride) {
+                                             float* acc_out, int ml_stride, int acc_stride, int t_new = -1,
+                                             const __nv_bfloat16* kn = nullptr,
+                                             const __nv_bfloat16* vn = nullptr) {
     const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
     const int H = a.kc.num_heads;
     float qv[NH][4], m[NH], l[NH], acc[NH][4];
@@ -1302,8 +1307,9 @@ __device__ __forceinline__ void window_state(const DecodeArgs& a, const Item& it
             uint2 kr = make_uint2(0u, 0u), vr = make_uint2(0u, 0u);
             if (ok[u]) {
                 const int64_t base = (row0 + tk) * kHeadDim + 4 * lane;
-                kr = *reinterpret_cast<const uint2*>(kw + base);
-                vr = *reinterpret_cast<const uint2*>(vw + base);
+                const bool fresh = tk == t_new;
+                kr = *reinterpret_cast<const uint2*>(fresh ? kn + 4 * lane : kw + base);
+                vr = *reinterpret_cast<const uint2*>(fresh ? vn + 4 * lane : vw + base);
             }
             kx[u][0] = __uint_as_float(kr.x << 16);
             kx[u][1] = __uint_as_float(kr.x & 0xffff0000u);
@@ -2123,6 +2129,10 @@ union ProSmem {
         float m[kProWarps][8], l[kProWarps][8];
         float o[kProWarps][8][kHeadDim];
     } win;
+    struct {
+        uint8_t idx[kProWarps][kHeadDim];  // fused window append: each warp's index bytes
+        float r[kProWarps][kHeadDim];      // and residual scratch
+    } app;
 };
 
 // Exclusive scan of x over the CTA; total gets the sum.
@@ -2226,8 +2236,19 @@ __device__ __forceinline__ void window_unit(const DecodeArgs& a, int group, int 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rows = group < NH ? group : NH;
     const int head0 = it.h * group + it.hg * 8;
+    // Fused window append: the slot the new token takes, if this decode reads it (as in append_vector).
+    int t_new = -1;
+    const __nv_bfloat16 *kn = nullptr, *vn = nullptr;
+    if (a.app_on) {
+        const int L = max(__ldg(a.seq_lens + it.b), 0), S = a.app_sinks, W = a.app_window;
+        const int slot = L < S ? L : (W > 0 ? S + (L - S) % W : -1);
+        if (slot >= 0 && slot < it.t1) t_new = slot;
+        const int64_t row = static_cast<int64_t>(it.b) * H + it.h;
+        kn = static_cast<const __nv_bfloat16*>(a.k_new) + row * kHeadDim;
+        vn = static_cast<const __nv_bfloat16*>(a.v_new) + row * kHeadDim;
+    }
     window_state<NH>(a, it, it.h, head0, rows, warp, kProWarps, lane, &s.m[warp][0], &s.l[warp][0], &s.o[warp][0][0],
-                 1, kHeadDim);
+                 1, kHeadDim, t_new, kn, vn);
     __syncthreads();
     float* rec = record_of(a, it.b, it.h, it.split, group) + it.hg * 8 * (kHeadDim + 2);
     for (int e = threadIdx.x; e < rows * kHeadDim; e += kProThreads) {
@@ -2382,7 +2403,7 @@ __device__ __forceinline__ void rotate_rows_dense(const DecodeArgs& a, int group
 template <int KMODE, int NH>
 __global__ void __launch_bounds__(kProThreads, NH == 4 ? 2 : 1) decode_prologue_kernel(DecodeArgs a, int group,
                                                                                       int head_groups,
-                                                                      int64_t n_rot) {
+                                                                                      int64_t n_rot, int64_t n_win) {
     __shared__ ProSmem sm;
     griddep_launch_dependents();
     // Launched as a dependent of whatever ran before in the stream (the step's window append, say):
@@ -2397,8 +2418,18 @@ __global__ void __launch_bounds__(kProThreads, NH == 4 ? 2 : 1) decode_prologue_
         else
             rotate_rows(a, group, static_cast<int64_t>(a.batch) * a.num_q_heads, blk - 1,
                         KMODE == kQjl ? a.qjl_q : nullptr, sm);
-    } else {
+    } else if (blk <= n_rot + n_win) {
         window_unit<NH>(a, group, head_groups, blk - 1 - n_rot, sm);
+    } else {
+        // fused window append: one warp per (sequence, KV head, K or V)
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int64_t vec = (blk - 1 - n_rot - n_win) * kProWarps + warp;
+        if (vec < static_cast<int64_t>(a.batch) * a.kc.num_heads * 2)
+            append_vector(a.kc, a.vc, vec, static_cast<const __nv_bfloat16*>(a.k_new),
+                          static_cast<const __nv_bfloat16*>(a.v_new), static_cast<__nv_bfloat16*>(a.k_win_w),
+                          static_cast<__nv_bfloat16*>(a.v_win_w), a.app_window, a.app_sinks, a.seq_lens,
+                          a.block_tables, a.max_blocks, a.k_pages_w, a.v_pages_w, a.num_blocks, a.block_size,
+                          a.d_err, sm.app.idx[warp], sm.app.r[warp], lane);
     }
 }
 
@@ -2453,10 +2484,11 @@ tq_status launch_fmt(const DecodeArgs& a, const LutValues& tv, int group, cudaSt
     const int64_t n_rot = (KF::MODE == kGroupwise || KF::MODE == kRecipe) ? static_cast<int64_t>(a.batch) * a.kc.num_heads
                                                  : (rows + kRotRows - 1) / kRotRows;
     const int64_t n_win = a.window > 0 ? static_cast<int64_t>(a.batch) * a.kc.num_heads * head_groups : 0;
-    if (1 + n_rot + n_win > INT32_MAX) return TQ_ERR_UNSUPPORTED;
+    const int64_t n_app = a.app_on ? (static_cast<int64_t>(a.batch) * a.kc.num_heads * 2 + kProWarps - 1) / kProWarps : 0;
+    if (1 + n_rot + n_win + n_app > INT32_MAX) return TQ_ERR_UNSUPPORTED;
     const cudaError_t pe = launch_dependent(decode_prologue_kernel<KF::MODE, NH>,
-                                            dim3(static_cast<unsigned>(1 + n_rot + n_win)), dim3(kProThreads), 0, s,
-                                            a, group, head_groups, n_rot);
+                                            dim3(static_cast<unsigned>(1 + n_rot + n_win + n_app)), dim3(kProThreads),
+                                            0, s, a, group, head_groups, n_rot, n_win);
     if (pe != cudaSuccess) return fail(TQ_ERR_CUDA, std::string("decode prologue launch: ") + cudaGetErrorString(pe));
     const int64_t units = static_cast<int64_t>(a.items_per_unit) * a.batch * head_groups *
                           (blk ? a.kc.num_heads / kBlkWarps : a.kc.num_heads);

@@ -81,12 +81,25 @@ struct DecodeArgs {
     int32_t split_tokens, max_splits, items_per_unit;
     float* ws;                     // records [B][H_kv][items_per_unit][G][2 + 128]
     float* qrot;                   // rotated, scaled queries [B][H_q][128] in K packed order
-    float* qjl_q;                  // QJL keys: sqrt(pi/2)/128 * S q_r of the scaled rotated query,
-                                   // [B][H_q][128] in projection order
+    float* qjl_q;                  // QJL and recipe keys: the projections of the scaled rotated query,
+                                   // [B][H_q][128], permuted so that each lane's B-fragment values of a
+                                   // sign k-step are adjacent
     int32_t* work_list;            // tensor-core kernels: (sequence, split) pairs of the non-empty
                                    // work items, [B * items_per_unit][2], built on the device
     int32_t* work_count;           // number of pairs in work_list
     int* d_err;
+    // Fused window append (tq_window_append_decode): extra prologue CTAs append the step's new token
+    // per (sequence, KV head) as tq_window_append would, and the prologue's window CTAs read the token
+    // from k_new / v_new for the dense slot it takes (the append may be writing that slot meanwhile).
+    // The decode then reads what it would read after a separate append. app_on = 0: no append.
+    int32_t app_on;
+    const void* k_new;             // bf16 [B][H_kv][128]
+    const void* v_new;
+    void* k_win_w;                 // the dense buffers and pages the append writes
+    void* v_win_w;
+    uint8_t* k_pages_w;
+    uint8_t* v_pages_w;
+    int32_t app_window, app_sinks; // the append's W and S (the decode's window is S + W)
     // Test hook (TQ_TEST_WITHHOLD_COPIES=1): the tensor-core kernels' producer
     // issues no copies, so the compute warps' bounded waits expire and report
     // TQ_DERR_TIMEOUT. Nothing sets it in normal use.
@@ -152,6 +165,13 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 #endif
+
+// The argument checks of tq_window_append (TQ_OK for batch == 0 as well).
+tq_status validate_window_append(const tq_codec* kc, const tq_codec* vc, const void* k_new, const void* v_new,
+                                 const void* k_win, const void* v_win, int32_t window, int32_t sinks,
+                                 const int32_t* seq_lens, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                 const void* k_pages, const void* v_pages, int64_t num_blocks, int32_t block_size,
+                                 int32_t batch);
 
 // Sets the thread-local error message and returns `st`.
 tq_status fail(tq_status st, const std::string& msg);

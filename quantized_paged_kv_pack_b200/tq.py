@@ -85,11 +85,14 @@ def lib():
         L.tq_static_workspace_bytes.restype = _SZ
         L.tq_window_append.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP, _I64,
                                        _I32, _I32, _VP, _VP]
+        L.tq_window_append_decode.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32,
+                                              _VP, _I32, _I32, _I32, ctypes.c_float, _I64, _I32, _VP, _VP, _SZ,
+                                              _VP, _VP]
         L.tq_byte_ledger.argtypes = [P(_FormatDesc), P(_FormatDesc), _I32, _VP, _I32, _I32, _I32, _I64, _I32,
                                      P(_Ledger)]
         for name in ("tq_codec_host_tables", "tq_codec_qjl_matrix", "tq_codec_group_rotation", "tq_make_codec", "tq_pack_kv", "tq_decode_paged",
                      "tq_decode_partials", "tq_decode_combine", "tq_byte_ledger", "tq_decode_paged_static",
-                     "tq_window_append"):
+                     "tq_window_append", "tq_window_append_decode"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -348,6 +351,50 @@ def window_append(kc: Codec, vc: Codec, k_new: torch.Tensor, v_new: torch.Tensor
                                   int(window), int(sinks), _ptr(seq_lens), _ptr(block_tables),
                                   int(block_tables.shape[1]), _ptr(k_pages), _ptr(v_pages), nb, int(block_size), B,
                                   _ptr(d_err), _stream(stream)))
+
+
+def window_append_decode(kc: Codec, vc: Codec, k_new: torch.Tensor, v_new: torch.Tensor,
+                         k_win: Optional[torch.Tensor], v_win: Optional[torch.Tensor], window: int, sinks: int,
+                         q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_size: int,
+                         block_tables: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int, softmax_scale: float,
+                         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                         d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step (tq_window_append_decode): window_append, then decode_paged with window
+    sinks + window and the same seq_lens, in fewer launches; returns fp32 [B][H_q][d]."""
+    if q.dim() != 3:
+        raise ValueError("q must be [batch][num_q_heads][head_dim]")
+    B, Hq, d = q.shape
+    H = kc.num_kv_heads
+    _need(q, torch.bfloat16, (B, Hq, kc.head_dim), "q")
+    _need(k_new, torch.bfloat16, (B, H, kc.head_dim), "k_new")
+    _need(v_new, torch.bfloat16, (B, H, kc.head_dim), "v_new")
+    dense = int(window) + int(sinks)
+    if dense > 0:
+        if k_win is None or v_win is None:
+            raise ValueError("sinks + window > 0 needs the dense buffers")
+        _need(k_win, torch.bfloat16, (B, H, dense, kc.head_dim), "k_win")
+        _need(v_win, torch.bfloat16, (B, H, dense, kc.head_dim), "v_win")
+    else:
+        k_win = v_win = None
+    _need(seq_lens, torch.int32, (B,), "seq_lens")
+    if block_tables.dim() != 2:
+        raise ValueError("block_tables must be [batch][max_blocks_per_seq]")
+    _need(block_tables, torch.int32, (B, block_tables.shape[1]), "block_tables")
+    nb = _pools(kc, vc, k_pages, v_pages, block_size)
+    bs = int(block_size)
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, (B, Hq, d), "out")
+    if workspace is None:
+        workspace = alloc_workspace(B, Hq, H, max_seq_len, bs, device=q.device)
+    if d_err is not None:
+        _need(d_err, torch.int32, (1,), "d_err")
+    _check(lib().tq_window_append_decode(kc.handle, vc.handle, _ptr(k_new), _ptr(v_new), _ptr(k_win), _ptr(v_win),
+                                         int(window), int(sinks), _ptr(q), _ptr(k_pages), _ptr(v_pages),
+                                         _ptr(block_tables), int(block_tables.shape[1]), _ptr(seq_lens), B, Hq,
+                                         int(max_seq_len), float(softmax_scale), nb, bs, _ptr(out), _ptr(workspace),
+                                         workspace.numel(), _ptr(d_err), _stream(stream)))
+    return out
 
 
 def decode_workspace_bytes(batch: int, num_q_heads: int, num_kv_heads: int, max_seq_len: int, block_size: int) -> int:
