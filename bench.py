@@ -244,15 +244,17 @@ class ClockSampler:
         self.sel = sel
 
     def _nvml_loop(self, nv, handle, stop):
-        mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+        mx = None
         while not stop.is_set():
             try:
+                if mx is None:
+                    mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
                 sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
                 bits = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((float(sm), float(mx), {n for n, b in self.REASON_BITS.items() if bits & b}))
             except Exception:
-                break
-            self.samples.append((float(sm), float(mx), {n for n, b in self.REASON_BITS.items() if bits & b}))
-            stop.wait(0.005)
+                pass  # a failed query is skipped, not fatal
+            stop.wait(0.002)
 
     def __enter__(self):
         try:
@@ -267,6 +269,7 @@ class ClockSampler:
             self.thread = threading.Thread(target=self._nvml_loop, args=(nv, handle, self.stop), daemon=True)
             self.thread.start()
             time.sleep(0.02)
+            self.first = len(self.samples)  # samples from here on fall inside the timed region
             return self
         except Exception:
             self.thread = None
@@ -304,11 +307,15 @@ class ClockSampler:
                 self.samples.append((sm, mx, {n for n, v in zip(names, parts[5:9]) if v.lower() == "active"}))
 
     def summary(self):
-        if not self.samples:
+        inside = self.samples[getattr(self, "first", 0):]
+        where = "timed region"
+        if not inside:  # a region shorter than the sampling interval: the samples just before it
+            inside, where = self.samples[-3:], "just before the timed region"
+        if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        reasons = set().union(*(r for _, _, r in self.samples))
-        return {"sm_mhz": statistics.median(sm for sm, _, _ in self.samples), "sm_max_mhz": self.samples[-1][1],
-                "reasons": sorted(reasons), "samples": len(self.samples),
+        reasons = set().union(*(r for _, _, r in inside))
+        return {"sm_mhz": statistics.median(sm for sm, _, _ in inside), "sm_max_mhz": inside[-1][1],
+                "reasons": sorted(reasons), "samples": len(inside), "sampled": where,
                 "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
