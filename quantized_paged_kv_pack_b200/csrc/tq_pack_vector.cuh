@@ -62,6 +62,22 @@ __device__ __forceinline__ unsigned short norm_fp16_bits(const float (&x)[4], fl
     return hb;
 }
 
+// Boundaries of a group's codebook below u (the index): the 15 loads are issued
+// together instead of one per loop trip (a lone vector is bound by this latency).
+__device__ __forceinline__ int pv_boundary_count(const float* bound, int levels, float u) {
+    int idx = 0;
+#pragma unroll
+    for (int q = 0; q < 15; ++q)
+        if (q < levels - 1) idx += (__ldg(bound + q) < u) ? 1 : 0;
+    return idx;
+}
+
+// (lb / b, lb % b) for a bit width b of 2, 3 or 4 and 0 <= lb < 2^16, without a division.
+__device__ __forceinline__ void pv_divmod(int lb, int b, int& q, int& r) {
+    q = b == 4 ? lb >> 2 : (b == 2 ? lb >> 1 : static_cast<int>((static_cast<unsigned>(lb) * 0xAAABu) >> 17));
+    r = lb - q * b;
+}
+
 // One warp quantizes the vector x (lane l holds elements 4l .. 4l+3) of KV
 // head h and writes its row at `offset` of the sub-page `sub` (block_size
 // rows). idx_buf: 128 bytes, r_buf: 128 floats of shared scratch owned by the
@@ -106,8 +122,7 @@ __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8
         const int g = (c.n_groups == 2 && p >= c.pos0[1]) ? 1 : 0;
         const float u = z[i] * inv;
         const int levels = 1 << c.bits[g];
-        int idx = 0;
-        for (int q = 0; q < levels - 1; ++q) idx += (c.bound[g * 16 + q] < u) ? 1 : 0;
+        const int idx = pv_boundary_count(c.bound + g * 16, levels, u);
         idx_buf[p] = static_cast<uint8_t>(idx);
         if (c.qjl) {
             const float r = u - c.cent[g * 16 + idx];  // residual, rotated coordinate j
@@ -122,11 +137,19 @@ __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8
     if (c.qjl) {
         g16 = __half_as_ushort(__float2half_rn(sqrtf(pv_warp_sum(rr))));
         float proj[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int j = 0; j < kHeadDim; ++j) {
-            const float r = r_buf[j];
-            const float* st = c.qjl_st + j * kHeadDim + lane;
+        // rows of S^T in batches of 8, their loads issued together (same accumulation order)
+        for (int j0 = 0; j0 < kHeadDim; j0 += 8) {
+            float sv[8][4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) proj[k] = fmaf(__ldg(st + 32 * k), r, proj[k]);
+            for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) sv[jj][k] = __ldg(c.qjl_st + (j0 + jj) * kHeadDim + lane + 32 * k);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const float r = r_buf[j0 + jj];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) proj[k] = fmaf(sv[jj][k], r, proj[k]);
+            }
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) sign_word[k] = __ballot_sync(kPvFull, proj[k] >= 0.0f);
@@ -139,7 +162,8 @@ __device__ void pack_vector(const DevCodec& c, const float (&x)[4], int h, uint8
             const int g = (c.n_groups == 2 && B >= 8 * c.byte_off[1]) ? 1 : 0;
             const int lb = B - 8 * c.byte_off[g];
             const int b = c.bits[g];
-            const int q = lb / b, r = lb - q * b;
+            int q, r;
+            pv_divmod(lb, b, q, r);
             word |= ((idx_buf[c.pos0[g] + q] >> r) & 1u) << i;
         }
     }
@@ -183,12 +207,24 @@ __device__ void pack_recipe_tail(const DevCodec& c, const float (&res)[4], const
     for (int g = 0; g < 2; ++g) {
         const int n = c.size[g], p0 = c.pos0[g];
         const float* st = c.qjl_st + (g ? static_cast<int64_t>(n0) * n0 : 0);
-        for (int j = 0; j < n; ++j) {
-            const float r = r_buf[p0 + j];
+        // rows of S_g^T in batches of 8 (group sizes are multiples of 8), loads issued together
+        for (int j0 = 0; j0 < n; j0 += 8) {
+            float sv[8][4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = lane + 32 * k - p0;
-                if (i >= 0 && i < n) proj[k] = fmaf(__ldg(st + j * n + i), r, proj[k]);
+            for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = lane + 32 * k - p0;
+                    sv[jj][k] = (i >= 0 && i < n) ? __ldg(st + (j0 + jj) * n + i) : 0.0f;
+                }
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const float r = r_buf[p0 + j0 + jj];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = lane + 32 * k - p0;
+                    if (i >= 0 && i < n) proj[k] = fmaf(sv[jj][k], r, proj[k]);
+                }
             }
         }
     }
@@ -204,14 +240,16 @@ __device__ void pack_recipe_tail(const DevCodec& c, const float (&res)[4], const
             const int B = 16 * hw + i;
             unsigned bit;
             if (B < 8 * c.sign_off[0]) {  // group 0 indices
-                const int q = B / c.bits[0], r = B - q * c.bits[0];
+                int q, r;
+                pv_divmod(B, c.bits[0], q, r);
                 bit = (idx_buf[q] >> r) & 1u;
             } else if (B < 8 * c.byte_off[1]) {  // group 0 signs
                 const int p = B - 8 * c.sign_off[0];
                 bit = (sw[p >> 5] >> (p & 31)) & 1u;
             } else if (B < 8 * c.sign_off[1]) {  // group 1 indices
                 const int lb = B - 8 * c.byte_off[1];
-                const int q = lb / c.bits[1], r = lb - q * c.bits[1];
+                int q, r;
+                pv_divmod(lb, c.bits[1], q, r);
                 bit = (idx_buf[n0 + q] >> r) & 1u;
             } else {  // group 1 signs
                 const int p = n0 + B - 8 * c.sign_off[1];
@@ -258,10 +296,19 @@ __device__ void pack_vector_groupwise(const DevCodec& c, const float (&x)[4], in
     __syncwarp();
     float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const float* rt = c.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim + lane;
-    for (int j = 0; j < kHeadDim; ++j) {
-        const float xj = x_buf[j];
+    // rows of R_h^T in batches of 8, their loads issued together (same accumulation order)
+    for (int j0 = 0; j0 < kHeadDim; j0 += 8) {
+        float rv[8][4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) y[k] = fmaf(__ldg(rt + j * kHeadDim + 32 * k), xj, y[k]);
+        for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) rv[jj][k] = __ldg(rt + (j0 + jj) * kHeadDim + 32 * k);
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+            const float xj = x_buf[j0 + jj];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) y[k] = fmaf(rv[jj][k], xj, y[k]);
+        }
     }
     float res[4];  // recipe row: residuals u - c[idx] of the lane's positions
 #pragma unroll
@@ -270,8 +317,7 @@ __device__ void pack_vector_groupwise(const DevCodec& c, const float (&x)[4], in
         const int g = p >= n0 ? 1 : 0;
         const float u = n32[g] > 0.0f ? y[k] / n32[g] : 0.0f;
         const int levels = 1 << c.bits[g];
-        int idx = 0;
-        for (int q = 0; q < levels - 1; ++q) idx += (c.bound[g * 16 + q] < u) ? 1 : 0;
+        const int idx = pv_boundary_count(c.bound + g * 16, levels, u);
         idx_buf[p] = static_cast<uint8_t>(idx);
         res[k] = u - c.cent[g * 16 + idx];
     }
@@ -288,7 +334,8 @@ __device__ void pack_vector_groupwise(const DevCodec& c, const float (&x)[4], in
             const int g = B >= 8 * c.byte_off[1] ? 1 : 0;
             const int lb = B - 8 * c.byte_off[g];
             const int b = c.bits[g];
-            const int q = lb / b, r = lb - q * b;
+            int q, r;
+            pv_divmod(lb, b, q, r);
             word |= ((idx_buf[c.pos0[g] + q] >> r) & 1u) << i;
         }
     }
