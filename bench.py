@@ -40,7 +40,8 @@ SMALL = "decode_gqa8_4k_4bit"
 DECODE_LAUNCHES = 3  # per step: prologue (work list, query rotation, windows, the append), decode, combine
 EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl",
          "decode_llama8b_3p5bit_groupwise", "decode_llama8b_3p5bit_recipe",
-         "pack_llama8b_4bit", "pack_llama70b_3p5bit", "pack_llama8b_2p5bit"]
+         "pack_llama8b_4bit", "pack_llama70b_3p5bit", "pack_llama8b_2p5bit", "pack_llama8b_3p5bit_qjl",
+         "pack_llama8b_3p5bit_groupwise"]
 D = 128
 METRIC = "paged TQ decode HBM GB/s (algorithmic bytes / step time)"
 

@@ -95,6 +95,18 @@ WORKLOADS = {
         description="pack 32 sequences x 8192 tokens, 8 KV heads, block 32, shuffled slot mapping, "
                     "K 2.5-bit (32 channels at 4 bits + 96 at 2 bits), V uniform 3-bit (the formats of "
                     "the batch-256 decode workload)"),
+    "pack_llama8b_3p5bit_qjl": Workload(
+        "pack_llama8b_3p5bit_qjl", "pack", 1011, 32, 32, 8, 128, 16, 0,
+        (3, 2), (64, 64), (4, 3), (64, 64), 61, 62, 8, True, "fixed:8192", k_qjl=True,
+        description="pack 32 sequences x 8192 tokens, 8 KV heads, block 16, shuffled slot mapping, the QJL "
+                    "decode workload's formats (K 2.5-bit MSE plus the 1-bit QJL stage, V 3.5-bit); general "
+                    "per-vector pack kernel"),
+    "pack_llama8b_3p5bit_groupwise": Workload(
+        "pack_llama8b_3p5bit_groupwise", "pack", 1012, 32, 32, 8, 128, 16, 0,
+        (4, 3), (64, 64), (4, 3), (64, 64), 71, 72, 8, True, "fixed:8192", groupwise=True,
+        description="pack 32 sequences x 8192 tokens, 8 KV heads, block 16, shuffled slot mapping, K and V "
+                    "3.5-bit group-wise (the group-wise decode workload's formats); general per-vector pack "
+                    "kernel"),
     "decode_llama8b_4bit": Workload(
         "decode_llama8b_4bit", "decode", 1003, 64, 32, 8, 128, 16, 64,
         (4,), (128,), (4,), (128,), 0, 1, 8, True, "uniform:1024:32768",
