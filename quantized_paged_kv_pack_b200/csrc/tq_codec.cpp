@@ -447,18 +447,21 @@ bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, i
 using namespace tq;
 
 namespace tq {
-void build_pack_cells(const float* boundaries, int levels, PackCell* out) {
+bool build_pack_cells(const float* boundaries, int levels, PackCell* out) {
+    bool ok = true;
     for (int e = 0; e < kPackCells; ++e) {
         const double lo = e - 64 - 0.5, hi = e - 64 + 0.5;
-        int below = 0;
+        int below = 0, inside = 0;
         float thr = INFINITY;
         for (int i = 0; i + 1 < levels; ++i) {
             const double bv = static_cast<double>(boundaries[i]) * kPackCellScale;
             if (bv < lo) ++below;
-            else if (bv <= hi) thr = static_cast<float>(bv);
+            else if (bv <= hi) thr = static_cast<float>(bv), ++inside;
         }
+        if (inside > 1) ok = false;  // one compare per lookup needs at most one boundary per cell
         out[e] = PackCell{thr, below};
     }
+    return ok;
 }
 }  // namespace tq
 
@@ -537,11 +540,18 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     const size_t off_s = (n_sign + 2 * n_cent + 2 * n_perm + 15) / 16 * 16;
     const size_t n_s = c->qjl_s.size() * sizeof(float);
     const size_t off_r = (off_s + n_s + 15) / 16 * 16, n_r = c->rot_t.size() * sizeof(float);
-    // plain codecs (no QJL stage, no group-wise rotation) also carry the tensor-core pack's
-    // quantizer cell table of each group
-    const bool plain = !desc->qjl && !desc->groupwise;
+    // codecs without the QJL stage also carry the tensor-core pack's quantizer cell table of
+    // each group (when every cell holds at most one boundary)
+    std::vector<PackCell> cells;
+    if (!desc->qjl) {
+        cells.resize(static_cast<size_t>(desc->n_groups) * kPackCells);
+        bool ok = true;
+        for (int g = 0; g < desc->n_groups; ++g)
+            ok = build_pack_cells(c->bound[g], 1 << desc->group_bits[g], cells.data() + g * kPackCells) && ok;
+        if (!ok) cells.clear();
+    }
     const size_t off_c = (off_r + n_r + 15) / 16 * 16;
-    const size_t n_c = plain ? static_cast<size_t>(desc->n_groups) * kPackCells * sizeof(PackCell) : 0;
+    const size_t n_c = cells.size() * sizeof(PackCell);
     const size_t total = off_c + n_c;
     std::vector<char> host(total);
     char* p = host.data();
@@ -566,8 +576,7 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
             for (int j = 0; j < d; ++j) st[static_cast<size_t>(j) * d + i] = c->qjl_s[static_cast<size_t>(i) * d + j];
     }
     if (n_r) std::memcpy(p + off_r, c->rot_t.data(), n_r);
-    for (int g = 0; n_c && g < desc->n_groups; ++g)
-        build_pack_cells(c->bound[g], 1 << desc->group_bits[g], reinterpret_cast<PackCell*>(p + off_c) + g * kPackCells);
+    if (n_c) std::memcpy(p + off_c, cells.data(), n_c);
     if (cudaGetDevice(&c->device) != cudaSuccess || cudaMalloc(&c->d_tables, total) != cudaSuccess) {
         cudaGetLastError();
         delete c;

@@ -21,17 +21,18 @@ constexpr int kMaxLevels = 16;  // 4-bit codebooks at most on the GPU path
 // rotated unit coordinate u, scaled to v = 64 u, falls into cell round(v) + 64
 // of 129 cells over [-64, 64]; a cell holds the number of decision boundaries
 // strictly below it and the one boundary inside it (in units of v; +inf when
-// none). At head_dim 128 adjacent boundaries of the 2-, 3- and 4-bit
-// codebooks are more than one unit of v apart, so no cell holds two. A plain
-// codec builds one per group on the host and copies them to the device with
-// its other tables.
+// none). Adjacent boundaries of the 2-, 3- and 4-bit codebooks of dimension
+// 128 (and of the wider ones of smaller groups) are more than one unit of v
+// apart, so no cell holds two; build_pack_cells returns false if one does. A
+// codec without the QJL stage builds one per group on the host and copies them
+// to the device with its other tables.
 constexpr int kPackCells = 129;
 constexpr float kPackCellScale = 64.0f;
 struct PackCell {
     float thr;       // boundary inside the cell, +inf if none
     int32_t below;   // boundaries strictly below the cell
 };
-void build_pack_cells(const float* boundaries, int levels, PackCell* out);
+bool build_pack_cells(const float* boundaries, int levels, PackCell* out);
 
 // Device-side view of one codec, passed to kernels by value.
 struct DevCodec {
@@ -58,7 +59,7 @@ struct DevCodec {
                             // (n_g, residual norm_g) per group; qjl_st is then S_0^T then S_1^T (n_g x n_g)
     int32_t sign_off[2];    // byte offset of each group's QJL sign bits in the index part (QJL: the one
                             // stream after the index bitstreams)
-    const PackCell* cells;  // plain codecs: the pack's quantizer cell table of each group [n_groups][129];
+    const PackCell* cells;  // codecs without the QJL stage: the pack's quantizer cell table of each group [n_groups][129];
                             // else null
 };
 

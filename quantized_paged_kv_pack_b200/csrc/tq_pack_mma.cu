@@ -64,6 +64,15 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
+// d += a b (accumulating form).
+__device__ __forceinline__ void mma_bf16_acc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Packed fp32 helpers on pairs held in one 64-bit register.
 __device__ __forceinline__ uint64_t pk(float lo, float hi) {
     uint64_t r;
@@ -311,8 +320,43 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_u4_kernel(DevCodec kc, DevCo
                         }
                     }
                 }
+                // A token whose norm is not below 3e37 (inf, NaN, or so near the bf16 limit that the
+                // fp32 rotation could overflow) is packed as the zero vector with its norm as computed,
+                // so that every cell lookup below stays inside the table: its input row is cleared
+                // (the second half reloads it) and so are this half's fragments.
+                const bool bad0 = !(n_tok[0] < 3.0e37f), bad1 = !(n_tok[1] < 3.0e37f);
+                if (__any_sync(kFull, bad0 || bad1)) {
+                    __syncwarp();  // the fragments of every lane are read
+                    const uint32_t row0 = xbuf0 + static_cast<uint32_t>((cur * 16 + r) * kRowPad + 64 * c);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (bad0)
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(row0 + 16 * k), "r"(0u)
+                                         : "memory");
+                        if (bad1)
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(row0 + 8 * kRowPad + 16 * k),
+                                         "r"(0u)
+                                         : "memory");
+                    }
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) {
+                        if (bad0) xa[a] = make_uint2(0u, 0u);
+                        if (bad1) xb[a] = make_uint2(0u, 0u);
+                    }
+                    __syncwarp();
+                }
             }
 
+            // A token whose norm is not below 3e37 (inf, NaN, or so near the bf16 limit that the fp32
+            // rotation could overflow) is packed as the zero vector with its norm as computed: every
+            // cell lookup below then stays inside the table.
+            if (__any_sync(kFull, !(n_tok[0] < 3.0e37f) || !(n_tok[1] < 3.0e37f))) {
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    if (!(n_tok[0] < 3.0e37f)) xa[a] = make_uint2(0u, 0u);
+                    if (!(n_tok[1] < 3.0e37f)) xb[a] = make_uint2(0u, 0u);
+                }
+            }
             // z = (H_16 D_s) per a on the tensor cores: columns b' = 8t + 2c + {0,1} of n-tile t.
             uint64_t zp[8][2];  // [a][token]: (columns 2c, 2c+1 of n-tile t)
 #pragma unroll
@@ -445,6 +489,35 @@ using PU4 = PackFmt<4, 128, 0, 0>;
 using PU3 = PackFmt<3, 128, 0, 0>;
 using PM43 = PackFmt<4, 64, 3, 64>;
 using PM42 = PackFmt<4, 32, 2, 96>;
+
+// Bit assembly of a warp's 16 staged index rows (one byte per packed position, pitch
+// kStagePitch): in round k lanes 0-15 take packed positions 16 k .. 16 k + 7 of token lane
+// and lanes 16-31 positions 16 k + 8 .. 16 k + 15 of token lane - 16 (one group for the
+// whole warp, since groups start on multiples of 16), into b bytes of the row, LSB-first.
+template <class F>
+__device__ __forceinline__ void assemble_rows(uint32_t stage, uint8_t (&rows)[16][72], int lane) {
+    const int tok = lane & 15, hi8 = (lane >> 4) * 8;
+    const uint32_t srow = stage + static_cast<uint32_t>(tok * kStagePitch);
+    uint8_t* drow = &rows[tok][0];
+    static_for<0, 8>([&](auto kc) {
+        constexpr int K = decltype(kc)::value;
+        constexpr bool G1 = F::NG == 2 && 16 * K >= F::N0;
+        constexpr int B = G1 ? F::B1 : F::B0;
+        const int p = 16 * K + hi8;
+        const uint32_t lo = lds32(srow + p), hi = lds32(srow + p + 4);
+        uint8_t* dst = drow + (G1 ? F::BOFF1 + (p - F::N0) * B / 8 : p * B / 8);
+        if constexpr (B == 4) {
+            *reinterpret_cast<uint32_t*>(dst) = pack8<4>(lo, hi);
+        } else if constexpr (B == 2) {
+            *reinterpret_cast<unsigned short*>(dst) = static_cast<unsigned short>(pack8<2>(lo, hi));
+        } else {
+            const uint32_t w = pack8<3>(lo, hi);
+            dst[0] = static_cast<uint8_t>(w);
+            dst[1] = static_cast<uint8_t>(w >> 8);
+            dst[2] = static_cast<uint8_t>(w >> 16);
+        }
+    });
+}
 
 template <class F>
 __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const __nv_bfloat16* __restrict__ src,
@@ -597,6 +670,41 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
                         }
                     }
                 }
+                // A token whose norm is not below 3e37 (inf, NaN, or so near the bf16 limit that the
+                // fp32 rotation could overflow) is packed as the zero vector with its norm as computed,
+                // so that every cell lookup below stays inside the table: its input row is cleared
+                // (the second half reloads it) and so are this half's fragments.
+                const bool bad0 = !(n_tok[0] < 3.0e37f), bad1 = !(n_tok[1] < 3.0e37f);
+                if (__any_sync(kFull, bad0 || bad1)) {
+                    __syncwarp();  // the fragments of every lane are read
+                    const uint32_t row0 = xbuf0 + static_cast<uint32_t>((cur * 16 + r) * kRowPad + 64 * c);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (bad0)
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(row0 + 16 * k), "r"(0u)
+                                         : "memory");
+                        if (bad1)
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(row0 + 8 * kRowPad + 16 * k),
+                                         "r"(0u)
+                                         : "memory");
+                    }
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) {
+                        if (bad0) xa[a] = make_uint2(0u, 0u);
+                        if (bad1) xb[a] = make_uint2(0u, 0u);
+                    }
+                    __syncwarp();
+                }
+            }
+            // A token whose norm is not below 3e37 (inf, NaN, or so near the bf16 limit that the fp32
+            // rotation could overflow) is packed as the zero vector with its norm as computed: every
+            // cell lookup below then stays inside the table.
+            if (__any_sync(kFull, !(n_tok[0] < 3.0e37f) || !(n_tok[1] < 3.0e37f))) {
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    if (!(n_tok[0] < 3.0e37f)) xa[a] = make_uint2(0u, 0u);
+                    if (!(n_tok[1] < 3.0e37f)) xb[a] = make_uint2(0u, 0u);
+                }
             }
             uint64_t kq2[2];  // v = z * 64 / (sqrt(128) n) per token
 #pragma unroll
@@ -683,32 +791,7 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
         }
         __syncwarp();
 
-        // Pack: in round k lanes 0-15 take packed positions 16 k .. 16 k + 7 of token lane and lanes
-        // 16-31 positions 16 k + 8 .. 16 k + 15 of token lane - 16 (one group for the whole warp,
-        // since groups start on multiples of 16), into b bytes of the row, LSB-first.
-        {
-            const int tok = lane & 15, hi8 = (lane >> 4) * 8;
-            const uint32_t srow = stage + static_cast<uint32_t>(tok * kStagePitch);
-            uint8_t* drow = &sm.rows[warp][tok][0];
-            static_for<0, 8>([&](auto kc) {
-                constexpr int K = decltype(kc)::value;
-                constexpr bool G1 = F::NG == 2 && 16 * K >= F::N0;
-                constexpr int B = G1 ? F::B1 : F::B0;
-                const int p = 16 * K + hi8;
-                const uint32_t lo = lds32(srow + p), hi = lds32(srow + p + 4);
-                uint8_t* dst = drow + (G1 ? F::BOFF1 + (p - F::N0) * B / 8 : p * B / 8);
-                if constexpr (B == 4) {
-                    *reinterpret_cast<uint32_t*>(dst) = pack8<4>(lo, hi);
-                } else if constexpr (B == 2) {
-                    *reinterpret_cast<unsigned short*>(dst) = static_cast<unsigned short>(pack8<2>(lo, hi));
-                } else {
-                    const uint32_t w = pack8<3>(lo, hi);
-                    dst[0] = static_cast<uint8_t>(w);
-                    dst[1] = static_cast<uint8_t>(w >> 8);
-                    dst[2] = static_cast<uint8_t>(w >> 16);
-                }
-            });
-        }
+        assemble_rows<F>(stage, sm.rows[warp], lane);
         __syncwarp();
 
         // Write the rows in 8-byte pieces (index rows are whole multiples of 8 bytes), and the norms.
@@ -733,35 +816,356 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
     }
 }
 
+
+// ==== tensor-core pack for group-wise formats ===================================
+//
+// Group-wise rotation: u = R_h x / n_g with R_h per KV head (rows are packed
+// positions, columns channels) and one norm per group over the group's original
+// channels. R_h's nonzero entries are +-1/sqrt(m) inside Hadamard blocks of size
+// m (powers of two, 16 to 128, starting on multiples of 16), so R_h = D Q with
+// Q of entries -1, 0, +1 (exact in bf16) and D the blocks' scales, constants of
+// the format. The channels reach the blocks through a per-head permutation, so
+// Q x runs on mma.sync m16n8k16 as the dense product of a unit's 16 x 128 inputs
+// with Q^T (8 k-steps x 16 n-tiles, fp32 accumulation); D and 64 / n_g then scale
+// it to the cell domain. A CTA works on one KV head and keeps Q^T's B fragments
+// (32 KB) in shared memory. The group norms are sums of squares of the inputs
+// masked per group. Quantizer, index staging (the product's output coordinate is
+// the packed position), bit assembly and row writes follow the plain kernel; a
+// row ends in the two fp16 group norms.
+
+struct PackGwSmem {
+    QuantCell cells[2][kCells][16];   // codebook cells of group 0 and group 1, 16 copies
+    uint32_t qfrag[8][16][32][2];     // [k-step][n-tile][lane][reg]: Q^T of the CTA's head, bf16 pairs
+    uint4 gmask[4][32];               // [word / 4][lane]: the lane's group-0 channels as bf16 half masks
+    uint8_t rows[kPW][16][72];        // staged index rows
+    uint32_t norms[kPW][16];          // the row's two fp16 group norms
+    int slot32[kPW][16];              // the unit's slots: -1 padding, capacity when past the pool
+    uint8_t xbuf[kPW][2][16][kRowPad];  // double-buffered input rows; the current one then stages indices
+};
+static_assert(sizeof(PackGwSmem) <= 232448, "fits the shared memory of one CTA");
+
+// 1/sqrt(m) of the Hadamard block that holds packed position p (each group's
+// blocks in decreasing powers of two, as the codec builds R_h).
+template <class F>
+__host__ __device__ constexpr float gw_block_scale(int p) {
+    const int n = p >= F::N0 ? F::N1 : F::N0;
+    int off = p >= F::N0 ? p - F::N0 : p;
+    for (int k = 7; k >= 0; --k) {
+        const int m = 1 << k;
+        if (!(n & m)) continue;
+        if (off < m)
+            return static_cast<float>(((k & 1) ? 0.70710678118654752440 : 1.0) / static_cast<double>(1 << (k / 2)));
+        off -= m;
+    }
+    return 0.0f;
+}
+
+template <class F>
+__global__ void __launch_bounds__(kPW * 32, 1) pack_gw_kernel(DevCodec cd, const __nv_bfloat16* __restrict__ src,
+                                                          const int64_t* __restrict__ slots, int num_tokens,
+                                                          uint8_t* __restrict__ pages, int capacity, int block_size,
+                                                          int bs_log2, int* __restrict__ d_err) {
+    static_assert(F::NG == 2 && F::N0 % 16 == 0, "two groups starting on a multiple of 16");
+    extern __shared__ __align__(16) uint8_t psm_raw[];
+    PackGwSmem& sm = *reinterpret_cast<PackGwSmem*>(psm_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, c = lane & 3;
+    const int H = cd.num_heads;
+    const int h = blockIdx.x % H, cta = blockIdx.x / H, ctas = gridDim.x / H;
+
+    // Cell tables (group g's cells at g * kCells in the codec's table).
+    for (int i = threadIdx.x; i < 2 * kCells * 16; i += kPW * 32) (&sm.cells[0][0][0])[i] = cd.cells[i >> 4];
+    // B fragment (k-step a, n-tile nt) of lane (rr, cc): B[k][n] = sign of R_h[8 nt + rr][16 a + k] for
+    // k = 2 cc + {0, 1} (reg 0) and 2 cc + 8 + {0, 1} (reg 1).
+    const float* rt = cd.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim;  // entry (j, p) = R_h[p][j]
+    for (int i = threadIdx.x; i < 8 * 16 * 32; i += kPW * 32) {
+        const int ln = i & 31, nt = (i >> 5) & 15, a = i >> 9;
+        const int p = 8 * nt + (ln >> 2), j0 = 16 * a + 2 * (ln & 3);
+        uint32_t regs[2];
+        for (int q = 0; q < 2; ++q) {
+            uint32_t w = 0;
+            for (int e = 0; e < 2; ++e) {
+                const float val = __ldg(rt + (j0 + 8 * q + e) * kHeadDim + p);
+                const uint32_t hb = val > 0.0f ? 0x3F80u : (val < 0.0f ? 0xBF80u : 0u);
+                w |= hb << (16 * e);
+            }
+            regs[q] = w;
+        }
+        sm.qfrag[a][nt][ln][0] = regs[0];
+        sm.qfrag[a][nt][ln][1] = regs[1];
+    }
+    // Mask word k = 2 a + q of lane l covers its fragment channels 16 a + 8 q + 2 (l % 4) + {0, 1}.
+    if (threadIdx.x < 128) {
+        const int ln = threadIdx.x & 31, w4 = threadIdx.x >> 5;
+        const int16_t* posh = cd.pos + h * kHeadDim;
+        uint32_t m[4];
+        for (int k = 0; k < 4; ++k) {
+            const int wd = 4 * w4 + k;
+            const int j = 16 * (wd >> 1) + 8 * (wd & 1) + 2 * (ln & 3);
+            m[k] = (posh[j] < F::N0 ? 0x0000FFFFu : 0u) | (posh[j + 1] < F::N0 ? 0xFFFF0000u : 0u);
+        }
+        sm.gmask[w4][ln] = make_uint4(m[0], m[1], m[2], m[3]);
+    }
+    __syncthreads();
+
+    const int tgroups = (num_tokens + 15) / 16;
+    // cell e of group g for this lane: cells_lane + (g * kCells + e) * 128
+    const uint32_t cells_lane = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.cells[0][0][lane & 15]));
+    const uint32_t xbuf0 = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.xbuf[warp][0][0][0]));
+    const uint32_t qf_lane = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.qfrag[0][0][lane][0]));
+    auto issue = [&](int tg_, int buf) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int piece = lane + 32 * i, tok = piece >> 4, part = piece & 15;
+            const int t = tg_ * 16 + tok;
+            const bool live = t < num_tokens;
+            const __nv_bfloat16* g = src + (static_cast<int64_t>(live ? t : 0) * H + h) * kHeadDim + 8 * part;
+            cp_async16(xbuf0 + (buf * 16 + tok) * kRowPad + 16 * part, g, live ? 16u : 0u);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    const int stride = ctas * kPW;
+    int tg = cta * kPW + warp;
+    if (tg < tgroups) issue(tg, 0);
+    for (int it = 0; tg < tgroups; tg += stride, ++it) {
+        const int cur = it & 1;
+        const int t0 = tg * 16;
+        if (lane < 16) {
+            int64_t sl = -1;
+            if (t0 + lane < num_tokens) sl = __ldg(slots + t0 + lane);
+            sm.slot32[warp][lane] = sl < 0 ? -1 : (sl >= capacity ? capacity : static_cast<int>(sl));
+        }
+        if (tg + stride < tgroups) {
+            issue(tg + stride, cur ^ 1);
+        } else {
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncwarp();
+
+        // A fragments: xa[a] = token r, channels 16 a + 2 c + {0, 1} (.x) and 16 a + 8 + 2 c + {0, 1} (.y);
+        // xb[a] the same for token r + 8.
+        const uint32_t frag_row = xbuf0 + (cur * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)) * kRowPad +
+                                  ((lane >> 4) & 1) * 16;
+        const uint32_t stage = xbuf0 + cur * 16 * kRowPad;  // [16][kStagePitch] index bytes, packed order
+        uint2 xa[8], xb[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) ldsm_x4(frag_row + 32 * a, xa[a].x, xb[a].x, xa[a].y, xb[a].y);
+        __syncwarp();  // every lane has read its fragments: the input buffer now stages the indices
+
+        // Group norms: sums of exact squares of the inputs masked per group (fp32), fp64 when the
+        // fp32 norm is too close to an fp16 rounding midpoint to call.
+        float n_tok[2][2];          // [group][token r, r + 8]
+        unsigned short n16[2][2];
+        {
+            uint32_t mw[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint4 m4 = sm.gmask[k][lane];
+                mw[4 * k] = m4.x;
+                mw[4 * k + 1] = m4.y;
+                mw[4 * k + 2] = m4.z;
+                mw[4 * k + 3] = m4.w;
+            }
+            uint64_t acc[2][2] = {{0, 0}, {0, 0}};
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint32_t m = mw[2 * a + q];
+                    const uint32_t lo = q ? xa[a].y : xa[a].x, hi = q ? xb[a].y : xb[a].x;
+                    const uint64_t l0 = bf16x2_to_f32x2(lo & m), l1 = bf16x2_to_f32x2(lo & ~m);
+                    const uint64_t h0 = bf16x2_to_f32x2(hi & m), h1 = bf16x2_to_f32x2(hi & ~m);
+                    acc[0][0] = fma2(l0, l0, acc[0][0]);
+                    acc[1][0] = fma2(l1, l1, acc[1][0]);
+                    acc[0][1] = fma2(h0, h0, acc[0][1]);
+                    acc[1][1] = fma2(h1, h1, acc[1][1]);
+                }
+            bool risky[2][2];
+            bool any_risky = false;
+#pragma unroll
+            for (int g = 0; g < 2; ++g)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    float p, q;
+                    upk(acc[g][i], p, q);
+                    float ss = p + q;
+                    ss += __shfl_xor_sync(kFull, ss, 1);
+                    ss += __shfl_xor_sync(kFull, ss, 2);
+                    const float n32 = sqrtf(ss);
+                    bool rk = !(ss > 1e-30f && ss < 1e30f) || n32 > 60000.0f;
+                    const __half hh = __float2half_rn(n32);
+                    const unsigned short hb = __half_as_ushort(hh);
+                    if (!rk) {
+                        const float hf = __half2float(hh);
+                        const float up = __half2float(__ushort_as_half(static_cast<unsigned short>(hb + 1)));
+                        const float dn = __half2float(__ushort_as_half(static_cast<unsigned short>(hb - 1)));
+                        const float tol = 1e-6f * n32;
+                        rk = fabsf(n32 - 0.5f * (hf + up)) <= tol || fabsf(n32 - 0.5f * (hf + dn)) <= tol;
+                    }
+                    risky[g][i] = rk;
+                    any_risky = any_risky || rk;
+                    n_tok[g][i] = n32;
+                    n16[g][i] = hb;
+                }
+            if (__any_sync(kFull, any_risky)) {
+                // Rare: fp64 sums (all lanes join the shuffles).
+                double d[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint32_t m = mw[2 * a + q];
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const uint32_t w = i ? (q ? xb[a].y : xb[a].x) : (q ? xa[a].y : xa[a].x);
+                            const double e0 = __uint_as_float(w << 16), e1 = __uint_as_float(w & 0xffff0000u);
+                            const bool in0 = (m & 0xFFFFu) != 0, in1 = (m >> 16) != 0;
+                            d[0][i] += (in0 ? e0 * e0 : 0.0) + (in1 ? e1 * e1 : 0.0);
+                            d[1][i] += (in0 ? 0.0 : e0 * e0) + (in1 ? 0.0 : e1 * e1);
+                        }
+                    }
+#pragma unroll
+                for (int g = 0; g < 2; ++g)
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const double sd = warp4_sum_d(d[g][i]);
+                        if (risky[g][i]) {
+                            const double nd = sqrt(sd);
+                            n16[g][i] = __half_as_ushort(__double2half(nd));
+                            n_tok[g][i] = static_cast<float>(nd);
+                        }
+                    }
+            }
+        }
+        // A token with a norm not below 3e37 (inf, NaN, or so near the bf16 limit that the fp32 product
+        // could overflow) is packed as the zero vector with its norms as computed: every cell lookup
+        // below then stays inside the table.
+        {
+            const bool bad0 = !(n_tok[0][0] < 3.0e37f) || !(n_tok[1][0] < 3.0e37f);
+            const bool bad1 = !(n_tok[0][1] < 3.0e37f) || !(n_tok[1][1] < 3.0e37f);
+            if (__any_sync(kFull, bad0 || bad1)) {
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    if (bad0) xa[a] = make_uint2(0u, 0u);
+                    if (bad1) xb[a] = make_uint2(0u, 0u);
+                }
+            }
+        }
+        float kq[2][2];  // 64 / n_g per token: v = 64 u = acc * D * kq
+#pragma unroll
+        for (int g = 0; g < 2; ++g)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float k = n_tok[g][i] > 0.0f ? kCellScale / n_tok[g][i] : 0.0f;
+                if (!(k < 3.0e38f)) k = 0.0f;  // norms too small to scale: the zero vector
+                kq[g][i] = k;
+            }
+
+        // Q x in two halves of 8 n-tiles (outputs 64 HALF .. 64 HALF + 63), each over the 8 k-steps;
+        // then quantize and stage bytes (p, p + 1), p = 8 nt + 2 c, of tokens r and r + 8.
+        static_for<0, 2>([&](auto hc) {
+            constexpr int HALF = decltype(hc)::value;
+            float acc[8][4];
+#pragma unroll
+            for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int n = 0; n < 8; ++n) {
+                    const uint2 bf = lds64(qf_lane + static_cast<uint32_t>((a * 16 + 8 * HALF + n) * 32 * 8));
+                    mma_bf16_acc(acc[n], xa[a].x, xb[a].x, xa[a].y, xb[a].y, bf.x, bf.y);
+                }
+            static_for<0, 8>([&](auto nc) {
+                constexpr int n = decltype(nc)::value;
+                constexpr int NT = 8 * HALF + n;
+                constexpr int G = 8 * NT >= F::N0 ? 1 : 0;
+                constexpr float kScale = gw_block_scale<F>(8 * NT);
+                // address of cell round(v) + 64 = bits(v + 1.5 * 2^23) - 0x4B400000 + 64
+                constexpr uint32_t kTab = static_cast<uint32_t>(G * kCells) * 128u + 64u * 128u - 0x4B400000u * 128u;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float kv = kq[G][i] * kScale;
+                    const uint64_t vv = mul2(pk(acc[n][2 * i], acc[n][2 * i + 1]), pk(kv, kv));
+                    const uint64_t mm = add2(vv, pk(12582912.0f, 12582912.0f));
+                    float v0, v1, m0, m1;
+                    upk(vv, v0, v1);
+                    upk(mm, m0, m1);
+                    const uint2 e0 = lds64(__float_as_uint(m0) * 128u + cells_lane + kTab);
+                    const uint2 e1 = lds64(__float_as_uint(m1) * 128u + cells_lane + kTab);
+                    const uint32_t i0 = e0.y + (v0 > __uint_as_float(e0.x) ? 1u : 0u);
+                    const uint32_t i1 = e1.y + (v1 > __uint_as_float(e1.x) ? 1u : 0u);
+                    const uint32_t at = stage + static_cast<uint32_t>((r + 8 * i) * kStagePitch + 8 * NT + 2 * c);
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(at), "h"(static_cast<unsigned short>(i0 | (i1 << 8)))
+                                 : "memory");
+                }
+            });
+        });
+        if (c == 0) {
+            sm.norms[warp][r] = static_cast<uint32_t>(n16[0][0]) | (static_cast<uint32_t>(n16[1][0]) << 16);
+            sm.norms[warp][r + 8] = static_cast<uint32_t>(n16[0][1]) | (static_cast<uint32_t>(n16[1][1]) << 16);
+        }
+        __syncwarp();
+        assemble_rows<F>(stage, sm.rows[warp], lane);
+        __syncwarp();
+
+        // Write the rows in 8-byte pieces, and the two norms.
+        constexpr int ib = F::IB, rb = F::IB + 4;
+        constexpr int pieces = ib / 8;
+        for (int q = lane; q < 16 * pieces; q += 32) {
+            const int row = q / pieces, part = q - row * pieces;
+            const int slot = sm.slot32[warp][row];
+            if (slot >= 0 && slot < capacity) {
+                const int blk = bs_log2 >= 0 ? slot >> bs_log2 : slot / block_size;
+                const int off = slot - blk * block_size;
+                uint8_t* sub = pages + (static_cast<int64_t>(blk) * H + h) * block_size * rb;
+                *reinterpret_cast<uint2*>(sub + off * ib + 8 * part) =
+                    *reinterpret_cast<const uint2*>(&sm.rows[warp][row][8 * part]);
+                if (part == 0) *reinterpret_cast<uint32_t*>(sub + block_size * ib + 4 * off) = sm.norms[warp][row];
+            } else if (slot >= capacity && part == 0 && d_err) {
+                atomicOr(d_err, TQ_DERR_SLOT);
+            }
+        }
+        __syncwarp();
+    }
+}
+
 }  // namespace
 
-// Launches a tensor-core pack (uniform 4-bit, or another plain format); TQ_ERR_UNSUPPORTED when none applies.
+// Launches a tensor-core pack (uniform 4-bit, another plain format, or a group-wise
+// format); TQ_ERR_UNSUPPORTED when one of the two codecs has none.
 tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
                          const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
                          int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream) {
-    // Uniform 4-bit K and V: the 4-bit kernel. Other plain formats (no QJL stage, no group-wise
-    // rotation) with 2-, 3- and 4-bit groups and whole 8-byte index rows: the general tensor-core kernel.
-    bool u4 = true, plain = true;
-    for (const tq_codec* c : {kc, vc}) {
-        const tq_format_desc& d = c->desc;
+    // Uniform 4-bit K and V: the 4-bit kernel. Otherwise one launch per codec: plain formats (no QJL
+    // stage, no group-wise rotation) and group-wise formats without the QJL stage, with groups of
+    // 4 bits on 64 channels and 3 on 64, or 4 bits on 32 and 2 on 96 (plain also uniform 3 and 4 bits).
+    enum Kind { kNone, kU4, kU3, kM43, kM42, kGw43, kGw42 };
+    Kind kind[2];
+    bool u4 = true;
+    for (int side = 0; side < 2; ++side) {
+        const tq_format_desc& d = (side ? vc : kc)->desc;
         if (d.n_groups != 1 || d.group_bits[0] != 4 || d.qjl || d.groupwise) u4 = false;
-        const bool inst = (d.n_groups == 1 && (d.group_bits[0] == 4 || d.group_bits[0] == 3)) ||
-                          (d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 64 && d.group_bits[1] == 3) ||
-                          (d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 32 && d.group_bits[1] == 2);
-        if (d.qjl || d.groupwise || !inst || !c->dev.cells) plain = false;
+        const bool m43 = d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 64 && d.group_bits[1] == 3;
+        const bool m42 = d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 32 && d.group_bits[1] == 2;
+        Kind kd = kNone;
+        if (d.qjl || !(side ? vc : kc)->dev.cells) kd = kNone;
+        else if (d.groupwise) kd = m43 ? kGw43 : (m42 ? kGw42 : kNone);
+        else if (d.n_groups == 1 && d.group_bits[0] == 4) kd = kU4;
+        else if (d.n_groups == 1 && d.group_bits[0] == 3) kd = kU3;
+        else kd = m43 ? kM43 : (m42 ? kM42 : kNone);
+        kind[side] = kd;
     }
-    if (!u4 && !plain) return TQ_ERR_UNSUPPORTED;
+    if (kind[0] == kNone || kind[1] == kNone) return TQ_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 15) return TQ_ERR_UNSUPPORTED;
     if (block_size % 8 != 0) return TQ_ERR_UNSUPPORTED;  // 16-byte aligned rows and norm arrays
     // 32-bit index arithmetic in the kernel: slots, tokens and work units must fit.
     const int64_t capacity = num_blocks * block_size;
-    const int64_t n_units = (num_tokens + 15) / 16 * kc->desc.num_kv_heads * 2;
+    const int H = kc->desc.num_kv_heads;
+    const int64_t n_units = (num_tokens + 15) / 16 * H * 2;
     if (capacity > INT32_MAX || n_units > INT32_MAX || num_tokens > INT32_MAX - 16) return TQ_ERR_UNSUPPORTED;
     const int bs_log2 = (block_size & (block_size - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(block_size)) : -1;
-    // The quantizer cell table comes with the K codec (every uniform 4-bit
-    // codebook is the same). The kernel's shared-memory size is set once per
-    // device.
-    if (!kc->dev.cells || !vc->dev.cells) return TQ_ERR_UNSUPPORTED;
+    // The kernels' shared-memory sizes are set once per device.
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice failed");
     const cudaError_t err = once_per_device(dev, [] {
@@ -771,15 +1175,20 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sizeof(PackTcSmem)));
+        for (auto kern : {pack_gw_kernel<PM43>, pack_gw_kernel<PM42>})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(PackGwSmem)));
         return e;
     });
     if (err != cudaSuccess) return fail(TQ_ERR_CUDA, "pack fast path setup failed");
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t want = (n_units + kPW - 1) / kPW;
-    const int grid = static_cast<int>(want < sms ? want : sms);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (u4) {
+        // The quantizer cell table comes with the K codec (every uniform 4-bit codebook is the same).
+        const int64_t want = (n_units + kPW - 1) / kPW;
+        const int grid = static_cast<int>(want < sms ? want : sms);
         pack_u4_kernel<<<grid, kPW * 32, sizeof(PackSmem), st>>>(
             kc->dev, vc->dev, kc->dev.cells, static_cast<const __nv_bfloat16*>(k),
             static_cast<const __nv_bfloat16*>(v), slot_mapping, static_cast<int>(num_tokens),
@@ -787,22 +1196,31 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
             bs_log2, d_err);
         return TQ_OK;
     }
-    // One launch per codec; the grid covers that codec's units (half of the pair's).
-    const int64_t want1 = ((num_tokens + 15) / 16 * kc->desc.num_kv_heads + kPW - 1) / kPW;
+    // One launch per codec. Plain kernels: the grid covers that codec's units (half of the pair's).
+    // Group-wise kernels: CTAs keep one KV head, as many per head as fill the SMs (at least one).
+    const int64_t tgroups = (num_tokens + 15) / 16;
+    const int64_t want1 = (tgroups * H + kPW - 1) / kPW;
     const int grid1 = static_cast<int>(want1 < sms ? want1 : sms);
+    const int64_t per_head_want = (tgroups + kPW - 1) / kPW;
+    const int64_t per_head_fit = sms / H > 0 ? sms / H : 1;
+    const int per_head = static_cast<int>(per_head_want < per_head_fit ? per_head_want : per_head_fit);
     const struct { const tq_codec* c; const void* x; void* pages; } sides[2] = {{kc, k, k_pages}, {vc, v, v_pages}};
-    for (const auto& sd : sides) {
-        const tq_format_desc& d = sd.c->desc;
-        auto go = [&](auto kernel) {
-            kernel<<<grid1, kPW * 32, sizeof(PackTcSmem), st>>>(sd.c->dev, static_cast<const __nv_bfloat16*>(sd.x),
-                                                              slot_mapping, static_cast<int>(num_tokens),
-                                                              static_cast<uint8_t*>(sd.pages),
-                                                              static_cast<int>(capacity), block_size, bs_log2, d_err);
+    for (int side = 0; side < 2; ++side) {
+        const auto& sd = sides[side];
+        auto go = [&](auto kernel, int grid, size_t smem) {
+            kernel<<<grid, kPW * 32, smem, st>>>(sd.c->dev, static_cast<const __nv_bfloat16*>(sd.x), slot_mapping,
+                                                 static_cast<int>(num_tokens), static_cast<uint8_t*>(sd.pages),
+                                                 static_cast<int>(capacity), block_size, bs_log2, d_err);
         };
-        if (d.n_groups == 1 && d.group_bits[0] == 4) go(pack_tc_kernel<PU4>);
-        else if (d.n_groups == 1 && d.group_bits[0] == 3) go(pack_tc_kernel<PU3>);
-        else if (d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 64 && d.group_bits[1] == 3) go(pack_tc_kernel<PM43>);
-        else go(pack_tc_kernel<PM42>);
+        switch (kind[side]) {
+            case kU4: go(pack_tc_kernel<PU4>, grid1, sizeof(PackTcSmem)); break;
+            case kU3: go(pack_tc_kernel<PU3>, grid1, sizeof(PackTcSmem)); break;
+            case kM43: go(pack_tc_kernel<PM43>, grid1, sizeof(PackTcSmem)); break;
+            case kM42: go(pack_tc_kernel<PM42>, grid1, sizeof(PackTcSmem)); break;
+            case kGw43: go(pack_gw_kernel<PM43>, per_head * H, sizeof(PackGwSmem)); break;
+            case kGw42: go(pack_gw_kernel<PM42>, per_head * H, sizeof(PackGwSmem)); break;
+            default: break;
+        }
     }
     return TQ_OK;
 }

@@ -105,8 +105,8 @@ WORKLOADS = {
         "pack_llama8b_3p5bit_groupwise", "pack", 1012, 32, 32, 8, 128, 16, 0,
         (4, 3), (64, 64), (4, 3), (64, 64), 71, 72, 8, True, "fixed:8192", groupwise=True,
         description="pack 32 sequences x 8192 tokens, 8 KV heads, block 16, shuffled slot mapping, K and V "
-                    "3.5-bit group-wise (the group-wise decode workload's formats); general per-vector pack "
-                    "kernel"),
+                    "3.5-bit group-wise (the group-wise decode workload's formats); tensor-core group-wise "
+                    "pack kernel"),
     "decode_llama8b_4bit": Workload(
         "decode_llama8b_4bit", "decode", 1003, 64, 32, 8, 128, 16, 64,
         (4,), (128,), (4,), (128,), 0, 1, 8, True, "uniform:1024:32768",

@@ -224,16 +224,18 @@ def test_pack_edge_values_uniform_4bit_fast_path():
     assert np.array_equal(vp.cpu().numpy(), rv)
 
 
-@pytest.mark.parametrize("kspec,vspec,bs", [(((4,), (128,)), ((4,), (128,)), 16),
-                                             (((4, 3), (64, 64)), ((4, 3), (64, 64)), 16),
-                                             (((4, 2), (32, 96)), ((3,), (128,)), 32),
-                                             (((2,), (128,)), ((4, 3), (64, 64)), 48)])
-def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs):
-    """The tensor-core packs (uniform 4-bit, and the plain 2/3/4-bit mixes) against the general
-    kernel and the oracle on the same tokens."""
+@pytest.mark.parametrize("kspec,vspec,bs,gw", [(((4,), (128,)), ((4,), (128,)), 16, False),
+                                                (((4, 3), (64, 64)), ((4, 3), (64, 64)), 16, False),
+                                                (((4, 2), (32, 96)), ((3,), (128,)), 32, False),
+                                                (((2,), (128,)), ((4, 3), (64, 64)), 48, False),
+                                                (((4, 3), (64, 64)), ((4, 2), (32, 96)), 16, True),
+                                                (((4, 2), (32, 96)), ((4, 3), (64, 64)), 40, True)])
+def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs, gw):
+    """The tensor-core packs (uniform 4-bit, the plain 2/3/4-bit mixes, and the group-wise 4/3 and
+    4/2 formats) against the general kernel and the oracle on the same tokens."""
     H, T = 4, 700
-    kc, kf = codec_pair(H, *kspec, 8)
-    vc, vf = codec_pair(H, *vspec, 9)
+    kc, kf = codec_pair(H, *kspec, 8, groupwise=gw)
+    vc, vf = codec_pair(H, *vspec, 9, groupwise=gw)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(5)
     k, v = random_kv(T, H, gen)
@@ -254,6 +256,45 @@ def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs):
             compare_rows(rows_of(pages, s, bs, f, H), x, f, range(H))
         same = (out[0][i] == out[1][i]).mean()
         assert same > 0.999
+
+
+@pytest.mark.parametrize("kspec,vspec,mode", [(((4,), (128,)), ((4,), (128,)), ""),
+                                              (((4, 3), (64, 64)), ((4, 2), (32, 96)), ""),
+                                              (((4, 3), (64, 64)), ((4, 2), (32, 96)), "gw")])
+def test_pack_tokens_not_finite(monkeypatch, kspec, vspec, mode):
+    """Tokens holding inf, NaN or values near the bf16 limit (norms far beyond fp16) pack without
+    an error flag in the tensor-core kernels and the general one, and leave the rows of the other
+    tokens as the oracle has them."""
+    H, T, bs = 4, 200, 16
+    kc, kf = codec_pair(H, *kspec, 13, groupwise=mode == "gw")
+    vc, vf = codec_pair(H, *vspec, 14, groupwise=mode == "gw")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(77)
+    k, v = random_kv(T, H, gen)
+    k[3, 1, 5] = float("inf")
+    k[10, 0, :] = float("nan")
+    k[11, 2, 64:] = -float("inf")
+    v[20, 2, 7] = -float("inf")
+    v[21, 3, 100] = float("nan")
+    k[33, 3, 0] = 3.0e38
+    v[50, 1, :] = 2.0e38
+    bad_tokens = {3, 10, 11, 20, 21, 33, 50}
+    nb = -(-T // bs) + 1
+    slots = torch.as_tensor(np.random.default_rng(3).permutation(nb * bs)[:T], device="cuda")
+    for kernel in ("fast", "general"):
+        if kernel == "general":
+            monkeypatch.setenv("TQ_PACK_KERNEL", "general")
+        kp, vp = tq.page_pool(kc, nb, bs), tq.page_pool(vc, nb, bs)
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        tq.pack_kv(kc, vc, k, v, slots, kp, vp, bs, d_err=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        good = np.array([t for t in range(T) if t not in bad_tokens])
+        s = slots.cpu().numpy()[good]
+        for pages, src, f in ((kp, k, kf), (vp, v, vf)):
+            x = src[torch.as_tensor(good, device="cuda")].float().cpu().numpy().astype(np.float64)
+            flips, total = compare_rows(rows_of(pages.cpu().numpy(), s, bs, f, H), x, f, range(H))
+            assert flips <= max(1, MAX_FLIP_FRACTION * total)
 
 
 def test_pack_workload_whole_sequence_and_mse_full_size():
