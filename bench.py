@@ -206,12 +206,27 @@ class PackSetup:
         return T * H * D * 2 * 2 + T * H * (self.kc.row_bytes + self.vc.row_bytes) + T * 8
 
     def launches(self):
-        """Kernels per tq_pack_kv call: one for uniform 4-bit K and V (both sides in one grid) or for
-        the general kernel (QJL or group-wise rows); one per side for the other tensor-core formats."""
+        """Kernels per tq_pack_kv call, as the library dispatches them: one for uniform 4-bit K and V
+        (both sides in one grid); one per side when both sides have a tensor-core pack (plain 3/4-bit,
+        4+3 and 4+2 mixes; group-wise 4+3 and 4+2; QJL 3+2, 4+3, uniform 3 and 2 bits); else one
+        general launch."""
         ks, vs = WL.codec_specs(self.w)
-        plain = not (ks.qjl or ks.groupwise or vs.qjl or vs.groupwise)
-        u4 = tuple(self.w.k_bits) == (4,) and tuple(self.w.v_bits) == (4,)
-        return 2 if plain and not u4 else 1
+
+        def fast(spec):
+            shape = (tuple(spec.group_bits), tuple(spec.group_size))
+            mixes = {((4, 3), (64, 64)), ((4, 2), (32, 96))}
+            if spec.qjl and spec.groupwise:
+                return False
+            if spec.qjl:
+                return shape in {((3, 2), (64, 64)), ((4, 3), (64, 64)), ((3,), (128,)), ((2,), (128,))}
+            if spec.groupwise:
+                return shape in mixes
+            return shape in mixes | {((4,), (128,)), ((3,), (128,))}
+
+        if self.w.block_size % 8 or not (fast(ks) and fast(vs)):
+            return 1
+        u4 = all(tuple(sp.group_bits) == (4,) and not sp.qjl for sp in (ks, vs))
+        return 1 if u4 else 2
 
     def step(self):
         tq.pack_kv(self.kc, self.vc, self.k, self.v, self.slots, self.kp, self.vp, self.w.block_size, d_err=self.err)

@@ -540,10 +540,10 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out) {
     const size_t off_s = (n_sign + 2 * n_cent + 2 * n_perm + 15) / 16 * 16;
     const size_t n_s = c->qjl_s.size() * sizeof(float);
     const size_t off_r = (off_s + n_s + 15) / 16 * 16, n_r = c->rot_t.size() * sizeof(float);
-    // codecs without the QJL stage also carry the tensor-core pack's quantizer cell table of
-    // each group (when every cell holds at most one boundary)
+    // every codec also carries the tensor-core pack's quantizer cell table of each group (when
+    // every cell holds at most one boundary)
     std::vector<PackCell> cells;
-    if (!desc->qjl) {
+    {
         cells.resize(static_cast<size_t>(desc->n_groups) * kPackCells);
         bool ok = true;
         for (int g = 0; g < desc->n_groups; ++g)

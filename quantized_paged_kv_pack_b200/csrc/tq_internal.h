@@ -24,8 +24,8 @@ constexpr int kMaxLevels = 16;  // 4-bit codebooks at most on the GPU path
 // none). Adjacent boundaries of the 2-, 3- and 4-bit codebooks of dimension
 // 128 (and of the wider ones of smaller groups) are more than one unit of v
 // apart, so no cell holds two; build_pack_cells returns false if one does. A
-// codec without the QJL stage builds one per group on the host and copies them
-// to the device with its other tables.
+// codec builds one per group on the host and copies them to the device with its
+// other tables.
 constexpr int kPackCells = 129;
 constexpr float kPackCellScale = 64.0f;
 struct PackCell {
@@ -59,8 +59,8 @@ struct DevCodec {
                             // (n_g, residual norm_g) per group; qjl_st is then S_0^T then S_1^T (n_g x n_g)
     int32_t sign_off[2];    // byte offset of each group's QJL sign bits in the index part (QJL: the one
                             // stream after the index bitstreams)
-    const PackCell* cells;  // codecs without the QJL stage: the pack's quantizer cell table of each group [n_groups][129];
-                            // else null
+    const PackCell* cells;  // the pack's quantizer cell table of each group [n_groups][129]; null when a
+                            // cell would hold two boundaries
 };
 
 // Arguments of the decode kernels (device pointers; see tq_decode_paged).

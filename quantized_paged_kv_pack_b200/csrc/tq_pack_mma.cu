@@ -450,15 +450,31 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_u4_kernel(DevCodec kc, DevCo
 
 constexpr int kStagePitch = 132;
 
-struct PackTcSmem {
+// Warps per CTA and staged row pitch: the QJL variant runs 8 warps, which leaves room for the
+// fragments of S, and its rows carry 16 sign bytes after the index bytes.
+template <bool QJL>
+struct TcShape {
+    static constexpr int W = QJL ? 8 : kPW;
+    static constexpr int RP = QJL ? 88 : 72;
+};
+
+template <bool QJL>
+struct PackTcSmemBase {
+    static constexpr int W = TcShape<QJL>::W, RP = TcShape<QJL>::RP;
     QuantCell cells[3][kCells][16];  // codebooks of 2, 3, 4 bits (index bits - 2), 16 copies
     uint32_t bfrag[1][8][2][32][2];  // [codec][a][n-tile][lane][reg]: B operands (+-1 bf16 pairs)
-    uint8_t rows[kPW][16][72];       // staged index rows of a warp's 16 tokens (pitch 72: 16 rows, 16 bank pairs)
-    unsigned short norms[kPW][16];
-    int slot32[kPW][16];             // the unit's slots: -1 padding, capacity when past the pool
-    uint8_t xbuf[kPW][2][16][kRowPad];  // double-buffered input rows (bf16); the current one then stages indices
+    uint8_t rows[W][16][RP];         // staged rows of a warp's 16 tokens (pitch 72: 16 rows, 16 bank pairs)
+    uint32_t norms[W][16];           // the row's fp16 norm (QJL: and the residual norm above it)
+    int slot32[W][16];               // the unit's slots: -1 padding, capacity when past the pool
+    uint8_t xbuf[W][2][16][kRowPad];  // double-buffered input rows (bf16); the current one then stages indices
 };
+struct PackQjlSmem : PackTcSmemBase<true> {
+    uint32_t sfrag[2][8][16][32][2];  // [hi / lo][k-step][n-tile][lane][reg]: S as bf16 hi + lo B operands
+    float centv[2][16][32];           // [group][index][lane]: 64 x centroid (v units), one copy per lane
+};
+using PackTcSmem = PackTcSmemBase<false>;
 static_assert(16 * kStagePitch <= 16 * kRowPad, "index staging fits in an input buffer");
+static_assert(sizeof(PackTcSmem) <= 232448 && sizeof(PackQjlSmem) <= 232448, "fits the shared memory of one CTA");
 
 // The 8 indices (bytes) x0..x7 of lo = [x0 x1 x2 x3], hi = [x4 x5 x6 x7], b bits each, LSB-first.
 template <int B>
@@ -489,13 +505,31 @@ using PU4 = PackFmt<4, 128, 0, 0>;
 using PU3 = PackFmt<3, 128, 0, 0>;
 using PM43 = PackFmt<4, 64, 3, 64>;
 using PM42 = PackFmt<4, 32, 2, 96>;
+using PM32 = PackFmt<3, 64, 2, 64>;
+using PU2 = PackFmt<2, 128, 0, 0>;
+
+// Two floats as bf16x2 (round to nearest even; lo in the low half).
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// x = bf16 hi + bf16 lo for both halves (lo is the rounded remainder).
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    hi = bf16x2_rn(x0, x1);
+    lo = bf16x2_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xffff0000u));
+}
+// Bits 0-3 of x to bits 0, 2, 4, 6.
+__device__ __forceinline__ uint32_t spread4(uint32_t x) {
+    return (x & 1u) | ((x & 2u) << 1) | ((x & 4u) << 2) | ((x & 8u) << 3);
+}
 
 // Bit assembly of a warp's 16 staged index rows (one byte per packed position, pitch
 // kStagePitch): in round k lanes 0-15 take packed positions 16 k .. 16 k + 7 of token lane
 // and lanes 16-31 positions 16 k + 8 .. 16 k + 15 of token lane - 16 (one group for the
 // whole warp, since groups start on multiples of 16), into b bytes of the row, LSB-first.
-template <class F>
-__device__ __forceinline__ void assemble_rows(uint32_t stage, uint8_t (&rows)[16][72], int lane) {
+template <class F, int RP>
+__device__ __forceinline__ void assemble_rows(uint32_t stage, uint8_t (&rows)[16][RP], int lane) {
     const int tok = lane & 15, hi8 = (lane >> 4) * 8;
     const uint32_t srow = stage + static_cast<uint32_t>(tok * kStagePitch);
     uint8_t* drow = &rows[tok][0];
@@ -519,23 +553,46 @@ __device__ __forceinline__ void assemble_rows(uint32_t stage, uint8_t (&rows)[16
     });
 }
 
-template <class F>
-__global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const __nv_bfloat16* __restrict__ src,
+template <class F, bool QJL>
+__global__ void __launch_bounds__(TcShape<QJL>::W * 32, 1) pack_tc_kernel(DevCodec cd, const __nv_bfloat16* __restrict__ src,
                                                           const int64_t* __restrict__ slots, int num_tokens,
                                                           uint8_t* __restrict__ pages, int capacity, int block_size,
                                                           int bs_log2, int* __restrict__ d_err) {
+    static_assert(!QJL || F::NG == 1 || F::B0 != F::B1, "cell tables by bit width");
+    constexpr int kW = TcShape<QJL>::W;
+    using Smem = std::conditional_t<QJL, PackQjlSmem, PackTcSmem>;
     extern __shared__ __align__(16) uint8_t psm_raw[];
-    PackTcSmem& sm = *reinterpret_cast<PackTcSmem*>(psm_raw);
+    Smem& sm = *reinterpret_cast<Smem*>(psm_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, c = lane & 3;
 
     // Cell tables of the format's groups.
     for (int g = 0; g < F::NG; ++g) {
         const int bi = (g ? F::B1 : F::B0) - 2;
-        for (int i = threadIdx.x; i < kCells * 16; i += kPW * 32)
+        for (int i = threadIdx.x; i < kCells * 16; i += kW * 32)
             sm.cells[bi][i >> 4][i & 15] = cd.cells[g * kCells + (i >> 4)];
     }
-    for (int i = threadIdx.x; i < 8 * 2 * 32; i += kPW * 32) {
+    if constexpr (QJL) {
+        // B fragment (k-step a, n-tile nt) of lane (rr, cc): B[k][n] = S[8 nt + rr][16 a + k] for
+        // k = 2 cc + {0, 1} (reg 0) and 2 cc + 8 + {0, 1} (reg 1), split into bf16 hi + lo.
+        for (int i = threadIdx.x; i < 8 * 16 * 32; i += kW * 32) {
+            const int ln = i & 31, nt = (i >> 5) & 15, a = i >> 9;
+            const int n = 8 * nt + (ln >> 2), j0 = 16 * a + 2 * (ln & 3);
+            for (int q = 0; q < 2; ++q) {
+                const float s0 = cd.qjl_st[(j0 + 8 * q) * kHeadDim + n];  // S^T: entry (j, i) = S[i][j]
+                const float s1 = cd.qjl_st[(j0 + 8 * q + 1) * kHeadDim + n];
+                uint32_t hi, lo;
+                split_bf16x2(s0, s1, hi, lo);
+                sm.sfrag[0][a][nt][ln][q] = hi;
+                sm.sfrag[1][a][nt][ln][q] = lo;
+            }
+        }
+        for (int i = threadIdx.x; i < 2 * 16 * 32; i += kW * 32) {
+            const int g = i >> 9, k = (i >> 5) & 15;
+            sm.centv[g][k][i & 31] = g < F::NG ? kCellScale * cd.cent[g * kMaxLevels + k] : 0.0f;
+        }
+    }
+    for (int i = threadIdx.x; i < 8 * 2 * 32; i += kW * 32) {
         const int ln = i & 31, t = (i >> 5) & 1, a = (i >> 6) & 7;
         const int rr = ln >> 2, cc = ln & 3;
         const int bp = 8 * t + rr;
@@ -572,8 +629,8 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    const int stride = gridDim.x * kPW;
-    int u = blockIdx.x * kPW + warp;
+    const int stride = gridDim.x * kW;
+    int u = blockIdx.x * kW + warp;
     if (u < units) issue(u, 0);
     for (int it = 0; u < units; u += stride, ++it) {
         const int cur = it & 1;
@@ -600,6 +657,10 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
         const uint32_t stage = xbuf0 + cur * 16 * kRowPad;  // [16][kStagePitch] index bytes, packed order
         float n_tok[2];
         unsigned short n16[2];
+        // QJL: the residuals r = u - c[idx] (in units of v = 64 u) as the S product's A fragments,
+        // bf16 hi + lo: [a][2 t + token] covers coordinates 16 a + 8 t + 2 c + {0, 1}
+        uint32_t rh[8][4], rl[8][4];
+        float rr[2] = {0.0f, 0.0f};  // sums of squared residuals per token (v units)
         // the lane's indices: idxr[t][a] bytes (j, token r), (j + 1, token r), (j, token r + 8), (j + 1, token r + 8)
         uint32_t idxr[2][8];
         const int16_t* posh = cd.pos + h * kHeadDim;
@@ -744,11 +805,12 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
                                            0x4B400000u * 128u;
                 constexpr uint32_t kTab1 = static_cast<uint32_t>(((F::NG == 2 ? F::B1 : F::B0) - 2) * kCells) * 128u +
                                            64u * 128u - 0x4B400000u * 128u;
-                uint32_t tab[2];
+                uint32_t tab[2], cen[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int pe = static_cast<int>((pp >> (16 * e)) & 0xffffu);
                     tab[e] = cells_lane + ((ng == 2 && pe >= n0) ? kTab1 : kTab0);
+                    cen[e] = (ng == 2 && pe >= n0) ? 16u * 128u : 0u;
                 }
                 uint32_t w = 0;
 #pragma unroll
@@ -763,6 +825,13 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
                     const uint32_t i0 = e0.y + (v0 > __uint_as_float(e0.x) ? 1u : 0u);
                     const uint32_t i1 = e1.y + (v1 > __uint_as_float(e1.x) ? 1u : 0u);
                     w |= (i0 | (i1 << 8)) << (16 * i);
+                    if constexpr (QJL) {
+                        const uint32_t cl = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.centv[0][0][lane]));
+                        const float q0 = v0 - __uint_as_float(lds32(cl + cen[0] + i0 * 128u));
+                        const float q1 = v1 - __uint_as_float(lds32(cl + cen[1] + i1 * 128u));
+                        rr[i] = fmaf(q0, q0, fmaf(q1, q1, rr[i]));
+                        split_bf16x2(q0, q1, rh[a][2 * t + i], rl[a][2 * t + i]);
+                    }
                 }
                 idxr[t][a] = w;
             }
@@ -785,17 +854,64 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
                                  : "memory");
                 }
             }
+        uint32_t g16[2] = {0u, 0u};
+        if constexpr (QJL) {
+            // Residual norms |r| = sqrt(sum of squares in v units) / 64, fp16.
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float q = rr[i];
+                q += __shfl_xor_sync(kFull, q, 1);
+                q += __shfl_xor_sync(kFull, q, 2);
+                g16[i] = __half_as_ushort(__float2half_rn(sqrtf(q) * (1.0f / kCellScale)));
+            }
+            // S r on the tensor cores (hi x hi + lo x hi + hi x lo, fp32 accumulation), four n-tiles
+            // at a time; sign bit of output i = 8 nt + 2 c + e is (S r)_i >= 0, byte nt of the sign
+            // stream, bit 2 c + e.
+            const uint32_t sf_lane = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.sfrag[0][0][0][lane][0]));
+            constexpr uint32_t kLoOff = 8u * 16u * 32u * 8u;
+#pragma unroll
+            for (int n4 = 0; n4 < 4; ++n4) {
+                float acc[4][4];
+#pragma unroll
+                for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) {
+                        const uint32_t off = static_cast<uint32_t>((a * 16 + 4 * n4 + n) * 32 * 8);
+                        const uint2 bh = lds64(sf_lane + off), bl = lds64(sf_lane + kLoOff + off);
+                        mma_bf16_acc(acc[n], rh[a][0], rh[a][1], rh[a][2], rh[a][3], bh.x, bh.y);
+                        mma_bf16_acc(acc[n], rl[a][0], rl[a][1], rl[a][2], rl[a][3], bh.x, bh.y);
+                        mma_bf16_acc(acc[n], rh[a][0], rh[a][1], rh[a][2], rh[a][3], bl.x, bl.y);
+                    }
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    const uint32_t s0 = __ballot_sync(kFull, acc[n][0] >= 0.0f);
+                    const uint32_t s1 = __ballot_sync(kFull, acc[n][1] >= 0.0f);
+                    const uint32_t s2 = __ballot_sync(kFull, acc[n][2] >= 0.0f);
+                    const uint32_t s3 = __ballot_sync(kFull, acc[n][3] >= 0.0f);
+                    if (c == 0) {
+                        const int sh = 4 * r;
+                        sm.rows[warp][r][F::IB + 4 * n4 + n] =
+                            static_cast<uint8_t>(spread4((s0 >> sh) & 0xFu) | (spread4((s1 >> sh) & 0xFu) << 1));
+                        sm.rows[warp][r + 8][F::IB + 4 * n4 + n] =
+                            static_cast<uint8_t>(spread4((s2 >> sh) & 0xFu) | (spread4((s3 >> sh) & 0xFu) << 1));
+                    }
+                }
+            }
+        }
         if (c == 0) {
-            sm.norms[warp][r] = n16[0];
-            sm.norms[warp][r + 8] = n16[1];
+            sm.norms[warp][r] = static_cast<uint32_t>(n16[0]) | (g16[0] << 16);
+            sm.norms[warp][r + 8] = static_cast<uint32_t>(n16[1]) | (g16[1] << 16);
         }
         __syncwarp();
 
         assemble_rows<F>(stage, sm.rows[warp], lane);
         __syncwarp();
 
-        // Write the rows in 8-byte pieces (index rows are whole multiples of 8 bytes), and the norms.
-        constexpr int ib = F::IB, rb = F::IB + 2;
+        // Write the rows in 8-byte pieces (index rows, and with QJL their 16 sign bytes, are whole
+        // multiples of 8 bytes), and the norms.
+        constexpr int ib = F::IB + (QJL ? 16 : 0), rb = ib + (QJL ? 4 : 2);
         const int pieces = ib / 8;
         for (int q = lane; q < 16 * pieces; q += 32) {
             const int row = q / pieces, part = q - row * pieces;
@@ -806,8 +922,13 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_tc_kernel(DevCodec cd, const
                 uint8_t* sub = pages + (static_cast<int64_t>(blk) * H + h) * block_size * rb;
                 *reinterpret_cast<uint2*>(sub + off * ib + 8 * part) =
                     *reinterpret_cast<const uint2*>(&sm.rows[warp][row][8 * part]);
-                if (part == 0)
-                    *reinterpret_cast<unsigned short*>(sub + block_size * ib + 2 * off) = sm.norms[warp][row];
+                if (part == 0) {
+                    if constexpr (QJL)
+                        *reinterpret_cast<uint32_t*>(sub + block_size * ib + 4 * off) = sm.norms[warp][row];
+                    else
+                        *reinterpret_cast<unsigned short*>(sub + block_size * ib + 2 * off) =
+                            static_cast<unsigned short>(sm.norms[warp][row]);
+                }
             } else if (slot >= capacity && part == 0 && d_err) {
                 atomicOr(d_err, TQ_DERR_SLOT);
             }
@@ -1139,8 +1260,10 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
                          int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream) {
     // Uniform 4-bit K and V: the 4-bit kernel. Otherwise one launch per codec: plain formats (no QJL
     // stage, no group-wise rotation) and group-wise formats without the QJL stage, with groups of
-    // 4 bits on 64 channels and 3 on 64, or 4 bits on 32 and 2 on 96 (plain also uniform 3 and 4 bits).
-    enum Kind { kNone, kU4, kU3, kM43, kM42, kGw43, kGw42 };
+    // 4 bits on 64 channels and 3 on 64, or 4 bits on 32 and 2 on 96 (plain also uniform 3 and 4
+    // bits); QJL formats (without group-wise rotation) of 3 bits on 64 channels and 2 on 64, 4 on 64
+    // and 3 on 64, or uniform 3 or 2 bits.
+    enum Kind { kNone, kU4, kU3, kM43, kM42, kGw43, kGw42, kQ32, kQ43, kQu3, kQu2 };
     Kind kind[2];
     bool u4 = true;
     for (int side = 0; side < 2; ++side) {
@@ -1148,8 +1271,15 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
         if (d.n_groups != 1 || d.group_bits[0] != 4 || d.qjl || d.groupwise) u4 = false;
         const bool m43 = d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 64 && d.group_bits[1] == 3;
         const bool m42 = d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 32 && d.group_bits[1] == 2;
+        const bool m32 = d.n_groups == 2 && d.group_bits[0] == 3 && d.group_size[0] == 64 && d.group_bits[1] == 2;
         Kind kd = kNone;
-        if (d.qjl || !(side ? vc : kc)->dev.cells) kd = kNone;
+        if (!(side ? vc : kc)->dev.cells || (d.qjl && d.groupwise)) kd = kNone;
+        else if (d.qjl)
+            kd = m32 ? kQ32
+                     : (m43 ? kQ43
+                            : (d.n_groups == 1 && d.group_bits[0] == 3
+                                   ? kQu3
+                                   : (d.n_groups == 1 && d.group_bits[0] == 2 ? kQu2 : kNone)));
         else if (d.groupwise) kd = m43 ? kGw43 : (m42 ? kGw42 : kNone);
         else if (d.n_groups == 1 && d.group_bits[0] == 4) kd = kU4;
         else if (d.n_groups == 1 && d.group_bits[0] == 3) kd = kU3;
@@ -1171,10 +1301,16 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
     const cudaError_t err = once_per_device(dev, [] {
         cudaError_t e = cudaFuncSetAttribute(pack_u4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(sizeof(PackSmem)));
-        for (auto kern : {pack_tc_kernel<PU4>, pack_tc_kernel<PU3>, pack_tc_kernel<PM43>, pack_tc_kernel<PM42>})
+        for (auto kern : {pack_tc_kernel<PU4, false>, pack_tc_kernel<PU3, false>, pack_tc_kernel<PM43, false>,
+                          pack_tc_kernel<PM42, false>})
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sizeof(PackTcSmem)));
+        for (auto kern : {pack_tc_kernel<PM32, true>, pack_tc_kernel<PM43, true>, pack_tc_kernel<PU3, true>,
+                          pack_tc_kernel<PU2, true>})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(PackQjlSmem)));
         for (auto kern : {pack_gw_kernel<PM43>, pack_gw_kernel<PM42>})
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1201,22 +1337,29 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
     const int64_t tgroups = (num_tokens + 15) / 16;
     const int64_t want1 = (tgroups * H + kPW - 1) / kPW;
     const int grid1 = static_cast<int>(want1 < sms ? want1 : sms);
+    constexpr int kQW = TcShape<true>::W;
+    const int64_t wantq = (tgroups * H + kQW - 1) / kQW;
+    const int gridq = static_cast<int>(wantq < sms ? wantq : sms);
     const int64_t per_head_want = (tgroups + kPW - 1) / kPW;
     const int64_t per_head_fit = sms / H > 0 ? sms / H : 1;
     const int per_head = static_cast<int>(per_head_want < per_head_fit ? per_head_want : per_head_fit);
     const struct { const tq_codec* c; const void* x; void* pages; } sides[2] = {{kc, k, k_pages}, {vc, v, v_pages}};
     for (int side = 0; side < 2; ++side) {
         const auto& sd = sides[side];
-        auto go = [&](auto kernel, int grid, size_t smem) {
-            kernel<<<grid, kPW * 32, smem, st>>>(sd.c->dev, static_cast<const __nv_bfloat16*>(sd.x), slot_mapping,
+        auto go = [&](auto kernel, int grid, size_t smem, int warps = kPW) {
+            kernel<<<grid, warps * 32, smem, st>>>(sd.c->dev, static_cast<const __nv_bfloat16*>(sd.x), slot_mapping,
                                                  static_cast<int>(num_tokens), static_cast<uint8_t*>(sd.pages),
                                                  static_cast<int>(capacity), block_size, bs_log2, d_err);
         };
         switch (kind[side]) {
-            case kU4: go(pack_tc_kernel<PU4>, grid1, sizeof(PackTcSmem)); break;
-            case kU3: go(pack_tc_kernel<PU3>, grid1, sizeof(PackTcSmem)); break;
-            case kM43: go(pack_tc_kernel<PM43>, grid1, sizeof(PackTcSmem)); break;
-            case kM42: go(pack_tc_kernel<PM42>, grid1, sizeof(PackTcSmem)); break;
+            case kU4: go(pack_tc_kernel<PU4, false>, grid1, sizeof(PackTcSmem)); break;
+            case kU3: go(pack_tc_kernel<PU3, false>, grid1, sizeof(PackTcSmem)); break;
+            case kM43: go(pack_tc_kernel<PM43, false>, grid1, sizeof(PackTcSmem)); break;
+            case kM42: go(pack_tc_kernel<PM42, false>, grid1, sizeof(PackTcSmem)); break;
+            case kQ32: go(pack_tc_kernel<PM32, true>, gridq, sizeof(PackQjlSmem), kQW); break;
+            case kQ43: go(pack_tc_kernel<PM43, true>, gridq, sizeof(PackQjlSmem), kQW); break;
+            case kQu3: go(pack_tc_kernel<PU3, true>, gridq, sizeof(PackQjlSmem), kQW); break;
+            case kQu2: go(pack_tc_kernel<PU2, true>, gridq, sizeof(PackQjlSmem), kQW); break;
             case kGw43: go(pack_gw_kernel<PM43>, per_head * H, sizeof(PackGwSmem)); break;
             case kGw42: go(pack_gw_kernel<PM42>, per_head * H, sizeof(PackGwSmem)); break;
             default: break;

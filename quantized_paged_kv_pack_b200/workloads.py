@@ -99,8 +99,8 @@ WORKLOADS = {
         "pack_llama8b_3p5bit_qjl", "pack", 1011, 32, 32, 8, 128, 16, 0,
         (3, 2), (64, 64), (4, 3), (64, 64), 61, 62, 8, True, "fixed:8192", k_qjl=True,
         description="pack 32 sequences x 8192 tokens, 8 KV heads, block 16, shuffled slot mapping, the QJL "
-                    "decode workload's formats (K 2.5-bit MSE plus the 1-bit QJL stage, V 3.5-bit); general "
-                    "per-vector pack kernel"),
+                    "decode workload's formats (K 2.5-bit MSE plus the 1-bit QJL stage, V 3.5-bit); QJL "
+                    "tensor-core pack for K, plain tensor-core pack for V"),
     "pack_llama8b_3p5bit_groupwise": Workload(
         "pack_llama8b_3p5bit_groupwise", "pack", 1012, 32, 32, 8, 128, 16, 0,
         (4, 3), (64, 64), (4, 3), (64, 64), 71, 72, 8, True, "fixed:8192", groupwise=True,

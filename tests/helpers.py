@@ -140,3 +140,46 @@ def workload_codecs(w):
     vf = O.Format(D, w.num_kv_heads, vs.group_bits, vs.group_size, vs.high_coords, vs.seed, qjl=vs.qjl,
                   groupwise=vs.groupwise)
     return kc, vc, kf, vf
+
+
+QJL_BOUNDARY_REL = 1e-5  # near-boundary exemption for index mismatches
+SIGN_REL = 1e-4  # a sign may differ only where |(S r)_i| is this small against |r| sqrt(d)
+
+
+def check_qjl_rows(rows, x, fmt, heads):
+    """GPU rows [N][H][row] against the oracle's QJL quantization of x [N][H][d]."""
+    compared = 0
+    for h in heads:
+        f1 = slice_format(fmt, h)
+        idx, n16, u, signs, g16 = O.quantize_qjl(x[:, h], f1, 0)
+        gidx, gn16, gsigns, gg16 = O.decode_rows(rows[:, h], f1)
+        assert np.array_equal(gn16.astype(np.float16).view(np.uint16), n16.astype(np.float16).view(np.uint16))
+        bad = np.any(gidx != idx, axis=-1)  # vectors with an index flip at a boundary
+        if bad.any():
+            margin = O.boundary_margin(u, f1)
+            flips = gidx != idx
+            assert np.all(margin[flips] <= QJL_BOUNDARY_REL), "index mismatch away from a codebook boundary"
+        ok = ~bad
+        # residual norms: fp16 of |r|, equal unless |r| sits at an fp16 rounding midpoint
+        gd = gg16[ok] != g16[ok]
+        if gd.any():
+            rel = np.abs(gg16[ok][gd] - g16[ok][gd]) / np.maximum(g16[ok][gd], 1e-30)
+            assert np.all(rel < 2e-3), "residual norm differs by more than one fp16 step"
+            assert gd.sum() <= max(2, 0.002 * ok.sum())
+        # signs: equal except where the projection is negligibly small
+        r = np.empty(u.shape)
+        perm = O.permutation(f1, 0)
+        start = 0
+        chat = np.empty(u.shape)
+        for b, size in zip(f1.group_bits, f1.group_size):
+            cb, _ = O.codebook(b, D)
+            chat[:, start:start + size] = cb[idx[:, start:start + size]]
+            start += size
+        r[:, perm] = u - chat
+        proj = r @ O.qjl_matrix(f1).T
+        scale = np.linalg.norm(r, axis=-1, keepdims=True) * math.sqrt(D)
+        diff = (gsigns != signs) & ok[:, None]
+        assert np.all(np.abs(proj[diff]) <= SIGN_REL * np.broadcast_to(scale, proj.shape)[diff]), \
+            "QJL sign mismatch away from zero"
+        compared += int(ok.sum())
+    return compared

@@ -11,7 +11,7 @@ from oracle import tq_oracle as O
 from quantized_paged_kv_pack_b200 import tq
 from quantized_paged_kv_pack_b200 import workloads as W
 
-from helpers import D, codec_pair, random_kv, slice_format, workload_codecs
+from helpers import D, check_qjl_rows, codec_pair, random_kv, slice_format, workload_codecs
 
 pytestmark = pytest.mark.gpu
 
@@ -224,26 +224,28 @@ def test_pack_edge_values_uniform_4bit_fast_path():
     assert np.array_equal(vp.cpu().numpy(), rv)
 
 
-@pytest.mark.parametrize("kspec,vspec,bs,gw", [(((4,), (128,)), ((4,), (128,)), 16, False),
-                                                (((4, 3), (64, 64)), ((4, 3), (64, 64)), 16, False),
-                                                (((4, 2), (32, 96)), ((3,), (128,)), 32, False),
-                                                (((2,), (128,)), ((4, 3), (64, 64)), 48, False),
-                                                (((4, 3), (64, 64)), ((4, 2), (32, 96)), 16, True),
-                                                (((4, 2), (32, 96)), ((4, 3), (64, 64)), 40, True)])
-def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs, gw):
-    """The tensor-core packs (uniform 4-bit, the plain 2/3/4-bit mixes, and the group-wise 4/3 and
-    4/2 formats) against the general kernel and the oracle on the same tokens."""
+@pytest.mark.parametrize("kspec,vspec,bs,mode", [(((4,), (128,)), ((4,), (128,)), 16, ""),
+                                                  (((4, 3), (64, 64)), ((4, 3), (64, 64)), 16, ""),
+                                                  (((4, 2), (32, 96)), ((3,), (128,)), 32, ""),
+                                                  (((2,), (128,)), ((4, 3), (64, 64)), 48, ""),
+                                                  (((4, 3), (64, 64)), ((4, 2), (32, 96)), 16, "gw"),
+                                                  (((4, 2), (32, 96)), ((4, 3), (64, 64)), 40, "gw"),
+                                                  (((3, 2), (64, 64)), ((4, 3), (64, 64)), 16, "qjl"),
+                                                  (((3,), (128,)), ((2,), (128,)), 24, "qjl")])
+def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs, mode):
+    """The tensor-core packs (uniform 4-bit, the plain 2/3/4-bit mixes, the group-wise 4/3 and 4/2
+    formats, and QJL formats) against the general kernel and the oracle on the same tokens."""
     H, T = 4, 700
-    kc, kf = codec_pair(H, *kspec, 8, groupwise=gw)
-    vc, vf = codec_pair(H, *vspec, 9, groupwise=gw)
+    kc, kf = codec_pair(H, *kspec, 8, qjl=mode == "qjl", groupwise=mode == "gw")
+    vc, vf = codec_pair(H, *vspec, 9, qjl=mode == "qjl", groupwise=mode == "gw")
     gen = torch.Generator(device="cuda")
     gen.manual_seed(5)
     k, v = random_kv(T, H, gen)
     nb = -(-T // bs) + 2
     slots = torch.as_tensor(np.random.default_rng(1).permutation(nb * bs)[:T], device="cuda")
     out = []
-    for mode in ("fast", "general"):
-        if mode == "general":
+    for kernel in ("fast", "general"):
+        if kernel == "general":
             monkeypatch.setenv("TQ_PACK_KERNEL", "general")
         kp, vp = tq.page_pool(kc, nb, bs), tq.page_pool(vc, nb, bs)
         tq.pack_kv(kc, vc, k, v, slots, kp, vp, bs)
@@ -253,21 +255,25 @@ def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs, gw):
     for i, (src, f) in enumerate(((k, kf), (v, vf))):
         x = src.float().cpu().numpy().astype(np.float64)
         for pages in (out[0][i], out[1][i]):
-            compare_rows(rows_of(pages, s, bs, f, H), x, f, range(H))
+            if mode == "qjl":
+                assert check_qjl_rows(rows_of(pages, s, bs, f, H), x, f, range(H)) > 0.99 * T * H
+            else:
+                compare_rows(rows_of(pages, s, bs, f, H), x, f, range(H))
         same = (out[0][i] == out[1][i]).mean()
         assert same > 0.999
 
 
 @pytest.mark.parametrize("kspec,vspec,mode", [(((4,), (128,)), ((4,), (128,)), ""),
                                               (((4, 3), (64, 64)), ((4, 2), (32, 96)), ""),
-                                              (((4, 3), (64, 64)), ((4, 2), (32, 96)), "gw")])
+                                              (((4, 3), (64, 64)), ((4, 2), (32, 96)), "gw"),
+                                              (((3, 2), (64, 64)), ((3,), (128,)), "qjl")])
 def test_pack_tokens_not_finite(monkeypatch, kspec, vspec, mode):
     """Tokens holding inf, NaN or values near the bf16 limit (norms far beyond fp16) pack without
     an error flag in the tensor-core kernels and the general one, and leave the rows of the other
     tokens as the oracle has them."""
     H, T, bs = 4, 200, 16
-    kc, kf = codec_pair(H, *kspec, 13, groupwise=mode == "gw")
-    vc, vf = codec_pair(H, *vspec, 14, groupwise=mode == "gw")
+    kc, kf = codec_pair(H, *kspec, 13, qjl=mode == "qjl", groupwise=mode == "gw")
+    vc, vf = codec_pair(H, *vspec, 14, qjl=mode == "qjl", groupwise=mode == "gw")
     gen = torch.Generator(device="cuda")
     gen.manual_seed(77)
     k, v = random_kv(T, H, gen)
@@ -293,8 +299,12 @@ def test_pack_tokens_not_finite(monkeypatch, kspec, vspec, mode):
         s = slots.cpu().numpy()[good]
         for pages, src, f in ((kp, k, kf), (vp, v, vf)):
             x = src[torch.as_tensor(good, device="cuda")].float().cpu().numpy().astype(np.float64)
-            flips, total = compare_rows(rows_of(pages.cpu().numpy(), s, bs, f, H), x, f, range(H))
-            assert flips <= max(1, MAX_FLIP_FRACTION * total)
+            rows = rows_of(pages.cpu().numpy(), s, bs, f, H)
+            if mode == "qjl":
+                assert check_qjl_rows(rows, x, f, range(H)) > 0.99 * len(good) * H
+            else:
+                flips, total = compare_rows(rows, x, f, range(H))
+                assert flips <= max(1, MAX_FLIP_FRACTION * total)
 
 
 def test_pack_workload_whole_sequence_and_mse_full_size():
