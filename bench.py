@@ -41,7 +41,7 @@ DECODE_LAUNCHES = 3  # per step: prologue (work list, query rotation, windows, t
 EXTRA = ["decode_llama8b_4bit", "decode_llama8b_2p5bit", "decode_llama8b_3p5bit_qjl",
          "decode_llama8b_3p5bit_groupwise", "decode_llama8b_3p5bit_recipe",
          "pack_llama8b_4bit", "pack_llama70b_3p5bit", "pack_llama8b_2p5bit", "pack_llama8b_3p5bit_qjl",
-         "pack_llama8b_3p5bit_groupwise"]
+         "pack_llama8b_3p5bit_groupwise", "pack_llama8b_3p5bit_recipe"]
 D = 128
 METRIC = "paged TQ decode HBM GB/s (algorithmic bytes / step time)"
 
@@ -208,15 +208,15 @@ class PackSetup:
     def launches(self):
         """Kernels per tq_pack_kv call, as the library dispatches them: one for uniform 4-bit K and V
         (both sides in one grid); one per side when both sides have a tensor-core pack (plain 3/4-bit,
-        4+3 and 4+2 mixes; group-wise 4+3 and 4+2; QJL 3+2, 4+3, uniform 3 and 2 bits); else one
-        general launch."""
+        4+3 and 4+2 mixes; group-wise 4+3 and 4+2; QJL 3+2, 4+3, uniform 3 and 2 bits; recipe rows
+        3+2 and 4+3); else one general launch."""
         ks, vs = WL.codec_specs(self.w)
 
         def fast(spec):
             shape = (tuple(spec.group_bits), tuple(spec.group_size))
             mixes = {((4, 3), (64, 64)), ((4, 2), (32, 96))}
             if spec.qjl and spec.groupwise:
-                return False
+                return shape in {((3, 2), (64, 64)), ((4, 3), (64, 64))}
             if spec.qjl:
                 return shape in {((3, 2), (64, 64)), ((4, 3), (64, 64)), ((3,), (128,)), ((2,), (128,))}
             if spec.groupwise:

@@ -954,16 +954,37 @@ __global__ void __launch_bounds__(TcShape<QJL>::W * 32, 1) pack_tc_kernel(DevCod
 // the packed position), bit assembly and row writes follow the plain kernel; a
 // row ends in the two fp16 group norms.
 
-struct PackGwSmem {
+// The recipe variant (group-wise rotation plus each group's QJL stage) runs 8 warps, which leaves
+// room for the fragments of S_0 and S_1.
+template <bool RECIPE>
+struct PackGwSmemBase {
+    static constexpr int W = RECIPE ? 8 : kPW;
     QuantCell cells[2][kCells][16];   // codebook cells of group 0 and group 1, 16 copies
     uint32_t qfrag[8][16][32][2];     // [k-step][n-tile][lane][reg]: Q^T of the CTA's head, bf16 pairs
     uint4 gmask[4][32];               // [word / 4][lane]: the lane's group-0 channels as bf16 half masks
-    uint8_t rows[kPW][16][72];        // staged index rows
-    uint32_t norms[kPW][16];          // the row's two fp16 group norms
-    int slot32[kPW][16];              // the unit's slots: -1 padding, capacity when past the pool
-    uint8_t xbuf[kPW][2][16][kRowPad];  // double-buffered input rows; the current one then stages indices
+    uint8_t rows[W][16][72];          // staged rows
+    uint2 norms[W][16];               // the row's fp16 norms: n_0 | n_1 << 16 (recipe: n_0, g_0, n_1, g_1)
+    int slot32[W][16];                // the unit's slots: -1 padding, capacity when past the pool
+    uint8_t xbuf[W][2][16][kRowPad];  // double-buffered input rows; the current one then stages indices
 };
-static_assert(sizeof(PackGwSmem) <= 232448, "fits the shared memory of one CTA");
+struct PackRecipeSmem : PackGwSmemBase<true> {
+    uint32_t sfrag[2][2][4][8][32][2];  // [group][hi / lo][k-step][n-tile][lane][reg]: S_g as bf16 hi + lo
+    float centv[2][16][32];             // [group][index][lane]: 64 x centroid (v units), one copy per lane
+};
+using PackGwSmem = PackGwSmemBase<false>;
+static_assert(sizeof(PackGwSmem) <= 232448 && sizeof(PackRecipeSmem) <= 232448, "fits the shared memory of one CTA");
+
+// Row layout of the recipe row (two groups, each [indices][QJL signs], then the four fp16 norms):
+// the same group fields as F with group 1's indices after group 0's sign bytes.
+template <class F>
+struct RecipeOf {
+    static constexpr int B0 = F::B0, N0 = F::N0, B1 = F::B1, N1 = F::N1, NG = 2;
+    static constexpr int SIGN0 = B0 * N0 / 8;                 // group 0's sign bytes
+    static constexpr int BOFF1 = SIGN0 + N0 / 8;              // group 1's index bytes
+    static constexpr int SIGN1 = BOFF1 + B1 * N1 / 8;         // group 1's sign bytes
+    static constexpr int IB = SIGN1 + N1 / 8;                 // index part of a row
+    static_assert(IB % 8 == 0 && IB <= 72, "whole 8-byte index parts within the staged row");
+};
 
 // 1/sqrt(m) of the Hadamard block that holds packed position p (each group's
 // blocks in decreasing powers of two, as the codec builds R_h).
@@ -981,25 +1002,29 @@ __host__ __device__ constexpr float gw_block_scale(int p) {
     return 0.0f;
 }
 
-template <class F>
-__global__ void __launch_bounds__(kPW * 32, 1) pack_gw_kernel(DevCodec cd, const __nv_bfloat16* __restrict__ src,
+template <class F, bool RECIPE>
+__global__ void __launch_bounds__(PackGwSmemBase<RECIPE>::W * 32, 1) pack_gw_kernel(DevCodec cd, const __nv_bfloat16* __restrict__ src,
                                                           const int64_t* __restrict__ slots, int num_tokens,
                                                           uint8_t* __restrict__ pages, int capacity, int block_size,
                                                           int bs_log2, int* __restrict__ d_err) {
     static_assert(F::NG == 2 && F::N0 % 16 == 0, "two groups starting on a multiple of 16");
+    static_assert(!RECIPE || (F::N0 == 64 && F::N1 == 64), "recipe rows: one group per half of the product");
+    constexpr int kW = PackGwSmemBase<RECIPE>::W;
+    using Smem = std::conditional_t<RECIPE, PackRecipeSmem, PackGwSmem>;
+    using FR = std::conditional_t<RECIPE, RecipeOf<F>, F>;  // the row layout
     extern __shared__ __align__(16) uint8_t psm_raw[];
-    PackGwSmem& sm = *reinterpret_cast<PackGwSmem*>(psm_raw);
+    Smem& sm = *reinterpret_cast<Smem*>(psm_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, c = lane & 3;
     const int H = cd.num_heads;
     const int h = blockIdx.x % H, cta = blockIdx.x / H, ctas = gridDim.x / H;
 
     // Cell tables (group g's cells at g * kCells in the codec's table).
-    for (int i = threadIdx.x; i < 2 * kCells * 16; i += kPW * 32) (&sm.cells[0][0][0])[i] = cd.cells[i >> 4];
+    for (int i = threadIdx.x; i < 2 * kCells * 16; i += kW * 32) (&sm.cells[0][0][0])[i] = cd.cells[i >> 4];
     // B fragment (k-step a, n-tile nt) of lane (rr, cc): B[k][n] = sign of R_h[8 nt + rr][16 a + k] for
     // k = 2 cc + {0, 1} (reg 0) and 2 cc + 8 + {0, 1} (reg 1).
     const float* rt = cd.rot_t + static_cast<int64_t>(h) * kHeadDim * kHeadDim;  // entry (j, p) = R_h[p][j]
-    for (int i = threadIdx.x; i < 8 * 16 * 32; i += kPW * 32) {
+    for (int i = threadIdx.x; i < 8 * 16 * 32; i += kW * 32) {
         const int ln = i & 31, nt = (i >> 5) & 15, a = i >> 9;
         const int p = 8 * nt + (ln >> 2), j0 = 16 * a + 2 * (ln & 3);
         uint32_t regs[2];
@@ -1014,6 +1039,26 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_gw_kernel(DevCodec cd, const
         }
         sm.qfrag[a][nt][ln][0] = regs[0];
         sm.qfrag[a][nt][ln][1] = regs[1];
+    }
+    if constexpr (RECIPE) {
+        // S_g's B fragment (k-step kk, n-tile nt) of lane (rr, cc): B[k][n] = S_g[8 nt + rr][16 kk + k] for
+        // k = 2 cc + {0, 1} (reg 0) and 2 cc + 8 + {0, 1} (reg 1), split into bf16 hi + lo; the codec
+        // stores S_0^T then S_1^T, entry (j, i) = S_g[i][j].
+        for (int i = threadIdx.x; i < 2 * 4 * 8 * 32; i += kW * 32) {
+            const int ln = i & 31, nt = (i >> 5) & 7, kk = (i >> 8) & 3, g = i >> 10;
+            const float* st = cd.qjl_st + g * F::N0 * F::N0;
+            const int n = 8 * nt + (ln >> 2), j0 = 16 * kk + 2 * (ln & 3);
+            for (int q = 0; q < 2; ++q) {
+                uint32_t hi, lo;
+                split_bf16x2(st[(j0 + 8 * q) * 64 + n], st[(j0 + 8 * q + 1) * 64 + n], hi, lo);
+                sm.sfrag[g][0][kk][nt][ln][q] = hi;
+                sm.sfrag[g][1][kk][nt][ln][q] = lo;
+            }
+        }
+        for (int i = threadIdx.x; i < 2 * 16 * 32; i += kW * 32) {
+            const int g = i >> 9, k = (i >> 5) & 15;
+            sm.centv[g][k][i & 31] = kCellScale * cd.cent[g * kMaxLevels + k];
+        }
     }
     // Mask word k = 2 a + q of lane l covers its fragment channels 16 a + 8 q + 2 (l % 4) + {0, 1}.
     if (threadIdx.x < 128) {
@@ -1045,8 +1090,8 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_gw_kernel(DevCodec cd, const
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    const int stride = ctas * kPW;
-    int tg = cta * kPW + warp;
+    const int stride = ctas * kW;
+    int tg = cta * kW + warp;
     if (tg < tgroups) issue(tg, 0);
     for (int it = 0; tg < tgroups; tg += stride, ++it) {
         const int cur = it & 1;
@@ -1184,9 +1229,15 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_gw_kernel(DevCodec cd, const
             }
 
         // Q x in two halves of 8 n-tiles (outputs 64 HALF .. 64 HALF + 63), each over the 8 k-steps;
-        // then quantize and stage bytes (p, p + 1), p = 8 nt + 2 c, of tokens r and r + 8.
+        // then quantize and stage bytes (p, p + 1), p = 8 nt + 2 c, of tokens r and r + 8. Recipe rows:
+        // each half is one group, whose QJL stage follows its quantization.
+        uint32_t g16[2][2] = {{0u, 0u}, {0u, 0u}};  // recipe: [group][token] residual norms
         static_for<0, 2>([&](auto hc) {
             constexpr int HALF = decltype(hc)::value;
+            // recipe: the group's residuals r = u - c[idx] (v units) as the S_g product's A fragments,
+            // bf16 hi + lo: [k-step][2 (n-tile & 1) + token] for n-tiles 2 k-step + {0, 1} of the half
+            uint32_t rh[4][4], rl[4][4];
+            float rr[2] = {0.0f, 0.0f};
             float acc[8][4];
 #pragma unroll
             for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
@@ -1219,19 +1270,76 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_gw_kernel(DevCodec cd, const
                     const uint32_t at = stage + static_cast<uint32_t>((r + 8 * i) * kStagePitch + 8 * NT + 2 * c);
                     asm volatile("st.shared.u16 [%0], %1;" ::"r"(at), "h"(static_cast<unsigned short>(i0 | (i1 << 8)))
                                  : "memory");
+                    if constexpr (RECIPE) {
+                        const uint32_t cl =
+                            static_cast<uint32_t>(__cvta_generic_to_shared(&sm.centv[G][0][lane]));
+                        const float q0 = v0 - __uint_as_float(lds32(cl + i0 * 128u));
+                        const float q1 = v1 - __uint_as_float(lds32(cl + i1 * 128u));
+                        rr[i] = fmaf(q0, q0, fmaf(q1, q1, rr[i]));
+                        split_bf16x2(q0, q1, rh[n >> 1][2 * (n & 1) + i], rl[n >> 1][2 * (n & 1) + i]);
+                    }
                 }
             });
+            if constexpr (RECIPE) {
+                // Residual norms of the group, then S_g r_g (hi x hi + lo x hi + hi x lo), four n-tiles at
+                // a time; bit 2 c + e of sign byte nt is (S_g r_g)_i >= 0 for i = 8 nt + 2 c + e.
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    float q = rr[i];
+                    q += __shfl_xor_sync(kFull, q, 1);
+                    q += __shfl_xor_sync(kFull, q, 2);
+                    g16[HALF][i] = __half_as_ushort(__float2half_rn(sqrtf(q) * (1.0f / kCellScale)));
+                }
+                const uint32_t sf_lane =
+                    static_cast<uint32_t>(__cvta_generic_to_shared(&sm.sfrag[HALF][0][0][0][lane][0]));
+                constexpr uint32_t kLoOff = 4u * 8u * 32u * 8u;
+                constexpr int kSign = HALF ? FR::SIGN1 : FR::SIGN0;
+#pragma unroll
+                for (int n4 = 0; n4 < 2; ++n4) {
+                    float sacc[4][4];
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.0f;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                        for (int n = 0; n < 4; ++n) {
+                            const uint32_t off = static_cast<uint32_t>((kk * 8 + 4 * n4 + n) * 32 * 8);
+                            const uint2 bh = lds64(sf_lane + off), bl = lds64(sf_lane + kLoOff + off);
+                            mma_bf16_acc(sacc[n], rh[kk][0], rh[kk][1], rh[kk][2], rh[kk][3], bh.x, bh.y);
+                            mma_bf16_acc(sacc[n], rl[kk][0], rl[kk][1], rl[kk][2], rl[kk][3], bh.x, bh.y);
+                            mma_bf16_acc(sacc[n], rh[kk][0], rh[kk][1], rh[kk][2], rh[kk][3], bl.x, bl.y);
+                        }
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) {
+                        const uint32_t s0 = __ballot_sync(kFull, sacc[n][0] >= 0.0f);
+                        const uint32_t s1 = __ballot_sync(kFull, sacc[n][1] >= 0.0f);
+                        const uint32_t s2 = __ballot_sync(kFull, sacc[n][2] >= 0.0f);
+                        const uint32_t s3 = __ballot_sync(kFull, sacc[n][3] >= 0.0f);
+                        if (c == 0) {
+                            const int sh = 4 * r;
+                            sm.rows[warp][r][kSign + 4 * n4 + n] = static_cast<uint8_t>(
+                                spread4((s0 >> sh) & 0xFu) | (spread4((s1 >> sh) & 0xFu) << 1));
+                            sm.rows[warp][r + 8][kSign + 4 * n4 + n] = static_cast<uint8_t>(
+                                spread4((s2 >> sh) & 0xFu) | (spread4((s3 >> sh) & 0xFu) << 1));
+                        }
+                    }
+                }
+            }
         });
         if (c == 0) {
-            sm.norms[warp][r] = static_cast<uint32_t>(n16[0][0]) | (static_cast<uint32_t>(n16[1][0]) << 16);
-            sm.norms[warp][r + 8] = static_cast<uint32_t>(n16[0][1]) | (static_cast<uint32_t>(n16[1][1]) << 16);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const uint32_t n0 = n16[0][i], n1 = n16[1][i];
+                sm.norms[warp][r + 8 * i] = RECIPE ? make_uint2(n0 | (g16[0][i] << 16), n1 | (g16[1][i] << 16))
+                                                   : make_uint2(n0 | (n1 << 16), 0u);
+            }
         }
         __syncwarp();
-        assemble_rows<F>(stage, sm.rows[warp], lane);
+        assemble_rows<FR>(stage, sm.rows[warp], lane);
         __syncwarp();
 
-        // Write the rows in 8-byte pieces, and the two norms.
-        constexpr int ib = F::IB, rb = F::IB + 4;
+        // Write the rows in 8-byte pieces, and the norms (two, recipe four).
+        constexpr int ib = FR::IB, rb = FR::IB + (RECIPE ? 8 : 4);
         constexpr int pieces = ib / 8;
         for (int q = lane; q < 16 * pieces; q += 32) {
             const int row = q / pieces, part = q - row * pieces;
@@ -1242,7 +1350,12 @@ __global__ void __launch_bounds__(kPW * 32, 1) pack_gw_kernel(DevCodec cd, const
                 uint8_t* sub = pages + (static_cast<int64_t>(blk) * H + h) * block_size * rb;
                 *reinterpret_cast<uint2*>(sub + off * ib + 8 * part) =
                     *reinterpret_cast<const uint2*>(&sm.rows[warp][row][8 * part]);
-                if (part == 0) *reinterpret_cast<uint32_t*>(sub + block_size * ib + 4 * off) = sm.norms[warp][row];
+                if (part == 0) {
+                    if constexpr (RECIPE)
+                        *reinterpret_cast<uint2*>(sub + block_size * ib + 8 * off) = sm.norms[warp][row];
+                    else
+                        *reinterpret_cast<uint32_t*>(sub + block_size * ib + 4 * off) = sm.norms[warp][row].x;
+                }
             } else if (slot >= capacity && part == 0 && d_err) {
                 atomicOr(d_err, TQ_DERR_SLOT);
             }
@@ -1263,7 +1376,9 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
     // 4 bits on 64 channels and 3 on 64, or 4 bits on 32 and 2 on 96 (plain also uniform 3 and 4
     // bits); QJL formats (without group-wise rotation) of 3 bits on 64 channels and 2 on 64, 4 on 64
     // and 3 on 64, or uniform 3 or 2 bits.
-    enum Kind { kNone, kU4, kU3, kM43, kM42, kGw43, kGw42, kQ32, kQ43, kQu3, kQu2 };
+    // Recipe rows (group-wise rotation with each group's QJL stage) of 3 bits on 64 channels and 2 on
+    // 64, or 4 and 3.
+    enum Kind { kNone, kU4, kU3, kM43, kM42, kGw43, kGw42, kQ32, kQ43, kQu3, kQu2, kR32, kR43 };
     Kind kind[2];
     bool u4 = true;
     for (int side = 0; side < 2; ++side) {
@@ -1273,7 +1388,8 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
         const bool m42 = d.n_groups == 2 && d.group_bits[0] == 4 && d.group_size[0] == 32 && d.group_bits[1] == 2;
         const bool m32 = d.n_groups == 2 && d.group_bits[0] == 3 && d.group_size[0] == 64 && d.group_bits[1] == 2;
         Kind kd = kNone;
-        if (!(side ? vc : kc)->dev.cells || (d.qjl && d.groupwise)) kd = kNone;
+        if (!(side ? vc : kc)->dev.cells) kd = kNone;
+        else if (d.qjl && d.groupwise) kd = m32 ? kR32 : (m43 ? kR43 : kNone);
         else if (d.qjl)
             kd = m32 ? kQ32
                      : (m43 ? kQ43
@@ -1311,10 +1427,14 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sizeof(PackQjlSmem)));
-        for (auto kern : {pack_gw_kernel<PM43>, pack_gw_kernel<PM42>})
+        for (auto kern : {pack_gw_kernel<PM43, false>, pack_gw_kernel<PM42, false>})
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sizeof(PackGwSmem)));
+        for (auto kern : {pack_gw_kernel<PM32, true>, pack_gw_kernel<PM43, true>})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(PackRecipeSmem)));
         return e;
     });
     if (err != cudaSuccess) return fail(TQ_ERR_CUDA, "pack fast path setup failed");
@@ -1340,9 +1460,12 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
     constexpr int kQW = TcShape<true>::W;
     const int64_t wantq = (tgroups * H + kQW - 1) / kQW;
     const int gridq = static_cast<int>(wantq < sms ? wantq : sms);
-    const int64_t per_head_want = (tgroups + kPW - 1) / kPW;
+    constexpr int kRW = PackGwSmemBase<true>::W;
     const int64_t per_head_fit = sms / H > 0 ? sms / H : 1;
-    const int per_head = static_cast<int>(per_head_want < per_head_fit ? per_head_want : per_head_fit);
+    auto per_head = [&](int warps) {
+        const int64_t want = (tgroups + warps - 1) / warps;
+        return static_cast<int>(want < per_head_fit ? want : per_head_fit);
+    };
     const struct { const tq_codec* c; const void* x; void* pages; } sides[2] = {{kc, k, k_pages}, {vc, v, v_pages}};
     for (int side = 0; side < 2; ++side) {
         const auto& sd = sides[side];
@@ -1360,8 +1483,10 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
             case kQ43: go(pack_tc_kernel<PM43, true>, gridq, sizeof(PackQjlSmem), kQW); break;
             case kQu3: go(pack_tc_kernel<PU3, true>, gridq, sizeof(PackQjlSmem), kQW); break;
             case kQu2: go(pack_tc_kernel<PU2, true>, gridq, sizeof(PackQjlSmem), kQW); break;
-            case kGw43: go(pack_gw_kernel<PM43>, per_head * H, sizeof(PackGwSmem)); break;
-            case kGw42: go(pack_gw_kernel<PM42>, per_head * H, sizeof(PackGwSmem)); break;
+            case kGw43: go(pack_gw_kernel<PM43, false>, per_head(kPW) * H, sizeof(PackGwSmem)); break;
+            case kGw42: go(pack_gw_kernel<PM42, false>, per_head(kPW) * H, sizeof(PackGwSmem)); break;
+            case kR32: go(pack_gw_kernel<PM32, true>, per_head(kRW) * H, sizeof(PackRecipeSmem), kRW); break;
+            case kR43: go(pack_gw_kernel<PM43, true>, per_head(kRW) * H, sizeof(PackRecipeSmem), kRW); break;
             default: break;
         }
     }

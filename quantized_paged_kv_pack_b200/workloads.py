@@ -107,6 +107,12 @@ WORKLOADS = {
         description="pack 32 sequences x 8192 tokens, 8 KV heads, block 16, shuffled slot mapping, K and V "
                     "3.5-bit group-wise (the group-wise decode workload's formats); tensor-core group-wise "
                     "pack kernel"),
+    "pack_llama8b_3p5bit_recipe": Workload(
+        "pack_llama8b_3p5bit_recipe", "pack", 1013, 32, 32, 8, 128, 16, 0,
+        (3, 2), (64, 64), (4, 3), (64, 64), 81, 82, 8, True, "fixed:8192", k_qjl=True, groupwise=True,
+        description="pack 32 sequences x 8192 tokens, 8 KV heads, block 16, shuffled slot mapping, the recipe "
+                    "decode workload's formats (K recipe rows: two group-wise groups, each with its QJL "
+                    "signs and norms; V 3.5-bit group-wise); tensor-core recipe and group-wise packs"),
     "decode_llama8b_4bit": Workload(
         "decode_llama8b_4bit", "decode", 1003, 64, 32, 8, 128, 16, 64,
         (4,), (128,), (4,), (128,), 0, 1, 8, True, "uniform:1024:32768",
@@ -146,7 +152,7 @@ WORKLOADS = {
                     "K in the recipe row as printed: two group-wise groups (64 original channels, the "
                     "outliers among them, at 3 bits + 64 at 2), each with its QJL signs, norm and residual "
                     "norm (3.5 bits per channel); V 3.5-bit group-wise; 128-token bf16 window; runs on the "
-                    "general CUDA-core decode kernel"),
+                    "tensor-core decode kernel"),
 }
 
 

@@ -183,3 +183,38 @@ def check_qjl_rows(rows, x, fmt, heads):
             "QJL sign mismatch away from zero"
         compared += int(ok.sum())
     return compared
+
+
+RECIPE_SIGN_REL = 1e-4  # a sign may differ only where |(S_g r_g)_i| is this small against |r_g| sqrt(n_g)
+
+
+def check_recipe_rows(rows, x, fmt, heads):
+    """GPU rows [N][H][row] against the oracle's recipe quantization of x [N][H][d]."""
+    compared = 0
+    for h in heads:
+        f1 = slice_format(fmt, h)
+        idx, n16, u, signs, g16 = O.quantize_qjl(x[:, h], f1, 0)
+        gidx, gn16, gsigns, gg16 = O.decode_rows(rows[:, h], f1)
+        assert np.array_equal(gn16.astype(np.float16).view(np.uint16), n16.astype(np.float16).view(np.uint16))
+        flips = gidx != idx
+        if flips.any():
+            margin = O.boundary_margin(u, f1)
+            assert np.all(margin[flips] <= QJL_BOUNDARY_REL), "index mismatch away from a codebook boundary"
+        ok = ~np.any(flips, axis=-1)
+        gd = gg16[ok] != g16[ok]
+        if gd.any():
+            rel = np.abs(gg16[ok][gd] - g16[ok][gd]) / np.maximum(g16[ok][gd], 1e-30)
+            assert np.all(rel < 2e-3), "residual norm differs by more than one fp16 step"
+            assert gd.sum() <= max(2, 0.002 * gd.size)
+        start = 0
+        for g, (b, n) in enumerate(zip(f1.group_bits, f1.group_size)):
+            c, _ = O.codebook(b, n)
+            r = u[:, start:start + n] - c[idx[:, start:start + n]]
+            proj = r @ O.recipe_qjl_matrix(f1, g).T
+            scale = np.linalg.norm(r, axis=-1, keepdims=True) * math.sqrt(n)
+            diff = (gsigns[:, start:start + n] != signs[:, start:start + n]) & ok[:, None]
+            assert np.all(np.abs(proj[diff]) <= RECIPE_SIGN_REL * np.broadcast_to(scale, proj.shape)[diff]), \
+                "QJL sign mismatch away from zero"
+            start += n
+        compared += int(ok.sum())
+    return compared

@@ -11,7 +11,7 @@ from oracle import tq_oracle as O
 from quantized_paged_kv_pack_b200 import tq
 from quantized_paged_kv_pack_b200 import workloads as W
 
-from helpers import D, check_qjl_rows, codec_pair, random_kv, slice_format, workload_codecs
+from helpers import D, check_qjl_rows, check_recipe_rows, codec_pair, random_kv, slice_format, workload_codecs
 
 pytestmark = pytest.mark.gpu
 
@@ -231,13 +231,17 @@ def test_pack_edge_values_uniform_4bit_fast_path():
                                                   (((4, 3), (64, 64)), ((4, 2), (32, 96)), 16, "gw"),
                                                   (((4, 2), (32, 96)), ((4, 3), (64, 64)), 40, "gw"),
                                                   (((3, 2), (64, 64)), ((4, 3), (64, 64)), 16, "qjl"),
-                                                  (((3,), (128,)), ((2,), (128,)), 24, "qjl")])
+                                                  (((3,), (128,)), ((2,), (128,)), 24, "qjl"),
+                                                  (((3, 2), (64, 64)), ((4, 3), (64, 64)), 16, "recipe"),
+                                                  (((4, 3), (64, 64)), ((3, 2), (64, 64)), 32, "recipe")])
 def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs, mode):
     """The tensor-core packs (uniform 4-bit, the plain 2/3/4-bit mixes, the group-wise 4/3 and 4/2
-    formats, and QJL formats) against the general kernel and the oracle on the same tokens."""
+    formats, QJL formats and recipe rows) against the general kernel and the oracle on the same
+    tokens."""
     H, T = 4, 700
-    kc, kf = codec_pair(H, *kspec, 8, qjl=mode == "qjl", groupwise=mode == "gw")
-    vc, vf = codec_pair(H, *vspec, 9, qjl=mode == "qjl", groupwise=mode == "gw")
+    qjl, gw = mode in ("qjl", "recipe"), mode in ("gw", "recipe")
+    kc, kf = codec_pair(H, *kspec, 8, qjl=qjl, groupwise=gw)
+    vc, vf = codec_pair(H, *vspec, 9, qjl=qjl, groupwise=gw)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(5)
     k, v = random_kv(T, H, gen)
@@ -257,6 +261,8 @@ def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs, mode
         for pages in (out[0][i], out[1][i]):
             if mode == "qjl":
                 assert check_qjl_rows(rows_of(pages, s, bs, f, H), x, f, range(H)) > 0.99 * T * H
+            elif mode == "recipe":
+                assert check_recipe_rows(rows_of(pages, s, bs, f, H), x, f, range(H)) > 0.99 * T * H
             else:
                 compare_rows(rows_of(pages, s, bs, f, H), x, f, range(H))
         same = (out[0][i] == out[1][i]).mean()
@@ -266,14 +272,16 @@ def test_fast_and_general_pack_kernels_agree(monkeypatch, kspec, vspec, bs, mode
 @pytest.mark.parametrize("kspec,vspec,mode", [(((4,), (128,)), ((4,), (128,)), ""),
                                               (((4, 3), (64, 64)), ((4, 2), (32, 96)), ""),
                                               (((4, 3), (64, 64)), ((4, 2), (32, 96)), "gw"),
-                                              (((3, 2), (64, 64)), ((3,), (128,)), "qjl")])
+                                              (((3, 2), (64, 64)), ((3,), (128,)), "qjl"),
+                                              (((3, 2), (64, 64)), ((4, 3), (64, 64)), "recipe")])
 def test_pack_tokens_not_finite(monkeypatch, kspec, vspec, mode):
     """Tokens holding inf, NaN or values near the bf16 limit (norms far beyond fp16) pack without
     an error flag in the tensor-core kernels and the general one, and leave the rows of the other
     tokens as the oracle has them."""
     H, T, bs = 4, 200, 16
-    kc, kf = codec_pair(H, *kspec, 13, qjl=mode == "qjl", groupwise=mode == "gw")
-    vc, vf = codec_pair(H, *vspec, 14, qjl=mode == "qjl", groupwise=mode == "gw")
+    qjl, gw = mode in ("qjl", "recipe"), mode in ("gw", "recipe")
+    kc, kf = codec_pair(H, *kspec, 13, qjl=qjl, groupwise=gw)
+    vc, vf = codec_pair(H, *vspec, 14, qjl=qjl, groupwise=gw)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(77)
     k, v = random_kv(T, H, gen)
@@ -302,6 +310,8 @@ def test_pack_tokens_not_finite(monkeypatch, kspec, vspec, mode):
             rows = rows_of(pages.cpu().numpy(), s, bs, f, H)
             if mode == "qjl":
                 assert check_qjl_rows(rows, x, f, range(H)) > 0.99 * len(good) * H
+            elif mode == "recipe":
+                assert check_recipe_rows(rows, x, f, range(H)) > 0.99 * len(good) * H
             else:
                 flips, total = compare_rows(rows, x, f, range(H))
                 assert flips <= max(1, MAX_FLIP_FRACTION * total)

@@ -10,47 +10,13 @@ import torch
 from oracle import tq_oracle as O
 from quantized_paged_kv_pack_b200 import tq
 
-from helpers import D, DecodeProblem, codec_pair, random_kv, slice_format
+from helpers import D, DecodeProblem, check_recipe_rows, codec_pair, random_kv, slice_format
 
 pytestmark = pytest.mark.gpu
 
-BOUNDARY_REL = 1e-5
-SIGN_REL = 1e-4  # a sign may differ only where |(S_g r_g)_i| is this small against |r_g| sqrt(n_g)
 
 
-def check_recipe_rows(rows, x, fmt, heads):
-    """GPU rows [N][H][row] against the oracle's recipe quantization of x [N][H][d]."""
-    compared = 0
-    for h in heads:
-        f1 = slice_format(fmt, h)
-        idx, n16, u, signs, g16 = O.quantize_qjl(x[:, h], f1, 0)
-        gidx, gn16, gsigns, gg16 = O.decode_rows(rows[:, h], f1)
-        assert np.array_equal(gn16.astype(np.float16).view(np.uint16), n16.astype(np.float16).view(np.uint16))
-        flips = gidx != idx
-        if flips.any():
-            margin = O.boundary_margin(u, f1)
-            assert np.all(margin[flips] <= BOUNDARY_REL), "index mismatch away from a codebook boundary"
-        ok = ~np.any(flips, axis=-1)
-        gd = gg16[ok] != g16[ok]
-        if gd.any():
-            rel = np.abs(gg16[ok][gd] - g16[ok][gd]) / np.maximum(g16[ok][gd], 1e-30)
-            assert np.all(rel < 2e-3), "residual norm differs by more than one fp16 step"
-            assert gd.sum() <= max(2, 0.002 * gd.size)
-        start = 0
-        for g, (b, n) in enumerate(zip(f1.group_bits, f1.group_size)):
-            c, _ = O.codebook(b, n)
-            r = u[:, start:start + n] - c[idx[:, start:start + n]]
-            proj = r @ O.recipe_qjl_matrix(f1, g).T
-            scale = np.linalg.norm(r, axis=-1, keepdims=True) * math.sqrt(n)
-            diff = (gsigns[:, start:start + n] != signs[:, start:start + n]) & ok[:, None]
-            assert np.all(np.abs(proj[diff]) <= SIGN_REL * np.broadcast_to(scale, proj.shape)[diff]), \
-                "QJL sign mismatch away from zero"
-            start += n
-        compared += int(ok.sum())
-    return compared
-
-
-@pytest.mark.parametrize("kfmt", [((4, 3), (64, 64)), ((4, 2), (32, 96)), ((3, 2), (16, 112))])
+@pytest.mark.parametrize("kfmt", [((4, 3), (64, 64)), ((3, 2), (64, 64)), ((4, 2), (32, 96)), ((3, 2), (16, 112))])
 @pytest.mark.parametrize("T,H,bs", [(37, 2, 16), (300, 8, 32)])
 def test_recipe_pack_matches_oracle(kfmt, T, H, bs):
     kc, kf = codec_pair(H, *kfmt, 51, qjl=True, groupwise=True)
@@ -123,9 +89,10 @@ def test_recipe_decode_tensor_core_matches_oracle_and_general(monkeypatch, H, G,
     assert worst <= 2e-3, worst
 
 
-def test_recipe_window_append_rows_equal_pack():
-    """tq_window_append packs an evicted token through the same routine: the row it writes for the
-    recipe format equals the row tq_pack_kv writes for that token."""
+def test_recipe_window_append_rows_equal_pack(monkeypatch):
+    """tq_window_append packs an evicted token through the general kernel's per-vector routine: the
+    row it writes for the recipe format equals the row that kernel writes for that token."""
+    monkeypatch.setenv("TQ_PACK_KERNEL", "general")
     H, bs, W = 2, 16, 4
     kc, kf = codec_pair(H, (4, 3), (64, 64), 71, qjl=True, groupwise=True)
     vc, vf = codec_pair(H, (4, 3), (64, 64), 72, groupwise=True)
