@@ -104,8 +104,7 @@ typedef enum {
  *                signs][group-1 indices][group-1 signs] and its norm area holds
  *                (n_0, |r_0|, n_1, |r_1|), 8 bytes. The key is, per group,
  *                n_g B_g^T (c_g + sqrt(pi/2)/group_size[g] |r_g| S_g^T z_g) on
- *                the group's channels. Decode accepts it for K only, on the
- *                general kernel.
+ *                the group's channels. Decode accepts it for K only.
  */
 typedef struct {
     int32_t head_dim;
@@ -182,7 +181,8 @@ tq_status tq_make_codec(const tq_format_desc* desc, tq_codec** out);
 void tq_free_codec(tq_codec* codec);
 
 /* Bytes of one packed row of this codec: index bytes of every group, the QJL
- * sign bytes of a QJL codec, and 2 norm bytes (4 for QJL and group-wise). */
+ * sign bytes of a QJL codec, and 2 norm bytes (4 for QJL and group-wise, 8 for
+ * the recipe row). */
 int32_t tq_codec_row_bytes(const tq_codec* codec);
 
 /*
@@ -203,7 +203,9 @@ int32_t tq_codec_row_bytes(const tq_codec* codec);
  * bytes of the block_size rows come first, row after row (offset * index
  * bytes), then the block_size norms (block_size * index bytes + 2 * offset),
  * so index rows stay 8-byte aligned. Each row is written whole; bytes of
- * other rows are untouched.
+ * other rows are untouched. A vector with an inf or NaN element, or a norm of
+ * 3e37 or more, gets its norm as computed (inf or NaN in fp16) and indices
+ * without meaning; no error flag is set for it.
  * Errors: TQ_ERR_VALUE for inconsistent arguments (num_kv_heads or head_dim
  * differing between the codecs, block_size < 1, null pointers with
  * num_tokens > 0). A slot >= num_blocks * block_size sets TQ_DERR_SLOT in
