@@ -305,8 +305,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partials_kernel(DecodeArgs
 // (win), all relative to the largest record max. The records are read in
 // parallel: first every max (thread j takes splits j, j + 128, ...), then per
 // chunk of 128 splits each thread's weight goes to shared memory and the
-// accumulator sums its column with eight loads in flight. fw: the group's 128
-// floats of shared scratch, red: its 4.
+// accumulator sums its column with WIDE loads in flight (WIDE = 16: unrolled
+// rounds with the loads past the last split skipped; 8: a loop unrolled by 8,
+// fewer registers, which the one-head-per-CTA combine's larger grids need).
+// fw: the group's 128 floats of shared scratch, red: its 4.
+template <int WIDE>
 __device__ __forceinline__ void merge_splits(const float* unit, int G, int g, int ns, int n_win, int max_splits,
                                              int j, float* fw, float* red, float& ls, float& rot, float& win) {
     auto rec = [&](int i) { return unit + (static_cast<int64_t>(i) * G + g) * (kHeadDim + 2); };
@@ -335,8 +338,20 @@ __device__ __forceinline__ void merge_splits(const float* unit, int G, int g, in
         fw[j] = f;
         __syncthreads();
         const int n = min(kHeadDim, ns - c0);
+        if constexpr (WIDE == 16) {
+            // past the last split the load is skipped and its weight is 0, so the sum keeps the split
+            // order and adds exact zeros
+            for (int k = 0; k < n; k += 16) {
+                float vals[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) vals[u] = k + u < n ? rec(c0 + k + u)[2 + j] : 0.0f;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) rot = fmaf(vals[u], fw[k + u], rot);
+            }
+        } else {
 #pragma unroll 8
-        for (int k = 0; k < n; ++k) rot = fmaf(rec(c0 + k)[2 + j], fw[k], rot);
+            for (int k = 0; k < n; ++k) rot = fmaf(rec(c0 + k)[2 + j], fw[k], rot);
+        }
         __syncthreads();  // fw is written again by the next chunk
     }
     lpart = warp_sum(lpart);
@@ -368,7 +383,7 @@ __global__ void __launch_bounds__(kHeadDim) decode_combine_kernel(DevCodec vc, c
     const int ns = (P + split_tokens - 1) / split_tokens;
     const float* unit = ws + (static_cast<int64_t>(b) * H + h) * items_per_unit * static_cast<int64_t>(G) * (kHeadDim + 2);
     float Ls, rot, win;
-    merge_splits(unit, G, g, ns, n_win, max_splits, j, y, red, Ls, rot, win);
+    merge_splits<8>(unit, G, g, ns, n_win, max_splits, j, y, red, Ls, rot, win);
     __syncthreads();  // y served as the merge's scratch
     float x;
     if (vc.groupwise) {
@@ -449,7 +464,7 @@ __global__ void __launch_bounds__(kHeadDim * kGwHeads) decode_combine_gw_kernel(
         // 16, so no group runs past G; were one to, it would repeat head G - 1 and write nothing.
         const int g = g0 + gl;
         float Ls, rot, win;
-        merge_splits(unit, G, g < G ? g : G - 1, ns, n_win, max_splits, j, ys + gl * kHeadDim, reds + gl * 4, Ls,
+        merge_splits<16>(unit, G, g < G ? g : G - 1, ns, n_win, max_splits, j, ys + gl * kHeadDim, reds + gl * 4, Ls,
                      rot, win);
         __syncthreads();  // ys served as the merge's scratch
         ys[gl * kHeadDim + j] = rot;  // packed positions
