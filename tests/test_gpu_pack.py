@@ -350,3 +350,37 @@ def test_pack_workload_whole_sequence_and_mse_full_size():
             mse_ref += ((O.dequantize_rows(ri, rn, f1, 0) - x[:, h]) ** 2).sum()
         assert abs(mse_gpu / mse_ref - 1) <= 0.02
     assert flips <= MAX_FLIP_FRACTION * total
+
+
+@pytest.mark.parametrize("name", ["pack_llama70b_3p5bit", "pack_llama8b_2p5bit", "pack_llama8b_3p5bit_qjl",
+                                  "pack_llama8b_3p5bit_groupwise", "pack_llama8b_3p5bit_recipe"])
+def test_pack_workloads_full_size_one_sequence(name):
+    """Each mixed-format pack workload in the benchmark's launch (32 x 8192 tokens, one call): every row
+    of one whole 8192-token sequence (all 8 KV heads, K and V) against the oracle, with its checks for
+    the format (index flips only at a boundary, norms bit-exact; QJL signs only where the projection is
+    negligible)."""
+    w = W.WORKLOADS[name]
+    kc, vc, kf, vf = workload_codecs(w)
+    k, v, slots, layout = W.pack_batch(w, device="cuda")
+    kp, vp = tq.page_pool(kc, layout.num_blocks, w.block_size), tq.page_pool(vc, layout.num_blocks, w.block_size)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.pack_kv(kc, vc, k, v, torch.as_tensor(slots, device="cuda"), kp, vp, w.block_size, d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    seq_len = int(layout.seq_lens[0])
+    b = 21  # a sequence late in the batch
+    pick = np.arange(b * seq_len, (b + 1) * seq_len)
+    s = slots[pick]
+    H = w.num_kv_heads
+    for pages, src, f in ((kp, k, kf), (vp, v, vf)):
+        sub = pages[torch.as_tensor(s // w.block_size, device="cuda")].cpu().numpy()
+        rows = np.stack([O.read_rows(sub, np.arange(len(s)), h, s % w.block_size, f, w.block_size)
+                         for h in range(H)], axis=1)
+        x = src[torch.as_tensor(pick, device="cuda")].float().cpu().numpy().astype(np.float64)
+        if f.qjl and f.groupwise:
+            assert check_recipe_rows(rows, x, f, range(H)) > 0.99 * len(s) * H
+        elif f.qjl:
+            assert check_qjl_rows(rows, x, f, range(H)) > 0.99 * len(s) * H
+        else:
+            flips, total = compare_rows(rows, x, f, range(H))
+            assert flips <= MAX_FLIP_FRACTION * total
