@@ -1293,33 +1293,43 @@ __device__ __forceinline__ void window_state(const DecodeArgs& a, const Item& it
     const __nv_bfloat16* vw = static_cast<const __nv_bfloat16*>(a.v_win);
     const int64_t row0 = (static_cast<int64_t>(it.b) * H + h) * a.window;
     const bool b4 = lane & 16, b3 = lane & 8;
-    // Four tokens at a time: their loads are issued together, and the four
-    // partial dot products of a head are summed over the warp by a transposed
-    // butterfly (the first two steps halve the values a lane carries; lane 8u
-    // ends with token u), then broadcast: 10 shuffles for 4 tokens instead of 20.
+    // Four tokens at a time: their loads are issued together (and those of the next
+    // four before this four is computed), and the four partial dot products of a
+    // head are summed over the warp by a transposed butterfly (the first two steps
+    // halve the values a lane carries; lane 8u ends with token u), then broadcast:
+    // 10 shuffles for 4 tokens instead of 20.
+    uint2 kr[4], vr[4];
+    auto load4 = [&](int t0_) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int tk = t0_ + u * t_step;
+            kr[u] = make_uint2(0u, 0u);
+            vr[u] = make_uint2(0u, 0u);
+            if (tk < it.t1) {
+                const int64_t base = (row0 + tk) * kHeadDim + 4 * lane;
+                const bool fresh = tk == t_new;
+                kr[u] = *reinterpret_cast<const uint2*>(fresh ? kn + 4 * lane : kw + base);
+                vr[u] = *reinterpret_cast<const uint2*>(fresh ? vn + 4 * lane : vw + base);
+            }
+        }
+    };
+    load4(t_first);
     for (int t0 = t_first; t0 < it.t1; t0 += 4 * t_step) {
         float kx[4][4], vx[4][4];
         bool ok[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int tk = t0 + u * t_step;
-            ok[u] = tk < it.t1;
-            uint2 kr = make_uint2(0u, 0u), vr = make_uint2(0u, 0u);
-            if (ok[u]) {
-                const int64_t base = (row0 + tk) * kHeadDim + 4 * lane;
-                const bool fresh = tk == t_new;
-                kr = *reinterpret_cast<const uint2*>(fresh ? kn + 4 * lane : kw + base);
-                vr = *reinterpret_cast<const uint2*>(fresh ? vn + 4 * lane : vw + base);
-            }
-            kx[u][0] = __uint_as_float(kr.x << 16);
-            kx[u][1] = __uint_as_float(kr.x & 0xffff0000u);
-            kx[u][2] = __uint_as_float(kr.y << 16);
-            kx[u][3] = __uint_as_float(kr.y & 0xffff0000u);
-            vx[u][0] = __uint_as_float(vr.x << 16);
-            vx[u][1] = __uint_as_float(vr.x & 0xffff0000u);
-            vx[u][2] = __uint_as_float(vr.y << 16);
-            vx[u][3] = __uint_as_float(vr.y & 0xffff0000u);
+            ok[u] = t0 + u * t_step < it.t1;
+            kx[u][0] = __uint_as_float(kr[u].x << 16);
+            kx[u][1] = __uint_as_float(kr[u].x & 0xffff0000u);
+            kx[u][2] = __uint_as_float(kr[u].y << 16);
+            kx[u][3] = __uint_as_float(kr[u].y & 0xffff0000u);
+            vx[u][0] = __uint_as_float(vr[u].x << 16);
+            vx[u][1] = __uint_as_float(vr[u].x & 0xffff0000u);
+            vx[u][2] = __uint_as_float(vr[u].y << 16);
+            vx[u][3] = __uint_as_float(vr[u].y & 0xffff0000u);
         }
+        load4(t0 + 4 * t_step);
 #pragma unroll
         for (int g = 0; g < NH; ++g) {
             if (g < rows) {
