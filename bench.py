@@ -355,6 +355,36 @@ def time_steps(fns, steps, stream):
     return sum(per_step), parts, per_step
 
 
+def capture_step(step, outputs):
+    """The step as a CUDA graph, so that a replay is one launch and a stall of the host thread
+    between the step's own launches cannot leave the GPU idle inside a timed step. The graph is
+    kept only if a replay, from zeroed outputs, gives the eager step's outputs bit for bit; else
+    (or if capture fails) the step runs eagerly. Returns (callable, how)."""
+    torch.cuda.synchronize()
+    step()
+    torch.cuda.synchronize()
+    ref = [o.clone() for o in outputs]
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+    except Exception as e:  # the library's launches could not be captured: time the eager step
+        torch.cuda.synchronize()
+        try:
+            step()  # clears a launch error a failed capture may have left for the next call
+        except Exception:
+            pass
+        torch.cuda.synchronize()
+        return step, f"eager (capture failed: {type(e).__name__})"
+    for o in outputs:
+        o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    if not all(torch.equal(o, r) for o, r in zip(outputs, ref)):
+        return step, "eager (graph replay differed)"
+    return g.replay, "cuda_graph"
+
+
 def percentiles(xs):
     q = np.percentile(np.asarray(xs, dtype=np.float64), [10, 50, 90])
     return {"p10": float(q[0]), "p50": float(q[1]), "p90": float(q[2])}
@@ -376,17 +406,20 @@ def measure_decode(setup: DecodeSetup, steps, warmup, dist_ctx=None, clocks=True
     torch.cuda.synchronize()
     if setup.err.item():
         raise RuntimeError(f"device error word {setup.err.item()} during warm-up")
+    timed, how = capture_step(step, [setup.out])
     barrier(dist_ctx)
     sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
     if sampler:
         sampler.__enter__()
-    total_ms, _, per_step = time_steps([step], steps, stream)
+    total_ms, _, per_step = time_steps([timed], steps, stream)
     if sampler:
         sampler.__exit__(None, None, None)
+    if setup.err.item():
+        raise RuntimeError(f"device error word {setup.err.item()} in the timed steps")
     _, parts, _ = time_steps(phases, steps, stream)
     barrier(dist_ctx)
     total_ms = max_over_ranks(total_ms, dist_ctx)
-    return total_ms / steps, parts, (sampler.summary() if sampler else None), per_step
+    return total_ms / steps, parts, (sampler.summary() if sampler else None), per_step, how
 
 
 def measure_latency(setup: DecodeSetup, reps, warmup, cold):
@@ -445,17 +478,20 @@ def measure_decode_e2e(setup: DecodeSetup, steps, warmup):
 
 
 def measure_pack(setup: PackSetup, steps, warmup, clocks=False):
+    """Returns (ms per step, clock summary or None, how the step was launched)."""
     for _ in range(warmup):
         setup.step()
     torch.cuda.synchronize()
+    timed, how = capture_step(setup.step, [setup.kp, setup.vp])
     sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
     if sampler:
         sampler.__enter__()
-    total, _, _ = time_steps([setup.step], steps, torch.cuda.current_stream())
+    total, _, _ = time_steps([timed], steps, torch.cuda.current_stream())
     if sampler:
         sampler.__exit__(None, None, None)
-        return total / steps, sampler.summary()
-    return total / steps
+    if setup.err.item():
+        raise RuntimeError(f"device error word {setup.err.item()} in the timed steps")
+    return total / steps, (sampler.summary() if sampler else None), how
 
 
 # --------------------------------------------------------------------------- distributed plumbing
@@ -679,7 +715,7 @@ def workload_of(args):
 def run_pack(args, w, dist_ctx, rank, world):
     """Headline on the pack workload: one step = tq_pack_kv over the whole batch."""
     setup = PackSetup(w)
-    ms, clocks = measure_pack(setup, args.steps, args.warmup, clocks=True)
+    ms, clocks, how = measure_pack(setup, args.steps, args.warmup, clocks=True)
     ms = max_over_ranks(ms, dist_ctx)
     peak, peak_kind = peaks()
     nbytes = setup.bytes()
@@ -702,7 +738,8 @@ def run_pack(args, w, dist_ctx, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
             "config": {"workload": w.name, "description": w.description, "batch": w.batch,
-                       "l2": f"no flush: {nbytes / 1e9:.2f} GB moved per step, L2 is 126 MB"},
+                       "l2": f"no flush: {nbytes / 1e9:.2f} GB moved per step, L2 is 126 MB",
+                       "step_launch": how},
             "tokens_per_s": world * setup.k.shape[0] / (ms * 1e-3),
             "roofline": {"bound": "hbm", "kernel": "pack", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / peak,
@@ -730,7 +767,7 @@ def run_ours(args):
             dist_ctx.destroy_process_group()
         return rc
     setup = DecodeSetup(w, seed_offset=rank)
-    step_ms, parts, clocks, per_step = measure_decode(setup, args.steps, args.warmup, dist_ctx)
+    step_ms, parts, clocks, per_step, how = measure_decode(setup, args.steps, args.warmup, dist_ctx)
     e2e_ms, h2d, d2h = measure_decode_e2e(setup, max(3, args.steps // 2), args.warmup)
     e2e_ms = max_over_ranks(e2e_ms, dist_ctx)
     peak, peak_kind = peaks()
@@ -748,7 +785,8 @@ def run_ours(args):
                    "k_format": {"bits": list(w.k_bits), "sizes": list(w.k_sizes)},
                    "v_format": {"bits": list(w.v_bits), "sizes": list(w.v_sizes)},
                    "parallelism": f"{world} independent replicas (no collective)",
-                   "l2": f"no flush: {split_bytes / 1e9:.2f} GB of pages read per step, L2 is 126 MB"},
+                   "l2": f"no flush: {split_bytes / 1e9:.2f} GB of pages read per step, L2 is 126 MB",
+                   "step_launch": how},
         "kv_tokens_per_s": world * setup.kv_tokens() / (step_ms * 1e-3),
         "step_ms_percentiles": percentiles(per_step),
         "step_breakdown_ms": {"window_append": parts[0], "decode_partials": parts[1], "decode_combine": parts[2]},
@@ -786,7 +824,7 @@ def run_ours(args):
                 torch.cuda.empty_cache()
                 setup = DecodeSetup(ew)
                 n_steps = max(5, args.steps // 2)
-                ms, p, _, _ = measure_decode(setup, n_steps, args.warmup, None, clocks=False)
+                ms, p, _, _, how_x = measure_decode(setup, n_steps, args.warmup, None, clocks=False)
                 line["gpu_launches"] += DECODE_LAUNCHES * n_steps
                 sb = setup.decode_split_bytes()
                 extra[name] = {"GB/s": setup.step_bytes() / (ms * 1e-3) / 1e9,
@@ -795,7 +833,7 @@ def run_ours(args):
                                                      "decode_combine": p[2]},
                                "decode_partials_GB/s": sb / (p[1] * 1e-3) / 1e9,
                                "decode_partials_frac": sb / (p[1] * 1e-3) / 1e9 / peak,
-                               "traffic": stored_traffic(name, "tq_decode_mma.cu")}
+                               "traffic": stored_traffic(name, "tq_decode_mma.cu"), "step_launch": how_x}
                 if not args.no_cpu_baseline:
                     extra[name]["cpu_oracle"] = guarded(lambda: oracle_decode_sample(
                         ew, setup.kspec, setup.vspec, setup.layout, lambda b, h: gpu_pages_unit(setup, b, h),
@@ -804,10 +842,11 @@ def run_ours(args):
                 del setup
                 torch.cuda.empty_cache()
                 setup = PackSetup(ew)
-                ms = measure_pack(setup, max(5, args.steps // 2), args.warmup)
+                ms, _, how_x = measure_pack(setup, max(5, args.steps // 2), args.warmup)
                 gbs = setup.bytes() / (ms * 1e-3) / 1e9
                 extra[name] = {"GB/s": gbs, "tokens_per_s": setup.k.shape[0] / (ms * 1e-3), "ms_per_step": ms,
-                               "frac": gbs / peak, "traffic": stored_traffic(name, "tq_pack_mma.cu")}
+                               "frac": gbs / peak, "traffic": stored_traffic(name, "tq_pack_mma.cu"),
+                               "step_launch": how_x}
                 if not args.no_cpu_baseline:
                     ks, vs = WL.codec_specs(ew)
                     extra[name]["cpu_oracle"] = guarded(lambda: oracle_pack_sample(ew, ks, vs, args.cpu_budget / 4))

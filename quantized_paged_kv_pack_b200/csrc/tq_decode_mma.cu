@@ -2174,10 +2174,13 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_tot, int& t
 
 // Work list of the tensor-core kernels: the (sequence, split) pairs of every
 // non-empty packed work item, longest first: every full split (sequence by
-// sequence), then the partial last splits by decreasing tile count (a
-// counting sort whose bucket offsets come from one scan over the CTA); and
-// their number. Dealt in snake order (item_of), this balances the persistent
-// CTAs about as well as greedy longest-first assignment.
+// sequence), then the partial last splits by decreasing tile count, in
+// sequence order within a tile count (a counting sort whose bucket offsets
+// come from one scan over the CTA); and their number. Dealt in snake order
+// (item_of), this balances the persistent CTAs about as well as greedy
+// longest-first assignment. The order is a function of the lengths alone, so
+// an item always runs on the same CTA after the same items: results are the
+// same bit for bit from call to call.
 __device__ __forceinline__ void build_work_list(const DecodeArgs& a, ProSmem& sm) {
     auto& s = sm.wl;
     const int tid = threadIdx.x;
@@ -2220,10 +2223,25 @@ __device__ __forceinline__ void build_work_list(const DecodeArgs& a, ProSmem& sm
         int n_full;
         const int of = block_exclusive_scan(nf, s.warp_tot, n_full);
         for (int j = 0; j < nf; ++j) list[s.base_full + of + j] = make_int2(b, j);
-        if (pt) list[atomicAdd(&s.cursor[pt], 1)] = make_int2(b, nf);
         __syncthreads();
         if (tid == 0) s.base_full += n_full;
         __syncthreads();
+    }
+    // Partial splits: one warp, 32 sequences at a time; lanes with the same tile count take
+    // consecutive places in lane order after that bucket's cursor.
+    if (tid < 32) {
+        for (int b0 = 0; b0 < a.batch; b0 += 32) {
+            const int b = b0 + tid;
+            int nf = 0, pt = 0;
+            if (b < a.batch) geometry(b, nf, pt);
+            const unsigned peers = __match_any_sync(kFull, pt);
+            const int rank = __popc(peers & ((1u << tid) - 1u));
+            const int base = pt ? s.cursor[pt] : 0;
+            __syncwarp();
+            if (pt && rank == 0) s.cursor[pt] = base + __popc(peers);
+            __syncwarp();
+            if (pt) list[base + rank] = make_int2(b, nf);
+        }
     }
 }
 

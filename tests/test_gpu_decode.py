@@ -327,3 +327,14 @@ def test_decode_many_sequences_work_list(monkeypatch, H):
             continue
         hq = int(rng.integers(prob.Hq))
         assert np.abs(got[b, hq] - prob.oracle(b, hq)).max() <= ATOL
+
+
+def test_decode_is_reproducible_bit_for_bit_on_ragged_lengths():
+    """Ragged lengths put several partial splits of one tile count in the work list; their order is a
+    function of the lengths alone, so repeated calls give the same output bit for bit."""
+    lens = [int(x) for x in np.random.default_rng(12).integers(1, 6000, size=48)]
+    prob = DecodeProblem(lens, 8, 4, ((4,), (128,), 3), ((4, 3), (64, 64), 4), window=16, block_size=16, seed=9)
+    outs = [prob.run().clone() for _ in range(4)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
