@@ -123,3 +123,21 @@ def test_oracle_pack_sample_and_guard():
     assert ok == {"GB/s": 1.0, "token_heads_per_s": 2.0, "cores": 3, "kind": "oracle", "sample": "d"}
     bad = bench.guarded(lambda: 1 / 0)
     assert bad["error"].startswith("ZeroDivisionError")
+
+
+def test_pack_launch_count_follows_the_dispatch():
+    """The benchmark's claim of kernels per tq_pack_kv call: one for uniform 4-bit K and V (one grid for
+    both), two (one per side) when both sides have a tensor-core pack, one general launch otherwise."""
+    expect = {"pack_llama8b_4bit": 1, "pack_llama70b_3p5bit": 2, "pack_llama8b_2p5bit": 2,
+              "pack_llama8b_3p5bit_qjl": 2, "pack_llama8b_3p5bit_groupwise": 2, "pack_llama8b_3p5bit_recipe": 2}
+    assert {n for n, w in WL.WORKLOADS.items() if w.kind == "pack"} == set(expect)
+    for name, n in expect.items():
+        setup = object.__new__(bench.PackSetup)
+        setup.w = WL.WORKLOADS[name]
+        assert setup.launches() == n, name
+    # a block size that is not a multiple of 8, or a format without a tensor-core pack: the general kernel
+    w = WL.WORKLOADS["pack_llama70b_3p5bit"]
+    for changed in ({"block_size": 12}, {"k_bits": (3, 2), "k_sizes": (16, 112)}):
+        setup = object.__new__(bench.PackSetup)
+        setup.w = WL.Workload(**{**w.__dict__, **changed})
+        assert setup.launches() == 1, changed
