@@ -1,11 +1,13 @@
 """Benchmark of the compressed paged KV cache on B200: one JSON line on rank 0.
 
 A step is one serving decode step of the whole hot path over the workload's
-batch: tq_pack_kv writes the step's new K/V vector per (sequence, KV head)
-into its page slot (the token that leaves the dense window), then
-tq_decode_paged attends every query head over the packed history plus the
-bf16 window. Inputs are resident in HBM before timing; the page pools are far
-larger than L2, so no flush is needed between steps.
+batch, one tq_window_append_decode call: the window append packs the token
+that leaves each (sequence, KV head)'s dense window into its page slot, then
+the decode attends every query head over the packed history plus the bf16
+window. Inputs are resident in HBM before timing; the page pools are far
+larger than L2, so no flush is needed between steps. Each timed step replays
+a CUDA graph of the call when the replay reproduces the eager call's output
+bit for bit (else the eager call runs); `config.step_launch` says which.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -237,7 +239,7 @@ class PackSetup:
 class ClockSampler:
     """SM clocks and throttle reasons sampled while the timed region runs.
 
-    NVML (read-only queries) from a thread every 5 ms, so that a timed region of
+    NVML (read-only queries) from a thread every 2 ms, so that a timed region of
     tens of milliseconds still gets several samples; nvidia-smi (-lms 100) when
     NVML is not importable. Nothing here changes a GPU setting.
     """
