@@ -309,6 +309,8 @@ size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num
  * workspace      device buffer of at least tq_decode_workspace_bytes(...)
  *                bytes, 256-byte aligned, owned by the caller; it holds the
  *                split-K partials and is fully rewritten by each call.
+ * Repeated calls on the same inputs give the same output bit for bit: the
+ * split-K work order and every summation order depend on the lengths alone.
  * Errors: TQ_ERR_VALUE for inconsistent sizes or a short workspace,
  * TQ_ERR_UNSUPPORTED for a format the kernels lack. A block id outside
  * [0, num_blocks) sets TQ_DERR_BLOCK (block 0 is read instead, no fault);
