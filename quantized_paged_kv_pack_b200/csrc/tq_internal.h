@@ -204,9 +204,10 @@ struct SplitPlan {
 bool make_split_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_seq_len,
                      int32_t block_size, int32_t sms, SplitPlan* plan);
 
-// Uniform 4-bit pack on the tensor cores; TQ_ERR_UNSUPPORTED (nothing
-// launched) for other formats or unaligned pools.
-tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
+// The tensor-core packs (uniform 4-bit, plain, QJL, group-wise and recipe
+// formats that have an instantiation); TQ_ERR_UNSUPPORTED (nothing launched)
+// when either codec has none, or for buffers not 16-byte aligned.
+tq_status launch_pack_tc(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
                          const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
                          int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream);
 // Launch-error check (and TQ_CHECKED synchronisation) after a pack launch.

@@ -100,11 +100,12 @@ extern "C" tq_status tq_pack_kv(const tq_codec* kc, const tq_codec* vc, const vo
     if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 1)
         return fail(TQ_ERR_VALUE, "page pools must be 2-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // Tensor-core path for uniform 4-bit codecs; the general kernel covers
-    // every other format. TQ_PACK_KERNEL=general selects the general kernel.
+    // Tensor-core packs where both codecs have one (and the buffers are 16-byte
+    // aligned); the general kernel covers every other call. TQ_PACK_KERNEL=general
+    // selects the general kernel.
     const char* force = std::getenv("TQ_PACK_KERNEL");
     if (!(force && std::string(force) == "general")) {
-        tq_status st = launch_pack_u4(kc, vc, k, v, slot_mapping, num_tokens, k_pages, v_pages, num_blocks,
+        tq_status st = launch_pack_tc(kc, vc, k, v, slot_mapping, num_tokens, k_pages, v_pages, num_blocks,
                                       block_size, d_err, stream);
         if (st != TQ_OK && st != TQ_ERR_UNSUPPORTED) return st;
         if (st == TQ_OK) return finish_pack(s, d_err);

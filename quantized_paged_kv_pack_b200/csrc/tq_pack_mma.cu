@@ -1368,7 +1368,7 @@ __global__ void __launch_bounds__(PackGwSmemBase<RECIPE>::W * 32, 1) pack_gw_ker
 
 // Launches a tensor-core pack (uniform 4-bit, another plain format, or a group-wise
 // format); TQ_ERR_UNSUPPORTED when one of the two codecs has none.
-tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
+tq_status launch_pack_tc(const tq_codec* kc, const tq_codec* vc, const void* k, const void* v,
                          const int64_t* slot_mapping, int64_t num_tokens, void* k_pages, void* v_pages,
                          int64_t num_blocks, int32_t block_size, int32_t* d_err, void* stream) {
     // Uniform 4-bit K and V: the 4-bit kernel. Otherwise one launch per codec: plain formats (no QJL
@@ -1403,6 +1403,9 @@ tq_status launch_pack_u4(const tq_codec* kc, const tq_codec* vc, const void* k, 
         kind[side] = kd;
     }
     if (kind[0] == kNone || kind[1] == kNone) return TQ_ERR_UNSUPPORTED;
+    // 16-byte copies of the input rows (cp.async) and 8-byte row stores: the general kernel takes
+    // inputs or pools aligned only as the call requires (8 and 2 bytes).
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15) return TQ_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 15) return TQ_ERR_UNSUPPORTED;
     if (block_size % 8 != 0) return TQ_ERR_UNSUPPORTED;  // 16-byte aligned rows and norm arrays
     // 32-bit index arithmetic in the kernel: slots, tokens and work units must fit.

@@ -384,3 +384,34 @@ def test_pack_workloads_full_size_one_sequence(name):
         else:
             flips, total = compare_rows(rows, x, f, range(H))
             assert flips <= MAX_FLIP_FRACTION * total
+
+
+def test_pack_inputs_aligned_to_8_bytes_only():
+    """K and V that start 8 bytes past a 16-byte boundary (the call's own requirement is 8) take the
+    general kernel, since the tensor-core packs copy 16-byte pieces of the input rows; rows match the
+    oracle."""
+    H, T, bs = 2, 50, 16
+    kc, kf = codec_pair(H, (4,), (128,), 21)
+    vc, vf = codec_pair(H, (4, 3), (64, 64), 22)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4)
+    k0, v0 = random_kv(T, H, gen)
+    kb = torch.empty(T * H * D + 4, dtype=torch.bfloat16, device="cuda")
+    vb = torch.empty(T * H * D + 4, dtype=torch.bfloat16, device="cuda")
+    k = kb[4:].view(T, H, D)
+    v = vb[4:].view(T, H, D)
+    k.copy_(k0)
+    v.copy_(v0)
+    assert k.data_ptr() % 16 == 8 and v.data_ptr() % 16 == 8
+    nb = -(-T // bs) + 1
+    slots = torch.arange(T, device="cuda")
+    kp, vp = tq.page_pool(kc, nb, bs), tq.page_pool(vc, nb, bs)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.pack_kv(kc, vc, k, v, slots, kp, vp, bs, d_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    s = np.arange(T)
+    for pages, src, f in ((kp, k0, kf), (vp, v0, vf)):
+        x = src.float().cpu().numpy().astype(np.float64)
+        flips, total = compare_rows(rows_of(pages.cpu().numpy(), s, bs, f, H), x, f, range(H))
+        assert flips <= max(1, MAX_FLIP_FRACTION * total)
