@@ -368,7 +368,8 @@ def capture_step(step, outputs):
     ref = [o.clone() for o in outputs]
     try:
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        # thread-local: other threads' CUDA calls (NCCL's watchdog under torchrun) stay legal during capture
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
             step()
     except Exception as e:  # the library's launches could not be captured: time the eager step
         torch.cuda.synchronize()
